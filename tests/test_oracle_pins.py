@@ -1,0 +1,299 @@
+"""Pins of the fp64 oracle against facts the pages and mathematics fix.
+
+Each test is chosen so that a plausible mistake in the oracle fails it:
+  * a dropped residual / wrong sign / transposed weight  -> closed forms at N=1, N=2
+  * a wrong softmax scale or key source (input vs output) -> N=2 closed form
+  * an off-by-one in the lowbit block ranges              -> brute-force coverage,
+                                                             blocked == naive
+  * a wrong head split or missing mask                    -> textbook causal layer
+  * a tanh-approximate GELU or misplaced eps              -> GELU / RMS values
+Source of the method: "Recurrent Transformer" paper page (www.lshu.cn/news/403416):
+paper §2 (notation: RMS, Attn), §2.1 (Transformer layer), §2.2 (RT layer,
+temporary and persistent pairs), notes §4.2 (blocked schedule, exactness).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import rtinputs
+from oracle import rt_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _problem(B, N, d, H, d_ff, sigma=0.02, seed=0):
+    W = rtinputs.weights(seed, d, d_ff, sigma=sigma, dtype="f32")
+    x = rtinputs.x_batch(seed, range(B), N, d, dtype="f32")
+    return x, W
+
+
+def _relerr(a, b):
+    return np.max(np.abs(a - b)) / np.max(np.abs(b))
+
+
+# --------------------------------------------------------------------------
+# scalar building blocks, against textbook values
+# --------------------------------------------------------------------------
+def test_gelu_matches_normal_cdf_values():
+    # GELU(y) = y * Phi(y); Phi(1) = 0.8413447460685429, Phi(2) = 0.9772498680518208
+    # (standard normal table values). The tanh approximation gives 0.841192 at 1.
+    g = O.gelu(np.array([0.0, 1.0, -1.0, 2.0]))
+    assert g[0] == 0.0
+    assert abs(g[1] - 0.8413447460685429) < 1e-15
+    assert abs(g[2] - (-1.0) * (1 - 0.8413447460685429)) < 1e-15
+    assert abs(g[3] - 2 * 0.9772498680518208) < 1e-15
+
+
+def test_rms_definition():
+    # RMS(x) = x / sqrt(mean x^2 + eps): [3, 4] has mean square 12.5.
+    r = O.rms(np.array([3.0, 4.0]))
+    np.testing.assert_allclose(r, np.array([3.0, 4.0]) / math.sqrt(12.5 + 1e-6), rtol=0, atol=1e-15)
+    # output has mean square 1 up to the eps term
+    v = np.random.default_rng(1).standard_normal(64) * 5
+    r = O.rms(v)
+    ms = np.mean(v * v)
+    assert abs(np.mean(r * r) - ms / (ms + 1e-6)) < 1e-14
+
+
+# --------------------------------------------------------------------------
+# the schedule
+# --------------------------------------------------------------------------
+def test_lowbit_worked_example_from_pages():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "lowbit_worked_example.txt"))
+            if l.strip() and not l.startswith("#")]
+    for t, lb, q0, q1 in (map(int, r) for r in rows):
+        assert O.lowbit(t) == lb
+        blocks = {tt: (keys, qs) for tt, keys, qs in O.lowbit_blocks(16)}
+        keys, qs = blocks[t]
+        assert qs == list(range(q0, q1 + 1))
+        assert keys == list(range(t - lb + 1, t + 1))
+
+
+def test_lowbit_values():
+    assert [O.lowbit(t) for t in range(1, 17)] == [1, 2, 1, 4, 1, 2, 1, 8, 1, 2, 1, 4, 1, 2, 1, 16]
+    with pytest.raises(ValueError):
+        O.lowbit(0)
+
+
+@pytest.mark.parametrize("N", list(range(1, 65)) + [100, 127, 128, 129, 255, 256])
+def test_schedule_covers_every_causal_pair_exactly_once(N):
+    count = np.zeros((N + 1, N + 1), dtype=np.int64)
+    for t, keys, queries in O.lowbit_blocks(N):
+        for j in queries:
+            assert t < j, "a fold must happen before its query is finalised"
+            for i in keys:
+                assert i <= t, "a key can only be folded once revealed"
+                count[j, i] += 1
+    for j in range(1, N + 1):
+        for i in range(1, N + 1):
+            assert count[j, i] == (1 if i < j else 0), (j, i)
+
+
+# --------------------------------------------------------------------------
+# exactness of the blocked schedule (notes §4.2: equal up to FP reordering)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("N", [1, 2, 3, 7, 8, 64])
+def test_blocked_equals_naive(N):
+    x, W = _problem(2, N, 16, 2, 32, sigma=0.3)
+    zn, Kn, Vn = O.rt_layer(x, W, 2)
+    zb, Kb, Vb = O.rt_layer_blocked(x, W, 2)
+    for a, b in ((zb, zn), (Kb, Kn), (Vb, Vn)):
+        assert _relerr(a, b) < 1e-12
+
+
+def test_blocked_equals_naive_peaky_attention():
+    # sigma = 0.2 at d=64 makes softmax peaky, exercising the max-rescaling path.
+    x, W = _problem(2, 40, 64, 2, 128, sigma=0.2)
+    zn, Kn, Vn = O.rt_layer(x, W, 2)
+    zb, Kb, Vb = O.rt_layer_blocked(x, W, 2)
+    for a, b in ((zb, zn), (Kb, Kn), (Vb, Vn)):
+        assert _relerr(a, b) < 1e-12
+    # confirm peakiness: over all queries and heads, some query puts most of
+    # its mass on one key and the score spread is wide
+    best, spread = 0.0, 0.0
+    for t in range(1, 40):
+        r = O.rms(x[0, t])
+        q = r @ W["W_q"].T
+        for h in range(2):
+            sl = slice(32 * h, 32 * h + 32)
+            s = (Kn[0, :t, sl] @ q[sl]) / math.sqrt(32)
+            p = np.exp(s - s.max()); p /= p.sum()
+            best, spread = max(best, p.max()), max(spread, s.max() - s.min())
+    assert best > 0.5 and spread > 8
+
+
+# --------------------------------------------------------------------------
+# the fold on its own
+# --------------------------------------------------------------------------
+def test_block_fold_equals_direct_softmax_and_is_associative():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((5, 8)); k = rng.standard_normal((7, 8)); v = rng.standard_normal((7, 8))
+    sc = 0.7
+    m0 = np.full(5, -np.inf); l0 = np.zeros(5); o0 = np.zeros((5, 8))
+    m, l, o = O.block_fold(q, k, v, m0, l0, o0, sc)
+    # direct: softmax rows (explicit loops)
+    for a in range(5):
+        s = [sc * sum(q[a, e] * k[i, e] for e in range(8)) for i in range(7)]
+        mx = max(s)
+        w = [math.exp(si - mx) for si in s]
+        ref = [sum(w[i] * v[i, e] for i in range(7)) / sum(w) for e in range(8)]
+        np.testing.assert_allclose(o[a] / l[a], ref, rtol=1e-13, atol=1e-14)
+        assert abs(m[a] - mx) < 1e-14 * abs(mx)
+    # two halves folded one after the other = one fold
+    m1, l1, o1 = O.block_fold(q, k[:3], v[:3], m0, l0, o0, sc)
+    m2, l2, o2 = O.block_fold(q, k[3:], v[3:], m1, l1, o1, sc)
+    np.testing.assert_allclose(o2 / l2[:, None], o / l[:, None], rtol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# closed forms (pure-Python loops, independent of the oracle's helpers)
+# --------------------------------------------------------------------------
+def _py_rms(v):
+    ms = sum(e * e for e in v) / len(v)
+    return [e / math.sqrt(ms + 1e-6) for e in v]
+
+
+def _py_mv(Wm, v):
+    return [sum(Wm[i][j] * v[j] for j in range(len(v))) for i in range(len(Wm))]
+
+
+def _py_gelu(y):
+    return 0.5 * y * (1.0 + math.erf(y / math.sqrt(2.0)))
+
+
+def _py_layer_tail(x, a, W):
+    """u = x + W_o a ; z = u + W_2 GELU(W_1 RMS(u))."""
+    u = [xi + oi for xi, oi in zip(x, _py_mv(W["W_o"], a))]
+    h = [_py_gelu(e) for e in _py_mv(W["W_1"], _py_rms(u))]
+    return [ui + mi for ui, mi in zip(u, _py_mv(W["W_2"], h))]
+
+
+def test_N1_closed_form_single_token_layer():
+    # With one position, softmax over the single temporary key is 1, so
+    # a = v~ = W_v RMS(x), and the layer is one pre-norm layer on one token.
+    d, H, d_ff = 8, 2, 16
+    x, W = _problem(3, 1, d, H, d_ff, sigma=0.4)
+    z, K, V = O.rt_layer(x, W, H)
+    Wl = {k: v.tolist() for k, v in W.items()}
+    for b in range(3):
+        xb = x[b, 0].tolist()
+        a = _py_mv(Wl["W_v"], _py_rms(xb))
+        zb = _py_layer_tail(xb, a, Wl)
+        np.testing.assert_allclose(z[b, 0], zb, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(K[b, 0], _py_mv(Wl["W_k"], _py_rms(zb)), rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(V[b, 0], _py_mv(Wl["W_v"], _py_rms(zb)), rtol=1e-13, atol=1e-14)
+
+
+def test_N2_closed_form_persistent_key_from_output():
+    # Position 2 attends to {persistent (k1, v1) from z1} + {temporary (k~2, v~2)}.
+    # Two-way softmax = logistic: a = sig(s1 - s2) v1 + sig(s2 - s1) v~2, per head,
+    # with s = <k, q> / sqrt(d_h).
+    d, H, d_ff = 8, 2, 16
+    dh = d // H
+    x, W = _problem(2, 2, d, H, d_ff, sigma=0.5)
+    z, K, V = O.rt_layer(x, W, H)
+    Wl = {k: v.tolist() for k, v in W.items()}
+    sig = lambda y: 1.0 / (1.0 + math.exp(-y))
+    for b in range(2):
+        x1, x2 = x[b, 0].tolist(), x[b, 1].tolist()
+        z1 = _py_layer_tail(x1, _py_mv(Wl["W_v"], _py_rms(x1)), Wl)
+        k1 = _py_mv(Wl["W_k"], _py_rms(z1)); v1 = _py_mv(Wl["W_v"], _py_rms(z1))
+        r2 = _py_rms(x2)
+        q2 = _py_mv(Wl["W_q"], r2); kt = _py_mv(Wl["W_k"], r2); vt = _py_mv(Wl["W_v"], r2)
+        a = []
+        for h in range(H):
+            sl = slice(h * dh, (h + 1) * dh)
+            s1 = sum(p * r for p, r in zip(q2[sl], k1[sl])) / math.sqrt(dh)
+            s2 = sum(p * r for p, r in zip(q2[sl], kt[sl])) / math.sqrt(dh)
+            a += [sig(s1 - s2) * e1 + sig(s2 - s1) * e2 for e1, e2 in zip(v1[sl], vt[sl])]
+        z2 = _py_layer_tail(x2, a, Wl)
+        np.testing.assert_allclose(z[b, 0], z1, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(z[b, 1], z2, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(K[b, 0], k1, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(V[b, 1], _py_mv(Wl["W_v"], _py_rms(z2)), rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# standard-layer special case (paper §2.1): a textbook causal pre-norm layer
+# written as one masked score matrix per head
+# --------------------------------------------------------------------------
+def _textbook_causal_layer(x, W, H):
+    B, N, d = x.shape
+    dh = d // H
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    r = x / np.sqrt(ms + 1e-6)
+    q = (r @ W["W_q"].T).reshape(B, N, H, dh).transpose(0, 2, 1, 3)
+    k = (r @ W["W_k"].T).reshape(B, N, H, dh).transpose(0, 2, 1, 3)
+    v = (r @ W["W_v"].T).reshape(B, N, H, dh).transpose(0, 2, 1, 3)
+    S = q @ k.transpose(0, 1, 3, 2) / np.sqrt(dh)                 # [B,H,N,N]
+    mask = np.triu(np.ones((N, N), dtype=bool), k=1)              # key index > query index
+    S = np.where(mask, -np.inf, S)
+    P = np.exp(S - S.max(axis=-1, keepdims=True))
+    P /= P.sum(axis=-1, keepdims=True)
+    a = (P @ v).transpose(0, 2, 1, 3).reshape(B, N, d)
+    u = x + a @ W["W_o"].T
+    ru = u / np.sqrt(np.mean(u * u, axis=-1, keepdims=True) + 1e-6)
+    pre = ru @ W["W_1"].T
+    from scipy.stats import norm
+    y = u + (pre * norm.cdf(pre)) @ W["W_2"].T
+    return y, k.transpose(0, 2, 1, 3).reshape(B, N, d), v.transpose(0, 2, 1, 3).reshape(B, N, d)
+
+
+@pytest.mark.parametrize("N,H", [(1, 1), (5, 2), (33, 4)])
+def test_input_kv_source_is_the_textbook_transformer_layer(N, H):
+    x, W = _problem(2, N, 16, H, 48, sigma=0.3)
+    z, K, V = O.rt_layer(x, W, H, kv_source="input")
+    zt, Kt, Vt = _textbook_causal_layer(x, W, H)
+    assert _relerr(z, zt) < 1e-12
+    assert _relerr(K, Kt) < 1e-12
+    assert _relerr(V, Vt) < 1e-12
+
+
+def test_rt_reduces_to_transformer_when_branches_vanish_and_differs_otherwise():
+    # With W_o = 0 and W_2 = 0 the layer output equals its input (z = x), so the
+    # persistent pair from z equals the one from x.
+    x, W = _problem(2, 12, 16, 2, 32, sigma=0.3)
+    W0 = dict(W, W_o=np.zeros_like(W["W_o"]), W_2=np.zeros_like(W["W_2"]))
+    a = O.rt_layer(x, W0, 2)
+    b = O.rt_layer(x, W0, 2, kv_source="input")
+    for u, v in zip(a, b):
+        assert _relerr(u, v) < 1e-14
+    zr, _, _ = O.rt_layer(x, W, 2)
+    zt, _, _ = O.rt_layer(x, W, 2, kv_source="input")
+    assert np.max(np.abs(zr - zt)) > 1e-6
+
+
+# --------------------------------------------------------------------------
+# invariants
+# --------------------------------------------------------------------------
+def test_prefix_batch_permutation_and_causality():
+    x, W = _problem(3, 20, 16, 2, 32, sigma=0.3)
+    z, K, V = O.rt_layer(x, W, 2)
+    # prefix: running the first 11 positions gives the first 11 outputs
+    zp, Kp, Vp = O.rt_layer(x[:, :11], W, 2)
+    np.testing.assert_array_equal(zp, z[:, :11])
+    np.testing.assert_array_equal(Kp, K[:, :11])
+    # batch permutation permutes outputs (sequences are independent)
+    perm = [2, 0, 1]
+    zq, _, _ = O.rt_layer(x[perm], W, 2)
+    np.testing.assert_allclose(zq, z[perm], rtol=1e-14, atol=1e-14)
+    # causality: perturbing x at position 15 leaves positions < 15 unchanged
+    x2 = x.copy(); x2[:, 14] += 1.0
+    z2, _, _ = O.rt_layer(x2, W, 2)
+    np.testing.assert_array_equal(z2[:, :14], z[:, :14])
+    assert np.max(np.abs(z2[:, 14:] - z[:, 14:])) > 1e-3
+
+
+def test_stack_chains_layers():
+    vocab, d, H, d_ff = 50, 16, 2, 32
+    E = rtinputs.embedding(0, vocab, d, dtype="f32")
+    ids = np.stack([rtinputs.token_ids(0, b, 6, vocab) for b in range(2)])
+    layers = [rtinputs.weights(0, d, d_ff, sigma=0.3, dtype="f32", layer=i) for i in range(3)]
+    zs, kv = O.rt_stack(ids, E, layers, H)
+    x = E[ids]
+    for i, W in enumerate(layers):
+        x, K, V = O.rt_layer(x, W, H)
+        np.testing.assert_array_equal(K, kv[i][0])
+    np.testing.assert_array_equal(x, zs)
