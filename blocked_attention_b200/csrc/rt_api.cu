@@ -1,0 +1,816 @@
+// rt_api.cu -- host side of librtlayer: argument validation, workspace plan,
+// TMA descriptors, the N-step driver (host loop or one CUDA-graph replay) and
+// the extern "C" entry points declared in include/rtlayer.h.
+//
+// One forward of the Recurrent Transformer layer ("Recurrent Transformer"
+// paper page, www.lshu.cn/news/403416, paper §2.2 and notes §4.2):
+//   1. inv_rms(x) for all B*N rows; batched projection QKV = [W_q;W_k;W_v] rms(x)
+//      (queries and temporary pairs of every position, position-major);
+//   2. for t = 1..N (j = t-1):
+//        finalise a_j (temporary-pair merge, a = o/l)      [naive: full attention]
+//        u = x_j + a W_o^T ; h = GELU(rms(u) W_1^T) ; z_j = u + h W_2^T
+//        (k_j, v_j) = rms(z_j) [W_k; W_v]^T  -> position-major K, V
+//        fold keys (t - lb, t] into queries (t, t + lb], lb = lowbit(t)   [blocked only]
+// No accumulator initialisation pass: at t = 2^k the block (0, t] x (t, 2t] is
+// the first fold into each of its queries, so those folds write (m, l, o)
+// without reading them, and position 1 is never folded into.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <vector>
+
+#include "../../include/rtlayer.h"
+#include "rt_attn.cuh"
+#include "rt_common.cuh"
+#include "rt_gemm_tc.cuh"
+#include "rt_simt.cuh"
+
+namespace rt {
+
+static constexpr float kEps = 1e-6f;
+typedef __nv_bfloat16 bf16;
+
+#define RT_CK(call)                                  \
+  do {                                               \
+    cudaError_t e_ = (call);                         \
+    if (e_ != cudaSuccess) return RT_ERR_CUDA;       \
+  } while (0)
+
+static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// device set-up
+// ---------------------------------------------------------------------------
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                      const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DevState {
+  bool ready = false;
+  int sms = 0;
+  cudaStream_t capture = nullptr;
+};
+static std::mutex g_dev_mu;
+static DevState g_dev[64];
+static PFN_encodeTiled_t g_encode = nullptr;
+
+template <int BN, int EPI>
+static cudaError_t set_tc_attr() {
+  constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
+  return cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)GemmCfg<BN, STAGES>::SMEM_BYTES);
+}
+template <int EPI>
+static cudaError_t set_tc_attrs_epi() {
+  cudaError_t e;
+  if ((e = set_tc_attr<32, EPI>()) != cudaSuccess) return e;
+  if ((e = set_tc_attr<64, EPI>()) != cudaSuccess) return e;
+  if ((e = set_tc_attr<128, EPI>()) != cudaSuccess) return e;
+  return set_tc_attr<256, EPI>();
+}
+
+// Checks the current device and performs one-time per-device set-up.
+static int device_setup(DevState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RT_ERR_DEVICE;
+  if (dev < 0 || dev >= 64) return RT_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevState& ds = g_dev[dev];
+  if (!ds.ready) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return RT_ERR_DEVICE;
+    if (major != 10) return RT_ERR_DEVICE;
+    if (cudaDeviceGetAttribute(&ds.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return RT_ERR_DEVICE;
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return RT_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_encodeTiled_t>(fn);
+    }
+    if (set_tc_attrs_epi<EPI_PLAIN>() != cudaSuccess || set_tc_attrs_epi<EPI_PROJ>() != cudaSuccess ||
+        set_tc_attrs_epi<EPI_WO>() != cudaSuccess || set_tc_attrs_epi<EPI_W1>() != cudaSuccess ||
+        set_tc_attrs_epi<EPI_W2>() != cudaSuccess || set_tc_attrs_epi<EPI_WKV>() != cudaSuccess)
+      return RT_ERR_CUDA;
+    if (cudaStreamCreateWithFlags(&ds.capture, cudaStreamNonBlocking) != cudaSuccess) return RT_ERR_CUDA;
+    ds.ready = true;
+  }
+  *out = &ds;
+  return RT_OK;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][inner] matrix; box 64 x box_rows,
+// 128-byte swizzle (the K-major UMMA operand layout). Out-of-range rows read 0.
+static bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output-tile width: the widest tile that still gives >= 120 tiles.
+static int choose_bn(int M, int N) {
+  const long ntm = (M + 127) / 128;
+  for (int bn : {256, 128, 64})
+    if (ntm * ((N + bn - 1) / bn) >= 120) return bn;
+  return 32;
+}
+
+template <int BN, int EPI>
+static cudaError_t launch_tc_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+                                const EpiParams& p, unsigned* err, int sms, cudaStream_t st) {
+  constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
+  using C = GemmCfg<BN, STAGES>;
+  const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN);
+  const int grid = (int)std::min<long>(tiles, sms);
+  k_gemm_tc<BN, STAGES, EPI><<<grid, 192, C::SMEM_BYTES, st>>>(ta, tb, M, N, K, p, err);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+static cudaError_t launch_tc(int bn, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+                             const EpiParams& p, unsigned* err, int sms, cudaStream_t st) {
+  switch (bn) {
+    case 256: return launch_tc_bn<256, EPI>(ta, tb, M, N, K, p, err, sms, st);
+    case 128: return launch_tc_bn<128, EPI>(ta, tb, M, N, K, p, err, sms, st);
+    case 64: return launch_tc_bn<64, EPI>(ta, tb, M, N, K, p, err, sms, st);
+    default: return launch_tc_bn<32, EPI>(ta, tb, M, N, K, p, err, sms, st);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// shapes and workspace plan
+// ---------------------------------------------------------------------------
+struct Shape {
+  int B, N, d, H, d_ff, dtype, schedule;
+  int dh() const { return d / H; }
+};
+
+static int validate(const Shape& s) {
+  if (s.B <= 0 || s.N <= 0 || s.d <= 0 || s.H <= 0 || s.d_ff <= 0) return RT_ERR_INVALID_ARG;
+  if (s.d % s.H != 0) return RT_ERR_INVALID_ARG;
+  if (s.dtype != RT_F32 && s.dtype != RT_BF16) return RT_ERR_INVALID_ARG;
+  if (s.schedule != RT_SCHED_BLOCKED && s.schedule != RT_SCHED_NAIVE) return RT_ERR_INVALID_ARG;
+  const long rows = (long)s.B * s.N;
+  if (rows > (1l << 30) || (long)s.B * s.H > 65535) return RT_ERR_UNSUPPORTED;
+  const int dh = s.dh();
+  if (s.dtype == RT_F32) {
+    if (dh != 32 && dh != 64 && dh != 128) return RT_ERR_UNSUPPORTED;
+    if ((rows + 63) / 64 > 65535) return RT_ERR_UNSUPPORTED;
+  } else {
+    if (dh != 64 || s.d % 64 != 0 || s.d_ff % 64 != 0) return RT_ERR_UNSUPPORTED;
+  }
+  return RT_OK;
+}
+
+struct Plan {
+  Shape s;
+  size_t esz;
+  size_t off_err, off_qkv, off_m, off_l, off_o, off_inv, off_xr, off_wqkv, off_a, off_u32, off_u16, off_ru,
+      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, total;
+};
+
+static Plan make_plan(const Shape& s) {
+  Plan P;
+  std::memset(&P, 0, sizeof(P));
+  P.s = s;
+  P.esz = s.dtype == RT_BF16 ? 2 : 4;
+  const size_t rows = (size_t)s.B * s.N, d = s.d, B = s.B;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  P.off_err = take(256);
+  P.off_qkv = take(rows * 3 * d * P.esz);
+  if (s.schedule == RT_SCHED_BLOCKED) {
+    P.off_m = take(rows * s.H * 4);
+    P.off_l = take(rows * s.H * 4);
+    P.off_o = take(rows * d * 4);
+  }
+  if (s.dtype == RT_BF16) P.off_inv = take(rows * 4);
+  else P.off_xr = take(rows * d * 4);
+  P.off_wqkv = take(3 * d * d * P.esz);
+  P.off_a = take(B * d * P.esz);
+  P.off_u32 = take(B * d * 4);
+  if (s.dtype == RT_BF16) P.off_u16 = take(B * d * 2);
+  else P.off_ru = take(B * d * 4);
+  P.off_h = take(B * (size_t)s.d_ff * P.esz);
+  P.off_zs = take(B * d * P.esz);
+  if (s.dtype == RT_F32) P.off_rz = take(B * d * 4);
+  P.off_ssq_u = take((d / 32 + 1) * B * 4);
+  P.off_ssq_z = take((d / 32 + 1) * B * 4);
+  P.total = off;
+  return P;
+}
+
+struct Ptrs {
+  const void *x, *Wq, *Wk, *Wv, *Wo, *W1, *W2;
+  void *z, *K, *V, *ws;
+};
+
+// ---------------------------------------------------------------------------
+// per-kernel-class event timing (stream driver only)
+// ---------------------------------------------------------------------------
+enum KernelClass {
+  KC_INV_RMS = 0, KC_PROJ, KC_ATTEND, KC_WO, KC_W1, KC_W2, KC_WKV, KC_FOLD_WARP, KC_FOLD_MMA, KC_NORM,
+  KC_COUNT
+};
+
+struct Timer {
+  std::vector<cudaEvent_t> pool;
+  std::vector<int> cls;   // class of each recorded pair
+  size_t used = 0;        // events used in the current forward
+  cudaError_t err = cudaSuccess;
+  cudaEvent_t next() {
+    if (used == pool.size()) {
+      cudaEvent_t e;
+      cudaError_t c = cudaEventCreate(&e);
+      if (c != cudaSuccess) { err = c; return nullptr; }
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+};
+
+struct TimedScope {
+  Timer* T;
+  cudaStream_t st;
+  TimedScope(Timer* t, int c, cudaStream_t s) : T(t), st(s) {
+    if (T) {
+      cudaEvent_t e = T->next();
+      if (e) cudaEventRecord(e, st);
+      T->cls.push_back(c);
+    }
+  }
+  ~TimedScope() {
+    if (T) {
+      cudaEvent_t e = T->next();
+      if (e) cudaEventRecord(e, st);
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// fold launch (shared by the layer and rt_block_fold)
+// ---------------------------------------------------------------------------
+template <class T>
+static cudaError_t launch_fold(const T* Q, int q_stride, const T* K, const T* V, int kv_stride, float* m,
+                               float* l, float* o, int B, int H, int dh, int q0, int nq, int k0, int nk,
+                               float sc2, int init, bool allow_mma, cudaStream_t st) {
+  const int pairs = B * H;
+  if constexpr (std::is_same<T, bf16>::value) {
+    if (allow_mma && dh == 64 && nk % 16 == 0) {
+      dim3 grid((nq + 63) / 64, pairs);
+      k_fold_mma<<<grid, 128, 0, st>>>(Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init);
+      return cudaGetLastError();
+    }
+  }
+  const int blocks = (pairs + 3) / 4;
+  switch (dh) {
+    case 32: k_fold_warp<T, 1><<<blocks, 128, 0, st>>>(Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init); break;
+    case 64: k_fold_warp<T, 2><<<blocks, 128, 0, st>>>(Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init); break;
+    default: k_fold_warp<T, 4><<<blocks, 128, 0, st>>>(Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init); break;
+  }
+  return cudaGetLastError();
+}
+
+template <class T, int DPL>
+static cudaError_t launch_attend(const Plan& P, const T* qkv, const T* K, const T* V, const float* m,
+                                 const float* l, const float* o, T* a, int j, float sc2, cudaStream_t st) {
+  const Shape& s = P.s;
+  const int blocks = (s.B * s.H + 3) / 4;
+  if (s.schedule == RT_SCHED_BLOCKED)
+    k_finalize<T, DPL><<<blocks, 128, 0, st>>>(qkv, m, l, o, a, s.B, s.H, j, sc2, j > 0 ? 1 : 0);
+  else
+    k_naive_attn<T, DPL><<<blocks, 128, 0, st>>>(qkv, K, V, a, s.B, s.H, j, sc2);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// bf16 forward
+// ---------------------------------------------------------------------------
+static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st, Timer* T) {
+  const Shape& s = P.s;
+  char* ws = static_cast<char*>(X.ws);
+  unsigned* err = reinterpret_cast<unsigned*>(ws + P.off_err);
+  bf16* qkv = reinterpret_cast<bf16*>(ws + P.off_qkv);
+  float* m = reinterpret_cast<float*>(ws + P.off_m);
+  float* l = reinterpret_cast<float*>(ws + P.off_l);
+  float* o = reinterpret_cast<float*>(ws + P.off_o);
+  float* inv = reinterpret_cast<float*>(ws + P.off_inv);
+  bf16* wqkv = reinterpret_cast<bf16*>(ws + P.off_wqkv);
+  bf16* a16 = reinterpret_cast<bf16*>(ws + P.off_a);
+  float* u32 = reinterpret_cast<float*>(ws + P.off_u32);
+  bf16* u16 = reinterpret_cast<bf16*>(ws + P.off_u16);
+  bf16* h16 = reinterpret_cast<bf16*>(ws + P.off_h);
+  bf16* z16 = reinterpret_cast<bf16*>(ws + P.off_zs);
+  float* ssq_u = reinterpret_cast<float*>(ws + P.off_ssq_u);
+  float* ssq_z = reinterpret_cast<float*>(ws + P.off_ssq_z);
+  const bf16* x = static_cast<const bf16*>(X.x);
+  bf16* K = static_cast<bf16*>(X.K);
+  bf16* V = static_cast<bf16*>(X.V);
+  const int B = s.B, N = s.N, d = s.d, H = s.H, dff = s.d_ff;
+  const size_t rows = (size_t)B * N;
+  const size_t dd = (size_t)d * d * 2;
+
+  RT_CK(cudaMemsetAsync(err, 0, sizeof(unsigned), st));
+  RT_CK(cudaMemcpyAsync(wqkv, X.Wq, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + dd, X.Wk, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + 2 * dd, X.Wv, dd, cudaMemcpyDeviceToDevice, st));
+
+  // 1. queries and temporary pairs of all positions
+  {
+    TimedScope ts(T, KC_INV_RMS, st);
+    k_row_inv_rms<bf16><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(x, inv, rows, d, kEps);
+  }
+  RT_CK(cudaGetLastError());
+  const int bn_p = choose_bn((int)rows, 3 * d);
+  CUtensorMap tA_x, tB_qkv;
+  if (!make_tmap(&tA_x, x, d, rows, 128) || !make_tmap(&tB_qkv, wqkv, d, 3 * d, bn_p)) return RT_ERR_INVALID_ARG;
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.B = B; ep.Nseq = N; ep.d = d; ep.d_ff = dff; ep.eps = kEps;
+  ep.inv_rms = inv; ep.qkv = qkv; ep.x = x; ep.u32 = u32; ep.u16 = u16; ep.h16 = h16;
+  ep.zout = static_cast<bf16*>(X.z); ep.z16 = z16; ep.Kout = K; ep.Vout = V;
+  {
+    TimedScope ts(T, KC_PROJ, st);
+    RT_CK(launch_tc<EPI_PROJ>(bn_p, tA_x, tB_qkv, (int)rows, 3 * d, d, ep, err, ds.sms, st));
+  }
+
+  // 2. the N-step loop
+  const int bn_o = choose_bn(B, d), bn_1 = choose_bn(B, dff), bn_2 = choose_bn(B, d), bn_kv = choose_bn(B, 2 * d);
+  CUtensorMap tA_a, tB_o, tA_u, tB_1, tA_h, tB_2, tA_z, tB_kv;
+  if (!make_tmap(&tA_a, a16, d, B, 128) || !make_tmap(&tB_o, X.Wo, d, d, bn_o) ||
+      !make_tmap(&tA_u, u16, d, B, 128) || !make_tmap(&tB_1, X.W1, d, dff, bn_1) ||
+      !make_tmap(&tA_h, h16, dff, B, 128) || !make_tmap(&tB_2, X.W2, dff, d, bn_2) ||
+      !make_tmap(&tA_z, z16, d, B, 128) || !make_tmap(&tB_kv, wqkv + (size_t)d * d, d, 2 * d, bn_kv))
+    return RT_ERR_INVALID_ARG;
+  const float sc2 = kLog2e / std::sqrt((float)s.dh());
+  const bool blocked = s.schedule == RT_SCHED_BLOCKED;
+  for (int j = 0; j < N; ++j) {
+    ep.j = j;
+    {
+      TimedScope ts(T, KC_ATTEND, st);
+      RT_CK((launch_attend<bf16, 2>(P, qkv, K, V, m, l, o, a16, j, sc2, st)));
+    }
+    ep.ssq_out = ssq_u;
+    {
+      TimedScope ts(T, KC_WO, st);
+      RT_CK(launch_tc<EPI_WO>(bn_o, tA_a, tB_o, B, d, d, ep, err, ds.sms, st));
+    }
+    ep.ssq_in = ssq_u; ep.ssq_tiles = (d + bn_o - 1) / bn_o;
+    {
+      TimedScope ts(T, KC_W1, st);
+      RT_CK(launch_tc<EPI_W1>(bn_1, tA_u, tB_1, B, dff, d, ep, err, ds.sms, st));
+    }
+    ep.ssq_out = ssq_z;
+    {
+      TimedScope ts(T, KC_W2, st);
+      RT_CK(launch_tc<EPI_W2>(bn_2, tA_h, tB_2, B, d, dff, ep, err, ds.sms, st));
+    }
+    ep.ssq_in = ssq_z; ep.ssq_tiles = (d + bn_2 - 1) / bn_2;
+    {
+      TimedScope ts(T, KC_WKV, st);
+      RT_CK(launch_tc<EPI_WKV>(bn_kv, tA_z, tB_kv, B, 2 * d, d, ep, err, ds.sms, st));
+    }
+    if (blocked) {
+      const int t = j + 1, lb = lowbit(t), nq = std::min(lb, N - t);
+      if (nq > 0) {
+        TimedScope ts(T, lb >= 16 ? KC_FOLD_MMA : KC_FOLD_WARP, st);
+        RT_CK(launch_fold<bf16>(qkv, 3 * d, K, V, d, m, l, o, B, H, 64, t, nq, t - lb, lb, sc2,
+                                t == lb ? 1 : 0, true, st));
+      }
+    }
+  }
+  return RT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// fp32 forward (SIMT)
+// ---------------------------------------------------------------------------
+template <int EPI>
+static cudaError_t launch_simt(const float* A, const float* W, int M, int N, int K, const SimtEpi& p,
+                               cudaStream_t st) {
+  dim3 grid((N + 63) / 64, (M + 63) / 64);
+  k_gemm_simt<EPI><<<grid, 256, 0, st>>>(A, W, M, N, K, p);
+  return cudaGetLastError();
+}
+
+static int enqueue_f32(const Plan& P, const Ptrs& X, cudaStream_t st, Timer* T) {
+  const Shape& s = P.s;
+  char* ws = static_cast<char*>(X.ws);
+  unsigned* err = reinterpret_cast<unsigned*>(ws + P.off_err);
+  float* qkv = reinterpret_cast<float*>(ws + P.off_qkv);
+  float* m = reinterpret_cast<float*>(ws + P.off_m);
+  float* l = reinterpret_cast<float*>(ws + P.off_l);
+  float* o = reinterpret_cast<float*>(ws + P.off_o);
+  float* xr = reinterpret_cast<float*>(ws + P.off_xr);
+  float* wqkv = reinterpret_cast<float*>(ws + P.off_wqkv);
+  float* a = reinterpret_cast<float*>(ws + P.off_a);
+  float* u = reinterpret_cast<float*>(ws + P.off_u32);
+  float* ru = reinterpret_cast<float*>(ws + P.off_ru);
+  float* h = reinterpret_cast<float*>(ws + P.off_h);
+  float* zs = reinterpret_cast<float*>(ws + P.off_zs);
+  float* rz = reinterpret_cast<float*>(ws + P.off_rz);
+  const float* x = static_cast<const float*>(X.x);
+  float* K = static_cast<float*>(X.K);
+  float* V = static_cast<float*>(X.V);
+  const int B = s.B, N = s.N, d = s.d, H = s.H, dff = s.d_ff, dh = s.dh();
+  const size_t rows = (size_t)B * N;
+  const size_t dd = (size_t)d * d * 4;
+
+  RT_CK(cudaMemsetAsync(err, 0, sizeof(unsigned), st));
+  RT_CK(cudaMemcpyAsync(wqkv, X.Wq, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + dd, X.Wk, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + 2 * dd, X.Wv, dd, cudaMemcpyDeviceToDevice, st));
+  k_rmsnorm_f32<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(x, xr, rows, d, kEps);
+  RT_CK(cudaGetLastError());
+  SimtEpi p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B; p.Nseq = N; p.d = d; p.d_ff = dff;
+  p.qkv = qkv; p.x = x; p.u = u; p.h = h; p.zout = static_cast<float*>(X.z); p.zs = zs; p.Kout = K; p.Vout = V;
+  RT_CK(launch_simt<EPI_PROJ>(xr, wqkv, (int)rows, 3 * d, d, p, st));
+
+  const float sc2 = kLog2e / std::sqrt((float)dh);
+  const bool blocked = s.schedule == RT_SCHED_BLOCKED;
+  for (int j = 0; j < N; ++j) {
+    p.j = j;
+    cudaError_t e;
+    if (dh == 32) e = launch_attend<float, 1>(P, qkv, K, V, m, l, o, a, j, sc2, st);
+    else if (dh == 64) e = launch_attend<float, 2>(P, qkv, K, V, m, l, o, a, j, sc2, st);
+    else e = launch_attend<float, 4>(P, qkv, K, V, m, l, o, a, j, sc2, st);
+    RT_CK(e);
+    RT_CK(launch_simt<EPI_WO>(a, static_cast<const float*>(X.Wo), B, d, d, p, st));
+    k_rmsnorm_f32<<<(B + 7) / 8, 256, 0, st>>>(u, ru, B, d, kEps);
+    RT_CK(cudaGetLastError());
+    RT_CK(launch_simt<EPI_W1>(ru, static_cast<const float*>(X.W1), B, dff, d, p, st));
+    RT_CK(launch_simt<EPI_W2>(h, static_cast<const float*>(X.W2), B, d, dff, p, st));
+    k_rmsnorm_f32<<<(B + 7) / 8, 256, 0, st>>>(zs, rz, B, d, kEps);
+    RT_CK(cudaGetLastError());
+    RT_CK(launch_simt<EPI_WKV>(rz, wqkv + (size_t)d * d, B, 2 * d, d, p, st));
+    if (blocked) {
+      const int t = j + 1, lb = lowbit(t), nq = std::min(lb, N - t);
+      TimedScope ts(nq > 0 ? T : nullptr, KC_FOLD_WARP, st);
+      if (nq > 0)
+        RT_CK(launch_fold<float>(qkv, 3 * d, K, V, d, m, l, o, B, H, dh, t, nq, t - lb, lb, sc2,
+                                 t == lb ? 1 : 0, false, st));
+    }
+  }
+  return RT_OK;
+}
+
+static int enqueue_forward(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st,
+                           Timer* T = nullptr) {
+  return P.s.dtype == RT_BF16 ? enqueue_bf16(P, X, ds, st, T) : enqueue_f32(P, X, st, T);
+}
+
+// Kernels one forward launches (must mirror enqueue_bf16 / enqueue_f32).
+static long launch_count(const Shape& s) {
+  long folds = 0;
+  if (s.schedule == RT_SCHED_BLOCKED)
+    for (int t = 1; t <= s.N; ++t) folds += (std::min(lowbit(t), s.N - t) > 0) ? 1 : 0;
+  if (s.dtype == RT_BF16) return 2 + 5l * s.N + folds;
+  return 2 + 8l * s.N + folds;
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-graph driver: the whole forward recorded once per argument set
+// ---------------------------------------------------------------------------
+struct GraphKey {
+  uintptr_t p[11];
+  int v[8];
+  bool operator<(const GraphKey& o) const {
+    int c = std::memcmp(p, o.p, sizeof(p));
+    if (c) return c < 0;
+    return std::memcmp(v, o.v, sizeof(v)) < 0;
+  }
+};
+struct GraphEntry {
+  cudaGraphExec_t exec;
+  unsigned long long last_use;
+};
+static std::mutex g_graph_mu;
+static std::map<GraphKey, GraphEntry> g_graphs;
+static unsigned long long g_graph_clock = 0;
+static constexpr size_t kMaxGraphs = 8;
+
+static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st) {
+  DevState* ds = nullptr;
+  int rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  RT_CK(cudaStreamIsCapturing(st, &cap));
+  if (driver == RT_DRIVER_STREAM || cap != cudaStreamCaptureStatusNone) return enqueue_forward(P, X, *ds, st);
+
+  int dev = 0;
+  RT_CK(cudaGetDevice(&dev));
+  GraphKey key;
+  std::memset(&key, 0, sizeof(key));
+  const void* ptrs[11] = {X.x, X.Wq, X.Wk, X.Wv, X.Wo, X.W1, X.W2, X.z, X.K, X.V, X.ws};
+  for (int i = 0; i < 11; ++i) key.p[i] = reinterpret_cast<uintptr_t>(ptrs[i]);
+  const int vals[8] = {P.s.B, P.s.N, P.s.d, P.s.H, P.s.d_ff, P.s.dtype, P.s.schedule, dev};
+  std::memcpy(key.v, vals, sizeof(vals));
+
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  auto it = g_graphs.find(key);
+  if (it == g_graphs.end()) {
+    cudaGraph_t graph = nullptr;
+    RT_CK(cudaStreamBeginCapture(ds->capture, cudaStreamCaptureModeThreadLocal));
+    rc = enqueue_forward(P, X, *ds, ds->capture);
+    cudaError_t ce = cudaStreamEndCapture(ds->capture, &graph);
+    if (rc != RT_OK) {
+      if (graph) cudaGraphDestroy(graph);
+      return rc;
+    }
+    if (ce != cudaSuccess) return RT_ERR_CUDA;
+    cudaGraphExec_t exec = nullptr;
+    ce = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ce != cudaSuccess) return RT_ERR_CUDA;
+    if (g_graphs.size() >= kMaxGraphs) {
+      auto victim = g_graphs.begin();
+      for (auto i2 = g_graphs.begin(); i2 != g_graphs.end(); ++i2)
+        if (i2->second.last_use < victim->second.last_use) victim = i2;
+      cudaGraphExecDestroy(victim->second.exec);
+      g_graphs.erase(victim);
+    }
+    it = g_graphs.emplace(key, GraphEntry{exec, 0}).first;
+  }
+  it->second.last_use = ++g_graph_clock;
+  RT_CK(cudaGraphLaunch(it->second.exec, st));
+  return RT_OK;
+}
+
+}  // namespace rt
+
+// ===========================================================================
+// extern "C" entry points
+// ===========================================================================
+using namespace rt;
+
+extern "C" int rt_version(void) { return 100; }
+
+extern "C" const char* rt_status_string(int status) {
+  switch (status) {
+    case RT_OK: return "ok";
+    case RT_ERR_INVALID_ARG: return "invalid argument";
+    case RT_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case RT_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case RT_ERR_CUDA: return "CUDA runtime error";
+    case RT_ERR_TIMEOUT: return "device-side wait timed out";
+    case RT_ERR_DEVICE: return "no usable sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+extern "C" size_t rt_layer_workspace_bytes(int B, int N, int d, int H, int d_ff, int dtype, int schedule) {
+  Shape s{B, N, d, H, d_ff, dtype, schedule};
+  if (validate(s) != RT_OK) return 0;
+  return make_plan(s).total;
+}
+
+extern "C" int rt_layer_forward(const void* x, const void* W_q, const void* W_k, const void* W_v,
+                                const void* W_o, const void* W_1, const void* W_2, int B, int N, int d, int H,
+                                int d_ff, int dtype, int schedule, int driver, void* z, void* K, void* V,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s{B, N, d, H, d_ff, dtype, schedule};
+  int rc = validate(s);
+  if (rc != RT_OK) return rc;
+  if (driver != RT_DRIVER_GRAPH && driver != RT_DRIVER_STREAM) return RT_ERR_INVALID_ARG;
+  if (!x || !W_q || !W_k || !W_v || !W_o || !W_1 || !W_2 || !z || !K || !V) return RT_ERR_INVALID_ARG;
+  const void* all[10] = {x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V};
+  for (const void* p : all)
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return RT_ERR_INVALID_ARG;
+  const Plan P = make_plan(s);
+  if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return RT_ERR_WORKSPACE;
+  Ptrs X{x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V, workspace};
+  return run_forward(P, X, driver, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int rt_layer_sync_status(void* workspace, void* stream) {
+  if (!workspace) return RT_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned h = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RT_ERR_CUDA;
+  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return RT_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(h), st) != cudaSuccess) return RT_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RT_ERR_CUDA;
+  if (h & RT_DEVERR_TIMEOUT) return RT_ERR_TIMEOUT;
+  if (h & RT_DEVERR_INDEX) return RT_ERR_INVALID_ARG;
+  return RT_OK;
+}
+
+static size_t host_io_bytes(const Shape& s, size_t esz) {
+  const size_t rows = (size_t)s.B * s.N, d = s.d;
+  size_t tot = 0;
+  tot += align_up(rows * d * esz, 256) * 4;                     // x, z, K, V
+  tot += align_up(d * d * esz, 256) * 4;                        // W_q, W_k, W_v, W_o
+  tot += align_up((size_t)s.d_ff * d * esz, 256) * 2;           // W_1, W_2
+  return tot;
+}
+
+extern "C" size_t rt_layer_host_workspace_bytes(int B, int N, int d, int H, int d_ff, int dtype, int schedule) {
+  Shape s{B, N, d, H, d_ff, dtype, schedule};
+  if (validate(s) != RT_OK) return 0;
+  const Plan P = make_plan(s);
+  return P.total + host_io_bytes(s, P.esz);
+}
+
+extern "C" int rt_layer_forward_host(const void* x, const void* W_q, const void* W_k, const void* W_v,
+                                     const void* W_o, const void* W_1, const void* W_2, int B, int N, int d,
+                                     int H, int d_ff, int dtype, int schedule, int driver, void* z, void* K,
+                                     void* V, void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s{B, N, d, H, d_ff, dtype, schedule};
+  int rc = validate(s);
+  if (rc != RT_OK) return rc;
+  if (!x || !W_q || !W_k || !W_v || !W_o || !W_1 || !W_2 || !z || !K || !V) return RT_ERR_INVALID_ARG;
+  const Plan P = make_plan(s);
+  if (!workspace || workspace_bytes < P.total + host_io_bytes(s, P.esz) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return RT_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t rows = (size_t)B * N;
+  const size_t act = rows * d * P.esz, wdd = (size_t)d * d * P.esz, wdf = (size_t)d_ff * d * P.esz;
+  char* base = static_cast<char*>(workspace) + P.total;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base + off;
+    off += align_up(bytes, 256);
+    return p;
+  };
+  char *xd = take(act), *zd = take(act), *Kd = take(act), *Vd = take(act);
+  char *Wqd = take(wdd), *Wkd = take(wdd), *Wvd = take(wdd), *Wod = take(wdd), *W1d = take(wdf), *W2d = take(wdf);
+  RT_CK(cudaMemcpyAsync(xd, x, act, cudaMemcpyHostToDevice, st));
+  RT_CK(cudaMemcpyAsync(Wqd, W_q, wdd, cudaMemcpyHostToDevice, st));
+  RT_CK(cudaMemcpyAsync(Wkd, W_k, wdd, cudaMemcpyHostToDevice, st));
+  RT_CK(cudaMemcpyAsync(Wvd, W_v, wdd, cudaMemcpyHostToDevice, st));
+  RT_CK(cudaMemcpyAsync(Wod, W_o, wdd, cudaMemcpyHostToDevice, st));
+  RT_CK(cudaMemcpyAsync(W1d, W_1, wdf, cudaMemcpyHostToDevice, st));
+  RT_CK(cudaMemcpyAsync(W2d, W_2, wdf, cudaMemcpyHostToDevice, st));
+  Ptrs X{xd, Wqd, Wkd, Wvd, Wod, W1d, W2d, zd, Kd, Vd, workspace};
+  rc = run_forward(P, X, driver, st);
+  if (rc != RT_OK) return rc;
+  RT_CK(cudaMemcpyAsync(z, zd, act, cudaMemcpyDeviceToHost, st));
+  RT_CK(cudaMemcpyAsync(K, Kd, act, cudaMemcpyDeviceToHost, st));
+  RT_CK(cudaMemcpyAsync(V, Vd, act, cudaMemcpyDeviceToHost, st));
+  return RT_OK;
+}
+
+extern "C" int rt_embed_forward(const int32_t* ids, const void* E, int B, int N, int vocab, int d, int dtype,
+                                void* x, void* workspace, void* stream) {
+  if (!ids || !E || !x || B <= 0 || N <= 0 || vocab <= 0 || d <= 0) return RT_ERR_INVALID_ARG;
+  if (dtype != RT_F32 && dtype != RT_BF16) return RT_ERR_INVALID_ARG;
+  DevState* ds = nullptr;
+  int rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* err = static_cast<unsigned*>(workspace);
+  const size_t rows = (size_t)B * N;
+  if (rows > 0x7fffffffu) return RT_ERR_UNSUPPORTED;
+  if (dtype == RT_BF16)
+    k_embed<bf16><<<(unsigned)rows, 128, 0, st>>>(ids, static_cast<const bf16*>(E), static_cast<bf16*>(x), rows,
+                                                  vocab, d, err);
+  else
+    k_embed<float><<<(unsigned)rows, 128, 0, st>>>(ids, static_cast<const float*>(E), static_cast<float*>(x),
+                                                   rows, vocab, d, err);
+  RT_CK(cudaGetLastError());
+  return RT_OK;
+}
+
+extern "C" int rt_block_fold(const void* Q, int q_stride, const void* K, const void* V, int kv_stride, float* m,
+                             float* l, float* o, int B, int H, int d_h, int q0, int nq, int k0, int nk, int dtype,
+                             void* stream) {
+  if (!Q || !K || !V || !m || !l || !o) return RT_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || nq <= 0 || nk <= 0 || q0 < 0 || k0 < 0) return RT_ERR_INVALID_ARG;
+  if (q_stride < H * d_h || kv_stride < H * d_h || (long)B * H > 65535) return RT_ERR_INVALID_ARG;
+  if (dtype == RT_BF16 && d_h != 64) return RT_ERR_UNSUPPORTED;
+  if (dtype == RT_F32 && d_h != 32 && d_h != 64 && d_h != 128) return RT_ERR_UNSUPPORTED;
+  if (dtype == RT_BF16 && (q_stride % 8 != 0 || kv_stride % 8 != 0)) return RT_ERR_UNSUPPORTED;
+  DevState* ds = nullptr;
+  int rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  const float sc2 = kLog2e / std::sqrt((float)d_h);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == RT_BF16)
+    e = launch_fold<bf16>(static_cast<const bf16*>(Q), q_stride, static_cast<const bf16*>(K),
+                          static_cast<const bf16*>(V), kv_stride, m, l, o, B, H, d_h, q0, nq, k0, nk, sc2, 0, true, st);
+  else if (dtype == RT_F32)
+    e = launch_fold<float>(static_cast<const float*>(Q), q_stride, static_cast<const float*>(K),
+                           static_cast<const float*>(V), kv_stride, m, l, o, B, H, d_h, q0, nq, k0, nk, sc2, 0, false,
+                           st);
+  else
+    return RT_ERR_INVALID_ARG;
+  return e == cudaSuccess ? RT_OK : RT_ERR_CUDA;
+}
+
+extern "C" int rt_project_qkv(const void* x, const void* W_qkv, int B, int N, int d, int dtype, void* QKV,
+                              void* scratch, void* stream) {
+  if (!x || !W_qkv || !QKV || !scratch || B <= 0 || N <= 0 || d <= 0) return RT_ERR_INVALID_ARG;
+  if (dtype == RT_BF16 && d % 64 != 0) return RT_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)B * N;
+  if (rows > (1u << 30)) return RT_ERR_UNSUPPORTED;
+  DevState* ds = nullptr;
+  int rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == RT_BF16) {
+    float* inv = static_cast<float*>(scratch);
+    k_row_inv_rms<bf16><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const bf16*>(x), inv, rows, d, kEps);
+    RT_CK(cudaGetLastError());
+    const int bn = choose_bn((int)rows, 3 * d);
+    CUtensorMap ta, tb;
+    if (!make_tmap(&ta, x, d, rows, 128) || !make_tmap(&tb, W_qkv, d, 3 * d, bn)) return RT_ERR_INVALID_ARG;
+    EpiParams ep;
+    std::memset(&ep, 0, sizeof(ep));
+    ep.B = B; ep.Nseq = N; ep.d = d; ep.inv_rms = inv; ep.qkv = static_cast<bf16*>(QKV);
+    RT_CK(launch_tc<EPI_PROJ>(bn, ta, tb, (int)rows, 3 * d, d, ep, nullptr, ds->sms, st));
+  } else if (dtype == RT_F32) {
+    if ((rows + 63) / 64 > 65535) return RT_ERR_UNSUPPORTED;
+    float* xr = static_cast<float*>(scratch);
+    k_rmsnorm_f32<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const float*>(x), xr, rows, d, kEps);
+    RT_CK(cudaGetLastError());
+    SimtEpi p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = B; p.Nseq = N; p.d = d; p.qkv = static_cast<float*>(QKV);
+    RT_CK(launch_simt<EPI_PROJ>(xr, static_cast<const float*>(W_qkv), (int)rows, 3 * d, d, p, st));
+  } else {
+    return RT_ERR_INVALID_ARG;
+  }
+  return RT_OK;
+}
+
+extern "C" int rt_gemm_bf16(const void* A, const void* W, float* C, int M, int Nout, int Kd, void* stream) {
+  if (!A || !W || !C || M <= 0 || Nout <= 0 || Kd <= 0) return RT_ERR_INVALID_ARG;
+  if (Kd % 64 != 0) return RT_ERR_UNSUPPORTED;
+  DevState* ds = nullptr;
+  int rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  const int bn = choose_bn(M, Nout);
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, A, Kd, M, 128) || !make_tmap(&tb, W, Kd, Nout, bn)) return RT_ERR_INVALID_ARG;
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.c32 = C;
+  RT_CK(launch_tc<EPI_PLAIN>(bn, ta, tb, M, Nout, Kd, ep, nullptr, ds->sms, static_cast<cudaStream_t>(stream)));
+  return RT_OK;
+}
+
+extern "C" long rt_layer_launch_count(int B, int N, int d, int H, int d_ff, int dtype, int schedule) {
+  Shape s{B, N, d, H, d_ff, dtype, schedule};
+  if (validate(s) != RT_OK) return -1;
+  return launch_count(s);
+}
+
+extern "C" int rt_layer_forward_timed(const void* x, const void* W_q, const void* W_k, const void* W_v,
+                                      const void* W_o, const void* W_1, const void* W_2, int B, int N, int d,
+                                      int H, int d_ff, int dtype, int schedule, void* z, void* K, void* V,
+                                      void* workspace, size_t workspace_bytes, void* stream, float* class_ms,
+                                      int* class_launches, int n_classes) {
+  Shape s{B, N, d, H, d_ff, dtype, schedule};
+  int rc = validate(s);
+  if (rc != RT_OK) return rc;
+  if (!x || !W_q || !W_k || !W_v || !W_o || !W_1 || !W_2 || !z || !K || !V || !class_ms || !class_launches)
+    return RT_ERR_INVALID_ARG;
+  const Plan P = make_plan(s);
+  if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return RT_ERR_WORKSPACE;
+  DevState* ds = nullptr;
+  rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  RT_CK(cudaStreamIsCapturing(st, &cap));
+  if (cap != cudaStreamCaptureStatusNone) return RT_ERR_INVALID_ARG;
+  static std::mutex mu;
+  static Timer timer;
+  std::lock_guard<std::mutex> lk(mu);
+  timer.used = 0;
+  timer.cls.clear();
+  timer.err = cudaSuccess;
+  Ptrs X{x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V, workspace};
+  rc = enqueue_forward(P, X, *ds, st, &timer);
+  if (rc != RT_OK) return rc;
+  if (timer.err != cudaSuccess) return RT_ERR_CUDA;
+  RT_CK(cudaStreamSynchronize(st));
+  for (int c = 0; c < n_classes; ++c) { class_ms[c] = 0.f; class_launches[c] = 0; }
+  for (size_t i = 0; i < timer.cls.size(); ++i) {
+    float ms = 0.f;
+    RT_CK(cudaEventElapsedTime(&ms, timer.pool[2 * i], timer.pool[2 * i + 1]));
+    const int c = timer.cls[i];
+    if (c < n_classes) { class_ms[c] += ms; class_launches[c] += 1; }
+  }
+  return RT_OK;
+}

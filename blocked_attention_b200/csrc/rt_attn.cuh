@@ -1,0 +1,472 @@
+// rt_attn.cuh -- attention side of the Recurrent Transformer layer.
+//
+// Source: "Recurrent Transformer" paper page (www.lshu.cn/news/403416):
+//   notes §2.2 / paper §2.2 : the temporary pair (from x_t) is used only by
+//                             position t's own attention;
+//   notes §4.2 / paper §5   : exact blocked schedule with online-softmax
+//                             statistics (running max m, normaliser l,
+//                             numerator o);
+//   notes §4.1              : the naive schedule (query t reads all revealed
+//                             pairs at step t), kept as the ablation;
+//   paper §6.3              : position-major KV cache.
+//
+// Storage (position-major; row (j, b) = position j of sequence b):
+//   QKV [N][B][3d]  : q | k~ | v~ of every position (from the projection)
+//   K, V [N][B][d]  : persistent pairs
+//   m, l [N][B][H]  : fp32 statistics; m is kept in log2 units of the scaled
+//                     score, s2 = <q, k> * log2(e) / sqrt(d_h)
+//   o [N][B][d]     : fp32 numerators
+// Head h occupies columns h*d_h .. h*d_h + d_h - 1 of every row.
+#pragma once
+
+#include "rt_common.cuh"
+
+namespace rt {
+
+template <class T, int DPL>
+__device__ __forceinline__ void load_lane(const T* src, float (&v)[DPL]) {
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) v[i] = to_f(src[i]);
+}
+
+// ---------------------------------------------------------------------------
+// finalise position j: merge the temporary pair into the accumulator of
+// query j, then a_j = o / l per head. One warp per (b, h).
+// has_acc = false: the accumulator of j was never folded into (position 1).
+// ---------------------------------------------------------------------------
+template <class T, int DPL>
+__global__ void __launch_bounds__(128)
+    k_finalize(const T* __restrict__ qkv, const float* __restrict__ m, const float* __restrict__ l,
+               const float* __restrict__ o, T* __restrict__ a_out, int B, int H, int j, float sc2,
+               int has_acc) {
+  constexpr int DH = DPL * 32;
+  const int pair = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (pair >= B * H) return;
+  const int b = pair / H, h = pair - b * H;
+  const int d = H * DH;
+  const size_t row = (size_t)j * B + b;
+  const T* qp = qkv + row * (size_t)(3 * d) + h * DH + lane * DPL;
+  float q[DPL], kt[DPL], vt[DPL];
+  load_lane<T, DPL>(qp, q);
+  load_lane<T, DPL>(qp + d, kt);
+  load_lane<T, DPL>(qp + 2 * d, vt);
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) dot += q[i] * kt[i];
+  const float s = warp_sum(dot) * sc2;
+  float mo = -INFINITY, lo = 0.f, oo[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) oo[i] = 0.f;
+  if (has_acc) {
+    mo = m[row * H + h];
+    lo = l[row * H + h];
+    const float* op = o + row * (size_t)d + h * DH + lane * DPL;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) oo[i] = op[i];
+  }
+  const float mn = fmaxf(mo, s);
+  const float al = rescale(mo, mn), pt = exp2f(s - mn);
+  const float ln = lo * al + pt;
+  const float inv = 1.f / ln;
+  T* ap = a_out + (size_t)b * d + h * DH + lane * DPL;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) ap[i] = from_f<T>((oo[i] * al + pt * vt[i]) * inv);
+}
+
+// ---------------------------------------------------------------------------
+// naive schedule (ablation): a_j from all persistent pairs i < j plus the
+// temporary pair, streaming keys 32 at a time. One warp per (b, h).
+// ---------------------------------------------------------------------------
+template <class T, int DPL>
+__global__ void __launch_bounds__(128)
+    k_naive_attn(const T* __restrict__ qkv, const T* __restrict__ K, const T* __restrict__ V,
+                 T* __restrict__ a_out, int B, int H, int j, float sc2) {
+  constexpr int DH = DPL * 32;
+  __shared__ float sq[4][DH];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x * 4 + w;
+  const bool active = pair < B * H;
+  const int b = active ? pair / H : 0, h = active ? pair - (pair / H) * H : 0;
+  const int d = H * DH;
+  const size_t row = (size_t)j * B + b;
+  const T* qp = qkv + row * (size_t)(3 * d) + h * DH;
+  if (active) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) sq[w][lane * DPL + i] = to_f(qp[lane * DPL + i]);
+  }
+  __syncwarp();
+  if (!active) return;
+  float mo = -INFINITY, lo = 0.f, oo[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) oo[i] = 0.f;
+  for (int c0 = 0; c0 < j; c0 += 32) {
+    const int n = min(32, j - c0);
+    float s = -INFINITY;
+    if (lane < n) {
+      const T* kp = K + ((size_t)(c0 + lane) * B + b) * d + h * DH;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int e = 0; e < DH; ++e) acc += sq[w][e] * to_f(kp[e]);
+      s = acc * sc2;
+    }
+    const float mn = fmaxf(mo, warp_max(s));
+    const float al = rescale(mo, mn);
+    const float pl = (lane < n) ? exp2f(s - mn) : 0.f;
+    lo = lo * al + warp_sum(pl);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) oo[i] *= al;
+    for (int i = 0; i < n; ++i) {
+      const float pi = __shfl_sync(0xffffffffu, pl, i);
+      const T* vp = V + ((size_t)(c0 + i) * B + b) * d + h * DH + lane * DPL;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) oo[e] += pi * to_f(vp[e]);
+    }
+    mo = mn;
+  }
+  // the temporary pair
+  float kt[DPL], vt[DPL], q[DPL];
+  load_lane<T, DPL>(qp + d + lane * DPL, kt);
+  load_lane<T, DPL>(qp + 2 * d + lane * DPL, vt);
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) q[i] = sq[w][lane * DPL + i];
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) dot += q[i] * kt[i];
+  const float s = warp_sum(dot) * sc2;
+  const float mn = fmaxf(mo, s);
+  const float al = rescale(mo, mn), pt = exp2f(s - mn);
+  const float inv = 1.f / (lo * al + pt);
+  T* ap = a_out + (size_t)b * d + h * DH + lane * DPL;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) ap[i] = from_f<T>((oo[i] * al + pt * vt[i]) * inv);
+}
+
+// ---------------------------------------------------------------------------
+// block fold, warp kernel: one warp per (b, h) folds keys [k0, k0+nk) into
+// queries [q0, q0+nq). Used for small blocks (lowbit(t) < 16) in bf16 and for
+// every block in fp32. init = 1: the queries' accumulators are empty (first
+// fold into them), so they are written without being read.
+// ---------------------------------------------------------------------------
+template <class T, int DPL>
+__global__ void __launch_bounds__(128)
+    k_fold_warp(const T* __restrict__ Q, int q_stride, const T* __restrict__ K,
+                const T* __restrict__ V, int kv_stride, float* __restrict__ m,
+                float* __restrict__ l, float* __restrict__ o, int B, int H, int q0, int nq,
+                int k0, int nk, float sc2, int init) {
+  constexpr int DH = DPL * 32, KC = 8;
+  const int pair = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (pair >= B * H) return;
+  const int b = pair / H, h = pair - b * H;
+  const int d = H * DH;
+  for (int jq = q0; jq < q0 + nq; ++jq) {
+    const size_t row = (size_t)jq * B + b;
+    float q[DPL];
+    load_lane<T, DPL>(Q + row * (size_t)q_stride + h * DH + lane * DPL, q);
+    float mo = -INFINITY, lo = 0.f, oo[DPL];
+    float* op = o + row * (size_t)d + h * DH + lane * DPL;
+    if (init) {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) oo[i] = 0.f;
+    } else {
+      mo = m[row * H + h];
+      lo = l[row * H + h];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) oo[i] = op[i];
+    }
+    for (int c0 = 0; c0 < nk; c0 += KC) {
+      const int n = min(KC, nk - c0);
+      float s[KC];
+      float cm = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < KC; ++i) {
+        s[i] = -INFINITY;
+        if (i < n) {
+          float kk[DPL];
+          load_lane<T, DPL>(K + ((size_t)(k0 + c0 + i) * B + b) * kv_stride + h * DH + lane * DPL, kk);
+          float dot = 0.f;
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) dot += q[e] * kk[e];
+          s[i] = warp_sum(dot) * sc2;
+          cm = fmaxf(cm, s[i]);
+        }
+      }
+      const float mn = fmaxf(mo, cm);
+      const float al = rescale(mo, mn);
+      lo *= al;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) oo[e] *= al;
+#pragma unroll
+      for (int i = 0; i < KC; ++i) {
+        if (i < n) {
+          const float p = exp2f(s[i] - mn);
+          float vv[DPL];
+          load_lane<T, DPL>(V + ((size_t)(k0 + c0 + i) * B + b) * kv_stride + h * DH + lane * DPL, vv);
+          lo += p;
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) oo[e] += p * vv[e];
+        }
+      }
+      mo = mn;
+    }
+    if (lane == 0) {
+      m[row * H + h] = mo;
+      l[row * H + h] = lo;
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) op[i] = oo[i];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// block fold, tensor-core kernel (bf16, d_h = 64, nk a multiple of 16):
+// S = Q K^T and O += P V with mma.sync m16n8k16 (fp32 accumulate), online
+// softmax over key chunks of 64, then one merge into the fp32 (m, l, o) of
+// each query. CTA = 4 warps = 64 queries of one (b, h); K/V chunks are
+// double-buffered in shared memory by cp.async.
+// ---------------------------------------------------------------------------
+namespace mma_detail {
+constexpr int LDS = 72;  // padded smem row (bf16): 144 bytes, conflict-free ldmatrix
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+}  // namespace mma_detail
+
+__global__ void __launch_bounds__(128)
+    k_fold_mma(const __nv_bfloat16* __restrict__ Q, int q_stride, const __nv_bfloat16* __restrict__ K,
+               const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m,
+               float* __restrict__ l, float* __restrict__ o, int B, int H, int q0, int nq, int k0,
+               int nk, float sc2, int init) {
+  using namespace mma_detail;
+  constexpr int DH = 64, QT = 64, KC = 64;
+  __shared__ __align__(128) __nv_bfloat16 sQ[QT * LDS];
+  __shared__ __align__(128) __nv_bfloat16 sK[2][KC * LDS];
+  __shared__ __align__(128) __nv_bfloat16 sV[2][KC * LDS];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pair = blockIdx.y;
+  const int b = pair / H, h = pair - b * H;
+  const int d = H * DH;
+  const int qt0 = q0 + blockIdx.x * QT;
+  const int nrows = min(QT, q0 + nq - qt0);
+
+  // Q tile (rows beyond nrows are zero)
+  for (int c = tid; c < QT * 8; c += 128) {
+    const int r = c >> 3, cc = c & 7;
+    __nv_bfloat16* dst = &sQ[r * LDS + cc * 8];
+    if (r < nrows)
+      cp_async16(dst, Q + ((size_t)(qt0 + r) * B + b) * q_stride + h * DH + cc * 8);
+    else
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+  }
+  auto load_kv = [&](int buf, int kc0, int kcn) {
+    for (int c = tid; c < kcn * 8; c += 128) {
+      const int r = c >> 3, cc = c & 7;
+      const size_t src = ((size_t)(k0 + kc0 + r) * B + b) * kv_stride + h * DH + cc * 8;
+      cp_async16(&sK[buf][r * LDS + cc * 8], K + src);
+      cp_async16(&sV[buf][r * LDS + cc * 8], V + src);
+    }
+  };
+  load_kv(0, 0, min(KC, nk));
+  cp_async_commit();
+
+  const int nchunks = (nk + KC - 1) / KC;
+  const bool warp_active = warp * 16 < nrows;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  float oacc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+  uint32_t qf[4][4];
+
+  for (int ci = 0; ci < nchunks; ++ci) {
+    const int buf = ci & 1;
+    if (ci + 1 < nchunks) {
+      load_kv(buf ^ 1, (ci + 1) * KC, min(KC, nk - (ci + 1) * KC));
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    if (warp_active) {
+      if (ci == 0) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          ldsm_x4(qf[ks], &sQ[(warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + ks * 16 + (lane >> 4) * 8]);
+      }
+      const int kcn = min(KC, nk - ci * KC);
+      const int ntiles = kcn >> 3;  // even: kcn is a multiple of 16
+      float sacc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+        if (nt < ntiles) {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            uint32_t r[4];
+            ldsm_x4(r, &sK[buf][(nt * 8 + (lane & 7)) * LDS + kk * 32 + (lane >> 3) * 8]);
+            mma16816(sacc[nt], qf[2 * kk], r[0], r[1]);
+            mma16816(sacc[nt], qf[2 * kk + 1], r[2], r[3]);
+          }
+        }
+      }
+      // online softmax: rows g = lane/4 (regs 0,1) and g+8 (regs 2,3)
+      float cmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        if (nt < ntiles) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[nt][e] *= sc2;
+          cmax[0] = fmaxf(cmax[0], fmaxf(sacc[nt][0], sacc[nt][1]));
+          cmax[1] = fmaxf(cmax[1], fmaxf(sacc[nt][2], sacc[nt][3]));
+        }
+      }
+      float al[2];
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        cmax[rr] = fmaxf(cmax[rr], __shfl_xor_sync(0xffffffffu, cmax[rr], 1));
+        cmax[rr] = fmaxf(cmax[rr], __shfl_xor_sync(0xffffffffu, cmax[rr], 2));
+        const float mn = fmaxf(mrow[rr], cmax[rr]);
+        al[rr] = rescale(mrow[rr], mn);
+        mrow[rr] = mn;
+        lrow[rr] *= al[rr];
+      }
+#pragma unroll
+      for (int nd = 0; nd < 8; ++nd) {
+        oacc[nd][0] *= al[0]; oacc[nd][1] *= al[0];
+        oacc[nd][2] *= al[1]; oacc[nd][3] *= al[1];
+      }
+#pragma unroll
+      for (int kj = 0; kj < 4; ++kj) {
+        if (2 * kj < ntiles) {
+          float p[2][4];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            p[u][0] = exp2f(sacc[2 * kj + u][0] - mrow[0]);
+            p[u][1] = exp2f(sacc[2 * kj + u][1] - mrow[0]);
+            p[u][2] = exp2f(sacc[2 * kj + u][2] - mrow[1]);
+            p[u][3] = exp2f(sacc[2 * kj + u][3] - mrow[1]);
+            lrow[0] += p[u][0] + p[u][1];
+            lrow[1] += p[u][2] + p[u][3];
+          }
+          uint32_t pa[4];
+          pa[0] = pack2(p[0][0], p[0][1]);
+          pa[1] = pack2(p[0][2], p[0][3]);
+          pa[2] = pack2(p[1][0], p[1][1]);
+          pa[3] = pack2(p[1][2], p[1][3]);
+#pragma unroll
+          for (int nd = 0; nd < 8; nd += 2) {
+            uint32_t r[4];
+            ldsm_x4_t(r, &sV[buf][(kj * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + nd * 8 + (lane >> 4) * 8]);
+            mma16816(oacc[nd], pa, r[0], r[1]);
+            mma16816(oacc[nd + 1], pa, r[2], r[3]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  if (!warp_active) return;
+  // merge the block result into the global statistics of each query row
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    float lsum = lrow[rr];
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+    const int r = warp * 16 + (lane >> 2) + rr * 8;
+    if (r >= nrows) continue;
+    const size_t row = (size_t)(qt0 + r) * B + b;
+    float mg = -INFINITY, lg = 0.f;
+    if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }
+    const float mn = fmaxf(mg, mrow[rr]);
+    const float ag = rescale(mg, mn), ab = rescale(mrow[rr], mn);
+    if ((lane & 3) == 0) {
+      m[row * H + h] = mn;
+      l[row * H + h] = lg * ag + lsum * ab;
+    }
+    float* op = o + row * (size_t)d + h * DH + (lane & 3) * 2;
+#pragma unroll
+    for (int nd = 0; nd < 8; ++nd) {
+      float2 og = make_float2(0.f, 0.f);
+      if (!init) og = *reinterpret_cast<const float2*>(op + nd * 8);
+      og.x = og.x * ag + oacc[nd][rr * 2 + 0] * ab;
+      og.y = og.y * ag + oacc[nd][rr * 2 + 1] * ab;
+      *reinterpret_cast<float2*>(op + nd * 8) = og;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// small helpers
+// ---------------------------------------------------------------------------
+// inv[r] = 1 / sqrt(mean(x_r^2) + eps), one warp per row of width d
+template <class T>
+__global__ void __launch_bounds__(256) k_row_inv_rms(const T* __restrict__ x, float* __restrict__ inv,
+                                                     size_t rows, int d, float eps) {
+  const size_t r = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const T* xr = x + r * d;
+  float s = 0.f;
+  for (int e = lane; e < d; e += 32) {
+    const float v = to_f(xr[e]);
+    s += v * v;
+  }
+  s = warp_sum(s);
+  if (lane == 0) inv[r] = rsqrtf(s / (float)d + eps);
+}
+
+// out[r] = in[r] / rms(in[r]) (fp32 path)
+__global__ void __launch_bounds__(256) k_rmsnorm_f32(const float* __restrict__ in, float* __restrict__ out,
+                                                     size_t rows, int d, float eps) {
+  const size_t r = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float* xr = in + r * d;
+  float s = 0.f;
+  for (int e = lane; e < d; e += 32) s += xr[e] * xr[e];
+  s = warp_sum(s);
+  const float inv = rsqrtf(s / (float)d + eps);
+  for (int e = lane; e < d; e += 32) out[r * d + e] = xr[e] * inv;
+}
+
+// x[r][:] = E[ids[r]][:]
+template <class T>
+__global__ void k_embed(const int32_t* __restrict__ ids, const T* __restrict__ E, T* __restrict__ x,
+                        size_t rows, int vocab, int d, unsigned* err) {
+  const size_t r = blockIdx.x;
+  if (r >= rows) return;
+  const int id = ids[r];
+  const bool ok = id >= 0 && id < vocab;
+  if (!ok && threadIdx.x == 0) set_error(err, RT_DEVERR_INDEX);
+  for (int e = threadIdx.x; e < d; e += blockDim.x)
+    x[r * d + e] = ok ? E[(size_t)id * d + e] : from_f<T>(0.f);
+}
+
+}  // namespace rt

@@ -1,0 +1,298 @@
+// rt_gemm_tc.cuh -- bf16 x bf16 -> fp32 GEMM on the sm_100a tensor cores
+// (tcgen05.mma, accumulators in tensor memory, operands staged by TMA), with
+// the fused epilogues of the Recurrent Transformer layer.
+//
+//   C[M][N] = A[M][K] * W[N][K]^T      (A, W row-major = K-major operands)
+//
+// Kernel shape: persistent CTAs of 192 threads.
+//   warp 0      : TMA producer (one elected lane), STAGES-deep smem ring
+//   warp 1      : tensor-memory allocator + MMA issuer (one lane)
+//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
+// Tile 128 x BN x 64; two TMEM accumulators of BN columns so that the
+// epilogue of tile i overlaps the MMAs of tile i+1.
+//
+// Epilogues (one thread owns one output row, 32 columns at a time):
+//   PLAIN : C fp32
+//   PROJ  : batched projection of all positions, scaled by 1/rms(x) of the
+//           row, written position-major [N][B][3d] (queries and temporary
+//           pairs, "Recurrent Transformer" paper page, notes §4.2: queries
+//           depend only on the layer input and are computed up front)
+//   WO    : u = x_t + a W_o^T (fp32 and bf16 copies) + per-tile sum of u^2
+//   W1    : h = GELU((u W_1^T) / rms(u))            (rms from the WO partials)
+//   W2    : z_t = u + h W_2^T -> output z, bf16 copy, per-tile sum of z^2
+//   WKV   : [k_t | v_t] = (z_t [W_k; W_v]^T) / rms(z_t) -> position-major K, V
+// The identity rms(v) W^T = (v W^T) / r(v), r(v) = sqrt(mean v^2 + eps), moves
+// each RMSNorm into the next GEMM's epilogue; it changes only rounding.
+#pragma once
+
+#include "rt_common.cuh"
+
+namespace rt {
+
+enum EpiKind { EPI_PLAIN = 0, EPI_PROJ = 1, EPI_WO = 2, EPI_W1 = 3, EPI_W2 = 4, EPI_WKV = 5 };
+
+struct EpiParams {
+  int B, Nseq, d, d_ff, j;   // batch, sequence length, width, MLP width, position (0-based)
+  float eps;
+  float* c32;                // PLAIN out [M][N]
+  const float* inv_rms;      // PROJ: 1/rms per input row [B*N]
+  __nv_bfloat16* qkv;        // PROJ out [N][B][3d]
+  const __nv_bfloat16* x;    // WO: layer input [B][N][d]
+  float* u32;                // WO out / W2 in: [B][d]
+  __nv_bfloat16* u16;        // WO out: [B][d]
+  float* ssq_out;            // WO / W2 out: [n_tiles][B]
+  const float* ssq_in;       // W1 / WKV in: [ssq_tiles][B]
+  int ssq_tiles;
+  __nv_bfloat16* h16;        // W1 out: [B][d_ff]
+  __nv_bfloat16* zout;       // W2 out: [B][N][d]
+  __nv_bfloat16* z16;        // W2 out: [B][d]
+  __nv_bfloat16* Kout;       // WKV out: [N][B][d]
+  __nv_bfloat16* Vout;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// store 32 floats as 32 bf16 (64 contiguous bytes, 16-byte aligned)
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+    w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+    w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+    w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+    d4[i] = w;
+  }
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 w = s4[i];
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 f = __bfloat1622float2(p[k]);
+      v[8 * i + 2 * k] = f.x;
+      v[8 * i + 2 * k + 1] = f.y;
+    }
+  }
+}
+
+template <int BN, int STAGES>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+  static constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256;
+  static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
+};
+
+// Row-wise epilogue for one 32-column chunk; returns the chunk's sum of squares
+// of the value that feeds the next RMSNorm (WO: u, W2: z), else 0.
+template <int EPI>
+__device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int col0, int N,
+                                                float (&v)[32], float row_scale) {
+  float ssq = 0.f;
+  if constexpr (EPI == EPI_PLAIN) {
+    float* dst = p.c32 + (size_t)row * N + col0;
+    if (col0 + 32 <= N && (N % 4) == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < N) dst[i] = v[i];
+    }
+  } else if constexpr (EPI == EPI_PROJ) {
+    const int b = row / p.Nseq, n = row - b * p.Nseq;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= row_scale;
+    store_bf16x32(p.qkv + ((size_t)n * p.B + b) * (size_t)(3 * p.d) + col0, v);
+  } else if constexpr (EPI == EPI_WO) {
+    const int b = row;
+    float xv[32];
+    load_bf16x32(p.x + ((size_t)b * p.Nseq + p.j) * p.d + col0, xv);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      v[i] += xv[i];
+      ssq += v[i] * v[i];
+    }
+    float4* u4 = reinterpret_cast<float4*>(p.u32 + (size_t)b * p.d + col0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    store_bf16x32(p.u16 + (size_t)b * p.d + col0, v);
+  } else if constexpr (EPI == EPI_W1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i] * row_scale);
+    store_bf16x32(p.h16 + (size_t)row * p.d_ff + col0, v);
+  } else if constexpr (EPI == EPI_W2) {
+    const int b = row;
+    const float4* u4 = reinterpret_cast<const float4*>(p.u32 + (size_t)b * p.d + col0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float4 w = u4[i];
+      v[4 * i] += w.x; v[4 * i + 1] += w.y; v[4 * i + 2] += w.z; v[4 * i + 3] += w.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ssq += v[i] * v[i];
+    store_bf16x32(p.zout + ((size_t)b * p.Nseq + p.j) * p.d + col0, v);
+    store_bf16x32(p.z16 + (size_t)b * p.d + col0, v);
+  } else if constexpr (EPI == EPI_WKV) {
+    const int b = row;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= row_scale;
+    const size_t base = ((size_t)p.j * p.B + b) * p.d;
+    if (col0 < p.d) store_bf16x32(p.Kout + base + col0, v);
+    else store_bf16x32(p.Vout + base + (col0 - p.d), v);
+  }
+  return ssq;
+}
+
+template <int EPI>
+__device__ __forceinline__ float row_scale_for(const EpiParams& p, int row) {
+  if constexpr (EPI == EPI_PROJ) {
+    return p.inv_rms[row];
+  } else if constexpr (EPI == EPI_W1 || EPI == EPI_WKV) {
+    float s = 0.f;
+    for (int t = 0; t < p.ssq_tiles; ++t) s += p.ssq_in[(size_t)t * p.B + row];
+    return rsqrtf(s / (float)p.d + p.eps);
+  } else {
+    return 1.f;
+  }
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              int M, int N, int K, EpiParams p, unsigned* err) {
+  using C = GemmCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;   // [2]
+  uint64_t* tempty = tfull + 2;       // [2]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntn = (N + BN - 1) / BN, ntm = (M + C::BM - 1) / C::BM;
+  const int num_tiles = ntn * ntm;
+  const int nk = K / C::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); }
+  if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mt = tile / ntn, nt = tile - mt * ntn;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, kb * C::BK, mt * C::BM);
+          tma_load_2d(&tmB, &full[s], sB + s * C::B_BYTES, kb * C::BK, nt * BN);
+        }
+      }
+      if (!ok) {
+        // wait (bounded) for copies still in flight before the CTA can exit
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+        for (uint32_t i = first; i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1u, err);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(C::BM, BN);
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+        const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* a_st = sA + s * C::A_BYTES;
+          const uint8_t* b_st = sB + s * C::B_BYTES;
+#pragma unroll
+          for (int k = 0; k < C::BK / 16; ++k) {
+            // advance 16 bf16 (32 bytes) along K inside the 128-byte swizzle atom
+            tc_mma_f16(d_tmem, smem_desc_sw128(a_st + k * 32), smem_desc_sw128(b_st + k * 32), idesc,
+                       (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        tc_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps ----------------
+    const int q = warp & 3;
+    uint32_t local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      const int mt = tile / ntn, nt = tile - mt * ntn;
+      const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&tfull[acc], aph, err) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int row = mt * C::BM + q * 32 + lane;
+      const bool row_ok = row < M;
+      const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
+      float ssq = 0.f;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c, r);
+        tmem_ld_wait();
+        const int col0 = nt * BN + c;
+        if (row_ok && col0 < N) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
+        }
+      }
+      if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
+        if (row_ok) p.ssq_out[(size_t)nt * p.B + row] = ssq;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace rt

@@ -1,0 +1,243 @@
+"""ctypes binding of librtlayer.so (the C ABI declared in include/rtlayer.h).
+
+Argument marshalling only: torch supplies device memory and streams; every
+step of the layer runs in the library's CUDA kernels. There is no fallback:
+if the library is missing or the device is not an sm_100 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librtlayer.so")
+
+RT_OK, RT_ERR_INVALID_ARG, RT_ERR_UNSUPPORTED, RT_ERR_WORKSPACE, RT_ERR_CUDA, RT_ERR_TIMEOUT, RT_ERR_DEVICE = \
+    0, -1, -2, -3, -4, -5, -6
+RT_F32, RT_BF16 = 0, 1
+RT_SCHED_BLOCKED, RT_SCHED_NAIVE = 0, 1
+RT_DRIVER_GRAPH, RT_DRIVER_STREAM = 0, 1
+
+SCHEDULES = {"blocked": RT_SCHED_BLOCKED, "naive": RT_SCHED_NAIVE}
+DRIVERS = {"graph": RT_DRIVER_GRAPH, "stream": RT_DRIVER_STREAM}
+WEIGHT_NAMES = ("W_q", "W_k", "W_v", "W_o", "W_1", "W_2")
+
+EXPORTS = ("rt_version", "rt_status_string", "rt_layer_workspace_bytes", "rt_layer_forward",
+           "rt_layer_sync_status", "rt_layer_host_workspace_bytes", "rt_layer_forward_host",
+           "rt_embed_forward", "rt_block_fold", "rt_project_qkv", "rt_gemm_bf16",
+           "rt_layer_launch_count", "rt_layer_forward_timed")
+
+KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
+                  "fold_warp", "fold_mma")
+RT_KC_COUNT = 10
+
+_lib = None
+
+
+class RTError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load librtlayer.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m blocked_attention_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    fp = ctypes.POINTER(ctypes.c_float)
+    L.rt_version.restype = i
+    L.rt_status_string.restype = ctypes.c_char_p
+    L.rt_status_string.argtypes = [i]
+    L.rt_layer_workspace_bytes.restype = sz
+    L.rt_layer_workspace_bytes.argtypes = [i] * 7
+    L.rt_layer_host_workspace_bytes.restype = sz
+    L.rt_layer_host_workspace_bytes.argtypes = [i] * 7
+    fwd_args = [vp] * 7 + [i] * 8 + [vp] * 4 + [sz, vp]
+    L.rt_layer_forward.restype = i
+    L.rt_layer_forward.argtypes = fwd_args
+    L.rt_layer_forward_host.restype = i
+    L.rt_layer_forward_host.argtypes = fwd_args
+    L.rt_layer_sync_status.restype = i
+    L.rt_layer_sync_status.argtypes = [vp, vp]
+    L.rt_embed_forward.restype = i
+    L.rt_embed_forward.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp]
+    L.rt_block_fold.restype = i
+    L.rt_block_fold.argtypes = [vp, i, vp, vp, i, fp, fp, fp] + [i] * 8 + [i, vp]
+    L.rt_project_qkv.restype = i
+    L.rt_project_qkv.argtypes = [vp, vp, i, i, i, i, vp, vp, vp]
+    L.rt_gemm_bf16.restype = i
+    L.rt_gemm_bf16.argtypes = [vp, vp, fp, i, i, i, vp]
+    L.rt_layer_launch_count.restype = ctypes.c_long
+    L.rt_layer_launch_count.argtypes = [i] * 7
+    L.rt_layer_forward_timed.restype = i
+    L.rt_layer_forward_timed.argtypes = [vp] * 7 + [i] * 7 + [vp] * 4 + [sz, vp, fp,
+                                                                         ctypes.POINTER(ctypes.c_int), i]
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().rt_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != RT_OK:
+        raise RTError(fn, status)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return RT_F32
+    if t == torch.bfloat16:
+        return RT_BF16
+    raise ValueError(f"unsupported dtype {t}")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _fptr(t):
+    return ctypes.cast(ctypes.c_void_p(t.data_ptr()), ctypes.POINTER(ctypes.c_float))
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# --------------------------------------------------------------------------
+# the layer
+# --------------------------------------------------------------------------
+def workspace_bytes(B, N, d, H, d_ff, dtype=torch.bfloat16, schedule="blocked") -> int:
+    return int(lib().rt_layer_workspace_bytes(B, N, d, H, d_ff, _dtype_code(dtype), SCHEDULES[schedule]))
+
+
+def host_workspace_bytes(B, N, d, H, d_ff, dtype=torch.bfloat16, schedule="blocked") -> int:
+    return int(lib().rt_layer_host_workspace_bytes(B, N, d, H, d_ff, _dtype_code(dtype), SCHEDULES[schedule]))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    # torch's caching allocator returns blocks aligned to at least 512 bytes
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def layer_forward(x: torch.Tensor, W: dict, H: int, d_ff: int | None = None, schedule: str = "blocked",
+                  driver: str = "graph", out=None, workspace: torch.Tensor | None = None, stream=None):
+    """rt_layer_forward on device tensors. x: [B, N, d] (fp32 or bf16, cuda);
+    W: dict of W_q, W_k, W_v, W_o [d, d], W_1 [d_ff, d], W_2 [d, d_ff].
+    Returns (z [B, N, d], K [N, B, d], V [N, B, d]) -- K, V position-major."""
+    B, N, d = x.shape
+    d_ff = d_ff or W["W_1"].shape[0]
+    code = _dtype_code(x.dtype)
+    for n in WEIGHT_NAMES:
+        if W[n].dtype != x.dtype or not W[n].is_contiguous() or W[n].device != x.device:
+            raise ValueError(f"weight {n} must be a contiguous {x.dtype} tensor on {x.device}")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if out is None:
+        z = torch.empty_like(x)
+        K = torch.empty((N, B, d), dtype=x.dtype, device=x.device)
+        V = torch.empty_like(K)
+    else:
+        z, K, V = out
+    nbytes = workspace_bytes(B, N, d, H, d_ff, x.dtype, schedule)
+    if nbytes == 0:
+        raise RTError("rt_layer_workspace_bytes", RT_ERR_UNSUPPORTED)
+    if workspace is None:
+        workspace = alloc_workspace(nbytes, x.device)
+    rc = lib().rt_layer_forward(_ptr(x), *[_ptr(W[n]) for n in WEIGHT_NAMES], B, N, d, H, d_ff, code,
+                                SCHEDULES[schedule], DRIVERS[driver], _ptr(z), _ptr(K), _ptr(V),
+                                _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("rt_layer_forward", rc)
+    return z, K, V
+
+
+def launch_count(B, N, d, H, d_ff, dtype=torch.bfloat16, schedule="blocked") -> int:
+    return int(lib().rt_layer_launch_count(B, N, d, H, d_ff, _dtype_code(dtype), SCHEDULES[schedule]))
+
+
+def layer_forward_timed(x: torch.Tensor, W: dict, H: int, out, workspace: torch.Tensor,
+                        d_ff: int | None = None, schedule: str = "blocked", stream=None) -> dict:
+    """rt_layer_forward_timed: one forward with CUDA events around every
+    kernel; returns {class: (total_ms, launches)} (synchronises the stream)."""
+    B, N, d = x.shape
+    d_ff = d_ff or W["W_1"].shape[0]
+    z, K, V = out
+    ms = (ctypes.c_float * RT_KC_COUNT)()
+    cnt = (ctypes.c_int * RT_KC_COUNT)()
+    rc = lib().rt_layer_forward_timed(_ptr(x), *[_ptr(W[n]) for n in WEIGHT_NAMES], B, N, d, H, d_ff,
+                                      _dtype_code(x.dtype), SCHEDULES[schedule], _ptr(z), _ptr(K), _ptr(V),
+                                      _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream),
+                                      ms, cnt, RT_KC_COUNT)
+    _check("rt_layer_forward_timed", rc)
+    return {name: (float(ms[i]), int(cnt[i])) for i, name in enumerate(KERNEL_CLASSES) if cnt[i] > 0}
+
+
+def sync_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(lib().rt_layer_sync_status(_ptr(workspace), _stream(stream)))
+
+
+def layer_forward_host(x: torch.Tensor, W: dict, H: int, out, workspace: torch.Tensor, d_ff: int | None = None,
+                       schedule: str = "blocked", driver: str = "graph", stream=None):
+    """rt_layer_forward_host: x, W and out=(z, K, V) are HOST tensors (pinned
+    for asynchronous copies); workspace is a device buffer of
+    host_workspace_bytes(...) bytes. Returns once enqueued."""
+    B, N, d = x.shape
+    d_ff = d_ff or W["W_1"].shape[0]
+    z, K, V = out
+    rc = lib().rt_layer_forward_host(_ptr(x), *[_ptr(W[n]) for n in WEIGHT_NAMES], B, N, d, H, d_ff,
+                                     _dtype_code(x.dtype), SCHEDULES[schedule], DRIVERS[driver], _ptr(z),
+                                     _ptr(K), _ptr(V), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                     _stream(stream))
+    _check("rt_layer_forward_host", rc)
+
+
+# --------------------------------------------------------------------------
+# stack front end and component entry points
+# --------------------------------------------------------------------------
+def embed_forward(ids: torch.Tensor, E: torch.Tensor, workspace: torch.Tensor | None = None, stream=None):
+    B, N = ids.shape
+    vocab, d = E.shape
+    x = torch.empty((B, N, d), dtype=E.dtype, device=E.device)
+    rc = lib().rt_embed_forward(_ptr(ids), _ptr(E), B, N, vocab, d, _dtype_code(E.dtype), _ptr(x),
+                                _ptr(workspace), _stream(stream))
+    _check("rt_embed_forward", rc)
+    return x
+
+
+def block_fold(Q, K, V, m, l, o, H: int, d_h: int, q0: int, nq: int, k0: int, nk: int, stream=None):
+    """rt_block_fold: Q [n_pos, B, q_stride], K/V [n_pos, B, kv_stride];
+    m, l [n_pos, B, H] and o [n_pos, B, H*d_h] fp32 updated in place."""
+    B = Q.shape[1]
+    rc = lib().rt_block_fold(_ptr(Q), Q.shape[2], _ptr(K), _ptr(V), K.shape[2], _fptr(m), _fptr(l), _fptr(o),
+                             B, H, d_h, q0, nq, k0, nk, _dtype_code(Q.dtype), _stream(stream))
+    _check("rt_block_fold", rc)
+
+
+def project_qkv(x: torch.Tensor, W_qkv: torch.Tensor, stream=None):
+    B, N, d = x.shape
+    qkv = torch.empty((N, B, 3 * d), dtype=x.dtype, device=x.device)
+    scratch = torch.empty(B * N * (1 if x.dtype == torch.bfloat16 else d), dtype=torch.float32, device=x.device)
+    rc = lib().rt_project_qkv(_ptr(x), _ptr(W_qkv), B, N, d, _dtype_code(x.dtype), _ptr(qkv), _ptr(scratch),
+                              _stream(stream))
+    _check("rt_project_qkv", rc)
+    return qkv
+
+
+def gemm_bf16(A: torch.Tensor, W: torch.Tensor, stream=None):
+    M, Kd = A.shape
+    Nout = W.shape[0]
+    C = torch.empty((M, Nout), dtype=torch.float32, device=A.device)
+    rc = lib().rt_gemm_bf16(_ptr(A), _ptr(W), _fptr(C), M, Nout, Kd, _stream(stream))
+    _check("rt_gemm_bf16", rc)
+    return C

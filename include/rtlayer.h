@@ -1,0 +1,205 @@
+/*
+ * rtlayer.h -- C ABI of librtlayer.so: the forward pass (prefill / training
+ * forward) of one Recurrent Transformer (RT) layer on an NVIDIA B200 (sm_100a),
+ * computed with the exact dyadic ("lowbit") blocked schedule.
+ *
+ * Source of the operation: "Recurrent Transformer" paper page
+ * (www.lshu.cn/news/403416):
+ *   - paper §2.2 (Recurrent Transformer layer): a layer maps x_1..x_N to
+ *     z_1..z_N; position i forms its query and a temporary (k, v) from its
+ *     input x_i, and a persistent (k_i, v_i) from its output z_i, which is
+ *     stored and used by every later position;
+ *   - notes §2.2 (temporary vs persistent key/value pairs);
+ *   - notes §4.2 / paper §5 (exact blocked schedule): queries are computed up
+ *     front; when (k_t, v_t) is revealed, keys (t - lowbit(t), t] are folded
+ *     into the online-softmax statistics (m, l, o) of queries
+ *     (t, t + lowbit(t)]; exact up to floating-point reordering;
+ *   - paper §6.3 (position-major KV cache).
+ *
+ * Layer (per sequence b, t = 1..N; rms(v) = v / sqrt(mean(v^2) + 1e-6)):
+ *   r = rms(x_t); q = W_q r; k~ = W_k r; v~ = W_v r
+ *   a_t = per head h (columns h*d_h .. h*d_h + d_h - 1, d_h = d/H):
+ *         softmax over {(k_i, v_i) : i < t} + {(k~, v~)} of <k, q_h>/sqrt(d_h)
+ *   u = x_t + W_o a_t ; z_t = u + W_2 GELU(W_1 rms(u))   (exact erf GELU)
+ *   k_t = W_k rms(z_t) ; v_t = W_v rms(z_t)               (persistent pair)
+ *
+ * Conventions for every entry point below
+ *   - Pointers named *_dev are device memory owned by the caller; the library
+ *     allocates no device memory on these paths. Pointers named *_host are
+ *     host memory owned by the caller (page-locked for asynchronous copies).
+ *   - Storage type: RT_F32 (all tensors fp32, SIMT fp32 arithmetic) or
+ *     RT_BF16 (tensors bf16, fp32 accumulation and fp32 softmax statistics).
+ *   - Weights use nn.Linear orientation [out][in] (row-major), y = W r:
+ *       W_q, W_k, W_v, W_o : [d][d]; W_1 : [d_ff][d]; W_2 : [d][d_ff].
+ *   - x and z are [B][N][d] row-major (sequence-major).
+ *   - K and V (the persistent pairs) are POSITION-MAJOR [N][B][d], i.e.
+ *     [N][B][H][d_h]: the pairs of one position for all sequences are
+ *     contiguous, so a block (t - lb, t] is one contiguous slice.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *     Calls are asynchronous on it. Host-detectable errors (null pointers,
+ *     unsupported shapes, workspace too small) are returned before anything is
+ *     enqueued. Device-side errors (a bounded wait that ran out) are recorded
+ *     in an error word inside the workspace and reported by
+ *     rt_layer_sync_status.
+ *   - Concurrent calls sharing one workspace race; use one workspace per
+ *     in-flight call.
+ *   - Supported shapes: RT_F32: d_h in {32, 64, 128}. RT_BF16: d_h = 64,
+ *     d and d_ff multiples of 64. B, N >= 1. Others: RT_ERR_UNSUPPORTED.
+ */
+#ifndef RTLAYER_H
+#define RTLAYER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RT_OK = 0,
+  RT_ERR_INVALID_ARG = -1,  /* null pointer, non-positive size, d % H != 0 */
+  RT_ERR_UNSUPPORTED = -2,  /* shape/dtype combination not implemented     */
+  RT_ERR_WORKSPACE = -3,    /* workspace pointer null or too small          */
+  RT_ERR_CUDA = -4,         /* a CUDA runtime call failed                   */
+  RT_ERR_TIMEOUT = -5,      /* a device-side bounded wait ran out           */
+  RT_ERR_DEVICE = -6        /* no usable sm_100 device                      */
+} rt_status;
+
+typedef enum { RT_F32 = 0, RT_BF16 = 1 } rt_dtype;
+
+/* RT_SCHED_BLOCKED: the exact lowbit schedule (the product path).
+ * RT_SCHED_NAIVE: query t attends to all persistent pairs i < t at step t,
+ * Theta(N^2) traffic (the ablation of notes §4.1). Same result up to rounding. */
+typedef enum { RT_SCHED_BLOCKED = 0, RT_SCHED_NAIVE = 1 } rt_schedule;
+
+/* RT_DRIVER_GRAPH: the whole N-step loop is recorded once into a CUDA graph
+ * (cached per argument set) and replayed with a single launch per call.
+ * RT_DRIVER_STREAM: every kernel is launched from the host loop. */
+typedef enum { RT_DRIVER_GRAPH = 0, RT_DRIVER_STREAM = 1 } rt_driver;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int rt_version(void);
+
+/* Text for a status code. Never NULL. */
+const char* rt_status_string(int status);
+
+/* Bytes of device workspace rt_layer_forward needs for this shape.
+ * Returns 0 for invalid or unsupported arguments. */
+size_t rt_layer_workspace_bytes(int B, int N, int d, int H, int d_ff, int dtype,
+                                int schedule);
+
+/* The layer forward (paper §2.2 with the schedule of notes §4.2).
+ * Inputs : x_dev [B][N][d]; weights as in the conventions.
+ * Outputs: z_dev [B][N][d]; K_dev, V_dev position-major [N][B][d].
+ * workspace_dev: >= rt_layer_workspace_bytes(...) bytes, 256-byte aligned.
+ * Returns RT_OK once the work is enqueued on `stream`. */
+int rt_layer_forward(const void* x_dev,
+                     const void* W_q_dev, const void* W_k_dev, const void* W_v_dev,
+                     const void* W_o_dev, const void* W_1_dev, const void* W_2_dev,
+                     int B, int N, int d, int H, int d_ff,
+                     int dtype, int schedule, int driver,
+                     void* z_dev, void* K_dev, void* V_dev,
+                     void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of a
+ * workspace used by rt_layer_forward. RT_OK, RT_ERR_TIMEOUT or RT_ERR_CUDA. */
+int rt_layer_sync_status(void* workspace_dev, void* stream);
+
+/* Device bytes rt_layer_forward_host needs: the workspace of
+ * rt_layer_forward plus device copies of x, the weights, z, K and V. */
+size_t rt_layer_host_workspace_bytes(int B, int N, int d, int H, int d_ff,
+                                     int dtype, int schedule);
+
+/* End-to-end form of rt_layer_forward with HOST buffers: copies x and the
+ * weights host->device, runs the layer, copies z, K, V device->host, all
+ * enqueued on `stream` (returns once enqueued; synchronise the stream before
+ * reading the outputs). All host pointers must stay valid until then.
+ * Layouts as in rt_layer_forward. */
+int rt_layer_forward_host(const void* x_host,
+                          const void* W_q_host, const void* W_k_host, const void* W_v_host,
+                          const void* W_o_host, const void* W_1_host, const void* W_2_host,
+                          int B, int N, int d, int H, int d_ff,
+                          int dtype, int schedule, int driver,
+                          void* z_host, void* K_host, void* V_host,
+                          void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Token-embedding front end of a layer stack: x[b][n][:] = E[ids[b][n]][:].
+ * ids_dev int32 [B][N], each in [0, vocab) (out-of-range ids produce a zero
+ * row and set the error word of `workspace_dev` if it is not NULL);
+ * E_dev [vocab][d]; x_dev [B][N][d]; storage type `dtype`. */
+int rt_embed_forward(const int32_t* ids_dev, const void* E_dev, int B, int N,
+                     int vocab, int d, int dtype, void* x_dev,
+                     void* workspace_dev, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Component entry points (the same kernels rt_layer_forward runs, exposed for
+ * unit parity tests and measurement).
+ * ------------------------------------------------------------------------ */
+
+/* One block fold of notes §4.2 on caller-provided state, position-major:
+ *   Q_dev  [n_pos][B][q_stride] (query of head h at column h*d_h),
+ *   K_dev, V_dev [n_pos][B][kv_stride],
+ *   m_dev, l_dev [n_pos][B][H] fp32, o_dev [n_pos][B][H*d_h] fp32.
+ * Folds keys [k0, k0 + nk) into queries [q0, q0 + nq) (0-based positions),
+ * updating (m, l, o) in place. m is stored in log2 units scaled by
+ * log2(e)/sqrt(d_h) (m = -inf marks an empty accumulator).
+ * RT_BF16 needs d_h = 64; nk that is a multiple of 16 uses the tensor-core
+ * kernel, other nk the warp kernel. */
+int rt_block_fold(const void* Q_dev, int q_stride, const void* K_dev,
+                  const void* V_dev, int kv_stride, float* m_dev, float* l_dev,
+                  float* o_dev, int B, int H, int d_h, int q0, int nq, int k0,
+                  int nk, int dtype, void* stream);
+
+/* Batched projection of all B*N positions (queries depend only on x):
+ *   QKV_dev[n][b][0:d] = W_q rms(x[b][n]), [d:2d] = W_k rms(..), [2d:3d] = W_v rms(..)
+ * position-major [N][B][3d]. W_qkv_dev is [3d][d] (W_q; W_k; W_v stacked).
+ * scratch_dev: >= B*N*4 bytes (RT_BF16) or B*N*d*4 bytes (RT_F32). */
+int rt_project_qkv(const void* x_dev, const void* W_qkv_dev, int B, int N, int d,
+                   int dtype, void* QKV_dev, void* scratch_dev, void* stream);
+
+/* Dense product C[M][Nout] = A[M][Kd] * W[Nout][Kd]^T in bf16 with fp32
+ * accumulation on the tcgen05 tensor-core kernel; C is fp32. Kd % 64 == 0. */
+int rt_gemm_bf16(const void* A_dev, const void* W_dev, float* C_dev, int M,
+                 int Nout, int Kd, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Measurement
+ * ------------------------------------------------------------------------ */
+
+/* Number of kernels one rt_layer_forward launches for this shape (the same
+ * count whichever driver runs them); -1 for invalid arguments. */
+long rt_layer_launch_count(int B, int N, int d, int H, int d_ff, int dtype, int schedule);
+
+/* Kernel classes reported by rt_layer_forward_timed. */
+enum {
+  RT_KC_INV_RMS = 0, /* 1/rms of every input row                          */
+  RT_KC_PROJ = 1,    /* batched Q / temporary-pair projection             */
+  RT_KC_ATTEND = 2,  /* finalise a_t (blocked) or full attention (naive)  */
+  RT_KC_WO = 3,      /* a W_o^T + residual                                */
+  RT_KC_W1 = 4,      /* GELU(rms(u) W_1^T)                                */
+  RT_KC_W2 = 5,      /* h W_2^T + residual = z_t                          */
+  RT_KC_WKV = 6,     /* persistent pair rms(z_t) [W_k; W_v]^T             */
+  RT_KC_FOLD_WARP = 7, /* block fold, warp kernel                         */
+  RT_KC_FOLD_MMA = 8,  /* block fold, tensor-core kernel                  */
+  RT_KC_COUNT = 10
+};
+
+/* rt_layer_forward with the host-loop driver and a CUDA event pair recorded
+ * on `stream` around every kernel; synchronises `stream`, then writes the
+ * summed device time (ms) and the launch count of each kernel class into
+ * class_ms[0..n_classes) and class_launches[0..n_classes). For measurement;
+ * not for use inside stream capture. */
+int rt_layer_forward_timed(const void* x_dev,
+                           const void* W_q_dev, const void* W_k_dev, const void* W_v_dev,
+                           const void* W_o_dev, const void* W_1_dev, const void* W_2_dev,
+                           int B, int N, int d, int H, int d_ff, int dtype, int schedule,
+                           void* z_dev, void* K_dev, void* V_dev,
+                           void* workspace_dev, size_t workspace_bytes, void* stream,
+                           float* class_ms, int* class_launches, int n_classes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTLAYER_H */

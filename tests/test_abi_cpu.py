@@ -1,0 +1,105 @@
+"""The C ABI on the host: the library loads, exports every function the header
+declares, and its host-side logic (validation, workspace plan, launch count)
+behaves as documented. No kernel runs here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from blocked_attention_b200 import build as B
+from blocked_attention_b200 import rtlayer as R
+
+HEADER = os.path.join(B.INCLUDE, "rtlayer.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return R.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_all_exported(L):
+    names = _declared()
+    assert "rt_layer_forward" in names and len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in rtlayer.h but not exported"
+    assert set(R.EXPORTS) == set(names)
+
+
+def test_version_and_status_strings(L):
+    assert L.rt_version() >= 100
+    for s in range(-6, 1):
+        assert R.status_string(s) not in ("", "unknown status")
+    assert R.status_string(-99) == "unknown status"
+
+
+def test_workspace_plan(L):
+    bf, f32 = R.RT_BF16, R.RT_F32
+    ws = L.rt_layer_workspace_bytes
+    assert ws(512, 2048, 1024, 16, 4096, bf, 0) > 0
+    # bf16 storage needs d_h = 64
+    assert ws(2, 64, 64, 2, 256, bf, 0) == 0
+    assert ws(2, 64, 64, 2, 256, f32, 0) > 0
+    assert ws(2, 64, 64, 3, 256, f32, 0) == 0          # d % H != 0
+    assert ws(0, 64, 64, 2, 256, f32, 0) == 0
+    assert ws(2, 64, 64, 2, 256, 7, 0) == 0             # bad dtype
+    # the blocked schedule keeps (m, l, o) per position; the naive one does not
+    assert ws(8, 256, 512, 8, 1024, bf, 0) > ws(8, 256, 512, 8, 1024, bf, 1)
+    # headline: q/k~/v~ (3 x 2.1 GB) + o (4.3 GB) + m, l dominate
+    hb = ws(512, 2048, 1024, 16, 4096, bf, 0)
+    assert 10.5e9 < hb < 11.5e9
+    assert L.rt_layer_host_workspace_bytes(512, 2048, 1024, 16, 4096, bf, 0) > hb + 4 * 2.1e9
+
+
+def test_launch_count_matches_schedule(L):
+    # bf16: 2 set-up kernels + 5 per step + one fold per step t < N (lowbit(t) >= 1)
+    for N in (1, 2, 7, 64, 2048):
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0) == 2 + 5 * N + (N - 1)
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 1) == 2 + 5 * N
+    assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_F32, 0) == 2 + 8 * 8 + 7
+    assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_BF16, 0) == -1
+
+
+def _fwd(L, ptr, B=2, N=8, d=64, H=2, d_ff=256, dtype=R.RT_F32, sched=0, driver=0, ws_bytes=1 << 30,
+         ws=None):
+    p = [ctypes.c_void_p(ptr)] * 7
+    out = [ctypes.c_void_p(ptr)] * 3
+    return L.rt_layer_forward(*p, B, N, d, H, d_ff, dtype, sched, driver, *out,
+                              ctypes.c_void_p(ptr if ws is None else ws), ctypes.c_size_t(ws_bytes), None)
+
+
+def test_forward_argument_validation_happens_before_any_launch(L):
+    fake = 1 << 40                                       # never dereferenced
+    assert _fwd(L, 0) == R.RT_ERR_INVALID_ARG           # null pointers
+    assert _fwd(L, fake + 4) == R.RT_ERR_INVALID_ARG    # misaligned tensors
+    assert _fwd(L, fake, dtype=5) == R.RT_ERR_INVALID_ARG
+    assert _fwd(L, fake, driver=9) == R.RT_ERR_INVALID_ARG
+    assert _fwd(L, fake, H=3) == R.RT_ERR_INVALID_ARG
+    assert _fwd(L, fake, dtype=R.RT_BF16) == R.RT_ERR_UNSUPPORTED   # d_h = 32 in bf16
+    assert _fwd(L, fake, ws_bytes=100) == R.RT_ERR_WORKSPACE
+    assert _fwd(L, fake, ws=fake + 128) == R.RT_ERR_WORKSPACE        # workspace not 256-aligned
+
+
+def test_no_device_is_reported_not_faked(L):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    # valid arguments: the library must refuse to run rather than compute on the CPU
+    assert _fwd(L, 1 << 40) == R.RT_ERR_DEVICE
+    assert L.rt_gemm_bf16(ctypes.c_void_p(1 << 40), ctypes.c_void_p(1 << 40),
+                          ctypes.cast(ctypes.c_void_p(1 << 40), ctypes.POINTER(ctypes.c_float)),
+                          128, 128, 64, None) == R.RT_ERR_DEVICE
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(R, "_lib", None)
+    monkeypatch.setattr(R, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        R.lib()

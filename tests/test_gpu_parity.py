@@ -1,0 +1,233 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs. Bars: max|gpu-ref|/max|ref| <= 1e-4 (fp32 storage),
+<= 2e-2 (bf16 storage, fp32 accumulation), per output tensor z, K, V."""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import rtinputs  # noqa: E402
+from oracle import rt_oracle as O  # noqa: E402
+from tests.parity_util import TOL, problem, rel_err, to_device, to_np  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+LOG2E = 1.0 / math.log(2.0)
+
+
+@pytest.fixture(scope="module")
+def rt():
+    from blocked_attention_b200 import rtlayer
+    rtlayer.lib()
+    return rtlayer
+
+
+def _weights_dev(W, dtype):
+    return {k: to_device(v, dtype) for k, v in W.items()}
+
+
+def _check_layer(rt, B, N, d, H, d_ff, dtype, schedule="blocked", driver="graph", sigma=0.02, seqs=None):
+    x, W = problem(B, N, d, H, d_ff, dtype, sigma=sigma)
+    z, K, V = rt.layer_forward(to_device(x, dtype), _weights_dev(W, dtype), H, schedule=schedule, driver=driver)
+    torch.cuda.synchronize()
+    sel = list(range(B)) if seqs is None else list(seqs)
+    zr, Kr, Vr = O.rt_layer(x[sel], W, H)
+    zg = to_np(z)[sel]
+    Kg = to_np(K).transpose(1, 0, 2)[sel]
+    Vg = to_np(V).transpose(1, 0, 2)[sel]
+    errs = (rel_err(zg, zr), rel_err(Kg, Kr), rel_err(Vg, Vr))
+    assert max(errs) <= TOL[dtype], errs
+    return errs, (z, K, V)
+
+
+# --------------------------------------------------------------------------
+# components
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("M,Nout,Kd", [(128, 256, 64), (300, 192, 128), (64, 1024, 512), (1000, 96, 320),
+                                       (2048, 3072, 1024), (1, 32, 64)])
+def test_tcgen05_gemm_matches_fp64_matmul(rt, M, Nout, Kd):
+    rng = np.random.default_rng(M + Nout + Kd)
+    A = rtinputs.to_grid(rng.standard_normal((M, Kd)), "bf16")
+    W = rtinputs.to_grid(rng.standard_normal((Nout, Kd)), "bf16")
+    C = rt.gemm_bf16(to_device(A, "bf16"), to_device(W, "bf16"))
+    torch.cuda.synchronize()
+    ref = A @ W.T
+    assert rel_err(to_np(C), ref) < 1e-5
+
+
+@pytest.mark.parametrize("dtype,B,N,d", [("bf16", 3, 37, 128), ("bf16", 2, 300, 512), ("f32", 2, 64, 64),
+                                         ("f32", 3, 17, 96)])
+def test_batched_projection_matches_oracle(rt, dtype, B, N, d):
+    x, W = problem(B, N, d, 2 if d % 64 == 0 else 3, 2 * d, dtype)
+    Wqkv = np.concatenate([W["W_q"], W["W_k"], W["W_v"]], axis=0)
+    qkv = rt.project_qkv(to_device(x, dtype), to_device(Wqkv, dtype))
+    torch.cuda.synchronize()
+    ref = O.rms(x) @ Wqkv.T                      # [B, N, 3d]
+    got = to_np(qkv).transpose(1, 0, 2)          # position-major -> [B, N, 3d]
+    assert rel_err(got, ref) <= (5e-3 if dtype == "bf16" else 1e-5)
+
+
+@pytest.mark.parametrize("dtype,nk,nq,init_empty", [
+    ("bf16", 1, 1, False), ("bf16", 2, 2, True), ("bf16", 8, 5, False),      # warp kernel
+    ("bf16", 16, 16, False), ("bf16", 32, 7, False), ("bf16", 64, 64, True),  # tensor-core kernel
+    ("bf16", 256, 100, False), ("bf16", 1024, 130, False),
+    ("f32", 3, 4, False), ("f32", 16, 16, True), ("f32", 64, 33, False)])
+def test_block_fold_matches_oracle(rt, dtype, nk, nq, init_empty):
+    B, H, dh = 3, 2, 64 if dtype == "bf16" else 32
+    d = H * dh
+    npos = nk + nq + 2
+    rng = np.random.default_rng(nk * 7 + nq)
+    Q = rtinputs.to_grid(rng.standard_normal((npos, B, d)), dtype)
+    Kc = rtinputs.to_grid(rng.standard_normal((npos, B, d)), dtype)
+    Vc = rtinputs.to_grid(rng.standard_normal((npos, B, d)), dtype)
+    scale = 1.0 / math.sqrt(dh)
+    # prior accumulator state of the queries (natural-log units for the oracle)
+    m0 = rng.standard_normal((npos, B, H)) * 2
+    l0 = rng.uniform(0.5, 3.0, (npos, B, H))
+    o0 = rng.standard_normal((npos, B, d))
+    if init_empty:
+        m0[:] = -np.inf; l0[:] = 0; o0[:] = 0
+    k0, q0 = 1, 1 + nk
+    mg = torch.tensor((m0 * LOG2E).astype(np.float32), device="cuda")
+    lg = torch.tensor(l0.astype(np.float32), device="cuda")
+    og = torch.tensor(o0.astype(np.float32), device="cuda")
+    rt.block_fold(to_device(Q, dtype), to_device(Kc, dtype), to_device(Vc, dtype), mg, lg, og, H, dh, q0, nq, k0, nk)
+    torch.cuda.synchronize()
+    # oracle, per (b, h)
+    qh = Q[q0:q0 + nq].reshape(nq, B, H, dh).transpose(1, 2, 0, 3)     # [B,H,nq,dh]
+    kh = Kc[k0:k0 + nk].reshape(nk, B, H, dh).transpose(1, 2, 0, 3)
+    vh = Vc[k0:k0 + nk].reshape(nk, B, H, dh).transpose(1, 2, 0, 3)
+    mr = m0[q0:q0 + nq].transpose(1, 2, 0).copy()
+    lr = l0[q0:q0 + nq].transpose(1, 2, 0).copy()
+    orr = o0[q0:q0 + nq].reshape(nq, B, H, dh).transpose(1, 2, 0, 3).copy()
+    mr, lr, orr = O.block_fold(qh, kh, vh, mr, lr, orr, scale)
+    m_got = to_np(mg)[q0:q0 + nq].transpose(1, 2, 0) / LOG2E
+    l_got = to_np(lg)[q0:q0 + nq].transpose(1, 2, 0)
+    o_got = to_np(og)[q0:q0 + nq].reshape(nq, B, H, dh).transpose(1, 2, 0, 3)
+    tol = 2e-3 if dtype == "bf16" else 1e-5      # bf16 P in the PV product
+    assert np.max(np.abs(m_got - mr)) < 1e-4 * max(1.0, np.max(np.abs(mr)))
+    # compare normalised outputs and the normaliser
+    assert rel_err(o_got / l_got[..., None], orr / lr[..., None]) < tol
+    assert rel_err(l_got, lr) < tol
+    # rows outside the query range are untouched
+    untouched = np.ones(npos, bool); untouched[q0:q0 + nq] = False
+    np.testing.assert_array_equal(to_np(og)[untouched], o0[untouched].astype(np.float32))
+
+
+# --------------------------------------------------------------------------
+# the layer
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("schedule", ["blocked", "naive"])
+@pytest.mark.parametrize("driver", ["graph", "stream"])
+def test_layer_f32_tiny_config(rt, schedule, driver):
+    # B=2 sequences, N=64, d=64, H=2 heads of 32, d_ff=256, fp32
+    _check_layer(rt, 2, 64, 64, 2, 256, "f32", schedule=schedule, driver=driver)
+
+
+@pytest.mark.parametrize("B,N,d,H,d_ff", [(3, 37, 128, 2, 256), (5, 100, 192, 3, 320), (1, 1, 64, 1, 64),
+                                          (2, 2, 64, 1, 128), (130, 20, 128, 2, 256)])
+def test_layer_bf16_ragged_shapes(rt, B, N, d, H, d_ff):
+    _check_layer(rt, B, N, d, H, d_ff, "bf16")
+
+
+def test_layer_f32_peaky_attention(rt):
+    _check_layer(rt, 2, 48, 64, 2, 128, "f32", sigma=0.2)
+
+
+def test_layer_bf16_peaky_attention(rt):
+    _check_layer(rt, 2, 70, 128, 2, 256, "bf16", sigma=0.1)
+
+
+@pytest.mark.parametrize("schedule", ["blocked", "naive"])
+def test_layer_bf16_config_B64_N1024_d512(rt, schedule):
+    # B=64, N=1024, d=512, H=8 heads of 64, d_ff=2048; sequences sampled for the oracle
+    _check_layer(rt, 64, 1024, 512, 8, 2048, "bf16", schedule=schedule, seqs=[0, 31, 63])
+
+
+def test_blocked_equals_naive_on_gpu(rt):
+    B, N, d, H, d_ff = 4, 200, 128, 2, 256
+    x, W = problem(B, N, d, H, d_ff, "bf16")
+    xd, Wd = to_device(x, "bf16"), _weights_dev(W, "bf16")
+    a = rt.layer_forward(xd, Wd, H, schedule="blocked")
+    b = rt.layer_forward(xd, Wd, H, schedule="naive")
+    torch.cuda.synchronize()
+    for u, v in zip(a, b):
+        assert rel_err(to_np(u), to_np(v)) < 1e-2
+
+
+def test_prefix_property_on_gpu(rt):
+    B, N, d, H, d_ff = 3, 90, 128, 2, 256
+    x, W = problem(B, N, d, H, d_ff, "f32")
+    Wd = _weights_dev(W, "f32")
+    z, K, V = rt.layer_forward(to_device(x, "f32"), Wd, H)
+    zp, Kp, Vp = rt.layer_forward(to_device(x[:, :50].copy(), "f32"), Wd, H)
+    torch.cuda.synchronize()
+    assert rel_err(to_np(zp), to_np(z)[:, :50]) < 1e-6
+    assert rel_err(to_np(Kp), to_np(K)[:50]) < 1e-6
+
+
+def test_graph_replay_is_deterministic_and_matches_stream(rt):
+    B, N, d, H, d_ff = 8, 130, 256, 4, 512
+    x, W = problem(B, N, d, H, d_ff, "bf16")
+    xd, Wd = to_device(x, "bf16"), _weights_dev(W, "bf16")
+    ws = rt.alloc_workspace(rt.workspace_bytes(B, N, d, H, d_ff))
+    outs = [torch.empty((B, N, d), dtype=torch.bfloat16, device="cuda"),
+            torch.empty((N, B, d), dtype=torch.bfloat16, device="cuda"),
+            torch.empty((N, B, d), dtype=torch.bfloat16, device="cuda")]
+    rt.layer_forward(xd, Wd, H, out=outs, workspace=ws, driver="graph")
+    first = [t.clone() for t in outs]
+    rt.layer_forward(xd, Wd, H, out=outs, workspace=ws, driver="graph")     # cached graph replay
+    assert rt.sync_status(ws) == 0
+    for a, b in zip(first, outs):
+        assert torch.equal(a, b)
+    s = rt.layer_forward(xd, Wd, H, driver="stream")
+    torch.cuda.synchronize()
+    for a, b in zip(first, s):
+        assert torch.equal(a, b)
+
+
+def test_host_buffer_entry_point(rt):
+    B, N, d, H, d_ff = 4, 40, 128, 2, 256
+    x, W = problem(B, N, d, H, d_ff, "bf16")
+    xh = to_device(x, "bf16", device="cpu").pin_memory()
+    Wh = {k: to_device(v, "bf16", device="cpu").pin_memory() for k, v in W.items()}
+    out = [torch.empty((B, N, d), dtype=torch.bfloat16).pin_memory(),
+           torch.empty((N, B, d), dtype=torch.bfloat16).pin_memory(),
+           torch.empty((N, B, d), dtype=torch.bfloat16).pin_memory()]
+    ws = rt.alloc_workspace(rt.host_workspace_bytes(B, N, d, H, d_ff))
+    rt.layer_forward_host(xh, Wh, H, out, ws)
+    torch.cuda.synchronize()
+    zr, Kr, Vr = O.rt_layer(x, W, H)
+    assert rel_err(to_np(out[0]), zr) < TOL["bf16"]
+    assert rel_err(to_np(out[1]).transpose(1, 0, 2), Kr) < TOL["bf16"]
+
+
+def test_stack_of_layers_with_embedding(rt):
+    # reduced stack: vocab 500, d=128 (2 heads of 64), d_ff=256, 3 layers, B=3, N=33
+    vocab, d, H, d_ff, B, N, L = 500, 128, 2, 256, 3, 33, 3
+    E = rtinputs.embedding(0, vocab, d, dtype="bf16")
+    ids = np.stack([rtinputs.token_ids(0, b, N, vocab) for b in range(B)])
+    layers = [rtinputs.weights(0, d, d_ff, dtype="bf16", layer=i) for i in range(L)]
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    x = rt.embed_forward(torch.tensor(ids, device="cuda"), to_device(E, "bf16"), workspace=ws)
+    kv = []
+    for W in layers:
+        x, K, V = rt.layer_forward(x, _weights_dev(W, "bf16"), H)
+        kv.append((K, V))
+    torch.cuda.synchronize()
+    assert rt.sync_status(ws) == 0
+    zr, kvr = O.rt_stack(ids, E, layers, H)
+    assert rel_err(to_np(x), zr) < TOL["bf16"]
+    for (K, V), (Kr, Vr) in zip(kv, kvr):
+        assert rel_err(to_np(K).transpose(1, 0, 2), Kr) < TOL["bf16"]
+
+
+def test_embedding_out_of_range_id_is_reported(rt):
+    E = to_device(rtinputs.embedding(0, 10, 64, dtype="bf16"), "bf16")
+    ids = torch.tensor([[1, 2, 10]], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    x = rt.embed_forward(ids, E, workspace=ws)
+    assert rt.sync_status(ws) == rt.RT_ERR_INVALID_ARG
+    assert torch.count_nonzero(x[0, 2]) == 0
