@@ -66,6 +66,27 @@ def parse():
 
 
 # --------------------------------------------------------------------------
+# multi-rank helpers (replicas: no collective on the data path)
+# --------------------------------------------------------------------------
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank scalar (the device-timed step time) over all ranks."""
+    import torch
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_input_seed(seed: int, rank: int) -> int:
+    """Each replica draws its own batch."""
+    return 1000 + 1000 * seed + rank
+
+
+def aggregate_tokens_per_s(world: int, B: int, N: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes B*N tokens per step."""
+    return world * B * N / (ms_per_step / 1e3)
+
+
+# --------------------------------------------------------------------------
 # clocks during the timed region
 # --------------------------------------------------------------------------
 class ClockSampler:
@@ -139,7 +160,7 @@ def lowbit(t: int) -> int:
     return t & -t
 
 
-def algorithmic_work(cfg: dict) -> dict:
+def algorithmic_work(cfg: dict, schedule: str = "blocked") -> dict:
     """{class: ("tensor", flops) | ("hbm", bytes)} summed over one forward."""
     B, N, d, H, dff = cfg["B"], cfg["N"], cfg["d"], cfg["H"], cfg["d_ff"]
     w = {
@@ -152,6 +173,10 @@ def algorithmic_work(cfg: dict) -> dict:
         # q, k~, v~ of position t (bf16), (m, l, o) of query t read (fp32), a_t written (bf16)
         "attend": ("hbm", float(N) * B * (6 * d + 4 * d + 8 * H + 2 * d)),
     }
+    if schedule == "naive":
+        # query t reads the t-1 persistent pairs (k, v bf16) plus its own q, k~, v~; writes a_t
+        w["attend"] = ("hbm", float(B) * (4 * d * N * (N - 1) / 2 + N * 8 * d))
+        return w
     warp_b, mma_b = 0.0, 0.0
     for t in range(1, N):
         lb = lowbit(t)
@@ -253,7 +278,7 @@ def main():
     Wnp = rtinputs.weights(args.seed, d, dff, dtype="bf16")
     W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16) for k, v in Wnp.items()}
     g = torch.Generator(device=dev)
-    g.manual_seed(1000 + rank)
+    g.manual_seed(rank_input_seed(args.seed, rank))
     x = torch.randn((Bsz, N, d), generator=g, device=dev, dtype=torch.bfloat16)
     z = torch.empty_like(x)
     K = torch.empty((N, Bsz, d), dtype=torch.bfloat16, device=dev)
@@ -288,18 +313,16 @@ def main():
     clocks = sampler.stop()
     ms_total = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+        ms_total = max_over_ranks(ms_total, dist, dev)
     st = R.sync_status(ws)
     if st != 0:
         raise RuntimeError(f"device error in the timed region: {R.status_string(st)}")
     ms_step = ms_total / args.steps
-    value = world * Bsz * N / (ms_step / 1e3)
+    value = aggregate_tokens_per_s(world, Bsz, N, ms_step)
 
     # per-kernel device time: one extra forward with CUDA events around every kernel
     classes = R.layer_forward_timed(x, W, H, (z, K, V), ws, schedule=args.schedule)
-    work = algorithmic_work(cfg)
+    work = algorithmic_work(cfg, args.schedule)
     peaks = measured_peaks()
     kernels = {}
     for name, (kms, launches) in classes.items():
@@ -351,13 +374,11 @@ def main():
         torch.cuda.synchronize()
         e_ms = h0.elapsed_time(h1)
         if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+            e_ms = max_over_ranks(e_ms, dist, dev)
         e_ms /= args.e2e_steps
         h2d = xh.numel() * 2 + sum(v.numel() * 2 for v in Wh.values())
         d2h = sum(t.numel() * 2 for t in outh)
-        e2e = {"value": world * Bsz * N / (e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e_ms,
+        e2e = {"value": aggregate_tokens_per_s(world, Bsz, N, e_ms), "unit": "tokens/s", "ms_per_step": e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "path": "rt_layer_forward_host (pinned host buffers; H2D, forward, D2H in the timed region)"}
 

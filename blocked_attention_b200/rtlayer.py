@@ -70,7 +70,7 @@ def lib() -> ctypes.CDLL:
     L.rt_embed_forward.restype = i
     L.rt_embed_forward.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp]
     L.rt_block_fold.restype = i
-    L.rt_block_fold.argtypes = [vp, i, vp, vp, i, fp, fp, fp] + [i] * 8 + [i, vp]
+    L.rt_block_fold.argtypes = [vp, i, vp, vp, i, fp, fp, fp] + [i] * 7 + [i, vp]
     L.rt_project_qkv.restype = i
     L.rt_project_qkv.argtypes = [vp, vp, i, i, i, i, vp, vp, vp]
     L.rt_gemm_bf16.restype = i

@@ -103,3 +103,21 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(R, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         R.lib()
+
+
+def _param_counts():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(rt_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_header(L):
+    counts = _param_counts()
+    assert len(counts) == len(R.EXPORTS)
+    for name, n in counts.items():
+        fn = getattr(L, name)
+        got = len(fn.argtypes) if fn.argtypes is not None else 0
+        assert got == n, f"{name}: binding declares {got} arguments, header {n}"
