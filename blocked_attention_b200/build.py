@@ -43,7 +43,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         return LIB
     cmd = [nvcc_path(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "--shared",
            "-Xcompiler", "-fPIC", "-I", INCLUDE, "-o", LIB + ".tmp",
-           os.path.join(CSRC, "rt_api.cu")]
+           *sorted(glob.glob(os.path.join(CSRC, "*.cu")))]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     if extra:

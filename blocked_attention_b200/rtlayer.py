@@ -27,7 +27,7 @@ WEIGHT_NAMES = ("W_q", "W_k", "W_v", "W_o", "W_1", "W_2")
 EXPORTS = ("rt_version", "rt_status_string", "rt_layer_workspace_bytes", "rt_layer_forward",
            "rt_layer_sync_status", "rt_layer_host_workspace_bytes", "rt_layer_forward_host",
            "rt_embed_forward", "rt_block_fold", "rt_project_qkv", "rt_gemm_bf16",
-           "rt_layer_launch_count", "rt_layer_forward_timed")
+           "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma")
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.rt_layer_forward_timed.restype = i
     L.rt_layer_forward_timed.argtypes = [vp] * 7 + [i] * 7 + [vp] * 4 + [sz, vp, fp,
                                                                          ctypes.POINTER(ctypes.c_int), i]
+    L.rt_project_qkv_noalloc.restype = i
+    L.rt_project_qkv_noalloc.argtypes = [vp, vp, i, i, i, vp, vp]
     _lib = L
     return L
 
@@ -232,6 +234,15 @@ def project_qkv(x: torch.Tensor, W_qkv: torch.Tensor, stream=None):
                               _stream(stream))
     _check("rt_project_qkv", rc)
     return qkv
+
+
+def project_qkv_noalloc(x: torch.Tensor, W_qkv: torch.Tensor, out: torch.Tensor, stream=None):
+    """rt_project_qkv_noalloc: bf16 projection into the caller's `out`
+    ([N, B, 3d]) with the library's fixed scratch array (B*N <= 1048576)."""
+    B, N, d = x.shape
+    rc = lib().rt_project_qkv_noalloc(_ptr(x), _ptr(W_qkv), B, N, d, _ptr(out), _stream(stream))
+    _check("rt_project_qkv_noalloc", rc)
+    return out
 
 
 def gemm_bf16(A: torch.Tensor, W: torch.Tensor, stream=None):

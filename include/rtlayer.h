@@ -163,6 +163,25 @@ int rt_project_qkv(const void* x_dev, const void* W_qkv_dev, int B, int N, int d
 int rt_gemm_bf16(const void* A_dev, const void* W_dev, float* C_dev, int M,
                  int Nout, int Kd, void* stream);
 
+/* rt_project_qkv for RT_BF16 storage without caller scratch: the per-row
+ * 1/rms values live in a fixed array inside the library, so the call needs no
+ * device memory beyond x_dev, W_qkv_dev and QKV_dev (same layouts as
+ * rt_project_qkv). The paper has no counterpart; this exists for callers that
+ * cannot allocate device memory where they call it (runtimes that plan all
+ * device memory at start-up, code running while another framework's caching
+ * allocator holds the free memory, latency-critical loops).
+ *   - Limit: B*N <= 1048576 rows (a 4 MiB array that every GPU loading the
+ *     library keeps until exit); larger sizes return RT_ERR_WORKSPACE before
+ *     anything is enqueued. d % 64 == 0.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address with cudaGetSymbolAddress; make that first call
+ *     before any stream capture.
+ *   - All calls share the array and overwrite the rows they use before
+ *     reading them; calls that overlap on the GPU race on it.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+int rt_project_qkv_noalloc(const void* x_dev, const void* W_qkv_dev, int B, int N,
+                           int d, void* QKV_dev, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Measurement
  * ------------------------------------------------------------------------ */
