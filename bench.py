@@ -62,6 +62,16 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--stack", action="store_true",
+                    help="6-layer stack with token embedding (B=64 N=2048 d=1280 H=20x64 d_ff=5120)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="sequence-length sweep, blocked vs naive (B=32 d=1024 H=16x64 d_ff=4096)")
+    ap.add_argument("--sweep-n", default="512,1024,2048,4096,8192,16384")
+    ap.add_argument("--profile-case", choices=["step", "fold"],
+                    help="run one small case for an ncu capture and exit: 'step' = one host-loop forward at "
+                         "B=512 N=64 d=1024 (the per-step GEMM shapes of the headline); 'fold' = one block fold "
+                         "of --lb keys into --lb queries at B=64 H=16 (position-major, larger than L2)")
+    ap.add_argument("--lb", type=int, default=1024)
     return ap.parse_args()
 
 
@@ -178,12 +188,7 @@ def algorithmic_work(cfg: dict, schedule: str = "blocked") -> dict:
         w["attend"] = ("hbm", float(B) * (4 * d * N * (N - 1) / 2 + N * 8 * d))
         return w
     warp_b, mma_b = 0.0, 0.0
-    for t in range(1, N):
-        lb = lowbit(t)
-        nq = min(lb, N - t)
-        init = (t == lb)
-        per_q = 2 * d + (4 * d if init else 8 * d) + (8 * H if init else 16 * H)   # q read; o, m, l (read+)write
-        by = B * (nq * per_q + lb * 4 * d)                                          # + keys' k, v read
+    for lb, (by, fl) in fold_level_work(cfg).items():
         if lb >= 16:
             mma_b += by
         else:
@@ -191,6 +196,25 @@ def algorithmic_work(cfg: dict, schedule: str = "blocked") -> dict:
     w["fold_warp"] = ("hbm", warp_b)
     w["fold_mma"] = ("hbm", mma_b)
     return w
+
+
+def fold_level_work(cfg: dict) -> dict:
+    """{block size: (algorithmic bytes, FLOPs)} of the folds of one forward.
+    Bytes per fold: every key's k, v (bf16) read once; every query's q (bf16)
+    read and its o (fp32), m, l read and written -- written only for the first
+    fold into a query (t a power of two). FLOPs: QK^T and PV, 4 d per pair."""
+    B, N, d, H = cfg["B"], cfg["N"], cfg["d"], cfg["H"]
+    out = {}
+    for t in range(1, N):
+        lb = lowbit(t)
+        nq = min(lb, N - t)
+        init = (t == lb)
+        per_q = 2 * d + (4 * d if init else 8 * d) + (8 * H if init else 16 * H)
+        by = B * (nq * per_q + lb * 4 * d)
+        fl = 4.0 * B * d * nq * lb
+        b0, f0 = out.get(lb, (0.0, 0.0))
+        out[lb] = (b0 + by, f0 + fl)
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -251,6 +275,100 @@ def workload_config(args, cfg, world) -> dict:
 
 
 # --------------------------------------------------------------------------
+STACK = dict(B=64, N=2048, d=1280, H=20, d_ff=5120, layers=6, vocab=32000)
+SWEEP = dict(B=32, d=1024, H=16, d_ff=4096)
+
+
+def run_stack(args, R, torch, rtinputs):
+    """Tokens/s of the 6-layer stack: embedding gather, then 6 layer forwards,
+    each layer's z feeding the next (one step = the whole stack)."""
+    c = STACK
+    dev = torch.device("cuda", 0)
+    Bsz, N, d, H, dff, L = c["B"], c["N"], c["d"], c["H"], c["d_ff"], c["layers"]
+    E = torch.randn((c["vocab"], d), device=dev, dtype=torch.bfloat16) * 0.02
+    ids = torch.randint(0, c["vocab"], (Bsz, N), device=dev, dtype=torch.int32)
+    Ws = [{k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
+           for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16", layer=i).items()} for i in range(L)]
+    xs = [torch.empty((Bsz, N, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    KV = [(torch.empty((N, Bsz, d), dtype=torch.bfloat16, device=dev),
+           torch.empty((N, Bsz, d), dtype=torch.bfloat16, device=dev)) for _ in range(L)]
+    ws = R.alloc_workspace(R.workspace_bytes(Bsz, N, d, H, dff), dev)
+
+    def step():
+        x0 = R.embed_forward(ids, E, workspace=ws)
+        xs[0].copy_(x0)
+        for i in range(L):
+            R.layer_forward(xs[i % 2], Ws[i], H, out=(xs[(i + 1) % 2], KV[i][0], KV[i][1]), workspace=ws)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    assert R.sync_status(ws) == 0
+    print(json.dumps({"metric": "RT 6-layer stack prefill tokens/s", "value": Bsz * N / (ms / 1e3),
+                      "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+                      "dtype": "bf16", "data": "synthetic", "config": {"workload": "6-layer RT stack", **c}}),
+          flush=True)
+
+
+def run_sweep(args, R, torch):
+    """Sequence-length sweep, blocked vs naive schedule: latency per forward."""
+    c = SWEEP
+    dev = torch.device("cuda", 0)
+    Bsz, d, H, dff = c["B"], c["d"], c["H"], c["d_ff"]
+    W = {k: (torch.randn(v, device=dev) * 0.02).to(torch.bfloat16) for k, v in
+         {"W_q": (d, d), "W_k": (d, d), "W_v": (d, d), "W_o": (d, d), "W_1": (dff, d), "W_2": (d, dff)}.items()}
+    for N in [int(v) for v in args.sweep_n.split(",")]:
+        x = torch.randn((Bsz, N, d), device=dev, dtype=torch.bfloat16)
+        out = (torch.empty_like(x), torch.empty((N, Bsz, d), dtype=torch.bfloat16, device=dev),
+               torch.empty((N, Bsz, d), dtype=torch.bfloat16, device=dev))
+        for sched in ("blocked", "naive"):
+            ws = R.alloc_workspace(R.workspace_bytes(Bsz, N, d, H, dff, torch.bfloat16, sched), dev)
+            steps = 1 if (sched == "naive" and N >= 8192) else 2
+            R.layer_forward(x, W, H, schedule=sched, out=out, workspace=ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                R.layer_forward(x, W, H, schedule=sched, out=out, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / steps
+            assert R.sync_status(ws) == 0
+            print(json.dumps({"sweep": True, "N": N, "schedule": sched, "ms_per_forward": ms,
+                              "tokens_per_s": Bsz * N / (ms / 1e3), **c}), flush=True)
+            del ws
+            torch.cuda.empty_cache()
+
+
+def run_profile_case(args, R, torch, rtinputs):
+    dev = torch.device("cuda", 0)
+    if args.profile_case == "step":
+        B, N, d, H, dff = 512, 64, 1024, 16, 4096
+        W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
+             for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16").items()}
+        x = torch.randn((B, N, d), device=dev, dtype=torch.bfloat16)
+        z, _, _ = R.layer_forward(x, W, H, driver="stream")
+    else:
+        LB, B, H, dh = args.lb, 64, 16, 64
+        d = H * dh
+        Q = torch.randn((2 * LB, B, 3 * d), device=dev, dtype=torch.bfloat16)
+        Kc = torch.randn((2 * LB, B, d), device=dev, dtype=torch.bfloat16)
+        Vc = torch.randn((2 * LB, B, d), device=dev, dtype=torch.bfloat16)
+        m = torch.zeros((2 * LB, B, H), device=dev)
+        l = torch.ones((2 * LB, B, H), device=dev)
+        z = torch.zeros((2 * LB, B, d), device=dev)
+        R.block_fold(Q, Kc, Vc, m, l, z, H, dh, LB, LB, 0, LB)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": args.profile_case, "ok": bool(torch.isfinite(z.float()).all())}))
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -268,6 +386,12 @@ def main():
     import rtinputs
 
     torch.cuda.set_device(local)
+    if args.profile_case:
+        run_profile_case(args, R, torch, rtinputs)
+        return
+    if args.stack or args.sweep:
+        (run_stack(args, R, torch, rtinputs) if args.stack else run_sweep(args, R, torch))
+        return
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
@@ -324,8 +448,15 @@ def main():
     classes = R.layer_forward_timed(x, W, H, (z, K, V), ws, schedule=args.schedule)
     work = algorithmic_work(cfg, args.schedule)
     peaks = measured_peaks()
-    kernels = {}
+    kernels, fold_levels = {}, {}
+    lvl_work = fold_level_work(cfg) if args.schedule == "blocked" else {}
     for name, (kms, launches) in classes.items():
+        if name.startswith("fold_lb"):
+            lb = int(name[7:])
+            by, fl = lvl_work.get(lb, (0.0, 0.0))
+            fold_levels[lb] = {"ms_total": round(kms, 3), "launches": launches,
+                               "GB/s": by / (kms / 1e3) / 1e9, "TFLOP/s": fl / (kms / 1e3) / 1e12}
+            continue
         kind, amount = work.get(name, ("hbm", 0.0))
         per_launch_ms = kms / launches
         per_launch = amount / launches
@@ -400,7 +531,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(args, cfg, world),
-        "roofline": roofline, "step_roofline": step_roof, "kernels": kernels,
+        "roofline": roofline, "step_roofline": step_roof, "kernels": kernels, "fold_levels": fold_levels,
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": R.launch_count(Bsz, N, d, H, dff, torch.bfloat16, args.schedule) * args.steps,
         "clocks": clocks,

@@ -24,6 +24,7 @@
 #include "../../include/rtlayer.h"
 #include "rt_attn.cuh"
 #include "rt_common.cuh"
+#include "rt_fold_tc.cuh"
 #include "rt_gemm_tc.cuh"
 #include "rt_simt.cuh"
 
@@ -39,6 +40,25 @@ typedef __nv_bfloat16 bf16;
   } while (0)
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Launch with programmatic stream serialisation: the kernel may start while the
+// previous kernel in the stream runs; every kernel calls pdl_wait() before it
+// reads its predecessor's outputs.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------------------
 // device set-up
@@ -97,6 +117,9 @@ static int device_setup(DevState** out) {
         set_tc_attrs_epi<EPI_WO>() != cudaSuccess || set_tc_attrs_epi<EPI_W1>() != cudaSuccess ||
         set_tc_attrs_epi<EPI_W2>() != cudaSuccess || set_tc_attrs_epi<EPI_WKV>() != cudaSuccess)
       return RT_ERR_CUDA;
+    if (cudaFuncSetAttribute(k_fold_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)FoldTcCfg::SMEM_BYTES) != cudaSuccess)
+      return RT_ERR_CUDA;
     if (cudaStreamCreateWithFlags(&ds.capture, cudaStreamNonBlocking) != cudaSuccess) return RT_ERR_CUDA;
     ds.ready = true;
   }
@@ -117,6 +140,19 @@ static bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map over a position-major [npos][B][stride] buffer: box of
+// 128 positions x one sequence x 64 elements (one head), 128-byte swizzle.
+static bool make_tmap_pm(CUtensorMap* m, const void* base, uint64_t stride, uint64_t B, uint64_t npos) {
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (stride * 2) % 16 != 0) return false;
+  cuuint64_t dims[3] = {stride, B, npos};
+  cuuint64_t strides[2] = {stride * 2, stride * 2 * B};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Output-tile width: the widest tile that still gives >= 120 tiles.
 static int choose_bn(int M, int N) {
   const long ntm = (M + 127) / 128;
@@ -125,15 +161,45 @@ static int choose_bn(int M, int N) {
   return 32;
 }
 
+// Per-step GEMMs (M = B rows): 128-wide output tiles; when that gives few
+// tiles, split K (power of two, >= 4 k-blocks per split) towards ~128 CTAs.
+struct TileCfg {
+  int bn, splits;
+};
+static TileCfg choose_tiles(int M, int N, int K, bool allow_split) {
+  if (!allow_split) return {choose_bn(M, N), 1};
+  const long ntm = (M + 127) / 128;
+  const int bn = (N % 128 == 0) ? 128 : 64;
+  const long mn = ntm * ((N + bn - 1) / bn);
+  if (mn >= 120) return {choose_bn(M, N), 1};
+  const int nkb = K / 64;
+  int splits = 1;
+  while (mn * splits * 2 <= 160 && nkb % (splits * 2) == 0 && nkb / (splits * 2) >= 4) splits *= 2;
+  return {bn, splits};
+}
+// Split-K measured slower at M = 512 (the last-CTA reduction lengthens the
+// per-step critical path), so the layer uses unsplit tiles.
+static constexpr bool kLayerSplitK = false;
+// The tcgen05 fold beat the mma.sync fold only from block size 1024 up.
+static constexpr int kFoldTcMinBlock = 1024;
+static size_t split_part_floats(int M, int N, const TileCfg& c) {
+  if (c.splits <= 1) return 0;
+  const size_t ntm = (M + 127) / 128, ntn = (N + c.bn - 1) / c.bn;
+  return (size_t)c.splits * ntm * 128 * ntn * c.bn;
+}
+static size_t split_tiles(int M, int N, const TileCfg& c) {
+  return (size_t)((M + 127) / 128) * ((N + c.bn - 1) / c.bn);
+}
+
 template <int BN, int EPI>
 static cudaError_t launch_tc_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
                                 const EpiParams& p, unsigned* err, int sms, cudaStream_t st) {
   constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   using C = GemmCfg<BN, STAGES>;
-  const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN);
+  const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN) * (p.splits > 1 ? p.splits : 1);
   const int grid = (int)std::min<long>(tiles, sms);
-  k_gemm_tc<BN, STAGES, EPI><<<grid, 192, C::SMEM_BYTES, st>>>(ta, tb, M, N, K, p, err);
-  return cudaGetLastError();
+  return launch_pdl(k_gemm_tc<BN, STAGES, EPI>, dim3(grid), dim3(192), C::SMEM_BYTES, st, ta, tb, M, N, K, p,
+                    err);
 }
 
 template <int EPI>
@@ -176,7 +242,8 @@ struct Plan {
   Shape s;
   size_t esz;
   size_t off_err, off_qkv, off_m, off_l, off_o, off_inv, off_xr, off_wqkv, off_a, off_u32, off_u16, off_ru,
-      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, total;
+      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, off_part, off_cnt, cnt_bytes, total;
+  TileCfg t_wo, t_w1, t_w2, t_wkv;
 };
 
 static Plan make_plan(const Shape& s) {
@@ -210,6 +277,19 @@ static Plan make_plan(const Shape& s) {
   if (s.dtype == RT_F32) P.off_rz = take(B * d * 4);
   P.off_ssq_u = take((d / 32 + 1) * B * 4);
   P.off_ssq_z = take((d / 32 + 1) * B * 4);
+  if (s.dtype == RT_BF16) {
+    P.t_wo = choose_tiles(s.B, s.d, s.d, kLayerSplitK);
+    P.t_w1 = choose_tiles(s.B, s.d_ff, s.d, kLayerSplitK);
+    P.t_w2 = choose_tiles(s.B, s.d, s.d_ff, kLayerSplitK);
+    P.t_wkv = choose_tiles(s.B, 2 * s.d, s.d, kLayerSplitK);
+    const size_t part = std::max(std::max(split_part_floats(s.B, s.d, P.t_wo), split_part_floats(s.B, s.d_ff, P.t_w1)),
+                                 std::max(split_part_floats(s.B, s.d, P.t_w2), split_part_floats(s.B, 2 * s.d, P.t_wkv)));
+    const size_t cnt = std::max(std::max(split_tiles(s.B, s.d, P.t_wo), split_tiles(s.B, s.d_ff, P.t_w1)),
+                                std::max(split_tiles(s.B, s.d, P.t_w2), split_tiles(s.B, 2 * s.d, P.t_wkv)));
+    P.off_part = take(std::max<size_t>(part, 1) * 4);
+    P.cnt_bytes = cnt * 4;
+    P.off_cnt = take(P.cnt_bytes);
+  }
   P.total = off;
   return P;
 }
@@ -224,8 +304,15 @@ struct Ptrs {
 // ---------------------------------------------------------------------------
 enum KernelClass {
   KC_INV_RMS = 0, KC_PROJ, KC_ATTEND, KC_WO, KC_W1, KC_W2, KC_WKV, KC_FOLD_WARP, KC_FOLD_MMA, KC_NORM,
-  KC_COUNT
+  KC_FOLD_LEVEL0 = 16,   // + log2(block size): per-level fold timing
+  KC_COUNT = 32
 };
+
+static int log2_int(int v) {
+  int r = 0;
+  while (v > 1) { v >>= 1; ++r; }
+  return r;
+}
 
 struct Timer {
   std::vector<cudaEvent_t> pool;
@@ -266,23 +353,38 @@ struct TimedScope {
 // ---------------------------------------------------------------------------
 template <class T>
 static cudaError_t launch_fold(const T* Q, int q_stride, const T* K, const T* V, int kv_stride, float* m,
-                               float* l, float* o, int B, int H, int dh, int q0, int nq, int k0, int nk,
-                               float sc2, int init, bool allow_mma, cudaStream_t st) {
+                               float* l, float* o, T* a_out, int B, int H, int dh, int q0, int nq, int k0,
+                               int nk, float sc2, int init, int fin, bool fast, cudaStream_t st,
+                               unsigned* err = nullptr, int min_tc_block = 128) {
   const int pairs = B * H;
   if constexpr (std::is_same<T, bf16>::value) {
-    if (allow_mma && dh == 64 && nk % 16 == 0) {
+    if (fast && dh == 64 && nk % 128 == 0 && nk >= min_tc_block && q_stride % 8 == 0 && kv_stride % 8 == 0) {
+      CUtensorMap tq, tk, tv;
+      if (!make_tmap_pm(&tq, Q, q_stride, B, q0 + nq) || !make_tmap_pm(&tk, K, kv_stride, B, k0 + nk) ||
+          !make_tmap_pm(&tv, V, kv_stride, B, k0 + nk))
+        return cudaErrorInvalidValue;
+      dim3 grid((nq + 127) / 128, pairs);
+      return launch_pdl(k_fold_tc, grid, dim3(192), FoldTcCfg::SMEM_BYTES, st, tq, tk, tv, Q, q_stride, m, l, o,
+                        a_out, B, H, q0, nq, k0, nk, sc2, init, fin, err);
+    }
+    if (fast && dh == 64 && nk % 16 == 0) {
       dim3 grid((nq + 63) / 64, pairs);
-      k_fold_mma<<<grid, 128, 0, st>>>(Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init);
-      return cudaGetLastError();
+      return launch_pdl(k_fold_mma, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B, H,
+                        q0, nq, k0, nk, sc2, init, fin);
+    }
+    if (fast && dh == 64 && nk <= 8 && q_stride % 8 == 0 && kv_stride % 8 == 0) {
+      const long threads = (long)pairs * nq * 8;
+      return launch_pdl(k_fold_small, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st, Q, q_stride, K, V,
+                        kv_stride, m, l, o, a_out, B, H, q0, nq, k0, nk, sc2, init, fin);
     }
   }
+  if (fin) return cudaErrorInvalidValue;   // only the bf16 kernels finalise
   const int blocks = (pairs + 3) / 4;
   switch (dh) {
-    case 32: k_fold_warp<T, 1><<<blocks, 128, 0, st>>>(Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init); break;
-    case 64: k_fold_warp<T, 2><<<blocks, 128, 0, st>>>(Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init); break;
-    default: k_fold_warp<T, 4><<<blocks, 128, 0, st>>>(Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init); break;
+    case 32: return launch_pdl(k_fold_warp<T, 1>, dim3(blocks), dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init);
+    case 64: return launch_pdl(k_fold_warp<T, 2>, dim3(blocks), dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init);
+    default: return launch_pdl(k_fold_warp<T, 4>, dim3(blocks), dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, B, H, q0, nq, k0, nk, sc2, init);
   }
-  return cudaGetLastError();
 }
 
 template <class T, int DPL>
@@ -291,10 +393,9 @@ static cudaError_t launch_attend(const Plan& P, const T* qkv, const T* K, const 
   const Shape& s = P.s;
   const int blocks = (s.B * s.H + 3) / 4;
   if (s.schedule == RT_SCHED_BLOCKED)
-    k_finalize<T, DPL><<<blocks, 128, 0, st>>>(qkv, m, l, o, a, s.B, s.H, j, sc2, j > 0 ? 1 : 0);
-  else
-    k_naive_attn<T, DPL><<<blocks, 128, 0, st>>>(qkv, K, V, a, s.B, s.H, j, sc2);
-  return cudaGetLastError();
+    return launch_pdl(k_finalize<T, DPL>, dim3(blocks), dim3(128), 0, st, qkv, m, l, o, a, s.B, s.H, j, sc2,
+                      j > 0 ? 1 : 0);
+  return launch_pdl(k_naive_attn<T, DPL>, dim3(blocks), dim3(128), 0, st, qkv, K, V, a, s.B, s.H, j, sc2);
 }
 
 // ---------------------------------------------------------------------------
@@ -328,6 +429,7 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
   RT_CK(cudaMemcpyAsync(wqkv, X.Wq, dd, cudaMemcpyDeviceToDevice, st));
   RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + dd, X.Wk, dd, cudaMemcpyDeviceToDevice, st));
   RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + 2 * dd, X.Wv, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemsetAsync(ws + P.off_cnt, 0, P.cnt_bytes, st));   // split-K arrival counters start at zero
 
   // 1. queries and temporary pairs of all positions
   {
@@ -349,47 +451,60 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
   }
 
   // 2. the N-step loop
-  const int bn_o = choose_bn(B, d), bn_1 = choose_bn(B, dff), bn_2 = choose_bn(B, d), bn_kv = choose_bn(B, 2 * d);
+  const int bn_o = P.t_wo.bn, bn_1 = P.t_w1.bn, bn_2 = P.t_w2.bn, bn_kv = P.t_wkv.bn;
   CUtensorMap tA_a, tB_o, tA_u, tB_1, tA_h, tB_2, tA_z, tB_kv;
   if (!make_tmap(&tA_a, a16, d, B, 128) || !make_tmap(&tB_o, X.Wo, d, d, bn_o) ||
       !make_tmap(&tA_u, u16, d, B, 128) || !make_tmap(&tB_1, X.W1, d, dff, bn_1) ||
       !make_tmap(&tA_h, h16, dff, B, 128) || !make_tmap(&tB_2, X.W2, dff, d, bn_2) ||
       !make_tmap(&tA_z, z16, d, B, 128) || !make_tmap(&tB_kv, wqkv + (size_t)d * d, d, 2 * d, bn_kv))
     return RT_ERR_INVALID_ARG;
+  ep.part = reinterpret_cast<float*>(ws + P.off_part);
+  ep.counters = reinterpret_cast<unsigned*>(ws + P.off_cnt);
   const float sc2 = kLog2e / std::sqrt((float)s.dh());
   const bool blocked = s.schedule == RT_SCHED_BLOCKED;
+  if (blocked) {
+    // position 1: only its temporary pair; every later position is finalised
+    // by the last fold into it (the fold of the previous step)
+    TimedScope ts(T, KC_ATTEND, st);
+    RT_CK((launch_attend<bf16, 2>(P, qkv, K, V, m, l, o, a16, 0, sc2, st)));
+  }
   for (int j = 0; j < N; ++j) {
     ep.j = j;
-    {
+    if (!blocked) {
       TimedScope ts(T, KC_ATTEND, st);
       RT_CK((launch_attend<bf16, 2>(P, qkv, K, V, m, l, o, a16, j, sc2, st)));
     }
     ep.ssq_out = ssq_u;
+    ep.splits = P.t_wo.splits;
     {
       TimedScope ts(T, KC_WO, st);
       RT_CK(launch_tc<EPI_WO>(bn_o, tA_a, tB_o, B, d, d, ep, err, ds.sms, st));
     }
     ep.ssq_in = ssq_u; ep.ssq_tiles = (d + bn_o - 1) / bn_o;
+    ep.splits = P.t_w1.splits;
     {
       TimedScope ts(T, KC_W1, st);
       RT_CK(launch_tc<EPI_W1>(bn_1, tA_u, tB_1, B, dff, d, ep, err, ds.sms, st));
     }
     ep.ssq_out = ssq_z;
+    ep.splits = P.t_w2.splits;
     {
       TimedScope ts(T, KC_W2, st);
       RT_CK(launch_tc<EPI_W2>(bn_2, tA_h, tB_2, B, d, dff, ep, err, ds.sms, st));
     }
     ep.ssq_in = ssq_z; ep.ssq_tiles = (d + bn_2 - 1) / bn_2;
+    ep.splits = P.t_wkv.splits;
     {
       TimedScope ts(T, KC_WKV, st);
       RT_CK(launch_tc<EPI_WKV>(bn_kv, tA_z, tB_kv, B, 2 * d, d, ep, err, ds.sms, st));
     }
     if (blocked) {
+      // fold keys (t - lb, t] into queries (t, t + lb] and finalise query t + 1
       const int t = j + 1, lb = lowbit(t), nq = std::min(lb, N - t);
       if (nq > 0) {
-        TimedScope ts(T, lb >= 16 ? KC_FOLD_MMA : KC_FOLD_WARP, st);
-        RT_CK(launch_fold<bf16>(qkv, 3 * d, K, V, d, m, l, o, B, H, 64, t, nq, t - lb, lb, sc2,
-                                t == lb ? 1 : 0, true, st));
+        TimedScope ts(T, KC_FOLD_LEVEL0 + log2_int(lb), st);
+        RT_CK(launch_fold<bf16>(qkv, 3 * d, K, V, d, m, l, o, a16, B, H, 64, t, nq, t - lb, lb, sc2,
+                                t == lb ? 1 : 0, 1, true, st, err, kFoldTcMinBlock));
       }
     }
   }
@@ -461,10 +576,10 @@ static int enqueue_f32(const Plan& P, const Ptrs& X, cudaStream_t st, Timer* T) 
     RT_CK(launch_simt<EPI_WKV>(rz, wqkv + (size_t)d * d, B, 2 * d, d, p, st));
     if (blocked) {
       const int t = j + 1, lb = lowbit(t), nq = std::min(lb, N - t);
-      TimedScope ts(nq > 0 ? T : nullptr, KC_FOLD_WARP, st);
+      TimedScope ts(nq > 0 ? T : nullptr, KC_FOLD_LEVEL0 + log2_int(lb), st);
       if (nq > 0)
-        RT_CK(launch_fold<float>(qkv, 3 * d, K, V, d, m, l, o, B, H, dh, t, nq, t - lb, lb, sc2,
-                                 t == lb ? 1 : 0, false, st));
+        RT_CK(launch_fold<float>(qkv, 3 * d, K, V, d, m, l, o, nullptr, B, H, dh, t, nq, t - lb, lb, sc2,
+                                 t == lb ? 1 : 0, 0, false, st));
     }
   }
   return RT_OK;
@@ -480,7 +595,11 @@ static long launch_count(const Shape& s) {
   long folds = 0;
   if (s.schedule == RT_SCHED_BLOCKED)
     for (int t = 1; t <= s.N; ++t) folds += (std::min(lowbit(t), s.N - t) > 0) ? 1 : 0;
-  if (s.dtype == RT_BF16) return 2 + 5l * s.N + folds;
+  if (s.dtype == RT_BF16) {
+    // blocked: finalise(position 1) + 4 GEMMs per step + folds (each finalises the next position)
+    if (s.schedule == RT_SCHED_BLOCKED) return 2 + 1 + 4l * s.N + folds;
+    return 2 + 5l * s.N;
+  }
   return 2 + 8l * s.N + folds;
 }
 
@@ -706,11 +825,12 @@ extern "C" int rt_block_fold(const void* Q, int q_stride, const void* K, const v
   cudaError_t e;
   if (dtype == RT_BF16)
     e = launch_fold<bf16>(static_cast<const bf16*>(Q), q_stride, static_cast<const bf16*>(K),
-                          static_cast<const bf16*>(V), kv_stride, m, l, o, B, H, d_h, q0, nq, k0, nk, sc2, 0, true, st);
+                          static_cast<const bf16*>(V), kv_stride, m, l, o, nullptr, B, H, d_h, q0, nq, k0, nk, sc2, 0,
+                          0, true, st);
   else if (dtype == RT_F32)
     e = launch_fold<float>(static_cast<const float*>(Q), q_stride, static_cast<const float*>(K),
-                           static_cast<const float*>(V), kv_stride, m, l, o, B, H, d_h, q0, nq, k0, nk, sc2, 0, false,
-                           st);
+                           static_cast<const float*>(V), kv_stride, m, l, o, nullptr, B, H, d_h, q0, nq, k0, nk, sc2, 0,
+                           0, false, st);
   else
     return RT_ERR_INVALID_ARG;
   return e == cudaSuccess ? RT_OK : RT_ERR_CUDA;
@@ -811,6 +931,10 @@ extern "C" int rt_layer_forward_timed(const void* x, const void* W_q, const void
     RT_CK(cudaEventElapsedTime(&ms, timer.pool[2 * i], timer.pool[2 * i + 1]));
     const int c = timer.cls[i];
     if (c < n_classes) { class_ms[c] += ms; class_launches[c] += 1; }
+    if (c >= KC_FOLD_LEVEL0) {   // per-level folds also count towards the kernel that ran them
+      const int kc = (s.dtype == RT_BF16 && c - KC_FOLD_LEVEL0 >= 4) ? KC_FOLD_MMA : KC_FOLD_WARP;
+      if (kc < n_classes) { class_ms[kc] += ms; class_launches[kc] += 1; }
+    }
   }
   return RT_OK;
 }

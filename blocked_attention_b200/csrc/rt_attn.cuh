@@ -40,6 +40,8 @@ __global__ void __launch_bounds__(128)
                const float* __restrict__ o, T* __restrict__ a_out, int B, int H, int j, float sc2,
                int has_acc) {
   constexpr int DH = DPL * 32;
+  pdl_launch_dependents();
+  pdl_wait();
   const int pair = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (pair >= B * H) return;
   const int b = pair / H, h = pair - b * H;
@@ -83,6 +85,8 @@ __global__ void __launch_bounds__(128)
                  T* __restrict__ a_out, int B, int H, int j, float sc2) {
   constexpr int DH = DPL * 32;
   __shared__ float sq[4][DH];
+  pdl_launch_dependents();
+  pdl_wait();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x * 4 + w;
   const bool active = pair < B * H;
@@ -154,6 +158,8 @@ __global__ void __launch_bounds__(128)
                 float* __restrict__ l, float* __restrict__ o, int B, int H, int q0, int nq,
                 int k0, int nk, float sc2, int init) {
   constexpr int DH = DPL * 32, KC = 8;
+  pdl_launch_dependents();
+  pdl_wait();
   const int pair = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (pair >= B * H) return;
   const int b = pair / H, h = pair - b * H;
@@ -218,6 +224,123 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
+// block fold for small blocks (nk <= 8 keys), bf16, d_h = 64: eight lanes per
+// (b, h, query), eight dims (16 bytes of q/k/v, 32 bytes of o) per lane.
+// fin = 1: the first query of the block (q0) receives no later fold, so it
+// is finalised here -- its temporary pair is merged and a_{q0} = o / l is
+// written to a_out [B][d]; its (m, l, o) are not stored.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(src);
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __bfloat1622float2(p[k]);
+    v[2 * k] = f.x;
+    v[2 * k + 1] = f.y;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    k_fold_small(const __nv_bfloat16* __restrict__ qkv, int q_stride, const __nv_bfloat16* __restrict__ K,
+                 const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m, float* __restrict__ l,
+                 float* __restrict__ o, __nv_bfloat16* __restrict__ a_out, int B, int H, int q0, int nq,
+                 int k0, int nk, float sc2, int init, int fin) {
+  constexpr int DH = 64, KMAX = 8;
+  pdl_launch_dependents();
+  pdl_wait();
+  const long item = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int sl = threadIdx.x & 7;
+  if (item >= (long)B * H * nq) return;   // whole octets leave together
+  const unsigned omask = 0xFFu << ((threadIdx.x & 31) & 24);
+  const int d = H * DH;
+  const int qi = (int)(item % nq);
+  const int pair = (int)(item / nq);
+  const int b = pair / H, h = pair - b * H;
+  const size_t row = (size_t)(q0 + qi) * B + b;
+  const __nv_bfloat16* qp = qkv + row * (size_t)q_stride + h * DH + sl * 8;
+  float q[8];
+  load_bf16x8(qp, q);
+  float mo = -INFINITY, lo = 0.f, oo[8];
+  float* op = o + row * (size_t)d + h * DH + sl * 8;
+  if (init) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) oo[e] = 0.f;
+  } else {
+    mo = m[row * H + h];
+    lo = l[row * H + h];
+    const float4 a0 = reinterpret_cast<const float4*>(op)[0], a1 = reinterpret_cast<const float4*>(op)[1];
+    oo[0] = a0.x; oo[1] = a0.y; oo[2] = a0.z; oo[3] = a0.w;
+    oo[4] = a1.x; oo[5] = a1.y; oo[6] = a1.z; oo[7] = a1.w;
+  }
+  float s[KMAX];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    s[i] = -INFINITY;
+    if (i < nk) {
+      float kk[8];
+      load_bf16x8(K + ((size_t)(k0 + i) * B + b) * kv_stride + h * DH + sl * 8, kk);
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
+      dot += __shfl_xor_sync(omask, dot, 1);
+      dot += __shfl_xor_sync(omask, dot, 2);
+      dot += __shfl_xor_sync(omask, dot, 4);
+      s[i] = dot * sc2;
+      mx = fmaxf(mx, s[i]);
+    }
+  }
+  const float mn = fmaxf(mo, mx);
+  const float al = rescale(mo, mn);
+  lo *= al;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) oo[e] *= al;
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    if (i < nk) {
+      const float p = exp2f(s[i] - mn);
+      float vv[8];
+      load_bf16x8(V + ((size_t)(k0 + i) * B + b) * kv_stride + h * DH + sl * 8, vv);
+      lo += p;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
+    }
+  }
+  if (fin && qi == 0) {
+    float kt[8], vt[8];
+    load_bf16x8(qp + d, kt);
+    load_bf16x8(qp + 2 * d, vt);
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dot += q[e] * kt[e];
+    dot += __shfl_xor_sync(omask, dot, 1);
+    dot += __shfl_xor_sync(omask, dot, 2);
+    dot += __shfl_xor_sync(omask, dot, 4);
+    const float st = dot * sc2;
+    const float m2 = fmaxf(mn, st);
+    const float a2 = rescale(mn, m2), pt = exp2f(st - m2);
+    const float inv = 1.f / (lo * a2 + pt);
+    uint4 w;
+    uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      __nv_bfloat162 v2 = __floats2bfloat162_rn((oo[2 * k] * a2 + pt * vt[2 * k]) * inv,
+                                                (oo[2 * k + 1] * a2 + pt * vt[2 * k + 1]) * inv);
+      wp[k] = *reinterpret_cast<uint32_t*>(&v2);
+    }
+    *reinterpret_cast<uint4*>(a_out + (size_t)b * d + h * DH + sl * 8) = w;
+  } else {
+    if (sl == 0) {
+      m[row * H + h] = mn;
+      l[row * H + h] = lo;
+    }
+    reinterpret_cast<float4*>(op)[0] = make_float4(oo[0], oo[1], oo[2], oo[3]);
+    reinterpret_cast<float4*>(op)[1] = make_float4(oo[4], oo[5], oo[6], oo[7]);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // block fold, tensor-core kernel (bf16, d_h = 64, nk a multiple of 16):
 // S = Q K^T and O += P V with mma.sync m16n8k16 (fp32 accumulate), online
 // softmax over key chunks of 64, then one merge into the fp32 (m, l, o) of
@@ -260,13 +383,15 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 __global__ void __launch_bounds__(128)
     k_fold_mma(const __nv_bfloat16* __restrict__ Q, int q_stride, const __nv_bfloat16* __restrict__ K,
                const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m,
-               float* __restrict__ l, float* __restrict__ o, int B, int H, int q0, int nq, int k0,
-               int nk, float sc2, int init) {
+               float* __restrict__ l, float* __restrict__ o, __nv_bfloat16* __restrict__ a_out, int B, int H,
+               int q0, int nq, int k0, int nk, float sc2, int init, int fin) {
   using namespace mma_detail;
   constexpr int DH = 64, QT = 64, KC = 64;
   __shared__ __align__(128) __nv_bfloat16 sQ[QT * LDS];
   __shared__ __align__(128) __nv_bfloat16 sK[2][KC * LDS];
   __shared__ __align__(128) __nv_bfloat16 sV[2][KC * LDS];
+  pdl_launch_dependents();
+  pdl_wait();
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int pair = blockIdx.y;
@@ -406,18 +531,46 @@ __global__ void __launch_bounds__(128)
     if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }
     const float mn = fmaxf(mg, mrow[rr]);
     const float ag = rescale(mg, mn), ab = rescale(mrow[rr], mn);
-    if ((lane & 3) == 0) {
-      m[row * H + h] = mn;
-      l[row * H + h] = lg * ag + lsum * ab;
-    }
+    const float ln = lg * ag + lsum * ab;
     float* op = o + row * (size_t)d + h * DH + (lane & 3) * 2;
+    float on[16];
 #pragma unroll
     for (int nd = 0; nd < 8; ++nd) {
       float2 og = make_float2(0.f, 0.f);
       if (!init) og = *reinterpret_cast<const float2*>(op + nd * 8);
-      og.x = og.x * ag + oacc[nd][rr * 2 + 0] * ab;
-      og.y = og.y * ag + oacc[nd][rr * 2 + 1] * ab;
-      *reinterpret_cast<float2*>(op + nd * 8) = og;
+      on[2 * nd] = og.x * ag + oacc[nd][rr * 2 + 0] * ab;
+      on[2 * nd + 1] = og.y * ag + oacc[nd][rr * 2 + 1] * ab;
+    }
+    if (fin && blockIdx.x == 0 && r == 0) {
+      // query q0 receives no later fold: merge its temporary pair, write a_{q0}
+      const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * DH + (lane & 3) * 2;
+      float dot = 0.f;
+#pragma unroll
+      for (int nd = 0; nd < 8; ++nd) {
+        const float2 kt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tp + d + nd * 8));
+        const float2 qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sQ[nd * 8 + (lane & 3) * 2]));
+        dot += qv.x * kt.x + qv.y * kt.y;
+      }
+      dot += __shfl_xor_sync(0xFu, dot, 1);
+      dot += __shfl_xor_sync(0xFu, dot, 2);
+      const float st = dot * sc2;
+      const float m2 = fmaxf(mn, st);
+      const float a2 = rescale(mn, m2), pt = exp2f(st - m2);
+      const float inv = 1.f / (ln * a2 + pt);
+      __nv_bfloat16* ap = a_out + (size_t)b * d + h * DH + (lane & 3) * 2;
+#pragma unroll
+      for (int nd = 0; nd < 8; ++nd) {
+        const float2 vt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tp + 2 * d + nd * 8));
+        *reinterpret_cast<__nv_bfloat162*>(ap + nd * 8) =
+            __floats2bfloat162_rn((on[2 * nd] * a2 + pt * vt.x) * inv, (on[2 * nd + 1] * a2 + pt * vt.y) * inv);
+      }
+    } else {
+      if ((lane & 3) == 0) {
+        m[row * H + h] = mn;
+        l[row * H + h] = ln;
+      }
+#pragma unroll
+      for (int nd = 0; nd < 8; ++nd) *reinterpret_cast<float2*>(op + nd * 8) = make_float2(on[2 * nd], on[2 * nd + 1]);
     }
   }
 }
@@ -429,6 +582,8 @@ __global__ void __launch_bounds__(128)
 template <class T>
 __global__ void __launch_bounds__(256) k_row_inv_rms(const T* __restrict__ x, float* __restrict__ inv,
                                                      size_t rows, int d, float eps) {
+  pdl_launch_dependents();
+  pdl_wait();
   const size_t r = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;

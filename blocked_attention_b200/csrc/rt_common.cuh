@@ -38,6 +38,18 @@ __device__ __forceinline__ void set_error(unsigned* err, unsigned bits) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while its predecessor runs; it must call
+// pdl_wait() before touching anything the predecessor writes, and every
+// kernel calls it before it can finish so that completion stays transitive.
+// Both are no-ops for a normal launch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // small numeric helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float to_f(float v) { return v; }

@@ -1,0 +1,334 @@
+// rt_fold_tc.cuh -- block fold on the sm_100a tensor cores for large blocks.
+//
+// Folds keys [k0, k0 + nk) into the online-softmax statistics (m, l, o) of
+// queries [q0, q0 + nq) ("Recurrent Transformer" paper page, notes §4.2 /
+// paper §5: when (k_t, v_t) is revealed, keys (t - lowbit(t), t] are folded
+// into queries (t, t + lowbit(t)]). bf16 q/k/v, d_h = 64, nk a multiple of 128.
+//
+// CTA = one (sequence b, head h) and 128 queries; 192 threads:
+//   warp 0     : TMA producer (3-D boxes over the position-major cache:
+//                128 positions x 64 dims of one (b, h))
+//   warp 1     : TMEM allocator + MMA issuer
+//   warps 2..5 : softmax / accumulate / merge; thread = one query row
+// For each 128-key chunk c (double-buffered everywhere):
+//   S_c = Q K_c^T         tcgen05.mma, M=128 N=128 K=64, fp32 in TMEM
+//   P_c = exp2(S_c*sc2 - m_c) in bf16, written by the softmax warps to shared
+//         memory in the 128-byte-swizzled K-major operand layout
+//   O_c = P_c V_c         tcgen05.mma, M=128 N=64 K=128, V as MN-major operand
+//   o  <- o * exp2(m_{c-1} - m_c) + O_c   (registers; one chunk behind, so the
+//         PV product of chunk c overlaps the softmax of chunk c+1)
+// Finally each row merges (m, l, o) into its global statistics, or, when
+// fin = 1 and the row is query q0, merges the temporary pair and writes a_{q0}.
+#pragma once
+
+#include "rt_common.cuh"
+#include "rt_gemm_tc.cuh"
+
+namespace rt {
+
+struct FoldTcCfg {
+  static constexpr int QT = 128, KC = 128, DH = 64;
+  static constexpr uint32_t Q_BYTES = QT * DH * 2;    // 16 KB
+  static constexpr uint32_t KV_BYTES = KC * DH * 2;   // 16 KB (K or V chunk)
+  static constexpr uint32_t P_BYTES = QT * KC * 2;    // 32 KB (two 64-key swizzle atoms)
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + 2 * KV_BYTES;
+  static constexpr uint32_t OFF_P = OFF_V + 2 * KV_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 256;
+  static constexpr uint32_t TMEM_COLS = 512;          // S[2] at 0/128, O[2] at 256/320
+};
+
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap* m, uint64_t* bar, void* dst, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// MN-major operand with 128-byte swizzle, one 64-element swizzle row along MN:
+// K rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(const void* p) {
+  const uint32_t a = smem_u32(p);
+  uint64_t d = 0;
+  d |= (uint64_t)((a >> 4) & 0x3FFFu);   // start address
+  d |= (uint64_t)(8192u >> 4) << 16;     // leading byte offset (next 64-element MN group; unused for N = 64)
+  d |= (uint64_t)(1024u >> 4) << 32;     // stride byte offset: 8 K rows x 128 B
+  d |= (uint64_t)1u << 46;               // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;               // layout: 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void fence_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(192, 1)
+    k_fold_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __nv_bfloat16* __restrict__ Q, int q_stride,
+              float* __restrict__ m, float* __restrict__ l, float* __restrict__ o,
+              __nv_bfloat16* __restrict__ a_out, int B, int H, int q0, int nq, int k0, int nk, float sc2,
+              int init, int fin, unsigned* err) {
+  using C = FoldTcCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;    // [2]
+  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* s_free = bars + 7;     // [2]
+  uint64_t* p_full = bars + 9;     // [2]
+  uint64_t* o_full = bars + 11;    // [2]
+  uint64_t* o_free = bars + 13;    // [2]
+  uint64_t* mma_done = bars + 15;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.y;
+  const int b = pair / H, h = pair - b * H;
+  const int d = H * C::DH;
+  const int qt0 = q0 + blockIdx.x * C::QT;
+  const int nrows = min(C::QT, q0 + nq - qt0);
+  const int nchunks = nk / C::KC;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_free[i], 4);
+    }
+    mbar_init(mma_done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  pdl_launch_dependents();
+  pdl_wait();
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+      tma_load_3d(&tmQ, q_full, sQ, h * C::DH, b, qt0);
+      int c = 0;
+      for (; c < nchunks; ++c) {
+        const int st = c & 1;
+        const uint32_t ph = (c >> 1) & 1u;
+        if (!mbar_wait(&kv_empty[st], ph ^ 1u, err)) break;
+        mbar_arrive_expect_tx(&kv_full[st], 2 * C::KV_BYTES);
+        tma_load_3d(&tmK, &kv_full[st], smem + C::OFF_K + st * C::KV_BYTES, h * C::DH, b, k0 + c * C::KC);
+        tma_load_3d(&tmV, &kv_full[st], smem + C::OFF_V + st * C::KV_BYTES, h * C::DH, b, k0 + c * C::KC);
+      }
+      if (c < nchunks) {
+        // aborted: wait (bounded) for the copies this thread issued
+        mbar_wait(q_full, 0, err);
+        for (int i = (c >= 2 ? c - 2 : 0); i < c; ++i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1u, err);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128);
+      const uint32_t idesc_o = idesc_bf16_f32(128, 64) | (1u << 16);   // B (= V) MN-major
+      bool ok = mbar_wait(q_full, 0, err);
+      auto issue_s = [&](int c) -> bool {
+        const int st = c & 1;
+        const uint32_t ph = (c >> 1) & 1u;
+        if (!mbar_wait(&kv_full[st], ph, err) || !mbar_wait(&s_free[st], ph ^ 1u, err)) return false;
+        tc_fence_after();
+        const uint8_t* kt = smem + C::OFF_K + st * C::KV_BYTES;
+#pragma unroll
+        for (int k = 0; k < C::DH / 16; ++k)
+          tc_mma_f16(tmem_base + st * 128, smem_desc_sw128(sQ + k * 32), smem_desc_sw128(kt + k * 32), idesc_s,
+                     k != 0 ? 1u : 0u);
+        tc_commit(&s_full[st]);
+        return true;
+      };
+      auto issue_pv = [&](int c) -> bool {
+        const int bb = c & 1;
+        const uint32_t ph = (c >> 1) & 1u;
+        if (!mbar_wait(&p_full[bb], ph, err) || !mbar_wait(&o_free[bb], ph ^ 1u, err)) return false;
+        tc_fence_after();
+        const uint8_t* pt = smem + C::OFF_P + bb * C::P_BYTES;
+        const uint8_t* vt = smem + C::OFF_V + bb * C::KV_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < C::KC / 16; ++ks) {
+          // A = P: K-major, 64-key atoms 16 KB apart, 32 bytes per 16 keys inside an atom
+          // B = V: MN-major, 16 keys = 16 rows of 128 bytes
+          tc_mma_f16(tmem_base + 256 + bb * 64, smem_desc_sw128(pt + (ks >> 2) * 16384 + (ks & 3) * 32),
+                     smem_desc_sw128_mn(vt + ks * 16 * 128), idesc_o, ks != 0 ? 1u : 0u);
+        }
+        tc_commit(&o_full[bb]);
+        tc_commit(&kv_empty[bb]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int c = 0; c < nchunks && ok; ++c) {
+        if (c + 1 < nchunks) ok = issue_s(c + 1);
+        if (ok) ok = issue_pv(c);
+      }
+      // every MMA this thread issued has finished before the CTA can free TMEM
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, err);
+    }
+  } else {
+    // ---------------- softmax / accumulate / merge ----------------
+    const int qq = warp & 3;
+    const int r = qq * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
+    uint8_t* sP = smem + C::OFF_P;
+    float m_run = -INFINITY, l_run = 0.f, alpha_prev = 0.f;
+    float oacc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) oacc[i] = 0.f;
+    bool ok = true;
+
+    auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
+      int v = 1;
+      if (lane == 0) v = mbar_wait(bar, parity, err) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, v, 0) != 0;
+    };
+    auto accumulate = [&](int c, float alpha) -> bool {
+      const int bb = c & 1;
+      if (!wait_warp(&o_full[bb], (c >> 1) & 1u)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t rv[32];
+        tmem_ld_32x32b_x32(tmem_base + lane_base + 256 + bb * 64 + half * 32, rv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) oacc[half * 32 + i] = oacc[half * 32 + i] * alpha + __uint_as_float(rv[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[bb]);
+      return true;
+    };
+
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int bb = c & 1;
+      if (!wait_warp(&s_full[bb], (c >> 1) & 1u)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sbase = tmem_base + lane_base + bb * 128;
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t rv[32];
+        tmem_ld_32x32b_x32(sbase + cc * 32, rv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(rv[i]));
+      }
+      const float m_new = fmaxf(m_run, mx * sc2);
+      const float alpha = rescale(m_run, m_new);
+      float lsum = 0.f;
+      uint8_t* prow = sP + bb * C::P_BYTES + r * 128;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t rv[32];
+        tmem_ld_32x32b_x32(sbase + cc * 32, rv);
+        tmem_ld_wait();
+        uint8_t* atom = prow + (cc >> 1) * 16384;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            p[e] = exp2f(__uint_as_float(rv[g * 8 + e]) * sc2 - m_new);
+            lsum += p[e];
+          }
+          uint4 w;
+          w.x = pack_bf16x2(p[0], p[1]);
+          w.y = pack_bf16x2(p[2], p[3]);
+          w.z = pack_bf16x2(p[4], p[5]);
+          w.w = pack_bf16x2(p[6], p[7]);
+          const int chunk = (cc & 1) * 4 + g;
+          *reinterpret_cast<uint4*>(atom + ((chunk ^ (r & 7)) << 4)) = w;
+        }
+      }
+      l_run = l_run * alpha + lsum;
+      m_run = m_new;
+      tc_fence_before();
+      fence_async_shared();   // P stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_free[bb]);
+        mbar_arrive(&p_full[bb]);
+      }
+      if (c > 0 && !accumulate(c - 1, alpha_prev)) { ok = false; break; }
+      alpha_prev = alpha;
+    }
+    if (ok && nchunks > 0) ok = accumulate(nchunks - 1, alpha_prev);
+
+    if (ok && r < nrows) {
+      const size_t row = (size_t)(qt0 + r) * B + b;
+      float mg = -INFINITY, lg = 0.f;
+      float* op = o + row * (size_t)d + h * C::DH;
+      if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }
+      const float mn = fmaxf(mg, m_run);
+      const float ag = rescale(mg, mn), ab = rescale(m_run, mn);
+      const float ln = lg * ag + l_run * ab;
+      if (fin && blockIdx.x == 0 && r == 0) {
+        // query q0 receives no later fold: merge its temporary pair, write a_{q0}
+        const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * C::DH;
+        float dot = 0.f;
+#pragma unroll 8
+        for (int e = 0; e < C::DH; ++e)
+          dot += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(sQ)[e]) * __bfloat162float(tp[d + e]);
+        const float s2 = dot * sc2;
+        const float m2 = fmaxf(mn, s2);
+        const float a2 = rescale(mn, m2), pt = exp2f(s2 - m2);
+        const float inv = 1.f / (ln * a2 + pt);
+        __nv_bfloat16* ap = a_out + (size_t)b * d + h * C::DH;
+#pragma unroll
+        for (int e = 0; e < C::DH; e += 2) {
+          float og0 = 0.f, og1 = 0.f;
+          if (!init) { og0 = op[e]; og1 = op[e + 1]; }
+          const float o0 = og0 * ag + oacc[e] * ab, o1 = og1 * ag + oacc[e + 1] * ab;
+          const float2 vt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tp + 2 * d + e));
+          *reinterpret_cast<__nv_bfloat162*>(ap + e) =
+              __floats2bfloat162_rn((o0 * a2 + pt * vt.x) * inv, (o1 * a2 + pt * vt.y) * inv);
+        }
+      } else {
+        m[row * H + h] = mn;
+        l[row * H + h] = ln;
+#pragma unroll
+        for (int e = 0; e < C::DH; e += 4) {
+          float4 og = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (!init) og = *reinterpret_cast<const float4*>(op + e);
+          og.x = og.x * ag + oacc[e] * ab;
+          og.y = og.y * ag + oacc[e + 1] * ab;
+          og.z = og.z * ag + oacc[e + 2] * ab;
+          og.w = og.w * ag + oacc[e + 3] * ab;
+          *reinterpret_cast<float4*>(op + e) = og;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace rt

@@ -48,6 +48,13 @@ struct EpiParams {
   __nv_bfloat16* z16;        // W2 out: [B][d]
   __nv_bfloat16* Kout;       // WKV out: [N][B][d]
   __nv_bfloat16* Vout;
+  // split-K: `splits` CTAs share one output tile, each over K/splits; they
+  // write fp32 partial tiles to `part`, and the last to arrive (counted in
+  // `counters`, one per output tile, left at zero) sums them in split order
+  // and runs the epilogue.
+  int splits;
+  float* part;
+  unsigned* counters;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -186,10 +193,14 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntn = (N + BN - 1) / BN, ntm = (M + C::BM - 1) / C::BM;
-  const int num_tiles = ntn * ntm;
-  const int nk = K / C::BK;
-
+  const int nmn = ntn * ntm;
+  const int splits = p.splits > 1 ? p.splits : 1;
+  const int num_tiles = nmn * splits;
+  const int nk = K / C::BK / splits;   // k-blocks per split (the host keeps this exact)
+  __shared__ int s_last, s_abort;
   if (threadIdx.x == 0) {
+    s_last = 0;
+    s_abort = 0;
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -200,6 +211,9 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // everything above overlaps the predecessor kernel; its outputs are read below
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -207,13 +221,15 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mt = tile / ntn, nt = tile - mt * ntn;
+        const int ks = tile / nmn, mn = tile - ks * nmn;
+        const int mt = mn / ntn, nt = mn - mt * ntn;
+        const int kb0 = ks * nk;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, err)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-          tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, kb * C::BK, mt * C::BM);
-          tma_load_2d(&tmB, &full[s], sB + s * C::B_BYTES, kb * C::BK, nt * BN);
+          tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, (kb0 + kb) * C::BK, mt * C::BM);
+          tma_load_2d(&tmB, &full[s], sB + s * C::B_BYTES, (kb0 + kb) * C::BK, nt * BN);
         }
       }
       if (!ok) {
@@ -255,37 +271,104 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;
     uint32_t local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-      const int mt = tile / ntn, nt = tile - mt * ntn;
+      const int ks = tile / nmn, mn = tile - ks * nmn;
+      const int mt = mn / ntn, nt = mn - mt * ntn;
       const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], aph, err) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (splits > 1) {
+        // the split path synchronises the four epilogue warps: leave together
+        if (!ok && lane == 0) s_abort = 1;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        ok = s_abort ? 0 : 1;
+      }
       if (!ok) break;
       tc_fence_after();
-      const int row = mt * C::BM + q * 32 + lane;
+      const int lrow = q * 32 + lane;
+      const int row = mt * C::BM + lrow;
       const bool row_ok = row < M;
-      const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
-      float ssq = 0.f;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if (splits == 1) {
+        const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
+        float ssq = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + c, r);
-        tmem_ld_wait();
-        const int col0 = nt * BN + c;
-        if (row_ok && col0 < N) {
-          float v[32];
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c, r);
+          tmem_ld_wait();
+          const int col0 = nt * BN + c;
+          if (row_ok && col0 < N) {
+            float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+            ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
+          }
         }
+        if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
+          if (row_ok) p.ssq_out[(size_t)nt * p.B + row] = ssq;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+      } else {
+        // 1. this split's partial tile row -> part[ks][mn][lrow][0:BN]
+        float* prow = p.part + ((size_t)(ks * nmn + mn) * C::BM + lrow) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c, r);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              reinterpret_cast<float4*>(prow + c)[i] =
+                  make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                              __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        // 2. count arrivals; the last CTA of this output tile reduces
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x == 64) {
+          const unsigned old = atomicAdd(&p.counters[mn], 1u);
+          const int last = old == (unsigned)(splits - 1);
+          if (last) p.counters[mn] = 0u;   // every split has arrived: reset for the next use
+          s_last = last;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (s_last) {
+          __threadfence();
+          const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
+          float ssq = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            const int col0 = nt * BN + c;
+            if (row_ok && col0 < N) {
+              float v[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = 0.f;
+              for (int sp = 0; sp < splits; ++sp) {
+                const float4* src =
+                    reinterpret_cast<const float4*>(p.part + ((size_t)(sp * nmn + mn) * C::BM + lrow) * BN + c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 w = __ldcg(src + i);
+                  v[4 * i] += w.x; v[4 * i + 1] += w.y; v[4 * i + 2] += w.z; v[4 * i + 3] += w.w;
+                }
+              }
+              ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
+            }
+          }
+          if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
+            if (row_ok) p.ssq_out[(size_t)nt * p.B + row] = ssq;
+          }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // s_last is reused by the next tile
       }
-      if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
-        if (row_ok) p.ssq_out[(size_t)nt * p.B + row] = ssq;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
     }
   }
   __syncthreads();

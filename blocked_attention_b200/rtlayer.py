@@ -31,7 +31,8 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_layer_workspace_bytes", "rt_lay
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma")
-RT_KC_COUNT = 10
+RT_KC_FOLD_LEVEL0 = 16
+RT_KC_COUNT = 32
 
 _lib = None
 
@@ -182,7 +183,12 @@ def layer_forward_timed(x: torch.Tensor, W: dict, H: int, out, workspace: torch.
                                       _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream),
                                       ms, cnt, RT_KC_COUNT)
     _check("rt_layer_forward_timed", rc)
-    return {name: (float(ms[i]), int(cnt[i])) for i, name in enumerate(KERNEL_CLASSES) if cnt[i] > 0}
+    out = {name: (float(ms[i]), int(cnt[i])) for i, name in enumerate(KERNEL_CLASSES) if cnt[i] > 0}
+    for lv in range(RT_KC_COUNT - RT_KC_FOLD_LEVEL0):
+        c = RT_KC_FOLD_LEVEL0 + lv
+        if cnt[c] > 0:
+            out[f"fold_lb{1 << lv}"] = (float(ms[c]), int(cnt[c]))
+    return out
 
 
 def sync_status(workspace: torch.Tensor, stream=None) -> int:

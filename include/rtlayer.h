@@ -199,9 +199,10 @@ enum {
   RT_KC_W1 = 4,      /* GELU(rms(u) W_1^T)                                */
   RT_KC_W2 = 5,      /* h W_2^T + residual = z_t                          */
   RT_KC_WKV = 6,     /* persistent pair rms(z_t) [W_k; W_v]^T             */
-  RT_KC_FOLD_WARP = 7, /* block fold, warp kernel                         */
-  RT_KC_FOLD_MMA = 8,  /* block fold, tensor-core kernel                  */
-  RT_KC_COUNT = 10
+  RT_KC_FOLD_WARP = 7, /* block fold, small-block / warp kernels          */
+  RT_KC_FOLD_MMA = 8,  /* block fold, tensor-core kernel (block >= 16)    */
+  RT_KC_FOLD_LEVEL0 = 16, /* + log2(block size): the same folds by level  */
+  RT_KC_COUNT = 32
 };
 
 /* rt_layer_forward with the host-loop driver and a CUDA event pair recorded

@@ -59,9 +59,10 @@ def test_workspace_plan(L):
 
 
 def test_launch_count_matches_schedule(L):
-    # bf16: 2 set-up kernels + 5 per step + one fold per step t < N (lowbit(t) >= 1)
+    # bf16 blocked: inv_rms + projection + finalise(position 1) + 4 GEMMs per step
+    # + one fold per step t < N (each also finalises position t + 1)
     for N in (1, 2, 7, 64, 2048):
-        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0) == 2 + 5 * N + (N - 1)
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0) == 3 + 4 * N + (N - 1)
         assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 1) == 2 + 5 * N
     assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_F32, 0) == 2 + 8 * 8 + 7
     assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_BF16, 0) == -1

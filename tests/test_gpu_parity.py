@@ -70,9 +70,12 @@ def test_batched_projection_matches_oracle(rt, dtype, B, N, d):
 
 
 @pytest.mark.parametrize("dtype,nk,nq,init_empty", [
-    ("bf16", 1, 1, False), ("bf16", 2, 2, True), ("bf16", 8, 5, False),      # warp kernel
-    ("bf16", 16, 16, False), ("bf16", 32, 7, False), ("bf16", 64, 64, True),  # tensor-core kernel
-    ("bf16", 256, 100, False), ("bf16", 1024, 130, False),
+    ("bf16", 1, 1, False), ("bf16", 2, 2, True), ("bf16", 8, 5, False),      # small-block kernel (nk <= 8)
+    ("bf16", 16, 16, False), ("bf16", 32, 7, False), ("bf16", 64, 64, True),  # mma.sync kernel
+    ("bf16", 48, 20, False),
+    ("bf16", 256, 100, False), ("bf16", 1024, 130, False),                     # tcgen05 kernel (nk % 128 == 0)
+    ("bf16", 128, 77, False), ("bf16", 128, 128, True), ("bf16", 512, 300, True), ("bf16", 384, 1, False),
+    ("bf16", 12, 3, False),                                                      # generic warp kernel
     ("f32", 3, 4, False), ("f32", 16, 16, True), ("f32", 64, 33, False)])
 def test_block_fold_matches_oracle(rt, dtype, nk, nq, init_empty):
     B, H, dh = 3, 2, 64 if dtype == "bf16" else 32
