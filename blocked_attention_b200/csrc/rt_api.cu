@@ -45,19 +45,31 @@ static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; 
 // previous kernel in the stream runs; every kernel calls pdl_wait() before it
 // reads its predecessor's outputs.
 template <typename... KArgs, typename... Args>
-static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                              Args&&... args) {
+static cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                      int cluster, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = at;
   cfg.numAttrs = 1;
+  if (cluster > 1) {
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = cluster;
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  cfg.attrs = at;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  return launch_pdl_cluster(kern, grid, block, smem, st, 1, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------------------
@@ -167,36 +179,35 @@ struct TileCfg {
   int bn, splits;
 };
 static TileCfg choose_tiles(int M, int N, int K, bool allow_split) {
-  if (!allow_split) return {choose_bn(M, N), 1};
+  // Measured at M = 512 (per-step GEMM latency, graph of back-to-back
+  // launches): plain tiles with >= 120 CTAs win for K = 1024; for long K
+  // (W_2, K = 4096) 64-wide tiles with a 2-CTA cluster split-K win
+  // (15.3 us vs 21.0 us); wider splits cost more in staging than they save.
   const long ntm = (M + 127) / 128;
-  const int bn = (N % 128 == 0) ? 128 : 64;
-  const long mn = ntm * ((N + bn - 1) / bn);
-  if (mn >= 120) return {choose_bn(M, N), 1};
-  const int nkb = K / 64;
-  int splits = 1;
-  while (mn * splits * 2 <= 160 && nkb % (splits * 2) == 0 && nkb / (splits * 2) >= 4) splits *= 2;
-  return {bn, splits};
+  if (allow_split && K / 64 >= 64 && N % 64 == 0) {
+    const long mn = ntm * (N / 64);
+    if (mn * 2 <= 160 && mn < 120) return {64, 2};
+  }
+  return {choose_bn(M, N), 1};
 }
-// Split-K measured slower at M = 512 (the last-CTA reduction lengthens the
-// per-step critical path), so the layer uses unsplit tiles.
-static constexpr bool kLayerSplitK = false;
-// The tcgen05 fold beat the mma.sync fold only from block size 1024 up.
+// Per-step GEMMs may use cluster split-K (see choose_tiles).
+static constexpr bool kLayerSplitK = true;
+// Smallest block size that uses the tcgen05 fold (smaller ones: mma.sync);
+// measured: mma.sync is faster up to 512, the tcgen05 fold at 1024.
 static constexpr int kFoldTcMinBlock = 1024;
-static size_t split_part_floats(int M, int N, const TileCfg& c) {
-  if (c.splits <= 1) return 0;
-  const size_t ntm = (M + 127) / 128, ntn = (N + c.bn - 1) / c.bn;
-  return (size_t)c.splits * ntm * 128 * ntn * c.bn;
-}
-static size_t split_tiles(int M, int N, const TileCfg& c) {
-  return (size_t)((M + 127) / 128) * ((N + c.bn - 1) / c.bn);
-}
 
 template <int BN, int EPI>
 static cudaError_t launch_tc_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
                                 const EpiParams& p, unsigned* err, int sms, cudaStream_t st) {
   constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   using C = GemmCfg<BN, STAGES>;
-  const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN) * (p.splits > 1 ? p.splits : 1);
+  if (p.splits > 1) {
+    // one output tile per cluster of `splits` CTAs, one tile per CTA
+    const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN) * p.splits;
+    return launch_pdl_cluster(k_gemm_tc<BN, STAGES, EPI>, dim3((unsigned)tiles), dim3(192), C::SMEM_BYTES, st,
+                              p.splits, ta, tb, M, N, K, p, err);
+  }
+  const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = (int)std::min<long>(tiles, sms);
   return launch_pdl(k_gemm_tc<BN, STAGES, EPI>, dim3(grid), dim3(192), C::SMEM_BYTES, st, ta, tb, M, N, K, p,
                     err);
@@ -242,7 +253,7 @@ struct Plan {
   Shape s;
   size_t esz;
   size_t off_err, off_qkv, off_m, off_l, off_o, off_inv, off_xr, off_wqkv, off_a, off_u32, off_u16, off_ru,
-      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, off_part, off_cnt, cnt_bytes, total;
+      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, total;
   TileCfg t_wo, t_w1, t_w2, t_wkv;
 };
 
@@ -282,13 +293,6 @@ static Plan make_plan(const Shape& s) {
     P.t_w1 = choose_tiles(s.B, s.d_ff, s.d, kLayerSplitK);
     P.t_w2 = choose_tiles(s.B, s.d, s.d_ff, kLayerSplitK);
     P.t_wkv = choose_tiles(s.B, 2 * s.d, s.d, kLayerSplitK);
-    const size_t part = std::max(std::max(split_part_floats(s.B, s.d, P.t_wo), split_part_floats(s.B, s.d_ff, P.t_w1)),
-                                 std::max(split_part_floats(s.B, s.d, P.t_w2), split_part_floats(s.B, 2 * s.d, P.t_wkv)));
-    const size_t cnt = std::max(std::max(split_tiles(s.B, s.d, P.t_wo), split_tiles(s.B, s.d_ff, P.t_w1)),
-                                std::max(split_tiles(s.B, s.d, P.t_w2), split_tiles(s.B, 2 * s.d, P.t_wkv)));
-    P.off_part = take(std::max<size_t>(part, 1) * 4);
-    P.cnt_bytes = cnt * 4;
-    P.off_cnt = take(P.cnt_bytes);
   }
   P.total = off;
   return P;
@@ -355,7 +359,7 @@ template <class T>
 static cudaError_t launch_fold(const T* Q, int q_stride, const T* K, const T* V, int kv_stride, float* m,
                                float* l, float* o, T* a_out, int B, int H, int dh, int q0, int nq, int k0,
                                int nk, float sc2, int init, int fin, bool fast, cudaStream_t st,
-                               unsigned* err = nullptr, int min_tc_block = 128) {
+                               unsigned* err = nullptr, int min_tc_block = 128, int sms = 148) {
   const int pairs = B * H;
   if constexpr (std::is_same<T, bf16>::value) {
     if (fast && dh == 64 && nk % 128 == 0 && nk >= min_tc_block && q_stride % 8 == 0 && kv_stride % 8 == 0) {
@@ -363,13 +367,25 @@ static cudaError_t launch_fold(const T* Q, int q_stride, const T* K, const T* V,
       if (!make_tmap_pm(&tq, Q, q_stride, B, q0 + nq) || !make_tmap_pm(&tk, K, kv_stride, B, k0 + nk) ||
           !make_tmap_pm(&tv, V, kv_stride, B, k0 + nk))
         return cudaErrorInvalidValue;
-      dim3 grid((nq + 127) / 128, pairs);
+      const long items = (long)pairs * ((nq + 127) / 128);
+      const dim3 grid((unsigned)std::min<long>(items, sms));   // persistent over (pair, query tile) items
       return launch_pdl(k_fold_tc, grid, dim3(192), FoldTcCfg::SMEM_BYTES, st, tq, tk, tv, Q, q_stride, m, l, o,
                         a_out, B, H, q0, nq, k0, nk, sc2, init, fin, err);
     }
-    if (fast && dh == 64 && nk % 16 == 0) {
+    if (fast && dh == 64 && nk >= 16 && nk % 16 == 0) {
+      // pack 4 / 2 (b, h) pairs per CTA for 16- / 32-key blocks so that no warp idles
+      if (nk <= 16) {
+        dim3 grid((nq + 15) / 16, (pairs + 3) / 4);
+        return launch_pdl(k_fold_mma<4>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B,
+                          H, q0, nq, k0, nk, sc2, init, fin);
+      }
+      if (nk <= 32) {
+        dim3 grid((nq + 31) / 32, (pairs + 1) / 2);
+        return launch_pdl(k_fold_mma<2>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B,
+                          H, q0, nq, k0, nk, sc2, init, fin);
+      }
       dim3 grid((nq + 63) / 64, pairs);
-      return launch_pdl(k_fold_mma, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B, H,
+      return launch_pdl(k_fold_mma<1>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B, H,
                         q0, nq, k0, nk, sc2, init, fin);
     }
     if (fast && dh == 64 && nk <= 8 && q_stride % 8 == 0 && kv_stride % 8 == 0) {
@@ -429,7 +445,6 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
   RT_CK(cudaMemcpyAsync(wqkv, X.Wq, dd, cudaMemcpyDeviceToDevice, st));
   RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + dd, X.Wk, dd, cudaMemcpyDeviceToDevice, st));
   RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + 2 * dd, X.Wv, dd, cudaMemcpyDeviceToDevice, st));
-  RT_CK(cudaMemsetAsync(ws + P.off_cnt, 0, P.cnt_bytes, st));   // split-K arrival counters start at zero
 
   // 1. queries and temporary pairs of all positions
   {
@@ -458,8 +473,6 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
       !make_tmap(&tA_h, h16, dff, B, 128) || !make_tmap(&tB_2, X.W2, dff, d, bn_2) ||
       !make_tmap(&tA_z, z16, d, B, 128) || !make_tmap(&tB_kv, wqkv + (size_t)d * d, d, 2 * d, bn_kv))
     return RT_ERR_INVALID_ARG;
-  ep.part = reinterpret_cast<float*>(ws + P.off_part);
-  ep.counters = reinterpret_cast<unsigned*>(ws + P.off_cnt);
   const float sc2 = kLog2e / std::sqrt((float)s.dh());
   const bool blocked = s.schedule == RT_SCHED_BLOCKED;
   if (blocked) {
@@ -504,7 +517,7 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
       if (nq > 0) {
         TimedScope ts(T, KC_FOLD_LEVEL0 + log2_int(lb), st);
         RT_CK(launch_fold<bf16>(qkv, 3 * d, K, V, d, m, l, o, a16, B, H, 64, t, nq, t - lb, lb, sc2,
-                                t == lb ? 1 : 0, 1, true, st, err, kFoldTcMinBlock));
+                                t == lb ? 1 : 0, 1, true, st, err, kFoldTcMinBlock, ds.sms));
       }
     }
   }
@@ -826,7 +839,7 @@ extern "C" int rt_block_fold(const void* Q, int q_stride, const void* K, const v
   if (dtype == RT_BF16)
     e = launch_fold<bf16>(static_cast<const bf16*>(Q), q_stride, static_cast<const bf16*>(K),
                           static_cast<const bf16*>(V), kv_stride, m, l, o, nullptr, B, H, d_h, q0, nq, k0, nk, sc2, 0,
-                          0, true, st);
+                          0, true, st, nullptr, 128, ds->sms);
   else if (dtype == RT_F32)
     e = launch_fold<float>(static_cast<const float*>(Q), q_stride, static_cast<const float*>(K),
                            static_cast<const float*>(V), kv_stride, m, l, o, nullptr, B, H, d_h, q0, nq, k0, nk, sc2, 0,
@@ -937,4 +950,26 @@ extern "C" int rt_layer_forward_timed(const void* x, const void* W_q, const void
     }
   }
   return RT_OK;
+}
+
+// Self-test of the bounded wait: one thread waits on a barrier that nothing
+// arrives on; the wait must give up after limit_ns and record the timeout.
+namespace rt {
+__global__ void k_selftest_wait(unsigned* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_wait(&bar, 0, err, limit_ns);   // phase 0 never completes
+  }
+}
+}  // namespace rt
+
+extern "C" int rt_selftest_wait_timeout(unsigned long long limit_ns, void* workspace, void* stream) {
+  if (!workspace || limit_ns == 0 || limit_ns > 10000000000ull) return RT_ERR_INVALID_ARG;
+  DevState* ds = nullptr;
+  int rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<unsigned*>(workspace), limit_ns);
+  return cudaGetLastError() == cudaSuccess ? RT_OK : RT_ERR_CUDA;
 }

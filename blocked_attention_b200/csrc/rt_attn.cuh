@@ -224,8 +224,9 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
-// block fold for small blocks (nk <= 8 keys), bf16, d_h = 64: eight lanes per
-// (b, h, query), eight dims (16 bytes of q/k/v, 32 bytes of o) per lane.
+// block fold for small blocks (used for up to 8 keys), bf16, d_h = 64: eight
+// lanes per (b, h, query), eight dims (16 bytes of q/k/v, 32 bytes of o) per
+// lane; keys in groups of eight with online rescaling between groups.
 // fin = 1: the first query of the block (q0) receives no later fold, so it
 // is finalised here -- its temporary pair is merged and a_{q0} = o / l is
 // written to a_out [B][d]; its (m, l, o) are not stored.
@@ -273,39 +274,44 @@ __global__ void __launch_bounds__(256)
     oo[0] = a0.x; oo[1] = a0.y; oo[2] = a0.z; oo[3] = a0.w;
     oo[4] = a1.x; oo[5] = a1.y; oo[6] = a1.z; oo[7] = a1.w;
   }
-  float s[KMAX];
-  float mx = -INFINITY;
+  float mn = mo;
+  for (int c0 = 0; c0 < nk; c0 += KMAX) {
+    const int n = min(KMAX, nk - c0);
+    float s[KMAX];
+    float mx = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    s[i] = -INFINITY;
-    if (i < nk) {
-      float kk[8];
-      load_bf16x8(K + ((size_t)(k0 + i) * B + b) * kv_stride + h * DH + sl * 8, kk);
-      float dot = 0.f;
+    for (int i = 0; i < KMAX; ++i) {
+      s[i] = -INFINITY;
+      if (i < n) {
+        float kk[8];
+        load_bf16x8(K + ((size_t)(k0 + c0 + i) * B + b) * kv_stride + h * DH + sl * 8, kk);
+        float dot = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
-      dot += __shfl_xor_sync(omask, dot, 1);
-      dot += __shfl_xor_sync(omask, dot, 2);
-      dot += __shfl_xor_sync(omask, dot, 4);
-      s[i] = dot * sc2;
-      mx = fmaxf(mx, s[i]);
+        for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
+        dot += __shfl_xor_sync(omask, dot, 1);
+        dot += __shfl_xor_sync(omask, dot, 2);
+        dot += __shfl_xor_sync(omask, dot, 4);
+        s[i] = dot * sc2;
+        mx = fmaxf(mx, s[i]);
+      }
     }
-  }
-  const float mn = fmaxf(mo, mx);
-  const float al = rescale(mo, mn);
-  lo *= al;
+    const float m_new = fmaxf(mn, mx);
+    const float al = rescale(mn, m_new);
+    lo *= al;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) oo[e] *= al;
+    for (int e = 0; e < 8; ++e) oo[e] *= al;
 #pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    if (i < nk) {
-      const float p = exp2f(s[i] - mn);
-      float vv[8];
-      load_bf16x8(V + ((size_t)(k0 + i) * B + b) * kv_stride + h * DH + sl * 8, vv);
-      lo += p;
+    for (int i = 0; i < KMAX; ++i) {
+      if (i < n) {
+        const float p = exp2f(s[i] - m_new);
+        float vv[8];
+        load_bf16x8(V + ((size_t)(k0 + c0 + i) * B + b) * kv_stride + h * DH + sl * 8, vv);
+        lo += p;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
+        for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
+      }
     }
+    mn = m_new;
   }
   if (fin && qi == 0) {
     float kt[8], vt[8];
@@ -380,13 +386,17 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 }
 }  // namespace mma_detail
 
+// P (b, h) pairs per CTA: P = 1 for blocks >= 64 keys (64 queries of one pair,
+// keys in 64-key chunks); P = 2 / 4 for 32- / 16-key blocks (64/P queries and
+// the 64/P keys of each pair share one 64-row tile), so no warp idles.
+template <int P>
 __global__ void __launch_bounds__(128)
     k_fold_mma(const __nv_bfloat16* __restrict__ Q, int q_stride, const __nv_bfloat16* __restrict__ K,
                const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m,
                float* __restrict__ l, float* __restrict__ o, __nv_bfloat16* __restrict__ a_out, int B, int H,
                int q0, int nq, int k0, int nk, float sc2, int init, int fin) {
   using namespace mma_detail;
-  constexpr int DH = 64, QT = 64, KC = 64;
+  constexpr int DH = 64, QT = 64, KC = 64, QTP = QT / P, KCP = KC / P;
   __shared__ __align__(128) __nv_bfloat16 sQ[QT * LDS];
   __shared__ __align__(128) __nv_bfloat16 sK[2][KC * LDS];
   __shared__ __align__(128) __nv_bfloat16 sV[2][KC * LDS];
@@ -394,34 +404,47 @@ __global__ void __launch_bounds__(128)
   pdl_wait();
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int pair = blockIdx.y;
-  const int b = pair / H, h = pair - b * H;
+  const int npairs = B * H;
   const int d = H * DH;
-  const int qt0 = q0 + blockIdx.x * QT;
-  const int nrows = min(QT, q0 + nq - qt0);
+  const int qt0 = q0 + blockIdx.x * QTP;                 // first query of every pair in this CTA
+  const int nrows = min(QTP, q0 + nq - qt0);             // valid query rows per pair
+  // pair of tile row r (query rows and key rows alike)
+  auto pair_of = [&](int r) { return (int)blockIdx.y * P + r / QTP; };
 
-  // Q tile (rows beyond nrows are zero)
+  // Q tile (rows beyond nrows, or of a missing pair, are zero)
   for (int c = tid; c < QT * 8; c += 128) {
     const int r = c >> 3, cc = c & 7;
+    const int pr = pair_of(r), qr = r % QTP;
     __nv_bfloat16* dst = &sQ[r * LDS + cc * 8];
-    if (r < nrows)
-      cp_async16(dst, Q + ((size_t)(qt0 + r) * B + b) * q_stride + h * DH + cc * 8);
-    else
+    if (qr < nrows && pr < npairs) {
+      const int b = pr / H, h = pr - b * H;
+      cp_async16(dst, Q + ((size_t)(qt0 + qr) * B + b) * q_stride + h * DH + cc * 8);
+    } else {
       *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
   }
+  // keys [kc0, kc0 + kcn) of every pair; pair p occupies rows p*KCP .. p*KCP + KCP - 1
   auto load_kv = [&](int buf, int kc0, int kcn) {
-    for (int c = tid; c < kcn * 8; c += 128) {
+    for (int c = tid; c < KC * 8; c += 128) {
       const int r = c >> 3, cc = c & 7;
-      const size_t src = ((size_t)(k0 + kc0 + r) * B + b) * kv_stride + h * DH + cc * 8;
-      cp_async16(&sK[buf][r * LDS + cc * 8], K + src);
-      cp_async16(&sV[buf][r * LDS + cc * 8], V + src);
+      const int pr = (int)blockIdx.y * P + r / KCP, kr = r % KCP;
+      if (kr < kcn && pr < npairs) {
+        const int b = pr / H, h = pr - b * H;
+        const size_t src = ((size_t)(k0 + kc0 + kr) * B + b) * kv_stride + h * DH + cc * 8;
+        cp_async16(&sK[buf][r * LDS + cc * 8], K + src);
+        cp_async16(&sV[buf][r * LDS + cc * 8], V + src);
+      }
     }
   };
-  load_kv(0, 0, min(KC, nk));
+  load_kv(0, 0, min(KCP, nk));
   cp_async_commit();
 
-  const int nchunks = (nk + KC - 1) / KC;
-  const bool warp_active = warp * 16 < nrows;
+  const int wpair = pair_of(warp * 16);                  // this warp's pair
+  const int wq0 = (warp * 16) % QTP;                     // its first query row within the pair
+  const int kbase = (warp * 16 / QTP) * KCP;             // its pair's first key row in sK / sV
+  const int b = wpair / H, h = wpair - (wpair / H) * H;
+  const int nchunks = (nk + KCP - 1) / KCP;
+  const bool warp_active = wq0 < nrows && wpair < npairs;
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
   float oacc[8][4];
 #pragma unroll
@@ -431,7 +454,7 @@ __global__ void __launch_bounds__(128)
   for (int ci = 0; ci < nchunks; ++ci) {
     const int buf = ci & 1;
     if (ci + 1 < nchunks) {
-      load_kv(buf ^ 1, (ci + 1) * KC, min(KC, nk - (ci + 1) * KC));
+      load_kv(buf ^ 1, (ci + 1) * KCP, min(KCP, nk - (ci + 1) * KCP));
       cp_async_commit();
       cp_async_wait<1>();
     } else {
@@ -444,7 +467,7 @@ __global__ void __launch_bounds__(128)
         for (int ks = 0; ks < 4; ++ks)
           ldsm_x4(qf[ks], &sQ[(warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + ks * 16 + (lane >> 4) * 8]);
       }
-      const int kcn = min(KC, nk - ci * KC);
+      const int kcn = min(KCP, nk - ci * KCP);
       const int ntiles = kcn >> 3;  // even: kcn is a multiple of 16
       float sacc[8][4];
 #pragma unroll
@@ -454,7 +477,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
             uint32_t r[4];
-            ldsm_x4(r, &sK[buf][(nt * 8 + (lane & 7)) * LDS + kk * 32 + (lane >> 3) * 8]);
+            ldsm_x4(r, &sK[buf][(kbase + nt * 8 + (lane & 7)) * LDS + kk * 32 + (lane >> 3) * 8]);
             mma16816(sacc[nt], qf[2 * kk], r[0], r[1]);
             mma16816(sacc[nt], qf[2 * kk + 1], r[2], r[3]);
           }
@@ -507,7 +530,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
           for (int nd = 0; nd < 8; nd += 2) {
             uint32_t r[4];
-            ldsm_x4_t(r, &sV[buf][(kj * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + nd * 8 + (lane >> 4) * 8]);
+            ldsm_x4_t(r, &sV[buf][(kbase + kj * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + nd * 8 + (lane >> 4) * 8]);
             mma16816(oacc[nd], pa, r[0], r[1]);
             mma16816(oacc[nd + 1], pa, r[2], r[3]);
           }
@@ -524,7 +547,7 @@ __global__ void __launch_bounds__(128)
     float lsum = lrow[rr];
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-    const int r = warp * 16 + (lane >> 2) + rr * 8;
+    const int r = wq0 + (lane >> 2) + rr * 8;             // query row within the pair
     if (r >= nrows) continue;
     const size_t row = (size_t)(qt0 + r) * B + b;
     float mg = -INFINITY, lg = 0.f;
@@ -544,11 +567,12 @@ __global__ void __launch_bounds__(128)
     if (fin && blockIdx.x == 0 && r == 0) {
       // query q0 receives no later fold: merge its temporary pair, write a_{q0}
       const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * DH + (lane & 3) * 2;
+      const __nv_bfloat16* qrow = &sQ[(warp * 16) * LDS];   // tile row of this pair's query q0
       float dot = 0.f;
 #pragma unroll
       for (int nd = 0; nd < 8; ++nd) {
         const float2 kt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tp + d + nd * 8));
-        const float2 qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sQ[nd * 8 + (lane & 3) * 2]));
+        const float2 qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qrow[nd * 8 + (lane & 3) * 2]));
         dot += qv.x * kt.x + qv.y * kt.y;
       }
       dot += __shfl_xor_sync(0xFu, dot, 1);

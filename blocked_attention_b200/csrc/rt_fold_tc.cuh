@@ -5,7 +5,8 @@
 // paper §5: when (k_t, v_t) is revealed, keys (t - lowbit(t), t] are folded
 // into queries (t, t + lowbit(t)]). bf16 q/k/v, d_h = 64, nk a multiple of 128.
 //
-// CTA = one (sequence b, head h) and 128 queries; 192 threads:
+// Persistent CTAs (one per SM) loop over work items = one (sequence b, head h)
+// and 128 queries each; 192 threads:
 //   warp 0     : TMA producer (3-D boxes over the position-major cache:
 //                128 positions x 64 dims of one (b, h))
 //   warp 1     : TMEM allocator + MMA issuer
@@ -27,14 +28,14 @@
 namespace rt {
 
 struct FoldTcCfg {
-  static constexpr int QT = 128, KC = 128, DH = 64;
+  static constexpr int QT = 128, KC = 128, DH = 64, KVS = 3;
   static constexpr uint32_t Q_BYTES = QT * DH * 2;    // 16 KB
   static constexpr uint32_t KV_BYTES = KC * DH * 2;   // 16 KB (K or V chunk)
   static constexpr uint32_t P_BYTES = QT * KC * 2;    // 32 KB (two 64-key swizzle atoms)
-  static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
-  static constexpr uint32_t OFF_V = OFF_K + 2 * KV_BYTES;
-  static constexpr uint32_t OFF_P = OFF_V + 2 * KV_BYTES;
+  static constexpr uint32_t OFF_Q = 0;                             // [2]
+  static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;           // [KVS]
+  static constexpr uint32_t OFF_V = OFF_K + KVS * KV_BYTES;        // [KVS]
+  static constexpr uint32_t OFF_P = OFF_V + KVS * KV_BYTES;        // [2]
   static constexpr uint32_t OFF_BAR = OFF_P + 2 * P_BYTES;
   static constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 256;
   static constexpr uint32_t TMEM_COLS = 512;          // S[2] at 0/128, O[2] at 256/320
@@ -66,6 +67,11 @@ __device__ __forceinline__ void fence_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Persistent: CTA i takes work items i, i + gridDim.x, ... where an item is one
+// (b, h) pair and one tile of 128 queries (query tile fastest). All its chunks
+// form one global sequence g = 0, 1, ... (chunk c = g % nch of local item
+// g / nch), so the K/V ring, S/P/O buffers and their barrier phases run on
+// across items and the next item's Q and K/V load while the current finishes.
 __global__ void __launch_bounds__(192, 1)
     k_fold_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __nv_bfloat16* __restrict__ Q, int q_stride,
@@ -75,37 +81,48 @@ __global__ void __launch_bounds__(192, 1)
   using C = FoldTcCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + C::OFF_Q;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;     // [2]
-  uint64_t* s_free = bars + 7;     // [2]
-  uint64_t* p_full = bars + 9;     // [2]
-  uint64_t* o_full = bars + 11;    // [2]
-  uint64_t* o_free = bars + 13;    // [2]
-  uint64_t* mma_done = bars + 15;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars + 0;     // [2]
+  uint64_t* q_empty = bars + 2;    // [2]
+  uint64_t* kv_full = bars + 4;    // [KVS]
+  uint64_t* kv_empty = bars + 7;   // [KVS]
+  uint64_t* s_full = bars + 10;    // [2]
+  uint64_t* s_free = bars + 12;    // [2]
+  uint64_t* p_full = bars + 14;    // [2]
+  uint64_t* o_full = bars + 16;    // [2]
+  uint64_t* o_free = bars + 18;    // [2]
+  uint64_t* mma_done = bars + 20;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 21);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.y;
-  const int b = pair / H, h = pair - b * H;
   const int d = H * C::DH;
-  const int qt0 = q0 + blockIdx.x * C::QT;
-  const int nrows = min(C::QT, q0 + nq - qt0);
-  const int nchunks = nk / C::KC;
+  const int ntq = (nq + C::QT - 1) / C::QT;
+  const int nitems = B * H * ntq;
+  const int nch = nk / C::KC;
+  // items of this CTA and its total chunk count
+  const int my_items = blockIdx.x < nitems ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int total = my_items * nch;
+  auto item_of = [&](int li, int& b, int& h, int& qt0) {
+    const int it = (int)blockIdx.x + li * (int)gridDim.x;
+    const int pair = it / ntq, qt = it - pair * ntq;
+    b = pair / H;
+    h = pair - b * H;
+    qt0 = q0 + qt * C::QT;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 5);   // the MMA thread's commit + the four softmax warps
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
       mbar_init(&p_full[i], 4);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_free[i], 4);
+    }
+    for (int i = 0; i < C::KVS; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
     mbar_init(mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -126,21 +143,30 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-      tma_load_3d(&tmQ, q_full, sQ, h * C::DH, b, qt0);
-      int c = 0;
-      for (; c < nchunks; ++c) {
-        const int st = c & 1;
-        const uint32_t ph = (c >> 1) & 1u;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1u, err)) break;
-        mbar_arrive_expect_tx(&kv_full[st], 2 * C::KV_BYTES);
-        tma_load_3d(&tmK, &kv_full[st], smem + C::OFF_K + st * C::KV_BYTES, h * C::DH, b, k0 + c * C::KC);
-        tma_load_3d(&tmV, &kv_full[st], smem + C::OFF_V + st * C::KV_BYTES, h * C::DH, b, k0 + c * C::KC);
+      int g = 0;
+      bool ok = true;
+      int issued_q = 0;
+      for (int li = 0; li < my_items && ok; ++li) {
+        int b, h, qt0;
+        item_of(li, b, h, qt0);
+        const int qb = li & 1;
+        if (!mbar_wait(&q_empty[qb], ((li >> 1) & 1u) ^ 1u, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
+        tma_load_3d(&tmQ, &q_full[qb], smem + C::OFF_Q + qb * C::Q_BYTES, h * C::DH, b, qt0);
+        ++issued_q;
+        for (int c = 0; c < nch; ++c, ++g) {
+          const int st = g % C::KVS;
+          const uint32_t ph = (g / C::KVS) & 1u;
+          if (!mbar_wait(&kv_empty[st], ph ^ 1u, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&kv_full[st], 2 * C::KV_BYTES);
+          tma_load_3d(&tmK, &kv_full[st], smem + C::OFF_K + st * C::KV_BYTES, h * C::DH, b, k0 + c * C::KC);
+          tma_load_3d(&tmV, &kv_full[st], smem + C::OFF_V + st * C::KV_BYTES, h * C::DH, b, k0 + c * C::KC);
+        }
       }
-      if (c < nchunks) {
+      if (!ok) {
         // aborted: wait (bounded) for the copies this thread issued
-        mbar_wait(q_full, 0, err);
-        for (int i = (c >= 2 ? c - 2 : 0); i < c; ++i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1u, err);
+        for (int i = (issued_q >= 2 ? issued_q - 2 : 0); i < issued_q; ++i) mbar_wait(&q_full[i & 1], (i >> 1) & 1u, err);
+        for (int i = (g >= C::KVS ? g - C::KVS : 0); i < g; ++i) mbar_wait(&kv_full[i % C::KVS], (i / C::KVS) & 1u, err);
       }
     }
   } else if (warp == 1) {
@@ -148,27 +174,31 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, 128);
       const uint32_t idesc_o = idesc_bf16_f32(128, 64) | (1u << 16);   // B (= V) MN-major
-      bool ok = mbar_wait(q_full, 0, err);
-      auto issue_s = [&](int c) -> bool {
-        const int st = c & 1;
-        const uint32_t ph = (c >> 1) & 1u;
-        if (!mbar_wait(&kv_full[st], ph, err) || !mbar_wait(&s_free[st], ph ^ 1u, err)) return false;
+      bool ok = true;
+      auto issue_s = [&](int g) -> bool {
+        const int li = g / nch, c = g - li * nch;
+        const int qb = li & 1, st = g % C::KVS, bb = g & 1;
+        if (c == 0 && !mbar_wait(&q_full[qb], (li >> 1) & 1u, err)) return false;
+        if (!mbar_wait(&kv_full[st], (g / C::KVS) & 1u, err) || !mbar_wait(&s_free[bb], ((g >> 1) & 1u) ^ 1u, err))
+          return false;
         tc_fence_after();
+        const uint8_t* qt = smem + C::OFF_Q + qb * C::Q_BYTES;
         const uint8_t* kt = smem + C::OFF_K + st * C::KV_BYTES;
 #pragma unroll
         for (int k = 0; k < C::DH / 16; ++k)
-          tc_mma_f16(tmem_base + st * 128, smem_desc_sw128(sQ + k * 32), smem_desc_sw128(kt + k * 32), idesc_s,
+          tc_mma_f16(tmem_base + bb * 128, smem_desc_sw128(qt + k * 32), smem_desc_sw128(kt + k * 32), idesc_s,
                      k != 0 ? 1u : 0u);
-        tc_commit(&s_full[st]);
+        tc_commit(&s_full[bb]);
         return true;
       };
-      auto issue_pv = [&](int c) -> bool {
-        const int bb = c & 1;
-        const uint32_t ph = (c >> 1) & 1u;
+      auto issue_pv = [&](int g) -> bool {
+        const int li = g / nch, c = g - li * nch;
+        const int st = g % C::KVS, bb = g & 1;
+        const uint32_t ph = (g >> 1) & 1u;
         if (!mbar_wait(&p_full[bb], ph, err) || !mbar_wait(&o_free[bb], ph ^ 1u, err)) return false;
         tc_fence_after();
         const uint8_t* pt = smem + C::OFF_P + bb * C::P_BYTES;
-        const uint8_t* vt = smem + C::OFF_V + bb * C::KV_BYTES;
+        const uint8_t* vt = smem + C::OFF_V + st * C::KV_BYTES;
 #pragma unroll
         for (int ks = 0; ks < C::KC / 16; ++ks) {
           // A = P: K-major, 64-key atoms 16 KB apart, 32 bytes per 16 keys inside an atom
@@ -177,13 +207,14 @@ __global__ void __launch_bounds__(192, 1)
                      smem_desc_sw128_mn(vt + ks * 16 * 128), idesc_o, ks != 0 ? 1u : 0u);
         }
         tc_commit(&o_full[bb]);
-        tc_commit(&kv_empty[bb]);
+        tc_commit(&kv_empty[st]);
+        if (c == nch - 1) tc_commit(&q_empty[li & 1]);   // the item's S products are all done
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int c = 0; c < nchunks && ok; ++c) {
-        if (c + 1 < nchunks) ok = issue_s(c + 1);
-        if (ok) ok = issue_pv(c);
+      if (total > 0) ok = issue_s(0);
+      for (int g = 0; g < total && ok; ++g) {
+        if (g + 1 < total) ok = issue_s(g + 1);
+        if (ok) ok = issue_pv(g);
       }
       // every MMA this thread issued has finished before the CTA can free TMEM
       tc_commit(mma_done);
@@ -197,8 +228,6 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* sP = smem + C::OFF_P;
     float m_run = -INFINITY, l_run = 0.f, alpha_prev = 0.f;
     float oacc[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) oacc[i] = 0.f;
     bool ok = true;
 
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -206,9 +235,9 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) v = mbar_wait(bar, parity, err) ? 1 : 0;
       return __shfl_sync(0xffffffffu, v, 0) != 0;
     };
-    auto accumulate = [&](int c, float alpha) -> bool {
-      const int bb = c & 1;
-      if (!wait_warp(&o_full[bb], (c >> 1) & 1u)) return false;
+    auto accumulate = [&](int g, float alpha) -> bool {
+      const int bb = g & 1;
+      if (!wait_warp(&o_full[bb], (g >> 1) & 1u)) return false;
       tc_fence_after();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -223,10 +252,75 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) mbar_arrive(&o_free[bb]);
       return true;
     };
+    // merge the finished item li into the global statistics (or finalise q0)
+    auto merge = [&](int li) {
+      int b, h, qt0;
+      item_of(li, b, h, qt0);
+      const int nrows = min(C::QT, q0 + nq - qt0);
+      if (r < nrows) {
+        const size_t row = (size_t)(qt0 + r) * B + b;
+        float mg = -INFINITY, lg = 0.f;
+        float* op = o + row * (size_t)d + h * C::DH;
+        if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }
+        const float mn = fmaxf(mg, m_run);
+        const float ag = rescale(mg, mn), ab = rescale(m_run, mn);
+        const float ln = lg * ag + l_run * ab;
+        if (fin && qt0 == q0 && r == 0) {
+          // query q0 receives no later fold: merge its temporary pair, write a_{q0}
+          const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * C::DH;
+          const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(smem + C::OFF_Q + (li & 1) * C::Q_BYTES);
+          float dot = 0.f;
+#pragma unroll 8
+          for (int e = 0; e < C::DH; ++e) dot += __bfloat162float(qrow[e]) * __bfloat162float(tp[d + e]);
+          const float s2 = dot * sc2;
+          const float m2 = fmaxf(mn, s2);
+          const float a2 = rescale(mn, m2), pt = exp2f(s2 - m2);
+          const float inv = 1.f / (ln * a2 + pt);
+          __nv_bfloat16* ap = a_out + (size_t)b * d + h * C::DH;
+#pragma unroll
+          for (int e = 0; e < C::DH; e += 2) {
+            float og0 = 0.f, og1 = 0.f;
+            if (!init) { og0 = op[e]; og1 = op[e + 1]; }
+            const float o0 = og0 * ag + oacc[e] * ab, o1 = og1 * ag + oacc[e + 1] * ab;
+            const float2 vt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tp + 2 * d + e));
+            *reinterpret_cast<__nv_bfloat162*>(ap + e) =
+                __floats2bfloat162_rn((o0 * a2 + pt * vt.x) * inv, (o1 * a2 + pt * vt.y) * inv);
+          }
+        } else {
+          m[row * H + h] = mn;
+          l[row * H + h] = ln;
+#pragma unroll
+          for (int e = 0; e < C::DH; e += 4) {
+            float4 og = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!init) og = *reinterpret_cast<const float4*>(op + e);
+            og.x = og.x * ag + oacc[e] * ab;
+            og.y = og.y * ag + oacc[e + 1] * ab;
+            og.z = og.z * ag + oacc[e + 2] * ab;
+            og.w = og.w * ag + oacc[e + 3] * ab;
+            *reinterpret_cast<float4*>(op + e) = og;
+          }
+        }
+      }
+      // this item's Q buffer may be refilled (the MMA thread also arrives)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[li & 1]);
+    };
 
-    for (int c = 0; c < nchunks && ok; ++c) {
-      const int bb = c & 1;
-      if (!wait_warp(&s_full[bb], (c >> 1) & 1u)) { ok = false; break; }
+    for (int g = 0; g < total && ok; ++g) {
+      const int li = g / nch, c = g - li * nch;
+      const int bb = g & 1;
+      if (c == 0) {
+        if (g > 0) {
+          // finish the previous item before its running state is reset
+          if (!accumulate(g - 1, alpha_prev)) { ok = false; break; }
+          merge(li - 1);
+        }
+        m_run = -INFINITY;
+        l_run = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) oacc[i] = 0.f;
+      }
+      if (!wait_warp(&s_full[bb], (g >> 1) & 1u)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sbase = tmem_base + lane_base + bb * 128;
       float mx = -INFINITY;
@@ -249,11 +343,11 @@ __global__ void __launch_bounds__(192, 1)
         tmem_ld_wait();
         uint8_t* atom = prow + (cc >> 1) * 16384;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int gq = 0; gq < 4; ++gq) {
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            p[e] = exp2f(__uint_as_float(rv[g * 8 + e]) * sc2 - m_new);
+            p[e] = exp2f(__uint_as_float(rv[gq * 8 + e]) * sc2 - m_new);
             lsum += p[e];
           }
           uint4 w;
@@ -261,7 +355,7 @@ __global__ void __launch_bounds__(192, 1)
           w.y = pack_bf16x2(p[2], p[3]);
           w.z = pack_bf16x2(p[4], p[5]);
           w.w = pack_bf16x2(p[6], p[7]);
-          const int chunk = (cc & 1) * 4 + g;
+          const int chunk = (cc & 1) * 4 + gq;
           *reinterpret_cast<uint4*>(atom + ((chunk ^ (r & 7)) << 4)) = w;
         }
       }
@@ -274,55 +368,10 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(&s_free[bb]);
         mbar_arrive(&p_full[bb]);
       }
-      if (c > 0 && !accumulate(c - 1, alpha_prev)) { ok = false; break; }
+      if (c > 0 && !accumulate(g - 1, alpha_prev)) { ok = false; break; }
       alpha_prev = alpha;
     }
-    if (ok && nchunks > 0) ok = accumulate(nchunks - 1, alpha_prev);
-
-    if (ok && r < nrows) {
-      const size_t row = (size_t)(qt0 + r) * B + b;
-      float mg = -INFINITY, lg = 0.f;
-      float* op = o + row * (size_t)d + h * C::DH;
-      if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }
-      const float mn = fmaxf(mg, m_run);
-      const float ag = rescale(mg, mn), ab = rescale(m_run, mn);
-      const float ln = lg * ag + l_run * ab;
-      if (fin && blockIdx.x == 0 && r == 0) {
-        // query q0 receives no later fold: merge its temporary pair, write a_{q0}
-        const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * C::DH;
-        float dot = 0.f;
-#pragma unroll 8
-        for (int e = 0; e < C::DH; ++e)
-          dot += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(sQ)[e]) * __bfloat162float(tp[d + e]);
-        const float s2 = dot * sc2;
-        const float m2 = fmaxf(mn, s2);
-        const float a2 = rescale(mn, m2), pt = exp2f(s2 - m2);
-        const float inv = 1.f / (ln * a2 + pt);
-        __nv_bfloat16* ap = a_out + (size_t)b * d + h * C::DH;
-#pragma unroll
-        for (int e = 0; e < C::DH; e += 2) {
-          float og0 = 0.f, og1 = 0.f;
-          if (!init) { og0 = op[e]; og1 = op[e + 1]; }
-          const float o0 = og0 * ag + oacc[e] * ab, o1 = og1 * ag + oacc[e + 1] * ab;
-          const float2 vt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tp + 2 * d + e));
-          *reinterpret_cast<__nv_bfloat162*>(ap + e) =
-              __floats2bfloat162_rn((o0 * a2 + pt * vt.x) * inv, (o1 * a2 + pt * vt.y) * inv);
-        }
-      } else {
-        m[row * H + h] = mn;
-        l[row * H + h] = ln;
-#pragma unroll
-        for (int e = 0; e < C::DH; e += 4) {
-          float4 og = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (!init) og = *reinterpret_cast<const float4*>(op + e);
-          og.x = og.x * ag + oacc[e] * ab;
-          og.y = og.y * ag + oacc[e + 1] * ab;
-          og.z = og.z * ag + oacc[e + 2] * ab;
-          og.w = og.w * ag + oacc[e + 3] * ab;
-          *reinterpret_cast<float4*>(op + e) = og;
-        }
-      }
-    }
+    if (ok && total > 0 && accumulate(total - 1, alpha_prev)) merge(my_items - 1);
   }
   __syncthreads();
   if (warp == 1) {

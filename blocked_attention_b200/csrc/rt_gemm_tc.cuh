@@ -48,14 +48,34 @@ struct EpiParams {
   __nv_bfloat16* z16;        // W2 out: [B][d]
   __nv_bfloat16* Kout;       // WKV out: [N][B][d]
   __nv_bfloat16* Vout;
-  // split-K: `splits` CTAs share one output tile, each over K/splits; they
-  // write fp32 partial tiles to `part`, and the last to arrive (counted in
-  // `counters`, one per output tile, left at zero) sums them in split order
-  // and runs the epilogue.
+  // split-K: `splits` CTAs (one thread-block cluster, launched with cluster
+  // dimension `splits`) share one output tile, each over K/splits; each
+  // stages its fp32 partial tile in its own shared memory, and after a
+  // cluster barrier CTA rank r sums rows [r*128/splits, (r+1)*128/splits) of
+  // all ranks' partials over distributed shared memory, in rank order, and
+  // runs the epilogue for them. BN/splits must be a multiple of 32.
   int splits;
-  float* part;
-  unsigned* counters;
 };
+
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 dsmem_ld_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -195,12 +215,11 @@ __global__ void __launch_bounds__(192, 1)
   const int ntn = (N + BN - 1) / BN, ntm = (M + C::BM - 1) / C::BM;
   const int nmn = ntn * ntm;
   const int splits = p.splits > 1 ? p.splits : 1;
+  // splits == 1: persistent loop over output tiles; splits > 1: one tile per
+  // CTA, tile = mn * splits + ks, so a cluster of `splits` CTAs holds one mn.
   const int num_tiles = nmn * splits;
   const int nk = K / C::BK / splits;   // k-blocks per split (the host keeps this exact)
-  __shared__ int s_last, s_abort;
   if (threadIdx.x == 0) {
-    s_last = 0;
-    s_abort = 0;
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -221,7 +240,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int ks = tile / nmn, mn = tile - ks * nmn;
+        const int mn = tile / splits, ks = tile - mn * splits;
         const int mt = mn / ntn, nt = mn - mt * ntn;
         const int kb0 = ks * nk;
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -271,18 +290,12 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;
     uint32_t local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-      const int ks = tile / nmn, mn = tile - ks * nmn;
+      const int mn = tile / splits;
       const int mt = mn / ntn, nt = mn - mt * ntn;
       const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], aph, err) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (splits > 1) {
-        // the split path synchronises the four epilogue warps: leave together
-        if (!ok && lane == 0) s_abort = 1;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        ok = s_abort ? 0 : 1;
-      }
       if (!ok) break;
       tc_fence_after();
       const int lrow = q * 32 + lane;
@@ -308,68 +321,67 @@ __global__ void __launch_bounds__(192, 1)
         if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
           if (row_ok) p.ssq_out[(size_t)nt * p.B + row] = ssq;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
       } else {
-        // 1. this split's partial tile row -> part[ks][mn][lrow][0:BN]
-        float* prow = p.part + ((size_t)(ks * nmn + mn) * C::BM + lrow) * BN;
+        // stage this CTA's partial tile (fp32, rows padded to BN + 4 floats) in the
+        // shared memory of the operand ring: every TMA load and MMA has completed
+        fence_proxy_async_smem();
+        float* stage = reinterpret_cast<float*>(smem) + (size_t)lrow * (BN + 4);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(taddr + c, r);
           tmem_ld_wait();
-          if (row_ok) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              reinterpret_cast<float4*>(prow + c)[i] =
-                  make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                              __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-          }
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(stage + c)[i] =
+                make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
+                            __uint_as_float(r[4 * i + 3]));
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
-        // 2. count arrivals; the last CTA of this output tile reduces
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (threadIdx.x == 64) {
-          const unsigned old = atomicAdd(&p.counters[mn], 1u);
-          const int last = old == (unsigned)(splits - 1);
-          if (last) p.counters[mn] = 0u;   // every split has arrived: reset for the next use
-          s_last = last;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (s_last) {
-          __threadfence();
-          const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
-          float ssq = 0.f;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  if (splits > 1) {
+    // one output tile per cluster: reduce the ranks' partials over DSMEM
+    cluster_sync();
+    if (warp >= 2) {
+      const int t = threadIdx.x - 64;                  // 0..127
+      const int rank = blockIdx.x % splits;            // == %cluster_ctarank for a 1-D cluster of `splits`
+      const int mn = blockIdx.x / splits;
+      const int mt = mn / ntn, nt = mn - mt * ntn;
+      const int rows_per = C::BM / splits, cpt = BN / splits;
+      const int lrow = rank * rows_per + t / splits;
+      const int cbase = (t % splits) * cpt;
+      const int row = mt * C::BM + lrow;
+      const bool row_ok = row < M && blockIdx.x < num_tiles;
+      const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
+      const uint32_t my = smem_u32(reinterpret_cast<float*>(smem) + (size_t)lrow * (BN + 4) + cbase);
+      float ssq = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
-            const int col0 = nt * BN + c;
-            if (row_ok && col0 < N) {
-              float v[32];
+      for (int c = 0; c < cpt; c += 32) {
+        float v[32];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = 0.f;
-              for (int sp = 0; sp < splits; ++sp) {
-                const float4* src =
-                    reinterpret_cast<const float4*>(p.part + ((size_t)(sp * nmn + mn) * C::BM + lrow) * BN + c);
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        for (int rr = 0; rr < splits; ++rr) {
+          const uint32_t src = dsmem_map(my + c * 4, (uint32_t)rr);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float4 w = __ldcg(src + i);
-                  v[4 * i] += w.x; v[4 * i + 1] += w.y; v[4 * i + 2] += w.z; v[4 * i + 3] += w.w;
-                }
-              }
-              ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
-            }
-          }
-          if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
-            if (row_ok) p.ssq_out[(size_t)nt * p.B + row] = ssq;
+          for (int i = 0; i < 8; ++i) {
+            const float4 w = dsmem_ld_f4(src + i * 16);
+            v[4 * i] += w.x; v[4 * i + 1] += w.y; v[4 * i + 2] += w.z; v[4 * i + 3] += w.w;
           }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");   // s_last is reused by the next tile
+        const int col0 = nt * BN + cbase + c;
+        if (row_ok && col0 < N) ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
+      }
+      if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
+        // the `splits` consecutive lanes sharing a row add their column sums
+        for (int o = 1; o < splits; o <<= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+        if (row_ok && (t % splits) == 0) p.ssq_out[(size_t)nt * p.B + row] = ssq;
       }
     }
+    cluster_sync();   // peers may still read this CTA's staging until here
   }
   __syncthreads();
   if (warp == 1) {

@@ -27,7 +27,8 @@ WEIGHT_NAMES = ("W_q", "W_k", "W_v", "W_o", "W_1", "W_2")
 EXPORTS = ("rt_version", "rt_status_string", "rt_layer_workspace_bytes", "rt_layer_forward",
            "rt_layer_sync_status", "rt_layer_host_workspace_bytes", "rt_layer_forward_host",
            "rt_embed_forward", "rt_block_fold", "rt_project_qkv", "rt_gemm_bf16",
-           "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc")
+           "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc",
+           "rt_selftest_wait_timeout")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma")
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
                                                                          ctypes.POINTER(ctypes.c_int), i]
     L.rt_project_qkv_noalloc.restype = i
     L.rt_project_qkv_noalloc.argtypes = [vp, vp, i, i, i, vp, vp]
+    L.rt_selftest_wait_timeout.restype = i
+    L.rt_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp, vp]
     _lib = L
     return L
 
@@ -189,6 +192,11 @@ def layer_forward_timed(x: torch.Tensor, W: dict, H: int, out, workspace: torch.
         if cnt[c] > 0:
             out[f"fold_lb{1 << lv}"] = (float(ms[c]), int(cnt[c]))
     return out
+
+
+def selftest_wait_timeout(limit_ns: int, workspace: torch.Tensor, stream=None):
+    """Enqueue the bounded-wait self-test (see rt_selftest_wait_timeout)."""
+    _check("rt_selftest_wait_timeout", lib().rt_selftest_wait_timeout(int(limit_ns), _ptr(workspace), _stream(stream)))
 
 
 def sync_status(workspace: torch.Tensor, stream=None) -> int:

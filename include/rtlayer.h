@@ -218,6 +218,15 @@ int rt_layer_forward_timed(const void* x_dev,
                            void* workspace_dev, size_t workspace_bytes, void* stream,
                            float* class_ms, int* class_launches, int n_classes);
 
+/* Failure-detection self-test: enqueues one kernel whose single thread waits
+ * on a shared-memory barrier that nothing ever arrives on, through the same
+ * bounded wait every kernel of this library uses, with a limit of limit_ns
+ * nanoseconds (1 .. 1e10). The wait gives up, records the timeout in the
+ * error word at workspace_dev (as rt_layer_forward's kernels do) and the
+ * kernel exits; rt_layer_sync_status(workspace_dev, stream) then returns
+ * RT_ERR_TIMEOUT. Nothing traps or hangs. */
+int rt_selftest_wait_timeout(unsigned long long limit_ns, void* workspace_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -72,10 +72,11 @@ def test_batched_projection_matches_oracle(rt, dtype, B, N, d):
 @pytest.mark.parametrize("dtype,nk,nq,init_empty", [
     ("bf16", 1, 1, False), ("bf16", 2, 2, True), ("bf16", 8, 5, False),      # small-block kernel (nk <= 8)
     ("bf16", 16, 16, False), ("bf16", 32, 7, False), ("bf16", 64, 64, True),  # mma.sync kernel
-    ("bf16", 48, 20, False),
+    ("bf16", 16, 40, False), ("bf16", 32, 70, True), ("bf16", 96, 65, False),  # (4 / 2 / 1 pairs per CTA)
+    ("bf16", 48, 20, False), ("bf16", 12, 3, False), ("bf16", 27, 9, True),    # generic warp kernel (12, 27)
     ("bf16", 256, 100, False), ("bf16", 1024, 130, False),                     # tcgen05 kernel (nk % 128 == 0)
     ("bf16", 128, 77, False), ("bf16", 128, 128, True), ("bf16", 512, 300, True), ("bf16", 384, 1, False),
-    ("bf16", 12, 3, False),                                                      # generic warp kernel
+    ("bf16", 40, 6, False),                                                      # generic warp kernel
     ("f32", 3, 4, False), ("f32", 16, 16, True), ("f32", 64, 33, False)])
 def test_block_fold_matches_oracle(rt, dtype, nk, nq, init_empty):
     B, H, dh = 3, 2, 64 if dtype == "bf16" else 32
@@ -234,3 +235,13 @@ def test_embedding_out_of_range_id_is_reported(rt):
     x = rt.embed_forward(ids, E, workspace=ws)
     assert rt.sync_status(ws) == rt.RT_ERR_INVALID_ARG
     assert torch.count_nonzero(x[0, 2]) == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_stays_usable(rt):
+    # a barrier nothing arrives on: the wait gives up after 1 ms and reports it
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    rt.selftest_wait_timeout(1_000_000, ws)
+    assert rt.sync_status(ws) == rt.RT_ERR_TIMEOUT
+    assert rt.sync_status(ws) == 0                       # the word was cleared
+    # the context is still usable: a normal forward runs and passes parity
+    _check_layer(rt, 2, 20, 128, 2, 256, "bf16")
