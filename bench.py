@@ -67,10 +67,11 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="sequence-length sweep, blocked vs naive (B=32 d=1024 H=16x64 d_ff=4096)")
     ap.add_argument("--sweep-n", default="512,1024,2048,4096,8192,16384")
-    ap.add_argument("--profile-case", choices=["step", "fold"],
+    ap.add_argument("--profile-case", choices=["step", "fold", "fwd"],
                     help="run one small case for an ncu capture and exit: 'step' = one host-loop forward at "
                          "B=512 N=64 d=1024 (the per-step GEMM shapes of the headline); 'fold' = one block fold "
-                         "of --lb keys into --lb queries at B=64 H=16 (position-major, larger than L2)")
+                         "of --lb keys into --lb queries at B=64 H=16 (position-major, larger than L2); "
+                         "'fwd' = one graph-driver forward at the headline widths with N = --lb")
     ap.add_argument("--lb", type=int, default=1024)
     return ap.parse_args()
 
@@ -349,12 +350,12 @@ def run_sweep(args, R, torch):
 
 def run_profile_case(args, R, torch, rtinputs):
     dev = torch.device("cuda", 0)
-    if args.profile_case == "step":
-        B, N, d, H, dff = 512, 64, 1024, 16, 4096
+    if args.profile_case in ("step", "fwd"):
+        B, N, d, H, dff = 512, (64 if args.profile_case == "step" else args.lb), 1024, 16, 4096
         W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
              for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16").items()}
         x = torch.randn((B, N, d), device=dev, dtype=torch.bfloat16)
-        z, _, _ = R.layer_forward(x, W, H, driver="stream")
+        z, _, _ = R.layer_forward(x, W, H, driver="stream" if args.profile_case == "step" else "graph")
     else:
         LB, B, H, dh = args.lb, 64, 16, 64
         d = H * dh

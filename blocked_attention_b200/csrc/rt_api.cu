@@ -130,7 +130,9 @@ static int device_setup(DevState** out) {
         set_tc_attrs_epi<EPI_W2>() != cudaSuccess || set_tc_attrs_epi<EPI_WKV>() != cudaSuccess)
       return RT_ERR_CUDA;
     if (cudaFuncSetAttribute(k_fold_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)FoldTcCfg::SMEM_BYTES) != cudaSuccess)
+                             (int)FoldTcCfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(k_fold_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)FoldTc2Cfg::SMEM_BYTES) != cudaSuccess)
       return RT_ERR_CUDA;
     if (cudaStreamCreateWithFlags(&ds.capture, cudaStreamNonBlocking) != cudaSuccess) return RT_ERR_CUDA;
     ds.ready = true;
@@ -192,8 +194,8 @@ static TileCfg choose_tiles(int M, int N, int K, bool allow_split) {
 }
 // Per-step GEMMs may use cluster split-K (see choose_tiles).
 static constexpr bool kLayerSplitK = true;
-// Smallest block size that uses the tcgen05 fold (smaller ones: mma.sync);
-// measured: mma.sync is faster up to 512, the tcgen05 fold at 1024.
+// Smallest block size that uses the tcgen05 folds (smaller ones: mma.sync);
+// measured at the headline shape: mma.sync wins up to 512, tcgen05 at 1024.
 static constexpr int kFoldTcMinBlock = 1024;
 
 template <int BN, int EPI>
@@ -367,6 +369,13 @@ static cudaError_t launch_fold(const T* Q, int q_stride, const T* K, const T* V,
       if (!make_tmap_pm(&tq, Q, q_stride, B, q0 + nq) || !make_tmap_pm(&tk, K, kv_stride, B, k0 + nk) ||
           !make_tmap_pm(&tv, V, kv_stride, B, k0 + nk))
         return cudaErrorInvalidValue;
+      if (nq > 128) {
+        // two 128-query tiles per item share every K/V chunk
+        const long items = (long)pairs * ((nq + 255) / 256);
+        const dim3 grid((unsigned)std::min<long>(items, sms));
+        return launch_pdl(k_fold_tc2, grid, dim3(320), FoldTc2Cfg::SMEM_BYTES, st, tq, tk, tv, Q, q_stride, m, l,
+                          o, a_out, B, H, q0, nq, k0, nk, sc2, init, fin, err);
+      }
       const long items = (long)pairs * ((nq + 127) / 128);
       const dim3 grid((unsigned)std::min<long>(items, sms));   // persistent over (pair, query tile) items
       return launch_pdl(k_fold_tc, grid, dim3(192), FoldTcCfg::SMEM_BYTES, st, tq, tk, tv, Q, q_stride, m, l, o,
@@ -411,7 +420,8 @@ static cudaError_t launch_attend(const Plan& P, const T* qkv, const T* K, const 
   if (s.schedule == RT_SCHED_BLOCKED)
     return launch_pdl(k_finalize<T, DPL>, dim3(blocks), dim3(128), 0, st, qkv, m, l, o, a, s.B, s.H, j, sc2,
                       j > 0 ? 1 : 0);
-  return launch_pdl(k_naive_attn<T, DPL>, dim3(blocks), dim3(128), 0, st, qkv, K, V, a, s.B, s.H, j, sc2);
+  // naive schedule: one CTA of 8 warps per (b, h), keys split across the warps
+  return launch_pdl(k_naive_attn<T, DPL>, dim3(s.B * s.H), dim3(256), 0, st, qkv, K, V, a, s.B, s.H, j, sc2);
 }
 
 // ---------------------------------------------------------------------------

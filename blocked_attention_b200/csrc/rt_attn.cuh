@@ -77,40 +77,52 @@ __global__ void __launch_bounds__(128)
 
 // ---------------------------------------------------------------------------
 // naive schedule (ablation): a_j from all persistent pairs i < j plus the
-// temporary pair, streaming keys 32 at a time. One warp per (b, h).
+// temporary pair. One CTA of 8 warps per (b, h): warp w scores keys
+// w*32 + lane, w*32 + 256 + lane, ... (one key per lane, 16-byte loads), keeps
+// its own online-softmax state, and the 8 partial states are merged in shared
+// memory at the end.
 // ---------------------------------------------------------------------------
 template <class T, int DPL>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     k_naive_attn(const T* __restrict__ qkv, const T* __restrict__ K, const T* __restrict__ V,
                  T* __restrict__ a_out, int B, int H, int j, float sc2) {
-  constexpr int DH = DPL * 32;
-  __shared__ float sq[4][DH];
+  constexpr int DH = DPL * 32, NW = 8;
+  __shared__ float sq[DH];
+  __shared__ float sm[NW], sl[NW], so[NW][DH];
   pdl_launch_dependents();
   pdl_wait();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x * 4 + w;
-  const bool active = pair < B * H;
-  const int b = active ? pair / H : 0, h = active ? pair - (pair / H) * H : 0;
+  const int pair = blockIdx.x;
+  const int b = pair / H, h = pair - b * H;
   const int d = H * DH;
   const size_t row = (size_t)j * B + b;
   const T* qp = qkv + row * (size_t)(3 * d) + h * DH;
-  if (active) {
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) sq[w][lane * DPL + i] = to_f(qp[lane * DPL + i]);
-  }
-  __syncwarp();
-  if (!active) return;
+  if (threadIdx.x < DH) sq[threadIdx.x] = to_f(qp[threadIdx.x]);
+  __syncthreads();
   float mo = -INFINITY, lo = 0.f, oo[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) oo[i] = 0.f;
-  for (int c0 = 0; c0 < j; c0 += 32) {
+  for (int c0 = w * 32; c0 < j; c0 += NW * 32) {
     const int n = min(32, j - c0);
     float s = -INFINITY;
     if (lane < n) {
       const T* kp = K + ((size_t)(c0 + lane) * B + b) * d + h * DH;
       float acc = 0.f;
+      if constexpr (sizeof(T) == 2 && DH % 8 == 0) {
+#pragma unroll
+        for (int e0 = 0; e0 < DH; e0 += 8) {
+          const uint4 wv = *reinterpret_cast<const uint4*>(kp + e0);
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(p2[k]);
+            acc += sq[e0 + 2 * k] * f.x + sq[e0 + 2 * k + 1] * f.y;
+          }
+        }
+      } else {
 #pragma unroll 8
-      for (int e = 0; e < DH; ++e) acc += sq[w][e] * to_f(kp[e]);
+        for (int e = 0; e < DH; ++e) acc += sq[e] * to_f(kp[e]);
+      }
       s = acc * sc2;
     }
     const float mn = fmaxf(mo, warp_max(s));
@@ -119,6 +131,7 @@ __global__ void __launch_bounds__(128)
     lo = lo * al + warp_sum(pl);
 #pragma unroll
     for (int i = 0; i < DPL; ++i) oo[i] *= al;
+#pragma unroll 8
     for (int i = 0; i < n; ++i) {
       const float pi = __shfl_sync(0xffffffffu, pl, i);
       const T* vp = V + ((size_t)(c0 + i) * B + b) * d + h * DH + lane * DPL;
@@ -127,22 +140,36 @@ __global__ void __launch_bounds__(128)
     }
     mo = mn;
   }
-  // the temporary pair
-  float kt[DPL], vt[DPL], q[DPL];
+  if (lane == 0) { sm[w] = mo; sl[w] = lo; }
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) so[w][lane * DPL + i] = oo[i];
+  __syncthreads();
+  if (w != 0) return;
+  // merge the warps' partial states, then the temporary pair
+  float mt = -INFINITY;
+  for (int k = 0; k < NW; ++k) mt = fmaxf(mt, sm[k]);
+  float lt = 0.f, ot[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) ot[i] = 0.f;
+  for (int k = 0; k < NW; ++k) {
+    const float f = rescale(sm[k], mt);
+    lt += sl[k] * f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) ot[i] += so[k][lane * DPL + i] * f;
+  }
+  float kt[DPL], vt[DPL];
   load_lane<T, DPL>(qp + d + lane * DPL, kt);
   load_lane<T, DPL>(qp + 2 * d + lane * DPL, vt);
-#pragma unroll
-  for (int i = 0; i < DPL; ++i) q[i] = sq[w][lane * DPL + i];
   float dot = 0.f;
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) dot += q[i] * kt[i];
+  for (int i = 0; i < DPL; ++i) dot += sq[lane * DPL + i] * kt[i];
   const float s = warp_sum(dot) * sc2;
-  const float mn = fmaxf(mo, s);
-  const float al = rescale(mo, mn), pt = exp2f(s - mn);
-  const float inv = 1.f / (lo * al + pt);
+  const float mn = fmaxf(mt, s);
+  const float al = rescale(mt, mn), pt = exp2f(s - mn);
+  const float inv = 1.f / (lt * al + pt);
   T* ap = a_out + (size_t)b * d + h * DH + lane * DPL;
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) ap[i] = from_f<T>((oo[i] * al + pt * vt[i]) * inv);
+  for (int i = 0; i < DPL; ++i) ap[i] = from_f<T>((ot[i] * al + pt * vt[i]) * inv);
 }
 
 // ---------------------------------------------------------------------------
@@ -224,9 +251,8 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
-// block fold for small blocks (used for up to 8 keys), bf16, d_h = 64: eight
-// lanes per (b, h, query), eight dims (16 bytes of q/k/v, 32 bytes of o) per
-// lane; keys in groups of eight with online rescaling between groups.
+// block fold for small blocks (at most 8 keys), bf16, d_h = 64: eight lanes
+// per (b, h, query), eight dims (16 bytes of q/k/v, 32 bytes of o) per lane.
 // fin = 1: the first query of the block (q0) receives no later fold, so it
 // is finalised here -- its temporary pair is merged and a_{q0} = o / l is
 // written to a_out [B][d]; its (m, l, o) are not stored.
@@ -242,6 +268,19 @@ __device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* src, float (&v)
   }
 }
 
+__device__ __forceinline__ void unpack_bf16x8(const uint4& w, float (&v)[8]) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __bfloat1622float2(p[k]);
+    v[2 * k] = f.x;
+    v[2 * k + 1] = f.y;
+  }
+}
+
+// All global loads of an octet are issued before any arithmetic (one round of
+// memory latency): q, the keys' k and v, the query's (m, l, o) and, for the
+// finalised query, its temporary pair.
 __global__ void __launch_bounds__(256)
     k_fold_small(const __nv_bfloat16* __restrict__ qkv, int q_stride, const __nv_bfloat16* __restrict__ K,
                  const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m, float* __restrict__ l,
@@ -260,8 +299,24 @@ __global__ void __launch_bounds__(256)
   const int b = pair / H, h = pair - b * H;
   const size_t row = (size_t)(q0 + qi) * B + b;
   const __nv_bfloat16* qp = qkv + row * (size_t)q_stride + h * DH + sl * 8;
-  float q[8];
-  load_bf16x8(qp, q);
+  const bool finrow = fin && qi == 0;
+  const int n = min(nk, KMAX);   // callers use this kernel for nk <= 8
+  // ---- loads ----
+  const uint4 qw = *reinterpret_cast<const uint4*>(qp);
+  uint4 kw[KMAX], vw[KMAX];
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    if (i < n) {
+      const size_t kr = ((size_t)(k0 + i) * B + b) * kv_stride + h * DH + sl * 8;
+      kw[i] = *reinterpret_cast<const uint4*>(K + kr);
+      vw[i] = *reinterpret_cast<const uint4*>(V + kr);
+    }
+  }
+  uint4 ktw = make_uint4(0, 0, 0, 0), vtw = make_uint4(0, 0, 0, 0);
+  if (finrow) {
+    ktw = *reinterpret_cast<const uint4*>(qp + d);
+    vtw = *reinterpret_cast<const uint4*>(qp + 2 * d);
+  }
   float mo = -INFINITY, lo = 0.f, oo[8];
   float* op = o + row * (size_t)d + h * DH + sl * 8;
   if (init) {
@@ -274,59 +329,62 @@ __global__ void __launch_bounds__(256)
     oo[0] = a0.x; oo[1] = a0.y; oo[2] = a0.z; oo[3] = a0.w;
     oo[4] = a1.x; oo[5] = a1.y; oo[6] = a1.z; oo[7] = a1.w;
   }
-  float mn = mo;
-  for (int c0 = 0; c0 < nk; c0 += KMAX) {
-    const int n = min(KMAX, nk - c0);
-    float s[KMAX];
-    float mx = -INFINITY;
+  // ---- scores ----
+  float q[8];
+  unpack_bf16x8(qw, q);
+  float s[KMAX];
+  float mx = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < KMAX; ++i) {
-      s[i] = -INFINITY;
-      if (i < n) {
-        float kk[8];
-        load_bf16x8(K + ((size_t)(k0 + c0 + i) * B + b) * kv_stride + h * DH + sl * 8, kk);
-        float dot = 0.f;
+  for (int i = 0; i < KMAX; ++i) {
+    s[i] = -INFINITY;
+    if (i < n) {
+      float kk[8];
+      unpack_bf16x8(kw[i], kk);
+      float dot = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
-        dot += __shfl_xor_sync(omask, dot, 1);
-        dot += __shfl_xor_sync(omask, dot, 2);
-        dot += __shfl_xor_sync(omask, dot, 4);
-        s[i] = dot * sc2;
-        mx = fmaxf(mx, s[i]);
-      }
+      for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
+      dot += __shfl_xor_sync(omask, dot, 1);
+      dot += __shfl_xor_sync(omask, dot, 2);
+      dot += __shfl_xor_sync(omask, dot, 4);
+      s[i] = dot * sc2;
+      mx = fmaxf(mx, s[i]);
     }
-    const float m_new = fmaxf(mn, mx);
-    const float al = rescale(mn, m_new);
-    lo *= al;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) oo[e] *= al;
-#pragma unroll
-    for (int i = 0; i < KMAX; ++i) {
-      if (i < n) {
-        const float p = exp2f(s[i] - m_new);
-        float vv[8];
-        load_bf16x8(V + ((size_t)(k0 + c0 + i) * B + b) * kv_stride + h * DH + sl * 8, vv);
-        lo += p;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
-      }
-    }
-    mn = m_new;
   }
-  if (fin && qi == 0) {
-    float kt[8], vt[8];
-    load_bf16x8(qp + d, kt);
-    load_bf16x8(qp + 2 * d, vt);
+  float st = -INFINITY;
+  if (finrow) {
+    float kt[8];
+    unpack_bf16x8(ktw, kt);
     float dot = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) dot += q[e] * kt[e];
     dot += __shfl_xor_sync(omask, dot, 1);
     dot += __shfl_xor_sync(omask, dot, 2);
     dot += __shfl_xor_sync(omask, dot, 4);
-    const float st = dot * sc2;
+    st = dot * sc2;
+  }
+  // ---- online-softmax merge (block keys, then the temporary pair if finalising) ----
+  const float mn = fmaxf(mo, mx);
+  const float al = rescale(mo, mn);
+  lo *= al;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) oo[e] *= al;
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    if (i < n) {
+      const float p = exp2f(s[i] - mn);
+      float vv[8];
+      unpack_bf16x8(vw[i], vv);
+      lo += p;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
+    }
+  }
+  if (finrow) {
     const float m2 = fmaxf(mn, st);
     const float a2 = rescale(mn, m2), pt = exp2f(st - m2);
     const float inv = 1.f / (lo * a2 + pt);
+    float vt[8];
+    unpack_bf16x8(vtw, vt);
     uint4 w;
     uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll

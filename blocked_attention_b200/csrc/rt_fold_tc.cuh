@@ -380,4 +380,340 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// k_fold_tc2: two softmax warpgroups. Work item = one (b, h) pair and a super
+// tile of 256 queries (tile A = queries 0..127, tile B = 128..255 of it), so
+// every K/V chunk feeds two 128-query tiles. 320 threads:
+//   warp 0 : TMA producer (Q of both tiles double-buffered per item; K/V ring)
+//   warp 1 : MMA issuer, ping-pong order S_A(0) S_B(0) | PV_A(g) S_A(g+1)
+//            PV_B(g) S_B(g+1) | ..., so each tile's softmax overlaps the
+//            other tile's tensor-core work
+//   warps 2..5 (tile A), 6..9 (tile B): softmax, accumulate, merge
+// TMEM: S_A 0..127, S_B 128..255, O_A[2] 256/320, O_B[2] 384/448.
+// ---------------------------------------------------------------------------
+struct FoldTc2Cfg {
+  static constexpr int QT = 128, KC = 128, DH = 64, KVS = 2;
+  static constexpr uint32_t Q_BYTES = QT * DH * 2;    // 16 KB per tile
+  static constexpr uint32_t KV_BYTES = KC * DH * 2;   // 16 KB
+  static constexpr uint32_t P_BYTES = QT * KC * 2;    // 32 KB per tile
+  static constexpr uint32_t OFF_Q = 0;                           // [2 buffers][2 tiles]
+  static constexpr uint32_t OFF_K = OFF_Q + 4 * Q_BYTES;         // [KVS]
+  static constexpr uint32_t OFF_V = OFF_K + KVS * KV_BYTES;      // [KVS]
+  static constexpr uint32_t OFF_P = OFF_V + KVS * KV_BYTES;      // [2 tiles]
+  static constexpr uint32_t OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 512;
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+__global__ void __launch_bounds__(320, 1)
+    k_fold_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __nv_bfloat16* __restrict__ Q, int q_stride,
+               float* __restrict__ m, float* __restrict__ l, float* __restrict__ o,
+               __nv_bfloat16* __restrict__ a_out, int B, int H, int q0, int nq, int k0, int nk, float sc2,
+               int init, int fin, unsigned* err) {
+  using C = FoldTc2Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;      // [2]
+  uint64_t* q_empty = bars + 2;     // [2]
+  uint64_t* kv_full = bars + 4;     // [KVS]
+  uint64_t* kv_empty = bars + 6;    // [KVS]
+  uint64_t* s_full = bars + 8;      // [tile]
+  uint64_t* s_free = bars + 10;     // [tile]
+  uint64_t* p_full = bars + 12;     // [tile]
+  uint64_t* p_free = bars + 14;     // [tile]
+  uint64_t* o_full = bars + 16;     // [tile][2]
+  uint64_t* o_free = bars + 20;     // [tile][2]
+  uint64_t* mma_done = bars + 24;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 25);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = H * C::DH;
+  const int nts = (nq + 2 * C::QT - 1) / (2 * C::QT);   // super tiles per pair
+  const int nitems = B * H * nts;
+  const int nch = nk / C::KC;
+  const int my_items = blockIdx.x < nitems ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int total = my_items * nch;
+  auto item_of = [&](int li, int& b, int& h, int& st0) {
+    const int it = (int)blockIdx.x + li * (int)gridDim.x;
+    const int pair = it / nts, stt = it - pair * nts;
+    b = pair / H;
+    h = pair - b * H;
+    st0 = q0 + stt * 2 * C::QT;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 9);   // MMA commit + 8 softmax warps
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_free[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_free[i], 4);
+    }
+    for (int i = 0; i < C::KVS; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  pdl_launch_dependents();
+  pdl_wait();
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int g = 0, issued_q = 0;
+      bool ok = true;
+      for (int li = 0; li < my_items && ok; ++li) {
+        int b, h, st0;
+        item_of(li, b, h, st0);
+        const int qb = li & 1;
+        if (!mbar_wait(&q_empty[qb], ((li >> 1) & 1u) ^ 1u, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&q_full[qb], 2 * C::Q_BYTES);
+        tma_load_3d(&tmQ, &q_full[qb], smem + C::OFF_Q + (qb * 2 + 0) * C::Q_BYTES, h * C::DH, b, st0);
+        tma_load_3d(&tmQ, &q_full[qb], smem + C::OFF_Q + (qb * 2 + 1) * C::Q_BYTES, h * C::DH, b, st0 + C::QT);
+        ++issued_q;
+        for (int c = 0; c < nch; ++c, ++g) {
+          const int st = g % C::KVS;
+          const uint32_t ph = (g / C::KVS) & 1u;
+          if (!mbar_wait(&kv_empty[st], ph ^ 1u, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&kv_full[st], 2 * C::KV_BYTES);
+          tma_load_3d(&tmK, &kv_full[st], smem + C::OFF_K + st * C::KV_BYTES, h * C::DH, b, k0 + c * C::KC);
+          tma_load_3d(&tmV, &kv_full[st], smem + C::OFF_V + st * C::KV_BYTES, h * C::DH, b, k0 + c * C::KC);
+        }
+      }
+      if (!ok) {
+        for (int i = (issued_q >= 2 ? issued_q - 2 : 0); i < issued_q; ++i) mbar_wait(&q_full[i & 1], (i >> 1) & 1u, err);
+        for (int i = (g >= C::KVS ? g - C::KVS : 0); i < g; ++i) mbar_wait(&kv_full[i % C::KVS], (i / C::KVS) & 1u, err);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128);
+      const uint32_t idesc_o = idesc_bf16_f32(128, 64) | (1u << 16);   // B (= V) MN-major
+      auto issue_s = [&](int g, int t) -> bool {
+        const int li = g / nch, c = g - li * nch;
+        const int qb = li & 1, st = g % C::KVS;
+        if (t == 0 && c == 0 && !mbar_wait(&q_full[qb], (li >> 1) & 1u, err)) return false;
+        if (t == 0 && !mbar_wait(&kv_full[st], (g / C::KVS) & 1u, err)) return false;
+        if (!mbar_wait(&s_free[t], (g & 1u) ^ 1u, err)) return false;
+        tc_fence_after();
+        const uint8_t* qt = smem + C::OFF_Q + (qb * 2 + t) * C::Q_BYTES;
+        const uint8_t* kt = smem + C::OFF_K + st * C::KV_BYTES;
+#pragma unroll
+        for (int k = 0; k < C::DH / 16; ++k)
+          tc_mma_f16(tmem_base + t * 128, smem_desc_sw128(qt + k * 32), smem_desc_sw128(kt + k * 32), idesc_s,
+                     k != 0 ? 1u : 0u);
+        tc_commit(&s_full[t]);
+        return true;
+      };
+      auto issue_pv = [&](int g, int t) -> bool {
+        const int li = g / nch, c = g - li * nch;
+        const int st = g % C::KVS, ob = g & 1;
+        if (!mbar_wait(&p_full[t], g & 1u, err) || !mbar_wait(&o_free[t * 2 + ob], ((g >> 1) & 1u) ^ 1u, err))
+          return false;
+        tc_fence_after();
+        const uint8_t* pt = smem + C::OFF_P + t * C::P_BYTES;
+        const uint8_t* vt = smem + C::OFF_V + st * C::KV_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < C::KC / 16; ++ks)
+          tc_mma_f16(tmem_base + 256 + t * 128 + ob * 64, smem_desc_sw128(pt + (ks >> 2) * 16384 + (ks & 3) * 32),
+                     smem_desc_sw128_mn(vt + ks * 16 * 128), idesc_o, ks != 0 ? 1u : 0u);
+        tc_commit(&o_full[t * 2 + ob]);
+        tc_commit(&p_free[t]);
+        if (t == 1) {
+          tc_commit(&kv_empty[st]);
+          if (c == nch - 1) tc_commit(&q_empty[li & 1]);
+        }
+        return true;
+      };
+      bool ok = true;
+      if (total > 0) ok = issue_s(0, 0) && issue_s(0, 1);
+      for (int g = 0; g < total && ok; ++g) {
+        ok = issue_pv(g, 0);
+        if (ok && g + 1 < total) ok = issue_s(g + 1, 0);
+        if (ok) ok = issue_pv(g, 1);
+        if (ok && g + 1 < total) ok = issue_s(g + 1, 1);
+      }
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, err);
+    }
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    const int t = (warp - 2) >> 2;          // tile of this warpgroup
+    const int qq = warp & 3;                // TMEM lane quarter of this warp
+    const int r = qq * 32 + lane;           // query row within the tile
+    const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
+    uint8_t* sP = smem + C::OFF_P + t * C::P_BYTES;
+    float m_run = -INFINITY, l_run = 0.f, alpha_prev = 0.f;
+    float oacc[64];
+    bool ok = true;
+
+    auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
+      int v = 1;
+      if (lane == 0) v = mbar_wait(bar, parity, err) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, v, 0) != 0;
+    };
+    auto accumulate = [&](int g, float alpha) -> bool {
+      const int ob = g & 1;
+      if (!wait_warp(&o_full[t * 2 + ob], (g >> 1) & 1u)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t rv[32];
+        tmem_ld_32x32b_x32(tmem_base + lane_base + 256 + t * 128 + ob * 64 + half * 32, rv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) oacc[half * 32 + i] = oacc[half * 32 + i] * alpha + __uint_as_float(rv[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[t * 2 + ob]);
+      return true;
+    };
+    auto merge = [&](int li) {
+      int b, h, st0;
+      item_of(li, b, h, st0);
+      const int qt0 = st0 + t * C::QT;
+      const int nrows = min(C::QT, q0 + nq - qt0);   // may be <= 0 for an empty tile B
+      if (r < nrows) {
+        const size_t row = (size_t)(qt0 + r) * B + b;
+        float mg = -INFINITY, lg = 0.f;
+        float* op = o + row * (size_t)d + h * C::DH;
+        if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }
+        const float mn = fmaxf(mg, m_run);
+        const float ag = rescale(mg, mn), ab = rescale(m_run, mn);
+        const float ln = lg * ag + l_run * ab;
+        if (fin && qt0 == q0 && r == 0) {
+          const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * C::DH;
+          const __nv_bfloat16* qrow =
+              reinterpret_cast<const __nv_bfloat16*>(smem + C::OFF_Q + ((li & 1) * 2 + t) * C::Q_BYTES);
+          float dot = 0.f;
+#pragma unroll 8
+          for (int e = 0; e < C::DH; ++e) dot += __bfloat162float(qrow[e]) * __bfloat162float(tp[d + e]);
+          const float s2 = dot * sc2;
+          const float m2 = fmaxf(mn, s2);
+          const float a2 = rescale(mn, m2), pt = exp2f(s2 - m2);
+          const float inv = 1.f / (ln * a2 + pt);
+          __nv_bfloat16* ap = a_out + (size_t)b * d + h * C::DH;
+#pragma unroll
+          for (int e = 0; e < C::DH; e += 2) {
+            float og0 = 0.f, og1 = 0.f;
+            if (!init) { og0 = op[e]; og1 = op[e + 1]; }
+            const float o0 = og0 * ag + oacc[e] * ab, o1 = og1 * ag + oacc[e + 1] * ab;
+            const float2 vt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tp + 2 * d + e));
+            *reinterpret_cast<__nv_bfloat162*>(ap + e) =
+                __floats2bfloat162_rn((o0 * a2 + pt * vt.x) * inv, (o1 * a2 + pt * vt.y) * inv);
+          }
+        } else {
+          m[row * H + h] = mn;
+          l[row * H + h] = ln;
+#pragma unroll
+          for (int e = 0; e < C::DH; e += 4) {
+            float4 og = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!init) og = *reinterpret_cast<const float4*>(op + e);
+            og.x = og.x * ag + oacc[e] * ab;
+            og.y = og.y * ag + oacc[e + 1] * ab;
+            og.z = og.z * ag + oacc[e + 2] * ab;
+            og.w = og.w * ag + oacc[e + 3] * ab;
+            *reinterpret_cast<float4*>(op + e) = og;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[li & 1]);
+    };
+
+    for (int g = 0; g < total && ok; ++g) {
+      const int li = g / nch, c = g - li * nch;
+      if (c == 0) {
+        if (g > 0) {
+          if (!accumulate(g - 1, alpha_prev)) { ok = false; break; }
+          merge(li - 1);
+        }
+        m_run = -INFINITY;
+        l_run = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) oacc[i] = 0.f;
+      }
+      if (!wait_warp(&s_full[t], g & 1u)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sbase = tmem_base + lane_base + t * 128;
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t rv[32];
+        tmem_ld_32x32b_x32(sbase + cc * 32, rv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(rv[i]));
+      }
+      const float m_new = fmaxf(m_run, mx * sc2);
+      const float alpha = rescale(m_run, m_new);
+      // P of the previous chunk must have been consumed by its PV product
+      if (!wait_warp(&p_free[t], (g & 1u) ^ 1u)) { ok = false; break; }
+      float lsum = 0.f;
+      uint8_t* prow = sP + r * 128;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t rv[32];
+        tmem_ld_32x32b_x32(sbase + cc * 32, rv);
+        tmem_ld_wait();
+        uint8_t* atom = prow + (cc >> 1) * 16384;
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            p[e] = exp2f(__uint_as_float(rv[gq * 8 + e]) * sc2 - m_new);
+            lsum += p[e];
+          }
+          uint4 w;
+          w.x = pack_bf16x2(p[0], p[1]);
+          w.y = pack_bf16x2(p[2], p[3]);
+          w.z = pack_bf16x2(p[4], p[5]);
+          w.w = pack_bf16x2(p[6], p[7]);
+          const int chunk = (cc & 1) * 4 + gq;
+          *reinterpret_cast<uint4*>(atom + ((chunk ^ (r & 7)) << 4)) = w;
+        }
+      }
+      l_run = l_run * alpha + lsum;
+      m_run = m_new;
+      tc_fence_before();
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_free[t]);
+        mbar_arrive(&p_full[t]);
+      }
+      if (c > 0 && !accumulate(g - 1, alpha_prev)) { ok = false; break; }
+      alpha_prev = alpha;
+    }
+    if (ok && total > 0 && accumulate(total - 1, alpha_prev)) merge(my_items - 1);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
 }  // namespace rt

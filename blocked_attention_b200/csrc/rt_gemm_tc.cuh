@@ -230,21 +230,39 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  // everything above overlaps the predecessor kernel; its outputs are read below
+  // everything above overlaps the predecessor kernel. The producer also loads
+  // the weight (B) tiles of its first pipeline stages before waiting: weights
+  // are never written by a predecessor. Every thread waits before touching
+  // anything a predecessor writes.
   pdl_launch_dependents();
-  pdl_wait();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
+      // weight tiles of the first tile's first stages (all stages start empty)
+      int pre = 0;
+      if ((int)blockIdx.x < num_tiles) {
+        const int mn = (int)blockIdx.x / splits, ks = (int)blockIdx.x - mn * splits;
+        const int nt = mn - (mn / ntn) * ntn;
+        pre = nk < STAGES ? nk : STAGES;
+        for (int kb = 0; kb < pre; ++kb) {
+          mbar_arrive_expect_tx(&full[kb], C::STAGE_BYTES);
+          tma_load_2d(&tmB, &full[kb], sB + kb * C::B_BYTES, (ks * nk + kb) * C::BK, nt * BN);
+        }
+      }
+      pdl_wait();
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mn = tile / splits, ks = tile - mn * splits;
         const int mt = mn / ntn, nt = mn - mt * ntn;
         const int kb0 = ks * nk;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          if ((int)it < pre) {   // B already in flight; add A
+            tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, (kb0 + kb) * C::BK, mt * C::BM);
+            continue;
+          }
           if (!mbar_wait(&empty[s], ph ^ 1u, err)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
           tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, (kb0 + kb) * C::BK, mt * C::BM);
@@ -259,6 +277,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    pdl_wait();
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(C::BM, BN);
       uint32_t it = 0, local = 0;
@@ -287,6 +306,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ---------------- epilogue warps ----------------
+    pdl_wait();
     const int q = warp & 3;
     uint32_t local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {

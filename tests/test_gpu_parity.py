@@ -74,7 +74,8 @@ def test_batched_projection_matches_oracle(rt, dtype, B, N, d):
     ("bf16", 16, 16, False), ("bf16", 32, 7, False), ("bf16", 64, 64, True),  # mma.sync kernel
     ("bf16", 16, 40, False), ("bf16", 32, 70, True), ("bf16", 96, 65, False),  # (4 / 2 / 1 pairs per CTA)
     ("bf16", 48, 20, False), ("bf16", 12, 3, False), ("bf16", 27, 9, True),    # generic warp kernel (12, 27)
-    ("bf16", 256, 100, False), ("bf16", 1024, 130, False),                     # tcgen05 kernel (nk % 128 == 0)
+    ("bf16", 256, 100, False), ("bf16", 1024, 130, False),                     # tcgen05 kernels (nk % 128 == 0)
+    ("bf16", 256, 256, False), ("bf16", 1024, 700, True), ("bf16", 256, 129, False),
     ("bf16", 128, 77, False), ("bf16", 128, 128, True), ("bf16", 512, 300, True), ("bf16", 384, 1, False),
     ("bf16", 40, 6, False),                                                      # generic warp kernel
     ("f32", 3, 4, False), ("f32", 16, 16, True), ("f32", 64, 33, False)])
