@@ -242,14 +242,21 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0;
       bool ok = true;
       // weight tiles of the first tile's first stages (all stages start empty)
+      // Each tile walks its k-blocks starting at a rotation that depends on its
+      // row and column tile, so that CTAs sharing an operand (same row tile:
+      // same A; same column tile: same B) request different k-blocks at any
+      // moment instead of hammering the same L2 lines together.
+      auto rot_of = [&](int mt, int nt) { return (3 * nt + 5 * mt) % nk; };
       int pre = 0;
       if ((int)blockIdx.x < num_tiles) {
         const int mn = (int)blockIdx.x / splits, ks = (int)blockIdx.x - mn * splits;
-        const int nt = mn - (mn / ntn) * ntn;
+        const int mt = mn / ntn, nt = mn - mt * ntn;
+        const int rot = rot_of(mt, nt);
         pre = nk < STAGES ? nk : STAGES;
         for (int kb = 0; kb < pre; ++kb) {
+          const int kk = ks * nk + (kb + rot) % nk;
           mbar_arrive_expect_tx(&full[kb], C::STAGE_BYTES);
-          tma_load_2d(&tmB, &full[kb], sB + kb * C::B_BYTES, (ks * nk + kb) * C::BK, nt * BN);
+          tma_load_2d(&tmB, &full[kb], sB + kb * C::B_BYTES, kk * C::BK, nt * BN);
         }
       }
       pdl_wait();
@@ -257,16 +264,18 @@ __global__ void __launch_bounds__(192, 1)
         const int mn = tile / splits, ks = tile - mn * splits;
         const int mt = mn / ntn, nt = mn - mt * ntn;
         const int kb0 = ks * nk;
+        const int rot = rot_of(mt, nt);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          const int kk = kb0 + (kb + rot) % nk;
           if ((int)it < pre) {   // B already in flight; add A
-            tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, (kb0 + kb) * C::BK, mt * C::BM);
+            tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, kk * C::BK, mt * C::BM);
             continue;
           }
           if (!mbar_wait(&empty[s], ph ^ 1u, err)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-          tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, (kb0 + kb) * C::BK, mt * C::BM);
-          tma_load_2d(&tmB, &full[s], sB + s * C::B_BYTES, (kb0 + kb) * C::BK, nt * BN);
+          tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, kk * C::BK, mt * C::BM);
+          tma_load_2d(&tmB, &full[s], sB + s * C::B_BYTES, kk * C::BK, nt * BN);
         }
       }
       if (!ok) {
