@@ -84,7 +84,17 @@ struct DevState {
   bool ready = false;
   int sms = 0;
   cudaStream_t capture = nullptr;
+  cudaStream_t h2d = nullptr, d2h = nullptr;   // transfer streams of the host-buffer entry point
+  std::vector<cudaEvent_t> events;             // fork/join events of the host-buffer entry point
 };
+// Overlapped transfers of rt_layer_forward_host: x goes up in kIoXChunks
+// chunks of sequences (each projected as soon as it lands) and z, K, V come
+// down in kIoOutChunks ranges of positions as soon as the step loop has
+// finished them.
+static constexpr int kIoXChunks = 32, kIoOutChunks = 64, kIoEvents = 3 + kIoXChunks + kIoOutChunks;
+static std::mutex g_io_mu;   // the transfer streams and events are per device
+// positions per uploaded chunk of x
+static int io_chunk_len(int N) { return (N + kIoXChunks - 1) / kIoXChunks; }
 static std::mutex g_dev_mu;
 static DevState g_dev[64];
 static PFN_encodeTiled_t g_encode = nullptr;
@@ -134,7 +144,13 @@ static int device_setup(DevState** out) {
         cudaFuncSetAttribute(k_fold_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)FoldTc2Cfg::SMEM_BYTES) != cudaSuccess)
       return RT_ERR_CUDA;
-    if (cudaStreamCreateWithFlags(&ds.capture, cudaStreamNonBlocking) != cudaSuccess) return RT_ERR_CUDA;
+    if (cudaStreamCreateWithFlags(&ds.capture, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&ds.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&ds.d2h, cudaStreamNonBlocking) != cudaSuccess)
+      return RT_ERR_CUDA;
+    ds.events.resize(kIoEvents);
+    for (auto& e : ds.events)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return RT_ERR_CUDA;
     ds.ready = true;
   }
   *out = &ds;
@@ -305,6 +321,14 @@ struct Ptrs {
   void *z, *K, *V, *ws;
 };
 
+// Host buffers of rt_layer_forward_host whose transfers the bf16 forward
+// overlaps with its own work (x up in sequence chunks, outputs down in
+// position ranges). Device-side copies are X.x / X.z / X.K / X.V.
+struct HostIo {
+  const void* x_host;
+  void *z_host, *K_host, *V_host;
+};
+
 // ---------------------------------------------------------------------------
 // per-kernel-class event timing (stream driver only)
 // ---------------------------------------------------------------------------
@@ -427,7 +451,8 @@ static cudaError_t launch_attend(const Plan& P, const T* qkv, const T* K, const 
 // ---------------------------------------------------------------------------
 // bf16 forward
 // ---------------------------------------------------------------------------
-static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st, Timer* T) {
+static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st, Timer* T,
+                        const HostIo* io = nullptr) {
   const Shape& s = P.s;
   char* ws = static_cast<char*>(X.ws);
   unsigned* err = reinterpret_cast<unsigned*>(ws + P.off_err);
@@ -457,23 +482,77 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
   RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + 2 * dd, X.Wv, dd, cudaMemcpyDeviceToDevice, st));
 
   // 1. queries and temporary pairs of all positions
-  {
-    TimedScope ts(T, KC_INV_RMS, st);
-    k_row_inv_rms<bf16><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(x, inv, rows, d, kEps);
-  }
-  RT_CK(cudaGetLastError());
   const int bn_p = choose_bn((int)rows, 3 * d);
-  CUtensorMap tA_x, tB_qkv;
-  if (!make_tmap(&tA_x, x, d, rows, 128) || !make_tmap(&tB_qkv, wqkv, d, 3 * d, bn_p)) return RT_ERR_INVALID_ARG;
+  CUtensorMap tB_qkv;
+  if (!make_tmap(&tB_qkv, wqkv, d, 3 * d, bn_p)) return RT_ERR_INVALID_ARG;
   EpiParams ep;
   std::memset(&ep, 0, sizeof(ep));
   ep.B = B; ep.Nseq = N; ep.d = d; ep.d_ff = dff; ep.eps = kEps;
   ep.inv_rms = inv; ep.qkv = qkv; ep.x = x; ep.u32 = u32; ep.u16 = u16; ep.h16 = h16;
   ep.zout = static_cast<bf16*>(X.z); ep.z16 = z16; ep.Kout = K; ep.Vout = V;
-  {
-    TimedScope ts(T, KC_PROJ, st);
-    RT_CK(launch_tc<EPI_PROJ>(bn_p, tA_x, tB_qkv, (int)rows, 3 * d, d, ep, err, ds.sms, st));
+  // x arrives in chunks of xc positions (the host-buffer path uploads chunk
+  // c while earlier chunks are projected and the step loop runs); chunk c
+  // is projected just before the first step that reads one of its
+  // positions. Device layout of x: [n_chunks][B][xc][d].
+  const int xc = io ? io_chunk_len(N) : N, n_chunks = (N + xc - 1) / xc;
+  ep.xc = xc;
+  int ev = 0;
+  if (io) {   // fork the transfer streams off the main stream; queue every upload
+    RT_CK(cudaEventRecord(ds.events[ev], st));
+    RT_CK(cudaStreamWaitEvent(ds.h2d, ds.events[ev], 0));
+    RT_CK(cudaStreamWaitEvent(ds.d2h, ds.events[ev], 0));
+    ++ev;
+    for (int c = 0; c < n_chunks; ++c) {
+      const int len = std::min(xc, N - c * xc);
+      RT_CK(cudaMemcpy2DAsync(const_cast<bf16*>(x) + (size_t)c * B * xc * d, (size_t)xc * d * 2,
+                              static_cast<const bf16*>(io->x_host) + (size_t)c * xc * d, (size_t)N * d * 2,
+                              (size_t)len * d * 2, B, cudaMemcpyHostToDevice, ds.h2d));
+      RT_CK(cudaEventRecord(ds.events[ev + c], ds.h2d));
+    }
   }
+  const int ev_x = ev;
+  if (io) ev += n_chunks;
+  int projected = 0;   // chunks projected so far
+  // project every chunk up to the one holding position `pos`
+  auto project_through = [&](int pos) -> int {
+    while (projected * xc <= pos) {
+      const int c = projected++;
+      const size_t nr = (size_t)B * xc;   // rows of the chunk, padding included
+      const bf16* xs = x + (size_t)c * B * xc * d;
+      if (io) RT_CK(cudaStreamWaitEvent(st, ds.events[ev_x + c], 0));
+      {
+        TimedScope ts(T, KC_INV_RMS, st);
+        k_row_inv_rms<bf16><<<(unsigned)((nr + 7) / 8), 256, 0, st>>>(xs, inv, nr, d, kEps);
+      }
+      RT_CK(cudaGetLastError());
+      CUtensorMap tA_x;
+      if (!make_tmap(&tA_x, xs, d, nr, 128)) return RT_ERR_INVALID_ARG;
+      EpiParams epp = ep;
+      epp.n0 = c * xc;
+      TimedScope ts(T, KC_PROJ, st);
+      RT_CK(launch_tc<EPI_PROJ>(bn_p, tA_x, tB_qkv, (int)nr, 3 * d, d, epp, err, ds.sms, st));
+    }
+    return RT_OK;
+  };
+  // outputs of positions [p0, p1) are final once step p1 - 1 has run
+  int out_done = 0;
+  auto ship_outputs = [&](int p1) -> int {
+    const int p0 = out_done;
+    if (!io || p1 <= p0) return RT_OK;
+    RT_CK(cudaEventRecord(ds.events[ev], st));
+    RT_CK(cudaStreamWaitEvent(ds.d2h, ds.events[ev], 0));
+    ++ev;
+    const size_t kv0 = (size_t)p0 * B * d, kvn = (size_t)(p1 - p0) * B * d;
+    RT_CK(cudaMemcpyAsync(static_cast<bf16*>(io->K_host) + kv0, K + kv0, kvn * 2, cudaMemcpyDeviceToHost, ds.d2h));
+    RT_CK(cudaMemcpyAsync(static_cast<bf16*>(io->V_host) + kv0, V + kv0, kvn * 2, cudaMemcpyDeviceToHost, ds.d2h));
+    // z[b][p0:p1][:] for every b: B rows of (p1 - p0) * d elements, pitch N * d
+    RT_CK(cudaMemcpy2DAsync(static_cast<bf16*>(io->z_host) + (size_t)p0 * d, (size_t)N * d * 2,
+                            static_cast<const bf16*>(X.z) + (size_t)p0 * d, (size_t)N * d * 2,
+                            (size_t)(p1 - p0) * d * 2, B, cudaMemcpyDeviceToHost, ds.d2h));
+    out_done = p1;
+    return RT_OK;
+  };
+  const int out_every = std::max(1, (N + kIoOutChunks - 1) / kIoOutChunks);
 
   // 2. the N-step loop
   const int bn_o = P.t_wo.bn, bn_1 = P.t_w1.bn, bn_2 = P.t_w2.bn, bn_kv = P.t_wkv.bn;
@@ -485,6 +564,12 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
     return RT_ERR_INVALID_ARG;
   const float sc2 = kLog2e / std::sqrt((float)s.dh());
   const bool blocked = s.schedule == RT_SCHED_BLOCKED;
+  // step j reads queries and temporary pairs of positions up to 2j + 1
+  // (the fold of step j covers queries j + 1 .. 2j + 1, 0-based) and x of j
+  {
+    const int rc = project_through(std::min(N - 1, 1));
+    if (rc != RT_OK) return rc;
+  }
   if (blocked) {
     // position 1: only its temporary pair; every later position is finalised
     // by the last fold into it (the fold of the previous step)
@@ -493,6 +578,10 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
   }
   for (int j = 0; j < N; ++j) {
     ep.j = j;
+    {
+      const int rc = project_through(std::min(N - 1, 2 * j + 1));
+      if (rc != RT_OK) return rc;
+    }
     if (!blocked) {
       TimedScope ts(T, KC_ATTEND, st);
       RT_CK((launch_attend<bf16, 2>(P, qkv, K, V, m, l, o, a16, j, sc2, st)));
@@ -530,6 +619,18 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
                                 t == lb ? 1 : 0, 1, true, st, err, kFoldTcMinBlock, ds.sms));
       }
     }
+    if (io && ((j + 1) % out_every == 0 || j + 1 == N)) {
+      const int rc = ship_outputs(j + 1);
+      if (rc != RT_OK) return rc;
+    }
+  }
+  if (io) {   // join the transfer streams back into the main stream
+    RT_CK(cudaEventRecord(ds.events[ev], ds.h2d));
+    RT_CK(cudaStreamWaitEvent(st, ds.events[ev], 0));
+    ++ev;
+    RT_CK(cudaEventRecord(ds.events[ev], ds.d2h));
+    RT_CK(cudaStreamWaitEvent(st, ds.events[ev], 0));
+    ++ev;
   }
   return RT_OK;
 }
@@ -609,7 +710,12 @@ static int enqueue_f32(const Plan& P, const Ptrs& X, cudaStream_t st, Timer* T) 
 }
 
 static int enqueue_forward(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st,
-                           Timer* T = nullptr) {
+                           Timer* T = nullptr, const HostIo* io = nullptr) {
+  if (io) {
+    if (P.s.dtype != RT_BF16) return RT_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_io_mu);
+    return enqueue_bf16(P, X, ds, st, T, io);
+  }
   return P.s.dtype == RT_BF16 ? enqueue_bf16(P, X, ds, st, T) : enqueue_f32(P, X, st, T);
 }
 
@@ -630,7 +736,7 @@ static long launch_count(const Shape& s) {
 // CUDA-graph driver: the whole forward recorded once per argument set
 // ---------------------------------------------------------------------------
 struct GraphKey {
-  uintptr_t p[11];
+  uintptr_t p[15];
   int v[8];
   bool operator<(const GraphKey& o) const {
     int c = std::memcmp(p, o.p, sizeof(p));
@@ -647,20 +753,23 @@ static std::map<GraphKey, GraphEntry> g_graphs;
 static unsigned long long g_graph_clock = 0;
 static constexpr size_t kMaxGraphs = 8;
 
-static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st) {
+static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st, const HostIo* io = nullptr) {
   DevState* ds = nullptr;
   int rc = device_setup(&ds);
   if (rc != RT_OK) return rc;
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   RT_CK(cudaStreamIsCapturing(st, &cap));
-  if (driver == RT_DRIVER_STREAM || cap != cudaStreamCaptureStatusNone) return enqueue_forward(P, X, *ds, st);
+  if (driver == RT_DRIVER_STREAM || cap != cudaStreamCaptureStatusNone)
+    return enqueue_forward(P, X, *ds, st, nullptr, io);
 
   int dev = 0;
   RT_CK(cudaGetDevice(&dev));
   GraphKey key;
   std::memset(&key, 0, sizeof(key));
-  const void* ptrs[11] = {X.x, X.Wq, X.Wk, X.Wv, X.Wo, X.W1, X.W2, X.z, X.K, X.V, X.ws};
-  for (int i = 0; i < 11; ++i) key.p[i] = reinterpret_cast<uintptr_t>(ptrs[i]);
+  const void* ptrs[15] = {X.x, X.Wq, X.Wk, X.Wv, X.Wo, X.W1, X.W2, X.z, X.K, X.V, X.ws,
+                          io ? io->x_host : nullptr, io ? io->z_host : nullptr,
+                          io ? io->K_host : nullptr, io ? io->V_host : nullptr};
+  for (int i = 0; i < 15; ++i) key.p[i] = reinterpret_cast<uintptr_t>(ptrs[i]);
   const int vals[8] = {P.s.B, P.s.N, P.s.d, P.s.H, P.s.d_ff, P.s.dtype, P.s.schedule, dev};
   std::memcpy(key.v, vals, sizeof(vals));
 
@@ -669,7 +778,7 @@ static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st
   if (it == g_graphs.end()) {
     cudaGraph_t graph = nullptr;
     RT_CK(cudaStreamBeginCapture(ds->capture, cudaStreamCaptureModeThreadLocal));
-    rc = enqueue_forward(P, X, *ds, ds->capture);
+    rc = enqueue_forward(P, X, *ds, ds->capture, nullptr, io);
     cudaError_t ce = cudaStreamEndCapture(ds->capture, &graph);
     if (rc != RT_OK) {
       if (graph) cudaGraphDestroy(graph);
@@ -757,7 +866,9 @@ extern "C" int rt_layer_sync_status(void* workspace, void* stream) {
 static size_t host_io_bytes(const Shape& s, size_t esz) {
   const size_t rows = (size_t)s.B * s.N, d = s.d;
   size_t tot = 0;
-  tot += align_up(rows * d * esz, 256) * 4;                     // x, z, K, V
+  const size_t xc = (size_t)io_chunk_len(s.N), x_rows = (size_t)s.B * xc * ((s.N + xc - 1) / xc);
+  tot += align_up(x_rows * d * esz, 256);                       // x, in chunks of positions
+  tot += align_up(rows * d * esz, 256) * 3;                     // z, K, V
   tot += align_up(d * d * esz, 256) * 4;                        // W_q, W_k, W_v, W_o
   tot += align_up((size_t)s.d_ff * d * esz, 256) * 2;           // W_1, W_2
   return tot;
@@ -768,6 +879,17 @@ extern "C" size_t rt_layer_host_workspace_bytes(int B, int N, int d, int H, int 
   if (validate(s) != RT_OK) return 0;
   const Plan P = make_plan(s);
   return P.total + host_io_bytes(s, P.esz);
+}
+
+// True when `p` is page-locked host memory known to CUDA (cudaHostAlloc /
+// cudaHostRegister); pageable memory cannot be copied asynchronously.
+static bool is_pinned(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
 }
 
 extern "C" int rt_layer_forward_host(const void* x, const void* W_q, const void* W_k, const void* W_v,
@@ -792,9 +914,9 @@ extern "C" int rt_layer_forward_host(const void* x, const void* W_q, const void*
     off += align_up(bytes, 256);
     return p;
   };
-  char *xd = take(act), *zd = take(act), *Kd = take(act), *Vd = take(act);
+  const size_t xc = (size_t)io_chunk_len(N), x_act = (size_t)B * xc * ((N + xc - 1) / xc) * d * P.esz;
+  char *xd = take(x_act), *zd = take(act), *Kd = take(act), *Vd = take(act);
   char *Wqd = take(wdd), *Wkd = take(wdd), *Wvd = take(wdd), *Wod = take(wdd), *W1d = take(wdf), *W2d = take(wdf);
-  RT_CK(cudaMemcpyAsync(xd, x, act, cudaMemcpyHostToDevice, st));
   RT_CK(cudaMemcpyAsync(Wqd, W_q, wdd, cudaMemcpyHostToDevice, st));
   RT_CK(cudaMemcpyAsync(Wkd, W_k, wdd, cudaMemcpyHostToDevice, st));
   RT_CK(cudaMemcpyAsync(Wvd, W_v, wdd, cudaMemcpyHostToDevice, st));
@@ -802,6 +924,13 @@ extern "C" int rt_layer_forward_host(const void* x, const void* W_q, const void*
   RT_CK(cudaMemcpyAsync(W1d, W_1, wdf, cudaMemcpyHostToDevice, st));
   RT_CK(cudaMemcpyAsync(W2d, W_2, wdf, cudaMemcpyHostToDevice, st));
   Ptrs X{xd, Wqd, Wkd, Wvd, Wod, W1d, W2d, zd, Kd, Vd, workspace};
+  // bf16 with page-locked x, z, K, V: the copies of x and of the outputs run
+  // on transfer streams, overlapped with the projection and the step loop
+  if (dtype == RT_BF16 && is_pinned(x) && is_pinned(z) && is_pinned(K) && is_pinned(V)) {
+    HostIo io{x, z, K, V};
+    return run_forward(P, X, driver, st, &io);
+  }
+  RT_CK(cudaMemcpyAsync(xd, x, act, cudaMemcpyHostToDevice, st));
   rc = run_forward(P, X, driver, st);
   if (rc != RT_OK) return rc;
   RT_CK(cudaMemcpyAsync(z, zd, act, cudaMemcpyDeviceToHost, st));
@@ -878,7 +1007,7 @@ extern "C" int rt_project_qkv(const void* x, const void* W_qkv, int B, int N, in
     if (!make_tmap(&ta, x, d, rows, 128) || !make_tmap(&tb, W_qkv, d, 3 * d, bn)) return RT_ERR_INVALID_ARG;
     EpiParams ep;
     std::memset(&ep, 0, sizeof(ep));
-    ep.B = B; ep.Nseq = N; ep.d = d; ep.inv_rms = inv; ep.qkv = static_cast<bf16*>(QKV);
+    ep.B = B; ep.Nseq = N; ep.xc = N; ep.d = d; ep.inv_rms = inv; ep.qkv = static_cast<bf16*>(QKV);
     RT_CK(launch_tc<EPI_PROJ>(bn, ta, tb, (int)rows, 3 * d, d, ep, nullptr, ds->sms, st));
   } else if (dtype == RT_F32) {
     if ((rows + 63) / 64 > 65535) return RT_ERR_UNSUPPORTED;

@@ -33,6 +33,10 @@ enum EpiKind { EPI_PLAIN = 0, EPI_PROJ = 1, EPI_WO = 2, EPI_W1 = 3, EPI_W2 = 4, 
 
 struct EpiParams {
   int B, Nseq, d, d_ff, j;   // batch, sequence length, width, MLP width, position (0-based)
+  // x is stored as [ceil(Nseq / xc)][B][xc][d]: chunks of xc positions, each
+  // chunk sequence-major (xc = Nseq is the plain [B][Nseq][d] layout)
+  int xc;
+  int n0;                    // PROJ: the launch's rows are one chunk, [B][xc], from position n0
   float eps;
   float* c32;                // PLAIN out [M][N]
   const float* inv_rms;      // PROJ: 1/rms per input row [B*N]
@@ -139,14 +143,16 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
         if (col0 + i < N) dst[i] = v[i];
     }
   } else if constexpr (EPI == EPI_PROJ) {
-    const int b = row / p.Nseq, n = row - b * p.Nseq;
+    const int b = row / p.xc, n = p.n0 + (row - b * p.xc);
+    if (n >= p.Nseq) return 0.f;   // padding rows of a last, shorter chunk
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] *= row_scale;
     store_bf16x32(p.qkv + ((size_t)n * p.B + b) * (size_t)(3 * p.d) + col0, v);
   } else if constexpr (EPI == EPI_WO) {
     const int b = row;
     float xv[32];
-    load_bf16x32(p.x + ((size_t)b * p.Nseq + p.j) * p.d + col0, xv);
+    const int c = p.j / p.xc;
+    load_bf16x32(p.x + (((size_t)c * p.B + b) * p.xc + (p.j - c * p.xc)) * p.d + col0, xv);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       v[i] += xv[i];
@@ -242,11 +248,9 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0;
       bool ok = true;
       // weight tiles of the first tile's first stages (all stages start empty)
-      // Each tile walks its k-blocks starting at a rotation that depends on its
-      // row and column tile, so that CTAs sharing an operand (same row tile:
-      // same A; same column tile: same B) request different k-blocks at any
-      // moment instead of hammering the same L2 lines together.
-      auto rot_of = [&](int mt, int nt) { return (3 * nt + 5 * mt) % nk; };
+      // k-blocks are walked in order (a per-tile rotation of the start, to
+      // spread concurrent requests over L2, measured no faster)
+      auto rot_of = [&](int, int) { return 0; };
       int pre = 0;
       if ((int)blockIdx.x < num_tiles) {
         const int mn = (int)blockIdx.x / splits, ks = (int)blockIdx.x - mn * splits;

@@ -145,7 +145,7 @@ extern "C" int rt_project_qkv_noalloc(const void* x, const void* W_qkv, int B, i
   if (!encode(&ta, x, d, rows, 128) || !encode(&tb, W_qkv, d, 3 * (uint64_t)d, bn)) return RT_ERR_INVALID_ARG;
   rt::EpiParams ep;
   memset(&ep, 0, sizeof(ep));
-  ep.B = B; ep.Nseq = N; ep.d = d; ep.inv_rms = s->scratch; ep.qkv = static_cast<__nv_bfloat16*>(QKV);
+  ep.B = B; ep.Nseq = N; ep.xc = N; ep.d = d; ep.inv_rms = s->scratch; ep.qkv = static_cast<__nv_bfloat16*>(QKV);
   cudaError_t e;
   switch (bn) {
     case 256: e = launch_proj<256>(ta, tb, (int)rows, 3 * d, d, ep, s->sms, st); break;

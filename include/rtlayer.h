@@ -115,7 +115,15 @@ size_t rt_layer_host_workspace_bytes(int B, int N, int d, int H, int d_ff,
  * weights host->device, runs the layer, copies z, K, V device->host, all
  * enqueued on `stream` (returns once enqueued; synchronise the stream before
  * reading the outputs). All host pointers must stay valid until then.
- * Layouts as in rt_layer_forward. */
+ * Layouts as in rt_layer_forward; results are bitwise those of
+ * rt_layer_forward.
+ * bf16 with x, z, K and V page-locked (cudaHostAlloc / cudaHostRegister):
+ * the copies overlap the compute -- x goes up in chunks of sequences on a
+ * library-owned transfer stream, each chunk projected as soon as it lands,
+ * and z, K, V come down in ranges of positions as soon as the step loop has
+ * finished them; the transfer streams fork from and join back into `stream`
+ * (and into the cached graph). Otherwise the copies run in sequence with the
+ * compute on `stream`. */
 int rt_layer_forward_host(const void* x_host,
                           const void* W_q_host, const void* W_k_host, const void* W_v_host,
                           const void* W_o_host, const void* W_1_host, const void* W_2_host,

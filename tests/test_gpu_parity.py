@@ -209,6 +209,38 @@ def test_host_buffer_entry_point(rt):
     assert rel_err(to_np(out[1]).transpose(1, 0, 2), Kr) < TOL["bf16"]
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+@pytest.mark.parametrize("driver", ["graph", "stream"])
+def test_host_entry_matches_device_entry(rt, pinned, driver):
+    # B=11 splits unevenly into the sequence chunks of the overlapped upload
+    # and N=37 into its output ranges; pinned buffers take the overlapped
+    # path, pageable ones the sequential one. Both must equal the
+    # device-buffer entry point bit for bit.
+    B, N, d, H, d_ff = 11, 37, 128, 2, 256
+    x, W = problem(B, N, d, H, d_ff, "bf16")
+    xd = to_device(x, "bf16")
+    z0, K0, V0 = rt.layer_forward(xd, _weights_dev(W, "bf16"), H, driver=driver)
+
+    def host(t):
+        return t.pin_memory() if pinned else t
+
+    xh = host(to_device(x, "bf16", device="cpu"))
+    Wh = {k: host(to_device(v, "bf16", device="cpu")) for k, v in W.items()}
+    out = [host(torch.full((B, N, d), 7.0, dtype=torch.bfloat16)),
+           host(torch.full((N, B, d), 7.0, dtype=torch.bfloat16)),
+           host(torch.full((N, B, d), 7.0, dtype=torch.bfloat16))]
+    ws = rt.alloc_workspace(rt.host_workspace_bytes(B, N, d, H, d_ff))
+    for _ in range(2):   # the second call replays the cached graph
+        rt.layer_forward_host(xh, Wh, H, out, ws, driver=driver)
+        torch.cuda.synchronize()
+        assert rt.sync_status(ws) == 0
+        assert torch.equal(out[0], z0.cpu())
+        assert torch.equal(out[1], K0.cpu())
+        assert torch.equal(out[2], V0.cpu())
+        for t in out:
+            t.fill_(7.0)
+
+
 def test_stack_of_layers_with_embedding(rt):
     # reduced stack: vocab 500, d=128 (2 heads of 64), d_ff=256, 3 layers, B=3, N=33
     vocab, d, H, d_ff, B, N, L = 500, 128, 2, 256, 3, 33, 3
