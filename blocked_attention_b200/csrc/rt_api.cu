@@ -101,9 +101,8 @@ static PFN_encodeTiled_t g_encode = nullptr;
 
 template <int BN, int EPI>
 static cudaError_t set_tc_attr() {
-  constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
-  return cudaFuncSetAttribute(k_gemm_tc<BN, STAGES, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)GemmCfg<BN, STAGES>::SMEM_BYTES);
+  return cudaFuncSetAttribute(k_gemm_tc<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)GemmCfg<BN>::SMEM_BYTES);
 }
 template <int EPI>
 static cudaError_t set_tc_attrs_epi() {
@@ -202,7 +201,7 @@ static TileCfg choose_tiles(int M, int N, int K, bool allow_split) {
   // (W_2, K = 4096) 64-wide tiles with a 2-CTA cluster split-K win
   // (15.3 us vs 21.0 us); wider splits cost more in staging than they save.
   const long ntm = (M + 127) / 128;
-  if (allow_split && K / 64 >= 64 && N % 64 == 0) {
+  if (allow_split && K / 64 >= 64 && K % (2 * GemmCfg<64>::KB) == 0 && N % 64 == 0) {
     const long mn = ntm * (N / 64);
     if (mn * 2 <= 160 && mn < 120) return {64, 2};
   }
@@ -217,18 +216,16 @@ static constexpr int kFoldTcMinBlock = 1024;
 template <int BN, int EPI>
 static cudaError_t launch_tc_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
                                 const EpiParams& p, unsigned* err, int sms, cudaStream_t st) {
-  constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
-  using C = GemmCfg<BN, STAGES>;
+  using C = GemmCfg<BN>;
   if (p.splits > 1) {
     // one output tile per cluster of `splits` CTAs, one tile per CTA
     const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN) * p.splits;
-    return launch_pdl_cluster(k_gemm_tc<BN, STAGES, EPI>, dim3((unsigned)tiles), dim3(192), C::SMEM_BYTES, st,
+    return launch_pdl_cluster(k_gemm_tc<BN, EPI>, dim3((unsigned)tiles), dim3(C::THREADS), C::SMEM_BYTES, st,
                               p.splits, ta, tb, M, N, K, p, err);
   }
   const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = (int)std::min<long>(tiles, sms);
-  return launch_pdl(k_gemm_tc<BN, STAGES, EPI>, dim3(grid), dim3(192), C::SMEM_BYTES, st, ta, tb, M, N, K, p,
-                    err);
+  return launch_pdl(k_gemm_tc<BN, EPI>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, ta, tb, M, N, K, p, err);
 }
 
 template <int EPI>
@@ -422,9 +419,14 @@ static cudaError_t launch_fold(const T* Q, int q_stride, const T* K, const T* V,
                         q0, nq, k0, nk, sc2, init, fin);
     }
     if (fast && dh == 64 && nk <= 8 && q_stride % 8 == 0 && kv_stride % 8 == 0) {
-      const long threads = (long)pairs * nq * 8;
-      return launch_pdl(k_fold_small, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st, Q, q_stride, K, V,
-                        kv_stride, m, l, o, a_out, B, H, q0, nq, k0, nk, sc2, init, fin);
+      // grid of k_fold_small: 32 / S pairs per CTA, or ceil(nq / 32) CTAs per pair
+      int S = 1;
+      while (S < nq || S < nk) S <<= 1;
+      S = std::min(S, 32);
+      const long ctas = (long)((pairs + 32 / S - 1) / (32 / S)) * ((nq + S - 1) / S);
+      if (ctas > 0x7fffffffL) return cudaErrorInvalidValue;
+      return launch_pdl(k_fold_small, dim3((unsigned)ctas), dim3(256), 0, st, Q, q_stride, K, V, kv_stride, m, l, o,
+                        a_out, B, H, q0, nq, k0, nk, sc2, init, fin);
     }
   }
   if (fin) return cudaErrorInvalidValue;   // only the bf16 kernels finalise

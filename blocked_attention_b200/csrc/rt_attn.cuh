@@ -278,60 +278,91 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& w, float (&v)[8]) {
   }
 }
 
-// All global loads of an octet are issued before any arithmetic (one round of
-// memory latency): q, the keys' k and v, the query's (m, l, o) and, for the
-// finalised query, its temporary pair.
-__global__ void __launch_bounds__(256)
+// Work split: a CTA holds 32 octets. With S = min(32, the power of two
+// >= max(nq, nk)) query slots per (b, h) pair, a CTA serves 32 / S pairs
+// (S < 32) or 32 queries of one pair (nq > 32, the pair's queries cut into
+// ceil(nq / 32) CTAs). The CTA's keys -- at most 32 (pair, key) rows of k and
+// of v -- are staged once in shared memory by cp.async, so every query of a
+// pair reads them from there; q, (m, l, o) and the temporary pair are loaded
+// per octet before the staging wait, so all global loads of the CTA are in
+// flight together (one round of memory latency).
+__device__ __forceinline__ int fold_small_slots(int nq, int nk) {
+  int s = 1;
+  while (s < nq || s < nk) s <<= 1;
+  return s < 32 ? s : 32;
+}
+
+__global__ void __launch_bounds__(256, 4)
     k_fold_small(const __nv_bfloat16* __restrict__ qkv, int q_stride, const __nv_bfloat16* __restrict__ K,
                  const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m, float* __restrict__ l,
                  float* __restrict__ o, __nv_bfloat16* __restrict__ a_out, int B, int H, int q0, int nq,
                  int k0, int nk, float sc2, int init, int fin) {
   constexpr int DH = 64, KMAX = 8;
+  __shared__ __align__(16) uint4 skv[2][32 * 8];   // [k | v][(pair_local * nk + key) * 8 + 16-byte part]
   pdl_launch_dependents();
   pdl_wait();
-  const long item = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
-  const int sl = threadIdx.x & 7;
-  if (item >= (long)B * H * nq) return;   // whole octets leave together
-  const unsigned omask = 0xFFu << ((threadIdx.x & 31) & 24);
+  const int pairs = B * H;
+  const int S = fold_small_slots(nq, nk);
+  const int chunks = (nq + S - 1) / S;               // > 1 only when S = 32
+  const int P = 32 / S;                              // pairs per CTA (1 when chunks > 1)
+  const int pair0 = (int)(blockIdx.x / chunks) * P;
+  const int qbase = (int)(blockIdx.x % chunks) * S;
+  const int n = min(nk, KMAX);                       // callers use this kernel for nk <= 8
   const int d = H * DH;
-  const int qi = (int)(item % nq);
-  const int pair = (int)(item / nq);
-  const int b = pair / H, h = pair - b * H;
-  const size_t row = (size_t)(q0 + qi) * B + b;
-  const __nv_bfloat16* qp = qkv + row * (size_t)q_stride + h * DH + sl * 8;
-  const bool finrow = fin && qi == 0;
-  const int n = min(nk, KMAX);   // callers use this kernel for nk <= 8
-  // ---- loads ----
-  const uint4 qw = *reinterpret_cast<const uint4*>(qp);
-  uint4 kw[KMAX], vw[KMAX];
-#pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    if (i < n) {
-      const size_t kr = ((size_t)(k0 + i) * B + b) * kv_stride + h * DH + sl * 8;
-      kw[i] = *reinterpret_cast<const uint4*>(K + kr);
-      vw[i] = *reinterpret_cast<const uint4*>(V + kr);
+
+  // ---- stage the keys of the CTA's pairs ----
+  const int E = P * n;                               // (pair, key) rows, <= 32
+  for (int u = threadIdx.x; u < 2 * E * 8; u += blockDim.x) {
+    const int kv = u / (E * 8), r = u - kv * (E * 8);
+    const int e = r >> 3, part = r & 7;
+    const int pl = e / n, i = e - pl * n;
+    const int pair = pair0 + pl;
+    if (pair < pairs) {
+      const int b = pair / H, h = pair - b * H;
+      const __nv_bfloat16* src = (kv ? V : K) + ((size_t)(k0 + i) * B + b) * kv_stride + h * DH + part * 8;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&skv[kv][e * 8 + part])), "l"(src)
+                   : "memory");
     }
   }
-  uint4 ktw = make_uint4(0, 0, 0, 0), vtw = make_uint4(0, 0, 0, 0);
-  if (finrow) {
-    ktw = *reinterpret_cast<const uint4*>(qp + d);
-    vtw = *reinterpret_cast<const uint4*>(qp + 2 * d);
-  }
-  float mo = -INFINITY, lo = 0.f, oo[8];
+  asm volatile("cp.async.commit_group;" ::: "memory");
+
+  // ---- this octet's query ----
+  const int oct = threadIdx.x >> 3, sl = threadIdx.x & 7;
+  const unsigned omask = 0xFFu << ((threadIdx.x & 31) & 24);
+  const int pl = oct / S, qi = qbase + (oct - pl * S);
+  const int pair = pair0 + pl;
+  const bool active = pair < pairs && qi < nq;
+  const int b = active ? pair / H : 0, h = active ? pair - b * H : 0;
+  const size_t row = (size_t)(q0 + (active ? qi : 0)) * B + b;
+  const __nv_bfloat16* qp = qkv + row * (size_t)q_stride + h * DH + sl * 8;
+  const bool finrow = active && fin && qi == 0;
   float* op = o + row * (size_t)d + h * DH + sl * 8;
-  if (init) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) oo[e] = 0.f;
-  } else {
-    mo = m[row * H + h];
-    lo = l[row * H + h];
-    const float4 a0 = reinterpret_cast<const float4*>(op)[0], a1 = reinterpret_cast<const float4*>(op)[1];
-    oo[0] = a0.x; oo[1] = a0.y; oo[2] = a0.z; oo[3] = a0.w;
-    oo[4] = a1.x; oo[5] = a1.y; oo[6] = a1.z; oo[7] = a1.w;
+  uint4 qw = make_uint4(0, 0, 0, 0), ktw = qw, vtw = qw;
+  float mo = -INFINITY, lo = 0.f;
+  float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;
+  if (active) {
+    qw = *reinterpret_cast<const uint4*>(qp);
+    if (finrow) {
+      ktw = *reinterpret_cast<const uint4*>(qp + d);
+      vtw = *reinterpret_cast<const uint4*>(qp + 2 * d);
+    }
+    if (!init) {
+      mo = m[row * H + h];
+      lo = l[row * H + h];
+      o0 = reinterpret_cast<const float4*>(op)[0];
+      o1 = reinterpret_cast<const float4*>(op)[1];
+    }
   }
-  // ---- scores ----
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  if (!active) return;   // whole octets leave together; no barrier follows
+
+  float oo[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
   float q[8];
   unpack_bf16x8(qw, q);
+  const uint4* sk = &skv[0][(pl * n) * 8 + sl];
+  const uint4* sv = &skv[1][(pl * n) * 8 + sl];
+  // ---- scores ----
   float s[KMAX];
   float mx = -INFINITY;
 #pragma unroll
@@ -339,7 +370,7 @@ __global__ void __launch_bounds__(256)
     s[i] = -INFINITY;
     if (i < n) {
       float kk[8];
-      unpack_bf16x8(kw[i], kk);
+      unpack_bf16x8(sk[i * 8], kk);
       float dot = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
@@ -373,7 +404,7 @@ __global__ void __launch_bounds__(256)
     if (i < n) {
       const float p = exp2f(s[i] - mn);
       float vv[8];
-      unpack_bf16x8(vw[i], vv);
+      unpack_bf16x8(sv[i * 8], vv);
       lo += p;
 #pragma unroll
       for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];

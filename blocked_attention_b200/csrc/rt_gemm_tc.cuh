@@ -115,15 +115,28 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v
   }
 }
 
-template <int BN, int STAGES>
+// Tile configuration. A pipeline stage holds KSUB 64-wide K slices of the A
+// tile (128 rows) and of the B tile (BN rows), each slice one 128-byte-swizzle
+// TMA box, so one mbarrier wait gates 4 * KSUB MMAs. For BN <= 128 two
+// MMA-issuing warps take alternate stages into their own TMEM accumulators
+// (summed in the epilogue): an mbarrier wait of the issuing thread costs
+// about as long as four 128 x BN x 16 MMAs at BN <= 128, so with one issuer
+// the tensor pipe drains at every wait; the second issuer's MMAs fill it.
+// BN = 256 MMAs outlast the wait: one issuer, one slice per stage.
+template <int BN>
 struct GemmCfg {
-  static constexpr int BM = 128, BK = 64;
-  static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr int BM = 128, BK = 64, KSUB = BN == 256 ? 1 : 2;
+  static constexpr int KB = BK * KSUB;                       // K per stage
+  static constexpr uint32_t A_SUB = BM * BK * 2, B_SUB = BN * BK * 2;
+  static constexpr uint32_t A_BYTES = A_SUB * KSUB, B_BYTES = B_SUB * KSUB;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;  // 5 / 4 / 3 / 4 for BN 32 / 64 / 128 / 256
+  static constexpr int NACC = BN == 256 ? 1 : 2;             // accumulators (issuing warps) per tile
+  static constexpr uint32_t TMEM_COLS = 2 * NACC * BN;       // two tiles in flight
+  static constexpr int THREADS = 224;                        // producer, 2 issuers, 4 epilogue warps
   static constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256;
   static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
+  static_assert(STAGES >= 2, "stages");
 };
 
 // Row-wise epilogue for one 32-column chunk; returns the chunk's sum of squares
@@ -189,6 +202,25 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
   return ssq;
 }
 
+// 32 columns of a tile's accumulator for this thread's row: the sum of the
+// two issuers' partial accumulators (BN columns apart) when both wrote one.
+template <int NACC, int BN>
+__device__ __forceinline__ void tmem_ld_acc(uint32_t taddr, bool two, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld_32x32b_x32(taddr, r);
+  if (NACC == 2 && two) {
+    uint32_t r2[32];
+    tmem_ld_32x32b_x32(taddr + BN, r2);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
+  } else {
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+
 template <int EPI>
 __device__ __forceinline__ float row_scale_for(const EpiParams& p, int row) {
   if constexpr (EPI == EPI_PROJ) {
@@ -202,11 +234,12 @@ __device__ __forceinline__ float row_scale_for(const EpiParams& p, int row) {
   }
 }
 
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
+template <int BN, int EPI>
+__global__ void __launch_bounds__(224, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               int M, int N, int K, EpiParams p, unsigned* err) {
-  using C = GemmCfg<BN, STAGES>;
+  using C = GemmCfg<BN>;
+  constexpr int STAGES = C::STAGES, NACC = C::NACC, KSUB = C::KSUB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -224,10 +257,15 @@ __global__ void __launch_bounds__(192, 1)
   // splits == 1: persistent loop over output tiles; splits > 1: one tile per
   // CTA, tile = mn * splits + ks, so a cluster of `splits` CTAs holds one mn.
   const int num_tiles = nmn * splits;
-  const int nk = K / C::BK / splits;   // k-blocks per split (the host keeps this exact)
+  // stages per tile (per split). K is a multiple of 64; a last stage with
+  // fewer than KSUB slices loads and multiplies only those. With splits > 1
+  // the host keeps K / splits a multiple of the stage depth.
+  const int nk = splits > 1 ? K / C::KB / splits : (K + C::KB - 1) / C::KB;
+  const int ksl = K / C::BK;   // 64-wide K slices in all
+  auto slices = [&](int kblock) { const int r = ksl - kblock * KSUB; return r < KSUB ? r : KSUB; };
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], NACC); mbar_init(&tempty[a], 4); }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -248,19 +286,16 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0;
       bool ok = true;
       // weight tiles of the first tile's first stages (all stages start empty)
-      // k-blocks are walked in order (a per-tile rotation of the start, to
-      // spread concurrent requests over L2, measured no faster)
-      auto rot_of = [&](int, int) { return 0; };
       int pre = 0;
       if ((int)blockIdx.x < num_tiles) {
         const int mn = (int)blockIdx.x / splits, ks = (int)blockIdx.x - mn * splits;
         const int mt = mn / ntn, nt = mn - mt * ntn;
-        const int rot = rot_of(mt, nt);
         pre = nk < STAGES ? nk : STAGES;
         for (int kb = 0; kb < pre; ++kb) {
-          const int kk = ks * nk + (kb + rot) % nk;
-          mbar_arrive_expect_tx(&full[kb], C::STAGE_BYTES);
-          tma_load_2d(&tmB, &full[kb], sB + kb * C::B_BYTES, kk * C::BK, nt * BN);
+          const int kk = (ks * nk + kb) * KSUB, ns = slices(ks * nk + kb);
+          mbar_arrive_expect_tx(&full[kb], ns * (C::A_SUB + C::B_SUB));
+          for (int j = 0; j < ns; ++j)
+            tma_load_2d(&tmB, &full[kb], sB + kb * C::B_BYTES + j * C::B_SUB, (kk + j) * C::BK, nt * BN);
         }
       }
       pdl_wait();
@@ -268,18 +303,21 @@ __global__ void __launch_bounds__(192, 1)
         const int mn = tile / splits, ks = tile - mn * splits;
         const int mt = mn / ntn, nt = mn - mt * ntn;
         const int kb0 = ks * nk;
-        const int rot = rot_of(mt, nt);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
-          const int kk = kb0 + (kb + rot) % nk;
+          const int kk = (kb0 + kb) * KSUB, ns = slices(kb0 + kb);
+          uint8_t* a_st = sA + s * C::A_BYTES;
           if ((int)it < pre) {   // B already in flight; add A
-            tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, kk * C::BK, mt * C::BM);
+            for (int j = 0; j < ns; ++j)
+              tma_load_2d(&tmA, &full[s], a_st + j * C::A_SUB, (kk + j) * C::BK, mt * C::BM);
             continue;
           }
           if (!mbar_wait(&empty[s], ph ^ 1u, err)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-          tma_load_2d(&tmA, &full[s], sA + s * C::A_BYTES, kk * C::BK, mt * C::BM);
-          tma_load_2d(&tmB, &full[s], sB + s * C::B_BYTES, kk * C::BK, nt * BN);
+          mbar_arrive_expect_tx(&full[s], ns * (C::A_SUB + C::B_SUB));
+          for (int j = 0; j < ns; ++j) {
+            tma_load_2d(&tmA, &full[s], a_st + j * C::A_SUB, (kk + j) * C::BK, mt * C::BM);
+            tma_load_2d(&tmB, &full[s], sB + s * C::B_BYTES + j * C::B_SUB, (kk + j) * C::BK, nt * BN);
+          }
         }
       }
       if (!ok) {
@@ -288,10 +326,11 @@ __global__ void __launch_bounds__(192, 1)
         for (uint32_t i = first; i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1u, err);
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers: stage kb of a tile goes to issuer kb % NACC ----------------
     pdl_wait();
-    if (lane == 0) {
+    const int par = warp - 1;
+    if (lane == 0 && par < NACC) {
       const uint32_t idesc = idesc_bf16_f32(C::BM, BN);
       uint32_t it = 0, local = 0;
       bool ok = true;
@@ -299,22 +338,30 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base + (acc * NACC + par) * BN;
+        uint32_t accumulate = 0;
+        const int kb0 = (tile - (tile / splits) * splits) * nk;
         for (int kb = 0; kb < nk; ++kb, ++it) {
+          if ((kb % NACC) != par) continue;
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
           if (!mbar_wait(&full[s], ph, err)) { ok = false; break; }
           tc_fence_after();
           const uint8_t* a_st = sA + s * C::A_BYTES;
           const uint8_t* b_st = sB + s * C::B_BYTES;
+          const int nmma = slices(kb0 + kb) * (C::BK / 16);
 #pragma unroll
-          for (int k = 0; k < C::BK / 16; ++k) {
-            // advance 16 bf16 (32 bytes) along K inside the 128-byte swizzle atom
-            tc_mma_f16(d_tmem, smem_desc_sw128(a_st + k * 32), smem_desc_sw128(b_st + k * 32), idesc,
-                       (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < KSUB * (C::BK / 16); ++k) {
+            if (k >= nmma) break;
+            // slice k / 4; inside it advance 16 bf16 (32 bytes) along K in the 128-byte swizzle atom
+            const int j = k / (C::BK / 16), kk = k % (C::BK / 16);
+            tc_mma_f16(d_tmem, smem_desc_sw128(a_st + j * C::A_SUB + kk * 32),
+                       smem_desc_sw128(b_st + j * C::B_SUB + kk * 32), idesc, accumulate);
+            accumulate = 1u;
           }
           tc_commit(&empty[s]);
         }
-        tc_commit(&tfull[acc]);
+        if (!ok) break;
+        tc_commit(&tfull[acc]);   // with no stage of its own in this tile it arrives at once
       }
     }
   } else {
@@ -334,22 +381,17 @@ __global__ void __launch_bounds__(192, 1)
       const int lrow = q * 32 + lane;
       const int row = mt * C::BM + lrow;
       const bool row_ok = row < M;
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * NACC * BN;
+      const bool two = NACC == 2 && nk >= 2;   // issuer 1 wrote its accumulator in this tile
       if (splits == 1) {
         const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
         float ssq = 0.f;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + c, r);
-          tmem_ld_wait();
+          float v[32];
+          tmem_ld_acc<NACC, BN>(taddr + c, two, v);
           const int col0 = nt * BN + c;
-          if (row_ok && col0 < N) {
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-            ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
-          }
+          if (row_ok && col0 < N) ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
         }
         if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
           if (row_ok) p.ssq_out[(size_t)nt * p.B + row] = ssq;
@@ -361,14 +403,11 @@ __global__ void __launch_bounds__(192, 1)
         float* stage = reinterpret_cast<float*>(smem) + (size_t)lrow * (BN + 4);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + c, r);
-          tmem_ld_wait();
+          float v[32];
+          tmem_ld_acc<NACC, BN>(taddr + c, two, v);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(stage + c)[i] =
-                make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
-                            __uint_as_float(r[4 * i + 3]));
+            reinterpret_cast<float4*>(stage + c)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
       }
       tc_fence_before();
@@ -379,8 +418,8 @@ __global__ void __launch_bounds__(192, 1)
   if (splits > 1) {
     // one output tile per cluster: reduce the ranks' partials over DSMEM
     cluster_sync();
-    if (warp >= 2) {
-      const int t = threadIdx.x - 64;                  // 0..127
+    if (warp >= 3) {
+      const int t = threadIdx.x - 96;                  // 0..127
       const int rank = blockIdx.x % splits;            // == %cluster_ctarank for a 1-D cluster of `splits`
       const int mn = blockIdx.x / splits;
       const int mt = mn / ntn, nt = mn - mt * ntn;

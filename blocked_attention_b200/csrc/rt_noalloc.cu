@@ -46,9 +46,8 @@ EncodeFn g_encode_fn = nullptr;
 
 template <int BN>
 cudaError_t set_proj_attr() {
-  constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
-  return cudaFuncSetAttribute(rt::k_gemm_tc<BN, STAGES, rt::EPI_PROJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)rt::GemmCfg<BN, STAGES>::SMEM_BYTES);
+  return cudaFuncSetAttribute(rt::k_gemm_tc<BN, rt::EPI_PROJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)rt::GemmCfg<BN>::SMEM_BYTES);
 }
 
 // One-time set-up of the current device: sm_100 check, SM count, tensor-map
@@ -113,11 +112,10 @@ __global__ void __launch_bounds__(256) k_inv_rms_rows(const __nv_bfloat16* __res
 template <int BN>
 cudaError_t launch_proj(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const rt::EpiParams& p,
                         int sms, cudaStream_t st) {
-  constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
-  rt::k_gemm_tc<BN, STAGES, rt::EPI_PROJ>
-      <<<grid, 192, rt::GemmCfg<BN, STAGES>::SMEM_BYTES, st>>>(ta, tb, M, N, K, p, nullptr);
+  rt::k_gemm_tc<BN, rt::EPI_PROJ>
+      <<<grid, rt::GemmCfg<BN>::THREADS, rt::GemmCfg<BN>::SMEM_BYTES, st>>>(ta, tb, M, N, K, p, nullptr);
   return cudaGetLastError();
 }
 

@@ -71,6 +71,8 @@ def test_batched_projection_matches_oracle(rt, dtype, B, N, d):
 
 @pytest.mark.parametrize("dtype,nk,nq,init_empty", [
     ("bf16", 1, 1, False), ("bf16", 2, 2, True), ("bf16", 8, 5, False),      # small-block kernel (nk <= 8)
+    ("bf16", 8, 1, False), ("bf16", 3, 1, True), ("bf16", 5, 12, False),     # (query slots per pair 8 / 4 / 16)
+    ("bf16", 4, 70, False), ("bf16", 8, 33, True),                           # (a pair's queries over 3 / 2 CTAs)
     ("bf16", 16, 16, False), ("bf16", 32, 7, False), ("bf16", 64, 64, True),  # mma.sync kernel
     ("bf16", 16, 40, False), ("bf16", 32, 70, True), ("bf16", 96, 65, False),  # (4 / 2 / 1 pairs per CTA)
     ("bf16", 48, 20, False), ("bf16", 12, 3, False), ("bf16", 27, 9, True),    # generic warp kernel (12, 27)
