@@ -33,10 +33,17 @@ namespace rt {
 static constexpr float kEps = 1e-6f;
 typedef __nv_bfloat16 bf16;
 
+// The CUDA error behind the calling thread's last RT_ERR_CUDA status
+// (rt_last_cuda_error reads it).
+static thread_local int g_last_cuda_error = 0;
+static inline int cuda_failure(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return RT_ERR_CUDA;
+}
 #define RT_CK(call)                                  \
   do {                                               \
     cudaError_t e_ = (call);                         \
-    if (e_ != cudaSuccess) return RT_ERR_CUDA;       \
+    if (e_ != cudaSuccess) return cuda_failure(e_);  \
   } while (0)
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -134,22 +141,20 @@ static int device_setup(DevState** out) {
         return RT_ERR_CUDA;
       g_encode = reinterpret_cast<PFN_encodeTiled_t>(fn);
     }
-    if (set_tc_attrs_epi<EPI_PLAIN>() != cudaSuccess || set_tc_attrs_epi<EPI_PROJ>() != cudaSuccess ||
-        set_tc_attrs_epi<EPI_WO>() != cudaSuccess || set_tc_attrs_epi<EPI_W1>() != cudaSuccess ||
-        set_tc_attrs_epi<EPI_W2>() != cudaSuccess || set_tc_attrs_epi<EPI_WKV>() != cudaSuccess)
-      return RT_ERR_CUDA;
-    if (cudaFuncSetAttribute(k_fold_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)FoldTcCfg::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(k_fold_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)FoldTc2Cfg::SMEM_BYTES) != cudaSuccess)
-      return RT_ERR_CUDA;
-    if (cudaStreamCreateWithFlags(&ds.capture, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaStreamCreateWithFlags(&ds.h2d, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaStreamCreateWithFlags(&ds.d2h, cudaStreamNonBlocking) != cudaSuccess)
-      return RT_ERR_CUDA;
+    RT_CK(set_tc_attrs_epi<EPI_PLAIN>());
+    RT_CK(set_tc_attrs_epi<EPI_PROJ>());
+    RT_CK(set_tc_attrs_epi<EPI_WO>());
+    RT_CK(set_tc_attrs_epi<EPI_W1>());
+    RT_CK(set_tc_attrs_epi<EPI_W2>());
+    RT_CK(set_tc_attrs_epi<EPI_WKV>());
+    RT_CK(cudaFuncSetAttribute(k_fold_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FoldTcCfg::SMEM_BYTES));
+    RT_CK(cudaFuncSetAttribute(k_fold_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)FoldTc2Cfg::SMEM_BYTES));
+    RT_CK(cudaStreamCreateWithFlags(&ds.capture, cudaStreamNonBlocking));
+    RT_CK(cudaStreamCreateWithFlags(&ds.h2d, cudaStreamNonBlocking));
+    RT_CK(cudaStreamCreateWithFlags(&ds.d2h, cudaStreamNonBlocking));
     ds.events.resize(kIoEvents);
-    for (auto& e : ds.events)
-      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return RT_ERR_CUDA;
+    for (auto& e : ds.events) RT_CK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
     ds.ready = true;
   }
   *out = &ds;
@@ -197,15 +202,20 @@ struct TileCfg {
 };
 static TileCfg choose_tiles(int M, int N, int K, bool allow_split) {
   // Measured at M = 512 (per-step GEMM latency, graph of back-to-back
-  // launches): plain tiles with >= 120 CTAs win for K = 1024; for long K
-  // (W_2, K = 4096) 64-wide tiles with a 2-CTA cluster split-K win
-  // (15.3 us vs 21.0 us); wider splits cost more in staging than they save.
+  // launches): for long K (W_2, K = 4096) 64-wide tiles with a 2-CTA cluster
+  // split-K win (11.6 us vs 13.3 us unsplit); wider splits cost more in
+  // staging than they save. For K = 1024: the widest tiles that still give
+  // >= 120 CTAs (W_1: 128, 8.1 us vs 9.8 us at 64; W_kv: 64, 6.2 us vs 7.5
+  // us at 128; W_o: 32 -- 64-wide tiles on 64 CTAs time alike in isolation
+  // but 1.5 us slower inside the layer's step).
   const long ntm = (M + 127) / 128;
   if (allow_split && K / 64 >= 64 && K % (2 * GemmCfg<64>::KB) == 0 && N % 64 == 0) {
     const long mn = ntm * (N / 64);
     if (mn * 2 <= 160 && mn < 120) return {64, 2};
   }
-  return {choose_bn(M, N), 1};
+  if (ntm * ((N + 127) / 128) >= 120) return {128, 1};
+  if (ntm * ((N + 63) / 64) >= 120) return {64, 1};
+  return {32, 1};
 }
 // Per-step GEMMs may use cluster split-K (see choose_tiles).
 static constexpr bool kLayerSplitK = true;
@@ -786,11 +796,11 @@ static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st
       if (graph) cudaGraphDestroy(graph);
       return rc;
     }
-    if (ce != cudaSuccess) return RT_ERR_CUDA;
+    if (ce != cudaSuccess) return cuda_failure(ce);
     cudaGraphExec_t exec = nullptr;
     ce = cudaGraphInstantiate(&exec, graph, 0);
     cudaGraphDestroy(graph);
-    if (ce != cudaSuccess) return RT_ERR_CUDA;
+    if (ce != cudaSuccess) return cuda_failure(ce);
     if (g_graphs.size() >= kMaxGraphs) {
       auto victim = g_graphs.begin();
       for (auto i2 = g_graphs.begin(); i2 != g_graphs.end(); ++i2)
@@ -813,6 +823,10 @@ static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st
 using namespace rt;
 
 extern "C" int rt_version(void) { return 100; }
+
+extern "C" int rt_last_cuda_error(void) { return g_last_cuda_error; }
+
+extern "C" const char* rt_cuda_error_string(int code) { return cudaGetErrorString((cudaError_t)code); }
 
 extern "C" const char* rt_status_string(int status) {
   switch (status) {
@@ -856,10 +870,10 @@ extern "C" int rt_layer_sync_status(void* workspace, void* stream) {
   if (!workspace) return RT_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned h = 0;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return RT_ERR_CUDA;
-  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return RT_ERR_CUDA;
-  if (cudaMemsetAsync(workspace, 0, sizeof(h), st) != cudaSuccess) return RT_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return RT_ERR_CUDA;
+  RT_CK(cudaStreamSynchronize(st));
+  RT_CK(cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st));
+  RT_CK(cudaMemsetAsync(workspace, 0, sizeof(h), st));
+  RT_CK(cudaStreamSynchronize(st));
   if (h & RT_DEVERR_TIMEOUT) return RT_ERR_TIMEOUT;
   if (h & RT_DEVERR_INDEX) return RT_ERR_INVALID_ARG;
   return RT_OK;
@@ -987,7 +1001,7 @@ extern "C" int rt_block_fold(const void* Q, int q_stride, const void* K, const v
                            0, false, st);
   else
     return RT_ERR_INVALID_ARG;
-  return e == cudaSuccess ? RT_OK : RT_ERR_CUDA;
+  return e == cudaSuccess ? RT_OK : cuda_failure(e);
 }
 
 extern "C" int rt_project_qkv(const void* x, const void* W_qkv, int B, int N, int d, int dtype, void* QKV,
@@ -1077,7 +1091,7 @@ extern "C" int rt_layer_forward_timed(const void* x, const void* W_q, const void
   Ptrs X{x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V, workspace};
   rc = enqueue_forward(P, X, *ds, st, &timer);
   if (rc != RT_OK) return rc;
-  if (timer.err != cudaSuccess) return RT_ERR_CUDA;
+  if (timer.err != cudaSuccess) return cuda_failure(timer.err);
   RT_CK(cudaStreamSynchronize(st));
   for (int c = 0; c < n_classes; ++c) { class_ms[c] = 0.f; class_launches[c] = 0; }
   for (size_t i = 0; i < timer.cls.size(); ++i) {

@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!ok) {
         // aborted: wait (bounded) for the copies this thread issued
-        for (int i = (issued_q >= 2 ? issued_q - 2 : 0); i < issued_q; ++i) mbar_wait(&q_full[i & 1], (i >> 1) & 1u, err);
+        if (issued_q > 0) mbar_wait(&q_full[0], (issued_q - 1) & 1u, err);
         for (int i = (g >= C::KVS ? g - C::KVS : 0); i < g; ++i) mbar_wait(&kv_full[i % C::KVS], (i / C::KVS) & 1u, err);
       }
     }
@@ -302,8 +302,6 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       // this item's Q buffer may be refilled (the MMA thread also arrives)
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&q_empty[li & 1]);
     };
 
     for (int g = 0; g < total && ok; ++g) {
@@ -384,25 +382,41 @@ __global__ void __launch_bounds__(192, 1)
 // k_fold_tc2: two softmax warpgroups. Work item = one (b, h) pair and a super
 // tile of 256 queries (tile A = queries 0..127, tile B = 128..255 of it), so
 // every K/V chunk feeds two 128-query tiles. 320 threads:
-//   warp 0 : TMA producer (Q of both tiles double-buffered per item; K/V ring)
+//   warp 0 : TMA producer (Q of both tiles per item; K/V ring)
 //   warp 1 : MMA issuer, ping-pong order S_A(0) S_B(0) | PV_A(g) S_A(g+1)
 //            PV_B(g) S_B(g+1) | ..., so each tile's softmax overlaps the
 //            other tile's tensor-core work
 //   warps 2..5 (tile A), 6..9 (tile B): softmax, accumulate, merge
+// P is double-buffered per tile, so the softmax of chunk g + 1 runs while
+// the PV product of chunk g still reads P(g). Q is single-buffered: the
+// producer reloads it once the item's last S products have completed.
 // TMEM: S_A 0..127, S_B 128..255, O_A[2] 256/320, O_B[2] 384/448.
 // ---------------------------------------------------------------------------
+// q . k over d_h = 64 bf16 elements (one thread; kept out of line so that the
+// finalising row's dot product adds no registers to the softmax loop)
+__device__ __noinline__ float dot64_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k) {
+  float dot = 0.f;
+  for (int e = 0; e < 64; e += 2) {
+    const float2 qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + e));
+    const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + e));
+    dot += qv.x * kv.x + qv.y * kv.y;
+  }
+  return dot;
+}
+
 struct FoldTc2Cfg {
   static constexpr int QT = 128, KC = 128, DH = 64, KVS = 2;
   static constexpr uint32_t Q_BYTES = QT * DH * 2;    // 16 KB per tile
   static constexpr uint32_t KV_BYTES = KC * DH * 2;   // 16 KB
-  static constexpr uint32_t P_BYTES = QT * KC * 2;    // 32 KB per tile
-  static constexpr uint32_t OFF_Q = 0;                           // [2 buffers][2 tiles]
-  static constexpr uint32_t OFF_K = OFF_Q + 4 * Q_BYTES;         // [KVS]
+  static constexpr uint32_t P_BYTES = QT * KC * 2;    // 32 KB per tile and buffer
+  static constexpr uint32_t OFF_Q = 0;                           // [2 tiles]
+  static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;         // [KVS]
   static constexpr uint32_t OFF_V = OFF_K + KVS * KV_BYTES;      // [KVS]
-  static constexpr uint32_t OFF_P = OFF_V + KVS * KV_BYTES;      // [2 tiles]
-  static constexpr uint32_t OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr uint32_t OFF_P = OFF_V + KVS * KV_BYTES;      // [2 tiles][2 buffers]
+  static constexpr uint32_t OFF_BAR = OFF_P + 4 * P_BYTES;
   static constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 512;
   static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 };
 
 __global__ void __launch_bounds__(320, 1)
@@ -415,18 +429,18 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* q_full = bars + 0;      // [2]
-  uint64_t* q_empty = bars + 2;     // [2]
+  uint64_t* q_full = bars + 0;      // [1]
+  uint64_t* q_empty = bars + 2;     // [1]
   uint64_t* kv_full = bars + 4;     // [KVS]
   uint64_t* kv_empty = bars + 6;    // [KVS]
   uint64_t* s_full = bars + 8;      // [tile]
   uint64_t* s_free = bars + 10;     // [tile]
-  uint64_t* p_full = bars + 12;     // [tile]
-  uint64_t* p_free = bars + 14;     // [tile]
-  uint64_t* o_full = bars + 16;     // [tile][2]
-  uint64_t* o_free = bars + 20;     // [tile][2]
-  uint64_t* mma_done = bars + 24;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 25);
+  uint64_t* p_full = bars + 12;     // [tile][2]
+  uint64_t* p_free = bars + 16;     // [tile][2]
+  uint64_t* o_full = bars + 20;     // [tile][2]
+  uint64_t* o_free = bars + 24;     // [tile][2]
+  uint64_t* mma_done = bars + 28;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 29);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = H * C::DH;
@@ -444,15 +458,15 @@ __global__ void __launch_bounds__(320, 1)
   };
 
   if (threadIdx.x == 0) {
+    mbar_init(&q_full[0], 1);
+    mbar_init(&q_empty[0], 1);   // MMA commit after the item's last S products
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 9);   // MMA commit + 8 softmax warps
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&p_free[i], 1);
     }
     for (int i = 0; i < 4; ++i) {
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_free[i], 1);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_free[i], 4);
     }
@@ -484,11 +498,10 @@ __global__ void __launch_bounds__(320, 1)
       for (int li = 0; li < my_items && ok; ++li) {
         int b, h, st0;
         item_of(li, b, h, st0);
-        const int qb = li & 1;
-        if (!mbar_wait(&q_empty[qb], ((li >> 1) & 1u) ^ 1u, err)) { ok = false; break; }
-        mbar_arrive_expect_tx(&q_full[qb], 2 * C::Q_BYTES);
-        tma_load_3d(&tmQ, &q_full[qb], smem + C::OFF_Q + (qb * 2 + 0) * C::Q_BYTES, h * C::DH, b, st0);
-        tma_load_3d(&tmQ, &q_full[qb], smem + C::OFF_Q + (qb * 2 + 1) * C::Q_BYTES, h * C::DH, b, st0 + C::QT);
+        if (!mbar_wait(&q_empty[0], (li & 1u) ^ 1u, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&q_full[0], 2 * C::Q_BYTES);
+        tma_load_3d(&tmQ, &q_full[0], smem + C::OFF_Q, h * C::DH, b, st0);
+        tma_load_3d(&tmQ, &q_full[0], smem + C::OFF_Q + C::Q_BYTES, h * C::DH, b, st0 + C::QT);
         ++issued_q;
         for (int c = 0; c < nch; ++c, ++g) {
           const int st = g % C::KVS;
@@ -500,7 +513,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (!ok) {
-        for (int i = (issued_q >= 2 ? issued_q - 2 : 0); i < issued_q; ++i) mbar_wait(&q_full[i & 1], (i >> 1) & 1u, err);
+        if (issued_q > 0) mbar_wait(&q_full[0], (issued_q - 1) & 1u, err);
         for (int i = (g >= C::KVS ? g - C::KVS : 0); i < g; ++i) mbar_wait(&kv_full[i % C::KVS], (i / C::KVS) & 1u, err);
       }
     }
@@ -511,38 +524,40 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t idesc_o = idesc_bf16_f32(128, 64) | (1u << 16);   // B (= V) MN-major
       auto issue_s = [&](int g, int t) -> bool {
         const int li = g / nch, c = g - li * nch;
-        const int qb = li & 1, st = g % C::KVS;
-        if (t == 0 && c == 0 && !mbar_wait(&q_full[qb], (li >> 1) & 1u, err)) return false;
+        const int st = g % C::KVS;
+        if (t == 0 && c == 0 && !mbar_wait(&q_full[0], li & 1u, err)) return false;
         if (t == 0 && !mbar_wait(&kv_full[st], (g / C::KVS) & 1u, err)) return false;
         if (!mbar_wait(&s_free[t], (g & 1u) ^ 1u, err)) return false;
         tc_fence_after();
-        const uint8_t* qt = smem + C::OFF_Q + (qb * 2 + t) * C::Q_BYTES;
+        const uint8_t* qt = smem + C::OFF_Q + t * C::Q_BYTES;
         const uint8_t* kt = smem + C::OFF_K + st * C::KV_BYTES;
 #pragma unroll
         for (int k = 0; k < C::DH / 16; ++k)
           tc_mma_f16(tmem_base + t * 128, smem_desc_sw128(qt + k * 32), smem_desc_sw128(kt + k * 32), idesc_s,
                      k != 0 ? 1u : 0u);
         tc_commit(&s_full[t]);
+        // the item's last S products release Q to the producer
+        if (t == 1 && c == nch - 1) tc_commit(&q_empty[0]);
         return true;
       };
       auto issue_pv = [&](int g, int t) -> bool {
         const int li = g / nch, c = g - li * nch;
         const int st = g % C::KVS, ob = g & 1;
-        if (!mbar_wait(&p_full[t], g & 1u, err) || !mbar_wait(&o_free[t * 2 + ob], ((g >> 1) & 1u) ^ 1u, err))
+        if (!mbar_wait(&p_full[t * 2 + ob], (g >> 1) & 1u, err) ||
+            !mbar_wait(&o_free[t * 2 + ob], ((g >> 1) & 1u) ^ 1u, err))
           return false;
         tc_fence_after();
-        const uint8_t* pt = smem + C::OFF_P + t * C::P_BYTES;
+        const uint8_t* pt = smem + C::OFF_P + (t * 2 + ob) * C::P_BYTES;
         const uint8_t* vt = smem + C::OFF_V + st * C::KV_BYTES;
 #pragma unroll
         for (int ks = 0; ks < C::KC / 16; ++ks)
           tc_mma_f16(tmem_base + 256 + t * 128 + ob * 64, smem_desc_sw128(pt + (ks >> 2) * 16384 + (ks & 3) * 32),
                      smem_desc_sw128_mn(vt + ks * 16 * 128), idesc_o, ks != 0 ? 1u : 0u);
         tc_commit(&o_full[t * 2 + ob]);
-        tc_commit(&p_free[t]);
-        if (t == 1) {
-          tc_commit(&kv_empty[st]);
-          if (c == nch - 1) tc_commit(&q_empty[li & 1]);
-        }
+        tc_commit(&p_free[t * 2 + ob]);
+        if (t == 1) tc_commit(&kv_empty[st]);
+        (void)li;
+        (void)c;
         return true;
       };
       bool ok = true;
@@ -562,7 +577,9 @@ __global__ void __launch_bounds__(320, 1)
     const int qq = warp & 3;                // TMEM lane quarter of this warp
     const int r = qq * 32 + lane;           // query row within the tile
     const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
-    uint8_t* sP = smem + C::OFF_P + t * C::P_BYTES;
+    uint8_t* const sP = smem + C::OFF_P + t * 2 * C::P_BYTES + r * 128;   // this row in P buffer 0
+    uint64_t* const pfull = p_full + t * 2;
+    uint64_t* const pfree = p_free + t * 2;
     float m_run = -INFINITY, l_run = 0.f, alpha_prev = 0.f;
     float oacc[64];
     bool ok = true;
@@ -603,12 +620,8 @@ __global__ void __launch_bounds__(320, 1)
         const float ag = rescale(mg, mn), ab = rescale(m_run, mn);
         const float ln = lg * ag + l_run * ab;
         if (fin && qt0 == q0 && r == 0) {
-          const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * C::DH;
-          const __nv_bfloat16* qrow =
-              reinterpret_cast<const __nv_bfloat16*>(smem + C::OFF_Q + ((li & 1) * 2 + t) * C::Q_BYTES);
-          float dot = 0.f;
-#pragma unroll 8
-          for (int e = 0; e < C::DH; ++e) dot += __bfloat162float(qrow[e]) * __bfloat162float(tp[d + e]);
+          const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * C::DH;   // q, then k_tmp at +d, v_tmp at +2d
+          const float dot = dot64_bf16(tp, tp + d);
           const float s2 = dot * sc2;
           const float m2 = fmaxf(mn, s2);
           const float a2 = rescale(mn, m2), pt = exp2f(s2 - m2);
@@ -638,8 +651,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&q_empty[li & 1]);
+      __syncwarp();   // reconverge the warp after the row-dependent branch
     };
 
     for (int g = 0; g < total && ok; ++g) {
@@ -668,10 +680,11 @@ __global__ void __launch_bounds__(320, 1)
       }
       const float m_new = fmaxf(m_run, mx * sc2);
       const float alpha = rescale(m_run, m_new);
-      // P of the previous chunk must have been consumed by its PV product
-      if (!wait_warp(&p_free[t], (g & 1u) ^ 1u)) { ok = false; break; }
+      // P buffer g % 2 must have been consumed by the PV product of chunk g - 2
+      const int pb = g & 1;
+      if (!wait_warp(pfree + pb, ((g >> 1) & 1u) ^ 1u)) { ok = false; break; }
       float lsum = 0.f;
-      uint8_t* prow = sP + r * 128;
+      uint8_t* prow = sP + (pb ? C::P_BYTES : 0u);
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t rv[32];
@@ -702,7 +715,7 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&s_free[t]);
-        mbar_arrive(&p_full[t]);
+        mbar_arrive(pfull + pb);
       }
       if (c > 0 && !accumulate(g - 1, alpha_prev)) { ok = false; break; }
       alpha_prev = alpha;

@@ -24,7 +24,8 @@ SCHEDULES = {"blocked": RT_SCHED_BLOCKED, "naive": RT_SCHED_NAIVE}
 DRIVERS = {"graph": RT_DRIVER_GRAPH, "stream": RT_DRIVER_STREAM}
 WEIGHT_NAMES = ("W_q", "W_k", "W_v", "W_o", "W_1", "W_2")
 
-EXPORTS = ("rt_version", "rt_status_string", "rt_layer_workspace_bytes", "rt_layer_forward",
+EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_error_string",
+           "rt_layer_workspace_bytes", "rt_layer_forward",
            "rt_layer_sync_status", "rt_layer_host_workspace_bytes", "rt_layer_forward_host",
            "rt_embed_forward", "rt_block_fold", "rt_project_qkv", "rt_gemm_bf16",
            "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc",
@@ -40,7 +41,12 @@ _lib = None
 
 class RTError(RuntimeError):
     def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        msg = f"{fn} failed: {status} ({status_string(status)})"
+        self.cuda_error = 0
+        if status == RT_ERR_CUDA:
+            self.cuda_error = int(lib().rt_last_cuda_error())
+            msg += f": CUDA error {self.cuda_error} ({lib().rt_cuda_error_string(self.cuda_error).decode()})"
+        super().__init__(msg)
         self.status = status
 
 
@@ -58,6 +64,10 @@ def lib() -> ctypes.CDLL:
     L.rt_version.restype = i
     L.rt_status_string.restype = ctypes.c_char_p
     L.rt_status_string.argtypes = [i]
+    L.rt_last_cuda_error.restype = i
+    L.rt_last_cuda_error.argtypes = []
+    L.rt_cuda_error_string.restype = ctypes.c_char_p
+    L.rt_cuda_error_string.argtypes = [i]
     L.rt_layer_workspace_bytes.restype = sz
     L.rt_layer_workspace_bytes.argtypes = [i] * 7
     L.rt_layer_host_workspace_bytes.restype = sz

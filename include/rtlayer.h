@@ -84,6 +84,13 @@ int rt_version(void);
 /* Text for a status code. Never NULL. */
 const char* rt_status_string(int status);
 
+/* The CUDA runtime error (a cudaError_t value) behind the calling thread's
+ * most recent RT_ERR_CUDA status; 0 if there was none. */
+int rt_last_cuda_error(void);
+
+/* CUDA's text for a cudaError_t value. Never NULL. */
+const char* rt_cuda_error_string(int code);
+
 /* Bytes of device workspace rt_layer_forward needs for this shape.
  * Returns 0 for invalid or unsupported arguments. */
 size_t rt_layer_workspace_bytes(int B, int N, int d, int H, int d_ff, int dtype,
