@@ -228,6 +228,7 @@ static cudaError_t launch_tc_bn(const CUtensorMap& ta, const CUtensorMap& tb, in
                                 const EpiParams& p, unsigned* err, int sms, cudaStream_t st) {
   using C = GemmCfg<BN>;
   if (p.splits > 1) {
+    if (!C::split_fits(p.splits) || p.splits > 8 || K % (C::KB * p.splits) != 0) return cudaErrorInvalidValue;
     // one output tile per cluster of `splits` CTAs, one tile per CTA
     const long tiles = (long)((M + 127) / 128) * ((N + BN - 1) / BN) * p.splits;
     return launch_pdl_cluster(k_gemm_tc<BN, EPI>, dim3((unsigned)tiles), dim3(C::THREADS), C::SMEM_BYTES, st,

@@ -66,13 +66,17 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t smem_addr, uint32_t rank)
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float4 dsmem_ld_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
+// bulk copy of `bytes` (multiple of 16, 16-byte aligned) from this CTA's shared
+// memory into the shared memory of a CTA of the cluster, completing on that
+// CTA's mbarrier (both addresses already mapped with mapa)
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
                : "memory");
-  return v;
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -134,6 +138,12 @@ struct GemmCfg {
   static constexpr int NACC = BN == 256 ? 1 : 2;             // accumulators (issuing warps) per tile
   static constexpr uint32_t TMEM_COLS = 2 * NACC * BN;       // two tiles in flight
   static constexpr int THREADS = 224;                        // producer, 2 issuers, 4 epilogue warps
+  // split-K staging in the ring: the CTA's partial tile plus splits - 1
+  // receive slots of one row block each (fp32 rows padded to BN + 4)
+  static constexpr bool split_fits(int splits) {
+    return splits >= 1 && (BN / splits) % 32 == 0 &&
+           (size_t)(BM + (splits - 1) * (BM / splits)) * (BN + 4) * 4 <= (size_t)STAGES * STAGE_BYTES;
+  }
   static constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256;
   static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
   static_assert(STAGES >= 2, "stages");
@@ -248,7 +258,8 @@ __global__ void __launch_bounds__(224, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;   // [2]
   uint64_t* tempty = tfull + 2;       // [2]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* rbar = tempty + 2;        // split-K: the other ranks' row blocks have landed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rbar + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntn = (N + BN - 1) / BN, ntm = (M + C::BM - 1) / C::BM;
@@ -266,6 +277,7 @@ __global__ void __launch_bounds__(224, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], NACC); mbar_init(&tempty[a], 4); }
+    mbar_init(rbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -416,20 +428,42 @@ __global__ void __launch_bounds__(224, 1)
     }
   }
   if (splits > 1) {
-    // one output tile per cluster: reduce the ranks' partials over DSMEM
-    cluster_sync();
+    // One output tile per cluster, reduce-scattered over distributed shared
+    // memory: rank r owns rows [r * rows_per, (r + 1) * rows_per) of the tile.
+    // Every rank bulk-copies each row block it does not own from its staged
+    // partial into that owner's receive slot (slot = sender's rank among the
+    // others); each owner sums its block over the ranks in rank order and runs
+    // the epilogue on it.
+    const int rank = blockIdx.x % splits;            // == %cluster_ctarank for a 1-D cluster of `splits`
+    const int rows_per = C::BM / splits, cpt = BN / splits;
+    const uint32_t rb_floats = (uint32_t)rows_per * (BN + 4), rb_bytes = rb_floats * 4u;
+    float* stage = reinterpret_cast<float*>(smem);
+    float* recv = stage + (size_t)C::BM * (BN + 4);
+    if (threadIdx.x == 96) mbar_arrive_expect_tx(rbar, (uint32_t)(splits - 1) * rb_bytes);
+    fence_proxy_async_smem();   // this thread's staging writes -> the bulk copies' reads
+    cluster_sync();             // every rank's partial is staged and its receive barrier armed
+    if (threadIdx.x == 96) {
+      for (int rr = 0; rr < splits; ++rr) {
+        if (rr == rank) continue;
+        const int slot = rank < rr ? rank : rank - 1;
+        bulk_copy_to_cluster(dsmem_map(smem_u32(recv + (size_t)slot * rb_floats), (uint32_t)rr),
+                             smem_u32(stage + (size_t)rr * rb_floats), rb_bytes,
+                             dsmem_map(smem_u32(rbar), (uint32_t)rr));
+      }
+      bulk_commit_group();
+    }
     if (warp >= 3) {
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(rbar, 0u, err) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
       const int t = threadIdx.x - 96;                  // 0..127
-      const int rank = blockIdx.x % splits;            // == %cluster_ctarank for a 1-D cluster of `splits`
       const int mn = blockIdx.x / splits;
       const int mt = mn / ntn, nt = mn - mt * ntn;
-      const int rows_per = C::BM / splits, cpt = BN / splits;
-      const int lrow = rank * rows_per + t / splits;
-      const int cbase = (t % splits) * cpt;
+      const int brow = t / splits, cbase = (t % splits) * cpt;
+      const int lrow = rank * rows_per + brow;
       const int row = mt * C::BM + lrow;
-      const bool row_ok = row < M && blockIdx.x < num_tiles;
+      const bool row_ok = ok && row < M && blockIdx.x < num_tiles;
       const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
-      const uint32_t my = smem_u32(reinterpret_cast<float*>(smem) + (size_t)lrow * (BN + 4) + cbase);
       float ssq = 0.f;
 #pragma unroll 1
       for (int c = 0; c < cpt; c += 32) {
@@ -437,10 +471,13 @@ __global__ void __launch_bounds__(224, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0.f;
         for (int rr = 0; rr < splits; ++rr) {
-          const uint32_t src = dsmem_map(my + c * 4, (uint32_t)rr);
+          const float* src = rr == rank ? stage + (size_t)lrow * (BN + 4)
+                                        : recv + (size_t)(rr < rank ? rr : rr - 1) * rb_floats +
+                                              (size_t)brow * (BN + 4);
+          const float4* s4 = reinterpret_cast<const float4*>(src + cbase + c);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float4 w = dsmem_ld_f4(src + i * 16);
+            const float4 w = s4[i];
             v[4 * i] += w.x; v[4 * i + 1] += w.y; v[4 * i + 2] += w.z; v[4 * i + 3] += w.w;
           }
         }
@@ -453,7 +490,9 @@ __global__ void __launch_bounds__(224, 1)
         if (row_ok && (t % splits) == 0) p.ssq_out[(size_t)nt * p.B + row] = ssq;
       }
     }
-    cluster_sync();   // peers may still read this CTA's staging until here
+    // this CTA's outgoing copies have read its staging before it can exit;
+    // incoming ones completed before the owner's barrier wait returned
+    if (threadIdx.x == 96) bulk_wait_read_all();
   }
   __syncthreads();
   if (warp == 1) {
