@@ -430,13 +430,18 @@ static cudaError_t launch_fold(const T* Q, int q_stride, const T* K, const T* V,
                         q0, nq, k0, nk, sc2, init, fin);
     }
     if (fast && dh == 64 && nk <= 8 && q_stride % 8 == 0 && kv_stride % 8 == 0) {
-      // grid of k_fold_small: 32 / S pairs per CTA, or ceil(nq / 32) CTAs per pair
-      int S = 1;
-      while (S < nq || S < nk) S <<= 1;
-      S = std::min(S, 32);
-      const long ctas = (long)((pairs + 32 / S - 1) / (32 / S)) * ((nq + S - 1) / S);
+      // grid of k_fold_small: 16 / S pairs per CTA, or ceil(nq / 16) CTAs per pair
+      const int S = fold_small_slots(nq, nk);
+      const long ctas = (long)((pairs + 16 / S - 1) / (16 / S)) * ((nq + S - 1) / S);
       if (ctas > 0x7fffffffL) return cudaErrorInvalidValue;
-      return launch_pdl(k_fold_small, dim3((unsigned)ctas), dim3(256), 0, st, Q, q_stride, K, V, kv_stride, m, l, o,
+      const dim3 grid((unsigned)ctas), block(128);
+      if (nq <= nk && (nk == 1 || nk == 2 || nk == 4 || nk == 8)) {
+        // the layer's blocks: compile-time key count (S == nk)
+        auto kern = nk == 1 ? k_fold_small<1> : nk == 2 ? k_fold_small<2> : nk == 4 ? k_fold_small<4> : k_fold_small<8>;
+        return launch_pdl(kern, grid, block, 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B, H, q0, nq, k0,
+                          nk, sc2, init, fin);
+      }
+      return launch_pdl(k_fold_small<0>, grid, block, 0, st, Q, q_stride, K, V, kv_stride, m, l, o,
                         a_out, B, H, q0, nq, k0, nk, sc2, init, fin);
     }
   }

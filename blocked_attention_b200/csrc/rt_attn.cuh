@@ -278,54 +278,40 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& w, float (&v)[8]) {
   }
 }
 
-// Work split: a CTA holds 32 octets. With S = min(32, the power of two
-// >= max(nq, nk)) query slots per (b, h) pair, a CTA serves 32 / S pairs
-// (S < 32) or 32 queries of one pair (nq > 32, the pair's queries cut into
-// ceil(nq / 32) CTAs). The CTA's keys -- at most 32 (pair, key) rows of k and
-// of v -- are staged once in shared memory by cp.async, so every query of a
-// pair reads them from there; q, (m, l, o) and the temporary pair are loaded
-// per octet before the staging wait, so all global loads of the CTA are in
-// flight together (one round of memory latency).
-__device__ __forceinline__ int fold_small_slots(int nq, int nk) {
+// Work split: a CTA of 128 threads holds 16 octets. With S = min(16, the
+// power of two >= max(nq, nk)) query slots per (b, h) pair, a CTA serves
+// 16 / S pairs (S < 16) or 16 queries of one pair (nq > 16: the pair's
+// queries cut into ceil(nq / 16) CTAs). For nk >= 2 the CTA's keys -- at
+// most 16 (pair, key) rows of k and of v -- are staged once in shared memory
+// by cp.async, so every query of a pair reads them from there; a single key
+// (nk = 1, half of all steps) has no reuse and is loaded by each octet
+// directly. All index arithmetic precedes the wait for the predecessor
+// kernel, and every global load of a thread is issued before the first use
+// (one round of memory latency). NK > 0 fixes nk = NK and S = NK at compile
+// time (the layer's blocks, nq <= nk); NK = 0 takes them at run time.
+__host__ __device__ __forceinline__ int fold_small_slots(int nq, int nk) {
   int s = 1;
   while (s < nq || s < nk) s <<= 1;
-  return s < 32 ? s : 32;
+  return s < 16 ? s : 16;
 }
 
-__global__ void __launch_bounds__(256, 4)
+template <int NK>
+__global__ void __launch_bounds__(128)
     k_fold_small(const __nv_bfloat16* __restrict__ qkv, int q_stride, const __nv_bfloat16* __restrict__ K,
                  const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m, float* __restrict__ l,
                  float* __restrict__ o, __nv_bfloat16* __restrict__ a_out, int B, int H, int q0, int nq,
-                 int k0, int nk, float sc2, int init, int fin) {
+                 int k0, int nk_rt, float sc2, int init, int fin) {
   constexpr int DH = 64, KMAX = 8;
-  __shared__ __align__(16) uint4 skv[2][32 * 8];   // [k | v][(pair_local * nk + key) * 8 + 16-byte part]
-  pdl_launch_dependents();
-  pdl_wait();
+  constexpr bool STAGED = NK != 1;
+  __shared__ __align__(16) uint4 skv[STAGED ? 2 : 1][STAGED ? 16 * 8 : 1];   // [k | v][(pair_local * n + key) * 8 + part]
+  const int n = NK > 0 ? NK : min(nk_rt, KMAX);      // callers use this kernel for nk <= 8
   const int pairs = B * H;
-  const int S = fold_small_slots(nq, nk);
-  const int chunks = (nq + S - 1) / S;               // > 1 only when S = 32
-  const int P = 32 / S;                              // pairs per CTA (1 when chunks > 1)
-  const int pair0 = (int)(blockIdx.x / chunks) * P;
-  const int qbase = (int)(blockIdx.x % chunks) * S;
-  const int n = min(nk, KMAX);                       // callers use this kernel for nk <= 8
+  const int S = NK > 0 ? NK : fold_small_slots(nq, n);
+  const int chunks = NK > 0 ? 1 : (nq + S - 1) / S;  // > 1 only when S = 16
+  const int P = 16 / S;                              // pairs per CTA (1 when chunks > 1)
+  const int pair0 = (chunks == 1 ? (int)blockIdx.x : (int)blockIdx.x / chunks) * P;
+  const int qbase = chunks == 1 ? 0 : ((int)blockIdx.x % chunks) * S;
   const int d = H * DH;
-
-  // ---- stage the keys of the CTA's pairs ----
-  const int E = P * n;                               // (pair, key) rows, <= 32
-  for (int u = threadIdx.x; u < 2 * E * 8; u += blockDim.x) {
-    const int kv = u / (E * 8), r = u - kv * (E * 8);
-    const int e = r >> 3, part = r & 7;
-    const int pl = e / n, i = e - pl * n;
-    const int pair = pair0 + pl;
-    if (pair < pairs) {
-      const int b = pair / H, h = pair - b * H;
-      const __nv_bfloat16* src = (kv ? V : K) + ((size_t)(k0 + i) * B + b) * kv_stride + h * DH + part * 8;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&skv[kv][e * 8 + part])), "l"(src)
-                   : "memory");
-    }
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-
   // ---- this octet's query ----
   const int oct = threadIdx.x >> 3, sl = threadIdx.x & 7;
   const unsigned omask = 0xFFu << ((threadIdx.x & 31) & 24);
@@ -337,11 +323,37 @@ __global__ void __launch_bounds__(256, 4)
   const __nv_bfloat16* qp = qkv + row * (size_t)q_stride + h * DH + sl * 8;
   const bool finrow = active && fin && qi == 0;
   float* op = o + row * (size_t)d + h * DH + sl * 8;
-  uint4 qw = make_uint4(0, 0, 0, 0), ktw = qw, vtw = qw;
+  const size_t kv0 = ((size_t)k0 * B + b) * kv_stride + h * DH + sl * 8;   // key k0 of this pair (nk = 1 path)
+
+  pdl_launch_dependents();
+  pdl_wait();
+
+  if (STAGED) {
+    // ---- stage the keys of the CTA's pairs ----
+    const int E = P * n;                             // (pair, key) rows, <= 16
+    for (int u = threadIdx.x; u < 2 * E * 8; u += blockDim.x) {
+      const int kv = u >= E * 8 ? 1 : 0, r = u - kv * (E * 8);
+      const int e = r >> 3, part = r & 7;
+      const int pe = e / n, i = e - pe * n;
+      const int pr = pair0 + pe;
+      if (pr < pairs) {
+        const int bb = pr / H, hh = pr - bb * H;
+        const __nv_bfloat16* src = (kv ? V : K) + ((size_t)(k0 + i) * B + bb) * kv_stride + hh * DH + part * 8;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&skv[kv][e * 8 + part])), "l"(src)
+                     : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  uint4 qw = make_uint4(0, 0, 0, 0), ktw = qw, vtw = qw, k1w = qw, v1w = qw;
   float mo = -INFINITY, lo = 0.f;
   float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;
   if (active) {
     qw = *reinterpret_cast<const uint4*>(qp);
+    if (!STAGED) {
+      k1w = *reinterpret_cast<const uint4*>(K + kv0);
+      v1w = *reinterpret_cast<const uint4*>(V + kv0);
+    }
     if (finrow) {
       ktw = *reinterpret_cast<const uint4*>(qp + d);
       vtw = *reinterpret_cast<const uint4*>(qp + 2 * d);
@@ -353,15 +365,17 @@ __global__ void __launch_bounds__(256, 4)
       o1 = reinterpret_cast<const float4*>(op)[1];
     }
   }
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();
+  if (STAGED) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+  }
   if (!active) return;   // whole octets leave together; no barrier follows
 
   float oo[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
   float q[8];
   unpack_bf16x8(qw, q);
-  const uint4* sk = &skv[0][(pl * n) * 8 + sl];
-  const uint4* sv = &skv[1][(pl * n) * 8 + sl];
+  const uint4* sk = &skv[0][STAGED ? (pl * n) * 8 + sl : 0];
+  const uint4* sv = &skv[STAGED ? 1 : 0][STAGED ? (pl * n) * 8 + sl : 0];
   // ---- scores ----
   float s[KMAX];
   float mx = -INFINITY;
@@ -370,7 +384,7 @@ __global__ void __launch_bounds__(256, 4)
     s[i] = -INFINITY;
     if (i < n) {
       float kk[8];
-      unpack_bf16x8(sk[i * 8], kk);
+      unpack_bf16x8(STAGED ? sk[i * 8] : k1w, kk);
       float dot = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
@@ -404,7 +418,7 @@ __global__ void __launch_bounds__(256, 4)
     if (i < n) {
       const float p = exp2f(s[i] - mn);
       float vv[8];
-      unpack_bf16x8(sv[i * 8], vv);
+      unpack_bf16x8(STAGED ? sv[i * 8] : v1w, vv);
       lo += p;
 #pragma unroll
       for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
