@@ -113,11 +113,19 @@ def test_block_fold_matches_oracle(rt, dtype, nk, nq, init_empty):
     m_got = to_np(mg)[q0:q0 + nq].transpose(1, 2, 0) / LOG2E
     l_got = to_np(lg)[q0:q0 + nq].transpose(1, 2, 0)
     o_got = to_np(og)[q0:q0 + nq].reshape(nq, B, H, dh).transpose(1, 2, 0, 3)
-    tol = 2e-3 if dtype == "bf16" else 1e-5      # bf16 P in the PV product
     assert np.max(np.abs(m_got - mr)) < 1e-4 * max(1.0, np.max(np.abs(mr)))
-    # compare normalised outputs and the normaliser
-    assert rel_err(o_got / l_got[..., None], orr / lr[..., None]) < tol
-    assert rel_err(l_got, lr) < tol
+    # compare normalised outputs and the normaliser. In bf16 the kernels round
+    # the probabilities P to bf16 (unit roundoff 2^-9) before the PV product
+    # while the normaliser sums them in fp32, so each normalised output
+    # element is a convex combination of the block's v values with weights
+    # off by at most 2^-9 relative: |error| <= 2^-9 * max|v| (+ fp32 sums).
+    if dtype == "bf16":
+        bound = 2.0 ** -9 * np.max(np.abs(Vc[k0:k0 + nk])) * 1.01 + 1e-5
+        assert np.max(np.abs(o_got / l_got[..., None] - orr / lr[..., None])) <= bound
+        assert rel_err(l_got, lr) < 2.0 ** -9 * 1.01
+    else:
+        assert rel_err(o_got / l_got[..., None], orr / lr[..., None]) < 1e-5
+        assert rel_err(l_got, lr) < 1e-5
     # rows outside the query range are untouched
     untouched = np.ones(npos, bool); untouched[q0:q0 + nq] = False
     np.testing.assert_array_equal(to_np(og)[untouched], o0[untouched].astype(np.float32))
