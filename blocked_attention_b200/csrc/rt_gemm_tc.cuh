@@ -149,6 +149,23 @@ struct GemmCfg {
   static_assert(STAGES >= 2, "stages");
 };
 
+// Pulls into L1 the residual operand the epilogue will read for `ncols`
+// columns of a row from col0 on (WO: x, bf16; W2: u, fp32).
+template <int EPI>
+__device__ __forceinline__ void epilogue_prefetch(const EpiParams& p, int row, int col0, int N, int ncols) {
+  for (int c = 0; c < ncols; c += 32) {
+    if (col0 + c >= N) break;
+    const void* ptr = nullptr;
+    if constexpr (EPI == EPI_WO) {
+      const int ch = p.j / p.xc;
+      ptr = p.x + (((size_t)ch * p.B + row) * p.xc + (p.j - ch * p.xc)) * p.d + col0 + c;
+    } else if constexpr (EPI == EPI_W2) {
+      ptr = p.u32 + (size_t)row * p.d + col0 + c;
+    }
+    if (ptr) asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));   // one 128-byte line per chunk
+  }
+}
+
 // Row-wise epilogue for one 32-column chunk; returns the chunk's sum of squares
 // of the value that feeds the next RMSNorm (WO: u, W2: z), else 0.
 template <int EPI>
@@ -385,18 +402,21 @@ __global__ void __launch_bounds__(224, 1)
       const int mn = tile / splits;
       const int mt = mn / ntn, nt = mn - mt * ntn;
       const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
+      const int lrow = q * 32 + lane;
+      const int row = mt * C::BM + lrow;
+      const bool row_ok = row < M;
+      // while the tile's MMAs run: the row's RMS scale (reads the previous
+      // kernel's partial sums) and the epilogue's residual operand into L1
+      const float rs = (splits == 1 && row_ok) ? row_scale_for<EPI>(p, row) : 0.f;
+      if (splits == 1 && row_ok) epilogue_prefetch<EPI>(p, row, nt * BN, N, BN);
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], aph, err) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int lrow = q * 32 + lane;
-      const int row = mt * C::BM + lrow;
-      const bool row_ok = row < M;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * NACC * BN;
       const bool two = NACC == 2 && nk >= 2;   // issuer 1 wrote its accumulator in this tile
       if (splits == 1) {
-        const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
         float ssq = 0.f;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -453,17 +473,20 @@ __global__ void __launch_bounds__(224, 1)
       bulk_commit_group();
     }
     if (warp >= 3) {
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(rbar, 0u, err) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       const int t = threadIdx.x - 96;                  // 0..127
       const int mn = blockIdx.x / splits;
       const int mt = mn / ntn, nt = mn - mt * ntn;
       const int brow = t / splits, cbase = (t % splits) * cpt;
       const int lrow = rank * rows_per + brow;
       const int row = mt * C::BM + lrow;
-      const bool row_ok = ok && row < M && blockIdx.x < num_tiles;
-      const float rs = row_ok ? row_scale_for<EPI>(p, row) : 0.f;
+      const bool in_range = row < M && blockIdx.x < num_tiles;
+      // while the other ranks' blocks are in flight
+      const float rs = in_range ? row_scale_for<EPI>(p, row) : 0.f;
+      if (in_range) epilogue_prefetch<EPI>(p, row, nt * BN + cbase, N, cpt);
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(rbar, 0u, err) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      const bool row_ok = ok && in_range;
       float ssq = 0.f;
 #pragma unroll 1
       for (int c = 0; c < cpt; c += 32) {
