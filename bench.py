@@ -39,7 +39,12 @@ METRIC = "RT-layer prefill tokens/s (B=512,N=2048,d=1024 bf16); % of roofline"
 # DRAM traffic per launch from an ncu capture, keyed by (kernel class, workload,
 # hash of the CUDA sources at capture time). Reported as null once the sources
 # change. Filled from the ncu summaries under profiles/.
-NCU_TRAFFIC: dict = {}
+NCU_TRAFFIC: dict = {
+    # W_2 GEMM, one launch at the headline's per-step shape (M = 512, N = 1024,
+    # K = 4096), ncu --set full with cache flush: dram__bytes_read.sum
+    # 14,719,744 + dram__bytes_write.sum 0 (profiles/gemm_w2_B512_d1024_dff4096.md)
+    ("gemm_w2", "headline", "28de274d9908"): 14719744,
+}
 
 
 def src_hash() -> str:
