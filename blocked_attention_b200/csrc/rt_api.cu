@@ -195,8 +195,7 @@ static int choose_bn(int M, int N) {
   return 32;
 }
 
-// Per-step GEMMs (M = B rows): 128-wide output tiles; when that gives few
-// tiles, split K (power of two, >= 4 k-blocks per split) towards ~128 CTAs.
+// Per-step GEMMs (M = B rows): output tile width and split-K factor.
 struct TileCfg {
   int bn, splits;
 };

@@ -174,9 +174,11 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------------------
 // block fold, warp kernel: one warp per (b, h) folds keys [k0, k0+nk) into
-// queries [q0, q0+nq). Used for small blocks (lowbit(t) < 16) in bf16 and for
-// every block in fp32. init = 1: the queries' accumulators are empty (first
-// fold into them), so they are written without being read.
+// queries [q0, q0+nq). Used for every block in fp32 and, through
+// rt_block_fold, for bf16 blocks whose key count none of the other kernels
+// takes (neither <= 8 nor a multiple of 16). init = 1: the queries'
+// accumulators are empty (first fold into them), so they are written without
+// being read.
 // ---------------------------------------------------------------------------
 template <class T, int DPL>
 __global__ void __launch_bounds__(128)

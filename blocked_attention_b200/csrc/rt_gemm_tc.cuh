@@ -4,12 +4,16 @@
 //
 //   C[M][N] = A[M][K] * W[N][K]^T      (A, W row-major = K-major operands)
 //
-// Kernel shape: persistent CTAs of 192 threads.
-//   warp 0      : TMA producer (one elected lane), STAGES-deep smem ring
-//   warp 1      : tensor-memory allocator + MMA issuer (one lane)
-//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31
-// Tile 128 x BN x 64; two TMEM accumulators of BN columns so that the
-// epilogue of tile i overlaps the MMAs of tile i+1.
+// Kernel shape: persistent CTAs of 224 threads (one output tile per CTA of a
+// thread-block cluster under split-K).
+//   warp 0      : TMA producer (one elected lane), STAGES-deep smem ring of
+//                 KSUB 64-wide K slices per stage
+//   warps 1, 2  : MMA issuers (one lane each; warp 1 also allocates TMEM),
+//                 taking alternate stages into their own accumulators
+//   warps 3..6  : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31 and sums
+//                 the issuers' accumulators
+// Tile 128 x BN; two tiles' accumulators in TMEM so that the epilogue of tile
+// i overlaps the MMAs of tile i+1.
 //
 // Epilogues (one thread owns one output row, 32 columns at a time):
 //   PLAIN : C fp32

@@ -40,6 +40,20 @@ def test_version_and_status_strings(L):
     assert R.status_string(-99) == "unknown status"
 
 
+def test_cuda_error_detail(L):
+    # no CUDA-runtime failure has happened on this thread yet
+    assert L.rt_last_cuda_error() == 0
+    assert L.rt_cuda_error_string(0).decode() == "no error"
+    # any code maps to some text (never NULL), including unknown ones
+    assert L.rt_cuda_error_string(2).decode()
+    assert L.rt_cuda_error_string(123456).decode()
+    # the binding's exception carries the CUDA error only for RT_ERR_CUDA
+    e = R.RTError("rt_layer_forward", R.RT_ERR_INVALID_ARG)
+    assert e.cuda_error == 0 and "CUDA error" not in str(e)
+    e = R.RTError("rt_layer_forward", R.RT_ERR_CUDA)
+    assert "CUDA error 0" in str(e)
+
+
 def test_workspace_plan(L):
     bf, f32 = R.RT_BF16, R.RT_F32
     ws = L.rt_layer_workspace_bytes
