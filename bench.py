@@ -69,6 +69,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--decode", action="store_true",
+                    help="time the autoregressive decode step (B sequences, one new position against a cache)")
+    ap.add_argument("--decode-t", type=int, default=0, help="decoded position (default: the workload's N)")
     ap.add_argument("--stack", action="store_true",
                     help="6-layer stack with token embedding (B=64 N=2048 d=1280 H=20x64 d_ff=5120)")
     ap.add_argument("--sweep", action="store_true",
@@ -325,6 +328,45 @@ def run_stack(args, R, torch, rtinputs):
           flush=True)
 
 
+def run_decode(args, R, torch, rtinputs):
+    """Tokens/s of the decode step at the workload's widths: B sequences each
+    produce one new position t against a cache of t - 1 persistent pairs (one
+    step = one rt_layer_decode_step; the same position is re-decoded every
+    step, overwriting cache row t - 1)."""
+    cfg = WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    Bsz, N, d, H, dff = cfg["B"], cfg["N"], cfg["d"], cfg["H"], cfg["d_ff"]
+    t = args.decode_t or N
+    W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
+         for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16").items()}
+    Kc = torch.randn((t, Bsz, d), device=dev, dtype=torch.bfloat16)
+    Vc = torch.randn((t, Bsz, d), device=dev, dtype=torch.bfloat16)
+    xt = torch.randn((Bsz, d), device=dev, dtype=torch.bfloat16)
+    z = torch.empty_like(xt)
+    ws = R.alloc_workspace(R.decode_workspace_bytes(Bsz, d, H, dff), dev)
+
+    def step():
+        R.layer_decode_step(xt, W, H, t, Kc, Vc, out=z, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    assert R.sync_status(ws) == 0
+    kv_bytes = 2 * (t - 1) * Bsz * d * 2          # the cached keys and values read once
+    print(json.dumps({"metric": "RT layer decode tokens/s", "value": Bsz / (ms / 1e3), "unit": "tokens/s",
+                      "ms_per_step": ms, "steps": args.steps, "warmup": max(args.warmup, 3), "dtype": "bf16",
+                      "data": "synthetic", "cache_read_GBps": kv_bytes / (ms / 1e3) / 1e9,
+                      "config": {"workload": f"decode position {t}, B={Bsz} d={d} H={H}x{d // H} d_ff={dff}",
+                                 "B": Bsz, "t": t, "d": d, "H": H, "d_ff": dff}}), flush=True)
+
+
 def run_sweep(args, R, torch):
     """Sequence-length sweep, blocked vs naive schedule: latency per forward."""
     c = SWEEP
@@ -396,6 +438,9 @@ def main():
     torch.cuda.set_device(local)
     if args.profile_case:
         run_profile_case(args, R, torch, rtinputs)
+        return
+    if args.decode:
+        run_decode(args, R, torch, rtinputs)
         return
     if args.stack or args.sweep:
         (run_stack(args, R, torch, rtinputs) if args.stack else run_sweep(args, R, torch))

@@ -462,7 +462,7 @@ static cudaError_t launch_attend(const Plan& P, const T* qkv, const T* K, const 
     return launch_pdl(k_finalize<T, DPL>, dim3(blocks), dim3(128), 0, st, qkv, m, l, o, a, s.B, s.H, j, sc2,
                       j > 0 ? 1 : 0);
   // naive schedule: one CTA of 8 warps per (b, h), keys split across the warps
-  return launch_pdl(k_naive_attn<T, DPL>, dim3(s.B * s.H), dim3(256), 0, st, qkv, K, V, a, s.B, s.H, j, sc2);
+  return launch_pdl(k_naive_attn<T, DPL>, dim3(s.B * s.H), dim3(256), 0, st, qkv, K, V, a, s.B, s.H, j, j, sc2);
 }
 
 // ---------------------------------------------------------------------------
@@ -1007,6 +1007,99 @@ extern "C" int rt_block_fold(const void* Q, int q_stride, const void* K, const v
   else
     return RT_ERR_INVALID_ARG;
   return e == cudaSuccess ? RT_OK : cuda_failure(e);
+}
+
+// ---------------------------------------------------------------------------
+// autoregressive decode step (RT paper §7.3)
+// ---------------------------------------------------------------------------
+static Shape decode_shape(int B, int d, int H, int d_ff) { return Shape{B, 1, d, H, d_ff, RT_BF16, RT_SCHED_NAIVE}; }
+
+extern "C" size_t rt_layer_decode_workspace_bytes(int B, int d, int H, int d_ff) {
+  const Shape s = decode_shape(B, d, H, d_ff);
+  if (validate(s) != RT_OK) return 0;
+  return make_plan(s).total;
+}
+
+// Position t of B sequences: projection of x_t, attention of its query over
+// the cached persistent pairs of positions 1..t-1 plus its temporary pair,
+// W_o, MLP, and the new persistent pair written to row t-1 of the caches.
+// The kernels are the layer's own (naive-schedule attention with the query
+// at row 0 of a one-position Q/K~/V~ buffer).
+extern "C" int rt_layer_decode_step(const void* x_t, const void* W_q, const void* W_k, const void* W_v,
+                                    const void* W_o, const void* W_1, const void* W_2, int B, int t, int capacity,
+                                    int d, int H, int d_ff, void* z_t, void* K_cache, void* V_cache,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  const Shape s = decode_shape(B, d, H, d_ff);
+  int rc = validate(s);
+  if (rc != RT_OK) return rc;
+  if (t < 1 || t > capacity || (long)capacity * B > (1l << 30)) return RT_ERR_INVALID_ARG;
+  if (!x_t || !W_q || !W_k || !W_v || !W_o || !W_1 || !W_2 || !z_t || !K_cache || !V_cache) return RT_ERR_INVALID_ARG;
+  const Plan P = make_plan(s);
+  if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return RT_ERR_WORKSPACE;
+  DevState* ds = nullptr;
+  rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  unsigned* err = reinterpret_cast<unsigned*>(ws + P.off_err);
+  bf16* qkv = reinterpret_cast<bf16*>(ws + P.off_qkv);
+  float* inv = reinterpret_cast<float*>(ws + P.off_inv);
+  bf16* wqkv = reinterpret_cast<bf16*>(ws + P.off_wqkv);
+  bf16* a16 = reinterpret_cast<bf16*>(ws + P.off_a);
+  float* ssq_u = reinterpret_cast<float*>(ws + P.off_ssq_u);
+  float* ssq_z = reinterpret_cast<float*>(ws + P.off_ssq_z);
+  const bf16* x = static_cast<const bf16*>(x_t);
+  const size_t dd = (size_t)d * d * 2;
+
+  RT_CK(cudaMemsetAsync(err, 0, sizeof(unsigned), st));
+  RT_CK(cudaMemcpyAsync(wqkv, W_q, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + dd, W_k, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + 2 * dd, W_v, dd, cudaMemcpyDeviceToDevice, st));
+  k_row_inv_rms<bf16><<<(unsigned)((B + 7) / 8), 256, 0, st>>>(x, inv, (size_t)B, d, kEps);
+  RT_CK(cudaGetLastError());
+
+  // x_t, z_t are [B][d]: one position (Nseq = 1, position index 0) for the
+  // projection, W_o and W_2 epilogues; K_cache / V_cache rows are positions
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.B = B; ep.Nseq = 1; ep.xc = 1; ep.d = d; ep.d_ff = d_ff; ep.eps = kEps;
+  ep.inv_rms = inv; ep.qkv = qkv; ep.x = x;
+  ep.u32 = reinterpret_cast<float*>(ws + P.off_u32); ep.u16 = reinterpret_cast<bf16*>(ws + P.off_u16);
+  ep.h16 = reinterpret_cast<bf16*>(ws + P.off_h); ep.zout = static_cast<bf16*>(z_t);
+  ep.z16 = reinterpret_cast<bf16*>(ws + P.off_zs);
+  ep.Kout = static_cast<bf16*>(K_cache); ep.Vout = static_cast<bf16*>(V_cache);
+  const int bn_p = choose_bn(B, 3 * d);
+  CUtensorMap tA_x, tB_qkv;
+  if (!make_tmap(&tA_x, x, d, B, 128) || !make_tmap(&tB_qkv, wqkv, d, 3 * d, bn_p)) return RT_ERR_INVALID_ARG;
+  RT_CK(launch_tc<EPI_PROJ>(bn_p, tA_x, tB_qkv, B, 3 * d, d, ep, err, ds->sms, st));
+
+  const float sc2 = kLog2e / std::sqrt((float)s.dh());
+  RT_CK(launch_pdl(k_naive_attn<bf16, 2>, dim3(B * H), dim3(256), 0, st, static_cast<const bf16*>(qkv),
+                   static_cast<const bf16*>(K_cache), static_cast<const bf16*>(V_cache), a16, B, H, t - 1, 0, sc2));
+
+  const int bn_o = P.t_wo.bn, bn_1 = P.t_w1.bn, bn_2 = P.t_w2.bn, bn_kv = P.t_wkv.bn;
+  CUtensorMap tA_a, tB_o, tA_u, tB_1, tA_h, tB_2, tA_z, tB_kv;
+  if (!make_tmap(&tA_a, a16, d, B, 128) || !make_tmap(&tB_o, W_o, d, d, bn_o) ||
+      !make_tmap(&tA_u, ep.u16, d, B, 128) || !make_tmap(&tB_1, W_1, d, d_ff, bn_1) ||
+      !make_tmap(&tA_h, ep.h16, d_ff, B, 128) || !make_tmap(&tB_2, W_2, d_ff, d, bn_2) ||
+      !make_tmap(&tA_z, ep.z16, d, B, 128) || !make_tmap(&tB_kv, wqkv + (size_t)d * d, d, 2 * d, bn_kv))
+    return RT_ERR_INVALID_ARG;
+  ep.j = 0;
+  ep.ssq_out = ssq_u;
+  ep.splits = P.t_wo.splits;
+  RT_CK(launch_tc<EPI_WO>(bn_o, tA_a, tB_o, B, d, d, ep, err, ds->sms, st));
+  ep.ssq_in = ssq_u; ep.ssq_tiles = (d + bn_o - 1) / bn_o;
+  ep.splits = P.t_w1.splits;
+  RT_CK(launch_tc<EPI_W1>(bn_1, tA_u, tB_1, B, d_ff, d, ep, err, ds->sms, st));
+  ep.ssq_out = ssq_z;
+  ep.splits = P.t_w2.splits;
+  RT_CK(launch_tc<EPI_W2>(bn_2, tA_h, tB_2, B, d, d_ff, ep, err, ds->sms, st));
+  ep.ssq_in = ssq_z; ep.ssq_tiles = (d + bn_2 - 1) / bn_2;
+  ep.splits = P.t_wkv.splits;
+  ep.j = t - 1;   // the new persistent pair's row in the caches
+  RT_CK(launch_tc<EPI_WKV>(bn_kv, tA_z, tB_kv, B, 2 * d, d, ep, err, ds->sms, st));
+  return RT_OK;
 }
 
 extern "C" int rt_project_qkv(const void* x, const void* W_qkv, int B, int N, int d, int dtype, void* QKV,

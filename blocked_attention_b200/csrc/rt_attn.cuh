@@ -76,8 +76,9 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
-// naive schedule (ablation): a_j from all persistent pairs i < j plus the
-// temporary pair. One CTA of 8 warps per (b, h): warp w scores keys
+// naive schedule (ablation; also the decode step's attention): a_j from all
+// persistent pairs i < j plus the temporary pair of the query at row qpos of
+// qkv. One CTA of 8 warps per (b, h): warp w scores keys
 // w*32 + lane, w*32 + 256 + lane, ... (one key per lane, 16-byte loads), keeps
 // its own online-softmax state, and the 8 partial states are merged in shared
 // memory at the end.
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(128)
 template <class T, int DPL>
 __global__ void __launch_bounds__(256)
     k_naive_attn(const T* __restrict__ qkv, const T* __restrict__ K, const T* __restrict__ V,
-                 T* __restrict__ a_out, int B, int H, int j, float sc2) {
+                 T* __restrict__ a_out, int B, int H, int j, int qpos, float sc2) {
   constexpr int DH = DPL * 32, NW = 8;
   __shared__ float sq[DH];
   __shared__ float sm[NW], sl[NW], so[NW][DH];
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(256)
   const int pair = blockIdx.x;
   const int b = pair / H, h = pair - b * H;
   const int d = H * DH;
-  const size_t row = (size_t)j * B + b;
+  const size_t row = (size_t)qpos * B + b;   // the query's row of qkv (the layer: qpos = j)
   const T* qp = qkv + row * (size_t)(3 * d) + h * DH;
   if (threadIdx.x < DH) sq[threadIdx.x] = to_f(qp[threadIdx.x]);
   __syncthreads();

@@ -29,7 +29,7 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_erro
            "rt_layer_sync_status", "rt_layer_host_workspace_bytes", "rt_layer_forward_host",
            "rt_embed_forward", "rt_block_fold", "rt_project_qkv", "rt_gemm_bf16",
            "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc",
-           "rt_selftest_wait_timeout")
+           "rt_selftest_wait_timeout", "rt_layer_decode_workspace_bytes", "rt_layer_decode_step")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma")
@@ -96,6 +96,10 @@ def lib() -> ctypes.CDLL:
     L.rt_project_qkv_noalloc.argtypes = [vp, vp, i, i, i, vp, vp]
     L.rt_selftest_wait_timeout.restype = i
     L.rt_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp, vp]
+    L.rt_layer_decode_workspace_bytes.restype = sz
+    L.rt_layer_decode_workspace_bytes.argtypes = [i] * 4
+    L.rt_layer_decode_step.restype = i
+    L.rt_layer_decode_step.argtypes = [vp] * 7 + [i] * 6 + [vp] * 4 + [sz, vp]
     _lib = L
     return L
 
@@ -207,6 +211,33 @@ def layer_forward_timed(x: torch.Tensor, W: dict, H: int, out, workspace: torch.
 def selftest_wait_timeout(limit_ns: int, workspace: torch.Tensor, stream=None):
     """Enqueue the bounded-wait self-test (see rt_selftest_wait_timeout)."""
     _check("rt_selftest_wait_timeout", lib().rt_selftest_wait_timeout(int(limit_ns), _ptr(workspace), _stream(stream)))
+
+
+def decode_workspace_bytes(B: int, d: int, H: int, d_ff: int) -> int:
+    return int(lib().rt_layer_decode_workspace_bytes(B, d, H, d_ff))
+
+
+def layer_decode_step(x_t: torch.Tensor, W: dict, H: int, t: int, K_cache: torch.Tensor, V_cache: torch.Tensor,
+                      out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """rt_layer_decode_step: x_t [B, d] bf16 on cuda; K_cache, V_cache
+    [capacity, B, d] bf16 holding positions 1..t-1 in rows 0..t-2. Writes the
+    new persistent pair to row t-1 of the caches and returns z_t [B, d]."""
+    B, d = x_t.shape
+    d_ff = W["W_1"].shape[0]
+    cap = K_cache.shape[0]
+    for tsr in (x_t, K_cache, V_cache, *[W[n] for n in WEIGHT_NAMES]):
+        if tsr.dtype != torch.bfloat16 or not tsr.is_contiguous() or tsr.device != x_t.device:
+            raise ValueError("decode step tensors must be contiguous bf16 tensors on one device")
+    if tuple(K_cache.shape) != (cap, B, d) or tuple(V_cache.shape) != (cap, B, d):
+        raise ValueError("K_cache, V_cache must be [capacity, B, d]")
+    z = out if out is not None else torch.empty_like(x_t)
+    if workspace is None:
+        workspace = alloc_workspace(decode_workspace_bytes(B, d, H, d_ff), x_t.device)
+    rc = lib().rt_layer_decode_step(_ptr(x_t), *[_ptr(W[n]) for n in WEIGHT_NAMES], B, t, cap, d, H, d_ff,
+                                    _ptr(z), _ptr(K_cache), _ptr(V_cache), _ptr(workspace),
+                                    ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("rt_layer_decode_step", rc)
+    return z
 
 
 def sync_status(workspace: torch.Tensor, stream=None) -> int:

@@ -139,6 +139,28 @@ int rt_layer_forward_host(const void* x_host,
                           void* z_host, void* K_host, void* V_host,
                           void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* Device bytes rt_layer_decode_step needs (bf16); 0 if unsupported. */
+size_t rt_layer_decode_workspace_bytes(int B, int d, int H, int d_ff);
+
+/* One autoregressive decode step of the layer (paper §7.3: a new token costs
+ * one query against the cached persistent pairs), bf16.
+ * Position t (1-based) of B sequences whose persistent pairs of positions
+ * 1..t-1 are rows 0..t-2 of K_cache_dev / V_cache_dev, position-major
+ * [capacity][B][d] as returned by rt_layer_forward.
+ * Inputs : x_t_dev [B][d]; weights as in rt_layer_forward.
+ * Outputs: z_t_dev [B][d]; the new persistent pair (k_t, v_t) is written to
+ *          row t-1 of the caches (rows >= t are not touched).
+ * 1 <= t <= capacity, else RT_ERR_INVALID_ARG. workspace_dev: >=
+ * rt_layer_decode_workspace_bytes(...) bytes, 256-byte aligned; its error
+ * word is read by rt_layer_sync_status. Enqueued on `stream`; the result is
+ * that of rt_layer_forward's position t up to floating-point order. */
+int rt_layer_decode_step(const void* x_t_dev,
+                         const void* W_q_dev, const void* W_k_dev, const void* W_v_dev,
+                         const void* W_o_dev, const void* W_1_dev, const void* W_2_dev,
+                         int B, int t, int capacity, int d, int H, int d_ff,
+                         void* z_t_dev, void* K_cache_dev, void* V_cache_dev,
+                         void* workspace_dev, size_t workspace_bytes, void* stream);
+
 /* Token-embedding front end of a layer stack: x[b][n][:] = E[ids[b][n]][:].
  * ids_dev int32 [B][N], each in [0, vocab) (out-of-range ids produce a zero
  * row and set the error word of `workspace_dev` if it is not NULL);

@@ -18,6 +18,10 @@ translation of the paper ("paper").
                              layer output z_i, stored for all later positions.
   [RT notes §2.2]            temporary vs persistent key/value pairs.
   [RT notes §4.1]            naive schedule: query t attends to all revealed KV.
+  [RT paper §7.3]            decoding: a new token costs one query against
+                             the cached persistent pairs, as in a standard
+                             Transformer (the recurrence is over positions
+                             already in the cache).
   [RT notes §4.2]            blocked schedule: queries precomputed; when
                              (k_t, v_t) is revealed a block is folded into the
                              online-softmax statistics (m, l, o) of a batch of
@@ -131,6 +135,38 @@ def rt_layer(x: np.ndarray, W: dict, H: int, kv_source: str = "output"):
     K = Kp.transpose(0, 2, 1, 3).reshape(B, N, d)
     V = Vp.transpose(0, 2, 1, 3).reshape(B, N, d)
     return z, K, V
+
+
+def rt_decode_step(x_t: np.ndarray, W: dict, H: int, K_prev: np.ndarray, V_prev: np.ndarray):
+    """One autoregressive step of the RT layer [RT paper §7.3, §2.2].
+
+    x_t: [B, d] inputs of position t; K_prev, V_prev: [B, t-1, d] persistent
+    pairs of positions 1..t-1 (head h in columns h*d_h .. (h+1)*d_h - 1).
+    Returns (z_t, k_t, v_t), each [B, d]: the new position's output and its
+    persistent pair, which the caller appends to the cache.
+
+    Query and temporary pair from RMS(x_t); per head, attention over the cached
+    keys plus the temporary key with scores <k, q_h> / sqrt(d_h); then W_o,
+    residual, MLP, and (k_t, v_t) = (W_k RMS(z_t), W_v RMS(z_t)).
+    """
+    x_t = np.asarray(x_t, dtype=np.float64)
+    B, d = x_t.shape
+    dh = d // H
+    K_prev = np.asarray(K_prev, dtype=np.float64).reshape(B, -1, H, dh).transpose(0, 2, 1, 3)   # [B,H,t-1,dh]
+    V_prev = np.asarray(V_prev, dtype=np.float64).reshape(B, -1, H, dh).transpose(0, 2, 1, 3)
+    r = rms(x_t)
+    q = _heads(r @ W["W_q"].T, H)
+    k_tmp = _heads(r @ W["W_k"].T, H)
+    v_tmp = _heads(r @ W["W_v"].T, H)
+    keys = np.concatenate([K_prev, k_tmp[:, :, None]], axis=2)       # [B,H,t,dh]
+    vals = np.concatenate([V_prev, v_tmp[:, :, None]], axis=2)
+    s = np.einsum("bhe,bhie->bhi", q, keys) / np.sqrt(dh)
+    w = np.exp(s - s.max(axis=-1, keepdims=True))
+    a = np.einsum("bhi,bhie->bhe", w, vals) / w.sum(axis=-1)[..., None]
+    u = x_t + a.reshape(B, d) @ W["W_o"].T
+    z_t = u + mlp(u, W)
+    rz = rms(z_t)
+    return z_t, rz @ W["W_k"].T, rz @ W["W_v"].T
 
 
 # --------------------------------------------------------------------------

@@ -54,6 +54,25 @@ def test_cuda_error_detail(L):
     assert "CUDA error 0" in str(e)
 
 
+def test_decode_step_validation_happens_before_any_launch(L):
+    B, d, H, d_ff = 4, 128, 2, 256
+    assert L.rt_layer_decode_workspace_bytes(B, d, H, d_ff) > 0
+    assert L.rt_layer_decode_workspace_bytes(B, 96, 2, d_ff) == 0    # d_h = 48: bf16 path needs 64
+    assert L.rt_layer_decode_workspace_bytes(0, d, H, d_ff) == 0
+    p = ctypes.c_void_p(1 << 40)   # never dereferenced: every call below fails validation first
+
+    def call(t, cap, Bv=B, dv=d, ws_bytes=1 << 30):
+        return L.rt_layer_decode_step(*([p] * 7), Bv, t, cap, dv, H, d_ff, p, p, p, p,
+                                      ctypes.c_size_t(ws_bytes), None)
+    assert call(0, 8) == R.RT_ERR_INVALID_ARG          # positions are 1-based
+    assert call(9, 8) == R.RT_ERR_INVALID_ARG          # beyond the cache capacity
+    assert call(1, 8, Bv=0) == R.RT_ERR_INVALID_ARG
+    assert call(1, 8, dv=96) == R.RT_ERR_UNSUPPORTED
+    assert call(1, 8, ws_bytes=16) == R.RT_ERR_WORKSPACE
+    assert L.rt_layer_decode_step(None, *([p] * 6), B, 1, 8, d, H, d_ff, p, p, p, p,
+                                  ctypes.c_size_t(1 << 30), None) == R.RT_ERR_INVALID_ARG
+
+
 def test_workspace_plan(L):
     bf, f32 = R.RT_BF16, R.RT_F32
     ws = L.rt_layer_workspace_bytes

@@ -215,6 +215,37 @@ def test_N2_closed_form_persistent_key_from_output():
         np.testing.assert_allclose(V[b, 1], _py_mv(Wl["W_v"], _py_rms(z2)), rtol=1e-12, atol=1e-13)
 
 
+def test_decode_step_N1_closed_form():
+    # an empty cache: the step is the single-token layer of the closed form above
+    d, H, d_ff = 8, 2, 16
+    x, W = _problem(3, 1, d, H, d_ff, sigma=0.4)
+    Wl = {k: v.tolist() for k, v in W.items()}
+    z, k, v = O.rt_decode_step(x[:, 0], W, H, np.zeros((3, 0, d)), np.zeros((3, 0, d)))
+    for b in range(3):
+        xb = x[b, 0].tolist()
+        zb = _py_layer_tail(xb, _py_mv(Wl["W_v"], _py_rms(xb)), Wl)
+        np.testing.assert_allclose(z[b], zb, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(k[b], _py_mv(Wl["W_k"], _py_rms(zb)), rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(v[b], _py_mv(Wl["W_v"], _py_rms(zb)), rtol=1e-13, atol=1e-14)
+
+
+def test_decode_from_empty_cache_reproduces_the_layer():
+    # Autoregressive consistency: feeding each step's own (k_t, v_t) back as
+    # cache reproduces the whole-sequence layer (naive definition and the
+    # blocked schedule), peaky attention included.
+    for sigma in (0.02, 0.3):
+        x, W = _problem(2, 19, 16, 2, 32, sigma=sigma)
+        z, K, V = O.rt_layer(x, W, 2)
+        zb, Kb, Vb = O.rt_layer_blocked(x, W, 2)
+        Kc = np.zeros((2, 0, 16)); Vc = np.zeros((2, 0, 16))
+        for t in range(19):
+            zt, kt, vt = O.rt_decode_step(x[:, t], W, 2, Kc, Vc)
+            for ref, got in ((z[:, t], zt), (K[:, t], kt), (V[:, t], vt), (zb[:, t], zt)):
+                np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+            Kc = np.concatenate([Kc, kt[:, None]], axis=1)
+            Vc = np.concatenate([Vc, vt[:, None]], axis=1)
+
+
 # --------------------------------------------------------------------------
 # standard-layer special case (paper §2.1): a textbook causal pre-norm layer
 # written as one masked score matrix per head
