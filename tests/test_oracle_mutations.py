@@ -42,6 +42,14 @@ MUTANTS = {
     "query block one short": (
         "queries = list(range(t + 1, min(t + lb, N) + 1))", "queries = list(range(t + 1, min(t + lb, N)))",
         ["test_schedule_covers_every_causal_pair_exactly_once"]),
+    "decode step: persistent pair from the input": (
+        "    rz = rms(z_t)\n    return z_t, rz @ W[\"W_k\"].T, rz @ W[\"W_v\"].T",
+        "    rz = rms(x_t)\n    return z_t, rz @ W[\"W_k\"].T, rz @ W[\"W_v\"].T",
+        ["test_decode_step_N1_closed_form", "test_decode_from_empty_cache_reproduces_the_layer"]),
+    "decode step: temporary key used as its value": (
+        "    vals = np.concatenate([V_prev, v_tmp[:, :, None]], axis=2)",
+        "    vals = np.concatenate([V_prev, k_tmp[:, :, None]], axis=2)",
+        ["test_decode_step_N1_closed_form", "test_decode_from_empty_cache_reproduces_the_layer"]),
     "wrong rescale sign in the fold": (
         "alpha = np.where(np.isneginf(m), 0.0, np.exp(m - m_new))",
         "alpha = np.where(np.isneginf(m), 0.0, np.exp(m_new - m))",
