@@ -170,6 +170,62 @@ def rt_decode_step(x_t: np.ndarray, W: dict, H: int, K_prev: np.ndarray, V_prev:
 
 
 # --------------------------------------------------------------------------
+# the paper's own parameterisation (not the single-layer configuration)
+# --------------------------------------------------------------------------
+def rms_unit(v: np.ndarray) -> np.ndarray:
+    """RMS(v) = sqrt(D) v / ||v||_2 over the last axis of width D, exactly as
+    written in [RT paper §2, notation] (no eps, unit gain)."""
+    return v * np.sqrt(v.shape[-1]) / np.linalg.norm(v, axis=-1, keepdims=True)
+
+
+def rt_layer_pages(x: np.ndarray, W: dict, H: int, L: int = 1, kv_source: str = "output"):
+    """RT layer in the paper's own parameterisation [RT paper §2 notation,
+    §2.1, §2.2]; naive per-step schedule.
+
+    Per position t and sequence b, with RMS = rms_unit and RMS_h = rms_unit
+    over each head's d_h entries (the query/key normalisation, applied per
+    head as the multi-head rule applies the single-head construction per head):
+        r = RMS(x_t); q = RMS_h(W_q r); k~ = RMS_h(W_k r); v~ = W_v r
+        per head: a_h = Attn(cached pairs + (k~, v~), q_h), scores <k, q_h>
+                  (no softmax scale)
+        u = x_t + W_o a / sqrt(L);  z_t = u + W_2 GELU(W_1 RMS(u)) / sqrt(L)
+        persistent k_t = RMS_h(W_k RMS(s_t)), v_t = W_v RMS(s_t)
+    with s_t = z_t (kv_source="output") or x_t ("input": the standard layer
+    of [RT paper §2.1]). The persistent-pair equations are cut off in the
+    extracted §2.2; they are read as the temporary ones applied to s_t.
+    Returns (z, K, V), each [B, N, d].
+    """
+    if kv_source not in ("output", "input"):
+        raise ValueError(kv_source)
+    x = np.asarray(x, dtype=np.float64)
+    B, N, d = x.shape
+    dh = d // H
+    inv_sqrt_L = 1.0 / np.sqrt(L)
+    z = np.empty_like(x)
+    Kp = np.empty((B, H, N, dh))
+    Vp = np.empty((B, H, N, dh))
+    for t in range(N):
+        r = rms_unit(x[:, t])
+        q = rms_unit(_heads(r @ W["W_q"].T, H))
+        kt = rms_unit(_heads(r @ W["W_k"].T, H))
+        vt = _heads(r @ W["W_v"].T, H)
+        keys = np.concatenate([Kp[:, :, :t], kt[:, :, None]], axis=2)
+        vals = np.concatenate([Vp[:, :, :t], vt[:, :, None]], axis=2)
+        s = np.einsum("bhe,bhie->bhi", q, keys)
+        w = np.exp(s - s.max(axis=-1, keepdims=True))
+        a = np.einsum("bhi,bhie->bhe", w, vals) / w.sum(axis=-1)[..., None]
+        u = x[:, t] + (a.reshape(B, d) @ W["W_o"].T) * inv_sqrt_L
+        zt = u + (gelu(rms_unit(u) @ W["W_1"].T) @ W["W_2"].T) * inv_sqrt_L
+        z[:, t] = zt
+        rs = rms_unit(zt if kv_source == "output" else x[:, t])
+        Kp[:, :, t] = rms_unit(_heads(rs @ W["W_k"].T, H))
+        Vp[:, :, t] = _heads(rs @ W["W_v"].T, H)
+    K = Kp.transpose(0, 2, 1, 3).reshape(B, N, d)
+    V = Vp.transpose(0, 2, 1, 3).reshape(B, N, d)
+    return z, K, V
+
+
+# --------------------------------------------------------------------------
 # blocked (lowbit) schedule, in the pages' order
 # --------------------------------------------------------------------------
 def lowbit_blocks(N: int):

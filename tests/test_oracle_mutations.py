@@ -50,6 +50,18 @@ MUTANTS = {
         "    vals = np.concatenate([V_prev, v_tmp[:, :, None]], axis=2)",
         "    vals = np.concatenate([V_prev, k_tmp[:, :, None]], axis=2)",
         ["test_decode_step_N1_closed_form", "test_decode_from_empty_cache_reproduces_the_layer"]),
+    "paper parameterisation: softmax scale kept": (
+        '        s = np.einsum("bhe,bhie->bhi", q, keys)\n        w = np.exp(s - s.max',
+        '        s = np.einsum("bhe,bhie->bhi", q, keys) / np.sqrt(dh)\n        w = np.exp(s - s.max',
+        ["test_pages_parameterisation_N1_N2_closed_forms", "test_pages_parameterisation_standard_layer_reduction"]),
+    "paper parameterisation: query norm over the whole width": (
+        '        q = rms_unit(_heads(r @ W["W_q"].T, H))',
+        '        q = _heads(rms_unit(r @ W["W_q"].T), H)',
+        ["test_pages_parameterisation_N1_N2_closed_forms", "test_pages_parameterisation_standard_layer_reduction"]),
+    "paper parameterisation: attention residual not scaled": (
+        '        u = x[:, t] + (a.reshape(B, d) @ W["W_o"].T) * inv_sqrt_L',
+        '        u = x[:, t] + (a.reshape(B, d) @ W["W_o"].T)',
+        ["test_pages_parameterisation_N1_N2_closed_forms"]),
     "wrong rescale sign in the fold": (
         "alpha = np.where(np.isneginf(m), 0.0, np.exp(m - m_new))",
         "alpha = np.where(np.isneginf(m), 0.0, np.exp(m_new - m))",

@@ -247,6 +247,92 @@ def test_decode_from_empty_cache_reproduces_the_layer():
 
 
 # --------------------------------------------------------------------------
+# the paper's own parameterisation (rt_layer_pages): pure-Python closed forms
+# --------------------------------------------------------------------------
+def _py_rms_unit(v):
+    """sqrt(D) v / ||v||_2 (paper §2 notation), no eps."""
+    n = math.sqrt(sum(e * e for e in v))
+    return [e * math.sqrt(len(v)) / n for e in v]
+
+
+def _py_heads_rms_unit(v, H):
+    dh = len(v) // H
+    out = []
+    for h in range(H):
+        out += _py_rms_unit(v[h * dh:(h + 1) * dh])
+    return out
+
+
+def _py_pages_tail(x, a, W, L):
+    """u = x + W_o a / sqrt(L); z = u + W_2 GELU(W_1 RMS(u)) / sqrt(L)."""
+    c = 1.0 / math.sqrt(L)
+    u = [xi + c * oi for xi, oi in zip(x, _py_mv(W["W_o"], a))]
+    h = [_py_gelu(e) for e in _py_mv(W["W_1"], _py_rms_unit(u))]
+    return [ui + c * mi for ui, mi in zip(u, _py_mv(W["W_2"], h))]
+
+
+def test_pages_parameterisation_N1_N2_closed_forms():
+    # N = 1: one key, a = v~ = W_v RMS(x). N = 2: per head a two-way softmax
+    # (logistic) of the unscaled scores <k1, q2>, <k~2, q2> with per-head
+    # unit-RMS keys and queries (|score| <= d_h by Cauchy-Schwarz).
+    d, H, d_ff, L = 8, 2, 16, 4
+    dh = d // H
+    x, W = _problem(2, 2, d, H, d_ff, sigma=0.5)
+    z, K, V = O.rt_layer_pages(x, W, H, L=L)
+    Wl = {k: v.tolist() for k, v in W.items()}
+    sig = lambda y: 1.0 / (1.0 + math.exp(-y))
+    for b in range(2):
+        x1, x2 = x[b, 0].tolist(), x[b, 1].tolist()
+        r1 = _py_rms_unit(x1)
+        z1 = _py_pages_tail(x1, _py_mv(Wl["W_v"], r1), Wl, L)
+        rz1 = _py_rms_unit(z1)
+        k1 = _py_heads_rms_unit(_py_mv(Wl["W_k"], rz1), H)
+        v1 = _py_mv(Wl["W_v"], rz1)
+        r2 = _py_rms_unit(x2)
+        q2 = _py_heads_rms_unit(_py_mv(Wl["W_q"], r2), H)
+        kt = _py_heads_rms_unit(_py_mv(Wl["W_k"], r2), H)
+        vt = _py_mv(Wl["W_v"], r2)
+        a = []
+        for h in range(H):
+            sl = slice(h * dh, (h + 1) * dh)
+            s1 = sum(p * r for p, r in zip(q2[sl], k1[sl]))
+            s2 = sum(p * r for p, r in zip(q2[sl], kt[sl]))
+            assert abs(s1) <= dh + 1e-9 and abs(s2) <= dh + 1e-9
+            a += [sig(s1 - s2) * e1 + sig(s2 - s1) * e2 for e1, e2 in zip(v1[sl], vt[sl])]
+        z2 = _py_pages_tail(x2, a, Wl, L)
+        np.testing.assert_allclose(z[b, 0], z1, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(K[b, 0], k1, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(V[b, 0], v1, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(z[b, 1], z2, rtol=1e-11, atol=1e-12)
+        rz2 = _py_rms_unit(z2)
+        np.testing.assert_allclose(K[b, 1], _py_heads_rms_unit(_py_mv(Wl["W_k"], rz2), H), rtol=1e-11, atol=1e-12)
+
+
+def test_pages_parameterisation_standard_layer_reduction():
+    # kv_source="input" is the paper's standard layer (§2.1): one masked score
+    # matrix per head with per-head unit-RMS q and k and no softmax scale
+    B, N, d, H, d_ff, L = 2, 9, 16, 4, 32, 3
+    dh = d // H
+    x, W = _problem(B, N, d, H, d_ff, sigma=0.3)
+    z, K, V = O.rt_layer_pages(x, W, H, L=L, kv_source="input")
+    unit = lambda v: v * np.sqrt(v.shape[-1]) / np.sqrt(np.sum(v * v, axis=-1, keepdims=True))
+    r = unit(x)
+    q = unit((r @ W["W_q"].T).reshape(B, N, H, dh)).transpose(0, 2, 1, 3)
+    k = unit((r @ W["W_k"].T).reshape(B, N, H, dh)).transpose(0, 2, 1, 3)
+    v = (r @ W["W_v"].T).reshape(B, N, H, dh).transpose(0, 2, 1, 3)
+    S = q @ k.transpose(0, 1, 3, 2)
+    S = np.where(np.triu(np.ones((N, N), dtype=bool), k=1), -np.inf, S)
+    P = np.exp(S - S.max(axis=-1, keepdims=True))
+    P /= P.sum(axis=-1, keepdims=True)
+    a = (P @ v).transpose(0, 2, 1, 3).reshape(B, N, d)
+    u = x + (a @ W["W_o"].T) / np.sqrt(L)
+    hid = unit(u) @ W["W_1"].T
+    zr = u + ((0.5 * hid * (1.0 + np.vectorize(math.erf)(hid / math.sqrt(2.0)))) @ W["W_2"].T) / np.sqrt(L)
+    np.testing.assert_allclose(z, zr, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(K, k.transpose(0, 2, 1, 3).reshape(B, N, d), rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
 # standard-layer special case (paper §2.1): a textbook causal pre-norm layer
 # written as one masked score matrix per head
 # --------------------------------------------------------------------------
