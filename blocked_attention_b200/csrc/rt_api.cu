@@ -1023,8 +1023,9 @@ extern "C" size_t rt_layer_decode_workspace_bytes(int B, int d, int H, int d_ff)
 // Position t of B sequences: projection of x_t, attention of its query over
 // the cached persistent pairs of positions 1..t-1 plus its temporary pair,
 // W_o, MLP, and the new persistent pair written to row t-1 of the caches.
-// The kernels are the layer's own (naive-schedule attention with the query
-// at row 0 of a one-position Q/K~/V~ buffer).
+// The projection and GEMMs are the layer's own; the attention is a decode
+// kernel (lanes own whole cached keys) with the query at row 0 of a
+// one-position Q/K~/V~ buffer.
 extern "C" int rt_layer_decode_step(const void* x_t, const void* W_q, const void* W_k, const void* W_v,
                                     const void* W_o, const void* W_1, const void* W_2, int B, int t, int capacity,
                                     int d, int H, int d_ff, void* z_t, void* K_cache, void* V_cache,
@@ -1075,8 +1076,8 @@ extern "C" int rt_layer_decode_step(const void* x_t, const void* W_q, const void
   RT_CK(launch_tc<EPI_PROJ>(bn_p, tA_x, tB_qkv, B, 3 * d, d, ep, err, ds->sms, st));
 
   const float sc2 = kLog2e / std::sqrt((float)s.dh());
-  RT_CK(launch_pdl(k_naive_attn<bf16, 2>, dim3(B * H), dim3(256), 0, st, static_cast<const bf16*>(qkv),
-                   static_cast<const bf16*>(K_cache), static_cast<const bf16*>(V_cache), a16, B, H, t - 1, 0, sc2));
+  RT_CK(launch_pdl(k_decode_attn, dim3(B * H), dim3(128), 0, st, static_cast<const bf16*>(qkv),
+                   static_cast<const bf16*>(K_cache), static_cast<const bf16*>(V_cache), a16, B, H, t - 1, sc2));
 
   const int bn_o = P.t_wo.bn, bn_1 = P.t_w1.bn, bn_2 = P.t_w2.bn, bn_kv = P.t_wkv.bn;
   CUtensorMap tA_a, tB_o, tA_u, tB_1, tA_h, tB_2, tA_z, tB_kv;

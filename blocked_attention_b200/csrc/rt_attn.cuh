@@ -453,6 +453,108 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
+// decode-step attention (bf16, d_h = 64): the query at row 0 of a
+// one-position qkv [B][3d] against cached keys 0..j-1 (position-major K, V
+// [.][B][d]) plus its temporary pair. One CTA of 4 warps per (b, h); each
+// lane owns whole keys (c = thread, thread + 128, ...): it loads the key's k
+// and v rows (2 x 128 bytes, sixteen 16-byte loads in flight), and keeps its
+// own online-softmax state (m, l) and 64-wide numerator. Lanes, then warps,
+// are merged at the end; warp 0 adds the temporary pair and writes a [B][d].
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+    k_decode_attn(const __nv_bfloat16* __restrict__ qkv, const __nv_bfloat16* __restrict__ K,
+                  const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __restrict__ a_out, int B, int H, int j,
+                  float sc2) {
+  constexpr int DH = 64, NW = 4;
+  __shared__ __align__(16) float sq[DH];
+  __shared__ float sm[NW], sl[NW];
+  __shared__ __align__(16) float so[NW][DH];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x;
+  const int b = pair / H, h = pair - b * H;
+  const int d = H * DH;
+  const __nv_bfloat16* qp = qkv + (size_t)b * (3 * d) + h * DH;
+  pdl_launch_dependents();
+  pdl_wait();
+  if (threadIdx.x < DH) sq[threadIdx.x] = __bfloat162float(qp[threadIdx.x]);
+  __syncthreads();
+  float m = -INFINITY, l = 0.f, oacc[DH];
+#pragma unroll
+  for (int i = 0; i < DH; ++i) oacc[i] = 0.f;
+  const float4* sq4 = reinterpret_cast<const float4*>(sq);
+  for (int c = threadIdx.x; c < j; c += blockDim.x) {
+    const size_t off = ((size_t)c * B + b) * d + h * DH;
+    const uint4* kp = reinterpret_cast<const uint4*>(K + off);
+    const uint4* vp = reinterpret_cast<const uint4*>(V + off);
+    uint4 kw[8], vw[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) kw[e] = kp[e];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vw[e] = vp[e];
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float kk[8];
+      unpack_bf16x8(kw[e], kk);
+      const float4 q0 = sq4[2 * e], q1 = sq4[2 * e + 1];
+      s += q0.x * kk[0] + q0.y * kk[1] + q0.z * kk[2] + q0.w * kk[3] + q1.x * kk[4] + q1.y * kk[5] +
+           q1.z * kk[6] + q1.w * kk[7];
+    }
+    s *= sc2;
+    if (s > m) {   // new running maximum of this lane: rescale its state
+      const float al = rescale(m, s);
+      l *= al;
+#pragma unroll
+      for (int i = 0; i < DH; ++i) oacc[i] *= al;
+      m = s;
+    }
+    const float p = exp2f(s - m);
+    l += p;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float vv[8];
+      unpack_bf16x8(vw[e], vv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) oacc[e * 8 + i] += p * vv[i];
+    }
+  }
+  // merge the warp's lanes (a lane without keys has m = -inf and weight 0)
+  const float mw = warp_max(m);
+  const float f = rescale(m, mw);
+  l = warp_sum(l * f);
+#pragma unroll
+  for (int i = 0; i < DH; ++i) oacc[i] = warp_sum(oacc[i] * f);
+  if (lane == 0) {
+    sm[w] = mw;
+    sl[w] = l;
+#pragma unroll
+    for (int i = 0; i < DH; ++i) so[w][i] = oacc[i];
+  }
+  __syncthreads();
+  if (w != 0) return;
+  // warp 0: merge the warps' states, then the temporary pair; lane owns dims 2*lane, 2*lane + 1
+  float mt = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < NW; ++k) mt = fmaxf(mt, sm[k]);
+  float lt = 0.f, ot0 = 0.f, ot1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < NW; ++k) {
+    const float fk = rescale(sm[k], mt);
+    lt += sl[k] * fk;
+    ot0 += so[k][2 * lane] * fk;
+    ot1 += so[k][2 * lane + 1] * fk;
+  }
+  const float2 kt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + d + 2 * lane));
+  const float2 vt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + 2 * d + 2 * lane));
+  const float st = warp_sum(sq[2 * lane] * kt.x + sq[2 * lane + 1] * kt.y) * sc2;
+  const float mn = fmaxf(mt, st);
+  const float al = rescale(mt, mn), pt = exp2f(st - mn);
+  const float inv = 1.f / (lt * al + pt);
+  *reinterpret_cast<__nv_bfloat162*>(a_out + (size_t)b * d + h * DH + 2 * lane) =
+      __floats2bfloat162_rn((ot0 * al + pt * vt.x) * inv, (ot1 * al + pt * vt.y) * inv);
+}
+
+// ---------------------------------------------------------------------------
 // block fold, tensor-core kernel (bf16, d_h = 64, nk a multiple of 16):
 // S = Q K^T and O += P V with mma.sync m16n8k16 (fp32 accumulate), online
 // softmax over key chunks of 64, then one merge into the fp32 (m, l, o) of
