@@ -18,6 +18,9 @@ translation of the paper ("paper").
                              layer output z_i, stored for all later positions.
   [RT notes §2.2]            temporary vs persistent key/value pairs.
   [RT notes §4.1]            naive schedule: query t attends to all revealed KV.
+  [RT paper §6.4]            backward pass (its body is missing from the
+                             extracted text): gradients here are the exact
+                             derivatives of the forward definition.
   [RT paper §7.3]            decoding: a new token costs one query against
                              the cached persistent pairs, as in a standard
                              Transformer (the recurrence is over positions
@@ -167,6 +170,61 @@ def rt_decode_step(x_t: np.ndarray, W: dict, H: int, K_prev: np.ndarray, V_prev:
     z_t = u + mlp(u, W)
     rz = rms(z_t)
     return z_t, rz @ W["W_k"].T, rz @ W["W_v"].T
+
+
+# --------------------------------------------------------------------------
+# gradients of the layer (groundwork for the backward pass)
+# --------------------------------------------------------------------------
+def rt_layer_backward(x: np.ndarray, W: dict, H: int, dz: np.ndarray, dK: np.ndarray, dV: np.ndarray):
+    """Gradients of the RT layer [RT paper §2.2] for upstream gradients dz, dK,
+    dV (each [B, N, d]): returns (dx [B, N, d], dW dict of the weight
+    gradients) of the scalar sum(z*dz) + sum(K*dK) + sum(V*dV).
+
+    The forward is the naive definition of rt_layer restated in float64
+    PyTorch CPU ops, and the gradients are PyTorch's reverse-mode derivatives
+    of it (the pages' own backward, paper §6.4, is missing from the extracted
+    text). Every persistent pair k_i, v_i receives gradient from all later
+    positions' attention, so the reverse pass runs over positions in reverse.
+    """
+    import torch
+    f64 = torch.float64
+    xt = torch.tensor(np.asarray(x, dtype=np.float64), dtype=f64, requires_grad=True)
+    Wt = {k: torch.tensor(np.asarray(v, dtype=np.float64), dtype=f64, requires_grad=True) for k, v in W.items()}
+    B, N, d = xt.shape
+    dh = d // H
+
+    def rms_t(v):
+        return v / torch.sqrt(torch.mean(v * v, dim=-1, keepdim=True) + EPS)
+
+    def heads_t(v):
+        return v.reshape(v.shape[:-1] + (H, dh))
+
+    zs, ks, vs = [], [], []
+    for t in range(N):
+        r = rms_t(xt[:, t])
+        q = heads_t(r @ Wt["W_q"].T)
+        kt = heads_t(r @ Wt["W_k"].T)
+        vt = heads_t(r @ Wt["W_v"].T)
+        keys = torch.stack(ks + [kt], dim=2)            # [B, H, t+1, dh]
+        vals = torch.stack(vs + [vt], dim=2)
+        sc = torch.einsum("bhe,bhie->bhi", q, keys) / np.sqrt(dh)
+        w = torch.softmax(sc, dim=-1)
+        a = torch.einsum("bhi,bhie->bhe", w, vals).reshape(B, d)
+        u = xt[:, t] + a @ Wt["W_o"].T
+        hid = rms_t(u) @ Wt["W_1"].T
+        zt = u + (0.5 * hid * (1.0 + torch.erf(hid / np.sqrt(2.0)))) @ Wt["W_2"].T
+        rz = rms_t(zt)
+        zs.append(zt)
+        ks.append(heads_t(rz @ Wt["W_k"].T))
+        vs.append(heads_t(rz @ Wt["W_v"].T))
+    z = torch.stack(zs, dim=1)
+    K = torch.stack(ks, dim=1).reshape(B, N, d)
+    V = torch.stack(vs, dim=1).reshape(B, N, d)
+    loss = (z * torch.tensor(dz, dtype=f64)).sum() + (K * torch.tensor(dK, dtype=f64)).sum() + \
+        (V * torch.tensor(dV, dtype=f64)).sum()
+    loss.backward()
+    dW = {k: v.grad.numpy().copy() for k, v in Wt.items()}
+    return xt.grad.numpy().copy(), dW, (z.detach().numpy(), K.detach().numpy(), V.detach().numpy())
 
 
 # --------------------------------------------------------------------------

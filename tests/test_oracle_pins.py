@@ -247,6 +247,48 @@ def test_decode_from_empty_cache_reproduces_the_layer():
 
 
 # --------------------------------------------------------------------------
+# gradients (rt_layer_backward): central finite differences of rt_layer
+# --------------------------------------------------------------------------
+def _loss(x, W, H, dz, dK, dV):
+    z, K, V = O.rt_layer(x, W, H)
+    return float(np.sum(z * dz) + np.sum(K * dK) + np.sum(V * dV))
+
+
+def test_backward_matches_finite_differences():
+    B, N, d, H, d_ff = 2, 4, 8, 2, 16
+    x, W = _problem(B, N, d, H, d_ff, sigma=0.5)
+    rng = np.random.default_rng(7)
+    dz, dK, dV = (rng.standard_normal((B, N, d)) for _ in range(3))
+    dx, dW, (z, K, V) = O.rt_layer_backward(x, W, H, dz, dK, dV)
+    zr, Kr, Vr = O.rt_layer(x, W, H)
+    np.testing.assert_allclose(z, zr, rtol=1e-12, atol=1e-13)      # the restated forward is the layer
+    np.testing.assert_allclose(K, Kr, rtol=1e-12, atol=1e-13)
+    h = 1e-5
+    for idx in [(0, 0, 0), (1, 3, 5), (0, 2, 7), (1, 1, 2)]:
+        xp = x.copy(); xp[idx] += h
+        xm = x.copy(); xm[idx] -= h
+        fd = (_loss(xp, W, H, dz, dK, dV) - _loss(xm, W, H, dz, dK, dV)) / (2 * h)
+        assert abs(fd - dx[idx]) <= 1e-6 * max(1.0, abs(fd)), (idx, fd, dx[idx])
+    for name, idx in [("W_q", (1, 2)), ("W_k", (3, 0)), ("W_v", (5, 6)), ("W_o", (0, 7)), ("W_1", (9, 4)),
+                      ("W_2", (6, 13))]:
+        Wp = {k: v.copy() for k, v in W.items()}; Wp[name][idx] += h
+        Wm = {k: v.copy() for k, v in W.items()}; Wm[name][idx] -= h
+        fd = (_loss(x, Wp, H, dz, dK, dV) - _loss(x, Wm, H, dz, dK, dV)) / (2 * h)
+        assert abs(fd - dW[name][idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd, dW[name][idx])
+
+
+def test_backward_is_causal():
+    # a gradient on z at position s reaches only the inputs of positions <= s
+    B, N, d, H, d_ff = 1, 6, 8, 2, 16
+    x, W = _problem(B, N, d, H, d_ff, sigma=0.4)
+    dz = np.zeros((B, N, d)); dz[0, 3] = 1.0
+    zero = np.zeros((B, N, d))
+    dx, _, _ = O.rt_layer_backward(x, W, H, dz, zero, zero)
+    assert np.all(dx[0, 4:] == 0.0)
+    assert np.all(np.abs(dx[0, :4]).max(axis=-1) > 0.0)
+
+
+# --------------------------------------------------------------------------
 # the paper's own parameterisation (rt_layer_pages): pure-Python closed forms
 # --------------------------------------------------------------------------
 def _py_rms_unit(v):
