@@ -173,6 +173,19 @@ def rt_decode_step(x_t: np.ndarray, W: dict, H: int, K_prev: np.ndarray, V_prev:
 
 
 # --------------------------------------------------------------------------
+# activation-checkpoint recompute and gradients (groundwork for training)
+# --------------------------------------------------------------------------
+def recompute_kv(z: np.ndarray, W: dict) -> tuple:
+    """Persistent pairs of every position rebuilt from the stored layer
+    outputs in one parallel step [RT paper §6.1, activation checkpointing:
+    with x stored, z is kept for free as the next layer's input and the
+    persistent pairs are rebuilt from it in parallel]: K = RMS(z) W_k^T,
+    V = RMS(z) W_v^T, each [B, N, d]."""
+    rz = rms(np.asarray(z, dtype=np.float64))
+    return rz @ W["W_k"].T, rz @ W["W_v"].T
+
+
+# --------------------------------------------------------------------------
 # gradients of the layer (groundwork for the backward pass)
 # --------------------------------------------------------------------------
 def rt_layer_backward(x: np.ndarray, W: dict, H: int, dz: np.ndarray, dK: np.ndarray, dV: np.ndarray):

@@ -254,6 +254,19 @@ def _loss(x, W, H, dz, dK, dV):
     return float(np.sum(z * dz) + np.sum(K * dK) + np.sum(V * dV))
 
 
+def test_checkpoint_recompute_rebuilds_the_persistent_pairs():
+    # the sequential layer and the one-step parallel rebuild from its z agree
+    x, W = _problem(3, 11, 16, 2, 32, sigma=0.3)
+    z, K, V = O.rt_layer(x, W, 2)
+    Kr, Vr = O.recompute_kv(z, W)
+    np.testing.assert_allclose(Kr, K, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(Vr, V, rtol=1e-13, atol=1e-14)
+    # and a persistent pair depends on its own position's output only
+    z2 = z.copy(); z2[:, 5] += 1.0
+    K2, _ = O.recompute_kv(z2, W)
+    assert np.array_equal(np.delete(K2, 5, axis=1), np.delete(Kr, 5, axis=1))
+
+
 def test_backward_matches_finite_differences():
     B, N, d, H, d_ff = 2, 4, 8, 2, 16
     x, W = _problem(B, N, d, H, d_ff, sigma=0.5)
