@@ -41,8 +41,12 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
     if not force and up_to_date():
         return LIB
+    # a per-process temporary, atomically renamed: concurrent builders (one
+    # process per GPU) never write the same file, and readers see either the
+    # old or the new library, whole
+    tmp = f"{LIB}.tmp{os.getpid()}"
     cmd = [nvcc_path(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "--shared",
-           "-Xcompiler", "-fPIC", "-I", INCLUDE, "-o", LIB + ".tmp",
+           "-Xcompiler", "-fPIC", "-I", INCLUDE, "-o", tmp,
            *sorted(glob.glob(os.path.join(CSRC, "*.cu")))]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -50,8 +54,10 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         cmd[1:1] = extra
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
+        if os.path.exists(tmp):
+            os.remove(tmp)
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     if verbose:
         sys.stdout.write(r.stdout + r.stderr)
     return LIB
