@@ -36,15 +36,11 @@ WORKLOADS = {
 }
 METRIC = "RT-layer prefill tokens/s (B=512,N=2048,d=1024 bf16); % of roofline"
 
-# DRAM traffic per launch from an ncu capture, keyed by (kernel class, workload,
-# hash of the CUDA sources at capture time). Reported as null once the sources
-# change. Filled from the ncu summaries under profiles/.
-NCU_TRAFFIC: dict = {
-    # W_2 GEMM, one launch at the headline's per-step shape (M = 512, N = 1024,
-    # K = 4096), ncu with cache flush: dram__bytes_read.sum 14,720,768 +
-    # dram__bytes_write.sum 0 (profiles/gemm_w2_B512_d1024_dff4096.md).
-    ("gemm_w2", "headline", "0679cf11600c"): 14720768,
-}
+# DRAM traffic per launch from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch), keyed by (kernel class, workload, hash
+# of the CUDA sources at capture time); reported as null once the sources
+# change.
+NCU_TRAFFIC: dict = {}
 
 
 def src_hash() -> str:
@@ -66,6 +62,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ablation", action="store_true", help="skip the naive-schedule ablation")
+    ap.add_argument("--ablation-steps", type=int, default=1)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--decode", action="store_true",
                     help="time the autoregressive decode step (B sequences, one new position against a cache)")
@@ -75,12 +73,14 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="sequence-length sweep, blocked vs naive (B=32 d=1024 H=16x64 d_ff=4096)")
     ap.add_argument("--sweep-n", default="512,1024,2048,4096,8192,16384")
-    ap.add_argument("--profile-case", choices=["step", "fold", "fwd"],
+    ap.add_argument("--profile-case", choices=["step", "fold", "fwd", "naive"],
                     help="run one small case for an ncu capture and exit: 'step' = one host-loop forward at "
                          "B=512 N=64 d=1024 (the per-step GEMM shapes of the headline); 'fold' = one block fold "
-                         "of --lb keys into --lb queries at B=64 H=16 (position-major, larger than L2); "
-                         "'fwd' = one graph-driver forward at the headline widths with N = --lb")
+                         "of --lb keys into --lb queries at B=--pB H=16 (position-major); 'fwd' = one "
+                         "graph-driver forward at the headline widths with N = --lb; 'naive' = one host-loop "
+                         "naive-schedule forward at B=--pB, N=--lb, d=1024 H=16x64 d_ff=4096")
     ap.add_argument("--lb", type=int, default=1024)
+    ap.add_argument("--pB", type=int, default=64, help="batch of the 'fold' and 'naive' profile cases")
     return ap.parse_args()
 
 
@@ -189,8 +189,9 @@ def algorithmic_work(cfg: dict, schedule: str = "blocked") -> dict:
         "gemm_w2": ("tensor", 2.0 * B * dff * d * N),
         "gemm_wkv": ("tensor", 2.0 * B * d * 2 * d * N),
         "inv_rms": ("hbm", 2.0 * B * N * d + 4.0 * B * N),
-        # q, k~, v~ of position t (bf16), (m, l, o) of query t read (fp32), a_t written (bf16)
-        "attend": ("hbm", float(N) * B * (6 * d + 4 * d + 8 * H + 2 * d)),
+        # blocked: only position 1 is finalised by this class (every later
+        # position by the last fold into it): q, k~, v~ read, a_1 written (bf16)
+        "attend": ("hbm", float(B) * (6 * d + 2 * d)),
     }
     if schedule == "naive":
         # query t reads the t-1 persistent pairs (k, v bf16) plus its own q, k~, v~; writes a_t
@@ -230,6 +231,7 @@ def fold_level_work(cfg: dict) -> dict:
 # the oracle as the CPU baseline / reference arm
 # --------------------------------------------------------------------------
 def blas_threads() -> int:
+    """Threads of numpy's BLAS pool: the threads the oracle's matrix products use."""
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
@@ -238,38 +240,48 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def time_oracle(cfg: dict, n_seq: int, n_pos: int, seed: int) -> tuple[float, float]:
-    """Runs the fp64 oracle (naive definition) on n_seq sequences x n_pos
-    positions of the workload; returns (tokens/s, seconds)."""
+# The oracle's timed sample: a subset of the workload's sequences at the full
+# sequence length. Sequences are independent, so the whole batch costs the
+# sample's time x B / ORACLE_SEQS and tokens/s is the sample's own.
+ORACLE_SEQS = 1
+
+
+def time_oracle(cfg: dict, n_seq: int, seed: int) -> tuple[float, float]:
+    """Runs the fp64 oracle (naive definition) on the first n_seq sequences of
+    the workload at its full length N; returns (tokens/s, seconds)."""
     import rtinputs
     from oracle import rt_oracle
     W = rtinputs.weights(seed, cfg["d"], cfg["d_ff"], dtype="bf16")
-    x = rtinputs.x_batch(seed, range(n_seq), n_pos, cfg["d"], dtype="bf16")
+    x = rtinputs.x_batch(seed, range(n_seq), cfg["N"], cfg["d"], dtype="bf16")
     t0 = time.perf_counter()
     rt_oracle.rt_layer(x, W, cfg["H"])
     dt = time.perf_counter() - t0
-    return n_seq * n_pos / dt, dt
+    return n_seq * cfg["N"] / dt, dt
+
+
+def oracle_sample_text(cfg: dict, secs: float | None = None) -> str:
+    t = f"; {secs:.1f} s" if secs is not None else ""
+    return (f"{ORACLE_SEQS} of the {cfg['B']} sequences at the full N={cfg['N']} (fp64 numpy oracle, naive "
+            f"schedule{t}); the whole batch takes B/{ORACLE_SEQS} times as long (sequences are independent)")
 
 
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
     cfg = WORKLOADS[args.workload]
-    n_seq, n_pos = 1, 256
     for _ in range(args.warmup):
-        time_oracle(cfg, n_seq, n_pos, args.seed)
-    secs = [time_oracle(cfg, n_seq, n_pos, args.seed)[1] for _ in range(args.steps)]
-    ms = 1e3 * sum(secs) / len(secs)
-    value = n_seq * n_pos / (ms / 1e3)
-    cores = blas_threads()
-    sample = (f"{n_seq} sequence x first {n_pos} positions of the {args.workload} workload per step "
-              f"(fp64 numpy oracle, naive schedule)")
+        time_oracle(cfg, ORACLE_SEQS, args.seed)
+    secs = [time_oracle(cfg, ORACLE_SEQS, args.seed)[1] for _ in range(args.steps)]
+    sample_s = sum(secs) / len(secs)
+    value = ORACLE_SEQS * cfg["N"] / sample_s
+    ms = 1e3 * sample_s * cfg["B"] / ORACLE_SEQS      # one step of the whole workload
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(args, cfg, world),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "nproc": os.cpu_count(),
+                         "kind": "oracle", "sample": oracle_sample_text(cfg, sample_s)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -403,8 +415,14 @@ def run_profile_case(args, R, torch, rtinputs):
              for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16").items()}
         x = torch.randn((B, N, d), device=dev, dtype=torch.bfloat16)
         z, _, _ = R.layer_forward(x, W, H, driver="stream" if args.profile_case == "step" else "graph")
+    elif args.profile_case == "naive":
+        B, N, d, H, dff = args.pB, args.lb, 1024, 16, 4096
+        W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
+             for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16").items()}
+        x = torch.randn((B, N, d), device=dev, dtype=torch.bfloat16)
+        z, _, _ = R.layer_forward(x, W, H, schedule="naive", driver="stream")
     else:
-        LB, B, H, dh = args.lb, 64, 16, 64
+        LB, B, H, dh = args.lb, args.pB, 16, 64
         d = H * dh
         Q = torch.randn((2 * LB, B, 3 * d), device=dev, dtype=torch.bfloat16)
         Kc = torch.randn((2 * LB, B, d), device=dev, dtype=torch.bfloat16)
@@ -499,6 +517,9 @@ def main():
     classes = R.layer_forward_timed(x, W, H, (z, K, V), ws, schedule=args.schedule)
     work = algorithmic_work(cfg, args.schedule)
     peaks = measured_peaks()
+    # a kernel timed at full clocks is compared with the burst GEMM peak; if
+    # the power cap throttled the timed region, with the sustained one
+    tensor_key = "bf16_tflops_sustained" if "sw_power_cap" in clocks.get("reasons", []) else "bf16_tflops"
     kernels, fold_levels = {}, {}
     lvl_work = fold_level_work(cfg) if args.schedule == "blocked" else {}
     for name, (kms, launches) in classes.items():
@@ -513,7 +534,7 @@ def main():
         per_launch = amount / launches
         if kind == "tensor":
             ach = per_launch / (per_launch_ms / 1e3) / 1e12
-            peak, unit = peaks["bf16_tflops_sustained"], "TFLOP/s"
+            peak, unit = peaks[tensor_key], "TFLOP/s"
         else:
             ach = per_launch / (per_launch_ms / 1e3) / 1e9
             peak, unit = peaks["hbm_gbs"], "GB/s"
@@ -525,12 +546,37 @@ def main():
     tr = NCU_TRAFFIC.get((dom, args.workload, src_hash()))
     roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
                 "unit": kd["unit"], "frac": kd["frac"], "traffic": tr,
-                "peak_source": f"{peaks['source']} ({'bf16_tflops_sustained' if kd['bound'] == 'tensor' else 'hbm_gbs'})"}
+                "peak_source": f"{peaks['source']} ({tensor_key if kd['bound'] == 'tensor' else 'hbm_gbs'})"}
     # whole-step roofline: the method's FLOPs against the bf16 tensor peak
     total_flops = sum(a for k, a in work.values() if k == "tensor") + 4.0 * Bsz * d * N * (N + 1) / 2
     step_roof = {"flops_per_step": total_flops,
                  "achieved_tflops": total_flops / (ms_step / 1e3) / 1e12,
-                 "frac_of_bf16_peak": total_flops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]}
+                 "frac_of_bf16_peak": total_flops / (ms_step / 1e3) / 1e12 / peaks[tensor_key],
+                 "peak_source": f"{peaks['source']} ({tensor_key})"}
+
+    # the naive Theta(N^2)-traffic schedule on the same inputs (the ablation)
+    ablation = None
+    if args.schedule == "blocked" and not args.no_ablation:
+        wsn = R.alloc_workspace(R.workspace_bytes(Bsz, N, d, H, dff, torch.bfloat16, "naive"), dev)
+        outn = (torch.empty_like(z), torch.empty_like(K), torch.empty_like(V))
+        R.layer_forward(x, W, H, schedule="naive", driver=args.driver, out=outn, workspace=wsn)
+        torch.cuda.synchronize()
+        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0.record(stream)
+        for _ in range(args.ablation_steps):
+            R.layer_forward(x, W, H, schedule="naive", driver=args.driver, out=outn, workspace=wsn)
+        n1.record(stream)
+        torch.cuda.synchronize()
+        if R.sync_status(wsn) != 0:
+            raise RuntimeError("device error in the naive-schedule ablation")
+        n_ms = n0.elapsed_time(n1) / args.ablation_steps
+        kv_bytes = 4.0 * Bsz * d * N * (N - 1) / 2
+        ablation = {"schedule": "naive", "ms_per_step": n_ms, "value": Bsz * N / (n_ms / 1e3),
+                    "unit": "tokens/s", "steps": args.ablation_steps,
+                    "kv_bytes_per_step": kv_bytes, "kv_GBps": kv_bytes / (n_ms / 1e3) / 1e9,
+                    "blocked_speedup": n_ms / ms_step}
+        del wsn, outn
+        torch.cuda.empty_cache()
 
     # end to end through the public C ABI with HOST buffers (copies in the timed region)
     e2e = None
@@ -566,11 +612,9 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_seq, n_pos = 2, N
-        val, secs = time_oracle(cfg, n_seq, n_pos, args.seed)
-        cpu = {"value": val, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{n_seq} sequences x all {n_pos} positions of the workload "
-                         f"(fp64 numpy oracle, naive schedule; {secs:.1f} s)"}
+        val, secs = time_oracle(cfg, ORACLE_SEQS, args.seed)
+        cpu = {"value": val, "unit": "tokens/s", "cores": blas_threads(), "nproc": os.cpu_count(),
+               "kind": "oracle", "sample": oracle_sample_text(cfg, secs)}
 
     if world > 1:
         dist.barrier()
@@ -583,6 +627,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(args, cfg, world),
         "roofline": roofline, "step_roofline": step_roof, "kernels": kernels, "fold_levels": fold_levels,
+        "ablation": ablation,
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": R.launch_count(Bsz, N, d, H, dff, torch.bfloat16, args.schedule) * args.steps,
         "clocks": clocks,

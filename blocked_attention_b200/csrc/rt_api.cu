@@ -26,17 +26,17 @@
 #include "rt_common.cuh"
 #include "rt_fold_tc.cuh"
 #include "rt_gemm_tc.cuh"
+#include "rt_host.h"
 #include "rt_simt.cuh"
 
 namespace rt {
 
-static constexpr float kEps = 1e-6f;
 typedef __nv_bfloat16 bf16;
 
 // The CUDA error behind the calling thread's last RT_ERR_CUDA status
 // (rt_last_cuda_error reads it).
 static thread_local int g_last_cuda_error = 0;
-static inline int cuda_failure(cudaError_t e) {
+int cuda_failure(cudaError_t e) {
   g_last_cuda_error = (int)e;
   return RT_ERR_CUDA;
 }
@@ -104,7 +104,21 @@ static std::mutex g_io_mu;   // the transfer streams and events are per device
 static int io_chunk_len(int N) { return (N + kIoXChunks - 1) / kIoXChunks; }
 static std::mutex g_dev_mu;
 static DevState g_dev[64];
+static std::mutex g_encode_mu;
 static PFN_encodeTiled_t g_encode = nullptr;
+
+bool load_tensor_map_encoder() {
+  std::lock_guard<std::mutex> lk(g_encode_mu);
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return false;
+  g_encode = reinterpret_cast<PFN_encodeTiled_t>(fn);
+  return true;
+}
 
 template <int BN, int EPI>
 static cudaError_t set_tc_attr() {
@@ -132,15 +146,7 @@ static int device_setup(DevState** out) {
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return RT_ERR_DEVICE;
     if (major != 10) return RT_ERR_DEVICE;
     if (cudaDeviceGetAttribute(&ds.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return RT_ERR_DEVICE;
-    if (!g_encode) {
-      void* fn = nullptr;
-      cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
-              cudaSuccess ||
-          q != cudaDriverEntryPointSuccess || !fn)
-        return RT_ERR_CUDA;
-      g_encode = reinterpret_cast<PFN_encodeTiled_t>(fn);
-    }
+    if (!load_tensor_map_encoder()) return RT_ERR_CUDA;
     RT_CK(set_tc_attrs_epi<EPI_PLAIN>());
     RT_CK(set_tc_attrs_epi<EPI_PROJ>());
     RT_CK(set_tc_attrs_epi<EPI_WO>());
@@ -161,9 +167,7 @@ static int device_setup(DevState** out) {
   return RT_OK;
 }
 
-// 2-D bf16 tensor map over a row-major [rows][inner] matrix; box 64 x box_rows,
-// 128-byte swizzle (the K-major UMMA operand layout). Out-of-range rows read 0.
-static bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
   if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * 2};
@@ -187,8 +191,7 @@ static bool make_tmap_pm(CUtensorMap* m, const void* base, uint64_t stride, uint
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Output-tile width: the widest tile that still gives >= 120 tiles.
-static int choose_bn(int M, int N) {
+int choose_bn(int M, int N) {
   const long ntm = (M + 127) / 128;
   for (int bn : {256, 128, 64})
     if (ntm * ((N + bn - 1) / bn) >= 120) return bn;
@@ -983,8 +986,9 @@ extern "C" int rt_embed_forward(const int32_t* ids, const void* E, int B, int N,
 
 extern "C" int rt_block_fold(const void* Q, int q_stride, const void* K, const void* V, int kv_stride, float* m,
                              float* l, float* o, int B, int H, int d_h, int q0, int nq, int k0, int nk, int dtype,
-                             void* stream) {
-  if (!Q || !K || !V || !m || !l || !o) return RT_ERR_INVALID_ARG;
+                             void* err_dev, void* stream) {
+  if (!Q || !K || !V || !m || !l || !o || !err_dev) return RT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(err_dev) & 3u) != 0) return RT_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || nq <= 0 || nk <= 0 || q0 < 0 || k0 < 0) return RT_ERR_INVALID_ARG;
   if (q_stride < H * d_h || kv_stride < H * d_h || (long)B * H > 65535) return RT_ERR_INVALID_ARG;
   if (dtype == RT_BF16 && d_h != 64) return RT_ERR_UNSUPPORTED;
@@ -999,7 +1003,7 @@ extern "C" int rt_block_fold(const void* Q, int q_stride, const void* K, const v
   if (dtype == RT_BF16)
     e = launch_fold<bf16>(static_cast<const bf16*>(Q), q_stride, static_cast<const bf16*>(K),
                           static_cast<const bf16*>(V), kv_stride, m, l, o, nullptr, B, H, d_h, q0, nq, k0, nk, sc2, 0,
-                          0, true, st, nullptr, 128, ds->sms);
+                          0, true, st, static_cast<unsigned*>(err_dev), 128, ds->sms);
   else if (dtype == RT_F32)
     e = launch_fold<float>(static_cast<const float*>(Q), q_stride, static_cast<const float*>(K),
                            static_cast<const float*>(V), kv_stride, m, l, o, nullptr, B, H, d_h, q0, nq, k0, nk, sc2, 0,
@@ -1104,8 +1108,9 @@ extern "C" int rt_layer_decode_step(const void* x_t, const void* W_q, const void
 }
 
 extern "C" int rt_project_qkv(const void* x, const void* W_qkv, int B, int N, int d, int dtype, void* QKV,
-                              void* scratch, void* stream) {
-  if (!x || !W_qkv || !QKV || !scratch || B <= 0 || N <= 0 || d <= 0) return RT_ERR_INVALID_ARG;
+                              void* scratch, void* err_dev, void* stream) {
+  if (!x || !W_qkv || !QKV || !scratch || !err_dev || B <= 0 || N <= 0 || d <= 0) return RT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(err_dev) & 3u) != 0) return RT_ERR_INVALID_ARG;
   if (dtype == RT_BF16 && d % 64 != 0) return RT_ERR_UNSUPPORTED;
   const size_t rows = (size_t)B * N;
   if (rows > (1u << 30)) return RT_ERR_UNSUPPORTED;
@@ -1123,7 +1128,7 @@ extern "C" int rt_project_qkv(const void* x, const void* W_qkv, int B, int N, in
     EpiParams ep;
     std::memset(&ep, 0, sizeof(ep));
     ep.B = B; ep.Nseq = N; ep.xc = N; ep.d = d; ep.inv_rms = inv; ep.qkv = static_cast<bf16*>(QKV);
-    RT_CK(launch_tc<EPI_PROJ>(bn, ta, tb, (int)rows, 3 * d, d, ep, nullptr, ds->sms, st));
+    RT_CK(launch_tc<EPI_PROJ>(bn, ta, tb, (int)rows, 3 * d, d, ep, static_cast<unsigned*>(err_dev), ds->sms, st));
   } else if (dtype == RT_F32) {
     if ((rows + 63) / 64 > 65535) return RT_ERR_UNSUPPORTED;
     float* xr = static_cast<float*>(scratch);
@@ -1139,8 +1144,10 @@ extern "C" int rt_project_qkv(const void* x, const void* W_qkv, int B, int N, in
   return RT_OK;
 }
 
-extern "C" int rt_gemm_bf16(const void* A, const void* W, float* C, int M, int Nout, int Kd, void* stream) {
-  if (!A || !W || !C || M <= 0 || Nout <= 0 || Kd <= 0) return RT_ERR_INVALID_ARG;
+extern "C" int rt_gemm_bf16(const void* A, const void* W, float* C, int M, int Nout, int Kd, void* err_dev,
+                            void* stream) {
+  if (!A || !W || !C || !err_dev || M <= 0 || Nout <= 0 || Kd <= 0) return RT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(err_dev) & 3u) != 0) return RT_ERR_INVALID_ARG;
   if (Kd % 64 != 0) return RT_ERR_UNSUPPORTED;
   DevState* ds = nullptr;
   int rc = device_setup(&ds);
@@ -1151,7 +1158,8 @@ extern "C" int rt_gemm_bf16(const void* A, const void* W, float* C, int M, int N
   EpiParams ep;
   std::memset(&ep, 0, sizeof(ep));
   ep.c32 = C;
-  RT_CK(launch_tc<EPI_PLAIN>(bn, ta, tb, M, Nout, Kd, ep, nullptr, ds->sms, static_cast<cudaStream_t>(stream)));
+  RT_CK(launch_tc<EPI_PLAIN>(bn, ta, tb, M, Nout, Kd, ep, static_cast<unsigned*>(err_dev), ds->sms,
+                             static_cast<cudaStream_t>(stream)));
   return RT_OK;
 }
 

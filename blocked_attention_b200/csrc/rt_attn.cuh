@@ -20,6 +20,7 @@
 #pragma once
 
 #include "rt_common.cuh"
+#include "rt_rownorm.cuh"
 
 namespace rt {
 
@@ -810,25 +811,6 @@ __global__ void __launch_bounds__(128)
 // ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------
-// inv[r] = 1 / sqrt(mean(x_r^2) + eps), one warp per row of width d
-template <class T>
-__global__ void __launch_bounds__(256) k_row_inv_rms(const T* __restrict__ x, float* __restrict__ inv,
-                                                     size_t rows, int d, float eps) {
-  pdl_launch_dependents();
-  pdl_wait();
-  const size_t r = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  const T* xr = x + r * d;
-  float s = 0.f;
-  for (int e = lane; e < d; e += 32) {
-    const float v = to_f(xr[e]);
-    s += v * v;
-  }
-  s = warp_sum(s);
-  if (lane == 0) inv[r] = rsqrtf(s / (float)d + eps);
-}
-
 // out[r] = in[r] / rms(in[r]) (fp32 path)
 __global__ void __launch_bounds__(256) k_rmsnorm_f32(const float* __restrict__ in, float* __restrict__ out,
                                                      size_t rows, int d, float eps) {

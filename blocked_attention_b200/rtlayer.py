@@ -29,7 +29,8 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_erro
            "rt_layer_sync_status", "rt_layer_host_workspace_bytes", "rt_layer_forward_host",
            "rt_embed_forward", "rt_block_fold", "rt_project_qkv", "rt_gemm_bf16",
            "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc",
-           "rt_selftest_wait_timeout", "rt_layer_decode_workspace_bytes", "rt_layer_decode_step")
+           "rt_selftest_wait_timeout", "rt_layer_decode_workspace_bytes", "rt_layer_decode_step",
+           "rt_project_qkv_noalloc_status")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma")
@@ -82,11 +83,11 @@ def lib() -> ctypes.CDLL:
     L.rt_embed_forward.restype = i
     L.rt_embed_forward.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp]
     L.rt_block_fold.restype = i
-    L.rt_block_fold.argtypes = [vp, i, vp, vp, i, fp, fp, fp] + [i] * 7 + [i, vp]
+    L.rt_block_fold.argtypes = [vp, i, vp, vp, i, fp, fp, fp] + [i] * 7 + [i, vp, vp]
     L.rt_project_qkv.restype = i
-    L.rt_project_qkv.argtypes = [vp, vp, i, i, i, i, vp, vp, vp]
+    L.rt_project_qkv.argtypes = [vp, vp, i, i, i, i, vp, vp, vp, vp]
     L.rt_gemm_bf16.restype = i
-    L.rt_gemm_bf16.argtypes = [vp, vp, fp, i, i, i, vp]
+    L.rt_gemm_bf16.argtypes = [vp, vp, fp, i, i, i, vp, vp]
     L.rt_layer_launch_count.restype = ctypes.c_long
     L.rt_layer_launch_count.argtypes = [i] * 7
     L.rt_layer_forward_timed.restype = i
@@ -94,6 +95,8 @@ def lib() -> ctypes.CDLL:
                                                                          ctypes.POINTER(ctypes.c_int), i]
     L.rt_project_qkv_noalloc.restype = i
     L.rt_project_qkv_noalloc.argtypes = [vp, vp, i, i, i, vp, vp]
+    L.rt_project_qkv_noalloc_status.restype = i
+    L.rt_project_qkv_noalloc_status.argtypes = [vp]
     L.rt_selftest_wait_timeout.restype = i
     L.rt_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp, vp]
     L.rt_layer_decode_workspace_bytes.restype = sz
@@ -272,22 +275,44 @@ def embed_forward(ids: torch.Tensor, E: torch.Tensor, workspace: torch.Tensor | 
     return x
 
 
-def block_fold(Q, K, V, m, l, o, H: int, d_h: int, q0: int, nq: int, k0: int, nk: int, stream=None):
+def _err_word(err, device):
+    """The caller's device error word, or a fresh zeroed one (owned here)."""
+    if err is not None:
+        return err, False
+    return torch.zeros(256, dtype=torch.uint8, device=device), True
+
+
+def _finish(fn: str, err, owned: bool, stream):
+    """When the binding owns the error word, read it (synchronises the stream)
+    and raise on a device-side error; otherwise the caller reads it with
+    sync_status(err)."""
+    if owned:
+        _check(fn, sync_status(err, stream))
+
+
+def block_fold(Q, K, V, m, l, o, H: int, d_h: int, q0: int, nq: int, k0: int, nk: int, err=None, stream=None):
     """rt_block_fold: Q [n_pos, B, q_stride], K/V [n_pos, B, kv_stride];
-    m, l [n_pos, B, H] and o [n_pos, B, H*d_h] fp32 updated in place."""
+    m, l [n_pos, B, H] and o [n_pos, B, H*d_h] fp32 updated in place.
+    err: device error word (None: a private one, checked before returning)."""
     B = Q.shape[1]
+    err, owned = _err_word(err, Q.device)
     rc = lib().rt_block_fold(_ptr(Q), Q.shape[2], _ptr(K), _ptr(V), K.shape[2], _fptr(m), _fptr(l), _fptr(o),
-                             B, H, d_h, q0, nq, k0, nk, _dtype_code(Q.dtype), _stream(stream))
+                             B, H, d_h, q0, nq, k0, nk, _dtype_code(Q.dtype), _ptr(err), _stream(stream))
     _check("rt_block_fold", rc)
+    _finish("rt_block_fold", err, owned, stream)
 
 
-def project_qkv(x: torch.Tensor, W_qkv: torch.Tensor, stream=None):
+def project_qkv(x: torch.Tensor, W_qkv: torch.Tensor, err=None, stream=None):
+    """rt_project_qkv: x [B, N, d] -> QKV position-major [N, B, 3d].
+    err: device error word (None: a private one, checked before returning)."""
     B, N, d = x.shape
     qkv = torch.empty((N, B, 3 * d), dtype=x.dtype, device=x.device)
     scratch = torch.empty(B * N * (1 if x.dtype == torch.bfloat16 else d), dtype=torch.float32, device=x.device)
+    err, owned = _err_word(err, x.device)
     rc = lib().rt_project_qkv(_ptr(x), _ptr(W_qkv), B, N, d, _dtype_code(x.dtype), _ptr(qkv), _ptr(scratch),
-                              _stream(stream))
+                              _ptr(err), _stream(stream))
     _check("rt_project_qkv", rc)
+    _finish("rt_project_qkv", err, owned, stream)
     return qkv
 
 
@@ -300,10 +325,20 @@ def project_qkv_noalloc(x: torch.Tensor, W_qkv: torch.Tensor, out: torch.Tensor,
     return out
 
 
-def gemm_bf16(A: torch.Tensor, W: torch.Tensor, stream=None):
+def project_qkv_noalloc_status(stream=None) -> int:
+    """rt_project_qkv_noalloc_status: synchronises the stream, then reads and
+    clears the library's error word of the allocation-free projection."""
+    return int(lib().rt_project_qkv_noalloc_status(_stream(stream)))
+
+
+def gemm_bf16(A: torch.Tensor, W: torch.Tensor, err=None, stream=None):
+    """rt_gemm_bf16: C = A W^T (bf16 operands, fp32 C).
+    err: device error word (None: a private one, checked before returning)."""
     M, Kd = A.shape
     Nout = W.shape[0]
     C = torch.empty((M, Nout), dtype=torch.float32, device=A.device)
-    rc = lib().rt_gemm_bf16(_ptr(A), _ptr(W), _fptr(C), M, Nout, Kd, _stream(stream))
+    err, owned = _err_word(err, A.device)
+    rc = lib().rt_gemm_bf16(_ptr(A), _ptr(W), _fptr(C), M, Nout, Kd, _ptr(err), _stream(stream))
     _check("rt_gemm_bf16", rc)
+    _finish("rt_gemm_bf16", err, owned, stream)
     return C

@@ -162,6 +162,9 @@ int rt_layer_decode_step(const void* x_t_dev,
                          void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /* Token-embedding front end of a layer stack: x[b][n][:] = E[ids[b][n]][:].
+ * Paper §6.1 stacks layers by feeding each layer's outputs z to the next
+ * layer as its inputs; the first layer's inputs are the embedded tokens, so a
+ * stack is this call followed by one rt_layer_forward per layer.
  * ids_dev int32 [B][N], each in [0, vocab) (out-of-range ids produce a zero
  * row and set the error word of `workspace_dev` if it is not NULL);
  * E_dev [vocab][d]; x_dev [B][N][d]; storage type `dtype`. */
@@ -181,24 +184,34 @@ int rt_embed_forward(const int32_t* ids_dev, const void* E_dev, int B, int N,
  * Folds keys [k0, k0 + nk) into queries [q0, q0 + nq) (0-based positions),
  * updating (m, l, o) in place. m is stored in log2 units scaled by
  * log2(e)/sqrt(d_h) (m = -inf marks an empty accumulator).
- * RT_BF16 needs d_h = 64; nk that is a multiple of 16 uses the tensor-core
- * kernel, other nk the warp kernel. */
+ * RT_BF16 needs d_h = 64. Kernel by key count nk: <= 8 the small-block
+ * kernel; multiples of 128 the tcgen05 kernels; other multiples of 16 the
+ * mma.sync kernel; anything else the warp kernel.
+ * err_dev: error word of the tcgen05 kernels' bounded waits, as in
+ * rt_project_qkv (read with rt_layer_sync_status). */
 int rt_block_fold(const void* Q_dev, int q_stride, const void* K_dev,
                   const void* V_dev, int kv_stride, float* m_dev, float* l_dev,
                   float* o_dev, int B, int H, int d_h, int q0, int nq, int k0,
-                  int nk, int dtype, void* stream);
+                  int nk, int dtype, void* err_dev, void* stream);
 
 /* Batched projection of all B*N positions (queries depend only on x):
  *   QKV_dev[n][b][0:d] = W_q rms(x[b][n]), [d:2d] = W_k rms(..), [2d:3d] = W_v rms(..)
  * position-major [N][B][3d]. W_qkv_dev is [3d][d] (W_q; W_k; W_v stacked).
- * scratch_dev: >= B*N*4 bytes (RT_BF16) or B*N*d*4 bytes (RT_F32). */
+ * scratch_dev: >= B*N*4 bytes (RT_BF16) or B*N*d*4 bytes (RT_F32).
+ * err_dev: a 4-byte-aligned device word (e.g. the first bytes of a layer
+ * workspace) into which the tensor-core kernel's bounded waits record a
+ * timeout; it is only ever OR-ed into, so it accumulates over calls until
+ * rt_layer_sync_status(err_dev, stream) reads and clears it. NULL is
+ * RT_ERR_INVALID_ARG. */
 int rt_project_qkv(const void* x_dev, const void* W_qkv_dev, int B, int N, int d,
-                   int dtype, void* QKV_dev, void* scratch_dev, void* stream);
+                   int dtype, void* QKV_dev, void* scratch_dev, void* err_dev,
+                   void* stream);
 
 /* Dense product C[M][Nout] = A[M][Kd] * W[Nout][Kd]^T in bf16 with fp32
- * accumulation on the tcgen05 tensor-core kernel; C is fp32. Kd % 64 == 0. */
+ * accumulation on the tcgen05 tensor-core kernel; C is fp32. Kd % 64 == 0.
+ * err_dev: error word as in rt_project_qkv (read with rt_layer_sync_status). */
 int rt_gemm_bf16(const void* A_dev, const void* W_dev, float* C_dev, int M,
-                 int Nout, int Kd, void* stream);
+                 int Nout, int Kd, void* err_dev, void* stream);
 
 /* rt_project_qkv for RT_BF16 storage without caller scratch: the per-row
  * 1/rms values live in a fixed array inside the library, so the call needs no
@@ -215,9 +228,19 @@ int rt_gemm_bf16(const void* A_dev, const void* W_dev, float* C_dev, int M,
  *     before any stream capture.
  *   - All calls share the array and overwrite the rows they use before
  *     reading them; calls that overlap on the GPU race on it.
+ *   - A bounded wait of the tensor-core kernel that runs out is recorded in a
+ *     device word that also lives inside the library (one per GPU, shared by
+ *     every call); rt_project_qkv_noalloc_status reads and clears it.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
 int rt_project_qkv_noalloc(const void* x_dev, const void* W_qkv_dev, int B, int N,
                            int d, void* QKV_dev, void* stream);
+
+/* Status of the rt_project_qkv_noalloc calls enqueued so far on the current
+ * device: synchronises `stream`, then reads and clears the library's error
+ * word. RT_OK, RT_ERR_TIMEOUT (a bounded wait ran out; that call's QKV_dev
+ * is incomplete), RT_ERR_CUDA, or RT_ERR_DEVICE if no call has set up the
+ * device yet. Allocates nothing. */
+int rt_project_qkv_noalloc_status(void* stream);
 
 /* ---------------------------------------------------------------------------
  * Measurement

@@ -129,7 +129,33 @@ def test_no_device_is_reported_not_faked(L):
     assert _fwd(L, 1 << 40) == R.RT_ERR_DEVICE
     assert L.rt_gemm_bf16(ctypes.c_void_p(1 << 40), ctypes.c_void_p(1 << 40),
                           ctypes.cast(ctypes.c_void_p(1 << 40), ctypes.POINTER(ctypes.c_float)),
-                          128, 128, 64, None) == R.RT_ERR_DEVICE
+                          128, 128, 64, ctypes.c_void_p(1 << 40), None) == R.RT_ERR_DEVICE
+    # the allocation-free projection sets up the device first, too
+    assert L.rt_project_qkv_noalloc(ctypes.c_void_p(1 << 40), ctypes.c_void_p(1 << 40), 2, 8, 64,
+                                    ctypes.c_void_p(1 << 40), None) == R.RT_ERR_DEVICE
+    assert L.rt_project_qkv_noalloc_status(None) == R.RT_ERR_DEVICE
+
+
+def test_component_entry_points_require_an_error_word(L):
+    # the tensor-core kernels behind these calls record bounded-wait timeouts
+    # in err_dev; a call without one (or with a misaligned one) is refused
+    # before anything is enqueued
+    p = ctypes.c_void_p(1 << 40)
+    fp = ctypes.cast(p, ctypes.POINTER(ctypes.c_float))
+    for err, want in ((None, R.RT_ERR_INVALID_ARG), (ctypes.c_void_p((1 << 40) + 2), R.RT_ERR_INVALID_ARG)):
+        assert L.rt_gemm_bf16(p, p, fp, 128, 128, 64, err, None) == want
+        assert L.rt_project_qkv(p, p, 2, 8, 64, R.RT_BF16, p, p, err, None) == want
+        assert L.rt_block_fold(p, 192, p, p, 64, fp, fp, fp, 2, 1, 64, 4, 4, 0, 4, R.RT_BF16, err, None) == want
+
+
+def test_noalloc_validation_happens_before_any_launch(L):
+    p = ctypes.c_void_p(1 << 40)
+    call = L.rt_project_qkv_noalloc
+    assert call(None, p, 2, 8, 64, p, None) == R.RT_ERR_INVALID_ARG
+    assert call(p, p, 0, 8, 64, p, None) == R.RT_ERR_INVALID_ARG
+    assert call(p, p, 2, 8, 96, p, None) == R.RT_ERR_UNSUPPORTED       # d % 64 != 0
+    # B*N = 2^20 + 1 rows: beyond the fixed scratch array
+    assert call(p, p, 1025, 1024, 64, p, None) == R.RT_ERR_WORKSPACE
 
 
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):

@@ -41,6 +41,24 @@ def test_headline_config_sampled_sequences():
     assert max(errs) <= TOL["bf16"], errs
 
 
+def test_long_sequence_exercises_blocks_of_2048_keys():
+    # N = 4096 at the headline widths: the fold of step 2048 folds a block of
+    # 2048 keys into 2048 queries (and step 1024 one of 1024), the block sizes
+    # of the sequence-length sweep's longer runs. One sequence is checked
+    # against the oracle; the other is filled on the device.
+    from blocked_attention_b200 import rtlayer as R
+    B, N, d, H, dff = 2, 4096, 1024, 16, 4096
+    seqs = [1]
+    W = rtinputs.weights(0, d, dff, dtype="bf16")
+    x, xs = _filled_batch(B, N, d, seqs, 0)
+    z, K, V = R.layer_forward(x, {k: to_device(v, "bf16") for k, v in W.items()}, H, driver="graph")
+    torch.cuda.synchronize()
+    zg, Kg, Vg = to_np(z[seqs]), to_np(K[:, seqs]).transpose(1, 0, 2), to_np(V[:, seqs]).transpose(1, 0, 2)
+    zr, Kr, Vr = O.rt_layer(xs, W, H)
+    errs = rel_err(zg, zr), rel_err(Kg, Kr), rel_err(Vg, Vr)
+    assert max(errs) <= TOL["bf16"], errs
+
+
 def test_stack_config_sampled_sequence():
     # 6 layers, d=1280 (20 heads of 64), d_ff=5120, vocab 32000, B=64, N=2048
     from blocked_attention_b200 import rtlayer as R

@@ -80,6 +80,7 @@ def test_batched_projection_matches_oracle(rt, dtype, B, N, d):
     ("bf16", 256, 256, False), ("bf16", 1024, 700, True), ("bf16", 256, 129, False),
     ("bf16", 128, 77, False), ("bf16", 128, 128, True), ("bf16", 512, 300, True), ("bf16", 384, 1, False),
     ("bf16", 40, 6, False),                                                      # generic warp kernel
+    ("bf16", 2048, 300, False), ("bf16", 4096, 129, True),                     # the blocks of N >= 4096
     ("f32", 3, 4, False), ("f32", 16, 16, True), ("f32", 64, 33, False)])
 def test_block_fold_matches_oracle(rt, dtype, nk, nq, init_empty):
     B, H, dh = 3, 2, 64 if dtype == "bf16" else 32
@@ -217,6 +218,7 @@ def test_host_buffer_entry_point(rt):
     zr, Kr, Vr = O.rt_layer(x, W, H)
     assert rel_err(to_np(out[0]), zr) < TOL["bf16"]
     assert rel_err(to_np(out[1]).transpose(1, 0, 2), Kr) < TOL["bf16"]
+    assert rel_err(to_np(out[2]).transpose(1, 0, 2), Vr) < TOL["bf16"]
 
 
 @pytest.mark.parametrize("pinned", [True, False])
@@ -269,6 +271,7 @@ def test_stack_of_layers_with_embedding(rt):
     assert rel_err(to_np(x), zr) < TOL["bf16"]
     for (K, V), (Kr, Vr) in zip(kv, kvr):
         assert rel_err(to_np(K).transpose(1, 0, 2), Kr) < TOL["bf16"]
+        assert rel_err(to_np(V).transpose(1, 0, 2), Vr) < TOL["bf16"]
 
 
 def test_embedding_out_of_range_id_is_reported(rt):
@@ -288,3 +291,19 @@ def test_bounded_wait_reports_timeout_and_context_stays_usable(rt):
     assert rt.sync_status(ws) == 0                       # the word was cleared
     # the context is still usable: a normal forward runs and passes parity
     _check_layer(rt, 2, 20, 128, 2, 256, "bf16")
+
+
+def test_component_entry_point_reports_through_its_error_word(rt):
+    # the error word a component entry point's tensor-core kernel records into
+    # is the one rt_layer_sync_status reads: a timeout recorded there (by the
+    # bounded-wait self-test) surfaces, is cleared, and a GEMM enqueued on the
+    # same word afterwards completes with the word still clear
+    err = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    rt.selftest_wait_timeout(1_000_000, err)
+    assert rt.sync_status(err) == rt.RT_ERR_TIMEOUT
+    rng = np.random.default_rng(5)
+    A = rtinputs.to_grid(rng.standard_normal((300, 256)), "bf16")
+    W = rtinputs.to_grid(rng.standard_normal((192, 256)), "bf16")
+    C = rt.gemm_bf16(to_device(A, "bf16"), to_device(W, "bf16"), err=err)
+    assert rt.sync_status(err) == 0
+    assert rel_err(to_np(C), A @ W.T) < 1e-5

@@ -469,3 +469,24 @@ def test_stack_chains_layers():
         x, K, V = O.rt_layer(x, W, H)
         np.testing.assert_array_equal(K, kv[i][0])
     np.testing.assert_array_equal(x, zs)
+
+
+def test_embedding_lookup_row_by_row():
+    # The stack's front end is a table lookup (the token id selects a row of
+    # the embedding table; RT paper §6.1 feeds the embedded tokens to the
+    # first layer). Hand-chosen ids -- the first and last rows of the table,
+    # repeats, and a [B, N] layout -- are checked one by one against a loop
+    # that copies the row by explicit index, so a transposed table, an
+    # off-by-one id or a flattened batch axis fails.
+    vocab, d = 7, 5
+    E = np.arange(vocab * d, dtype=np.float64).reshape(vocab, d) * 0.5 - 3.0
+    ids = np.array([[0, 6, 3], [6, 6, 0]], dtype=np.int32)
+    x = O.embed(ids, E)
+    assert x.shape == (2, 3, d)
+    for b in range(ids.shape[0]):
+        for n in range(ids.shape[1]):
+            row = [E[int(ids[b, n]), e] for e in range(d)]
+            assert list(x[b, n]) == row
+    # row 0 of the table is -3.0, -2.5, ... and row vocab-1 ends at the last entry
+    assert list(x[0, 0]) == [-3.0, -2.5, -2.0, -1.5, -1.0]
+    assert x[0, 1, -1] == E.flat[-1] == (vocab * d - 1) * 0.5 - 3.0
