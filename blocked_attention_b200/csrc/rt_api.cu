@@ -28,6 +28,7 @@
 #include "rt_gemm_tc.cuh"
 #include "rt_host.h"
 #include "rt_simt.cuh"
+#include "rt_steps.cuh"
 
 namespace rt {
 
@@ -77,6 +78,22 @@ template <typename... KArgs, typename... Args>
 static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                               Args&&... args) {
   return launch_pdl_cluster(kern, grid, block, smem, st, 1, std::forward<Args>(args)...);
+}
+
+// The persistent step kernel: one CTA per SM, all co-resident (cooperative
+// launch), since its tasks wait on flags set by other CTAs.
+static cudaError_t launch_steps(const StepsParams& sp, int sms, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)sms);
+  cfg.blockDim = dim3(StepsCfg::THREADS);
+  cfg.dynamicSmemBytes = StepsCfg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_steps, sp);
 }
 
 // ---------------------------------------------------------------------------
@@ -153,9 +170,11 @@ static int device_setup(DevState** out) {
     RT_CK(set_tc_attrs_epi<EPI_W1>());
     RT_CK(set_tc_attrs_epi<EPI_W2>());
     RT_CK(set_tc_attrs_epi<EPI_WKV>());
+    RT_CK(set_tc_attrs_epi<EPI_RKV>());
     RT_CK(cudaFuncSetAttribute(k_fold_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FoldTcCfg::SMEM_BYTES));
     RT_CK(cudaFuncSetAttribute(k_fold_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)FoldTc2Cfg::SMEM_BYTES));
+    RT_CK(cudaFuncSetAttribute(k_steps, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StepsCfg::SMEM_BYTES));
     RT_CK(cudaStreamCreateWithFlags(&ds.capture, cudaStreamNonBlocking));
     RT_CK(cudaStreamCreateWithFlags(&ds.h2d, cudaStreamNonBlocking));
     RT_CK(cudaStreamCreateWithFlags(&ds.d2h, cudaStreamNonBlocking));
@@ -277,12 +296,45 @@ static int validate(const Shape& s) {
   return RT_OK;
 }
 
+// Tile widths and splits of the persistent step kernel (bf16, blocked
+// schedule). ok = false: a shape the step kernel does not take (flag ranges
+// beyond its per-lane polling); the step loop then launches one GEMM kernel
+// per phase and one fold per step.
+struct StepsPlan {
+  bool ok;
+  GemmPhase g[4];
+  int nrb, G;
+};
+static StepsPlan plan_steps(const Shape& s) {
+  StepsPlan sp;
+  std::memset(&sp, 0, sizeof(sp));
+  if (s.dtype != RT_BF16 || s.schedule != RT_SCHED_BLOCKED) return sp;
+  const int d = s.d, dff = s.d_ff;
+  auto phase = [](int N, int K, int BN, int S) { return GemmPhase{N, K, BN, S, N / BN}; };
+  // W_o: 64-wide tiles (short tasks on the critical path); W_1, W_2, W_kv:
+  // 128-wide where the width allows (fewer operand bytes per output); the
+  // 4096-deep W_2 reduction split so that every task streams about 1024 of K.
+  sp.g[PH_WO] = phase(d, d, 64, 1);
+  sp.g[PH_W1] = phase(dff, d, dff % 128 == 0 ? 128 : 64, 1);
+  const int s2 = std::max(1, std::min(4, (dff / 64) / 8));
+  sp.g[PH_W2] = phase(d, dff, d % 128 == 0 ? 128 : 64, s2);
+  sp.g[PH_WKV] = phase(2 * d, d, 128, 1);
+  sp.nrb = (s.B + 127) / 128;
+  sp.G = (std::min(s.B, 128) + kFoldSeqs - 1) / kFoldSeqs;
+  // flag ranges one producer lane set polls (3 per lane) and the flag stride
+  const int w2_split_tiles = (dff / s2 + sp.g[PH_W1].BN - 1) / sp.g[PH_W1].BN + 1;
+  sp.ok = s.H * sp.G <= 96 && sp.g[PH_WO].tiles <= 96 && w2_split_tiles <= 96 && sp.g[PH_W2].tiles <= 96 &&
+          sp.g[PH_W1].tiles <= kFlagStride && sp.g[PH_WKV].tiles <= kFlagStride && s.H * sp.G <= kFlagStride;
+  return sp;
+}
+
 struct Plan {
   Shape s;
   size_t esz;
   size_t off_err, off_qkv, off_m, off_l, off_o, off_inv, off_xr, off_wqkv, off_a, off_u32, off_u16, off_ru,
-      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, total;
+      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, off_flags, off_w2cnt, off_w2part, total;
   TileCfg t_wo, t_w1, t_w2, t_wkv;
+  StepsPlan sp;
 };
 
 static Plan make_plan(const Shape& s) {
@@ -316,6 +368,13 @@ static Plan make_plan(const Shape& s) {
   if (s.dtype == RT_F32) P.off_rz = take(B * d * 4);
   P.off_ssq_u = take((d / 32 + 1) * B * 4);
   P.off_ssq_z = take((d / 32 + 1) * B * 4);
+  P.sp = plan_steps(s);
+  if (P.sp.ok) {
+    const GemmPhase& g2 = P.sp.g[PH_W2];
+    P.off_flags = take((size_t)PH_COUNT * P.sp.nrb * kFlagStride * 4);
+    P.off_w2cnt = take((size_t)P.sp.nrb * g2.tiles * 4);
+    P.off_w2part = take((size_t)P.sp.nrb * g2.tiles * g2.S * g2.BN * StepsCfg::BM * 4);
+  }
   if (s.dtype == RT_BF16) {
     P.t_wo = choose_tiles(s.B, s.d, s.d, kLayerSplitK);
     P.t_w1 = choose_tiles(s.B, s.d_ff, s.d, kLayerSplitK);
@@ -343,7 +402,7 @@ struct HostIo {
 // per-kernel-class event timing (stream driver only)
 // ---------------------------------------------------------------------------
 enum KernelClass {
-  KC_INV_RMS = 0, KC_PROJ, KC_ATTEND, KC_WO, KC_W1, KC_W2, KC_WKV, KC_FOLD_WARP, KC_FOLD_MMA, KC_NORM,
+  KC_INV_RMS = 0, KC_PROJ, KC_ATTEND, KC_WO, KC_W1, KC_W2, KC_WKV, KC_FOLD_WARP, KC_FOLD_MMA, KC_STEPS,
   KC_FOLD_LEVEL0 = 16,   // + log2(block size): per-level fold timing
   KC_COUNT = 32
 };
@@ -596,7 +655,67 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
     TimedScope ts(T, KC_ATTEND, st);
     RT_CK((launch_attend<bf16, 2>(P, qkv, K, V, m, l, o, a16, 0, sc2, st)));
   }
-  for (int j = 0; j < N; ++j) {
+  if (P.sp.ok) {
+    // persistent step kernel: one launch per segment of steps whose folds
+    // have at most 8 keys; the segment's last fold (>= 16 keys) follows it
+    StepsParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    const bf16* A_of[4] = {a16, u16, h16, z16};
+    const void* W_of[4] = {X.Wo, X.W1, X.W2, wqkv + (size_t)d * d};
+    for (int ph = 0; ph < 4; ++ph) {
+      const GemmPhase& g = P.sp.g[ph];
+      sp.g[ph] = g;
+      if (!make_tmap(&sp.tA[ph], A_of[ph], g.K, B, 128) || !make_tmap(&sp.tB[ph], W_of[ph], g.K, g.N, g.BN))
+        return RT_ERR_INVALID_ARG;
+    }
+    sp.ep = ep;
+    sp.ssq_u = ssq_u;
+    sp.ssq_z = ssq_z;
+    sp.qkv = qkv;
+    sp.m = m;
+    sp.l = l;
+    sp.o = o;
+    sp.a16 = a16;
+    sp.flags = reinterpret_cast<unsigned*>(ws + P.off_flags);
+    sp.w2cnt = reinterpret_cast<unsigned*>(ws + P.off_w2cnt);
+    sp.w2part = reinterpret_cast<float*>(ws + P.off_w2part);
+    sp.err = err;
+    sp.sc2 = sc2;
+    sp.H = H;
+    sp.nrb = P.sp.nrb;
+    sp.G = P.sp.G;
+    RT_CK(cudaMemsetAsync(sp.flags, 0, (size_t)PH_COUNT * P.sp.nrb * kFlagStride * 4, st));
+    RT_CK(cudaMemsetAsync(sp.w2cnt, 0, (size_t)P.sp.nrb * P.sp.g[PH_W2].tiles * 4, st));
+    for (int j = 0; j < N;) {
+      // steps j .. j1-1; the last one reveals position t = j1, whose fold has
+      // >= 16 keys (or which is the last position)
+      int j1 = j + 1;
+      while (j1 < N && lowbit(j1) < 16) ++j1;
+      {
+        const int rc = project_through(std::min(N - 1, 2 * (j1 - 1) + 1));
+        if (rc != RT_OK) return rc;
+      }
+      sp.j0 = j;
+      sp.j1 = j1;
+      {
+        TimedScope ts(T, KC_STEPS, st);
+        RT_CK(launch_steps(sp, ds.sms, st));
+      }
+      const int t = j1;
+      if (t < N) {
+        const int lb = lowbit(t), nq = std::min(lb, N - t);
+        TimedScope ts(T, KC_FOLD_LEVEL0 + log2_int(lb), st);
+        RT_CK(launch_fold<bf16>(qkv, 3 * d, K, V, d, m, l, o, a16, B, H, 64, t, nq, t - lb, lb, sc2,
+                                t == lb ? 1 : 0, 1, true, st, err, kFoldTcMinBlock, ds.sms));
+      }
+      if (io && (j1 - out_done >= out_every || j1 == N)) {
+        const int rc = ship_outputs(j1);
+        if (rc != RT_OK) return rc;
+      }
+      j = j1;
+    }
+  }
+  for (int j = 0; j < N && !P.sp.ok; ++j) {
     ep.j = j;
     {
       const int rc = project_through(std::min(N - 1, 2 * j + 1));
@@ -745,6 +864,16 @@ static long launch_count(const Shape& s) {
   if (s.schedule == RT_SCHED_BLOCKED)
     for (int t = 1; t <= s.N; ++t) folds += (std::min(lowbit(t), s.N - t) > 0) ? 1 : 0;
   if (s.dtype == RT_BF16) {
+    if (s.schedule == RT_SCHED_BLOCKED && plan_steps(s).ok) {
+      // finalise(position 1) + one step kernel per segment + the folds of
+      // >= 16 keys that end segments (each finalises the next position)
+      long segments = 0, big = 0;
+      for (int t = 1; t <= s.N; ++t) {
+        if (t == s.N || lowbit(t) >= 16) ++segments;
+        if (t < s.N && lowbit(t) >= 16) ++big;
+      }
+      return 2 + 1 + segments + big;
+    }
     // blocked: finalise(position 1) + 4 GEMMs per step + folds (each finalises the next position)
     if (s.schedule == RT_SCHED_BLOCKED) return 2 + 1 + 4l * s.N + folds;
     return 2 + 5l * s.N;
@@ -1141,6 +1270,53 @@ extern "C" int rt_project_qkv(const void* x, const void* W_qkv, int B, int N, in
   } else {
     return RT_ERR_INVALID_ARG;
   }
+  return RT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// activation-checkpoint recompute of the persistent pairs (RT paper §6.1)
+// ---------------------------------------------------------------------------
+static size_t recompute_ws_bytes(int B, int N, int d) {
+  return align_up(256, 256) + align_up((size_t)B * N * 4, 256) + align_up((size_t)2 * d * d * 2, 256);
+}
+
+extern "C" size_t rt_layer_recompute_workspace_bytes(int B, int N, int d) {
+  if (B <= 0 || N <= 0 || d <= 0 || d % 64 != 0 || (long)B * N > (1l << 30)) return 0;
+  return recompute_ws_bytes(B, N, d);
+}
+
+extern "C" int rt_layer_recompute_kv(const void* z, const void* W_k, const void* W_v, int B, int N, int d, void* K,
+                                     void* V, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!z || !W_k || !W_v || !K || !V || B <= 0 || N <= 0 || d <= 0) return RT_ERR_INVALID_ARG;
+  if (d % 64 != 0 || (long)B * N > (1l << 30)) return RT_ERR_UNSUPPORTED;
+  const void* all[5] = {z, W_k, W_v, K, V};
+  for (const void* p : all)
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return RT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < recompute_ws_bytes(B, N, d) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return RT_ERR_WORKSPACE;
+  DevState* ds = nullptr;
+  int rc = device_setup(&ds);
+  if (rc != RT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  unsigned* err = reinterpret_cast<unsigned*>(ws);
+  float* inv = reinterpret_cast<float*>(ws + 256);
+  bf16* wkv = reinterpret_cast<bf16*>(ws + 256 + align_up((size_t)B * N * 4, 256));
+  const size_t rows = (size_t)B * N, dd = (size_t)d * d * 2;
+  RT_CK(cudaMemsetAsync(err, 0, sizeof(unsigned), st));
+  RT_CK(cudaMemcpyAsync(wkv, W_k, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wkv) + dd, W_v, dd, cudaMemcpyDeviceToDevice, st));
+  k_row_inv_rms<bf16><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const bf16*>(z), inv, rows, d, kEps);
+  RT_CK(cudaGetLastError());
+  const int bn = choose_bn((int)rows, 2 * d);
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, z, d, rows, 128) || !make_tmap(&tb, wkv, d, 2 * d, bn)) return RT_ERR_INVALID_ARG;
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.B = B; ep.Nseq = N; ep.xc = N; ep.d = d; ep.inv_rms = inv;
+  ep.Kout = static_cast<bf16*>(K); ep.Vout = static_cast<bf16*>(V);
+  RT_CK(launch_tc<EPI_RKV>(bn, ta, tb, (int)rows, 2 * d, d, ep, err, ds->sms, st));
   return RT_OK;
 }
 

@@ -25,6 +25,9 @@
 //   W1    : h = GELU((u W_1^T) / rms(u))            (rms from the WO partials)
 //   W2    : z_t = u + h W_2^T -> output z, bf16 copy, per-tile sum of z^2
 //   WKV   : [k_t | v_t] = (z_t [W_k; W_v]^T) / rms(z_t) -> position-major K, V
+//   RKV   : the same for all B*N rows of a stored output z [B][N][d] at once
+//           (activation-checkpoint recompute of the persistent pairs, paper
+//           §6.1), scaled by 1/rms(z) of the row -> position-major K, V
 // The identity rms(v) W^T = (v W^T) / r(v), r(v) = sqrt(mean v^2 + eps), moves
 // each RMSNorm into the next GEMM's epilogue; it changes only rounding.
 #pragma once
@@ -33,7 +36,7 @@
 
 namespace rt {
 
-enum EpiKind { EPI_PLAIN = 0, EPI_PROJ = 1, EPI_WO = 2, EPI_W1 = 3, EPI_W2 = 4, EPI_WKV = 5 };
+enum EpiKind { EPI_PLAIN = 0, EPI_PROJ = 1, EPI_WO = 2, EPI_W1 = 3, EPI_W2 = 4, EPI_WKV = 5, EPI_RKV = 6 };
 
 struct EpiParams {
   int B, Nseq, d, d_ff, j;   // batch, sequence length, width, MLP width, position (0-based)
@@ -154,7 +157,7 @@ struct GemmCfg {
 };
 
 // Pulls into L1 the residual operand the epilogue will read for `ncols`
-// columns of a row from col0 on (WO: x, bf16; W2: u, fp32).
+// columns of a row from col0 on (WO: the layer input x, bf16).
 template <int EPI>
 __device__ __forceinline__ void epilogue_prefetch(const EpiParams& p, int row, int col0, int N, int ncols) {
   for (int c = 0; c < ncols; c += 32) {
@@ -163,8 +166,6 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& p, int row, i
     if constexpr (EPI == EPI_WO) {
       const int ch = p.j / p.xc;
       ptr = p.x + (((size_t)ch * p.B + row) * p.xc + (p.j - ch * p.xc)) * p.d + col0 + c;
-    } else if constexpr (EPI == EPI_W2) {
-      ptr = p.u32 + (size_t)row * p.d + col0 + c;
     }
     if (ptr) asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));   // one 128-byte line per chunk
   }
@@ -212,10 +213,11 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
     store_bf16x32(p.h16 + (size_t)row * p.d_ff + col0, v);
   } else if constexpr (EPI == EPI_W2) {
     const int b = row;
+    // u was written by other CTAs (L2-coherent loads: no stale L1 lines)
     const float4* u4 = reinterpret_cast<const float4*>(p.u32 + (size_t)b * p.d + col0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float4 w = u4[i];
+      float4 w = __ldcg(u4 + i);
       v[4 * i] += w.x; v[4 * i + 1] += w.y; v[4 * i + 2] += w.z; v[4 * i + 3] += w.w;
     }
 #pragma unroll
@@ -227,6 +229,14 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] *= row_scale;
     const size_t base = ((size_t)p.j * p.B + b) * p.d;
+    if (col0 < p.d) store_bf16x32(p.Kout + base + col0, v);
+    else store_bf16x32(p.Vout + base + (col0 - p.d), v);
+  } else if constexpr (EPI == EPI_RKV) {
+    // row = b * Nseq + n of z [B][N][d]; outputs position-major [N][B][d]
+    const int b = row / p.Nseq, n = row - b * p.Nseq;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= row_scale;
+    const size_t base = ((size_t)n * p.B + b) * p.d;
     if (col0 < p.d) store_bf16x32(p.Kout + base + col0, v);
     else store_bf16x32(p.Vout + base + (col0 - p.d), v);
   }
@@ -254,11 +264,11 @@ __device__ __forceinline__ void tmem_ld_acc(uint32_t taddr, bool two, float (&v)
 
 template <int EPI>
 __device__ __forceinline__ float row_scale_for(const EpiParams& p, int row) {
-  if constexpr (EPI == EPI_PROJ) {
+  if constexpr (EPI == EPI_PROJ || EPI == EPI_RKV) {
     return p.inv_rms[row];
   } else if constexpr (EPI == EPI_W1 || EPI == EPI_WKV) {
     float s = 0.f;
-    for (int t = 0; t < p.ssq_tiles; ++t) s += p.ssq_in[(size_t)t * p.B + row];
+    for (int t = 0; t < p.ssq_tiles; ++t) s += __ldcg(p.ssq_in + (size_t)t * p.B + row);
     return rsqrtf(s / (float)p.d + p.eps);
   } else {
     return 1.f;

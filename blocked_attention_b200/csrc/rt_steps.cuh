@@ -1,0 +1,689 @@
+// rt_steps.cuh -- the layer's N-step loop as one persistent kernel per segment
+// of steps (sm_100a: tcgen05 tensor cores, TMEM accumulators, TMA operands).
+//
+// Source: "Recurrent Transformer" paper page (www.lshu.cn/news/403416):
+//   paper §2.2  : the per-position chain u = x_t + W_o a_t ->
+//                 z_t = u + W_2 GELU(W_1 rms(u)) -> (k_t, v_t) = [W_k; W_v] rms(z_t);
+//   notes §4.2  : when (k_t, v_t) is revealed, keys (t - lowbit(t), t] are
+//                 folded into the online-softmax statistics of queries
+//                 (t, t + lowbit(t)];
+//   paper §6.2  : O(N) medium-sized launches dominate a per-step loop.
+//
+// A segment is a run of steps j0 .. j1-1 (0-based positions; step j reveals
+// the pair of position t = j + 1) whose folds all have at most 8 keys, except
+// the fold of its last step, which has >= 16 keys (run afterwards by the block
+// fold kernels) or does not exist (t = N). Sequences never interact, so the
+// batch is cut into row blocks of 128 sequences (the GEMM tile height) and
+// every dependency below stays inside one row block: the row blocks run as
+// independent chains that overlap on the machine.
+//
+// Work of one step, per row block rb ("tasks"):
+//   WO   : u = x_j + a W_o^T (+ per-tile sums of u^2)        tiles of BN_o columns
+//   W1   : h = GELU((u W_1^T) / r(u))                         tiles of BN_1
+//   W2   : z_j = u + h W_2^T (+ sums of z^2)                  tiles of BN_2, K split S ways
+//   WKV  : [k_j | v_j] = (z_j [W_k; W_v]^T) / r(z_j)          tiles of BN_kv
+//   FOLD : keys (t - lb, t] into queries (t, t + lb] for one head and 32
+//          sequences; the first query (t + 1) is finalised: its temporary pair
+//          is merged and a_{t+1} = o / l is written (the A operand of the next
+//          step's WO).                                        lb <= 8, not on the segment's last step
+// Tasks are numbered in the order (step, phase, row block, tile, split) and
+// dealt round-robin to the grid's CTAs (one per SM, co-resident: cooperative
+// launch); each CTA processes its tasks in that order. Every task waits only
+// for tasks earlier in the order, so the earliest unfinished task can always
+// run: no deadlock.
+//
+// Dependencies are per-tile flags in global memory holding "last step done +
+// 1" (monotonic within a forward; cleared before it). A task's TMA producer
+// polls the flags of the tiles its A operand is made of, K slice by K slice,
+// so a GEMM starts on the first columns of its input while the producing
+// phase is still finishing them. Every thread that reads data another CTA
+// wrote first observes (acquire) the flag that covers it, then fences, and
+// reads that data through L2 (ld.global.cg or TMA), never from a possibly
+// stale L1 line; every writer fences its stores (also to the async proxy,
+// since the next phase reads them with TMA) before it releases its flag. The W_2 split-K partial
+// tiles go to global slots; an arrival counter elects the last split, which
+// sums the slots in split order (deterministic) and runs the epilogue.
+//
+// Every poll and every mbarrier wait is bounded by %globaltimer. A poll that
+// runs out records RT_DEVERR_TIMEOUT and returns; once the error word is set,
+// every later poll returns at once and the tasks run on with whatever data is
+// there, so the kernel always ends. An mbarrier wait that runs out (or sees
+// the error word set) stops its warp's task loop; before the CTA frees its
+// tensor memory, the MMA warps wait (bounded) for their issued MMAs and the
+// producer for its copies in flight.
+#pragma once
+
+#include "rt_common.cuh"
+#include "rt_gemm_tc.cuh"
+
+namespace rt {
+
+enum StepPhase { PH_WO = 0, PH_W1 = 1, PH_W2 = 2, PH_WKV = 3, PH_FOLD = 4, PH_COUNT = 5 };
+
+constexpr int kFlagStride = 256;   // flags per (phase, row block): tiles, or heads x fold groups
+constexpr int kFoldSeqs = 32;      // sequences per fold task
+constexpr int kSmallFoldMax = 8;   // largest block folded inside the step kernel
+
+struct StepsCfg {
+  static constexpr int BM = 128, BK = 64, KSUB = 2, BN_MAX = 128;
+  static constexpr uint32_t A_SUB = BM * BK * 2;            // one 64-wide K slice of A (16 KB)
+  static constexpr uint32_t B_SUB = BN_MAX * BK * 2;        // slot for one K slice of B (16 KB)
+  static constexpr uint32_t A_BYTES = A_SUB * KSUB, B_BYTES = B_SUB * KSUB;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 3;
+  static constexpr uint32_t TMEM_COLS = 512;                // 2 tiles in flight x 2 issuers x 128
+  static constexpr int THREADS = 224;                       // producer, 2 MMA issuers, 4 epilogue warps
+  static constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+};
+
+// One GEMM phase: C[B][N] = A[B][K] W[N][K]^T, output tiles of 128 x BN, the
+// reduction split S ways (S > 1 only for W2).
+struct GemmPhase {
+  int N, K, BN, S, tiles;
+};
+
+struct StepsParams {
+  CUtensorMap tA[4], tB[4];    // per GEMM phase: A (activations, box 64 x 128) and W (box 64 x BN)
+  GemmPhase g[4];
+  EpiParams ep;                // shapes, x, u32, u16, h16, zout, z16, Kout, Vout, xc, eps
+  float* ssq_u;                // [d / BN_o][B]
+  float* ssq_z;                // [d / BN_2][B]
+  const __nv_bfloat16* qkv;    // [N][B][3d]
+  float* m;                    // [N][B][H]
+  float* l;
+  float* o;                    // [N][B][d]
+  __nv_bfloat16* a16;          // [B][d]
+  unsigned* flags;             // [PH_COUNT][nrb][kFlagStride]
+  unsigned* w2cnt;             // [nrb][tiles of W2]: split arrivals, cumulative over the forward
+  float* w2part;               // [nrb][tiles][S][BN_2][128] fp32 partial tiles
+  unsigned* err;
+  float sc2;                   // log2(e) / sqrt(d_h)
+  int H, nrb, G;               // heads, row blocks, fold groups of 32 sequences per row block
+  int j0, j1;                  // the segment's steps
+};
+
+// ---------------------------------------------------------------------------
+// synchronisation helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ unsigned ld_volatile_u32(const unsigned* p) {
+  return *reinterpret_cast<const volatile unsigned*>(p);
+}
+// generic-proxy global stores <-> async-proxy (TMA) global accesses
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// barrier of the four epilogue warps (named barrier 1, 128 threads)
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Bounded poll until *f >= target (acquire). Returns at once once the error
+// word is set; a poll that runs out sets RT_DEVERR_TIMEOUT. Either way the
+// caller proceeds.
+__device__ __noinline__ void poll_ge(const unsigned* f, unsigned target, unsigned* err) {
+  if (ld_acquire_u32(f) >= target) return;
+  const unsigned long long t0 = globaltimer();
+  for (unsigned it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_u32(f) >= target) return;
+    if ((it & 15u) == 0) {
+      if (ld_volatile_u32(err) != 0) return;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        set_error(err, RT_DEVERR_TIMEOUT);
+        return;
+      }
+    }
+  }
+}
+
+// mbarrier wait bounded by time and abandoned once the error word is set.
+__device__ __forceinline__ bool mbar_wait_g(uint64_t* bar, unsigned parity, unsigned* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (unsigned it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (ld_volatile_u32(err) != 0) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        set_error(err, RT_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// task enumeration (identical in every warp role of a CTA)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int phase_tasks(const StepsParams& P, int ph, int j) {
+  if (ph < 4) return P.nrb * P.g[ph].tiles * P.g[ph].S;
+  return (j + 1 < P.j1) ? P.nrb * P.H * P.G : 0;   // the segment's last fold runs elsewhere
+}
+
+// Calls f(phase, step, local index) for this CTA's tasks in order; stops when
+// f returns false.
+template <class F>
+__device__ __forceinline__ void for_my_tasks(const StepsParams& P, F&& f) {
+  const long G = gridDim.x, bid = blockIdx.x;
+  long base = 0;
+  for (int j = P.j0; j < P.j1; ++j) {
+    for (int ph = 0; ph < PH_COUNT; ++ph) {
+      const int n = phase_tasks(P, ph, j);
+      long first = (bid - base) % G;
+      if (first < 0) first += G;
+      for (long loc = first; loc < n; loc += G)
+        if (!f(ph, j, (int)loc)) return;
+      base += n;
+    }
+  }
+}
+
+struct GemmTask {
+  int rb, tile, split, sl0, sl1;   // row block, output tile, K split, 64-wide K slices [sl0, sl1)
+};
+__device__ __forceinline__ GemmTask decode_gemm(const GemmPhase& g, int loc) {
+  GemmTask t;
+  const int per_rb = g.tiles * g.S;
+  t.rb = loc / per_rb;
+  const int r = loc - t.rb * per_rb;
+  t.tile = r / g.S;
+  t.split = r - t.tile * g.S;
+  const int ksl = g.K / 64;
+  t.sl0 = t.split * ksl / g.S;
+  t.sl1 = (t.split + 1) * ksl / g.S;
+  return t;
+}
+
+__device__ __forceinline__ unsigned* flag_ptr(const StepsParams& P, int ph, int rb, int i) {
+  return P.flags + ((size_t)(ph * P.nrb + rb) * kFlagStride + i);
+}
+
+// The flags the A operand of a GEMM task depends on: K slice kk of phase ph
+// is made by flags [lo(kk), hi(kk)) of phase dep_phase(ph), complete once
+// they reach dep_target.
+__device__ __forceinline__ int dep_phase(int ph) { return ph == PH_WO ? PH_FOLD : ph - 1; }
+__device__ __forceinline__ void slice_flags(const StepsParams& P, int ph, int kk, int& lo, int& hi) {
+  if (ph == PH_WO) {   // a of head kk (d_h = 64): the fold groups of head kk
+    lo = kk * P.G;
+    hi = lo + P.G;
+  } else {
+    lo = kk * 64 / P.g[ph - 1].BN;
+    hi = lo + 1;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// small block fold (at most 8 keys), one task = one head of up to 32
+// sequences: every (sequence, query) unit is served by an octet of lanes
+// holding 8 of the head's 64 dims; each thread takes R units at a time and
+// issues all their loads before any use. The first query of the block is
+// finalised (temporary pair merged, a = o / l written, statistics not
+// stored); the others' (m, l, o) are updated in place, or written when the
+// fold is the first into them (init).
+// ---------------------------------------------------------------------------
+template <int NK, int R>
+__device__ __forceinline__ void fold_small_units(const StepsParams& P, int q0, int nq, int k0, int init, int h,
+                                                 int s0, int ns, int tid) {
+  const int B = P.ep.B, H = P.H, d = P.ep.d;
+  const int oct = tid >> 3, sl = tid & 7;
+  const unsigned omask = 0xFFu << ((tid & 31) & 24);
+  const int U = ns * nq;
+  const __nv_bfloat16* K = P.ep.Kout;
+  const __nv_bfloat16* V = P.ep.Vout;
+  for (int u0 = 0; u0 < U; u0 += 16 * R) {
+    uint4 qw[R], kw[R][NK], vw[R][NK], ktw[R], vtw[R];
+    float4 oa[R], ob[R];
+    float mo[R], lo[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int u = u0 + r * 16 + oct;
+      const bool act = u < U;
+      const int s = act ? u / nq : 0, qi = act ? u - s * nq : 0;
+      const int b = s0 + s;
+      const size_t row = (size_t)(q0 + qi) * B + b;
+      const __nv_bfloat16* qp = P.qkv + row * (size_t)(3 * d) + h * 64 + sl * 8;
+      qw[r] = ktw[r] = vtw[r] = make_uint4(0, 0, 0, 0);
+      oa[r] = ob[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      mo[r] = -INFINITY;
+      lo[r] = 0.f;
+#pragma unroll
+      for (int i = 0; i < NK; ++i) kw[r][i] = vw[r][i] = make_uint4(0, 0, 0, 0);
+      if (act) {
+        // k, v, m, l and o were written by other CTAs of this kernel: loads
+        // through L2 only (no stale L1 lines); q and the temporary pair come
+        // from the projection kernel
+        qw[r] = *reinterpret_cast<const uint4*>(qp);
+#pragma unroll
+        for (int i = 0; i < NK; ++i) {
+          const size_t kv = ((size_t)(k0 + i) * B + b) * d + h * 64 + sl * 8;
+          kw[r][i] = __ldcg(reinterpret_cast<const uint4*>(K + kv));
+          vw[r][i] = __ldcg(reinterpret_cast<const uint4*>(V + kv));
+        }
+        if (qi == 0) {   // the finalised query's temporary pair
+          ktw[r] = *reinterpret_cast<const uint4*>(qp + d);
+          vtw[r] = *reinterpret_cast<const uint4*>(qp + 2 * d);
+        }
+        if (!init) {
+          const float* op = P.o + row * (size_t)d + h * 64 + sl * 8;
+          mo[r] = __ldcg(P.m + row * H + h);
+          lo[r] = __ldcg(P.l + row * H + h);
+          oa[r] = __ldcg(reinterpret_cast<const float4*>(op));
+          ob[r] = __ldcg(reinterpret_cast<const float4*>(op) + 1);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int u = u0 + r * 16 + oct;
+      if (u >= U) continue;   // whole octets together; shuffles stay inside the octet
+      const int s = u / nq, qi = u - s * nq;
+      const int b = s0 + s;
+      const size_t row = (size_t)(q0 + qi) * B + b;
+      float q[8];
+      unpack_bf16x8(qw[r], q);
+      float sc[NK];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < NK; ++i) {
+        float kk[8];
+        unpack_bf16x8(kw[r][i], kk);
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
+        dot += __shfl_xor_sync(omask, dot, 1);
+        dot += __shfl_xor_sync(omask, dot, 2);
+        dot += __shfl_xor_sync(omask, dot, 4);
+        sc[i] = dot * P.sc2;
+        mx = fmaxf(mx, sc[i]);
+      }
+      float oo[8] = {oa[r].x, oa[r].y, oa[r].z, oa[r].w, ob[r].x, ob[r].y, ob[r].z, ob[r].w};
+      const float mn = fmaxf(mo[r], mx);
+      const float al = rescale(mo[r], mn);
+      float ln = lo[r] * al;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) oo[e] *= al;
+#pragma unroll
+      for (int i = 0; i < NK; ++i) {
+        const float p = exp2f(sc[i] - mn);
+        float vv[8];
+        unpack_bf16x8(vw[r][i], vv);
+        ln += p;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
+      }
+      if (qi == 0) {
+        float kt[8];
+        unpack_bf16x8(ktw[r], kt);
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dot += q[e] * kt[e];
+        dot += __shfl_xor_sync(omask, dot, 1);
+        dot += __shfl_xor_sync(omask, dot, 2);
+        dot += __shfl_xor_sync(omask, dot, 4);
+        const float st = dot * P.sc2;
+        const float m2 = fmaxf(mn, st);
+        const float a2 = rescale(mn, m2), pt = exp2f(st - m2);
+        const float inv = 1.f / (ln * a2 + pt);
+        float vt[8];
+        unpack_bf16x8(vtw[r], vt);
+        uint4 w;
+        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          __nv_bfloat162 v2 = __floats2bfloat162_rn((oo[2 * k] * a2 + pt * vt[2 * k]) * inv,
+                                                    (oo[2 * k + 1] * a2 + pt * vt[2 * k + 1]) * inv);
+          wp[k] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+        *reinterpret_cast<uint4*>(P.a16 + (size_t)b * d + h * 64 + sl * 8) = w;
+      } else {
+        float* op = P.o + row * (size_t)d + h * 64 + sl * 8;
+        if (sl == 0) {
+          P.m[row * H + h] = mn;
+          P.l[row * H + h] = ln;
+        }
+        reinterpret_cast<float4*>(op)[0] = make_float4(oo[0], oo[1], oo[2], oo[3]);
+        reinterpret_cast<float4*>(op)[1] = make_float4(oo[4], oo[5], oo[6], oo[7]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// epilogue of one GEMM tile (split == whole K): 32 columns at a time, the sum
+// of the two issuers' accumulators
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_ld_pair(uint32_t taddr, bool two, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld_32x32b_x32(taddr, r);
+  if (two) {
+    uint32_t r2[32];
+    tmem_ld_32x32b_x32(taddr + StepsCfg::BN_MAX, r2);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
+  } else {
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool row_ok, int col_base, int BN, int N,
+                                               uint32_t taddr, bool two, float rs) {
+  float ssq = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    float v[32];
+    tmem_ld_pair(taddr + c, two, v);
+    if (row_ok) ssq += epilogue_chunk<EPI>(e, row, col_base + c, N, v, rs);
+  }
+  return ssq;
+}
+
+// The epilogue-side dependencies of a task, polled in parallel by the 128
+// epilogue threads (thread i polls flag i of a contiguous range), then one
+// fence per polling thread and the epilogue barrier.
+__device__ __forceinline__ void epi_poll_range(const StepsParams& P, int ph, int rb, int lo, int hi, unsigned target,
+                                               int tid) {
+  bool polled = false;
+  for (int i = lo + tid; i < hi; i += 128) {
+    poll_ge(flag_ptr(P, ph, rb, i), target, P.err);
+    polled = true;
+  }
+  if (polled) __threadfence();
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_constant__ StepsParams P) {
+  using C = StepsCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;   // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* drain = tempty + 2;          // [2]: an issuer's MMAs have all completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
+  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 2); mbar_init(&tempty[a], 4); mbar_init(&drain[a], 1); }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0)
+    for (int i = 0; i < 4; ++i) { tma_prefetch_desc(&P.tA[i]); tma_prefetch_desc(&P.tB[i]); }
+  if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (lane 0 issues; the warp polls flags) ----------------
+    uint32_t it = 0;
+    bool ok = true;
+    for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
+      if (ph == PH_FOLD) return true;
+      const GemmPhase& g = P.g[ph];
+      const GemmTask T = decode_gemm(g, loc);
+      const bool deps = !(ph == PH_WO && j == P.j0);   // a of the first step comes from an earlier kernel
+      const int dph = dep_phase(ph);
+      const unsigned target = ph == PH_WO ? (unsigned)j : (unsigned)(j + 1);
+      int flo = 0, fhi = 0, tmp;
+      if (deps) {
+        slice_flags(P, ph, T.sl0, flo, tmp);
+        slice_flags(P, ph, T.sl1 - 1, tmp, fhi);
+      }
+      // flags flo + lane + 32 i, i < 3: readiness bits of this lane
+      unsigned rdy = 0;
+      const uint32_t bn_bytes = (uint32_t)g.BN * C::BK * 2;
+      for (int kb = T.sl0; kb < T.sl1; kb += C::KSUB, ++it) {
+        const int ns = min(C::KSUB, T.sl1 - kb);
+        const uint32_t s = it % C::STAGES, par = (it / C::STAGES) & 1u;
+        int w = 1;
+        if (lane == 0) w = mbar_wait_g(&empty[s], par ^ 1u, P.err) ? 1 : 0;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) { ok = false; return false; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], ns * (C::A_SUB + bn_bytes));
+          for (int q = 0; q < ns; ++q)
+            tma_load_2d(&P.tB[ph], &full[s], sB + s * C::B_BYTES + q * C::B_SUB, (kb + q) * C::BK, T.tile * g.BN);
+        }
+        if (deps) {
+          int lo, hi, t2;
+          slice_flags(P, ph, kb, lo, t2);
+          slice_flags(P, ph, kb + ns - 1, t2, hi);
+          for (int i = 0; i < 3; ++i) {
+            const int f = flo + lane + 32 * i;
+            if (f >= lo && f < hi && f < fhi && !(rdy >> i & 1u)) {
+              poll_ge(flag_ptr(P, dph, T.rb, f), target, P.err);
+              rdy |= 1u << i;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) fence_proxy_async_global();
+        }
+        if (lane == 0)
+          for (int q = 0; q < ns; ++q)
+            tma_load_2d(&P.tA[ph], &full[s], sA + s * C::A_BYTES + q * C::A_SUB, (kb + q) * C::BK, T.rb * C::BM);
+      }
+      return true;
+    });
+    if (!ok && lane == 0) {
+      // wait (bounded) for copies still in flight before the CTA can exit
+      const uint32_t first = it > (uint32_t)C::STAGES ? it - C::STAGES : 0u;
+      for (uint32_t i = first; i < it; ++i) mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1u, P.err);
+    }
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers: stage kb of a task goes to issuer kb % 2 ----------------
+    const int par = warp - 1;
+    if (lane == 0) {
+      uint32_t it = 0, local = 0;
+      for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
+        if (ph == PH_FOLD) return true;
+        const GemmPhase& g = P.g[ph];
+        const GemmTask T = decode_gemm(g, loc);
+        const int nst = (T.sl1 - T.sl0 + C::KSUB - 1) / C::KSUB;
+        const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
+        ++local;
+        if (!mbar_wait_g(&tempty[acc], aph ^ 1u, P.err)) return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (acc * 2 + par) * C::BN_MAX;
+        const uint32_t idesc = idesc_bf16_f32(C::BM, g.BN);
+        uint32_t accumulate = 0;
+        for (int kb = 0; kb < nst; ++kb, ++it) {
+          if ((kb & 1) != par) continue;
+          const uint32_t s = it % C::STAGES, sp = (it / C::STAGES) & 1u;
+          if (!mbar_wait_g(&full[s], sp, P.err)) return false;
+          tc_fence_after();
+          const uint8_t* a_st = sA + s * C::A_BYTES;
+          const uint8_t* b_st = sB + s * C::B_BYTES;
+          const int nmma = min(C::KSUB, T.sl1 - T.sl0 - kb * C::KSUB) * (C::BK / 16);
+#pragma unroll
+          for (int k = 0; k < C::KSUB * (C::BK / 16); ++k) {
+            if (k >= nmma) break;
+            const int q = k / (C::BK / 16), kk = k % (C::BK / 16);
+            tc_mma_f16(d_tmem, smem_desc_sw128(a_st + q * C::A_SUB + kk * 32),
+                       smem_desc_sw128(b_st + q * C::B_SUB + kk * 32), idesc, accumulate);
+            accumulate = 1u;
+          }
+          tc_commit(&empty[s]);
+        }
+        tc_commit(&tfull[acc]);   // with no stage of its own in this task it arrives at once
+        return true;
+      });
+      // every MMA this thread issued has completed before the CTA frees TMEM
+      tc_commit(&drain[par]);
+      mbar_wait(&drain[par], 0u, P.err);
+    }
+  } else {
+    // ---------------- epilogue warps: GEMM epilogues and small folds ----------------
+    const int tid = threadIdx.x - 96;   // 0..127
+    const int q = warp & 3;             // TMEM lanes 32q .. 32q + 31
+    const int lrow = q * 32 + lane;
+    uint32_t local = 0;
+    for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
+      if (ph == PH_FOLD) {
+        const int per_rb = P.H * P.G;
+        const int rb = loc / per_rb, r = loc - rb * per_rb;
+        const int h = r / P.G, gi = r - h * P.G;
+        const int t = j + 1, lb = lowbit(t), nq = min(lb, P.ep.Nseq - t);
+        // this head's k and v of step j (and, through them, everything before)
+        const int kt = (64 * h) / P.g[PH_WKV].BN, vt = (P.ep.d + 64 * h) / P.g[PH_WKV].BN;
+        if (tid == 0) { poll_ge(flag_ptr(P, PH_WKV, rb, kt), j + 1, P.err); __threadfence(); }
+        if (tid == 32) { poll_ge(flag_ptr(P, PH_WKV, rb, vt), j + 1, P.err); __threadfence(); }
+        epi_bar();
+        const int s0 = rb * 128 + gi * kFoldSeqs;
+        const int ns = min(kFoldSeqs, min(P.ep.B - s0, (rb + 1) * 128 - s0));
+        if (ns > 0 && nq > 0) {
+          const int init = t == lb ? 1 : 0;
+          switch (lb) {
+            case 1: fold_small_units<1, 4>(P, t, nq, t - 1, init, h, s0, ns, tid); break;
+            case 2: fold_small_units<2, 4>(P, t, nq, t - 2, init, h, s0, ns, tid); break;
+            case 4: fold_small_units<4, 3>(P, t, nq, t - 4, init, h, s0, ns, tid); break;
+            default: fold_small_units<8, 2>(P, t, nq, t - 8, init, h, s0, ns, tid); break;
+          }
+        }
+        fence_proxy_async_global();   // a is read by the next step's TMA loads
+        __threadfence();
+        epi_bar();
+        if (tid == 0) st_release_u32(flag_ptr(P, PH_FOLD, rb, h * P.G + gi), (unsigned)(j + 1));
+        return true;
+      }
+      const GemmPhase& g = P.g[ph];
+      const GemmTask T = decode_gemm(g, loc);
+      const int nst = (T.sl1 - T.sl0 + C::KSUB - 1) / C::KSUB;
+      const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
+      ++local;
+      const int row = T.rb * C::BM + lrow;
+      const bool row_ok = row < P.ep.B;
+      const int col_base = T.tile * g.BN;
+      // dependencies of what this epilogue reads or overwrites (see the file comment)
+      if (ph == PH_WO) {
+        if (j > P.j0) epi_poll_range(P, PH_FOLD, T.rb, 0, P.H * P.G, (unsigned)j, tid);
+      } else if (ph == PH_W1) {
+        epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);
+      } else if (ph == PH_W2) {
+        // the residual u (a split's epilogue reads only tensor memory; the
+        // last split polls these before it sums the partial tiles)
+        if (g.S == 1) epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);
+      } else {
+        epi_poll_range(P, PH_W2, T.rb, 0, P.g[PH_W2].tiles, (unsigned)(j + 1), tid);
+      }
+      epi_bar();
+      EpiParams e = P.ep;
+      e.j = j;
+      float rs = 1.f;
+      if (ph == PH_W1) {
+        e.ssq_in = P.ssq_u; e.ssq_tiles = P.g[PH_WO].tiles;
+        if (row_ok) rs = row_scale_for<EPI_W1>(e, row);
+      } else if (ph == PH_WKV) {
+        e.ssq_in = P.ssq_z; e.ssq_tiles = P.g[PH_W2].tiles;
+        if (row_ok) rs = row_scale_for<EPI_WKV>(e, row);
+      }
+      if (row_ok && ph == PH_WO) epilogue_prefetch<EPI_WO>(e, row, col_base, g.N, g.BN);
+      // A wait that gives up (error word set) does not end the task: the four
+      // epilogue warps must reach every named barrier together, so they run
+      // on with whatever tensor memory holds.
+      if (lane == 0) mbar_wait_g(&tfull[acc], aph, P.err);
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * 2 * C::BN_MAX;
+      const bool two = nst >= 2;
+      bool done = true;   // this task finished its tile (else: a non-final split)
+      if (g.S == 1) {
+        float ssq = 0.f;
+        switch (ph) {
+          case PH_WO: ssq = epi_tile_tmem<EPI_WO>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs); break;
+          case PH_W1: epi_tile_tmem<EPI_W1>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs); break;
+          case PH_W2: ssq = epi_tile_tmem<EPI_W2>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs); break;
+          default: epi_tile_tmem<EPI_WKV>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs); break;
+        }
+        if (row_ok && ph == PH_WO) P.ssq_u[(size_t)T.tile * P.ep.B + row] = ssq;
+        if (row_ok && ph == PH_W2) P.ssq_z[(size_t)T.tile * P.ep.B + row] = ssq;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+      } else {
+        // split of W2: this split's partial tile to its slot ([col][row], so
+        // that a warp's stores and loads are 128-byte lines)
+        float* slot = P.w2part + (((size_t)T.rb * g.tiles + T.tile) * g.S + T.split) * (size_t)g.BN * C::BM;
+#pragma unroll 1
+        for (int c = 0; c < g.BN; c += 32) {
+          float v[32];
+          tmem_ld_pair(taddr + c, two, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) slot[(size_t)(c + i) * C::BM + lrow] = v[i];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        __threadfence();
+        epi_bar();
+        if (tid == 0) {
+          unsigned* cnt = P.w2cnt + (size_t)T.rb * g.tiles + T.tile;
+          const unsigned old = atom_add_acq_rel(cnt, 1u);
+          *s_last = (old == (unsigned)(g.S * j + g.S - 1)) ? 1 : 0;
+          __threadfence();
+        }
+        epi_bar();
+        done = *s_last != 0;
+        epi_bar();   // s_last is read by every thread before the next split task can rewrite it
+        if (done) {
+          // the last split: every split's partial is in its slot; sum them in
+          // split order and run the W2 epilogue
+          __threadfence();
+          epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);
+          epi_bar();
+          const float* slots = P.w2part + ((size_t)T.rb * g.tiles + T.tile) * g.S * (size_t)g.BN * C::BM;
+          float ssq = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < g.BN; c += 32) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            for (int sp = 0; sp < g.S; ++sp) {
+              const float* src = slots + (size_t)sp * g.BN * C::BM + (size_t)c * C::BM + lrow;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] += __ldcg(src + (size_t)i * C::BM);
+            }
+            if (row_ok) ssq += epilogue_chunk<EPI_W2>(e, row, col_base + c, g.N, v, 1.f);
+          }
+          if (row_ok) P.ssq_z[(size_t)T.tile * P.ep.B + row] = ssq;
+        }
+      }
+      if (done) {
+        fence_proxy_async_global();   // the next phase reads these outputs with TMA
+        __threadfence();
+        epi_bar();
+        if (tid == 0) st_release_u32(flag_ptr(P, ph, T.rb, T.tile), (unsigned)(j + 1));
+      }
+      return true;
+    });
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace rt

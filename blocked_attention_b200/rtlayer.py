@@ -30,7 +30,7 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_erro
            "rt_embed_forward", "rt_block_fold", "rt_project_qkv", "rt_gemm_bf16",
            "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc",
            "rt_selftest_wait_timeout", "rt_layer_decode_workspace_bytes", "rt_layer_decode_step",
-           "rt_project_qkv_noalloc_status")
+           "rt_project_qkv_noalloc_status", "rt_layer_recompute_workspace_bytes", "rt_layer_recompute_kv")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma")
@@ -97,6 +97,10 @@ def lib() -> ctypes.CDLL:
     L.rt_project_qkv_noalloc.argtypes = [vp, vp, i, i, i, vp, vp]
     L.rt_project_qkv_noalloc_status.restype = i
     L.rt_project_qkv_noalloc_status.argtypes = [vp]
+    L.rt_layer_recompute_workspace_bytes.restype = sz
+    L.rt_layer_recompute_workspace_bytes.argtypes = [i] * 3
+    L.rt_layer_recompute_kv.restype = i
+    L.rt_layer_recompute_kv.argtypes = [vp] * 3 + [i] * 3 + [vp] * 3 + [sz, vp]
     L.rt_selftest_wait_timeout.restype = i
     L.rt_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp, vp]
     L.rt_layer_decode_workspace_bytes.restype = sz
@@ -241,6 +245,31 @@ def layer_decode_step(x_t: torch.Tensor, W: dict, H: int, t: int, K_cache: torch
                                     ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("rt_layer_decode_step", rc)
     return z
+
+
+def recompute_kv(z: torch.Tensor, W_k: torch.Tensor, W_v: torch.Tensor, out=None,
+                 workspace: torch.Tensor | None = None, stream=None):
+    """rt_layer_recompute_kv: the persistent pairs of every position rebuilt
+    from stored outputs z [B, N, d] (bf16, cuda). Returns (K, V), each
+    position-major [N, B, d]."""
+    B, N, d = z.shape
+    for tsr in (z, W_k, W_v):
+        if tsr.dtype != torch.bfloat16 or not tsr.is_contiguous() or tsr.device != z.device:
+            raise ValueError("recompute tensors must be contiguous bf16 tensors on one device")
+    if out is None:
+        K = torch.empty((N, B, d), dtype=z.dtype, device=z.device)
+        V = torch.empty_like(K)
+    else:
+        K, V = out
+    nbytes = int(lib().rt_layer_recompute_workspace_bytes(B, N, d))
+    if nbytes == 0:
+        raise RTError("rt_layer_recompute_workspace_bytes", RT_ERR_UNSUPPORTED)
+    if workspace is None:
+        workspace = alloc_workspace(nbytes, z.device)
+    rc = lib().rt_layer_recompute_kv(_ptr(z), _ptr(W_k), _ptr(W_v), B, N, d, _ptr(K), _ptr(V), _ptr(workspace),
+                                     ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("rt_layer_recompute_kv", rc)
+    return K, V
 
 
 def sync_status(workspace: torch.Tensor, stream=None) -> int:

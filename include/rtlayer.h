@@ -161,6 +161,26 @@ int rt_layer_decode_step(const void* x_t_dev,
                          void* z_t_dev, void* K_cache_dev, void* V_cache_dev,
                          void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* Device bytes rt_layer_recompute_kv needs (bf16); 0 if unsupported. */
+size_t rt_layer_recompute_workspace_bytes(int B, int N, int d);
+
+/* Activation-checkpoint recompute of the persistent pairs (paper §6.1: with
+ * the layer's inputs and outputs stored, the persistent pairs of every
+ * position are rebuilt from the outputs in one parallel step):
+ *   K[n][b] = W_k rms(z[b][n]),  V[n][b] = W_v rms(z[b][n])
+ * for all B*N positions at once, bf16 storage, fp32 accumulation (one
+ * tensor-core GEMM of [B*N][d] x [2d][d]^T with the 1/rms(z) row scale in its
+ * epilogue). z_dev [B][N][d]; K_dev, V_dev position-major [N][B][d], as
+ * rt_layer_forward returns them. d % 64 == 0, B*N <= 2^30.
+ * workspace_dev: >= rt_layer_recompute_workspace_bytes(B, N, d) bytes,
+ * 256-byte aligned; its first word is the error word (rt_layer_sync_status).
+ * Enqueued on `stream`. The forward forms each pair from the bf16 copy of
+ * z_t with the fp32 sum of squares of z_t; from the stored bf16 z the result
+ * agrees up to that rounding. */
+int rt_layer_recompute_kv(const void* z_dev, const void* W_k_dev, const void* W_v_dev,
+                          int B, int N, int d, void* K_dev, void* V_dev,
+                          void* workspace_dev, size_t workspace_bytes, void* stream);
+
 /* Token-embedding front end of a layer stack: x[b][n][:] = E[ids[b][n]][:].
  * Paper §6.1 stacks layers by feeding each layer's outputs z to the next
  * layer as its inputs; the first layer's inputs are the embedded tokens, so a

@@ -91,12 +91,22 @@ def test_workspace_plan(L):
     assert L.rt_layer_host_workspace_bytes(512, 2048, 1024, 16, 4096, bf, 0) > hb + 4 * 2.1e9
 
 
+def _step_kernel_launches(N):
+    # the persistent step kernel runs segments of steps ending at a position t
+    # whose fold has >= 16 keys (that fold follows as its own launch) or t = N
+    segments = sum(1 for t in range(1, N + 1) if t == N or (t & -t) >= 16)
+    big_folds = sum(1 for t in range(1, N) if (t & -t) >= 16)
+    return segments + big_folds
+
+
 def test_launch_count_matches_schedule(L):
-    # bf16 blocked: inv_rms + projection + finalise(position 1) + 4 GEMMs per step
-    # + one fold per step t < N (each also finalises position t + 1)
-    for N in (1, 2, 7, 64, 2048):
-        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0) == 3 + 4 * N + (N - 1)
+    # bf16 blocked: inv_rms + projection + finalise(position 1) + the step
+    # kernel's segments + the folds of >= 16 keys between them
+    for N in (1, 2, 7, 16, 17, 64, 2048):
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0) == 3 + _step_kernel_launches(N)
         assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 1) == 2 + 5 * N
+    # the headline: 128 segments and 127 large folds
+    assert L.rt_layer_launch_count(512, 2048, 1024, 16, 4096, R.RT_BF16, 0) == 3 + 128 + 127
     assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_F32, 0) == 2 + 8 * 8 + 7
     assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_BF16, 0) == -1
 
@@ -181,3 +191,16 @@ def test_binding_signatures_match_header(L):
         fn = getattr(L, name)
         got = len(fn.argtypes) if fn.argtypes is not None else 0
         assert got == n, f"{name}: binding declares {got} arguments, header {n}"
+
+
+def test_recompute_validation_happens_before_any_launch(L):
+    assert L.rt_layer_recompute_workspace_bytes(4, 16, 128) >= 256 + 4 * 16 * 4 + 2 * 128 * 128 * 2
+    assert L.rt_layer_recompute_workspace_bytes(4, 16, 96) == 0          # d % 64 != 0
+    assert L.rt_layer_recompute_workspace_bytes(0, 16, 128) == 0
+    p = ctypes.c_void_p(1 << 40)
+    big = ctypes.c_size_t(1 << 30)
+    call = L.rt_layer_recompute_kv
+    assert call(None, p, p, 4, 16, 128, p, p, p, big, None) == R.RT_ERR_INVALID_ARG
+    assert call(p, p, p, 4, 16, 96, p, p, p, big, None) == R.RT_ERR_UNSUPPORTED
+    assert call(ctypes.c_void_p((1 << 40) + 8), p, p, 4, 16, 128, p, p, p, big, None) == R.RT_ERR_INVALID_ARG
+    assert call(p, p, p, 4, 16, 128, p, p, p, ctypes.c_size_t(64), None) == R.RT_ERR_WORKSPACE
