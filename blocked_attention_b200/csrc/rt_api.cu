@@ -276,7 +276,14 @@ static cudaError_t launch_tc(int bn, const CUtensorMap& ta, const CUtensorMap& t
 // ---------------------------------------------------------------------------
 struct Shape {
   int B, N, d, H, d_ff, dtype, schedule;
+  // pages = 1: the paper's own parameterisation (per-head unit-RMS queries
+  // and keys, no softmax scale, RMS without eps, branches scaled by
+  // 1/sqrt(L)); 0: the single-layer configuration
+  int pages = 0, L = 1;
   int dh() const { return d / H; }
+  float eps() const { return pages ? 0.f : kEps; }
+  // softmax scale in log2 units: log2(e) / sqrt(d_h), or log2(e) unscaled
+  float sc2() const { return pages ? kLog2e : kLog2e / std::sqrt((float)dh()); }
 };
 
 static int validate(const Shape& s) {
@@ -293,6 +300,8 @@ static int validate(const Shape& s) {
   } else {
     if (dh != 64 || s.d % 64 != 0 || s.d_ff % 64 != 0) return RT_ERR_UNSUPPORTED;
   }
+  if (s.pages && (s.dtype != RT_BF16 || s.schedule != RT_SCHED_BLOCKED)) return RT_ERR_UNSUPPORTED;
+  if (s.L < 1) return RT_ERR_INVALID_ARG;
   return RT_OK;
 }
 
@@ -561,12 +570,14 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
   RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + 2 * dd, X.Wv, dd, cudaMemcpyDeviceToDevice, st));
 
   // 1. queries and temporary pairs of all positions
-  const int bn_p = choose_bn((int)rows, 3 * d);
+  // (the paper's per-head normalisation needs whole 64-column heads per tile)
+  const int bn_p = std::max(s.pages ? 64 : 32, choose_bn((int)rows, 3 * d));
   CUtensorMap tB_qkv;
   if (!make_tmap(&tB_qkv, wqkv, d, 3 * d, bn_p)) return RT_ERR_INVALID_ARG;
   EpiParams ep;
   std::memset(&ep, 0, sizeof(ep));
-  ep.B = B; ep.Nseq = N; ep.d = d; ep.d_ff = dff; ep.eps = kEps;
+  ep.B = B; ep.Nseq = N; ep.d = d; ep.d_ff = dff; ep.eps = s.eps();
+  ep.pages = s.pages; ep.inv_sqrt_L = 1.f / std::sqrt((float)s.L);
   ep.inv_rms = inv; ep.qkv = qkv; ep.x = x; ep.u32 = u32; ep.u16 = u16; ep.h16 = h16;
   ep.zout = static_cast<bf16*>(X.z); ep.z16 = z16; ep.Kout = K; ep.Vout = V;
   // x arrives in chunks of xc positions (the host-buffer path uploads chunk
@@ -601,7 +612,7 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
       if (io) RT_CK(cudaStreamWaitEvent(st, ds.events[ev_x + c], 0));
       {
         TimedScope ts(T, KC_INV_RMS, st);
-        k_row_inv_rms<bf16><<<(unsigned)((nr + 7) / 8), 256, 0, st>>>(xs, inv, nr, d, kEps);
+        k_row_inv_rms<bf16><<<(unsigned)((nr + 7) / 8), 256, 0, st>>>(xs, inv, nr, d, s.eps());
       }
       RT_CK(cudaGetLastError());
       CUtensorMap tA_x;
@@ -641,7 +652,8 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
       !make_tmap(&tA_h, h16, dff, B, 128) || !make_tmap(&tB_2, X.W2, dff, d, bn_2) ||
       !make_tmap(&tA_z, z16, d, B, 128) || !make_tmap(&tB_kv, wqkv + (size_t)d * d, d, 2 * d, bn_kv))
     return RT_ERR_INVALID_ARG;
-  const float sc2 = kLog2e / std::sqrt((float)s.dh());
+  const float sc2 = s.sc2();
+  if (s.pages && !P.sp.ok) return RT_ERR_UNSUPPORTED;   // head normalisation lives in the step kernel
   const bool blocked = s.schedule == RT_SCHED_BLOCKED;
   // step j reads queries and temporary pairs of positions up to 2j + 1
   // (the fold of step j covers queries j + 1 .. 2j + 1, 0-based) and x of j
@@ -886,7 +898,7 @@ static long launch_count(const Shape& s) {
 // ---------------------------------------------------------------------------
 struct GraphKey {
   uintptr_t p[15];
-  int v[8];
+  int v[10];
   bool operator<(const GraphKey& o) const {
     int c = std::memcmp(p, o.p, sizeof(p));
     if (c) return c < 0;
@@ -919,7 +931,7 @@ static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st
                           io ? io->x_host : nullptr, io ? io->z_host : nullptr,
                           io ? io->K_host : nullptr, io ? io->V_host : nullptr};
   for (int i = 0; i < 15; ++i) key.p[i] = reinterpret_cast<uintptr_t>(ptrs[i]);
-  const int vals[8] = {P.s.B, P.s.N, P.s.d, P.s.H, P.s.d_ff, P.s.dtype, P.s.schedule, dev};
+  const int vals[10] = {P.s.B, P.s.N, P.s.d, P.s.H, P.s.d_ff, P.s.dtype, P.s.schedule, dev, P.s.pages, P.s.L};
   std::memcpy(key.v, vals, sizeof(vals));
 
   std::lock_guard<std::mutex> lk(g_graph_mu);
@@ -1001,6 +1013,27 @@ extern "C" int rt_layer_forward(const void* x, const void* W_q, const void* W_k,
     return RT_ERR_WORKSPACE;
   Ptrs X{x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V, workspace};
   return run_forward(P, X, driver, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int rt_layer_forward_pages(const void* x, const void* W_q, const void* W_k, const void* W_v,
+                                      const void* W_o, const void* W_1, const void* W_2, int B, int N, int d, int H,
+                                      int d_ff, int L, void* z, void* K, void* V, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  Shape s{B, N, d, H, d_ff, RT_BF16, RT_SCHED_BLOCKED};
+  s.pages = 1;
+  s.L = L;
+  int rc = validate(s);
+  if (rc != RT_OK) return rc;
+  if (!x || !W_q || !W_k || !W_v || !W_o || !W_1 || !W_2 || !z || !K || !V) return RT_ERR_INVALID_ARG;
+  const void* all[10] = {x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V};
+  for (const void* p : all)
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return RT_ERR_INVALID_ARG;
+  const Plan P = make_plan(s);
+  if (!P.sp.ok) return RT_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return RT_ERR_WORKSPACE;
+  Ptrs X{x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V, workspace};
+  return run_forward(P, X, RT_DRIVER_GRAPH, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int rt_layer_sync_status(void* workspace, void* stream) {

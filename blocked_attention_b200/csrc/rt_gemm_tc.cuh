@@ -66,6 +66,13 @@ struct EpiParams {
   // all ranks' partials over distributed shared memory, in rank order, and
   // runs the epilogue for them. BN/splits must be a multiple of 32.
   int splits;
+  // the paper's own parameterisation ("Recurrent Transformer" paper page,
+  // paper §2 notation and §2.1): pages = 1 normalises every head of q, k~
+  // (PROJ) and k (WKV, RKV) to unit RMS, and scales the W_o and W_2 branches
+  // by inv_sqrt_L = 1/sqrt(L) (the caller also sets eps = 0 and drops the
+  // softmax scale). pages = 0: the single-layer configuration.
+  int pages;
+  float inv_sqrt_L;
 };
 
 __device__ __forceinline__ uint32_t dsmem_map(uint32_t smem_addr, uint32_t rank) {
@@ -198,6 +205,10 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
     float xv[32];
     const int c = p.j / p.xc;
     load_bf16x32(p.x + (((size_t)c * p.B + b) * p.xc + (p.j - c * p.xc)) * p.d + col0, xv);
+    if (p.pages) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= p.inv_sqrt_L;
+    }
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       v[i] += xv[i];
@@ -215,6 +226,10 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
     const int b = row;
     // u was written by other CTAs (L2-coherent loads: no stale L1 lines)
     const float4* u4 = reinterpret_cast<const float4*>(p.u32 + (size_t)b * p.d + col0);
+    if (p.pages) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= p.inv_sqrt_L;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       float4 w = __ldcg(u4 + i);
@@ -241,6 +256,30 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
     else store_bf16x32(p.Vout + base + (col0 - p.d), v);
   }
   return ssq;
+}
+
+// The paper's per-head query/key normalisation (paper §2.1, RMS applied to
+// each head's d_h = 64 entries): 64 columns = one head of one row, scaled by
+// the row factor, then, for the q / k~ columns of PROJ ([0, 2d)) and the k
+// columns of WKV and RKV ([0, d)), normalised to unit RMS; then stored by the
+// 32-column epilogue with a row factor of 1.
+template <int EPI>
+__device__ __forceinline__ void epilogue_head64(const EpiParams& p, int row, int col0, int N, float (&va)[32],
+                                                float (&vb)[32], float row_scale) {
+  static_assert(EPI == EPI_PROJ || EPI == EPI_WKV || EPI == EPI_RKV, "head normalisation epilogues");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) { va[i] *= row_scale; vb[i] *= row_scale; }
+  const bool normed = EPI == EPI_PROJ ? col0 < 2 * p.d : col0 < p.d;
+  if (normed) {
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ss += va[i] * va[i] + vb[i] * vb[i];
+    const float sc = rsqrtf(ss * (1.f / 64.f));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) { va[i] *= sc; vb[i] *= sc; }
+  }
+  epilogue_chunk<EPI>(p, row, col0, N, va, 1.f);
+  epilogue_chunk<EPI>(p, row, col0 + 32, N, vb, 1.f);
 }
 
 // 32 columns of a tile's accumulator for this thread's row: the sum of the
@@ -432,8 +471,21 @@ __global__ void __launch_bounds__(224, 1)
       const bool two = NACC == 2 && nk >= 2;   // issuer 1 wrote its accumulator in this tile
       if (splits == 1) {
         float ssq = 0.f;
+        bool head_norm = false;
+        if constexpr ((EPI == EPI_PROJ || EPI == EPI_WKV || EPI == EPI_RKV) && BN >= 64) head_norm = p.pages != 0;
+        if (head_norm) {
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+          for (int c = 0; c < BN; c += 64) {
+            float va[32], vb[32];
+            tmem_ld_acc<NACC, BN>(taddr + c, two, va);
+            tmem_ld_acc<NACC, BN>(taddr + c + 32, two, vb);
+            const int col0 = nt * BN + c;
+            if constexpr ((EPI == EPI_PROJ || EPI == EPI_WKV || EPI == EPI_RKV) && BN >= 64)
+              if (row_ok && col0 < N) epilogue_head64<EPI>(p, row, col0, N, va, vb, rs);
+          }
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN && !head_norm; c += 32) {
           float v[32];
           tmem_ld_acc<NACC, BN>(taddr + c, two, v);
           const int col0 = nt * BN + c;

@@ -383,6 +383,18 @@ template <int EPI>
 __device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool row_ok, int col_base, int BN, int N,
                                                uint32_t taddr, bool two, float rs) {
   float ssq = 0.f;
+  if constexpr (EPI == EPI_WKV) {
+    if (e.pages) {   // per-head unit RMS of k (the paper's parameterisation)
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 64) {
+        float va[32], vb[32];
+        tmem_ld_pair(taddr + c, two, va);
+        tmem_ld_pair(taddr + c + 32, two, vb);
+        if (row_ok) epilogue_head64<EPI_WKV>(e, row, col_base + c, N, va, vb, rs);
+      }
+      return 0.f;
+    }
+  }
 #pragma unroll 1
   for (int c = 0; c < BN; c += 32) {
     float v[32];

@@ -30,7 +30,8 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_erro
            "rt_embed_forward", "rt_block_fold", "rt_project_qkv", "rt_gemm_bf16",
            "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc",
            "rt_selftest_wait_timeout", "rt_layer_decode_workspace_bytes", "rt_layer_decode_step",
-           "rt_project_qkv_noalloc_status", "rt_layer_recompute_workspace_bytes", "rt_layer_recompute_kv")
+           "rt_project_qkv_noalloc_status", "rt_layer_recompute_workspace_bytes", "rt_layer_recompute_kv",
+           "rt_layer_forward_pages")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma")
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.rt_layer_forward.argtypes = fwd_args
     L.rt_layer_forward_host.restype = i
     L.rt_layer_forward_host.argtypes = fwd_args
+    L.rt_layer_forward_pages.restype = i
+    L.rt_layer_forward_pages.argtypes = [vp] * 7 + [i] * 6 + [vp] * 4 + [sz, vp]
     L.rt_layer_sync_status.restype = i
     L.rt_layer_sync_status.argtypes = [vp, vp]
     L.rt_embed_forward.restype = i
@@ -186,6 +189,33 @@ def layer_forward(x: torch.Tensor, W: dict, H: int, d_ff: int | None = None, sch
                                 SCHEDULES[schedule], DRIVERS[driver], _ptr(z), _ptr(K), _ptr(V),
                                 _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("rt_layer_forward", rc)
+    return z, K, V
+
+
+def layer_forward_pages(x: torch.Tensor, W: dict, H: int, L: int = 1, out=None,
+                        workspace: torch.Tensor | None = None, stream=None):
+    """rt_layer_forward_pages: the layer in the paper's own parameterisation
+    (per-head unit-RMS queries and keys, no softmax scale, RMS without eps,
+    branches scaled by 1/sqrt(L)); bf16 device tensors as in layer_forward."""
+    B, N, d = x.shape
+    d_ff = W["W_1"].shape[0]
+    for n in WEIGHT_NAMES:
+        if W[n].dtype != torch.bfloat16 or not W[n].is_contiguous() or W[n].device != x.device:
+            raise ValueError(f"weight {n} must be a contiguous bf16 tensor on {x.device}")
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 tensor")
+    if out is None:
+        z = torch.empty_like(x)
+        K = torch.empty((N, B, d), dtype=x.dtype, device=x.device)
+        V = torch.empty_like(K)
+    else:
+        z, K, V = out
+    if workspace is None:
+        workspace = alloc_workspace(workspace_bytes(B, N, d, H, d_ff), x.device)
+    rc = lib().rt_layer_forward_pages(_ptr(x), *[_ptr(W[n]) for n in WEIGHT_NAMES], B, N, d, H, d_ff, L,
+                                      _ptr(z), _ptr(K), _ptr(V), _ptr(workspace),
+                                      ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("rt_layer_forward_pages", rc)
     return z, K, V
 
 

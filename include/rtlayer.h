@@ -109,6 +109,25 @@ int rt_layer_forward(const void* x_dev,
                      void* z_dev, void* K_dev, void* V_dev,
                      void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* The layer in the paper's own parameterisation (paper §2 notation, §2.1 and
+ * §2.2, rather than the single-layer configuration above), bf16, blocked
+ * schedule, graph driver:
+ *   RMS(v) = sqrt(D) v / ||v|| (no eps, unit gain); RMS_h = the same over
+ *   each head's 64 entries;
+ *   r = RMS(x_t); q = RMS_h(W_q r); k~ = RMS_h(W_k r); v~ = W_v r
+ *   a_t: per head softmax of <k, q_h> with no scale
+ *   u = x_t + W_o a_t / sqrt(L); z_t = u + W_2 GELU(W_1 RMS(u)) / sqrt(L)
+ *   k_t = RMS_h(W_k RMS(z_t)); v_t = W_v RMS(z_t)
+ * L >= 1 is the depth of the stack the layer belongs to. Arguments, layouts
+ * and workspace (rt_layer_workspace_bytes with RT_BF16, RT_SCHED_BLOCKED) as
+ * in rt_layer_forward. */
+int rt_layer_forward_pages(const void* x_dev,
+                           const void* W_q_dev, const void* W_k_dev, const void* W_v_dev,
+                           const void* W_o_dev, const void* W_1_dev, const void* W_2_dev,
+                           int B, int N, int d, int H, int d_ff, int L,
+                           void* z_dev, void* K_dev, void* V_dev,
+                           void* workspace_dev, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of a
  * workspace used by rt_layer_forward. RT_OK, RT_ERR_TIMEOUT or RT_ERR_CUDA. */
 int rt_layer_sync_status(void* workspace_dev, void* stream);

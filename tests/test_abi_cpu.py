@@ -204,3 +204,16 @@ def test_recompute_validation_happens_before_any_launch(L):
     assert call(p, p, p, 4, 16, 96, p, p, p, big, None) == R.RT_ERR_UNSUPPORTED
     assert call(ctypes.c_void_p((1 << 40) + 8), p, p, 4, 16, 128, p, p, p, big, None) == R.RT_ERR_INVALID_ARG
     assert call(p, p, p, 4, 16, 128, p, p, p, ctypes.c_size_t(64), None) == R.RT_ERR_WORKSPACE
+
+
+def test_pages_entry_point_validation_happens_before_any_launch(L):
+    p = ctypes.c_void_p(1 << 40)
+
+    def call(Lv=1, d=128, H=2, ws_bytes=1 << 34):
+        return L.rt_layer_forward_pages(*([p] * 7), 2, 16, d, H, 256, Lv, p, p, p, p, ctypes.c_size_t(ws_bytes),
+                                        None)
+    assert call(Lv=0) == R.RT_ERR_INVALID_ARG          # the stack depth L >= 1
+    assert call(d=96, H=2) == R.RT_ERR_UNSUPPORTED       # bf16 needs d_h = 64
+    assert call(ws_bytes=16) == R.RT_ERR_WORKSPACE
+    assert L.rt_layer_forward_pages(None, *([p] * 6), 2, 16, 128, 2, 256, 1, p, p, p, p,
+                                    ctypes.c_size_t(1 << 34), None) == R.RT_ERR_INVALID_ARG
