@@ -1,0 +1,455 @@
+// rt_backward.cu -- backward pass of the Recurrent Transformer layer, fp32
+// storage and arithmetic (SIMT; the 1e-4 parity mode).
+//
+// Source: "Recurrent Transformer" paper page (www.lshu.cn/news/403416):
+//   paper §2.2 : the layer (queries and temporary pairs from x_t, persistent
+//                pairs from z_t);
+//   paper §6.1 : activation checkpointing -- with the layer's inputs x and
+//                outputs z (and the persistent pairs K, V) stored, every
+//                intermediate of the forward is rebuilt in parallel;
+//   notes §5.3 : the backward's weight gradients batched outside the
+//                per-position loop;
+//   paper §6.4 : the backward pass itself (its body is missing from the
+//                extracted text; the steps below are the exact derivatives of
+//                the forward definition).
+//
+// Gradients of the scalar sum(z * dz) + sum(K * dK) + sum(V * dV):
+//  1. Rebuild (all B*N positions at once): r = rms(x), q / k~ / v~, the
+//     attention output a_t and its log-sum-exp per head (over the stored
+//     persistent pairs of positions < t plus the temporary pair), u, rms(u),
+//     the MLP pre-activation, rms(z).
+//  2. Reverse loop over positions t = N..1, M = B rows per step:
+//       dk_t, dv_t are complete (every later query has contributed);
+//       d rms(z_t) = dk_t W_k + dv_t W_v;  dz_t += rms'(z_t) ...
+//       MLP backward -> du_t;  da_t = du_t W_o;
+//       attention backward of query t: its contributions to dk_i, dv_i of
+//       every earlier position (added in place), to its own dq and to the
+//       temporary pair's dk~, dv~.
+//  3. Batched over all positions: dx = du + rms'(x)(dq W_q + dk~ W_k +
+//     dv~ W_v), and every weight gradient as one [out][B*N] x [B*N][in]
+//     product.
+// Per-position buffers are position-major (row t*B + b), like K and V.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "../../include/rtlayer.h"
+#include "rt_common.cuh"
+#include "rt_host.h"
+
+namespace rt {
+namespace bwd {
+
+// C[m][n] (+)= sum_k A(m, k) * W(n, k), fp32, 64 x 64 tile per CTA of 256
+// threads; A(m, k) = ta ? A[k * lda + m] : A[m * lda + k], likewise W.
+__global__ void __launch_bounds__(256) k_gemm(const float* __restrict__ A, int lda, int ta,
+                                              const float* __restrict__ W, int ldw, int tw, float* __restrict__ C,
+                                              int ldc, int M, int N, int K, int accumulate) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Ws[16][64 + 4];
+  const int row0 = blockIdx.y * 64, col0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 1024; i += 256) {
+      // ta / tw: consecutive threads walk the non-K index (coalesced for the
+      // transposed operand), else the K index
+      int r, kk;
+      if (ta) { kk = i >> 6; r = i & 63; } else { r = i >> 4; kk = i & 15; }
+      const int gr = row0 + r, gk = k0 + kk;
+      As[kk][r] = (gr < M && gk < K) ? (ta ? A[(size_t)gk * lda + gr] : A[(size_t)gr * lda + gk]) : 0.f;
+      int c, kw;
+      if (tw) { kw = i >> 6; c = i & 63; } else { c = i >> 4; kw = i & 15; }
+      const int gc = col0 + c, gkw = k0 + kw;
+      Ws[kw][c] = (gc < N && gkw < K) ? (tw ? W[(size_t)gkw * ldw + gc] : W[(size_t)gc * ldw + gkw]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; w[i] = Ws[kk][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = row0 + ty * 4 + i, c = col0 + tx * 4 + j;
+      if (r < M && c < N) {
+        float* dst = C + (size_t)r * ldc + c;
+        *dst = accumulate ? *dst + acc[i][j] : acc[i][j];
+      }
+    }
+}
+
+// dst[n][b][:] = src[b][n][:] (to = 1), or the inverse (to = 0)
+__global__ void k_permute(const float* __restrict__ src, float* __restrict__ dst, int B, int N, int d, int to) {
+  const size_t total = (size_t)B * N * d;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int e = (int)(i % d);
+    const size_t r = i / d;
+    if (to) {   // i indexes src [B][N][d]
+      const int n = (int)(r % N), b = (int)(r / N);
+      dst[((size_t)n * B + b) * d + e] = src[i];
+    } else {    // i indexes src [N][B][d]
+      const int b = (int)(r % B), n = (int)(r / B);
+      dst[((size_t)b * N + n) * d + e] = src[i];
+    }
+  }
+}
+
+// out[r] = in[r] * c_r, c_r = 1 / sqrt(mean(in[r]^2) + eps); one warp per row
+__global__ void __launch_bounds__(256) k_rms_rows(const float* __restrict__ in, float* __restrict__ out,
+                                                  float* __restrict__ cinv, size_t rows, int d, float eps) {
+  const size_t r = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float* v = in + r * d;
+  float s = 0.f;
+  for (int e = lane; e < d; e += 32) s += v[e] * v[e];
+  s = warp_sum(s);
+  const float c = rsqrtf(s / (float)d + eps);
+  for (int e = lane; e < d; e += 32) out[r * d + e] = v[e] * c;
+  if (lane == 0) cinv[r] = c;
+}
+
+// Backward of y = v * c(v), c = (mean(v^2) + eps)^(-1/2), for upstream g:
+//   dv = c g - c^3 (v . g) / d * v;   out[r] = add[r] + dv  (add may be null)
+__global__ void __launch_bounds__(256) k_rms_bwd(const float* __restrict__ v, const float* __restrict__ g,
+                                                 const float* __restrict__ cinv, const float* __restrict__ add,
+                                                 float* __restrict__ out, size_t rows, int d) {
+  const size_t r = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float* vr = v + r * d;
+  const float* gr = g + r * d;
+  float s = 0.f;
+  for (int e = lane; e < d; e += 32) s += vr[e] * gr[e];
+  s = warp_sum(s);
+  const float c = cinv[r];
+  const float k = c * c * c * s / (float)d;
+  for (int e = lane; e < d; e += 32) {
+    const float dv = c * gr[e] - k * vr[e];
+    out[r * d + e] = (add ? add[r * d + e] : 0.f) + dv;
+  }
+}
+
+// y = GELU(h) (exact erf form) and its derivative dGELU/dh = Phi(h) + h phi(h)
+__global__ void k_gelu(const float* __restrict__ h, float* __restrict__ y, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    y[i] = gelu_erf(h[i]);
+}
+__global__ void k_gelu_bwd(const float* __restrict__ dy, const float* __restrict__ h, float* __restrict__ dh,
+                           size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const float x = h[i];
+    const float Phi = 0.5f * (1.f + erff(x * 0.70710678118654752f));
+    const float phi = 0.39894228040143268f * expf(-0.5f * x * x);
+    dh[i] = dy[i] * (Phi + x * phi);
+  }
+}
+
+// Attention of every position at once over the stored persistent pairs
+// (rows 0..t-1 of K, V) plus its temporary pair, natural-log units:
+//   a_t = sum_i softmax(s)_i v_i,  lse_t = log sum_i exp(s_i),  s_i = <q, k_i> * scale.
+// One warp per (t, b, h); lanes split the keys, then merge.
+__global__ void __launch_bounds__(128) k_attn_lse(const float* __restrict__ qkv, const float* __restrict__ K,
+                                                  const float* __restrict__ V, float* __restrict__ a,
+                                                  float* __restrict__ lse, int B, int N, int H, int dh,
+                                                  float scale) {
+  const long w = (long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= (long)N * B * H) return;
+  const int h = (int)(w % H);
+  const long rb = w / H;                       // position-major row t * B + b
+  const int b = (int)(rb % B), t = (int)(rb / B);
+  const int d = H * dh;
+  const float* q = qkv + (size_t)rb * 3 * d + h * dh;
+  // scores: lane handles keys lane, lane + 32, ...; key t (index t) is the temporary pair
+  float m = -INFINITY;
+  for (int i = lane; i <= t; i += 32) {
+    const float* k = i < t ? K + ((size_t)i * B + b) * d + h * dh : q + d;
+    float s = 0.f;
+    for (int e = 0; e < dh; ++e) s += q[e] * k[e];
+    m = fmaxf(m, s * scale);
+  }
+  m = warp_max(m);
+  float l = 0.f;
+  for (int i = lane; i <= t; i += 32) {
+    const float* k = i < t ? K + ((size_t)i * B + b) * d + h * dh : q + d;
+    float s = 0.f;
+    for (int e = 0; e < dh; ++e) s += q[e] * k[e];
+    l += expf(s * scale - m);
+  }
+  l = warp_sum(l);
+  const float L = m + logf(l);
+  // a: lane handles dims lane, lane + 32, ... (keys in order)
+  for (int e = lane; e < dh; e += 32) {
+    float acc = 0.f;
+    for (int i = 0; i <= t; ++i) {
+      const float* k = i < t ? K + ((size_t)i * B + b) * d + h * dh : q + d;
+      const float* v = i < t ? V + ((size_t)i * B + b) * d + h * dh : q + 2 * d;
+      float s = 0.f;
+      for (int f = 0; f < dh; ++f) s += q[f] * k[f];
+      acc += expf(s * scale - L) * v[e];
+    }
+    a[(size_t)rb * d + h * dh + e] = acc;
+  }
+  if (lane == 0) lse[(size_t)rb * H + h] = L;
+}
+
+// Attention backward of query t (all sequences and heads): one warp per
+// (b, h). With p_i = exp(s_i - lse), dp_i = <da, v_i>, delta = <da, a>,
+// ds_i = p_i (dp_i - delta):
+//   dk_i += scale ds_i q,  dv_i += p_i da      (persistent pairs i < t, in place)
+//   dq = scale sum_i ds_i k_i,  dk~ = scale ds~ q,  dv~ = p~ da   (temporary pair)
+// Each (i, b, h) row of dK, dV is updated by exactly one warp.
+__global__ void __launch_bounds__(128) k_attn_bwd_step(const float* __restrict__ qkv, const float* __restrict__ K,
+                                                       const float* __restrict__ V, const float* __restrict__ a,
+                                                       const float* __restrict__ lse, const float* __restrict__ da,
+                                                       float* __restrict__ dK, float* __restrict__ dV,
+                                                       float* __restrict__ dqkv, int B, int H, int dh, int t,
+                                                       float scale) {
+  const int w = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= B * H) return;
+  const int b = w / H, h = w - b * H;
+  const int d = H * dh;
+  const size_t rt_ = (size_t)t * B + b;
+  const float* q = qkv + rt_ * 3 * d + h * dh;
+  const float* dav = da + rt_ * d + h * dh;
+  const float* av = a + rt_ * d + h * dh;
+  const float L = lse[rt_ * H + h];
+  float delta = 0.f;
+  for (int e = lane; e < dh; e += 32) delta += dav[e] * av[e];
+  delta = warp_sum(delta);
+  float* dq = dqkv + rt_ * 3 * d + h * dh;
+  // dq accumulates in registers: lane owns dims lane, lane + 32, ... (dh <= 128)
+  float dqr[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int i = 0; i <= t; ++i) {
+    const bool temp = i == t;
+    const float* k = temp ? q + d : K + ((size_t)i * B + b) * d + h * dh;
+    const float* v = temp ? q + 2 * d : V + ((size_t)i * B + b) * d + h * dh;
+    float s = 0.f, dp = 0.f;
+    for (int e = lane; e < dh; e += 32) {
+      s += q[e] * k[e];
+      dp += dav[e] * v[e];
+    }
+    s = warp_sum(s);
+    dp = warp_sum(dp);
+    const float p = expf(s * scale - L);
+    const float ds = p * (dp - delta);
+    float* dk = temp ? dq + d : dK + ((size_t)i * B + b) * d + h * dh;
+    float* dv = temp ? dq + 2 * d : dV + ((size_t)i * B + b) * d + h * dh;
+    for (int e = lane, c = 0; e < dh; e += 32, ++c) {
+      dqr[c] += scale * ds * k[e];
+      if (temp) {
+        dk[e] = scale * ds * q[e];
+        dv[e] = p * dav[e];
+      } else {
+        dk[e] += scale * ds * q[e];
+        dv[e] += p * dav[e];
+      }
+    }
+  }
+  for (int e = lane, c = 0; e < dh; e += 32, ++c) dq[e] = dqr[c];
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+struct BwdPlan {
+  size_t off_err, off_xp, off_xr, off_cx, off_qkv, off_a, off_lse, off_u, off_ur, off_cu, off_hp, off_g, off_zp,
+      off_zr, off_cz, off_dzu, off_dKa, off_dVa, off_dZ, off_dH, off_dU, off_dA, off_dqkv, off_dzr, off_dg,
+      off_dur, off_dxr, off_dxp, total;
+};
+
+static size_t al(size_t x) { return (x + 255) / 256 * 256; }
+
+static BwdPlan bwd_plan(int B, int N, int d, int H, int d_ff) {
+  BwdPlan P;
+  std::memset(&P, 0, sizeof(P));
+  const size_t R = (size_t)B * N, f = 4;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off += al(bytes); return o; };
+  P.off_err = take(256);
+  P.off_xp = take(R * d * f);
+  P.off_xr = take(R * d * f);
+  P.off_cx = take(R * f);
+  P.off_qkv = take(R * 3 * d * f);
+  P.off_a = take(R * d * f);
+  P.off_lse = take(R * H * f);
+  P.off_u = take(R * d * f);
+  P.off_ur = take(R * d * f);
+  P.off_cu = take(R * f);
+  P.off_hp = take(R * d_ff * f);
+  P.off_g = take(R * d_ff * f);
+  P.off_zp = take(R * d * f);
+  P.off_zr = take(R * d * f);
+  P.off_cz = take(R * f);
+  P.off_dzu = take(R * d * f);
+  P.off_dKa = take(R * d * f);
+  P.off_dVa = take(R * d * f);
+  P.off_dZ = take(R * d * f);
+  P.off_dH = take(R * d_ff * f);
+  P.off_dU = take(R * d * f);
+  P.off_dA = take(R * d * f);
+  P.off_dqkv = take(R * 3 * d * f);
+  P.off_dzr = take((size_t)B * d * f);
+  P.off_dg = take((size_t)B * d_ff * f);
+  P.off_dur = take((size_t)B * d * f);
+  P.off_dxr = take(R * d * f);
+  P.off_dxp = take(R * d * f);
+  P.total = off;
+  return P;
+}
+
+static int bwd_validate(int B, int N, int d, int H, int d_ff, int dtype) {
+  if (B <= 0 || N <= 0 || d <= 0 || H <= 0 || d_ff <= 0 || d % H != 0) return RT_ERR_INVALID_ARG;
+  if (dtype != RT_F32) return dtype == RT_BF16 ? RT_ERR_UNSUPPORTED : RT_ERR_INVALID_ARG;
+  const int dh = d / H;
+  if (dh > 128 || (long)B * N > (1l << 24)) return RT_ERR_UNSUPPORTED;
+  return RT_OK;
+}
+
+static cudaError_t gemm(const float* A, int lda, int ta, const float* W, int ldw, int tw, float* C, int ldc, int M,
+                        int N, int K, int acc, cudaStream_t st) {
+  dim3 grid((N + 63) / 64, (M + 63) / 64);
+  k_gemm<<<grid, 256, 0, st>>>(A, lda, ta, W, ldw, tw, C, ldc, M, N, K, acc);
+  return cudaGetLastError();
+}
+
+static unsigned grid_for(size_t n) { return (unsigned)std::min<size_t>((n + 255) / 256, 65535); }
+
+}  // namespace bwd
+}  // namespace rt
+
+using namespace rt;
+using namespace rt::bwd;
+
+extern "C" size_t rt_layer_backward_workspace_bytes(int B, int N, int d, int H, int d_ff, int dtype) {
+  if (bwd_validate(B, N, d, H, d_ff, dtype) != RT_OK) return 0;
+  return bwd_plan(B, N, d, H, d_ff).total;
+}
+
+#define RT_BCK(call)                                    \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return rt::cuda_failure(e_); \
+  } while (0)
+
+extern "C" int rt_layer_backward(const void* x_, const void* Wq_, const void* Wk_, const void* Wv_, const void* Wo_,
+                                 const void* W1_, const void* W2_, const void* z_, const void* K_, const void* V_,
+                                 const void* dz_, const void* dK_, const void* dV_, int B, int N, int d, int H,
+                                 int d_ff, int dtype, void* dx_, void* dWq_, void* dWk_, void* dWv_, void* dWo_,
+                                 void* dW1_, void* dW2_, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = bwd_validate(B, N, d, H, d_ff, dtype);
+  if (rc != RT_OK) return rc;
+  const void* in[13] = {x_, Wq_, Wk_, Wv_, Wo_, W1_, W2_, z_, K_, V_, dz_, dK_, dV_};
+  void* out[7] = {dx_, dWq_, dWk_, dWv_, dWo_, dW1_, dW2_};
+  for (const void* p : in)
+    if (!p) return RT_ERR_INVALID_ARG;
+  for (void* p : out)
+    if (!p) return RT_ERR_INVALID_ARG;
+  const BwdPlan P = bwd_plan(B, N, d, H, d_ff);
+  if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return RT_ERR_WORKSPACE;
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) !=
+                                                cudaSuccess || major != 10)
+    return RT_ERR_DEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  const float *x = static_cast<const float*>(x_), *z = static_cast<const float*>(z_);
+  const float *Wq = static_cast<const float*>(Wq_), *Wk = static_cast<const float*>(Wk_),
+              *Wv = static_cast<const float*>(Wv_), *Wo = static_cast<const float*>(Wo_),
+              *W1 = static_cast<const float*>(W1_), *W2 = static_cast<const float*>(W2_);
+  const float *K = static_cast<const float*>(K_), *V = static_cast<const float*>(V_);
+  const float *dz = static_cast<const float*>(dz_), *dK = static_cast<const float*>(dK_),
+              *dV = static_cast<const float*>(dV_);
+  float *dx = static_cast<float*>(dx_), *dWq = static_cast<float*>(dWq_), *dWk = static_cast<float*>(dWk_),
+        *dWv = static_cast<float*>(dWv_), *dWo = static_cast<float*>(dWo_), *dW1 = static_cast<float*>(dW1_),
+        *dW2 = static_cast<float*>(dW2_);
+  float *xp = F(P.off_xp), *xr = F(P.off_xr), *cx = F(P.off_cx), *qkv = F(P.off_qkv), *a = F(P.off_a),
+        *lse = F(P.off_lse), *u = F(P.off_u), *ur = F(P.off_ur), *cu = F(P.off_cu), *hp = F(P.off_hp),
+        *g = F(P.off_g), *zp = F(P.off_zp), *zr = F(P.off_zr), *cz = F(P.off_cz), *dzu = F(P.off_dzu),
+        *dKa = F(P.off_dKa), *dVa = F(P.off_dVa), *dZ = F(P.off_dZ), *dH = F(P.off_dH), *dU = F(P.off_dU),
+        *dA = F(P.off_dA), *dqkv = F(P.off_dqkv), *dzr = F(P.off_dzr), *dg = F(P.off_dg), *dur = F(P.off_dur),
+        *dxr = F(P.off_dxr), *dxp = F(P.off_dxp);
+  const size_t R = (size_t)B * N;
+  const int dh = d / H;
+  const float scale = 1.f / std::sqrt((float)dh);
+  const unsigned rows_grid = (unsigned)((R + 7) / 8);
+
+  // 1. rebuild the forward's intermediates, all positions at once
+  k_permute<<<grid_for(R * d), 256, 0, st>>>(x, xp, B, N, d, 1);
+  k_permute<<<grid_for(R * d), 256, 0, st>>>(z, zp, B, N, d, 1);
+  k_permute<<<grid_for(R * d), 256, 0, st>>>(dz, dzu, B, N, d, 1);
+  RT_BCK(cudaGetLastError());
+  k_rms_rows<<<rows_grid, 256, 0, st>>>(xp, xr, cx, R, d, kEps);
+  k_rms_rows<<<rows_grid, 256, 0, st>>>(zp, zr, cz, R, d, kEps);
+  RT_BCK(cudaGetLastError());
+  RT_BCK(gemm(xr, d, 0, Wq, d, 0, qkv, 3 * d, (int)R, d, d, 0, st));
+  RT_BCK(gemm(xr, d, 0, Wk, d, 0, qkv + d, 3 * d, (int)R, d, d, 0, st));
+  RT_BCK(gemm(xr, d, 0, Wv, d, 0, qkv + 2 * d, 3 * d, (int)R, d, d, 0, st));
+  k_attn_lse<<<(unsigned)((R * H + 3) / 4), 128, 0, st>>>(qkv, K, V, a, lse, B, N, H, dh, scale);
+  RT_BCK(cudaGetLastError());
+  RT_BCK(cudaMemcpyAsync(u, xp, R * d * 4, cudaMemcpyDeviceToDevice, st));
+  RT_BCK(gemm(a, d, 0, Wo, d, 0, u, d, (int)R, d, d, 1, st));
+  k_rms_rows<<<rows_grid, 256, 0, st>>>(u, ur, cu, R, d, kEps);
+  RT_BCK(cudaGetLastError());
+  RT_BCK(gemm(ur, d, 0, W1, d, 0, hp, d_ff, (int)R, d_ff, d, 0, st));
+  k_gelu<<<grid_for(R * d_ff), 256, 0, st>>>(hp, g, R * d_ff);
+  RT_BCK(cudaGetLastError());
+
+  // 2. reverse loop over positions
+  RT_BCK(cudaMemcpyAsync(dKa, dK, R * d * 4, cudaMemcpyDeviceToDevice, st));
+  RT_BCK(cudaMemcpyAsync(dVa, dV, R * d * 4, cudaMemcpyDeviceToDevice, st));
+  const unsigned brows = (unsigned)((B + 7) / 8);
+  for (int t = N - 1; t >= 0; --t) {
+    const size_t r0 = (size_t)t * B;
+    // d rms(z_t) = dk_t W_k + dv_t W_v; dz_t = dz(upstream) + rms'(z_t)
+    RT_BCK(gemm(dKa + r0 * d, d, 0, Wk, d, 1, dzr, d, B, d, d, 0, st));
+    RT_BCK(gemm(dVa + r0 * d, d, 0, Wv, d, 1, dzr, d, B, d, d, 1, st));
+    k_rms_bwd<<<brows, 256, 0, st>>>(zp + r0 * d, dzr, cz + r0, dzu + r0 * d, dZ + r0 * d, B, d);
+    RT_BCK(cudaGetLastError());
+    // MLP: dh = dz W_2 ; dpre = dh * GELU'(pre) ; d rms(u) = dpre W_1 ; du = dz + rms'(u)
+    RT_BCK(gemm(dZ + r0 * d, d, 0, W2, d_ff, 1, dg, d_ff, B, d_ff, d, 0, st));
+    k_gelu_bwd<<<grid_for((size_t)B * d_ff), 256, 0, st>>>(dg, hp + r0 * d_ff, dH + r0 * d_ff, (size_t)B * d_ff);
+    RT_BCK(cudaGetLastError());
+    RT_BCK(gemm(dH + r0 * d_ff, d_ff, 0, W1, d, 1, dur, d, B, d, d_ff, 0, st));
+    k_rms_bwd<<<brows, 256, 0, st>>>(u + r0 * d, dur, cu + r0, dZ + r0 * d, dU + r0 * d, B, d);
+    RT_BCK(cudaGetLastError());
+    // da = du W_o, then the attention backward of query t
+    RT_BCK(gemm(dU + r0 * d, d, 0, Wo, d, 1, dA + r0 * d, d, B, d, d, 0, st));
+    k_attn_bwd_step<<<(unsigned)((B * H + 3) / 4), 128, 0, st>>>(qkv, K, V, a, lse, dA, dKa, dVa, dqkv, B, H, dh, t,
+                                                                 scale);
+    RT_BCK(cudaGetLastError());
+  }
+
+  // 3. batched: dx and the weight gradients
+  RT_BCK(gemm(dqkv, 3 * d, 0, Wq, d, 1, dxr, d, (int)R, d, d, 0, st));
+  RT_BCK(gemm(dqkv + d, 3 * d, 0, Wk, d, 1, dxr, d, (int)R, d, d, 1, st));
+  RT_BCK(gemm(dqkv + 2 * d, 3 * d, 0, Wv, d, 1, dxr, d, (int)R, d, d, 1, st));
+  k_rms_bwd<<<rows_grid, 256, 0, st>>>(xp, dxr, cx, dU, dxp, R, d);
+  RT_BCK(cudaGetLastError());
+  k_permute<<<grid_for(R * d), 256, 0, st>>>(dxp, dx, B, N, d, 0);
+  RT_BCK(cudaGetLastError());
+  const int Ri = (int)R;
+  RT_BCK(gemm(dqkv, 3 * d, 1, xr, d, 1, dWq, d, d, d, Ri, 0, st));
+  RT_BCK(gemm(dqkv + d, 3 * d, 1, xr, d, 1, dWk, d, d, d, Ri, 0, st));
+  RT_BCK(gemm(dKa, d, 1, zr, d, 1, dWk, d, d, d, Ri, 1, st));
+  RT_BCK(gemm(dqkv + 2 * d, 3 * d, 1, xr, d, 1, dWv, d, d, d, Ri, 0, st));
+  RT_BCK(gemm(dVa, d, 1, zr, d, 1, dWv, d, d, d, Ri, 1, st));
+  RT_BCK(gemm(dU, d, 1, a, d, 1, dWo, d, d, d, Ri, 0, st));
+  RT_BCK(gemm(dH, d_ff, 1, ur, d, 1, dW1, d, d_ff, d, Ri, 0, st));
+  RT_BCK(gemm(dZ, d, 1, g, d_ff, 1, dW2, d_ff, d, d_ff, Ri, 0, st));
+  return RT_OK;
+}

@@ -31,7 +31,7 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_erro
            "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc",
            "rt_selftest_wait_timeout", "rt_layer_decode_workspace_bytes", "rt_layer_decode_step",
            "rt_project_qkv_noalloc_status", "rt_layer_recompute_workspace_bytes", "rt_layer_recompute_kv",
-           "rt_layer_forward_pages")
+           "rt_layer_forward_pages", "rt_layer_backward_workspace_bytes", "rt_layer_backward")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma")
@@ -79,6 +79,10 @@ def lib() -> ctypes.CDLL:
     L.rt_layer_forward.argtypes = fwd_args
     L.rt_layer_forward_host.restype = i
     L.rt_layer_forward_host.argtypes = fwd_args
+    L.rt_layer_backward_workspace_bytes.restype = sz
+    L.rt_layer_backward_workspace_bytes.argtypes = [i] * 6
+    L.rt_layer_backward.restype = i
+    L.rt_layer_backward.argtypes = [vp] * 13 + [i] * 6 + [vp] * 8 + [sz, vp]
     L.rt_layer_forward_pages.restype = i
     L.rt_layer_forward_pages.argtypes = [vp] * 7 + [i] * 6 + [vp] * 4 + [sz, vp]
     L.rt_layer_sync_status.restype = i
@@ -217,6 +221,34 @@ def layer_forward_pages(x: torch.Tensor, W: dict, H: int, L: int = 1, out=None,
                                       ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("rt_layer_forward_pages", rc)
     return z, K, V
+
+
+def layer_backward(x: torch.Tensor, W: dict, H: int, z: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                   dz: torch.Tensor, dK: torch.Tensor, dV: torch.Tensor, workspace: torch.Tensor | None = None,
+                   stream=None):
+    """rt_layer_backward (fp32): gradients of sum(z*dz) + sum(K*dK) + sum(V*dV)
+    for x [B, N, d], the weights W, the forward's outputs z [B, N, d] and
+    K, V [N, B, d] (position-major), and upstream dz, dK, dV of the same
+    shapes. Returns (dx, {name: dW})."""
+    B, N, d = x.shape
+    d_ff = W["W_1"].shape[0]
+    tensors = (x, z, K, V, dz, dK, dV, *[W[n] for n in WEIGHT_NAMES])
+    for tsr in tensors:
+        if tsr.dtype != torch.float32 or not tsr.is_contiguous() or tsr.device != x.device:
+            raise ValueError("backward tensors must be contiguous fp32 tensors on one device")
+    dx = torch.empty_like(x)
+    dW = {n: torch.empty_like(W[n]) for n in WEIGHT_NAMES}
+    nbytes = int(lib().rt_layer_backward_workspace_bytes(B, N, d, H, d_ff, RT_F32))
+    if nbytes == 0:
+        raise RTError("rt_layer_backward_workspace_bytes", RT_ERR_UNSUPPORTED)
+    if workspace is None:
+        workspace = alloc_workspace(nbytes, x.device)
+    rc = lib().rt_layer_backward(_ptr(x), *[_ptr(W[n]) for n in WEIGHT_NAMES], _ptr(z), _ptr(K), _ptr(V),
+                                 _ptr(dz), _ptr(dK), _ptr(dV), B, N, d, H, d_ff, RT_F32, _ptr(dx),
+                                 *[_ptr(dW[n]) for n in WEIGHT_NAMES], _ptr(workspace),
+                                 ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("rt_layer_backward", rc)
+    return dx, dW
 
 
 def launch_count(B, N, d, H, d_ff, dtype=torch.bfloat16, schedule="blocked") -> int:

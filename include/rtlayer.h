@@ -200,6 +200,41 @@ int rt_layer_recompute_kv(const void* z_dev, const void* W_k_dev, const void* W_
                           int B, int N, int d, void* K_dev, void* V_dev,
                           void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* Device bytes rt_layer_backward needs; 0 if unsupported (RT_F32 only,
+ * d_h <= 128). */
+size_t rt_layer_backward_workspace_bytes(int B, int N, int d, int H, int d_ff, int dtype);
+
+/* Backward pass of the layer (paper §6.4, whose body is missing from the
+ * extracted text: these are the exact derivatives of the forward of paper
+ * §2.2), fp32 storage and arithmetic (RT_F32; RT_BF16 returns
+ * RT_ERR_UNSUPPORTED). Gradients of the scalar
+ *   sum(z * dz) + sum(K * dK) + sum(V * dV)
+ * with respect to x and the six weights, given the forward's inputs and its
+ * stored outputs:
+ *   x_dev, z_dev, dz_dev : [B][N][d];  K_dev, V_dev, dK_dev, dV_dev :
+ *   position-major [N][B][d] (as rt_layer_forward returns K and V);
+ *   weights as in rt_layer_forward.
+ * Outputs: dx_dev [B][N][d]; dW_*_dev with the shapes of the weights
+ * (overwritten, not accumulated).
+ * Method: every intermediate of the forward is rebuilt from (x, z, K, V) in
+ * parallel (paper §6.1, activation checkpointing); a reverse loop over
+ * positions carries the gradient of each persistent pair back through z_t,
+ * the MLP, W_o and the attention of query t (whose contributions to the
+ * pairs of earlier positions are added in place); dx and the weight
+ * gradients are then formed for all positions at once (the backward batched
+ * outside the loop, notes §5.3).
+ * workspace_dev: >= rt_layer_backward_workspace_bytes(...) bytes, 256-byte
+ * aligned. Enqueued on `stream`. */
+int rt_layer_backward(const void* x_dev,
+                      const void* W_q_dev, const void* W_k_dev, const void* W_v_dev,
+                      const void* W_o_dev, const void* W_1_dev, const void* W_2_dev,
+                      const void* z_dev, const void* K_dev, const void* V_dev,
+                      const void* dz_dev, const void* dK_dev, const void* dV_dev,
+                      int B, int N, int d, int H, int d_ff, int dtype,
+                      void* dx_dev, void* dW_q_dev, void* dW_k_dev, void* dW_v_dev,
+                      void* dW_o_dev, void* dW_1_dev, void* dW_2_dev,
+                      void* workspace_dev, size_t workspace_bytes, void* stream);
+
 /* Token-embedding front end of a layer stack: x[b][n][:] = E[ids[b][n]][:].
  * Paper §6.1 stacks layers by feeding each layer's outputs z to the next
  * layer as its inputs; the first layer's inputs are the embedded tokens, so a
