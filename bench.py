@@ -193,6 +193,9 @@ def algorithmic_work(cfg: dict, schedule: str = "blocked") -> dict:
         # position by the last fold into it): q, k~, v~ read, a_1 written (bf16)
         "attend": ("hbm", float(B) * (6 * d + 2 * d)),
     }
+    # the persistent step kernel: the four per-step GEMMs of every step (its
+    # small folds are accounted in fold_level_work)
+    w["steps"] = ("tensor", 2.0 * B * N * (d * d + 2 * d * dff + 2 * d * d))
     if schedule == "naive":
         # query t reads the t-1 persistent pairs (k, v bf16) plus its own q, k~, v~; writes a_t
         w["attend"] = ("hbm", float(B) * (4 * d * N * (N - 1) / 2 + N * 8 * d))

@@ -34,7 +34,7 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_erro
            "rt_layer_forward_pages", "rt_layer_backward_workspace_bytes", "rt_layer_backward")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
-                  "fold_warp", "fold_mma")
+                  "fold_warp", "fold_mma", "steps")
 RT_KC_FOLD_LEVEL0 = 16
 RT_KC_COUNT = 32
 
