@@ -603,7 +603,7 @@ __global__ void __launch_bounds__(128)
     k_fold_mma(const __nv_bfloat16* __restrict__ Q, int q_stride, const __nv_bfloat16* __restrict__ K,
                const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m,
                float* __restrict__ l, float* __restrict__ o, __nv_bfloat16* __restrict__ a_out, int B, int H,
-               int q0, int nq, int k0, int nk, float sc2, int init, int fin) {
+               int q0, int nq, int k0, int nk, float sc2, int init, int fin, unsigned* err) {
   using namespace mma_detail;
   constexpr int DH = 64, QT = 64, KC = 64, QTP = QT / P, KCP = KC / P;
   __shared__ __align__(128) __nv_bfloat16 sQ[QT * LDS];
@@ -758,6 +758,8 @@ __global__ void __launch_bounds__(128)
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
     const int r = wq0 + (lane >> 2) + rr * 8;             // query row within the pair
     if (r >= nrows) continue;
+    // (uniform across the four lanes of a row, like the test above)
+    if (!idx_ok(qt0 + r >= q0 && qt0 + r < q0 + nq && b < B && h < H, err)) continue;
     const size_t row = (size_t)(qt0 + r) * B + b;
     float mg = -INFINITY, lg = 0.f;
     if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }

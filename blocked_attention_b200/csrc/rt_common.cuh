@@ -37,6 +37,21 @@ __device__ __forceinline__ void set_error(unsigned* err, unsigned bits) {
   if (err) atomicOr(err, bits);
 }
 
+// Debug build (compiled with -DRT_BOUNDS_CHECK, library librtlayer_check.so):
+// the global indexes the layer's kernels compute are checked against the
+// ranges their arguments declare; a failed check records RT_DEVERR_INDEX in
+// the error word (rt_layer_sync_status then returns RT_ERR_INVALID_ARG) and
+// the access is skipped. Nothing traps. In the normal build the check is the
+// constant true and compiles away.
+#ifdef RT_BOUNDS_CHECK
+__device__ __forceinline__ bool idx_ok(bool ok, unsigned* err) {
+  if (!ok) set_error(err, RT_DEVERR_INDEX);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool idx_ok(bool, unsigned*) { return true; }
+#endif
+
 // ---------------------------------------------------------------------------
 // programmatic dependent launch: a kernel launched with programmatic stream
 // serialisation may start while its predecessor runs; it must call

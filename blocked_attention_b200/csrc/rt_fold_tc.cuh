@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(192, 1)
       int b, h, qt0;
       item_of(li, b, h, qt0);
       const int nrows = min(C::QT, q0 + nq - qt0);
-      if (r < nrows) {
+      if (r < nrows && idx_ok(qt0 + r >= q0 && qt0 + r < q0 + nq && b < B && h < H, err)) {
         const size_t row = (size_t)(qt0 + r) * B + b;
         float mg = -INFINITY, lg = 0.f;
         float* op = o + row * (size_t)d + h * C::DH;
@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(320, 1)
       item_of(li, b, h, st0);
       const int qt0 = st0 + t * C::QT;
       const int nrows = min(C::QT, q0 + nq - qt0);   // may be <= 0 for an empty tile B
-      if (r < nrows) {
+      if (r < nrows && idx_ok(qt0 + r >= q0 && qt0 + r < q0 + nq && b < B && h < H, err)) {
         const size_t row = (size_t)(qt0 + r) * B + b;
         float mg = -INFINITY, lg = 0.f;
         float* op = o + row * (size_t)d + h * C::DH;

@@ -206,6 +206,8 @@ __device__ __forceinline__ GemmTask decode_gemm(const GemmPhase& g, int loc) {
 }
 
 __device__ __forceinline__ unsigned* flag_ptr(const StepsParams& P, int ph, int rb, int i) {
+  if (!idx_ok(ph >= 0 && ph < PH_COUNT && rb >= 0 && rb < P.nrb && i >= 0 && i < kFlagStride, P.err))
+    i = 0, rb = 0, ph = 0;   // (debug build) a bad flag index reads flag 0 instead
   return P.flags + ((size_t)(ph * P.nrb + rb) * kFlagStride + i);
 }
 
@@ -245,20 +247,23 @@ __device__ __forceinline__ void fold_small_units(const StepsParams& P, int q0, i
     uint4 qw[R], kw[R][NK], vw[R][NK], ktw[R], vtw[R];
     float4 oa[R], ob[R];
     float mo[R], lo[R];
+    bool live[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int u = u0 + r * 16 + oct;
-      const bool act = u < U;
+      bool act = u < U;
       const int s = act ? u / nq : 0, qi = act ? u - s * nq : 0;
       const int b = s0 + s;
       const size_t row = (size_t)(q0 + qi) * B + b;
       const __nv_bfloat16* qp = P.qkv + row * (size_t)(3 * d) + h * 64 + sl * 8;
       qw[r] = ktw[r] = vtw[r] = make_uint4(0, 0, 0, 0);
+      act = act && idx_ok(b < B && q0 + qi < P.ep.Nseq && k0 >= 0 && k0 + NK <= q0 && h < H, P.err);
       oa[r] = ob[r] = make_float4(0.f, 0.f, 0.f, 0.f);
       mo[r] = -INFINITY;
       lo[r] = 0.f;
 #pragma unroll
       for (int i = 0; i < NK; ++i) kw[r][i] = vw[r][i] = make_uint4(0, 0, 0, 0);
+      live[r] = act;
       if (act) {
         // k, v, m, l and o were written by other CTAs of this kernel: loads
         // through L2 only (no stale L1 lines); q and the temporary pair come
@@ -286,7 +291,7 @@ __device__ __forceinline__ void fold_small_units(const StepsParams& P, int q0, i
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int u = u0 + r * 16 + oct;
-      if (u >= U) continue;   // whole octets together; shuffles stay inside the octet
+      if (!live[r]) continue;   // whole octets together; shuffles stay inside the octet
       const int s = u / nq, qi = u - s * nq;
       const int b = s0 + s;
       const size_t row = (size_t)(q0 + qi) * B + b;
@@ -586,8 +591,9 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
       ++local;
       const int row = T.rb * C::BM + lrow;
-      const bool row_ok = row < P.ep.B;
       const int col_base = T.tile * g.BN;
+      const bool row_ok = row < P.ep.B &&
+                          idx_ok(T.rb < P.nrb && col_base + g.BN <= g.N && T.sl1 <= g.K / 64 && j < P.ep.Nseq, P.err);
       // dependencies of what this epilogue reads or overwrites (see the file comment)
       if (ph == PH_WO) {
         if (j > P.j0) epi_poll_range(P, PH_FOLD, T.rb, 0, P.H * P.G, (unsigned)j, tid);
