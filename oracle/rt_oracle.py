@@ -297,6 +297,58 @@ def rt_layer_pages(x: np.ndarray, W: dict, H: int, L: int = 1, kv_source: str = 
 
 
 # --------------------------------------------------------------------------
+# block-wise (chunked) recurrence
+# --------------------------------------------------------------------------
+def rt_layer_chunked(x: np.ndarray, W: dict, H: int, C: int):
+    """RT layer with the recurrence executed block-wise, in chunks of C
+    positions [RT notes §8 and paper §9 (discussion and conclusion): running the recurrence over blocks of steps
+    trades depth for speed; named as future work without a definition].
+
+    Reading (ours): the positions are cut into consecutive chunks of C; a
+    position's persistent pair (from its output z) becomes visible only to
+    the positions of later chunks, and inside its own chunk a position
+    attends to the temporary pairs (from the inputs x) of the chunk's
+    positions up to and including itself. Per position t of chunk c
+    (positions c*C .. c*C + C - 1):
+        keys = {(k_i, v_i): i < c*C} + {(k~_s, v~_s): c*C <= s <= t}
+    and everything else is the layer of rt_layer. C = 1 is rt_layer itself;
+    C >= N is the standard causal Transformer layer of [RT paper §2.1] (every
+    pair temporary), whose persistent pairs are then W_{k,v} RMS(z).
+    Naive schedule, fp64. Returns (z, K, V), each [B, N, d].
+    """
+    if C < 1:
+        raise ValueError("chunk length C >= 1")
+    x = np.asarray(x, dtype=np.float64)
+    B, N, d = x.shape
+    dh = d // H
+    scale = 1.0 / np.sqrt(dh)
+    z = np.empty_like(x)
+    Kp = np.empty((B, H, N, dh))
+    Vp = np.empty((B, H, N, dh))
+    r = rms(x)
+    Qt = _heads(r @ W["W_q"].T, H)              # [B, N, H, dh]
+    Kt = _heads(r @ W["W_k"].T, H)
+    Vt = _heads(r @ W["W_v"].T, H)
+    for c0 in range(0, N, C):
+        c1 = min(N, c0 + C)
+        for t in range(c0, c1):
+            keys = np.concatenate([Kp[:, :, :c0], Kt[:, c0:t + 1].transpose(0, 2, 1, 3)], axis=2)
+            vals = np.concatenate([Vp[:, :, :c0], Vt[:, c0:t + 1].transpose(0, 2, 1, 3)], axis=2)
+            sc = np.einsum("bhe,bhie->bhi", Qt[:, t], keys) * scale
+            sc = sc - sc.max(axis=-1, keepdims=True)
+            w = np.exp(sc)
+            a = np.einsum("bhi,bhie->bhe", w, vals) / w.sum(axis=-1)[..., None]
+            u = x[:, t] + a.reshape(B, d) @ W["W_o"].T
+            z[:, t] = u + mlp(u, W)
+        rz = rms(z[:, c0:c1])                    # the chunk's persistent pairs, revealed together
+        Kp[:, :, c0:c1] = _heads(rz @ W["W_k"].T, H).transpose(0, 2, 1, 3)
+        Vp[:, :, c0:c1] = _heads(rz @ W["W_v"].T, H).transpose(0, 2, 1, 3)
+    K = Kp.transpose(0, 2, 1, 3).reshape(B, N, d)
+    V = Vp.transpose(0, 2, 1, 3).reshape(B, N, d)
+    return z, K, V
+
+
+# --------------------------------------------------------------------------
 # blocked (lowbit) schedule, in the pages' order
 # --------------------------------------------------------------------------
 def lowbit_blocks(N: int):

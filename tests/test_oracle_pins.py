@@ -490,3 +490,55 @@ def test_embedding_lookup_row_by_row():
     # row 0 of the table is -3.0, -2.5, ... and row vocab-1 ends at the last entry
     assert list(x[0, 0]) == [-3.0, -2.5, -2.0, -1.5, -1.0]
     assert x[0, 1, -1] == E.flat[-1] == (vocab * d - 1) * 0.5 - 3.0
+
+
+# --------------------------------------------------------------------------
+# block-wise (chunked) recurrence: the two ends of the depth/speed trade-off
+# --------------------------------------------------------------------------
+def test_chunked_recurrence_with_chunks_of_one_is_the_rt_layer():
+    x, W = _problem(2, 13, 32, 2, 64, sigma=0.2)
+    got = O.rt_layer_chunked(x, W, 2, 1)
+    ref = O.rt_layer(x, W, 2)
+    for g, r in zip(got, ref):
+        assert _relerr(g, r) < 1e-12
+
+
+@pytest.mark.parametrize("N,C", [(9, 9), (9, 16)])
+def test_chunked_recurrence_with_one_chunk_is_the_standard_layer(N, C):
+    # every pair temporary: the causal pre-norm Transformer layer (its own
+    # textbook pin is test_input_kv_source_is_the_textbook_transformer_layer)
+    x, W = _problem(2, N, 32, 2, 64, sigma=0.2)
+    z, K, V = O.rt_layer_chunked(x, W, 2, C)
+    zr, _, _ = O.rt_layer(x, W, 2, kv_source="input")
+    assert _relerr(z, zr) < 1e-12
+    Kr, Vr = O.recompute_kv(z, W)               # persistent pairs of the outputs
+    assert _relerr(K, Kr) < 1e-12 and _relerr(V, Vr) < 1e-12
+
+
+def test_chunked_recurrence_two_positions_closed_form():
+    # N = 2 in one chunk of 2: position 2 sees the TEMPORARY pairs of
+    # positions 1 and 2 (with C = 1 it would see position 1's persistent pair)
+    x, W = _problem(1, 2, 16, 1, 32, sigma=0.3)
+    z, _, _ = O.rt_layer_chunked(x, W, 1, 2)
+    r = O.rms(x[0])
+    q, kt, vt = r @ W["W_q"].T, r @ W["W_k"].T, r @ W["W_v"].T
+    s = np.array([q[1] @ kt[0], q[1] @ kt[1]]) / 4.0
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    a = p[0] * vt[0] + p[1] * vt[1]
+    u = x[0, 1] + W["W_o"] @ a
+    z2 = u + W["W_2"] @ O.gelu(W["W_1"] @ O.rms(u))
+    assert _relerr(z[0, 1], z2) < 1e-12
+    # position 1 attends to its own temporary pair only: a_1 = v~_1
+    u1 = x[0, 0] + W["W_o"] @ vt[0]
+    assert _relerr(z[0, 0], u1 + W["W_2"] @ O.gelu(W["W_1"] @ O.rms(u1))) < 1e-12
+
+
+def test_chunked_recurrence_is_causal_and_chunk_local():
+    x, W = _problem(1, 12, 32, 2, 64, sigma=0.2)
+    z, _, _ = O.rt_layer_chunked(x, W, 2, 4)
+    x2 = x.copy()
+    x2[:, 9] += 1.0                              # chunk 2 (positions 9..12, 1-based)
+    z2, _, _ = O.rt_layer_chunked(x2, W, 2, 4)
+    np.testing.assert_array_equal(z2[:, :9], z[:, :9])
+    assert np.max(np.abs(z2[:, 9:] - z[:, 9:])) > 1e-3
