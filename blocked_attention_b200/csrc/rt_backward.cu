@@ -1,5 +1,7 @@
-// rt_backward.cu -- backward pass of the Recurrent Transformer layer, fp32
-// storage and arithmetic (SIMT; the 1e-4 parity mode).
+// rt_backward.cu -- backward pass of the Recurrent Transformer layer: fp32
+// arithmetic (SIMT), fp32 storage (the 1e-4 parity mode) or bf16 storage
+// (inputs widened to fp32 working copies, gradients rounded to bf16 at the
+// end).
 //
 // Source: "Recurrent Transformer" paper page (www.lshu.cn/news/403416):
 //   paper §2.2 : the layer (queries and temporary pairs from x_t, persistent
@@ -86,6 +88,16 @@ __global__ void __launch_bounds__(256) k_gemm(const float* __restrict__ A, int l
         *dst = accumulate ? *dst + acc[i][j] : acc[i][j];
       }
     }
+}
+
+// dst[i] = float(src[i]) (bf16 storage -> the fp32 working copies) and back
+__global__ void k_bf16_to_f32(const __nv_bfloat16* __restrict__ src, float* __restrict__ dst, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = __bfloat162float(src[i]);
+}
+__global__ void k_f32_to_bf16(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
 }
 
 // dst[n][b][:] = src[b][n][:] (to = 1), or the inverse (to = 0)
@@ -265,6 +277,7 @@ __global__ void __launch_bounds__(128) k_attn_bwd_step(const float* __restrict__
 // host side
 // ---------------------------------------------------------------------------
 struct BwdPlan {
+  size_t off_in, off_out;   // bf16 storage: fp32 copies of the 13 inputs / the 7 outputs
   size_t off_err, off_xp, off_xr, off_cx, off_qkv, off_a, off_lse, off_u, off_ur, off_cu, off_hp, off_g, off_zp,
       off_zr, off_cz, off_dzu, off_dKa, off_dVa, off_dZ, off_dH, off_dU, off_dA, off_dqkv, off_dzr, off_dg,
       off_dur, off_dxr, off_dxp, total;
@@ -272,12 +285,30 @@ struct BwdPlan {
 
 static size_t al(size_t x) { return (x + 255) / 256 * 256; }
 
-static BwdPlan bwd_plan(int B, int N, int d, int H, int d_ff) {
+// element counts of the backward's inputs (x, W_q, W_k, W_v, W_o, W_1, W_2,
+// z, K, V, dz, dK, dV) and outputs (dx, dW_q, dW_k, dW_v, dW_o, dW_1, dW_2)
+static void bwd_counts(int B, int N, int d, int d_ff, size_t (&in)[13], size_t (&out)[7]) {
+  const size_t act = (size_t)B * N * d, dd = (size_t)d * d, df = (size_t)d * d_ff;
+  const size_t i_[13] = {act, dd, dd, dd, dd, df, df, act, act, act, act, act, act};
+  const size_t o_[7] = {act, dd, dd, dd, dd, df, df};
+  for (int i = 0; i < 13; ++i) in[i] = i_[i];
+  for (int i = 0; i < 7; ++i) out[i] = o_[i];
+}
+
+static BwdPlan bwd_plan(int B, int N, int d, int H, int d_ff, int dtype) {
   BwdPlan P;
   std::memset(&P, 0, sizeof(P));
   const size_t R = (size_t)B * N, f = 4;
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off += al(bytes); return o; };
+  if (dtype == RT_BF16) {
+    size_t in[13], out[7], ni = 0, no = 0;
+    bwd_counts(B, N, d, d_ff, in, out);
+    for (size_t c : in) ni += al(c * f);
+    for (size_t c : out) no += al(c * f);
+    P.off_in = take(ni);
+    P.off_out = take(no);
+  }
   P.off_err = take(256);
   P.off_xp = take(R * d * f);
   P.off_xr = take(R * d * f);
@@ -312,7 +343,7 @@ static BwdPlan bwd_plan(int B, int N, int d, int H, int d_ff) {
 
 static int bwd_validate(int B, int N, int d, int H, int d_ff, int dtype) {
   if (B <= 0 || N <= 0 || d <= 0 || H <= 0 || d_ff <= 0 || d % H != 0) return RT_ERR_INVALID_ARG;
-  if (dtype != RT_F32) return dtype == RT_BF16 ? RT_ERR_UNSUPPORTED : RT_ERR_INVALID_ARG;
+  if (dtype != RT_F32 && dtype != RT_BF16) return RT_ERR_INVALID_ARG;
   const int dh = d / H;
   if (dh > 128 || (long)B * N > (1l << 24)) return RT_ERR_UNSUPPORTED;
   return RT_OK;
@@ -335,7 +366,7 @@ using namespace rt::bwd;
 
 extern "C" size_t rt_layer_backward_workspace_bytes(int B, int N, int d, int H, int d_ff, int dtype) {
   if (bwd_validate(B, N, d, H, d_ff, dtype) != RT_OK) return 0;
-  return bwd_plan(B, N, d, H, d_ff).total;
+  return bwd_plan(B, N, d, H, d_ff, dtype).total;
 }
 
 #define RT_BCK(call)                                    \
@@ -357,7 +388,7 @@ extern "C" int rt_layer_backward(const void* x_, const void* Wq_, const void* Wk
     if (!p) return RT_ERR_INVALID_ARG;
   for (void* p : out)
     if (!p) return RT_ERR_INVALID_ARG;
-  const BwdPlan P = bwd_plan(B, N, d, H, d_ff);
+  const BwdPlan P = bwd_plan(B, N, d, H, d_ff, dtype);
   if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return RT_ERR_WORKSPACE;
   int dev = 0, major = 0;
@@ -366,6 +397,29 @@ extern "C" int rt_layer_backward(const void* x_, const void* Wq_, const void* Wk
     return RT_ERR_DEVICE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
+  // bf16 storage: widen the inputs into fp32 working copies, run the fp32
+  // backward on them, round the results to bf16 at the end
+  void* out_dst[7] = {dx_, dWq_, dWk_, dWv_, dWo_, dW1_, dW2_};
+  size_t in_n[13], out_n[7];
+  bwd_counts(B, N, d, d_ff, in_n, out_n);
+  if (dtype == RT_BF16) {
+    size_t o = P.off_in;
+    for (int i = 0; i < 13; ++i) {
+      float* dst = reinterpret_cast<float*>(ws + o);
+      k_bf16_to_f32<<<grid_for(in_n[i]), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in[i]), dst, in_n[i]);
+      in[i] = dst;
+      o += al(in_n[i] * 4);
+    }
+    o = P.off_out;
+    for (int i = 0; i < 7; ++i) {
+      out[i] = ws + o;
+      o += al(out_n[i] * 4);
+    }
+    RT_BCK(cudaGetLastError());
+    x_ = in[0]; Wq_ = in[1]; Wk_ = in[2]; Wv_ = in[3]; Wo_ = in[4]; W1_ = in[5]; W2_ = in[6];
+    z_ = in[7]; K_ = in[8]; V_ = in[9]; dz_ = in[10]; dK_ = in[11]; dV_ = in[12];
+    dx_ = out[0]; dWq_ = out[1]; dWk_ = out[2]; dWv_ = out[3]; dWo_ = out[4]; dW1_ = out[5]; dW2_ = out[6];
+  }
   auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
   const float *x = static_cast<const float*>(x_), *z = static_cast<const float*>(z_);
   const float *Wq = static_cast<const float*>(Wq_), *Wk = static_cast<const float*>(Wk_),
@@ -451,5 +505,11 @@ extern "C" int rt_layer_backward(const void* x_, const void* Wq_, const void* Wk
   RT_BCK(gemm(dU, d, 1, a, d, 1, dWo, d, d, d, Ri, 0, st));
   RT_BCK(gemm(dH, d_ff, 1, ur, d, 1, dW1, d, d_ff, d, Ri, 0, st));
   RT_BCK(gemm(dZ, d, 1, g, d_ff, 1, dW2, d_ff, d, d_ff, Ri, 0, st));
+  if (dtype == RT_BF16) {
+    for (int i = 0; i < 7; ++i)
+      k_f32_to_bf16<<<grid_for(out_n[i]), 256, 0, st>>>(static_cast<const float*>(out[i]),
+                                                       static_cast<__nv_bfloat16*>(out_dst[i]), out_n[i]);
+    RT_BCK(cudaGetLastError());
+  }
   return RT_OK;
 }

@@ -226,25 +226,27 @@ def layer_forward_pages(x: torch.Tensor, W: dict, H: int, L: int = 1, out=None,
 def layer_backward(x: torch.Tensor, W: dict, H: int, z: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                    dz: torch.Tensor, dK: torch.Tensor, dV: torch.Tensor, workspace: torch.Tensor | None = None,
                    stream=None):
-    """rt_layer_backward (fp32): gradients of sum(z*dz) + sum(K*dK) + sum(V*dV)
-    for x [B, N, d], the weights W, the forward's outputs z [B, N, d] and
-    K, V [N, B, d] (position-major), and upstream dz, dK, dV of the same
-    shapes. Returns (dx, {name: dW})."""
+    """rt_layer_backward: gradients of sum(z*dz) + sum(K*dK) + sum(V*dV) for
+    x [B, N, d], the weights W, the forward's outputs z [B, N, d] and K, V
+    [N, B, d] (position-major), and upstream dz, dK, dV of the same shapes;
+    all fp32 or all bf16 (fp32 arithmetic either way). Returns
+    (dx, {name: dW})."""
     B, N, d = x.shape
     d_ff = W["W_1"].shape[0]
+    code = _dtype_code(x.dtype)
     tensors = (x, z, K, V, dz, dK, dV, *[W[n] for n in WEIGHT_NAMES])
     for tsr in tensors:
-        if tsr.dtype != torch.float32 or not tsr.is_contiguous() or tsr.device != x.device:
-            raise ValueError("backward tensors must be contiguous fp32 tensors on one device")
+        if tsr.dtype != x.dtype or not tsr.is_contiguous() or tsr.device != x.device:
+            raise ValueError("backward tensors must be contiguous tensors of one dtype on one device")
     dx = torch.empty_like(x)
     dW = {n: torch.empty_like(W[n]) for n in WEIGHT_NAMES}
-    nbytes = int(lib().rt_layer_backward_workspace_bytes(B, N, d, H, d_ff, RT_F32))
+    nbytes = int(lib().rt_layer_backward_workspace_bytes(B, N, d, H, d_ff, code))
     if nbytes == 0:
         raise RTError("rt_layer_backward_workspace_bytes", RT_ERR_UNSUPPORTED)
     if workspace is None:
         workspace = alloc_workspace(nbytes, x.device)
     rc = lib().rt_layer_backward(_ptr(x), *[_ptr(W[n]) for n in WEIGHT_NAMES], _ptr(z), _ptr(K), _ptr(V),
-                                 _ptr(dz), _ptr(dK), _ptr(dV), B, N, d, H, d_ff, RT_F32, _ptr(dx),
+                                 _ptr(dz), _ptr(dK), _ptr(dV), B, N, d, H, d_ff, code, _ptr(dx),
                                  *[_ptr(dW[n]) for n in WEIGHT_NAMES], _ptr(workspace),
                                  ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("rt_layer_backward", rc)

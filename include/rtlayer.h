@@ -200,14 +200,15 @@ int rt_layer_recompute_kv(const void* z_dev, const void* W_k_dev, const void* W_
                           int B, int N, int d, void* K_dev, void* V_dev,
                           void* workspace_dev, size_t workspace_bytes, void* stream);
 
-/* Device bytes rt_layer_backward needs; 0 if unsupported (RT_F32 only,
- * d_h <= 128). */
+/* Device bytes rt_layer_backward needs; 0 if unsupported (d_h <= 128). */
 size_t rt_layer_backward_workspace_bytes(int B, int N, int d, int H, int d_ff, int dtype);
 
 /* Backward pass of the layer (paper §6.4, whose body is missing from the
  * extracted text: these are the exact derivatives of the forward of paper
- * §2.2), fp32 storage and arithmetic (RT_F32; RT_BF16 returns
- * RT_ERR_UNSUPPORTED). Gradients of the scalar
+ * §2.2), fp32 arithmetic; storage RT_F32, or RT_BF16 (every input and
+ * output bf16; the inputs are widened to fp32 working copies inside the
+ * workspace and the gradients rounded to bf16 at the end). Gradients of the
+ * scalar
  *   sum(z * dz) + sum(K * dK) + sum(V * dV)
  * with respect to x and the six weights, given the forward's inputs and its
  * stored outputs:
