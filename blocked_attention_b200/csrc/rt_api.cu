@@ -280,7 +280,13 @@ struct Shape {
   // and keys, no softmax scale, RMS without eps, branches scaled by
   // 1/sqrt(L)); 0: the single-layer configuration
   int pages = 0, L = 1;
+  // chunk > 0: the block-wise recurrence with chunks of `chunk` positions
+  // (a position's persistent pair is seen from the next chunk on; inside a
+  // chunk, causal attention over the temporary pairs); 0: per position
+  int chunk = 0;
   int dh() const { return d / H; }
+  // rows of the per-step GEMMs: B sequences x positions per step
+  int step_rows() const { return chunk > 0 ? B * std::min(chunk, N) : B; }
   float eps() const { return pages ? 0.f : kEps; }
   // softmax scale in log2 units: log2(e) / sqrt(d_h), or log2(e) unscaled
   float sc2() const { return pages ? kLog2e : kLog2e / std::sqrt((float)dh()); }
@@ -301,6 +307,9 @@ static int validate(const Shape& s) {
     if (dh != 64 || s.d % 64 != 0 || s.d_ff % 64 != 0) return RT_ERR_UNSUPPORTED;
   }
   if (s.pages && (s.dtype != RT_BF16 || s.schedule != RT_SCHED_BLOCKED)) return RT_ERR_UNSUPPORTED;
+  if (s.chunk < 0) return RT_ERR_INVALID_ARG;
+  if (s.chunk > 0 && (s.dtype != RT_BF16 || s.schedule != RT_SCHED_BLOCKED || s.pages)) return RT_ERR_UNSUPPORTED;
+  if ((long)s.step_rows() * s.d_ff > (1l << 31)) return RT_ERR_UNSUPPORTED;
   if (s.L < 1) return RT_ERR_INVALID_ARG;
   return RT_OK;
 }
@@ -317,7 +326,7 @@ struct StepsPlan {
 static StepsPlan plan_steps(const Shape& s) {
   StepsPlan sp;
   std::memset(&sp, 0, sizeof(sp));
-  if (s.dtype != RT_BF16 || s.schedule != RT_SCHED_BLOCKED) return sp;
+  if (s.dtype != RT_BF16 || s.schedule != RT_SCHED_BLOCKED || s.chunk > 0) return sp;
   const int d = s.d, dff = s.d_ff;
   auto phase = [](int N, int K, int BN, int S) { return GemmPhase{N, K, BN, S, N / BN}; };
   // W_o: 64-wide tiles (short tasks on the critical path); W_1, W_2, W_kv:
@@ -351,7 +360,7 @@ static Plan make_plan(const Shape& s) {
   std::memset(&P, 0, sizeof(P));
   P.s = s;
   P.esz = s.dtype == RT_BF16 ? 2 : 4;
-  const size_t rows = (size_t)s.B * s.N, d = s.d, B = s.B;
+  const size_t rows = (size_t)s.B * s.N, d = s.d, B = (size_t)s.step_rows();   // B: rows per step
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -385,10 +394,11 @@ static Plan make_plan(const Shape& s) {
     P.off_w2part = take((size_t)P.sp.nrb * g2.tiles * g2.S * g2.BN * StepsCfg::BM * 4);
   }
   if (s.dtype == RT_BF16) {
-    P.t_wo = choose_tiles(s.B, s.d, s.d, kLayerSplitK);
-    P.t_w1 = choose_tiles(s.B, s.d_ff, s.d, kLayerSplitK);
-    P.t_w2 = choose_tiles(s.B, s.d, s.d_ff, kLayerSplitK);
-    P.t_wkv = choose_tiles(s.B, 2 * s.d, s.d, kLayerSplitK);
+    const int M = s.step_rows();
+    P.t_wo = choose_tiles(M, s.d, s.d, kLayerSplitK);
+    P.t_w1 = choose_tiles(M, s.d_ff, s.d, kLayerSplitK);
+    P.t_w2 = choose_tiles(M, s.d, s.d_ff, kLayerSplitK);
+    P.t_wkv = choose_tiles(M, 2 * s.d, s.d, kLayerSplitK);
   }
   P.total = off;
   return P;
@@ -860,8 +870,119 @@ static int enqueue_f32(const Plan& P, const Ptrs& X, cudaStream_t st, Timer* T) 
   return RT_OK;
 }
 
+// ---------------------------------------------------------------------------
+// block-wise (chunked) recurrence, bf16: per chunk of C positions, the
+// chunk's attention (fold state + causal temporary pairs), the four GEMMs at
+// M = B * C rows (position-major), and the dyadic block fold at chunk
+// granularity: when chunk cc (1-based) has revealed its persistent pairs,
+// the pairs of chunks (cc - lb, cc] are folded into the queries of chunks
+// (cc, cc + lb], lb = lowbit(cc).
+// ---------------------------------------------------------------------------
+static int enqueue_chunked(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st, Timer* T) {
+  const Shape& s = P.s;
+  char* ws = static_cast<char*>(X.ws);
+  unsigned* err = reinterpret_cast<unsigned*>(ws + P.off_err);
+  bf16* qkv = reinterpret_cast<bf16*>(ws + P.off_qkv);
+  float* m = reinterpret_cast<float*>(ws + P.off_m);
+  float* l = reinterpret_cast<float*>(ws + P.off_l);
+  float* o = reinterpret_cast<float*>(ws + P.off_o);
+  float* inv = reinterpret_cast<float*>(ws + P.off_inv);
+  bf16* wqkv = reinterpret_cast<bf16*>(ws + P.off_wqkv);
+  bf16* a16 = reinterpret_cast<bf16*>(ws + P.off_a);
+  bf16* u16 = reinterpret_cast<bf16*>(ws + P.off_u16);
+  bf16* h16 = reinterpret_cast<bf16*>(ws + P.off_h);
+  bf16* z16 = reinterpret_cast<bf16*>(ws + P.off_zs);
+  float* ssq_u = reinterpret_cast<float*>(ws + P.off_ssq_u);
+  float* ssq_z = reinterpret_cast<float*>(ws + P.off_ssq_z);
+  const bf16* x = static_cast<const bf16*>(X.x);
+  bf16* K = static_cast<bf16*>(X.K);
+  bf16* V = static_cast<bf16*>(X.V);
+  const int B = s.B, N = s.N, d = s.d, H = s.H, dff = s.d_ff, C = std::min(s.chunk, s.N);
+  const int Mmax = s.step_rows();
+  const size_t rows = (size_t)B * N, dd = (size_t)d * d * 2;
+  RT_CK(cudaMemsetAsync(err, 0, sizeof(unsigned), st));
+  RT_CK(cudaMemcpyAsync(wqkv, X.Wq, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + dd, X.Wk, dd, cudaMemcpyDeviceToDevice, st));
+  RT_CK(cudaMemcpyAsync(reinterpret_cast<char*>(wqkv) + 2 * dd, X.Wv, dd, cudaMemcpyDeviceToDevice, st));
+  // queries and temporary pairs of every position
+  {
+    TimedScope ts(T, KC_INV_RMS, st);
+    k_row_inv_rms<bf16><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(x, inv, rows, d, kEps);
+  }
+  RT_CK(cudaGetLastError());
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.B = B; ep.Nseq = N; ep.xc = N; ep.d = d; ep.d_ff = dff; ep.eps = kEps;
+  ep.inv_rms = inv; ep.qkv = qkv; ep.x = x; ep.u32 = reinterpret_cast<float*>(ws + P.off_u32); ep.u16 = u16;
+  ep.h16 = h16; ep.zout = static_cast<bf16*>(X.z); ep.z16 = z16; ep.Kout = K; ep.Vout = V;
+  {
+    const int bn_p = choose_bn((int)rows, 3 * d);
+    CUtensorMap tA_x, tB_qkv;
+    if (!make_tmap(&tA_x, x, d, rows, 128) || !make_tmap(&tB_qkv, wqkv, d, 3 * d, bn_p)) return RT_ERR_INVALID_ARG;
+    TimedScope ts(T, KC_PROJ, st);
+    RT_CK(launch_tc<EPI_PROJ>(bn_p, tA_x, tB_qkv, (int)rows, 3 * d, d, ep, err, ds.sms, st));
+  }
+  const int bn_o = P.t_wo.bn, bn_1 = P.t_w1.bn, bn_2 = P.t_w2.bn, bn_kv = P.t_wkv.bn;
+  CUtensorMap tA_a, tB_o, tA_u, tB_1, tA_h, tB_2, tA_z, tB_kv;
+  if (!make_tmap(&tA_a, a16, d, Mmax, 128) || !make_tmap(&tB_o, X.Wo, d, d, bn_o) ||
+      !make_tmap(&tA_u, u16, d, Mmax, 128) || !make_tmap(&tB_1, X.W1, d, dff, bn_1) ||
+      !make_tmap(&tA_h, h16, dff, Mmax, 128) || !make_tmap(&tB_2, X.W2, dff, d, bn_2) ||
+      !make_tmap(&tA_z, z16, d, Mmax, 128) || !make_tmap(&tB_kv, wqkv + (size_t)d * d, d, 2 * d, bn_kv))
+    return RT_ERR_INVALID_ARG;
+  const float sc2 = s.sc2();
+  const int nchunks = (N + C - 1) / C;
+  for (int c = 0; c < nchunks; ++c) {
+    const int p0 = c * C, nc = std::min(C, N - p0), M = B * nc;
+    {
+      TimedScope ts(T, KC_ATTEND, st);
+      const long units = (long)M * H;
+      RT_CK(launch_pdl(k_chunk_attend, dim3((unsigned)((units + 15) / 16)), dim3(128), 0, st,
+                       static_cast<const bf16*>(qkv), static_cast<const float*>(m), static_cast<const float*>(l),
+                       static_cast<const float*>(o), a16, B, H, p0, nc, sc2, c > 0 ? 1 : 0, err));
+    }
+    ep.j = p0;
+    ep.ssq_rows = M;
+    ep.ssq_out = ssq_u;
+    ep.splits = P.t_wo.splits;
+    {
+      TimedScope ts(T, KC_WO, st);
+      RT_CK(launch_tc<EPI_WO>(bn_o, tA_a, tB_o, M, d, d, ep, err, ds.sms, st));
+    }
+    ep.ssq_in = ssq_u; ep.ssq_tiles = (d + bn_o - 1) / bn_o;
+    ep.splits = P.t_w1.splits;
+    {
+      TimedScope ts(T, KC_W1, st);
+      RT_CK(launch_tc<EPI_W1>(bn_1, tA_u, tB_1, M, dff, d, ep, err, ds.sms, st));
+    }
+    ep.ssq_out = ssq_z;
+    ep.splits = P.t_w2.splits;
+    {
+      TimedScope ts(T, KC_W2, st);
+      RT_CK(launch_tc<EPI_W2>(bn_2, tA_h, tB_2, M, d, dff, ep, err, ds.sms, st));
+    }
+    ep.ssq_in = ssq_z; ep.ssq_tiles = (d + bn_2 - 1) / bn_2;
+    ep.splits = P.t_wkv.splits;
+    {
+      TimedScope ts(T, KC_WKV, st);
+      RT_CK(launch_tc<EPI_WKV>(bn_kv, tA_z, tB_kv, M, 2 * d, d, ep, err, ds.sms, st));
+    }
+    const int cc = c + 1;   // chunks revealed so far
+    if (cc * C < N) {
+      const int lb = lowbit(cc), q0 = cc * C, nq = std::min(lb * C, N - q0);
+      TimedScope ts(T, KC_FOLD_LEVEL0 + log2_int(lb * C), st);
+      RT_CK(launch_fold<bf16>(qkv, 3 * d, K, V, d, m, l, o, nullptr, B, H, 64, q0, nq, (cc - lb) * C, lb * C, sc2,
+                              cc == lb ? 1 : 0, 0, true, st, err, kFoldTcMinBlock, ds.sms));
+    }
+  }
+  return RT_OK;
+}
+
 static int enqueue_forward(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st,
                            Timer* T = nullptr, const HostIo* io = nullptr) {
+  if (P.s.chunk > 0) {
+    if (io) return RT_ERR_UNSUPPORTED;
+    return enqueue_chunked(P, X, ds, st, T);
+  }
   if (io) {
     if (P.s.dtype != RT_BF16) return RT_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_io_mu);
@@ -875,6 +996,11 @@ static long launch_count(const Shape& s) {
   long folds = 0;
   if (s.schedule == RT_SCHED_BLOCKED)
     for (int t = 1; t <= s.N; ++t) folds += (std::min(lowbit(t), s.N - t) > 0) ? 1 : 0;
+  if (s.dtype == RT_BF16 && s.chunk > 0) {
+    // inv_rms + projection; per chunk: attend + 4 GEMMs (+ a fold unless it is the last)
+    const int C = std::min(s.chunk, s.N), nchunks = (s.N + C - 1) / C;
+    return 2 + 5l * nchunks + (nchunks - 1);
+  }
   if (s.dtype == RT_BF16) {
     if (s.schedule == RT_SCHED_BLOCKED && plan_steps(s).ok) {
       // finalise(position 1) + one step kernel per segment + the folds of
@@ -898,7 +1024,7 @@ static long launch_count(const Shape& s) {
 // ---------------------------------------------------------------------------
 struct GraphKey {
   uintptr_t p[15];
-  int v[10];
+  int v[11];
   bool operator<(const GraphKey& o) const {
     int c = std::memcmp(p, o.p, sizeof(p));
     if (c) return c < 0;
@@ -931,7 +1057,8 @@ static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st
                           io ? io->x_host : nullptr, io ? io->z_host : nullptr,
                           io ? io->K_host : nullptr, io ? io->V_host : nullptr};
   for (int i = 0; i < 15; ++i) key.p[i] = reinterpret_cast<uintptr_t>(ptrs[i]);
-  const int vals[10] = {P.s.B, P.s.N, P.s.d, P.s.H, P.s.d_ff, P.s.dtype, P.s.schedule, dev, P.s.pages, P.s.L};
+  const int vals[11] = {P.s.B, P.s.N, P.s.d, P.s.H, P.s.d_ff, P.s.dtype, P.s.schedule, dev, P.s.pages, P.s.L,
+                        P.s.chunk};
   std::memcpy(key.v, vals, sizeof(vals));
 
   std::lock_guard<std::mutex> lk(g_graph_mu);
@@ -1030,6 +1157,33 @@ extern "C" int rt_layer_forward_pages(const void* x, const void* W_q, const void
     if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return RT_ERR_INVALID_ARG;
   const Plan P = make_plan(s);
   if (!P.sp.ok) return RT_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return RT_ERR_WORKSPACE;
+  Ptrs X{x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V, workspace};
+  return run_forward(P, X, RT_DRIVER_GRAPH, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t rt_layer_chunked_workspace_bytes(int B, int N, int d, int H, int d_ff, int C) {
+  Shape s{B, N, d, H, d_ff, RT_BF16, RT_SCHED_BLOCKED};
+  s.chunk = C;
+  if (C < 1 || validate(s) != RT_OK) return 0;
+  return make_plan(s).total;
+}
+
+extern "C" int rt_layer_forward_chunked(const void* x, const void* W_q, const void* W_k, const void* W_v,
+                                        const void* W_o, const void* W_1, const void* W_2, int B, int N, int d,
+                                        int H, int d_ff, int C, void* z, void* K, void* V, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  Shape s{B, N, d, H, d_ff, RT_BF16, RT_SCHED_BLOCKED};
+  s.chunk = C;
+  if (C < 1) return RT_ERR_INVALID_ARG;
+  int rc = validate(s);
+  if (rc != RT_OK) return rc;
+  if (!x || !W_q || !W_k || !W_v || !W_o || !W_1 || !W_2 || !z || !K || !V) return RT_ERR_INVALID_ARG;
+  const void* all[10] = {x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V};
+  for (const void* p : all)
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return RT_ERR_INVALID_ARG;
+  const Plan P = make_plan(s);
   if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return RT_ERR_WORKSPACE;
   Ptrs X{x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V, workspace};

@@ -454,6 +454,73 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
+// block-wise (chunked) recurrence, bf16, d_h = 64: the attention of the nc
+// positions p0 .. p0 + nc - 1 of one chunk. Query t of sequence b, head h
+// has folded into its (m, l, o) every persistent pair of the earlier chunks
+// (has_acc = 0 for the first chunk: none); it now attends causally to the
+// temporary pairs of the chunk's positions p0 .. t, merged one by one into
+// the same online-softmax statistics, and writes a_t = o / l to row
+// (t - p0) * B + b of a_out [nc * B][d]. An octet of lanes (8 dims each) per
+// (position, sequence, head); 16 octets per CTA.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+    k_chunk_attend(const __nv_bfloat16* __restrict__ qkv, const float* __restrict__ m,
+                   const float* __restrict__ l, const float* __restrict__ o, __nv_bfloat16* __restrict__ a_out,
+                   int B, int H, int p0, int nc, float sc2, int has_acc, unsigned* err) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int oct = threadIdx.x >> 3, sl = threadIdx.x & 7;
+  const unsigned omask = 0xFFu << ((threadIdx.x & 31) & 24);
+  const long unit = (long)blockIdx.x * 16 + oct;           // ((t - p0) * B + b) * H + h
+  if (unit >= (long)nc * B * H) return;                     // whole octets together
+  const int h = (int)(unit % H);
+  const long rb = unit / H;                                 // chunk row (t - p0) * B + b
+  const int b = (int)(rb % B), i = (int)(rb / B);
+  const int d = H * 64;
+  const int t = p0 + i;
+  if (!idx_ok(i < nc && b < B, err)) return;
+  const size_t row = (size_t)t * B + b;
+  float q[8];
+  load_bf16x8(qkv + row * (size_t)(3 * d) + h * 64 + sl * 8, q);
+  float mo = -INFINITY, lo = 0.f, oo[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (has_acc) {
+    mo = m[row * H + h];
+    lo = l[row * H + h];
+    const float4* op = reinterpret_cast<const float4*>(o + row * (size_t)d + h * 64 + sl * 8);
+    const float4 a0 = op[0], a1 = op[1];
+    oo[0] = a0.x; oo[1] = a0.y; oo[2] = a0.z; oo[3] = a0.w; oo[4] = a1.x; oo[5] = a1.y; oo[6] = a1.z; oo[7] = a1.w;
+  }
+  for (int s = p0; s <= t; ++s) {
+    const __nv_bfloat16* tp = qkv + ((size_t)s * B + b) * (size_t)(3 * d) + h * 64 + sl * 8;
+    float kt[8], vt[8];
+    load_bf16x8(tp + d, kt);
+    load_bf16x8(tp + 2 * d, vt);
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dot += q[e] * kt[e];
+    dot += __shfl_xor_sync(omask, dot, 1);
+    dot += __shfl_xor_sync(omask, dot, 2);
+    dot += __shfl_xor_sync(omask, dot, 4);
+    const float sc = dot * sc2;
+    const float mn = fmaxf(mo, sc);
+    const float al = rescale(mo, mn), p = exp2f(sc - mn);
+    lo = lo * al + p;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) oo[e] = oo[e] * al + p * vt[e];
+    mo = mn;
+  }
+  const float inv = 1.f / lo;
+  uint4 w;
+  uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 v2 = __floats2bfloat162_rn(oo[2 * k] * inv, oo[2 * k + 1] * inv);
+    wp[k] = *reinterpret_cast<uint32_t*>(&v2);
+  }
+  *reinterpret_cast<uint4*>(a_out + (size_t)rb * d + h * 64 + sl * 8) = w;
+}
+
+// ---------------------------------------------------------------------------
 // decode-step attention (bf16, d_h = 64): the query at row 0 of a
 // one-position qkv [B][3d] against cached keys 0..j-1 (position-major K, V
 // [.][B][d]) plus its temporary pair. One CTA of 4 warps per (b, h); each

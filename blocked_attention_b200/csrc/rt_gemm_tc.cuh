@@ -73,7 +73,15 @@ struct EpiParams {
   // softmax scale). pages = 0: the single-layer configuration.
   int pages;
   float inv_sqrt_L;
+  // Rows of the per-position GEMMs (WO, W1, W2, WKV) are position-major:
+  // row r is sequence r % B at position j + r / B (one position per launch:
+  // row = sequence; a chunk of positions: B rows per position). ssq_rows is
+  // the row count of the launch, the stride of the sum-of-squares partials
+  // (0 = B).
+  int ssq_rows;
 };
+
+__device__ __forceinline__ int ssq_stride(const EpiParams& p) { return p.ssq_rows ? p.ssq_rows : p.B; }
 
 __device__ __forceinline__ uint32_t dsmem_map(uint32_t smem_addr, uint32_t rank) {
   uint32_t r;
@@ -171,8 +179,9 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& p, int row, i
     if (col0 + c >= N) break;
     const void* ptr = nullptr;
     if constexpr (EPI == EPI_WO) {
-      const int ch = p.j / p.xc;
-      ptr = p.x + (((size_t)ch * p.B + row) * p.xc + (p.j - ch * p.xc)) * p.d + col0 + c;
+      const int b = row % p.B, jj = p.j + row / p.B;
+      const int ch = jj / p.xc;
+      ptr = p.x + (((size_t)ch * p.B + b) * p.xc + (jj - ch * p.xc)) * p.d + col0 + c;
     }
     if (ptr) asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));   // one 128-byte line per chunk
   }
@@ -201,10 +210,10 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
     for (int i = 0; i < 32; ++i) v[i] *= row_scale;
     store_bf16x32(p.qkv + ((size_t)n * p.B + b) * (size_t)(3 * p.d) + col0, v);
   } else if constexpr (EPI == EPI_WO) {
-    const int b = row;
+    const int b = row % p.B, jj = p.j + row / p.B;
     float xv[32];
-    const int c = p.j / p.xc;
-    load_bf16x32(p.x + (((size_t)c * p.B + b) * p.xc + (p.j - c * p.xc)) * p.d + col0, xv);
+    const int c = jj / p.xc;
+    load_bf16x32(p.x + (((size_t)c * p.B + b) * p.xc + (jj - c * p.xc)) * p.d + col0, xv);
     if (p.pages) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] *= p.inv_sqrt_L;
@@ -214,18 +223,18 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
       v[i] += xv[i];
       ssq += v[i] * v[i];
     }
-    float4* u4 = reinterpret_cast<float4*>(p.u32 + (size_t)b * p.d + col0);
+    float4* u4 = reinterpret_cast<float4*>(p.u32 + (size_t)row * p.d + col0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) u4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    store_bf16x32(p.u16 + (size_t)b * p.d + col0, v);
+    store_bf16x32(p.u16 + (size_t)row * p.d + col0, v);
   } else if constexpr (EPI == EPI_W1) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i] * row_scale);
     store_bf16x32(p.h16 + (size_t)row * p.d_ff + col0, v);
   } else if constexpr (EPI == EPI_W2) {
-    const int b = row;
+    const int b = row % p.B, jj = p.j + row / p.B;
     // u was written by other CTAs (L2-coherent loads: no stale L1 lines)
-    const float4* u4 = reinterpret_cast<const float4*>(p.u32 + (size_t)b * p.d + col0);
+    const float4* u4 = reinterpret_cast<const float4*>(p.u32 + (size_t)row * p.d + col0);
     if (p.pages) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] *= p.inv_sqrt_L;
@@ -237,13 +246,12 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
     }
 #pragma unroll
     for (int i = 0; i < 32; ++i) ssq += v[i] * v[i];
-    store_bf16x32(p.zout + ((size_t)b * p.Nseq + p.j) * p.d + col0, v);
-    store_bf16x32(p.z16 + (size_t)b * p.d + col0, v);
+    store_bf16x32(p.zout + ((size_t)b * p.Nseq + jj) * p.d + col0, v);
+    store_bf16x32(p.z16 + (size_t)row * p.d + col0, v);
   } else if constexpr (EPI == EPI_WKV) {
-    const int b = row;
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] *= row_scale;
-    const size_t base = ((size_t)p.j * p.B + b) * p.d;
+    const size_t base = ((size_t)p.j * p.B + row) * p.d;   // position j + row / B, sequence row % B
     if (col0 < p.d) store_bf16x32(p.Kout + base + col0, v);
     else store_bf16x32(p.Vout + base + (col0 - p.d), v);
   } else if constexpr (EPI == EPI_RKV) {
@@ -307,7 +315,7 @@ __device__ __forceinline__ float row_scale_for(const EpiParams& p, int row) {
     return p.inv_rms[row];
   } else if constexpr (EPI == EPI_W1 || EPI == EPI_WKV) {
     float s = 0.f;
-    for (int t = 0; t < p.ssq_tiles; ++t) s += __ldcg(p.ssq_in + (size_t)t * p.B + row);
+    for (int t = 0; t < p.ssq_tiles; ++t) s += __ldcg(p.ssq_in + (size_t)t * ssq_stride(p) + row);
     return rsqrtf(s / (float)p.d + p.eps);
   } else {
     return 1.f;
@@ -492,7 +500,7 @@ __global__ void __launch_bounds__(224, 1)
           if (row_ok && col0 < N) ssq += epilogue_chunk<EPI>(p, row, col0, N, v, rs);
         }
         if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
-          if (row_ok) p.ssq_out[(size_t)nt * p.B + row] = ssq;
+          if (row_ok) p.ssq_out[(size_t)nt * ssq_stride(p) + row] = ssq;
         }
       } else {
         // stage this CTA's partial tile (fp32, rows padded to BN + 4 floats) in the
@@ -576,7 +584,7 @@ __global__ void __launch_bounds__(224, 1)
       if constexpr (EPI == EPI_WO || EPI == EPI_W2) {
         // the `splits` consecutive lanes sharing a row add their column sums
         for (int o = 1; o < splits; o <<= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
-        if (row_ok && (t % splits) == 0) p.ssq_out[(size_t)nt * p.B + row] = ssq;
+        if (row_ok && (t % splits) == 0) p.ssq_out[(size_t)nt * ssq_stride(p) + row] = ssq;
       }
     }
     // this CTA's outgoing copies have read its staging before it can exit;

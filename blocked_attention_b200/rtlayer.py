@@ -31,7 +31,8 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_erro
            "rt_layer_launch_count", "rt_layer_forward_timed", "rt_project_qkv_noalloc",
            "rt_selftest_wait_timeout", "rt_layer_decode_workspace_bytes", "rt_layer_decode_step",
            "rt_project_qkv_noalloc_status", "rt_layer_recompute_workspace_bytes", "rt_layer_recompute_kv",
-           "rt_layer_forward_pages", "rt_layer_backward_workspace_bytes", "rt_layer_backward")
+           "rt_layer_forward_pages", "rt_layer_backward_workspace_bytes", "rt_layer_backward",
+           "rt_layer_chunked_workspace_bytes", "rt_layer_forward_chunked")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
                   "fold_warp", "fold_mma", "steps")
@@ -83,6 +84,10 @@ def lib() -> ctypes.CDLL:
     L.rt_layer_backward_workspace_bytes.argtypes = [i] * 6
     L.rt_layer_backward.restype = i
     L.rt_layer_backward.argtypes = [vp] * 13 + [i] * 6 + [vp] * 8 + [sz, vp]
+    L.rt_layer_chunked_workspace_bytes.restype = sz
+    L.rt_layer_chunked_workspace_bytes.argtypes = [i] * 6
+    L.rt_layer_forward_chunked.restype = i
+    L.rt_layer_forward_chunked.argtypes = [vp] * 7 + [i] * 6 + [vp] * 4 + [sz, vp]
     L.rt_layer_forward_pages.restype = i
     L.rt_layer_forward_pages.argtypes = [vp] * 7 + [i] * 6 + [vp] * 4 + [sz, vp]
     L.rt_layer_sync_status.restype = i
@@ -251,6 +256,35 @@ def layer_backward(x: torch.Tensor, W: dict, H: int, z: torch.Tensor, K: torch.T
                                  ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check("rt_layer_backward", rc)
     return dx, dW
+
+
+def layer_forward_chunked(x: torch.Tensor, W: dict, H: int, C: int, out=None,
+                          workspace: torch.Tensor | None = None, stream=None):
+    """rt_layer_forward_chunked: the block-wise recurrence with chunks of C
+    positions; bf16 device tensors as in layer_forward."""
+    B, N, d = x.shape
+    d_ff = W["W_1"].shape[0]
+    for n in WEIGHT_NAMES:
+        if W[n].dtype != torch.bfloat16 or not W[n].is_contiguous() or W[n].device != x.device:
+            raise ValueError(f"weight {n} must be a contiguous bf16 tensor on {x.device}")
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 tensor")
+    if out is None:
+        z = torch.empty_like(x)
+        K = torch.empty((N, B, d), dtype=x.dtype, device=x.device)
+        V = torch.empty_like(K)
+    else:
+        z, K, V = out
+    if workspace is None:
+        nbytes = int(lib().rt_layer_chunked_workspace_bytes(B, N, d, H, d_ff, C))
+        if nbytes == 0:
+            raise RTError("rt_layer_chunked_workspace_bytes", RT_ERR_UNSUPPORTED)
+        workspace = alloc_workspace(nbytes, x.device)
+    rc = lib().rt_layer_forward_chunked(_ptr(x), *[_ptr(W[n]) for n in WEIGHT_NAMES], B, N, d, H, d_ff, C,
+                                        _ptr(z), _ptr(K), _ptr(V), _ptr(workspace),
+                                        ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check("rt_layer_forward_chunked", rc)
+    return z, K, V
 
 
 def launch_count(B, N, d, H, d_ff, dtype=torch.bfloat16, schedule="blocked") -> int:

@@ -128,6 +128,30 @@ int rt_layer_forward_pages(const void* x_dev,
                            void* z_dev, void* K_dev, void* V_dev,
                            void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* Device bytes rt_layer_forward_chunked needs for chunks of C positions;
+ * 0 if unsupported. */
+size_t rt_layer_chunked_workspace_bytes(int B, int N, int d, int H, int d_ff, int C);
+
+/* The layer with its recurrence executed block-wise, in chunks of C >= 1
+ * positions (paper §9 and notes §8 name this depth-for-speed trade-off
+ * without defining it; this is our reading): the positions are cut into
+ * consecutive chunks of C; a position's persistent pair is visible only to
+ * the positions of later chunks, and inside its own chunk a position attends
+ * to the temporary pairs of the chunk's positions up to itself. C = 1 is the
+ * layer of rt_layer_forward; C >= N the standard causal Transformer layer
+ * (paper §2.1), whose K, V outputs are then W_{k,v} rms(z).
+ * bf16, the exact blocked schedule at chunk granularity, graph driver: per
+ * chunk one attention launch, the four GEMMs with B * C rows, and one block
+ * fold (chunks (c - lowbit(c), c] into chunks (c, c + lowbit(c)]).
+ * Arguments and layouts as in rt_layer_forward; workspace_dev >=
+ * rt_layer_chunked_workspace_bytes(...) bytes, 256-byte aligned. */
+int rt_layer_forward_chunked(const void* x_dev,
+                             const void* W_q_dev, const void* W_k_dev, const void* W_v_dev,
+                             const void* W_o_dev, const void* W_1_dev, const void* W_2_dev,
+                             int B, int N, int d, int H, int d_ff, int C,
+                             void* z_dev, void* K_dev, void* V_dev,
+                             void* workspace_dev, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of a
  * workspace used by rt_layer_forward. RT_OK, RT_ERR_TIMEOUT or RT_ERR_CUDA. */
 int rt_layer_sync_status(void* workspace_dev, void* stream);

@@ -217,3 +217,17 @@ def test_pages_entry_point_validation_happens_before_any_launch(L):
     assert call(ws_bytes=16) == R.RT_ERR_WORKSPACE
     assert L.rt_layer_forward_pages(None, *([p] * 6), 2, 16, 128, 2, 256, 1, p, p, p, p,
                                     ctypes.c_size_t(1 << 34), None) == R.RT_ERR_INVALID_ARG
+
+
+def test_chunked_entry_point_validation_happens_before_any_launch(L):
+    assert L.rt_layer_chunked_workspace_bytes(4, 64, 128, 2, 256, 16) > L.rt_layer_chunked_workspace_bytes(
+        4, 64, 128, 2, 256, 1)                                        # per-step buffers hold B x C rows
+    assert L.rt_layer_chunked_workspace_bytes(4, 64, 128, 2, 256, 0) == 0
+    assert L.rt_layer_chunked_workspace_bytes(4, 64, 96, 2, 256, 4) == 0   # bf16 needs d_h = 64
+    p = ctypes.c_void_p(1 << 40)
+
+    def call(C=4, ws_bytes=1 << 34):
+        return L.rt_layer_forward_chunked(*([p] * 7), 4, 64, 128, 2, 256, C, p, p, p, p,
+                                          ctypes.c_size_t(ws_bytes), None)
+    assert call(C=0) == R.RT_ERR_INVALID_ARG
+    assert call(ws_bytes=16) == R.RT_ERR_WORKSPACE
