@@ -73,6 +73,14 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="sequence-length sweep, blocked vs naive (B=32 d=1024 H=16x64 d_ff=4096)")
     ap.add_argument("--sweep-n", default="512,1024,2048,4096,8192,16384")
+    ap.add_argument("--pages", action="store_true",
+                    help="the paper's own parameterisation (rt_layer_forward_pages) at the workload's shape")
+    ap.add_argument("--chunked", type=int, default=0, metavar="C",
+                    help="the block-wise recurrence with chunks of C positions at the workload's shape")
+    ap.add_argument("--recompute", action="store_true",
+                    help="activation-checkpoint recompute of K, V from z over all B*N rows")
+    ap.add_argument("--backward", action="store_true",
+                    help="backward pass (bf16 storage) at B=64 N=1024 d=512 H=8x64 d_ff=2048")
     ap.add_argument("--profile-case", choices=["step", "fold", "fwd", "naive"],
                     help="run one small case for an ncu capture and exit: 'step' = one host-loop forward at "
                          "B=512 N=64 d=1024 (the per-step GEMM shapes of the headline); 'fold' = one block fold "
@@ -410,6 +418,78 @@ def run_sweep(args, R, torch):
             torch.cuda.empty_cache()
 
 
+def _timed(torch, fn, steps: int, warmup: int) -> float:
+    """ms per call of fn on the current stream (CUDA events), after warm-up."""
+    for _ in range(max(warmup, 1)):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_next_rows(args, R, torch, rtinputs):
+    """Measurements of the rows beyond the forward: the paper's own
+    parameterisation, the block-wise recurrence, the checkpoint recompute
+    and the backward pass. One JSON line each."""
+    dev = torch.device("cuda", 0)
+    peaks = measured_peaks()
+    if args.backward:
+        Bsz, N, d, H, dff = 64, 1024, 512, 8, 2048
+    else:
+        c = WORKLOADS[args.workload]
+        Bsz, N, d, H, dff = c["B"], c["N"], c["d"], c["H"], c["d_ff"]
+    W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
+         for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16").items()}
+    x = torch.randn((Bsz, N, d), device=dev, dtype=torch.bfloat16)
+    shape = {"B": Bsz, "N": N, "d": d, "H": H, "d_ff": dff}
+    line = {"dtype": "bf16", "data": "synthetic", "steps": args.steps, "warmup": args.warmup}
+    if args.pages or args.chunked:
+        out = (torch.empty_like(x), torch.empty((N, Bsz, d), dtype=torch.bfloat16, device=dev),
+               torch.empty((N, Bsz, d), dtype=torch.bfloat16, device=dev))
+        if args.pages:
+            ws = R.alloc_workspace(R.workspace_bytes(Bsz, N, d, H, dff), dev)
+            fn = lambda: R.layer_forward_pages(x, W, H, 1, out=out, workspace=ws)
+            name, extra = "RT-layer prefill tokens/s, the paper's own parameterisation", {}
+        else:
+            ws = R.alloc_workspace(int(R.lib().rt_layer_chunked_workspace_bytes(Bsz, N, d, H, dff, args.chunked)), dev)
+            fn = lambda: R.layer_forward_chunked(x, W, H, args.chunked, out=out, workspace=ws)
+            name, extra = "RT-layer prefill tokens/s, block-wise recurrence", {"chunk": args.chunked}
+        ms = _timed(torch, fn, args.steps, args.warmup)
+        assert R.sync_status(ws) == 0
+        flops = 2.0 * Bsz * N * (6 * d * d + 2 * d * dff) + 4.0 * Bsz * d * N * (N + 1) / 2
+        line.update({"metric": name, "value": Bsz * N / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+                     "tflops": flops / (ms / 1e3) / 1e12, "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 /
+                     peaks["bf16_tflops"], "config": {"workload": "RT layer forward", **shape, **extra}})
+    elif args.recompute:
+        z = x
+        K = torch.empty((N, Bsz, d), dtype=torch.bfloat16, device=dev)
+        V = torch.empty_like(K)
+        ws = R.alloc_workspace(int(R.lib().rt_layer_recompute_workspace_bytes(Bsz, N, d)), dev)
+        ms = _timed(torch, lambda: R.recompute_kv(z, W["W_k"], W["W_v"], out=(K, V), workspace=ws), args.steps,
+                    args.warmup)
+        assert R.sync_status(ws) == 0
+        flops = 2.0 * Bsz * N * d * 2 * d
+        line.update({"metric": "checkpoint recompute of K, V from z, tokens/s", "value": Bsz * N / (ms / 1e3),
+                     "unit": "tokens/s", "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                     "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                     "config": {"workload": "recompute", **shape}})
+    else:
+        z, K, V = R.layer_forward(x, W, H)
+        dz, dK, dV = torch.randn_like(z), torch.randn_like(K), torch.randn_like(V)
+        ws = R.alloc_workspace(int(R.lib().rt_layer_backward_workspace_bytes(Bsz, N, d, H, dff, R.RT_BF16)), dev)
+        ms = _timed(torch, lambda: R.layer_backward(x, W, H, z, K, V, dz, dK, dV, workspace=ws), args.steps,
+                    args.warmup)
+        line.update({"metric": "RT-layer backward tokens/s (bf16 storage, fp32 arithmetic)",
+                     "value": Bsz * N / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+                     "config": {"workload": "backward", **shape}})
+    print(json.dumps(line), flush=True)
+
+
 def run_profile_case(args, R, torch, rtinputs):
     dev = torch.device("cuda", 0)
     if args.profile_case in ("step", "fwd"):
@@ -460,6 +540,9 @@ def main():
         return
     if args.decode:
         run_decode(args, R, torch, rtinputs)
+        return
+    if args.pages or args.chunked or args.recompute or args.backward:
+        run_next_rows(args, R, torch, rtinputs)
         return
     if args.stack or args.sweep:
         (run_stack(args, R, torch, rtinputs) if args.stack else run_sweep(args, R, torch))
