@@ -170,50 +170,49 @@ __global__ void k_gelu_bwd(const float* __restrict__ dy, const float* __restrict
 // Attention of every position at once over the stored persistent pairs
 // (rows 0..t-1 of K, V) plus its temporary pair, natural-log units:
 //   a_t = sum_i softmax(s)_i v_i,  lse_t = log sum_i exp(s_i),  s_i = <q, k_i> * scale.
-// One warp per (t, b, h); lanes split the keys, then merge.
+// One warp per (t, b, h); lane i owns keys i, i + 32, ... (key t is the
+// temporary pair) with whole-row dot products, its own online-softmax state
+// and DH-wide numerator; the lanes are merged at the end.
+template <int DH>
 __global__ void __launch_bounds__(128) k_attn_lse(const float* __restrict__ qkv, const float* __restrict__ K,
                                                   const float* __restrict__ V, float* __restrict__ a,
-                                                  float* __restrict__ lse, int B, int N, int H, int dh,
-                                                  float scale) {
+                                                  float* __restrict__ lse, int B, int N, int H, float scale) {
   const long w = (long)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= (long)N * B * H) return;
   const int h = (int)(w % H);
   const long rb = w / H;                       // position-major row t * B + b
   const int b = (int)(rb % B), t = (int)(rb / B);
-  const int d = H * dh;
-  const float* q = qkv + (size_t)rb * 3 * d + h * dh;
-  // scores: lane handles keys lane, lane + 32, ...; key t (index t) is the temporary pair
-  float m = -INFINITY;
+  const int d = H * DH;
+  const float* q = qkv + (size_t)rb * 3 * d + h * DH;
+  float qr[DH], acc[DH];
+#pragma unroll
+  for (int e = 0; e < DH; ++e) { qr[e] = q[e]; acc[e] = 0.f; }
+  float m = -INFINITY, l = 0.f;
   for (int i = lane; i <= t; i += 32) {
-    const float* k = i < t ? K + ((size_t)i * B + b) * d + h * dh : q + d;
+    const float* k = i < t ? K + ((size_t)i * B + b) * d + h * DH : q + d;
+    const float* v = i < t ? V + ((size_t)i * B + b) * d + h * DH : q + 2 * d;
     float s = 0.f;
-    for (int e = 0; e < dh; ++e) s += q[e] * k[e];
-    m = fmaxf(m, s * scale);
+#pragma unroll
+    for (int e = 0; e < DH; ++e) s += qr[e] * k[e];
+    s *= scale;
+    const float mn = fmaxf(m, s);
+    const float al = m == -INFINITY ? 0.f : expf(m - mn), p = expf(s - mn);
+    l = l * al + p;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) acc[e] = acc[e] * al + p * v[e];
+    m = mn;
   }
-  m = warp_max(m);
-  float l = 0.f;
-  for (int i = lane; i <= t; i += 32) {
-    const float* k = i < t ? K + ((size_t)i * B + b) * d + h * dh : q + d;
-    float s = 0.f;
-    for (int e = 0; e < dh; ++e) s += q[e] * k[e];
-    l += expf(s * scale - m);
+  // merge the lanes' states
+  const float M = warp_max(m);
+  const float f = m == -INFINITY ? 0.f : expf(m - M);
+  const float L = warp_sum(l * f);
+#pragma unroll
+  for (int e = 0; e < DH; ++e) {
+    const float v = warp_sum(acc[e] * f);
+    if (lane == (e & 31)) a[(size_t)rb * d + h * DH + e] = v / L;
   }
-  l = warp_sum(l);
-  const float L = m + logf(l);
-  // a: lane handles dims lane, lane + 32, ... (keys in order)
-  for (int e = lane; e < dh; e += 32) {
-    float acc = 0.f;
-    for (int i = 0; i <= t; ++i) {
-      const float* k = i < t ? K + ((size_t)i * B + b) * d + h * dh : q + d;
-      const float* v = i < t ? V + ((size_t)i * B + b) * d + h * dh : q + 2 * d;
-      float s = 0.f;
-      for (int f = 0; f < dh; ++f) s += q[f] * k[f];
-      acc += expf(s * scale - L) * v[e];
-    }
-    a[(size_t)rb * d + h * dh + e] = acc;
-  }
-  if (lane == 0) lse[(size_t)rb * H + h] = L;
+  if (lane == 0) lse[(size_t)rb * H + h] = M + logf(L);
 }
 
 // Attention backward of query t (all sequences and heads): one warp per
@@ -221,56 +220,62 @@ __global__ void __launch_bounds__(128) k_attn_lse(const float* __restrict__ qkv,
 // ds_i = p_i (dp_i - delta):
 //   dk_i += scale ds_i q,  dv_i += p_i da      (persistent pairs i < t, in place)
 //   dq = scale sum_i ds_i k_i,  dk~ = scale ds~ q,  dv~ = p~ da   (temporary pair)
-// Each (i, b, h) row of dK, dV is updated by exactly one warp.
+// Lane i owns keys i, i + 32, ... (whole rows; each (i, b, h) row of dK, dV
+// is updated by exactly one lane) and a partial dq, summed over the lanes at
+// the end.
+template <int DH>
 __global__ void __launch_bounds__(128) k_attn_bwd_step(const float* __restrict__ qkv, const float* __restrict__ K,
                                                        const float* __restrict__ V, const float* __restrict__ a,
                                                        const float* __restrict__ lse, const float* __restrict__ da,
                                                        float* __restrict__ dK, float* __restrict__ dV,
-                                                       float* __restrict__ dqkv, int B, int H, int dh, int t,
-                                                       float scale) {
+                                                       float* __restrict__ dqkv, int B, int H, int t, float scale) {
   const int w = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= B * H) return;
   const int b = w / H, h = w - b * H;
-  const int d = H * dh;
+  const int d = H * DH;
   const size_t rt_ = (size_t)t * B + b;
-  const float* q = qkv + rt_ * 3 * d + h * dh;
-  const float* dav = da + rt_ * d + h * dh;
-  const float* av = a + rt_ * d + h * dh;
+  const float* q = qkv + rt_ * 3 * d + h * DH;
+  const float* dav = da + rt_ * d + h * DH;
+  const float* av = a + rt_ * d + h * DH;
   const float L = lse[rt_ * H + h];
+  float qr[DH], dar[DH], dq[DH];
   float delta = 0.f;
-  for (int e = lane; e < dh; e += 32) delta += dav[e] * av[e];
-  delta = warp_sum(delta);
-  float* dq = dqkv + rt_ * 3 * d + h * dh;
-  // dq accumulates in registers: lane owns dims lane, lane + 32, ... (dh <= 128)
-  float dqr[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int i = 0; i <= t; ++i) {
+#pragma unroll
+  for (int e = 0; e < DH; ++e) {
+    qr[e] = q[e];
+    dar[e] = dav[e];
+    dq[e] = 0.f;
+    delta += dar[e] * av[e];
+  }
+  float* dqrow = dqkv + rt_ * 3 * d + h * DH;
+  for (int i = lane; i <= t; i += 32) {
     const bool temp = i == t;
-    const float* k = temp ? q + d : K + ((size_t)i * B + b) * d + h * dh;
-    const float* v = temp ? q + 2 * d : V + ((size_t)i * B + b) * d + h * dh;
+    const float* k = temp ? q + d : K + ((size_t)i * B + b) * d + h * DH;
+    const float* v = temp ? q + 2 * d : V + ((size_t)i * B + b) * d + h * DH;
     float s = 0.f, dp = 0.f;
-    for (int e = lane; e < dh; e += 32) {
-      s += q[e] * k[e];
-      dp += dav[e] * v[e];
+#pragma unroll
+    for (int e = 0; e < DH; ++e) {
+      s += qr[e] * k[e];
+      dp += dar[e] * v[e];
     }
-    s = warp_sum(s);
-    dp = warp_sum(dp);
     const float p = expf(s * scale - L);
     const float ds = p * (dp - delta);
-    float* dk = temp ? dq + d : dK + ((size_t)i * B + b) * d + h * dh;
-    float* dv = temp ? dq + 2 * d : dV + ((size_t)i * B + b) * d + h * dh;
-    for (int e = lane, c = 0; e < dh; e += 32, ++c) {
-      dqr[c] += scale * ds * k[e];
-      if (temp) {
-        dk[e] = scale * ds * q[e];
-        dv[e] = p * dav[e];
-      } else {
-        dk[e] += scale * ds * q[e];
-        dv[e] += p * dav[e];
-      }
+    float* dk = temp ? dqrow + d : dK + ((size_t)i * B + b) * d + h * DH;
+    float* dv = temp ? dqrow + 2 * d : dV + ((size_t)i * B + b) * d + h * DH;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) {
+      dq[e] += scale * ds * k[e];
+      const float gk = scale * ds * qr[e], gv = p * dar[e];
+      if (temp) { dk[e] = gk; dv[e] = gv; }
+      else { dk[e] += gk; dv[e] += gv; }
     }
   }
-  for (int e = lane, c = 0; e < dh; e += 32, ++c) dq[e] = dqr[c];
+#pragma unroll
+  for (int e = 0; e < DH; ++e) {
+    const float v = warp_sum(dq[e]);
+    if (lane == (e & 31)) dqrow[e] = v;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -345,7 +350,7 @@ static int bwd_validate(int B, int N, int d, int H, int d_ff, int dtype) {
   if (B <= 0 || N <= 0 || d <= 0 || H <= 0 || d_ff <= 0 || d % H != 0) return RT_ERR_INVALID_ARG;
   if (dtype != RT_F32 && dtype != RT_BF16) return RT_ERR_INVALID_ARG;
   const int dh = d / H;
-  if (dh > 128 || (long)B * N > (1l << 24)) return RT_ERR_UNSUPPORTED;
+  if ((dh != 32 && dh != 64 && dh != 128) || (long)B * N > (1l << 24)) return RT_ERR_UNSUPPORTED;
   return RT_OK;
 }
 
@@ -453,7 +458,12 @@ extern "C" int rt_layer_backward(const void* x_, const void* Wq_, const void* Wk
   RT_BCK(gemm(xr, d, 0, Wq, d, 0, qkv, 3 * d, (int)R, d, d, 0, st));
   RT_BCK(gemm(xr, d, 0, Wk, d, 0, qkv + d, 3 * d, (int)R, d, d, 0, st));
   RT_BCK(gemm(xr, d, 0, Wv, d, 0, qkv + 2 * d, 3 * d, (int)R, d, d, 0, st));
-  k_attn_lse<<<(unsigned)((R * H + 3) / 4), 128, 0, st>>>(qkv, K, V, a, lse, B, N, H, dh, scale);
+  {
+    const unsigned g = (unsigned)((R * H + 3) / 4);
+    if (dh == 32) k_attn_lse<32><<<g, 128, 0, st>>>(qkv, K, V, a, lse, B, N, H, scale);
+    else if (dh == 64) k_attn_lse<64><<<g, 128, 0, st>>>(qkv, K, V, a, lse, B, N, H, scale);
+    else k_attn_lse<128><<<g, 128, 0, st>>>(qkv, K, V, a, lse, B, N, H, scale);
+  }
   RT_BCK(cudaGetLastError());
   RT_BCK(cudaMemcpyAsync(u, xp, R * d * 4, cudaMemcpyDeviceToDevice, st));
   RT_BCK(gemm(a, d, 0, Wo, d, 0, u, d, (int)R, d, d, 1, st));
@@ -483,8 +493,12 @@ extern "C" int rt_layer_backward(const void* x_, const void* Wq_, const void* Wk
     RT_BCK(cudaGetLastError());
     // da = du W_o, then the attention backward of query t
     RT_BCK(gemm(dU + r0 * d, d, 0, Wo, d, 1, dA + r0 * d, d, B, d, d, 0, st));
-    k_attn_bwd_step<<<(unsigned)((B * H + 3) / 4), 128, 0, st>>>(qkv, K, V, a, lse, dA, dKa, dVa, dqkv, B, H, dh, t,
-                                                                 scale);
+    {
+      const unsigned g = (unsigned)((B * H + 3) / 4);
+      if (dh == 32) k_attn_bwd_step<32><<<g, 128, 0, st>>>(qkv, K, V, a, lse, dA, dKa, dVa, dqkv, B, H, t, scale);
+      else if (dh == 64) k_attn_bwd_step<64><<<g, 128, 0, st>>>(qkv, K, V, a, lse, dA, dKa, dVa, dqkv, B, H, t, scale);
+      else k_attn_bwd_step<128><<<g, 128, 0, st>>>(qkv, K, V, a, lse, dA, dKa, dVa, dqkv, B, H, t, scale);
+    }
     RT_BCK(cudaGetLastError());
   }
 
