@@ -24,9 +24,9 @@
 //       dk_t, dv_t are complete (every later query has contributed);
 //       d rms(z_t) = dk_t W_k + dv_t W_v;  dz_t += rms'(z_t) ...
 //       MLP backward -> du_t;  da_t = du_t W_o;
-//       attention backward of query t: its contributions to dk_i, dv_i of
-//       every earlier position (added in place), to its own dq and to the
-//       temporary pair's dk~, dv~.
+//       attention backward: query t's temporary pair, then the forward's
+//       block whose earliest query is t (its keys' dk, dv and its queries'
+//       dq, added in place) -- the exact blocked schedule in reverse.
 //  3. Batched over all positions: dx = du + rms'(x)(dq W_q + dk~ W_k +
 //     dv~ W_v), and every weight gradient as one [out][B*N] x [B*N][in]
 //     product.
@@ -215,67 +215,119 @@ __global__ void __launch_bounds__(128) k_attn_lse(const float* __restrict__ qkv,
   if (lane == 0) lse[(size_t)rb * H + h] = M + logf(L);
 }
 
-// Attention backward of query t (all sequences and heads): one warp per
-// (b, h). With p_i = exp(s_i - lse), dp_i = <da, v_i>, delta = <da, a>,
-// ds_i = p_i (dp_i - delta):
-//   dk_i += scale ds_i q,  dv_i += p_i da      (persistent pairs i < t, in place)
-//   dq = scale sum_i ds_i k_i,  dk~ = scale ds~ q,  dv~ = p~ da   (temporary pair)
-// Lane i owns keys i, i + 32, ... (whole rows; each (i, b, h) row of dK, dV
-// is updated by exactly one lane) and a partial dq, summed over the lanes at
-// the end.
+// Attention backward, exact blocked schedule (the forward's dyadic blocks in
+// reverse). With p_ji = exp(s_ji - lse_j), s_ji = <q_j, k_i> * scale,
+// dp_ji = <da_j, v_i>, delta_j = <da_j, a_j>, ds_ji = p_ji (dp_ji - delta_j):
+//   dk_i += scale sum_j ds_ji q_j,  dv_i += sum_j p_ji da_j,  dq_j += scale sum_i ds_ji k_i.
+// The pairs (key i < query j) are the forward's blocks: the block the forward
+// folds at step t (keys (t - lb, t], queries (t, t + lb]) is back-propagated
+// in the reverse loop right after query t + 1's gradient da is known (every
+// other query of the block is later, so already done) and before key t's
+// gradient is needed; each pair once, Theta(N log N) traffic like the forward.
+//
+// The temporary pair of query t: dk~ = scale ds~ q, dv~ = p~ da, and dq_t is
+// initialised with its term (the blocks add the rest later); delta_t stored.
+// One warp per (b, h); lanes over dims.
 template <int DH>
-__global__ void __launch_bounds__(128) k_attn_bwd_step(const float* __restrict__ qkv, const float* __restrict__ K,
-                                                       const float* __restrict__ V, const float* __restrict__ a,
+__global__ void __launch_bounds__(128) k_attn_bwd_temp(const float* __restrict__ qkv, const float* __restrict__ a,
                                                        const float* __restrict__ lse, const float* __restrict__ da,
-                                                       float* __restrict__ dK, float* __restrict__ dV,
-                                                       float* __restrict__ dqkv, int B, int H, int t, float scale) {
+                                                       float* __restrict__ delta, float* __restrict__ dqkv, int B,
+                                                       int H, int t, float scale) {
   const int w = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= B * H) return;
   const int b = w / H, h = w - b * H;
   const int d = H * DH;
-  const size_t rt_ = (size_t)t * B + b;
-  const float* q = qkv + rt_ * 3 * d + h * DH;
-  const float* dav = da + rt_ * d + h * DH;
-  const float* av = a + rt_ * d + h * DH;
-  const float L = lse[rt_ * H + h];
-  float qr[DH], dar[DH], dq[DH];
-  float delta = 0.f;
-#pragma unroll
-  for (int e = 0; e < DH; ++e) {
-    qr[e] = q[e];
-    dar[e] = dav[e];
-    dq[e] = 0.f;
-    delta += dar[e] * av[e];
+  const size_t r = (size_t)t * B + b;
+  const float* q = qkv + r * 3 * d + h * DH;
+  const float* dav = da + r * d + h * DH;
+  const float* av = a + r * d + h * DH;
+  float s = 0.f, dp = 0.f, dl = 0.f;
+  for (int e = lane; e < DH; e += 32) {
+    s += q[e] * q[d + e];
+    dp += dav[e] * q[2 * d + e];
+    dl += dav[e] * av[e];
   }
-  float* dqrow = dqkv + rt_ * 3 * d + h * DH;
-  for (int i = lane; i <= t; i += 32) {
-    const bool temp = i == t;
-    const float* k = temp ? q + d : K + ((size_t)i * B + b) * d + h * DH;
-    const float* v = temp ? q + 2 * d : V + ((size_t)i * B + b) * d + h * DH;
+  s = warp_sum(s);
+  dp = warp_sum(dp);
+  dl = warp_sum(dl);
+  const float p = expf(s * scale - lse[r * H + h]);
+  const float ds = p * (dp - dl);
+  float* dq = dqkv + r * 3 * d + h * DH;
+  for (int e = lane; e < DH; e += 32) {
+    dq[e] = scale * ds * q[d + e];
+    dq[d + e] = scale * ds * q[e];
+    dq[2 * d + e] = p * dav[e];
+  }
+  if (lane == 0) delta[r * H + h] = dl;
+}
+
+// One block, key side: thread = key row i of keys [k0, k0 + nk), all of one
+// (b, h) per blockIdx.x; loops over the block's queries.
+template <int DH>
+__global__ void __launch_bounds__(128) k_attn_bwd_block_kv(const float* __restrict__ qkv, const float* __restrict__ K,
+                                                           const float* __restrict__ V,
+                                                           const float* __restrict__ lse,
+                                                           const float* __restrict__ delta,
+                                                           const float* __restrict__ da, float* __restrict__ dK,
+                                                           float* __restrict__ dV, int B, int H, int q0, int nq,
+                                                           int k0, int nk, float scale) {
+  const int b = blockIdx.x / H, h = blockIdx.x - b * H;
+  const int i = k0 + blockIdx.y * 128 + threadIdx.x;
+  if (i >= k0 + nk) return;
+  const int d = H * DH;
+  const size_t ri = (size_t)i * B + b;
+  float k[DH], v[DH], gk[DH], gv[DH];
+#pragma unroll
+  for (int e = 0; e < DH; ++e) { k[e] = K[ri * d + h * DH + e]; v[e] = V[ri * d + h * DH + e]; gk[e] = gv[e] = 0.f; }
+  for (int j = q0; j < q0 + nq; ++j) {
+    const size_t rj = (size_t)j * B + b;
+    const float* q = qkv + rj * 3 * d + h * DH;
+    const float* dav = da + rj * d + h * DH;
     float s = 0.f, dp = 0.f;
 #pragma unroll
-    for (int e = 0; e < DH; ++e) {
-      s += qr[e] * k[e];
-      dp += dar[e] * v[e];
-    }
-    const float p = expf(s * scale - L);
-    const float ds = p * (dp - delta);
-    float* dk = temp ? dqrow + d : dK + ((size_t)i * B + b) * d + h * DH;
-    float* dv = temp ? dqrow + 2 * d : dV + ((size_t)i * B + b) * d + h * DH;
+    for (int e = 0; e < DH; ++e) { s += q[e] * k[e]; dp += dav[e] * v[e]; }
+    const float p = expf(s * scale - lse[rj * H + h]);
+    const float ds = p * (dp - delta[rj * H + h]);
 #pragma unroll
-    for (int e = 0; e < DH; ++e) {
-      dq[e] += scale * ds * k[e];
-      const float gk = scale * ds * qr[e], gv = p * dar[e];
-      if (temp) { dk[e] = gk; dv[e] = gv; }
-      else { dk[e] += gk; dv[e] += gv; }
-    }
+    for (int e = 0; e < DH; ++e) { gk[e] += scale * ds * q[e]; gv[e] += p * dav[e]; }
   }
 #pragma unroll
-  for (int e = 0; e < DH; ++e) {
-    const float v = warp_sum(dq[e]);
-    if (lane == (e & 31)) dqrow[e] = v;
+  for (int e = 0; e < DH; ++e) { dK[ri * d + h * DH + e] += gk[e]; dV[ri * d + h * DH + e] += gv[e]; }
+}
+
+// One block, query side: thread = query row j of queries [q0, q0 + nq);
+// adds its block term to dq_j.
+template <int DH>
+__global__ void __launch_bounds__(128) k_attn_bwd_block_q(const float* __restrict__ qkv, const float* __restrict__ K,
+                                                          const float* __restrict__ V,
+                                                          const float* __restrict__ lse,
+                                                          const float* __restrict__ delta,
+                                                          const float* __restrict__ da, float* __restrict__ dqkv,
+                                                          int B, int H, int q0, int nq, int k0, int nk,
+                                                          float scale) {
+  const int b = blockIdx.x / H, h = blockIdx.x - b * H;
+  const int j = q0 + blockIdx.y * 128 + threadIdx.x;
+  if (j >= q0 + nq) return;
+  const int d = H * DH;
+  const size_t rj = (size_t)j * B + b;
+  float q[DH], dav[DH], gq[DH];
+#pragma unroll
+  for (int e = 0; e < DH; ++e) { q[e] = qkv[rj * 3 * d + h * DH + e]; dav[e] = da[rj * d + h * DH + e]; gq[e] = 0.f; }
+  const float L = lse[rj * H + h], dl = delta[rj * H + h];
+  for (int i = k0; i < k0 + nk; ++i) {
+    const size_t ri = (size_t)i * B + b;
+    const float* k = K + ri * d + h * DH;
+    const float* v = V + ri * d + h * DH;
+    float s = 0.f, dp = 0.f;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) { s += q[e] * k[e]; dp += dav[e] * v[e]; }
+    const float ds = expf(s * scale - L) * (dp - dl);
+#pragma unroll
+    for (int e = 0; e < DH; ++e) gq[e] += scale * ds * k[e];
   }
+#pragma unroll
+  for (int e = 0; e < DH; ++e) dqkv[rj * 3 * d + h * DH + e] += gq[e];
 }
 
 // ---------------------------------------------------------------------------
@@ -283,7 +335,7 @@ __global__ void __launch_bounds__(128) k_attn_bwd_step(const float* __restrict__
 // ---------------------------------------------------------------------------
 struct BwdPlan {
   size_t off_in, off_out;   // bf16 storage: fp32 copies of the 13 inputs / the 7 outputs
-  size_t off_err, off_xp, off_xr, off_cx, off_qkv, off_a, off_lse, off_u, off_ur, off_cu, off_hp, off_g, off_zp,
+  size_t off_err, off_xp, off_xr, off_cx, off_qkv, off_a, off_lse, off_delta, off_u, off_ur, off_cu, off_hp, off_g, off_zp,
       off_zr, off_cz, off_dzu, off_dKa, off_dVa, off_dZ, off_dH, off_dU, off_dA, off_dqkv, off_dzr, off_dg,
       off_dur, off_dxr, off_dxp, total;
 };
@@ -321,6 +373,7 @@ static BwdPlan bwd_plan(int B, int N, int d, int H, int d_ff, int dtype) {
   P.off_qkv = take(R * 3 * d * f);
   P.off_a = take(R * d * f);
   P.off_lse = take(R * H * f);
+  P.off_delta = take(R * H * f);
   P.off_u = take(R * d * f);
   P.off_ur = take(R * d * f);
   P.off_cu = take(R * f);
@@ -362,6 +415,32 @@ static cudaError_t gemm(const float* A, int lda, int ta, const float* W, int ldw
 }
 
 static unsigned grid_for(size_t n) { return (unsigned)std::min<size_t>((n + 255) / 256, 65535); }
+
+// Attention backward of reverse step t (0-based position row t): the
+// temporary pair of query t, then the forward's block of step t (1-based:
+// keys rows [t - lb, t), queries rows [t, t + lb) clipped at N), whose
+// earliest query is row t.
+template <int DH>
+static cudaError_t attn_bwd_dh(const float* qkv, const float* K, const float* V, const float* a, const float* lse,
+                               const float* da, float* delta, float* dK, float* dV, float* dqkv, int B, int N, int H,
+                               int t, float scale, cudaStream_t st) {
+  k_attn_bwd_temp<DH><<<(unsigned)((B * H + 3) / 4), 128, 0, st>>>(qkv, a, lse, da, delta, dqkv, B, H, t, scale);
+  if (t >= 1) {
+    const int lb = lowbit(t), nq = std::min(lb, N - t), k0 = t - lb;
+    k_attn_bwd_block_kv<DH><<<dim3((unsigned)(B * H), (unsigned)((lb + 127) / 128)), 128, 0, st>>>(
+        qkv, K, V, lse, delta, da, dK, dV, B, H, t, nq, k0, lb, scale);
+    k_attn_bwd_block_q<DH><<<dim3((unsigned)(B * H), (unsigned)((nq + 127) / 128)), 128, 0, st>>>(
+        qkv, K, V, lse, delta, da, dqkv, B, H, t, nq, k0, lb, scale);
+  }
+  return cudaGetLastError();
+}
+static cudaError_t attn_bwd(int dh, const float* qkv, const float* K, const float* V, const float* a,
+                            const float* lse, const float* da, float* delta, float* dK, float* dV, float* dqkv, int B,
+                            int N, int H, int t, float scale, cudaStream_t st) {
+  if (dh == 32) return attn_bwd_dh<32>(qkv, K, V, a, lse, da, delta, dK, dV, dqkv, B, N, H, t, scale, st);
+  if (dh == 64) return attn_bwd_dh<64>(qkv, K, V, a, lse, da, delta, dK, dV, dqkv, B, N, H, t, scale, st);
+  return attn_bwd_dh<128>(qkv, K, V, a, lse, da, delta, dK, dV, dqkv, B, N, H, t, scale, st);
+}
 
 }  // namespace bwd
 }  // namespace rt
@@ -437,7 +516,7 @@ extern "C" int rt_layer_backward(const void* x_, const void* Wq_, const void* Wk
         *dWv = static_cast<float*>(dWv_), *dWo = static_cast<float*>(dWo_), *dW1 = static_cast<float*>(dW1_),
         *dW2 = static_cast<float*>(dW2_);
   float *xp = F(P.off_xp), *xr = F(P.off_xr), *cx = F(P.off_cx), *qkv = F(P.off_qkv), *a = F(P.off_a),
-        *lse = F(P.off_lse), *u = F(P.off_u), *ur = F(P.off_ur), *cu = F(P.off_cu), *hp = F(P.off_hp),
+        *lse = F(P.off_lse), *delta = F(P.off_delta), *u = F(P.off_u), *ur = F(P.off_ur), *cu = F(P.off_cu), *hp = F(P.off_hp),
         *g = F(P.off_g), *zp = F(P.off_zp), *zr = F(P.off_zr), *cz = F(P.off_cz), *dzu = F(P.off_dzu),
         *dKa = F(P.off_dKa), *dVa = F(P.off_dVa), *dZ = F(P.off_dZ), *dH = F(P.off_dH), *dU = F(P.off_dU),
         *dA = F(P.off_dA), *dqkv = F(P.off_dqkv), *dzr = F(P.off_dzr), *dg = F(P.off_dg), *dur = F(P.off_dur),
@@ -493,12 +572,7 @@ extern "C" int rt_layer_backward(const void* x_, const void* Wq_, const void* Wk
     RT_BCK(cudaGetLastError());
     // da = du W_o, then the attention backward of query t
     RT_BCK(gemm(dU + r0 * d, d, 0, Wo, d, 1, dA + r0 * d, d, B, d, d, 0, st));
-    {
-      const unsigned g = (unsigned)((B * H + 3) / 4);
-      if (dh == 32) k_attn_bwd_step<32><<<g, 128, 0, st>>>(qkv, K, V, a, lse, dA, dKa, dVa, dqkv, B, H, t, scale);
-      else if (dh == 64) k_attn_bwd_step<64><<<g, 128, 0, st>>>(qkv, K, V, a, lse, dA, dKa, dVa, dqkv, B, H, t, scale);
-      else k_attn_bwd_step<128><<<g, 128, 0, st>>>(qkv, K, V, a, lse, dA, dKa, dVa, dqkv, B, H, t, scale);
-    }
+    RT_BCK(attn_bwd(dh, qkv, K, V, a, lse, dA, delta, dKa, dVa, dqkv, B, N, H, t, scale, st));
     RT_BCK(cudaGetLastError());
   }
 
