@@ -80,9 +80,13 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return launch_pdl_cluster(kern, grid, block, smem, st, 1, std::forward<Args>(args)...);
 }
 
-// The persistent step kernel: one CTA per SM, all co-resident (cooperative
-// launch), since its tasks wait on flags set by other CTAs.
-static cudaError_t launch_steps(const StepsParams& sp, int sms, cudaStream_t st) {
+// The persistent step kernel: one CTA per SM, all co-resident, since its
+// tasks wait on flags set by other CTAs. The launch is cooperative (the
+// driver guarantees co-residency or refuses); `coop` = false launches the
+// same grid plainly -- one CTA per SM fits (shared memory allows no second)
+// and the previous kernel of the stream has finished, so the CTAs are
+// resident together in practice, and every wait is bounded regardless.
+static cudaError_t launch_steps(const StepsParams& sp, int sms, cudaStream_t st, bool coop) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)sms);
   cfg.blockDim = dim3(StepsCfg::THREADS);
@@ -92,7 +96,7 @@ static cudaError_t launch_steps(const StepsParams& sp, int sms, cudaStream_t st)
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = coop ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k_steps, sp);
 }
 
@@ -107,6 +111,9 @@ typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint3
 struct DevState {
   bool ready = false;
   int sms = 0;
+  // the step kernel's launches are cooperative unless this device's driver
+  // refused a cooperative launch (then plain, see launch_steps)
+  bool coop = true;
   cudaStream_t capture = nullptr;
   cudaStream_t h2d = nullptr, d2h = nullptr;   // transfer streams of the host-buffer entry point
   std::vector<cudaEvent_t> events;             // fork/join events of the host-buffer entry point
@@ -721,7 +728,14 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
       sp.j1 = j1;
       {
         TimedScope ts(T, KC_STEPS, st);
-        RT_CK(launch_steps(sp, ds.sms, st));
+        cudaError_t e = launch_steps(sp, ds.sms, st, ds.coop);
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (e != cudaSuccess && ds.coop && cudaStreamIsCapturing(st, &cs) == cudaSuccess &&
+            cs == cudaStreamCaptureStatusNone) {
+          cudaGetLastError();   // outside capture: the same grid, launched plainly
+          e = launch_steps(sp, ds.sms, st, false);
+        }
+        RT_CK(e);
       }
       const int t = j1;
       if (t < N) {
@@ -1065,9 +1079,22 @@ static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st
   auto it = g_graphs.find(key);
   if (it == g_graphs.end()) {
     cudaGraph_t graph = nullptr;
-    RT_CK(cudaStreamBeginCapture(ds->capture, cudaStreamCaptureModeThreadLocal));
-    rc = enqueue_forward(P, X, *ds, ds->capture, nullptr, io);
-    cudaError_t ce = cudaStreamEndCapture(ds->capture, &graph);
+    cudaError_t ce = cudaSuccess;
+    for (int attempt = 0; attempt < 2; ++attempt) {
+      RT_CK(cudaStreamBeginCapture(ds->capture, cudaStreamCaptureModeThreadLocal));
+      rc = enqueue_forward(P, X, *ds, ds->capture, nullptr, io);
+      ce = cudaStreamEndCapture(ds->capture, &graph);
+      // a capture that failed on the step kernel's cooperative launch is
+      // recorded once more with plain launches
+      if ((rc == RT_ERR_CUDA || ce != cudaSuccess) && P.sp.ok && ds->coop && attempt == 0) {
+        if (graph) cudaGraphDestroy(graph);
+        graph = nullptr;
+        cudaGetLastError();
+        ds->coop = false;
+        continue;
+      }
+      break;
+    }
     if (rc != RT_OK) {
       if (graph) cudaGraphDestroy(graph);
       return rc;
