@@ -1346,7 +1346,7 @@ extern "C" int rt_block_fold(const void* Q, int q_stride, const void* K, const v
   if (dtype == RT_BF16)
     e = launch_fold<bf16>(static_cast<const bf16*>(Q), q_stride, static_cast<const bf16*>(K),
                           static_cast<const bf16*>(V), kv_stride, m, l, o, nullptr, B, H, d_h, q0, nq, k0, nk, sc2, 0,
-                          0, true, st, static_cast<unsigned*>(err_dev), 128, ds->sms);
+                          0, true, st, static_cast<unsigned*>(err_dev), kFoldTcMinBlock, ds->sms);
   else if (dtype == RT_F32)
     e = launch_fold<float>(static_cast<const float*>(Q), q_stride, static_cast<const float*>(K),
                            static_cast<const float*>(V), kv_stride, m, l, o, nullptr, B, H, d_h, q0, nq, k0, nk, sc2, 0,

@@ -302,6 +302,8 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       // this item's Q buffer may be refilled (the MMA thread also arrives)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[li & 1]);
     };
 
     for (int g = 0; g < total && ok; ++g) {

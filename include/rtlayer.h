@@ -283,9 +283,10 @@ int rt_embed_forward(const int32_t* ids_dev, const void* E_dev, int B, int N,
  * Folds keys [k0, k0 + nk) into queries [q0, q0 + nq) (0-based positions),
  * updating (m, l, o) in place. m is stored in log2 units scaled by
  * log2(e)/sqrt(d_h) (m = -inf marks an empty accumulator).
- * RT_BF16 needs d_h = 64. Kernel by key count nk: <= 8 the small-block
- * kernel; multiples of 128 the tcgen05 kernels; other multiples of 16 the
- * mma.sync kernel; anything else the warp kernel.
+ * RT_BF16 needs d_h = 64. The kernel is the one rt_layer_forward runs for a
+ * block of nk keys: <= 8 the small-block kernel; multiples of 128 from 1024
+ * on the tcgen05 kernels; other multiples of 16 the mma.sync kernel; anything
+ * else the warp kernel.
  * err_dev: error word of the tcgen05 kernels' bounded waits, as in
  * rt_project_qkv (read with rt_layer_sync_status). */
 int rt_block_fold(const void* Q_dev, int q_stride, const void* K_dev,

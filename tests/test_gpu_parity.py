@@ -81,6 +81,7 @@ def test_batched_projection_matches_oracle(rt, dtype, B, N, d):
     ("bf16", 128, 77, False), ("bf16", 128, 128, True), ("bf16", 512, 300, True), ("bf16", 384, 1, False),
     ("bf16", 40, 6, False),                                                      # generic warp kernel
     ("bf16", 2048, 300, False), ("bf16", 4096, 129, True),                     # the blocks of N >= 4096
+    ("bf16", 1024, 100, False), ("bf16", 1024, 128, True),                     # one-tile tcgen05 kernel
     ("f32", 3, 4, False), ("f32", 16, 16, True), ("f32", 64, 33, False)])
 def test_block_fold_matches_oracle(rt, dtype, nk, nq, init_empty):
     B, H, dh = 3, 2, 64 if dtype == "bf16" else 32
@@ -307,3 +308,37 @@ def test_component_entry_point_reports_through_its_error_word(rt):
     C = rt.gemm_bf16(to_device(A, "bf16"), to_device(W, "bf16"), err=err)
     assert rt.sync_status(err) == 0
     assert rel_err(to_np(C), A @ W.T) < 1e-5
+
+
+@pytest.mark.parametrize("nk,nq", [(1024, 64), (1024, 300)])
+def test_tcgen05_fold_with_several_items_per_cta(rt, nk, nq):
+    # 28 sequences x 16 heads: every persistent CTA of the tcgen05 folds takes
+    # three or more (pair, query tile) items, so the query buffers are
+    # refilled (the buffer release by the softmax warps is exercised); the
+    # error word must stay clear and sampled pairs match the oracle
+    B, H, dh = 28, 16, 64
+    d = H * dh
+    npos = nk + nq
+    rng = np.random.default_rng(nk + nq)
+    Q = rtinputs.to_grid(rng.standard_normal((npos, B, d)), "bf16")
+    Kc = rtinputs.to_grid(rng.standard_normal((npos, B, d)), "bf16")
+    Vc = rtinputs.to_grid(rng.standard_normal((npos, B, d)), "bf16")
+    mg = torch.full((npos, B, H), -float("inf"), device="cuda")
+    lg = torch.zeros((npos, B, H), device="cuda")
+    og = torch.zeros((npos, B, d), device="cuda")
+    err = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    rt.block_fold(to_device(Q, "bf16"), to_device(Kc, "bf16"), to_device(Vc, "bf16"), mg, lg, og, H, dh, nk, nq, 0, nk,
+                  err=err)
+    assert rt.sync_status(err) == 0
+    sb = [0, 27]
+    qh = Q[nk:, sb].reshape(nq, 2, H, dh).transpose(1, 2, 0, 3)
+    kh = Kc[:nk, sb].reshape(nk, 2, H, dh).transpose(1, 2, 0, 3)
+    vh = Vc[:nk, sb].reshape(nk, 2, H, dh).transpose(1, 2, 0, 3)
+    mr = np.full((2, H, nq), -np.inf)
+    lr = np.zeros((2, H, nq))
+    orr = np.zeros((2, H, nq, dh))
+    mr, lr, orr = O.block_fold(qh, kh, vh, mr, lr, orr, 1.0 / math.sqrt(dh))
+    l_got = to_np(lg)[nk:, sb].transpose(1, 2, 0)
+    o_got = to_np(og)[nk:, sb].reshape(nq, 2, H, dh).transpose(1, 2, 0, 3)
+    bound = 2.0 ** -9 * np.max(np.abs(Vc[:nk, sb])) * 1.01 + 1e-5
+    assert np.max(np.abs(o_got / l_got[..., None] - orr / lr[..., None])) <= bound
