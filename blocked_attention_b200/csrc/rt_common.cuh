@@ -43,13 +43,26 @@ __device__ __forceinline__ void set_error(unsigned* err, unsigned bits) {
 // the error word (rt_layer_sync_status then returns RT_ERR_INVALID_ARG) and
 // the access is skipped. Nothing traps. In the normal build the check is the
 // constant true and compiles away.
+// The first failed check also leaves a record after the error word: word 1 =
+// the check's id (1-based), words 2 and 3 = two of its values (the caller's
+// error word must have room for four words; the layer's workspace reserves
+// 256 bytes).
 #ifdef RT_BOUNDS_CHECK
-__device__ __forceinline__ bool idx_ok(bool ok, unsigned* err) {
-  if (!ok) set_error(err, RT_DEVERR_INDEX);
+__device__ __forceinline__ bool idx_ok(bool ok, unsigned* err, unsigned id = 0, long long a = 0,
+                                       long long b = 0) {
+  if (!ok) {
+    set_error(err, RT_DEVERR_INDEX);
+    if (err && id && atomicCAS(err + 1, 0u, id) == 0u) {
+      err[2] = (unsigned)a;
+      err[3] = (unsigned)b;
+    }
+  }
   return ok;
 }
 #else
-__device__ __forceinline__ constexpr bool idx_ok(bool, unsigned*) { return true; }
+__device__ __forceinline__ constexpr bool idx_ok(bool, unsigned*, unsigned = 0, long long = 0, long long = 0) {
+  return true;
+}
 #endif
 
 // ---------------------------------------------------------------------------

@@ -191,8 +191,16 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& p, int row, i
 // of the value that feeds the next RMSNorm (WO: u, W2: z), else 0.
 template <int EPI>
 __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int col0, int N,
-                                                float (&v)[32], float row_scale) {
+                                                float (&v)[32], float row_scale, unsigned* dbg_err = nullptr) {
   float ssq = 0.f;
+  if constexpr (EPI == EPI_WO || EPI == EPI_W2 || EPI == EPI_WKV) {
+    // (debug build) the step rows and the output columns
+    if (!idx_ok(p.j + row / p.B < p.Nseq && col0 + 32 <= (EPI == EPI_WKV ? 2 * p.d : p.d) && (col0 & 31) == 0,
+                dbg_err, 20 + EPI, row, col0))
+      return 0.f;
+  } else if constexpr (EPI == EPI_W1) {
+    if (!idx_ok(col0 + 32 <= p.d_ff && (col0 & 31) == 0, dbg_err, 20 + EPI, row, col0)) return 0.f;
+  }
   if constexpr (EPI == EPI_PLAIN) {
     float* dst = p.c32 + (size_t)row * N + col0;
     if (col0 + 32 <= N && (N % 4) == 0) {

@@ -350,7 +350,8 @@ __device__ __forceinline__ void fold_small_units(const StepsParams& P, int q0, i
                                                     (oo[2 * k + 1] * a2 + pt * vt[2 * k + 1]) * inv);
           wp[k] = *reinterpret_cast<uint32_t*>(&v2);
         }
-        *reinterpret_cast<uint4*>(P.a16 + (size_t)b * d + h * 64 + sl * 8) = w;
+        if (idx_ok(b < B && h < H, P.err, 16, b, h))
+          *reinterpret_cast<uint4*>(P.a16 + (size_t)b * d + h * 64 + sl * 8) = w;
       } else {
         float* op = P.o + row * (size_t)d + h * 64 + sl * 8;
         if (sl == 0) {
@@ -386,7 +387,7 @@ __device__ __forceinline__ void tmem_ld_pair(uint32_t taddr, bool two, float (&v
 
 template <int EPI>
 __device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool row_ok, int col_base, int BN, int N,
-                                               uint32_t taddr, bool two, float rs) {
+                                               uint32_t taddr, bool two, float rs, unsigned* dbg_err) {
   float ssq = 0.f;
   if constexpr (EPI == EPI_WKV) {
     if (e.pages) {   // per-head unit RMS of k (the paper's parameterisation)
@@ -404,7 +405,7 @@ __device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool
   for (int c = 0; c < BN; c += 32) {
     float v[32];
     tmem_ld_pair(taddr + c, two, v);
-    if (row_ok) ssq += epilogue_chunk<EPI>(e, row, col_base + c, N, v, rs);
+    if (row_ok) ssq += epilogue_chunk<EPI>(e, row, col_base + c, N, v, rs, dbg_err);
   }
   return ssq;
 }
@@ -482,7 +483,9 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], ns * (C::A_SUB + bn_bytes));
           for (int q = 0; q < ns; ++q)
-            tma_load_2d(&P.tB[ph], &full[s], sB + s * C::B_BYTES + q * C::B_SUB, (kb + q) * C::BK, T.tile * g.BN);
+            if (idx_ok((kb + q + 1) * C::BK <= g.K && (T.tile + 1) * g.BN <= g.N && s < (uint32_t)C::STAGES &&
+                           g.BN <= C::BN_MAX, P.err, 11, kb + q, T.tile))
+              tma_load_2d(&P.tB[ph], &full[s], sB + s * C::B_BYTES + q * C::B_SUB, (kb + q) * C::BK, T.tile * g.BN);
         }
         if (deps) {
           int lo, hi, t2;
@@ -500,7 +503,8 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         }
         if (lane == 0)
           for (int q = 0; q < ns; ++q)
-            tma_load_2d(&P.tA[ph], &full[s], sA + s * C::A_BYTES + q * C::A_SUB, (kb + q) * C::BK, T.rb * C::BM);
+            if (idx_ok((kb + q + 1) * C::BK <= g.K && T.rb * C::BM < P.ep.B, P.err, 12, kb + q, T.rb))
+              tma_load_2d(&P.tA[ph], &full[s], sA + s * C::A_BYTES + q * C::A_SUB, (kb + q) * C::BK, T.rb * C::BM);
       }
       return true;
     });
@@ -524,6 +528,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         if (!mbar_wait_g(&tempty[acc], aph ^ 1u, P.err)) return false;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (acc * 2 + par) * C::BN_MAX;
+        idx_ok((acc * 2 + par) * C::BN_MAX + g.BN <= C::TMEM_COLS && nst >= 1, P.err, 13, acc, nst);
         const uint32_t idesc = idesc_bf16_f32(C::BM, g.BN);
         uint32_t accumulate = 0;
         for (int kb = 0; kb < nst; ++kb, ++it) {
@@ -630,20 +635,24 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       if (g.S == 1) {
         float ssq = 0.f;
         switch (ph) {
-          case PH_WO: ssq = epi_tile_tmem<EPI_WO>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs); break;
-          case PH_W1: epi_tile_tmem<EPI_W1>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs); break;
-          case PH_W2: ssq = epi_tile_tmem<EPI_W2>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs); break;
-          default: epi_tile_tmem<EPI_WKV>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs); break;
+          case PH_WO: ssq = epi_tile_tmem<EPI_WO>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs, P.err); break;
+          case PH_W1: epi_tile_tmem<EPI_W1>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs, P.err); break;
+          case PH_W2: ssq = epi_tile_tmem<EPI_W2>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs, P.err); break;
+          default: epi_tile_tmem<EPI_WKV>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs, P.err); break;
         }
-        if (row_ok && ph == PH_WO) P.ssq_u[(size_t)T.tile * P.ep.B + row] = ssq;
-        if (row_ok && ph == PH_W2) P.ssq_z[(size_t)T.tile * P.ep.B + row] = ssq;
+        if (row_ok && ph == PH_WO && idx_ok(T.tile <= P.ep.d / 32, P.err, 15, T.tile, 0))
+          P.ssq_u[(size_t)T.tile * P.ep.B + row] = ssq;
+        if (row_ok && ph == PH_W2 && idx_ok(T.tile <= P.ep.d / 32, P.err, 15, T.tile, 1))
+          P.ssq_z[(size_t)T.tile * P.ep.B + row] = ssq;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
       } else {
         // split of W2: this split's partial tile to its slot ([col][row], so
         // that a warp's stores and loads are 128-byte lines)
-        float* slot = P.w2part + (((size_t)T.rb * g.tiles + T.tile) * g.S + T.split) * (size_t)g.BN * C::BM;
+        const size_t slot_i = ((size_t)T.rb * g.tiles + T.tile) * g.S + T.split;
+        idx_ok(slot_i < (size_t)P.nrb * g.tiles * g.S && T.split < g.S, P.err, 14, (long long)slot_i, T.split);
+        float* slot = P.w2part + slot_i * (size_t)g.BN * C::BM;
 #pragma unroll 1
         for (int c = 0; c < g.BN; c += 32) {
           float v[32];
@@ -683,7 +692,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] += __ldcg(src + (size_t)i * C::BM);
             }
-            if (row_ok) ssq += epilogue_chunk<EPI_W2>(e, row, col_base + c, g.N, v, 1.f);
+            if (row_ok) ssq += epilogue_chunk<EPI_W2>(e, row, col_base + c, g.N, v, 1.f, P.err);
           }
           if (row_ok) P.ssq_z[(size_t)T.tile * P.ep.B + row] = ssq;
         }
