@@ -59,10 +59,19 @@ __device__ __forceinline__ bool idx_ok(bool ok, unsigned* err, unsigned id = 0, 
   }
   return ok;
 }
+// (debug build) the first bounded wait that ran out leaves the same kind of
+// record: id, then two values describing the wait
+__device__ __forceinline__ void timeout_record(unsigned* err, unsigned id, long long a, long long b) {
+  if (err && atomicCAS(err + 1, 0u, id) == 0u) {
+    err[2] = (unsigned)a;
+    err[3] = (unsigned)b;
+  }
+}
 #else
 __device__ __forceinline__ constexpr bool idx_ok(bool, unsigned*, unsigned = 0, long long = 0, long long = 0) {
   return true;
 }
+__device__ __forceinline__ void timeout_record(unsigned*, unsigned, long long, long long) {}
 #endif
 
 // ---------------------------------------------------------------------------

@@ -35,7 +35,7 @@ namespace {
 
 constexpr size_t kMaxRows = size_t(1) << 20;   // B*N limit: 4 MiB of fp32
 static __device__ __align__(256) float g_inv_rms_scratch[kMaxRows];
-static __device__ unsigned g_noalloc_err;
+static __device__ unsigned g_noalloc_err[4];   // error word (+ the debug build's failure record)
 
 struct DeviceSlot {
   bool ready = false;
@@ -76,7 +76,7 @@ int setup_current_device(DeviceSlot** out) {
     void* q = nullptr;
     if ((e = cudaGetSymbolAddress(&q, g_noalloc_err)) != cudaSuccess) return rt::cuda_failure(e);
     if (!q) return RT_ERR_CUDA;
-    if ((e = cudaMemset(q, 0, sizeof(unsigned))) != cudaSuccess) return rt::cuda_failure(e);
+    if ((e = cudaMemset(q, 0, sizeof(g_noalloc_err))) != cudaSuccess) return rt::cuda_failure(e);
     s.scratch = static_cast<float*>(p);
     s.err = static_cast<unsigned*>(q);
     s.ready = true;

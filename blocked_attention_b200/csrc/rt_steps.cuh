@@ -131,16 +131,21 @@ __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: 
 // Bounded poll until *f >= target (acquire). Returns at once once the error
 // word is set; a poll that runs out sets RT_DEVERR_TIMEOUT. Either way the
 // caller proceeds.
-__device__ __noinline__ void poll_ge(const unsigned* f, unsigned target, unsigned* err) {
+// (debug build: a wait that runs out records `id` and `where`, and the value
+// it saw, after the error word)
+__device__ __noinline__ void poll_ge(const unsigned* f, unsigned target, unsigned* err, unsigned id = 0,
+                                     long long where = 0) {
   if (ld_acquire_u32(f) >= target) return;
   const unsigned long long t0 = globaltimer();
   for (unsigned it = 1;; ++it) {
     __nanosleep(64);
-    if (ld_acquire_u32(f) >= target) return;
+    const unsigned v = ld_acquire_u32(f);
+    if (v >= target) return;
     if ((it & 15u) == 0) {
       if (ld_volatile_u32(err) != 0) return;
       if (globaltimer() - t0 > kWaitLimitNs) {
         set_error(err, RT_DEVERR_TIMEOUT);
+        timeout_record(err, id, where, ((long long)v << 16) | (target & 0xffff));
         return;
       }
     }
@@ -148,7 +153,8 @@ __device__ __noinline__ void poll_ge(const unsigned* f, unsigned target, unsigne
 }
 
 // mbarrier wait bounded by time and abandoned once the error word is set.
-__device__ __forceinline__ bool mbar_wait_g(uint64_t* bar, unsigned parity, unsigned* err) {
+__device__ __forceinline__ bool mbar_wait_g(uint64_t* bar, unsigned parity, unsigned* err, unsigned id = 0,
+                                            long long where = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (unsigned it = 1;; ++it) {
@@ -157,10 +163,16 @@ __device__ __forceinline__ bool mbar_wait_g(uint64_t* bar, unsigned parity, unsi
       if (ld_volatile_u32(err) != 0) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
         set_error(err, RT_DEVERR_TIMEOUT);
+        timeout_record(err, id, where, parity);
         return false;
       }
     }
   }
+}
+
+// where a wait is: CTA, step, phase and the task's index in its phase
+__device__ __forceinline__ long long wait_site(int ph, int j, int loc) {
+  return ((long long)blockIdx.x << 24) | ((long long)(j & 0xfff) << 12) | ((ph & 7) << 9) | (loc & 0x1ff);
 }
 
 // ---------------------------------------------------------------------------
@@ -414,10 +426,10 @@ __device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool
 // epilogue threads (thread i polls flag i of a contiguous range), then one
 // fence per polling thread and the epilogue barrier.
 __device__ __forceinline__ void epi_poll_range(const StepsParams& P, int ph, int rb, int lo, int hi, unsigned target,
-                                               int tid) {
+                                               int tid, int task_ph = 7, int task_loc = 0) {
   bool polled = false;
   for (int i = lo + tid; i < hi; i += 128) {
-    poll_ge(flag_ptr(P, ph, rb, i), target, P.err);
+    poll_ge(flag_ptr(P, ph, rb, i), target, P.err, 46, wait_site(task_ph, (int)target, (ph << 6) | (i & 63)));
     polled = true;
   }
   if (polled) __threadfence();
@@ -477,7 +489,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         const int ns = min(C::KSUB, T.sl1 - kb);
         const uint32_t s = it % C::STAGES, par = (it / C::STAGES) & 1u;
         int w = 1;
-        if (lane == 0) w = mbar_wait_g(&empty[s], par ^ 1u, P.err) ? 1 : 0;
+        if (lane == 0) w = mbar_wait_g(&empty[s], par ^ 1u, P.err, 41, wait_site(ph, j, loc)) ? 1 : 0;
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) { ok = false; return false; }
         if (lane == 0) {
@@ -494,7 +506,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
           for (int i = 0; i < 3; ++i) {
             const int f = flo + lane + 32 * i;
             if (f >= lo && f < hi && f < fhi && !(rdy >> i & 1u)) {
-              poll_ge(flag_ptr(P, dph, T.rb, f), target, P.err);
+              poll_ge(flag_ptr(P, dph, T.rb, f), target, P.err, 42, wait_site(ph, j, f));
               rdy |= 1u << i;
             }
           }
@@ -525,7 +537,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         const int nst = (T.sl1 - T.sl0 + C::KSUB - 1) / C::KSUB;
         const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
         ++local;
-        if (!mbar_wait_g(&tempty[acc], aph ^ 1u, P.err)) return false;
+        if (!mbar_wait_g(&tempty[acc], aph ^ 1u, P.err, 43, wait_site(ph, j, loc))) return false;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (acc * 2 + par) * C::BN_MAX;
         idx_ok((acc * 2 + par) * C::BN_MAX + g.BN <= C::TMEM_COLS && nst >= 1, P.err, 13, acc, nst);
@@ -534,7 +546,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         for (int kb = 0; kb < nst; ++kb, ++it) {
           if ((kb & 1) != par) continue;
           const uint32_t s = it % C::STAGES, sp = (it / C::STAGES) & 1u;
-          if (!mbar_wait_g(&full[s], sp, P.err)) return false;
+          if (!mbar_wait_g(&full[s], sp, P.err, 44, wait_site(ph, j, loc))) return false;
           tc_fence_after();
           const uint8_t* a_st = sA + s * C::A_BYTES;
           const uint8_t* b_st = sB + s * C::B_BYTES;
@@ -570,8 +582,8 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         const int t = j + 1, lb = lowbit(t), nq = min(lb, P.ep.Nseq - t);
         // this head's k and v of step j (and, through them, everything before)
         const int kt = (64 * h) / P.g[PH_WKV].BN, vt = (P.ep.d + 64 * h) / P.g[PH_WKV].BN;
-        if (tid == 0) { poll_ge(flag_ptr(P, PH_WKV, rb, kt), j + 1, P.err); __threadfence(); }
-        if (tid == 32) { poll_ge(flag_ptr(P, PH_WKV, rb, vt), j + 1, P.err); __threadfence(); }
+        if (tid == 0) { poll_ge(flag_ptr(P, PH_WKV, rb, kt), j + 1, P.err, 47, wait_site(ph, j, kt)); __threadfence(); }
+        if (tid == 32) { poll_ge(flag_ptr(P, PH_WKV, rb, vt), j + 1, P.err, 47, wait_site(ph, j, vt)); __threadfence(); }
         epi_bar();
         const int s0 = rb * 128 + gi * kFoldSeqs;
         const int ns = min(kFoldSeqs, min(P.ep.B - s0, (rb + 1) * 128 - s0));
@@ -626,7 +638,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       // A wait that gives up (error word set) does not end the task: the four
       // epilogue warps must reach every named barrier together, so they run
       // on with whatever tensor memory holds.
-      if (lane == 0) mbar_wait_g(&tfull[acc], aph, P.err);
+      if (lane == 0) mbar_wait_g(&tfull[acc], aph, P.err, 45, wait_site(ph, j, loc));
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * 2 * C::BN_MAX;

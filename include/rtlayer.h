@@ -298,10 +298,12 @@ int rt_block_fold(const void* Q_dev, int q_stride, const void* K_dev,
  *   QKV_dev[n][b][0:d] = W_q rms(x[b][n]), [d:2d] = W_k rms(..), [2d:3d] = W_v rms(..)
  * position-major [N][B][3d]. W_qkv_dev is [3d][d] (W_q; W_k; W_v stacked).
  * scratch_dev: >= B*N*4 bytes (RT_BF16) or B*N*d*4 bytes (RT_F32).
- * err_dev: a 4-byte-aligned device word (e.g. the first bytes of a layer
- * workspace) into which the tensor-core kernel's bounded waits record a
- * timeout; it is only ever OR-ed into, so it accumulates over calls until
- * rt_layer_sync_status(err_dev, stream) reads and clears it. NULL is
+ * err_dev: 16 bytes of device memory, 4-byte aligned (e.g. the first bytes
+ * of a layer workspace), whose first word is the error word into which the
+ * tensor-core kernel's bounded waits record a timeout; it is only ever OR-ed
+ * into, so it accumulates over calls until rt_layer_sync_status(err_dev,
+ * stream) reads and clears it (the debug library, librtlayer_check.so, also
+ * writes a record of the first failure into the next three words). NULL is
  * RT_ERR_INVALID_ARG. */
 int rt_project_qkv(const void* x_dev, const void* W_qkv_dev, int B, int N, int d,
                    int dtype, void* QKV_dev, void* scratch_dev, void* err_dev,
