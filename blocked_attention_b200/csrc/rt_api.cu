@@ -357,7 +357,7 @@ struct Plan {
   Shape s;
   size_t esz;
   size_t off_err, off_qkv, off_m, off_l, off_o, off_inv, off_xr, off_wqkv, off_a, off_u32, off_u16, off_ru,
-      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, off_flags, off_w2cnt, off_w2part, total;
+      off_h, off_zs, off_rz, off_ssq_u, off_ssq_z, off_flags, off_w2cnt, off_w2part, off_progress, total;
   TileCfg t_wo, t_w1, t_w2, t_wkv;
   StepsPlan sp;
 };
@@ -399,6 +399,7 @@ static Plan make_plan(const Shape& s) {
     P.off_flags = take((size_t)PH_COUNT * P.sp.nrb * kFlagStride * 4);
     P.off_w2cnt = take((size_t)P.sp.nrb * g2.tiles * 4);
     P.off_w2part = take((size_t)P.sp.nrb * g2.tiles * g2.S * g2.BN * StepsCfg::BM * 4);
+    P.off_progress = take((size_t)1024 * 4 * 4);   // the debug build's per-CTA progress record
   }
   if (s.dtype == RT_BF16) {
     const int M = s.step_rows();
@@ -709,6 +710,7 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
     sp.w2cnt = reinterpret_cast<unsigned*>(ws + P.off_w2cnt);
     sp.w2part = reinterpret_cast<float*>(ws + P.off_w2part);
     sp.err = err;
+    sp.progress = reinterpret_cast<unsigned*>(ws + P.off_progress);
     sp.sc2 = sc2;
     sp.H = H;
     sp.nrb = P.sp.nrb;

@@ -97,6 +97,7 @@ struct StepsParams {
   unsigned* w2cnt;             // [nrb][tiles of W2]: split arrivals, cumulative over the forward
   float* w2part;               // [nrb][tiles][S][BN_2][128] fp32 partial tiles
   unsigned* err;
+  unsigned* progress;          // (debug build) [gridDim][4]: the task each role of each CTA is at
   float sc2;                   // log2(e) / sqrt(d_h)
   int H, nrb, G;               // heads, row blocks, fold groups of 32 sequences per row block
   int j0, j1;                  // the segment's steps
@@ -173,6 +174,27 @@ __device__ __forceinline__ bool mbar_wait_g(uint64_t* bar, unsigned parity, unsi
 // where a wait is: CTA, step, phase and the task's index in its phase
 __device__ __forceinline__ long long wait_site(int ph, int j, int loc) {
   return ((long long)blockIdx.x << 24) | ((long long)(j & 0xfff) << 12) | ((ph & 7) << 9) | (loc & 0x1ff);
+}
+
+// (debug build) after an error the flags stay as they were, so that the
+// record shows the dependency state at the first failure
+__device__ __forceinline__ bool release_allowed(const StepsParams& P) {
+#ifdef RT_BOUNDS_CHECK
+  return ld_volatile_u32(P.err) == 0;
+#else
+  return true;
+#endif
+}
+
+// (debug build) role r of this CTA is at task (ph, j, loc): producer 0, MMA
+// issuers 1 and 2, epilogue 3
+__device__ __forceinline__ void note_progress(const StepsParams& P, int role, int ph, int j, int loc) {
+#ifdef RT_BOUNDS_CHECK
+  // frozen once the error word is set: the record shows where each role was
+  if (P.progress && ld_volatile_u32(P.err) == 0)
+    *reinterpret_cast<volatile unsigned*>(P.progress + blockIdx.x * 4 + role) =
+        ((unsigned)(j & 0xfff) << 12) | ((ph & 7) << 9) | (loc & 0x1ff) | 0x80000000u;
+#endif
 }
 
 // ---------------------------------------------------------------------------
@@ -472,6 +494,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
     bool ok = true;
     for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
       if (ph == PH_FOLD) return true;
+      if (lane == 0) note_progress(P, 0, ph, j, loc);
       const GemmPhase& g = P.g[ph];
       const GemmTask T = decode_gemm(g, loc);
       const bool deps = !(ph == PH_WO && j == P.j0);   // a of the first step comes from an earlier kernel
@@ -532,6 +555,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       uint32_t it = 0, local = 0;
       for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
         if (ph == PH_FOLD) return true;
+        note_progress(P, 1 + par, ph, j, loc);
         const GemmPhase& g = P.g[ph];
         const GemmTask T = decode_gemm(g, loc);
         const int nst = (T.sl1 - T.sl0 + C::KSUB - 1) / C::KSUB;
@@ -575,6 +599,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
     const int lrow = q * 32 + lane;
     uint32_t local = 0;
     for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
+      if (tid == 0) note_progress(P, 3, ph, j, loc);
       if (ph == PH_FOLD) {
         const int per_rb = P.H * P.G;
         const int rb = loc / per_rb, r = loc - rb * per_rb;
@@ -599,7 +624,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         fence_proxy_async_global();   // a is read by the next step's TMA loads
         __threadfence();
         epi_bar();
-        if (tid == 0) st_release_u32(flag_ptr(P, PH_FOLD, rb, h * P.G + gi), (unsigned)(j + 1));
+        if (tid == 0 && release_allowed(P)) st_release_u32(flag_ptr(P, PH_FOLD, rb, h * P.G + gi), (unsigned)(j + 1));
         return true;
       }
       const GemmPhase& g = P.g[ph];
@@ -713,7 +738,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         fence_proxy_async_global();   // the next phase reads these outputs with TMA
         __threadfence();
         epi_bar();
-        if (tid == 0) st_release_u32(flag_ptr(P, ph, T.rb, T.tile), (unsigned)(j + 1));
+        if (tid == 0 && release_allowed(P)) st_release_u32(flag_ptr(P, ph, T.rb, T.tile), (unsigned)(j + 1));
       }
       return true;
     });
