@@ -187,13 +187,23 @@ __device__ __forceinline__ bool release_allowed(const StepsParams& P) {
 }
 
 // (debug build) role r of this CTA is at task (ph, j, loc): producer 0, MMA
-// issuers 1 and 2, epilogue 3
+// issuers 1 and 2, epilogue 3 (word 2r), and in which wait (word 2r + 1:
+// kind in bits 28..30 -- 1 ring slot free, 2 dependency flag, 3 accumulator
+// free, 4 stage loaded, 5 accumulator full, 6 epilogue flag, 7 fold flag --
+// then the ring stage counter or task counter in bits 0..27)
 __device__ __forceinline__ void note_progress(const StepsParams& P, int role, int ph, int j, int loc) {
 #ifdef RT_BOUNDS_CHECK
   // frozen once the error word is set: the record shows where each role was
   if (P.progress && ld_volatile_u32(P.err) == 0)
-    *reinterpret_cast<volatile unsigned*>(P.progress + blockIdx.x * 4 + role) =
+    *reinterpret_cast<volatile unsigned*>(P.progress + blockIdx.x * 8 + 2 * role) =
         ((unsigned)(j & 0xfff) << 12) | ((ph & 7) << 9) | (loc & 0x1ff) | 0x80000000u;
+#endif
+}
+__device__ __forceinline__ void note_wait(const StepsParams& P, int role, unsigned kind, unsigned counter) {
+#ifdef RT_BOUNDS_CHECK
+  if (P.progress && ld_volatile_u32(P.err) == 0)
+    *reinterpret_cast<volatile unsigned*>(P.progress + blockIdx.x * 8 + 2 * role + 1) =
+        (kind << 28) | (counter & 0x0fffffffu) | 0x80000000u;
 #endif
 }
 
@@ -512,6 +522,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         const int ns = min(C::KSUB, T.sl1 - kb);
         const uint32_t s = it % C::STAGES, par = (it / C::STAGES) & 1u;
         int w = 1;
+        if (lane == 0) note_wait(P, 0, 1, it);
         if (lane == 0) w = mbar_wait_g(&empty[s], par ^ 1u, P.err, 41, wait_site(ph, j, loc)) ? 1 : 0;
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) { ok = false; return false; }
@@ -526,6 +537,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
           int lo, hi, t2;
           slice_flags(P, ph, kb, lo, t2);
           slice_flags(P, ph, kb + ns - 1, t2, hi);
+          if (lane == 0) note_wait(P, 0, 2, it);
           for (int i = 0; i < 3; ++i) {
             const int f = flo + lane + 32 * i;
             if (f >= lo && f < hi && f < fhi && !(rdy >> i & 1u)) {
@@ -561,6 +573,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         const int nst = (T.sl1 - T.sl0 + C::KSUB - 1) / C::KSUB;
         const uint32_t acc = local & 1u, aph = (local >> 1) & 1u;
         ++local;
+        note_wait(P, 1 + par, 3, local - 1);
         if (!mbar_wait_g(&tempty[acc], aph ^ 1u, P.err, 43, wait_site(ph, j, loc))) return false;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (acc * 2 + par) * C::BN_MAX;
@@ -570,6 +583,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         for (int kb = 0; kb < nst; ++kb, ++it) {
           if ((kb & 1) != par) continue;
           const uint32_t s = it % C::STAGES, sp = (it / C::STAGES) & 1u;
+          note_wait(P, 1 + par, 4, it);
           if (!mbar_wait_g(&full[s], sp, P.err, 44, wait_site(ph, j, loc))) return false;
           tc_fence_after();
           const uint8_t* a_st = sA + s * C::A_BYTES;
@@ -663,6 +677,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       // A wait that gives up (error word set) does not end the task: the four
       // epilogue warps must reach every named barrier together, so they run
       // on with whatever tensor memory holds.
+      if (tid == 0) note_wait(P, 3, 5, local - 1);
       if (lane == 0) mbar_wait_g(&tfull[acc], aph, P.err, 45, wait_site(ph, j, loc));
       __syncwarp();
       tc_fence_after();
