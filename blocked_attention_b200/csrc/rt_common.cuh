@@ -165,6 +165,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsign
   }
 }
 
+// Rings consumed by two issuers that take alternate stages: the previous
+// round of a slot may belong to the other issuer, and if that round's copy
+// has not landed yet when this issuer reaches the slot, a parity wait for
+// the slot's next round reads the pending phase as "the one before" and
+// passes with the wrong data. So each issuer records, per slot, the last
+// round whose data it saw land (seen[s] = round + 1), and before waiting on a
+// slot's barrier for round r an issuer waits (bounded) for seen[s] >= r. The
+// barrier is then exactly one phase from round r, which the parity tells
+// apart.
+// (debug build: a wait that runs out records `id` and `where`)
+__device__ __forceinline__ bool ring_round_wait(const volatile uint32_t* seen, uint32_t round, unsigned* err,
+                                                unsigned id = 0, long long where = 0,
+                                                unsigned long long limit_ns = kWaitLimitNs) {
+  if (*seen >= round) return true;
+  const unsigned long long t0 = globaltimer();
+  for (unsigned it = 0;; ++it) {
+    if (*seen >= round) return true;
+    if ((it & 255u) == 255u) {
+      if (*reinterpret_cast<volatile unsigned*>(err) != 0) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        set_error(err, RT_DEVERR_TIMEOUT);
+        if (id) timeout_record(err, id, where, round);
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tiled, no multicast)
 // ---------------------------------------------------------------------------

@@ -346,6 +346,7 @@ __global__ void __launch_bounds__(224, 1)
   uint64_t* tempty = tfull + 2;       // [2]
   uint64_t* rbar = tempty + 2;        // split-K: the other ranks' row blocks have landed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rbar + 1);
+  volatile uint32_t* seen = tmem_holder + 1;   // [STAGES]: see ring_round_wait
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntn = (N + BN - 1) / BN, ntm = (M + C::BM - 1) / C::BM;
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(224, 1)
   const int ksl = K / C::BK;   // 64-wide K slices in all
   auto slices = [&](int kblock) { const int r = ksl - kblock * KSUB; return r < KSUB ? r : KSUB; };
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); seen[s] = 0; }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], NACC); mbar_init(&tempty[a], 4); }
     mbar_init(rbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -442,7 +443,9 @@ __global__ void __launch_bounds__(224, 1)
         for (int kb = 0; kb < nk; ++kb, ++it) {
           if ((kb % NACC) != par) continue;
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          if (NACC > 1 && !ring_round_wait(&seen[s], it / STAGES, err)) { ok = false; break; }
           if (!mbar_wait(&full[s], ph, err)) { ok = false; break; }
+          if (NACC > 1) seen[s] = it / STAGES + 1;
           tc_fence_after();
           const uint8_t* a_st = sA + s * C::A_BYTES;
           const uint8_t* b_st = sB + s * C::B_BYTES;

@@ -189,7 +189,7 @@ __device__ __forceinline__ bool release_allowed(const StepsParams& P) {
 // (debug build) role r of this CTA is at task (ph, j, loc): producer 0, MMA
 // issuers 1 and 2, epilogue 3 (word 2r), and in which wait (word 2r + 1:
 // kind in bits 28..30 -- 1 ring slot free, 2 dependency flag, 3 accumulator
-// free, 4 stage loaded, 5 accumulator full, 6 epilogue flag, 7 fold flag --
+// free, 4 stage loaded, 5 accumulator full, 6 slot's previous round seen --
 // then the ring stage counter or task counter in bits 0..27)
 __device__ __forceinline__ void note_progress(const StepsParams& P, int role, int ph, int j, int loc) {
 #ifdef RT_BOUNDS_CHECK
@@ -483,10 +483,11 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
   uint64_t* drain = tempty + 2;          // [2]: an issuer's MMAs have all completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile uint32_t* seen = tmem_holder + 2;   // [STAGES]: see ring_round_wait
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); seen[s] = 0; }
     for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 2); mbar_init(&tempty[a], 4); mbar_init(&drain[a], 1); }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -583,8 +584,11 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         for (int kb = 0; kb < nst; ++kb, ++it) {
           if ((kb & 1) != par) continue;
           const uint32_t s = it % C::STAGES, sp = (it / C::STAGES) & 1u;
+          note_wait(P, 1 + par, 6, it);
+          if (!ring_round_wait(&seen[s], it / C::STAGES, P.err, 48, wait_site(ph, j, loc))) return false;
           note_wait(P, 1 + par, 4, it);
           if (!mbar_wait_g(&full[s], sp, P.err, 44, wait_site(ph, j, loc))) return false;
+          seen[s] = it / C::STAGES + 1;
           tc_fence_after();
           const uint8_t* a_st = sA + s * C::A_BYTES;
           const uint8_t* b_st = sB + s * C::B_BYTES;

@@ -1,7 +1,10 @@
 """Shared helpers of the parity tests: seeded problems (from rtinputs) on both
 sides, oracle runs on sampled sequences, and the error metric.
 
-Error metric (per output tensor): max |gpu - ref| / max |ref|.
+Error metric (per output tensor): max |gpu - ref| / max |ref|; where the
+reference is identically zero (for example the gradients of W_q and W_k of a
+one-token sequence, whose single softmax weight is constant) the metric is
+the absolute max |gpu|.
 Bars: 1e-4 for the fp32 storage mode, 2e-2 for bf16 storage with fp32
 accumulation."""
 from __future__ import annotations
@@ -16,7 +19,9 @@ TOL = {"f32": 1e-4, "bf16": 2e-2}
 def rel_err(got, ref) -> float:
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
-    return float(np.max(np.abs(got - ref)) / np.max(np.abs(ref)))
+    scale = float(np.max(np.abs(ref))) if ref.size else 0.0
+    diff = float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    return diff / scale if scale > 0.0 else diff
 
 
 def torch_dtype(dtype: str):
