@@ -86,7 +86,30 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // same grid plainly -- one CTA per SM fits (shared memory allows no second)
 // and the previous kernel of the stream has finished, so the CTAs are
 // resident together in practice, and every wait is bounded regardless.
-static cudaError_t launch_steps(const StepsParams& sp, int sms, cudaStream_t st, bool coop) {
+#ifdef RT_TRACE
+// (trace build) the segment starting at step g_trace_j0 records its task
+// events into g_trace (kTraceSlots times per task), if it has room for them
+static unsigned long long* g_trace = nullptr;
+static size_t g_trace_bytes = 0;
+static int g_trace_j0 = -1;
+extern "C" void rt_debug_trace_segment(void* buf, size_t bytes, int j0) {
+  g_trace = static_cast<unsigned long long*>(buf);
+  g_trace_bytes = bytes;
+  g_trace_j0 = j0;
+}
+#endif
+static cudaError_t launch_steps(const StepsParams& sp_in, int sms, cudaStream_t st, bool coop) {
+  StepsParams sp = sp_in;
+#ifdef RT_TRACE
+  if (g_trace && sp.j0 == g_trace_j0) {
+    size_t tasks = 0;
+    for (int j = sp.j0; j < sp.j1; ++j) {
+      for (int ph = 0; ph < 4; ++ph) tasks += (size_t)sp.nrb * sp.g[ph].tiles * sp.g[ph].S;
+      if (j + 1 < sp.j1) tasks += (size_t)sp.nrb * sp.H * sp.G;
+    }
+    if (tasks * kTraceSlots * 8 <= g_trace_bytes) sp.trace = g_trace;
+  }
+#endif
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)sms);
   cfg.blockDim = dim3(StepsCfg::THREADS);
@@ -341,15 +364,16 @@ static StepsPlan plan_steps(const Shape& s) {
   // 4096-deep W_2 reduction split so that every task streams about 1024 of K.
   sp.g[PH_WO] = phase(d, d, 64, 1);
   sp.g[PH_W1] = phase(dff, d, dff % 128 == 0 ? 128 : 64, 1);
-  const int s2 = std::max(1, std::min(4, (dff / 64) / 8));
-  sp.g[PH_W2] = phase(d, dff, d % 128 == 0 ? 128 : 64, s2);
+  const int bn2 = d % 128 == 0 ? 128 : 64;
+  // every split finishes BN_2 / S >= 32 of its tile's columns
+  const int s2 = std::max(1, std::min(std::min(4, bn2 / 32), (dff / 64) / 8));
+  sp.g[PH_W2] = phase(d, dff, bn2, s2);
   sp.g[PH_WKV] = phase(2 * d, d, 128, 1);
   sp.nrb = (s.B + 127) / 128;
   sp.G = (std::min(s.B, 128) + kFoldSeqs - 1) / kFoldSeqs;
-  // flag ranges one producer lane set polls (3 per lane) and the flag stride
-  const int w2_split_tiles = (dff / s2 + sp.g[PH_W1].BN - 1) / sp.g[PH_W1].BN + 1;
-  sp.ok = s.H * sp.G <= 96 && sp.g[PH_WO].tiles <= 96 && w2_split_tiles <= 96 && sp.g[PH_W2].tiles <= 96 &&
-          sp.g[PH_W1].tiles <= kFlagStride && sp.g[PH_WKV].tiles <= kFlagStride && s.H * sp.G <= kFlagStride;
+  // the flags of a phase fit its flag stride
+  sp.ok = s.H * sp.G <= kFlagStride && sp.g[PH_WO].tiles <= kFlagStride && sp.g[PH_W1].tiles <= kFlagStride &&
+          sp.g[PH_W2].tiles * s2 <= kFlagStride && sp.g[PH_WKV].tiles <= kFlagStride;
   return sp;
 }
 

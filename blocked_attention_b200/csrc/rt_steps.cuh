@@ -29,20 +29,23 @@
 // Tasks are numbered in the order (step, phase, row block, tile, split) and
 // dealt round-robin to the grid's CTAs (one per SM, co-resident: cooperative
 // launch); each CTA processes its tasks in that order. Every task waits only
-// for tasks earlier in the order, so the earliest unfinished task can always
-// run: no deadlock.
+// for tasks earlier in the order, except that the S splits of a W_2 tile wait
+// for one another's partial tiles; those are S consecutive tasks of one phase
+// on S different CTAs, each reached after earlier tasks only, so the earliest
+// unfinished task can always run: no deadlock.
 //
-// Dependencies are per-tile flags in global memory holding "last step done +
-// 1" (monotonic within a forward; cleared before it). A task's TMA producer
-// polls the flags of the tiles its A operand is made of, K slice by K slice,
-// so a GEMM starts on the first columns of its input while the producing
-// phase is still finishing them. Every thread that reads data another CTA
+// Dependencies are flags in global memory holding "last step done + 1"
+// (monotonic within a forward; cleared before it), one per output tile, or per
+// 1 / S of a W_2 tile. A task's TMA producer loads the weight operand of its
+// first pipeline stages, then polls every flag its A operand depends on (the
+// warp's lanes in parallel) and streams A. Every thread that reads data another CTA
 // wrote first observes (acquire) the flag that covers it, then fences, and
 // reads that data through L2 (ld.global.cg or TMA), never from a possibly
 // stale L1 line; every writer fences its stores (also to the async proxy,
-// since the next phase reads them with TMA) before it releases its flag. The W_2 split-K partial
-// tiles go to global slots; an arrival counter elects the last split, which
-// sums the slots in split order (deterministic) and runs the epilogue.
+// since the next phase reads them with TMA) before it releases its flag. The
+// W_2 split-K partial tiles go to global slots; once all S have arrived, every
+// split sums its 1 / S of the columns over the S slots in split order
+// (deterministic) and runs the epilogue on them.
 //
 // Every poll and every mbarrier wait is bounded by %globaltimer. A poll that
 // runs out records RT_DEVERR_TIMEOUT and returns; once the error word is set,
@@ -58,7 +61,18 @@
 
 namespace rt {
 
-enum StepPhase { PH_WO = 0, PH_W1 = 1, PH_W2 = 2, PH_WKV = 3, PH_FOLD = 4, PH_COUNT = 5 };
+enum StepPhase { PH_WO = 0, PH_W1 = 1, PH_W2 = 2, PH_WKV = 3, PH_FOLD = 4, PH_DEFER = 5, PH_COUNT = 6 };
+// the order of the phases inside a step
+__device__ __forceinline__ int phase_at(int i) {
+  switch (i) {
+    case 0: return PH_WO;
+    case 1: return PH_W1;
+    case 2: return PH_DEFER;
+    case 3: return PH_W2;
+    case 4: return PH_WKV;
+    default: return PH_FOLD;
+  }
+}
 
 constexpr int kFlagStride = 256;   // flags per (phase, row block): tiles, or heads x fold groups
 constexpr int kFoldSeqs = 32;      // sequences per fold task
@@ -97,7 +111,8 @@ struct StepsParams {
   unsigned* w2cnt;             // [nrb][tiles of W2]: split arrivals, cumulative over the forward
   float* w2part;               // [nrb][tiles][S][BN_2][128] fp32 partial tiles
   unsigned* err;
-  unsigned* progress;          // (debug build) [gridDim][4]: the task each role of each CTA is at
+  unsigned* progress;          // (debug build) [gridDim][8]: the task and the wait each role of each CTA is at
+  unsigned long long* trace;   // (trace build) [tasks of the segment][16] event times, or null
   float sc2;                   // log2(e) / sqrt(d_h)
   int H, nrb, G;               // heads, row blocks, fold groups of 32 sequences per row block
   int j0, j1;                  // the segment's steps
@@ -207,27 +222,49 @@ __device__ __forceinline__ void note_wait(const StepsParams& P, int role, unsign
 #endif
 }
 
+// (trace build) event ev of the segment's task gi happened now (%globaltimer
+// ns): 0 producer starts the task, 1 producer issued its last A load (every
+// dependency seen), 2 / 3 issuer 0 / 1 has its accumulator, 4 / 5 issuer 0 /
+// 1 issued its last MMA, 6 epilogue starts, 7 epilogue dependencies seen, 8
+// accumulator full, 9 flag released (a fold: 6, 7 and 9); per pipeline stage
+// k < 16: 16 + k producer has the slot, 48 + k an issuer saw the stage
+// loaded; 32 producer saw every dependency; epilogue sub-steps: 10 outputs
+// stored, 11 fences done
+constexpr int kTraceSlots = 64;
+__device__ __forceinline__ void trace_ev(const StepsParams& P, int gi, int ev) {
+#ifdef RT_TRACE
+  if (P.trace && ev < kTraceSlots) P.trace[(size_t)gi * kTraceSlots + ev] = globaltimer();
+#endif
+}
+
 // ---------------------------------------------------------------------------
 // task enumeration (identical in every warp role of a CTA)
 // ---------------------------------------------------------------------------
+// Queries of the block folded at step j - 1 (t = j) after its first one: the
+// deferred part of that fold, run at step j (0 when the block has one query).
+__device__ __forceinline__ int deferred_queries(const StepsParams& P, int j) {
+  return min(lowbit(j), P.ep.Nseq - j) - 1;
+}
 __device__ __forceinline__ int phase_tasks(const StepsParams& P, int ph, int j) {
   if (ph < 4) return P.nrb * P.g[ph].tiles * P.g[ph].S;
-  return (j + 1 < P.j1) ? P.nrb * P.H * P.G : 0;   // the segment's last fold runs elsewhere
+  if (ph == PH_FOLD) return (j + 1 < P.j1) ? P.nrb * P.H * P.G : 0;   // the segment's last fold runs elsewhere
+  return (j > P.j0 && deferred_queries(P, j) > 0) ? P.nrb * P.H * P.G : 0;
 }
 
-// Calls f(phase, step, local index) for this CTA's tasks in order; stops when
-// f returns false.
+// Calls f(phase, step, local index, index in the segment) for this CTA's
+// tasks in order; stops when f returns false.
 template <class F>
 __device__ __forceinline__ void for_my_tasks(const StepsParams& P, F&& f) {
   const long G = gridDim.x, bid = blockIdx.x;
   long base = 0;
   for (int j = P.j0; j < P.j1; ++j) {
-    for (int ph = 0; ph < PH_COUNT; ++ph) {
+    for (int oi = 0; oi < PH_COUNT; ++oi) {
+      const int ph = phase_at(oi);
       const int n = phase_tasks(P, ph, j);
       long first = (bid - base) % G;
       if (first < 0) first += G;
       for (long loc = first; loc < n; loc += G)
-        if (!f(ph, j, (int)loc)) return;
+        if (!f(ph, j, (int)loc, (int)(base + loc))) return;
       base += n;
     }
   }
@@ -259,13 +296,18 @@ __device__ __forceinline__ unsigned* flag_ptr(const StepsParams& P, int ph, int 
 // is made by flags [lo(kk), hi(kk)) of phase dep_phase(ph), complete once
 // they reach dep_target.
 __device__ __forceinline__ int dep_phase(int ph) { return ph == PH_WO ? PH_FOLD : ph - 1; }
+// Columns one flag of a GEMM phase covers: a tile, or with a split
+// reduction one tile / S (every split finishes that share of its tile).
+__device__ __forceinline__ int flag_cols(const GemmPhase& g) { return g.BN / g.S; }
+__device__ __forceinline__ int phase_flags(const GemmPhase& g) { return g.tiles * g.S; }
 __device__ __forceinline__ void slice_flags(const StepsParams& P, int ph, int kk, int& lo, int& hi) {
   if (ph == PH_WO) {   // a of head kk (d_h = 64): the fold groups of head kk
     lo = kk * P.G;
     hi = lo + P.G;
-  } else {
-    lo = kk * 64 / P.g[ph - 1].BN;
-    hi = lo + 1;
+  } else {             // columns [64 kk, 64 kk + 64) of the previous phase's output
+    const int fc = flag_cols(P.g[ph - 1]);
+    lo = (64 * kk) / fc;
+    hi = (64 * kk + 63) / fc + 1;
   }
 }
 
@@ -273,14 +315,14 @@ __device__ __forceinline__ void slice_flags(const StepsParams& P, int ph, int kk
 // small block fold (at most 8 keys), one task = one head of up to 32
 // sequences: every (sequence, query) unit is served by an octet of lanes
 // holding 8 of the head's 64 dims; each thread takes R units at a time and
-// issues all their loads before any use. The first query of the block is
+// issues all their loads before any use. With fin, the first query q0 is
 // finalised (temporary pair merged, a = o / l written, statistics not
-// stored); the others' (m, l, o) are updated in place, or written when the
-// fold is the first into them (init).
+// stored); the other queries' (m, l, o) are updated in place, or written when
+// the fold is the first into them (init).
 // ---------------------------------------------------------------------------
 template <int NK, int R>
 __device__ __forceinline__ void fold_small_units(const StepsParams& P, int q0, int nq, int k0, int init, int h,
-                                                 int s0, int ns, int tid) {
+                                                 int s0, int ns, int tid, int fin) {
   const int B = P.ep.B, H = P.H, d = P.ep.d;
   const int oct = tid >> 3, sl = tid & 7;
   const unsigned omask = 0xFFu << ((tid & 31) & 24);
@@ -319,7 +361,7 @@ __device__ __forceinline__ void fold_small_units(const StepsParams& P, int q0, i
           kw[r][i] = __ldcg(reinterpret_cast<const uint4*>(K + kv));
           vw[r][i] = __ldcg(reinterpret_cast<const uint4*>(V + kv));
         }
-        if (qi == 0) {   // the finalised query's temporary pair
+        if (fin && qi == 0) {   // the finalised query's temporary pair
           ktw[r] = *reinterpret_cast<const uint4*>(qp + d);
           vtw[r] = *reinterpret_cast<const uint4*>(qp + 2 * d);
         }
@@ -371,7 +413,7 @@ __device__ __forceinline__ void fold_small_units(const StepsParams& P, int q0, i
 #pragma unroll
         for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
       }
-      if (qi == 0) {
+      if (fin && qi == 0) {
         float kt[8];
         unpack_bf16x8(ktw[r], kt);
         float dot = 0.f;
@@ -482,7 +524,6 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
   uint64_t* tempty = tfull + 2;          // [2]
   uint64_t* drain = tempty + 2;          // [2]: an issuer's MMAs have all completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
-  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile uint32_t* seen = tmem_holder + 2;   // [STAGES]: see ring_round_wait
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -503,9 +544,10 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
     // ---------------- TMA producer (lane 0 issues; the warp polls flags) ----------------
     uint32_t it = 0;
     bool ok = true;
-    for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
-      if (ph == PH_FOLD) return true;
+    for_my_tasks(P, [&](int ph, int j, int loc, int gi) -> bool {
+      if (ph >= PH_FOLD) return true;
       if (lane == 0) note_progress(P, 0, ph, j, loc);
+      if (lane == 0) trace_ev(P, gi, 0);
       const GemmPhase& g = P.g[ph];
       const GemmTask T = decode_gemm(g, loc);
       const bool deps = !(ph == PH_WO && j == P.j0);   // a of the first step comes from an earlier kernel
@@ -516,44 +558,68 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         slice_flags(P, ph, T.sl0, flo, tmp);
         slice_flags(P, ph, T.sl1 - 1, tmp, fhi);
       }
-      // flags flo + lane + 32 i, i < 3: readiness bits of this lane
-      unsigned rdy = 0;
+      // The weight (B) halves of the first ring stages are loaded before the
+      // dependencies are seen (weights are never written here); then the
+      // lanes poll every flag the task's A operand depends on at once, one
+      // fence orders those writes before the async-proxy loads, and the A
+      // halves follow.
       const uint32_t bn_bytes = (uint32_t)g.BN * C::BK * 2;
-      for (int kb = T.sl0; kb < T.sl1; kb += C::KSUB, ++it) {
-        const int ns = min(C::KSUB, T.sl1 - kb);
-        const uint32_t s = it % C::STAGES, par = (it / C::STAGES) & 1u;
+      const int nst = (T.sl1 - T.sl0 + C::KSUB - 1) / C::KSUB;
+      const int pre = deps ? min(nst, C::STAGES) : 0;
+      auto take_slot = [&](int k) -> bool {   // wait for stage k's slot, then arm it and load its B half
+        const uint32_t ik = it + k, s = ik % C::STAGES, par = (ik / C::STAGES) & 1u;
+        const int kb = T.sl0 + k * C::KSUB, ns = min(C::KSUB, T.sl1 - kb);
         int w = 1;
-        if (lane == 0) note_wait(P, 0, 1, it);
+        if (lane == 0) note_wait(P, 0, 1, ik);
         if (lane == 0) w = mbar_wait_g(&empty[s], par ^ 1u, P.err, 41, wait_site(ph, j, loc)) ? 1 : 0;
         w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) { ok = false; return false; }
+        if (!w) return false;
         if (lane == 0) {
+          trace_ev(P, gi, 16 + min(k, 15));
           mbar_arrive_expect_tx(&full[s], ns * (C::A_SUB + bn_bytes));
           for (int q = 0; q < ns; ++q)
             if (idx_ok((kb + q + 1) * C::BK <= g.K && (T.tile + 1) * g.BN <= g.N && s < (uint32_t)C::STAGES &&
                            g.BN <= C::BN_MAX, P.err, 11, kb + q, T.tile))
               tma_load_2d(&P.tB[ph], &full[s], sB + s * C::B_BYTES + q * C::B_SUB, (kb + q) * C::BK, T.tile * g.BN);
         }
-        if (deps) {
-          int lo, hi, t2;
-          slice_flags(P, ph, kb, lo, t2);
-          slice_flags(P, ph, kb + ns - 1, t2, hi);
-          if (lane == 0) note_wait(P, 0, 2, it);
-          for (int i = 0; i < 3; ++i) {
-            const int f = flo + lane + 32 * i;
-            if (f >= lo && f < hi && f < fhi && !(rdy >> i & 1u)) {
-              poll_ge(flag_ptr(P, dph, T.rb, f), target, P.err, 42, wait_site(ph, j, f));
-              rdy |= 1u << i;
-            }
-          }
-          __syncwarp();
-          if (lane == 0) fence_proxy_async_global();
-        }
+        return true;
+      };
+      auto load_a = [&](int k) {
+        const uint32_t ik = it + k, s = ik % C::STAGES;
+        const int kb = T.sl0 + k * C::KSUB, ns = min(C::KSUB, T.sl1 - kb);
         if (lane == 0)
           for (int q = 0; q < ns; ++q)
             if (idx_ok((kb + q + 1) * C::BK <= g.K && T.rb * C::BM < P.ep.B, P.err, 12, kb + q, T.rb))
               tma_load_2d(&P.tA[ph], &full[s], sA + s * C::A_BYTES + q * C::A_SUB, (kb + q) * C::BK, T.rb * C::BM);
+      };
+      // (an abort leaves no armed stage without its A half, so that every
+      // copy in flight completes its barrier before the CTA exits)
+      for (int k = 0; k < pre; ++k)
+        if (!take_slot(k)) {
+          for (int q = 0; q < k; ++q) load_a(q);
+          it += k;
+          ok = false;
+          return false;
+        }
+      if (deps) {
+        if (lane == 0) note_wait(P, 0, 2, it);
+        for (int f = flo + lane; f < fhi; f += 32)
+          poll_ge(flag_ptr(P, dph, T.rb, f), target, P.err, 42, wait_site(ph, j, f));
+        __syncwarp();
+        if (lane == 0) fence_proxy_async_global();
+        if (lane == 0) trace_ev(P, gi, 32);
       }
+      for (int k = 0; k < pre; ++k) load_a(k);
+      for (int k = pre; k < nst; ++k) {
+        if (!take_slot(k)) {
+          it += k;
+          ok = false;
+          return false;
+        }
+        load_a(k);
+      }
+      it += nst;
+      if (lane == 0) trace_ev(P, gi, 1);
       return true;
     });
     if (!ok && lane == 0) {
@@ -566,8 +632,8 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
     const int par = warp - 1;
     if (lane == 0) {
       uint32_t it = 0, local = 0;
-      for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
-        if (ph == PH_FOLD) return true;
+      for_my_tasks(P, [&](int ph, int j, int loc, int gi) -> bool {
+        if (ph >= PH_FOLD) return true;
         note_progress(P, 1 + par, ph, j, loc);
         const GemmPhase& g = P.g[ph];
         const GemmTask T = decode_gemm(g, loc);
@@ -576,6 +642,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         ++local;
         note_wait(P, 1 + par, 3, local - 1);
         if (!mbar_wait_g(&tempty[acc], aph ^ 1u, P.err, 43, wait_site(ph, j, loc))) return false;
+        trace_ev(P, gi, 2 + par);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (acc * 2 + par) * C::BN_MAX;
         idx_ok((acc * 2 + par) * C::BN_MAX + g.BN <= C::TMEM_COLS && nst >= 1, P.err, 13, acc, nst);
@@ -589,6 +656,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
           note_wait(P, 1 + par, 4, it);
           if (!mbar_wait_g(&full[s], sp, P.err, 44, wait_site(ph, j, loc))) return false;
           seen[s] = it / C::STAGES + 1;
+          trace_ev(P, gi, 48 + min(kb, 15));
           tc_fence_after();
           const uint8_t* a_st = sA + s * C::A_BYTES;
           const uint8_t* b_st = sB + s * C::B_BYTES;
@@ -604,6 +672,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
           tc_commit(&empty[s]);
         }
         tc_commit(&tfull[acc]);   // with no stage of its own in this task it arrives at once
+        trace_ev(P, gi, 4 + par);
         return true;
       });
       // every MMA this thread issued has completed before the CTA frees TMEM
@@ -616,33 +685,55 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
     const int q = warp & 3;             // TMEM lanes 32q .. 32q + 31
     const int lrow = q * 32 + lane;
     uint32_t local = 0;
-    for_my_tasks(P, [&](int ph, int j, int loc) -> bool {
+    for_my_tasks(P, [&](int ph, int j, int loc, int gi) -> bool {
       if (tid == 0) note_progress(P, 3, ph, j, loc);
-      if (ph == PH_FOLD) {
+      if (tid == 0) trace_ev(P, gi, 6);
+      if (ph == PH_FOLD || ph == PH_DEFER) {
+        // FOLD (step j, t = j + 1): the block's keys into its first query t,
+        // which is finalised (a_t, read by the next step's W_o). DEFER (step
+        // j, t = j): the same block of the previous step into its other
+        // queries t + 1 .. t + nq - 1, off the critical path; the fold of
+        // step j (query t + 1 = j + 1) waits for it.
+        const bool urgent = ph == PH_FOLD;
         const int per_rb = P.H * P.G;
         const int rb = loc / per_rb, r = loc - rb * per_rb;
-        const int h = r / P.G, gi = r - h * P.G;
-        const int t = j + 1, lb = lowbit(t), nq = min(lb, P.ep.Nseq - t);
-        // this head's k and v of step j (and, through them, everything before)
+        const int h = r / P.G, gq = r - h * P.G;
+        const int t = urgent ? j + 1 : j, lb = lowbit(t), nq = min(lb, P.ep.Nseq - t);
+        const unsigned kv_ready = urgent ? (unsigned)(j + 1) : (unsigned)j;   // k, v of position t - 1
+        // this head's k and v of step t - 1 (and, through them, everything before)
         const int kt = (64 * h) / P.g[PH_WKV].BN, vt = (P.ep.d + 64 * h) / P.g[PH_WKV].BN;
-        if (tid == 0) { poll_ge(flag_ptr(P, PH_WKV, rb, kt), j + 1, P.err, 47, wait_site(ph, j, kt)); __threadfence(); }
-        if (tid == 32) { poll_ge(flag_ptr(P, PH_WKV, rb, vt), j + 1, P.err, 47, wait_site(ph, j, vt)); __threadfence(); }
+        if (tid == 0) { poll_ge(flag_ptr(P, PH_WKV, rb, kt), kv_ready, P.err, 47, wait_site(ph, j, kt)); __threadfence(); }
+        if (tid == 32) { poll_ge(flag_ptr(P, PH_WKV, rb, vt), kv_ready, P.err, 47, wait_site(ph, j, vt)); __threadfence(); }
+        if (urgent && tid == 64 && phase_tasks(P, PH_DEFER, j) > 0) {
+          poll_ge(flag_ptr(P, PH_DEFER, rb, r), (unsigned)(j + 1), P.err, 50, wait_site(ph, j, r));
+          __threadfence();
+        }
         epi_bar();
-        const int s0 = rb * 128 + gi * kFoldSeqs;
+        if (tid == 0) trace_ev(P, gi, 7);
+        const int s0 = rb * 128 + gq * kFoldSeqs;
         const int ns = min(kFoldSeqs, min(P.ep.B - s0, (rb + 1) * 128 - s0));
-        if (ns > 0 && nq > 0) {
-          const int init = t == lb ? 1 : 0;
+        const int init = t == lb ? 1 : 0;
+        if (ns > 0 && urgent && nq > 0) {
           switch (lb) {
-            case 1: fold_small_units<1, 4>(P, t, nq, t - 1, init, h, s0, ns, tid); break;
-            case 2: fold_small_units<2, 4>(P, t, nq, t - 2, init, h, s0, ns, tid); break;
-            case 4: fold_small_units<4, 3>(P, t, nq, t - 4, init, h, s0, ns, tid); break;
-            default: fold_small_units<8, 2>(P, t, nq, t - 8, init, h, s0, ns, tid); break;
+            case 1: fold_small_units<1, 2>(P, t, 1, t - 1, init, h, s0, ns, tid, 1); break;
+            case 2: fold_small_units<2, 2>(P, t, 1, t - 2, init, h, s0, ns, tid, 1); break;
+            case 4: fold_small_units<4, 2>(P, t, 1, t - 4, init, h, s0, ns, tid, 1); break;
+            default: fold_small_units<8, 2>(P, t, 1, t - 8, init, h, s0, ns, tid, 1); break;
+          }
+        } else if (ns > 0 && !urgent && nq > 1) {
+          switch (lb) {
+            case 2: fold_small_units<2, 4>(P, t + 1, nq - 1, t - 2, init, h, s0, ns, tid, 0); break;
+            case 4: fold_small_units<4, 3>(P, t + 1, nq - 1, t - 4, init, h, s0, ns, tid, 0); break;
+            default: fold_small_units<8, 2>(P, t + 1, nq - 1, t - 8, init, h, s0, ns, tid, 0); break;
           }
         }
+        if (tid == 0) trace_ev(P, gi, 10);
         fence_proxy_async_global();   // a is read by the next step's TMA loads
         __threadfence();
+        if (tid == 0) trace_ev(P, gi, 11);
         epi_bar();
-        if (tid == 0 && release_allowed(P)) st_release_u32(flag_ptr(P, PH_FOLD, rb, h * P.G + gi), (unsigned)(j + 1));
+        if (tid == 0 && release_allowed(P)) st_release_u32(flag_ptr(P, ph, rb, r), (unsigned)(j + 1));
+        if (tid == 0) trace_ev(P, gi, 9);
         return true;
       }
       const GemmPhase& g = P.g[ph];
@@ -664,9 +755,10 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         // last split polls these before it sums the partial tiles)
         if (g.S == 1) epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);
       } else {
-        epi_poll_range(P, PH_W2, T.rb, 0, P.g[PH_W2].tiles, (unsigned)(j + 1), tid);
+        epi_poll_range(P, PH_W2, T.rb, 0, phase_flags(P.g[PH_W2]), (unsigned)(j + 1), tid);
       }
       epi_bar();
+      if (tid == 0) trace_ev(P, gi, 7);
       EpiParams e = P.ep;
       e.j = j;
       float rs = 1.f;
@@ -674,7 +766,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         e.ssq_in = P.ssq_u; e.ssq_tiles = P.g[PH_WO].tiles;
         if (row_ok) rs = row_scale_for<EPI_W1>(e, row);
       } else if (ph == PH_WKV) {
-        e.ssq_in = P.ssq_z; e.ssq_tiles = P.g[PH_W2].tiles;
+        e.ssq_in = P.ssq_z; e.ssq_tiles = phase_flags(P.g[PH_W2]);
         if (row_ok) rs = row_scale_for<EPI_WKV>(e, row);
       }
       if (row_ok && ph == PH_WO) epilogue_prefetch<EPI_WO>(e, row, col_base, g.N, g.BN);
@@ -683,11 +775,12 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       // on with whatever tensor memory holds.
       if (tid == 0) note_wait(P, 3, 5, local - 1);
       if (lane == 0) mbar_wait_g(&tfull[acc], aph, P.err, 45, wait_site(ph, j, loc));
+      if (tid == 0) trace_ev(P, gi, 8);
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * 2 * C::BN_MAX;
       const bool two = nst >= 2;
-      bool done = true;   // this task finished its tile (else: a non-final split)
+      const int fu = T.tile * g.S + T.split;   // the flag (and Σ² unit) this task finishes
       if (g.S == 1) {
         float ssq = 0.f;
         switch (ph) {
@@ -698,15 +791,16 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         }
         if (row_ok && ph == PH_WO && idx_ok(T.tile <= P.ep.d / 32, P.err, 15, T.tile, 0))
           P.ssq_u[(size_t)T.tile * P.ep.B + row] = ssq;
-        if (row_ok && ph == PH_W2 && idx_ok(T.tile <= P.ep.d / 32, P.err, 15, T.tile, 1))
-          P.ssq_z[(size_t)T.tile * P.ep.B + row] = ssq;
+        if (row_ok && ph == PH_W2 && idx_ok(fu <= P.ep.d / 32, P.err, 15, fu, 1))
+          P.ssq_z[(size_t)fu * P.ep.B + row] = ssq;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
       } else {
         // split of W2: this split's partial tile to its slot ([col][row], so
         // that a warp's stores and loads are 128-byte lines)
-        const size_t slot_i = ((size_t)T.rb * g.tiles + T.tile) * g.S + T.split;
+        const size_t tile_i = (size_t)T.rb * g.tiles + T.tile;
+        const size_t slot_i = tile_i * g.S + T.split;
         idx_ok(slot_i < (size_t)P.nrb * g.tiles * g.S && T.split < g.S, P.err, 14, (long long)slot_i, T.split);
         float* slot = P.w2part + slot_i * (size_t)g.BN * C::BM;
 #pragma unroll 1
@@ -721,44 +815,45 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         if (lane == 0) mbar_arrive(&tempty[acc]);
         __threadfence();
         epi_bar();
+        // Every split of the tile has written its slot once the tile's
+        // arrival count reaches S (j + 1). The S splits run on S different
+        // CTAs at about the same time, and each then sums its 1 / S of the
+        // tile's columns over the S slots (in split order: deterministic)
+        // and runs the W2 epilogue on them. (The wait ends: a split's
+        // arrival needs only its own MMAs and earlier tasks of its CTA, and
+        // those never wait on this phase of this step.)
         if (tid == 0) {
-          unsigned* cnt = P.w2cnt + (size_t)T.rb * g.tiles + T.tile;
-          const unsigned old = atom_add_acq_rel(cnt, 1u);
-          *s_last = (old == (unsigned)(g.S * j + g.S - 1)) ? 1 : 0;
+          unsigned* cnt = P.w2cnt + tile_i;
+          atom_add_acq_rel(cnt, 1u);
+          poll_ge(cnt, (unsigned)(g.S * (j + 1)), P.err, 49, wait_site(ph, j, loc));
           __threadfence();
         }
+        epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);   // the residual u
         epi_bar();
-        done = *s_last != 0;
-        epi_bar();   // s_last is read by every thread before the next split task can rewrite it
-        if (done) {
-          // the last split: every split's partial is in its slot; sum them in
-          // split order and run the W2 epilogue
-          __threadfence();
-          epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);
-          epi_bar();
-          const float* slots = P.w2part + ((size_t)T.rb * g.tiles + T.tile) * g.S * (size_t)g.BN * C::BM;
-          float ssq = 0.f;
+        const int fc = flag_cols(g), c0 = T.split * fc;
+        const float* slots = P.w2part + tile_i * g.S * (size_t)g.BN * C::BM;
+        float ssq = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < g.BN; c += 32) {
-            float v[32];
+        for (int c = c0; c < c0 + fc; c += 32) {
+          float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
-            for (int sp = 0; sp < g.S; ++sp) {
-              const float* src = slots + (size_t)sp * g.BN * C::BM + (size_t)c * C::BM + lrow;
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          for (int sp = 0; sp < g.S; ++sp) {
+            const float* src = slots + (size_t)sp * g.BN * C::BM + (size_t)c * C::BM + lrow;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] += __ldcg(src + (size_t)i * C::BM);
-            }
-            if (row_ok) ssq += epilogue_chunk<EPI_W2>(e, row, col_base + c, g.N, v, 1.f, P.err);
+            for (int i = 0; i < 32; ++i) v[i] += __ldcg(src + (size_t)i * C::BM);
           }
-          if (row_ok) P.ssq_z[(size_t)T.tile * P.ep.B + row] = ssq;
+          if (row_ok) ssq += epilogue_chunk<EPI_W2>(e, row, col_base + c, g.N, v, 1.f, P.err);
         }
+        if (row_ok && idx_ok(fu <= P.ep.d / 32, P.err, 15, fu, 2)) P.ssq_z[(size_t)fu * P.ep.B + row] = ssq;
       }
-      if (done) {
-        fence_proxy_async_global();   // the next phase reads these outputs with TMA
-        __threadfence();
-        epi_bar();
-        if (tid == 0 && release_allowed(P)) st_release_u32(flag_ptr(P, ph, T.rb, T.tile), (unsigned)(j + 1));
-      }
+      if (tid == 0) trace_ev(P, gi, 10);
+      fence_proxy_async_global();   // the next phase reads these outputs with TMA
+      __threadfence();
+      if (tid == 0) trace_ev(P, gi, 11);
+      epi_bar();
+      if (tid == 0 && release_allowed(P)) st_release_u32(flag_ptr(P, ph, T.rb, fu), (unsigned)(j + 1));
+      if (tid == 0) trace_ev(P, gi, 9);
       return true;
     });
   }
