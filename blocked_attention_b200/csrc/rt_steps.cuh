@@ -229,7 +229,8 @@ __device__ __forceinline__ void note_wait(const StepsParams& P, int role, unsign
 // accumulator full, 9 flag released (a fold: 6, 7 and 9); per pipeline stage
 // k < 16: 16 + k producer has the slot, 48 + k an issuer saw the stage
 // loaded; 32 producer saw every dependency; epilogue sub-steps: 10 outputs
-// stored, 11 fences done
+// stored, 11 fences done, 40 + 2c / 41 + 2c chunk c (< 4) read from tensor
+// memory / written
 constexpr int kTraceSlots = 64;
 __device__ __forceinline__ void trace_ev(const StepsParams& P, int gi, int ev) {
 #ifdef RT_TRACE
@@ -472,8 +473,9 @@ __device__ __forceinline__ void tmem_ld_pair(uint32_t taddr, bool two, float (&v
 }
 
 template <int EPI>
-__device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool row_ok, int col_base, int BN, int N,
-                                               uint32_t taddr, bool two, float rs, unsigned* dbg_err) {
+__device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool row_ok, int col_base, int BN,
+                                               uint32_t taddr, bool two, float rs, unsigned* dbg_err,
+                                               const StepsParams& P, int gi) {
   float ssq = 0.f;
   if constexpr (EPI == EPI_WKV) {
     if (e.pages) {   // per-head unit RMS of k (the paper's parameterisation)
@@ -482,7 +484,7 @@ __device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool
         float va[32], vb[32];
         tmem_ld_pair(taddr + c, two, va);
         tmem_ld_pair(taddr + c + 32, two, vb);
-        if (row_ok) epilogue_head64<EPI_WKV>(e, row, col_base + c, N, va, vb, rs);
+        if (row_ok) epilogue_head64<EPI_WKV>(e, row, col_base + c, e.d * 2, va, vb, rs);
       }
       return 0.f;
     }
@@ -491,22 +493,21 @@ __device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool
   for (int c = 0; c < BN; c += 32) {
     float v[32];
     tmem_ld_pair(taddr + c, two, v);
-    if (row_ok) ssq += epilogue_chunk<EPI>(e, row, col_base + c, N, v, rs, dbg_err);
+    if (threadIdx.x == 96 && c < 128) trace_ev(P, gi, 40 + (c >> 4));
+    if (row_ok) ssq += epilogue_chunk<EPI>(e, row, col_base + c, EPI == EPI_W1 ? e.d_ff : (EPI == EPI_WKV ? 2 * e.d : e.d), v, rs, dbg_err);
+    if (threadIdx.x == 96 && c < 128) trace_ev(P, gi, 41 + (c >> 4));
   }
   return ssq;
 }
 
 // The epilogue-side dependencies of a task, polled in parallel by the 128
-// epilogue threads (thread i polls flag i of a contiguous range), then one
-// fence per polling thread and the epilogue barrier.
+// epilogue threads (thread i polls flag i of a contiguous range; the polls
+// are acquire loads), then the epilogue barrier, which orders every epilogue
+// thread's later loads after those acquires.
 __device__ __forceinline__ void epi_poll_range(const StepsParams& P, int ph, int rb, int lo, int hi, unsigned target,
                                                int tid, int task_ph = 7, int task_loc = 0) {
-  bool polled = false;
-  for (int i = lo + tid; i < hi; i += 128) {
+  for (int i = lo + tid; i < hi; i += 128)
     poll_ge(flag_ptr(P, ph, rb, i), target, P.err, 46, wait_site(task_ph, (int)target, (ph << 6) | (i & 63)));
-    polled = true;
-  }
-  if (polled) __threadfence();
 }
 
 // ---------------------------------------------------------------------------
@@ -702,12 +703,10 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         const unsigned kv_ready = urgent ? (unsigned)(j + 1) : (unsigned)j;   // k, v of position t - 1
         // this head's k and v of step t - 1 (and, through them, everything before)
         const int kt = (64 * h) / P.g[PH_WKV].BN, vt = (P.ep.d + 64 * h) / P.g[PH_WKV].BN;
-        if (tid == 0) { poll_ge(flag_ptr(P, PH_WKV, rb, kt), kv_ready, P.err, 47, wait_site(ph, j, kt)); __threadfence(); }
-        if (tid == 32) { poll_ge(flag_ptr(P, PH_WKV, rb, vt), kv_ready, P.err, 47, wait_site(ph, j, vt)); __threadfence(); }
-        if (urgent && tid == 64 && phase_tasks(P, PH_DEFER, j) > 0) {
+        if (tid == 0) poll_ge(flag_ptr(P, PH_WKV, rb, kt), kv_ready, P.err, 47, wait_site(ph, j, kt));
+        if (tid == 32) poll_ge(flag_ptr(P, PH_WKV, rb, vt), kv_ready, P.err, 47, wait_site(ph, j, vt));
+        if (urgent && tid == 64 && phase_tasks(P, PH_DEFER, j) > 0)
           poll_ge(flag_ptr(P, PH_DEFER, rb, r), (unsigned)(j + 1), P.err, 50, wait_site(ph, j, r));
-          __threadfence();
-        }
         epi_bar();
         if (tid == 0) trace_ev(P, gi, 7);
         const int s0 = rb * 128 + gq * kFoldSeqs;
@@ -728,11 +727,13 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
           }
         }
         if (tid == 0) trace_ev(P, gi, 10);
-        fence_proxy_async_global();   // a is read by the next step's TMA loads
-        __threadfence();
-        if (tid == 0) trace_ev(P, gi, 11);
         epi_bar();
-        if (tid == 0 && release_allowed(P)) st_release_u32(flag_ptr(P, ph, rb, r), (unsigned)(j + 1));
+        if (tid == 0) {
+          fence_proxy_async_global();   // a is read by the next step's TMA loads
+          __threadfence();
+          trace_ev(P, gi, 11);
+          if (release_allowed(P)) st_release_u32(flag_ptr(P, ph, rb, r), (unsigned)(j + 1));
+        }
         if (tid == 0) trace_ev(P, gi, 9);
         return true;
       }
@@ -784,10 +785,10 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       if (g.S == 1) {
         float ssq = 0.f;
         switch (ph) {
-          case PH_WO: ssq = epi_tile_tmem<EPI_WO>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs, P.err); break;
-          case PH_W1: epi_tile_tmem<EPI_W1>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs, P.err); break;
-          case PH_W2: ssq = epi_tile_tmem<EPI_W2>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs, P.err); break;
-          default: epi_tile_tmem<EPI_WKV>(e, row, row_ok, col_base, g.BN, g.N, taddr, two, rs, P.err); break;
+          case PH_WO: ssq = epi_tile_tmem<EPI_WO>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi); break;
+          case PH_W1: epi_tile_tmem<EPI_W1>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi); break;
+          case PH_W2: ssq = epi_tile_tmem<EPI_W2>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi); break;
+          default: epi_tile_tmem<EPI_WKV>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi); break;
         }
         if (row_ok && ph == PH_WO && idx_ok(T.tile <= P.ep.d / 32, P.err, 15, T.tile, 0))
           P.ssq_u[(size_t)T.tile * P.ep.B + row] = ssq;
@@ -813,7 +814,6 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
-        __threadfence();
         epi_bar();
         // Every split of the tile has written its slot once the tile's
         // arrival count reaches S (j + 1). The S splits run on S different
@@ -824,9 +824,9 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         // those never wait on this phase of this step.)
         if (tid == 0) {
           unsigned* cnt = P.w2cnt + tile_i;
+          __threadfence();   // the CTA's slot stores (ordered before by the barrier)
           atom_add_acq_rel(cnt, 1u);
           poll_ge(cnt, (unsigned)(g.S * (j + 1)), P.err, 49, wait_site(ph, j, loc));
-          __threadfence();
         }
         epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);   // the residual u
         epi_bar();
@@ -847,12 +847,17 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         }
         if (row_ok && idx_ok(fu <= P.ep.d / 32, P.err, 15, fu, 2)) P.ssq_z[(size_t)fu * P.ep.B + row] = ssq;
       }
+      // every thread's stores are issued; after the epilogue barrier one
+      // thread fences (also toward the async proxy: the next phase reads
+      // these outputs with TMA) and releases the flag
       if (tid == 0) trace_ev(P, gi, 10);
-      fence_proxy_async_global();   // the next phase reads these outputs with TMA
-      __threadfence();
-      if (tid == 0) trace_ev(P, gi, 11);
       epi_bar();
-      if (tid == 0 && release_allowed(P)) st_release_u32(flag_ptr(P, ph, T.rb, fu), (unsigned)(j + 1));
+      if (tid == 0) {
+        fence_proxy_async_global();
+        __threadfence();
+        trace_ev(P, gi, 11);
+        if (release_allowed(P)) st_release_u32(flag_ptr(P, ph, T.rb, fu), (unsigned)(j + 1));
+      }
       if (tid == 0) trace_ev(P, gi, 9);
       return true;
     });
