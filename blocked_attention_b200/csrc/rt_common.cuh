@@ -113,6 +113,30 @@ __device__ __forceinline__ float gelu_erf(float y) {
   return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f));
 }
 
+// erf by the rational approximation of Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (|error| <= 1.5e-7 for x >= 0; erf
+// is odd): erf(x) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-x^2),
+// t = 1 / (1 + p x). One reciprocal and one base-2 exponential (the PTX
+// approximate instructions) and six FMAs.
+__device__ __forceinline__ float erf_as7126(float x) {
+  const float ax = fabsf(x);
+  float t;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, ax, 1.f)));
+  float poly = fmaf(t, 1.061405429f, -1.453152027f);
+  poly = fmaf(t, poly, 1.421413741f);
+  poly = fmaf(t, poly, -0.284496736f);
+  poly = fmaf(t, poly, 0.254829592f);
+  poly *= t;
+  float e;   // exp(-x^2) = 2^(-x^2 log2 e)
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-ax * ax * 1.44269504088896341f));
+  return copysignf(fmaf(-poly, e, 1.f), x);
+}
+// GELU with that erf: the layer's bf16 path (its outputs are bf16-rounded,
+// 2^-9 relative, far above the approximation's error)
+__device__ __forceinline__ float gelu_as7126(float y) {
+  return 0.5f * y * (1.0f + erf_as7126(y * 0.70710678118654752f));
+}
+
 // scale of an empty accumulator: exp2(m_old - m_new) with m_old = -inf -> 0
 __device__ __forceinline__ float rescale(float m_old, float m_new) {
   return (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);

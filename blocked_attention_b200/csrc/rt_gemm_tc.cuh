@@ -237,7 +237,7 @@ __device__ __forceinline__ float epilogue_chunk(const EpiParams& p, int row, int
     store_bf16x32(p.u16 + (size_t)row * p.d + col0, v);
   } else if constexpr (EPI == EPI_W1) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i] * row_scale);
+    for (int i = 0; i < 32; ++i) v[i] = gelu_as7126(v[i] * row_scale);
     store_bf16x32(p.h16 + (size_t)row * p.d_ff + col0, v);
   } else if constexpr (EPI == EPI_W2) {
     const int b = row % p.B, jj = p.j + row / p.B;

@@ -230,7 +230,8 @@ __device__ __forceinline__ void note_wait(const StepsParams& P, int role, unsign
 // k < 16: 16 + k producer has the slot, 48 + k an issuer saw the stage
 // loaded; 32 producer saw every dependency; epilogue sub-steps: 10 outputs
 // stored, 11 fences done, 40 + 2c / 41 + 2c chunk c (< 4) read from tensor
-// memory / written
+// memory / written; a W2 split: 12 partial written, 13 every split arrived,
+// 14 its columns summed
 constexpr int kTraceSlots = 64;
 __device__ __forceinline__ void trace_ev(const StepsParams& P, int gi, int ev) {
 #ifdef RT_TRACE
@@ -814,6 +815,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
+        if (tid == 0) trace_ev(P, gi, 12);
         epi_bar();
         // Every split of the tile has written its slot once the tile's
         // arrival count reaches S (j + 1). The S splits run on S different
@@ -830,6 +832,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         }
         epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);   // the residual u
         epi_bar();
+        if (tid == 0) trace_ev(P, gi, 13);
         const int fc = flag_cols(g), c0 = T.split * fc;
         const float* slots = P.w2part + tile_i * g.S * (size_t)g.BN * C::BM;
         float ssq = 0.f;
@@ -843,6 +846,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] += __ldcg(src + (size_t)i * C::BM);
           }
+          if (tid == 0 && c == c0) trace_ev(P, gi, 14);
           if (row_ok) ssq += epilogue_chunk<EPI_W2>(e, row, col_base + c, g.N, v, 1.f, P.err);
         }
         if (row_ok && idx_ok(fu <= P.ep.d / 32, P.err, 15, fu, 2)) P.ssq_z[(size_t)fu * P.ep.B + row] = ssq;
