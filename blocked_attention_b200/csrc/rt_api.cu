@@ -423,7 +423,7 @@ static Plan make_plan(const Shape& s) {
     P.off_flags = take((size_t)PH_COUNT * P.sp.nrb * kFlagStride * 4);
     P.off_w2cnt = take((size_t)P.sp.nrb * g2.tiles * 4);
     P.off_w2part = take((size_t)P.sp.nrb * g2.tiles * g2.S * g2.BN * StepsCfg::BM * 4);
-    P.off_progress = take((size_t)1024 * 8 * 4);   // the debug build's per-CTA progress record
+    P.off_progress = take((size_t)1024 * 10 * 4);   // the debug build's per-CTA progress record
   }
   if (s.dtype == RT_BF16) {
     const int M = s.step_rows();

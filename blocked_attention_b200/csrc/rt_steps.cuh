@@ -86,7 +86,7 @@ struct StepsCfg {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = 3;
   static constexpr uint32_t TMEM_COLS = 512;                // 2 tiles in flight x 2 issuers x 128
-  static constexpr int THREADS = 224;                       // producer, 2 MMA issuers, 4 epilogue warps
+  static constexpr int THREADS = 352;                       // producer, 2 MMA issuers, 4 epilogue, 4 fold warps
   static constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 };
 
@@ -111,7 +111,7 @@ struct StepsParams {
   unsigned* w2cnt;             // [nrb][tiles of W2]: split arrivals, cumulative over the forward
   float* w2part;               // [nrb][tiles][S][BN_2][128] fp32 partial tiles
   unsigned* err;
-  unsigned* progress;          // (debug build) [gridDim][8]: the task and the wait each role of each CTA is at
+  unsigned* progress;          // (debug build) [gridDim][10]: the task and the wait each role of each CTA is at
   unsigned long long* trace;   // (trace build) [tasks of the segment][16] event times, or null
   float sc2;                   // log2(e) / sqrt(d_h)
   int H, nrb, G;               // heads, row blocks, fold groups of 32 sequences per row block
@@ -143,6 +143,8 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 // barrier of the four epilogue warps (named barrier 1, 128 threads)
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// barrier of the four fold warps (named barrier 2, 128 threads)
+__device__ __forceinline__ void fold_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 // Bounded poll until *f >= target (acquire). Returns at once once the error
 // word is set; a poll that runs out sets RT_DEVERR_TIMEOUT. Either way the
@@ -202,7 +204,7 @@ __device__ __forceinline__ bool release_allowed(const StepsParams& P) {
 }
 
 // (debug build) role r of this CTA is at task (ph, j, loc): producer 0, MMA
-// issuers 1 and 2, epilogue 3 (word 2r), and in which wait (word 2r + 1:
+// issuers 1 and 2, epilogue 3, folds 4 (word 2r), and in which wait (word 2r + 1:
 // kind in bits 28..30 -- 1 ring slot free, 2 dependency flag, 3 accumulator
 // free, 4 stage loaded, 5 accumulator full, 6 slot's previous round seen --
 // then the ring stage counter or task counter in bits 0..27)
@@ -210,14 +212,14 @@ __device__ __forceinline__ void note_progress(const StepsParams& P, int role, in
 #ifdef RT_BOUNDS_CHECK
   // frozen once the error word is set: the record shows where each role was
   if (P.progress && ld_volatile_u32(P.err) == 0)
-    *reinterpret_cast<volatile unsigned*>(P.progress + blockIdx.x * 8 + 2 * role) =
+    *reinterpret_cast<volatile unsigned*>(P.progress + blockIdx.x * 10 + 2 * role) =
         ((unsigned)(j & 0xfff) << 12) | ((ph & 7) << 9) | (loc & 0x1ff) | 0x80000000u;
 #endif
 }
 __device__ __forceinline__ void note_wait(const StepsParams& P, int role, unsigned kind, unsigned counter) {
 #ifdef RT_BOUNDS_CHECK
   if (P.progress && ld_volatile_u32(P.err) == 0)
-    *reinterpret_cast<volatile unsigned*>(P.progress + blockIdx.x * 8 + 2 * role + 1) =
+    *reinterpret_cast<volatile unsigned*>(P.progress + blockIdx.x * 10 + 2 * role + 1) =
         (kind << 28) | (counter & 0x0fffffffu) | 0x80000000u;
 #endif
 }
@@ -681,63 +683,16 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       tc_commit(&drain[par]);
       mbar_wait(&drain[par], 0u, P.err);
     }
-  } else {
-    // ---------------- epilogue warps: GEMM epilogues and small folds ----------------
+  } else if (warp < 7) {
+    // ---------------- epilogue warps: the GEMM epilogues ----------------
     const int tid = threadIdx.x - 96;   // 0..127
     const int q = warp & 3;             // TMEM lanes 32q .. 32q + 31
     const int lrow = q * 32 + lane;
     uint32_t local = 0;
     for_my_tasks(P, [&](int ph, int j, int loc, int gi) -> bool {
+      if (ph >= PH_FOLD) return true;   // the fold warps' tasks
       if (tid == 0) note_progress(P, 3, ph, j, loc);
       if (tid == 0) trace_ev(P, gi, 6);
-      if (ph == PH_FOLD || ph == PH_DEFER) {
-        // FOLD (step j, t = j + 1): the block's keys into its first query t,
-        // which is finalised (a_t, read by the next step's W_o). DEFER (step
-        // j, t = j): the same block of the previous step into its other
-        // queries t + 1 .. t + nq - 1, off the critical path; the fold of
-        // step j (query t + 1 = j + 1) waits for it.
-        const bool urgent = ph == PH_FOLD;
-        const int per_rb = P.H * P.G;
-        const int rb = loc / per_rb, r = loc - rb * per_rb;
-        const int h = r / P.G, gq = r - h * P.G;
-        const int t = urgent ? j + 1 : j, lb = lowbit(t), nq = min(lb, P.ep.Nseq - t);
-        const unsigned kv_ready = urgent ? (unsigned)(j + 1) : (unsigned)j;   // k, v of position t - 1
-        // this head's k and v of step t - 1 (and, through them, everything before)
-        const int kt = (64 * h) / P.g[PH_WKV].BN, vt = (P.ep.d + 64 * h) / P.g[PH_WKV].BN;
-        if (tid == 0) poll_ge(flag_ptr(P, PH_WKV, rb, kt), kv_ready, P.err, 47, wait_site(ph, j, kt));
-        if (tid == 32) poll_ge(flag_ptr(P, PH_WKV, rb, vt), kv_ready, P.err, 47, wait_site(ph, j, vt));
-        if (urgent && tid == 64 && phase_tasks(P, PH_DEFER, j) > 0)
-          poll_ge(flag_ptr(P, PH_DEFER, rb, r), (unsigned)(j + 1), P.err, 50, wait_site(ph, j, r));
-        epi_bar();
-        if (tid == 0) trace_ev(P, gi, 7);
-        const int s0 = rb * 128 + gq * kFoldSeqs;
-        const int ns = min(kFoldSeqs, min(P.ep.B - s0, (rb + 1) * 128 - s0));
-        const int init = t == lb ? 1 : 0;
-        if (ns > 0 && urgent && nq > 0) {
-          switch (lb) {
-            case 1: fold_small_units<1, 2>(P, t, 1, t - 1, init, h, s0, ns, tid, 1); break;
-            case 2: fold_small_units<2, 2>(P, t, 1, t - 2, init, h, s0, ns, tid, 1); break;
-            case 4: fold_small_units<4, 2>(P, t, 1, t - 4, init, h, s0, ns, tid, 1); break;
-            default: fold_small_units<8, 2>(P, t, 1, t - 8, init, h, s0, ns, tid, 1); break;
-          }
-        } else if (ns > 0 && !urgent && nq > 1) {
-          switch (lb) {
-            case 2: fold_small_units<2, 4>(P, t + 1, nq - 1, t - 2, init, h, s0, ns, tid, 0); break;
-            case 4: fold_small_units<4, 3>(P, t + 1, nq - 1, t - 4, init, h, s0, ns, tid, 0); break;
-            default: fold_small_units<8, 2>(P, t + 1, nq - 1, t - 8, init, h, s0, ns, tid, 0); break;
-          }
-        }
-        if (tid == 0) trace_ev(P, gi, 10);
-        epi_bar();
-        if (tid == 0) {
-          fence_proxy_async_global();   // a is read by the next step's TMA loads
-          __threadfence();
-          trace_ev(P, gi, 11);
-          if (release_allowed(P)) st_release_u32(flag_ptr(P, ph, rb, r), (unsigned)(j + 1));
-        }
-        if (tid == 0) trace_ev(P, gi, 9);
-        return true;
-      }
       const GemmPhase& g = P.g[ph];
       const GemmTask T = decode_gemm(g, loc);
       const int nst = (T.sl1 - T.sl0 + C::KSUB - 1) / C::KSUB;
@@ -863,6 +818,60 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         if (release_allowed(P)) st_release_u32(flag_ptr(P, ph, T.rb, fu), (unsigned)(j + 1));
       }
       if (tid == 0) trace_ev(P, gi, 9);
+      return true;
+    });
+  } else {
+    // ---------------- fold warps: the small folds (FOLD and DEFER tasks) ----------------
+    const int ftid = threadIdx.x - 224;   // 0..127
+    for_my_tasks(P, [&](int ph, int j, int loc, int gi) -> bool {
+      if (ph < PH_FOLD) return true;
+      if (ftid == 0) note_progress(P, 4, ph, j, loc);
+      if (ftid == 0) trace_ev(P, gi, 6);
+      // FOLD (step j, t = j + 1): the block's keys into its first query t,
+      // which is finalised (a_t, read by the next step's W_o). DEFER (step
+      // j, t = j): the same block of the previous step into its other
+      // queries t + 1 .. t + nq - 1, off the critical path; the fold of
+      // step j (query t + 1 = j + 1) waits for it.
+      const bool urgent = ph == PH_FOLD;
+      const int per_rb = P.H * P.G;
+      const int rb = loc / per_rb, r = loc - rb * per_rb;
+      const int h = r / P.G, gq = r - h * P.G;
+      const int t = urgent ? j + 1 : j, lb = lowbit(t), nq = min(lb, P.ep.Nseq - t);
+      const unsigned kv_ready = urgent ? (unsigned)(j + 1) : (unsigned)j;   // k, v of position t - 1
+      // this head's k and v of step t - 1 (and, through them, everything before)
+      const int kt = (64 * h) / P.g[PH_WKV].BN, vt = (P.ep.d + 64 * h) / P.g[PH_WKV].BN;
+      if (ftid == 0) poll_ge(flag_ptr(P, PH_WKV, rb, kt), kv_ready, P.err, 47, wait_site(ph, j, kt));
+      if (ftid == 32) poll_ge(flag_ptr(P, PH_WKV, rb, vt), kv_ready, P.err, 47, wait_site(ph, j, vt));
+      if (urgent && ftid == 64 && phase_tasks(P, PH_DEFER, j) > 0)
+        poll_ge(flag_ptr(P, PH_DEFER, rb, r), (unsigned)(j + 1), P.err, 50, wait_site(ph, j, r));
+      fold_bar();
+      if (ftid == 0) trace_ev(P, gi, 7);
+      const int s0 = rb * 128 + gq * kFoldSeqs;
+      const int ns = min(kFoldSeqs, min(P.ep.B - s0, (rb + 1) * 128 - s0));
+      const int init = t == lb ? 1 : 0;
+      if (ns > 0 && urgent && nq > 0) {
+        switch (lb) {
+          case 1: fold_small_units<1, 2>(P, t, 1, t - 1, init, h, s0, ns, ftid, 1); break;
+          case 2: fold_small_units<2, 2>(P, t, 1, t - 2, init, h, s0, ns, ftid, 1); break;
+          case 4: fold_small_units<4, 2>(P, t, 1, t - 4, init, h, s0, ns, ftid, 1); break;
+          default: fold_small_units<8, 1>(P, t, 1, t - 8, init, h, s0, ns, ftid, 1); break;
+        }
+      } else if (ns > 0 && !urgent && nq > 1) {
+        switch (lb) {
+          case 2: fold_small_units<2, 2>(P, t + 1, nq - 1, t - 2, init, h, s0, ns, ftid, 0); break;
+          case 4: fold_small_units<4, 2>(P, t + 1, nq - 1, t - 4, init, h, s0, ns, ftid, 0); break;
+          default: fold_small_units<8, 1>(P, t + 1, nq - 1, t - 8, init, h, s0, ns, ftid, 0); break;
+        }
+      }
+      if (ftid == 0) trace_ev(P, gi, 10);
+      fold_bar();
+      if (ftid == 0) {
+        fence_proxy_async_global();   // a is read by the next step's TMA loads
+        __threadfence();
+        trace_ev(P, gi, 11);
+        if (release_allowed(P)) st_release_u32(flag_ptr(P, ph, rb, r), (unsigned)(j + 1));
+      }
+      if (ftid == 0) trace_ev(P, gi, 9);
       return true;
     });
   }
