@@ -503,6 +503,65 @@ __device__ __forceinline__ float epi_tile_tmem(const EpiParams& e, int row, bool
   return ssq;
 }
 
+// W_o tile epilogue (BN = 64) with the residual x already in registers (the
+// epilogue loads it before it waits for the accumulator): u = x + a W_o^T,
+// written fp32 and bf16; returns the row's sum of squares over the tile.
+__device__ __forceinline__ float epi_wo_tile64(const EpiParams& e, int row, bool row_ok, int col_base,
+                                               uint32_t taddr, bool two, const uint4 (&xw)[8], unsigned* dbg_err) {
+  float ssq = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float v[32];
+    tmem_ld_pair(taddr + 32 * h, two, v);
+    const int col0 = col_base + 32 * h;
+    if (!row_ok || !idx_ok(e.j + row / e.B < e.Nseq && col0 + 32 <= e.d, dbg_err, 20 + EPI_WO, row, col0)) continue;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float xf[8];
+      unpack_bf16x8(xw[4 * h + k], xf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float w = v[8 * k + i];
+        if (e.pages) w *= e.inv_sqrt_L;
+        w += xf[i];
+        v[8 * k + i] = w;
+        ssq += w * w;
+      }
+    }
+    float4* u4 = reinterpret_cast<float4*>(e.u32 + (size_t)row * e.d + col0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    store_bf16x32(e.u16 + (size_t)row * e.d + col0, v);
+  }
+  return ssq;
+}
+
+// W_2 epilogue of one 32-column chunk with the residual u already in
+// registers: z = u + h W_2^T, written to the layer output and the bf16
+// operand of W_kv; returns the chunk's sum of squares.
+__device__ __forceinline__ float epi_w2_chunk_pre(const EpiParams& e, int row, bool row_ok, int col0,
+                                                  float (&v)[32], const uint4 (&uw)[8], unsigned* dbg_err) {
+  if (!row_ok || !idx_ok(e.j + row / e.B < e.Nseq && col0 + 32 <= e.d, dbg_err, 20 + EPI_W2, row, col0)) return 0.f;
+  const int b = row % e.B, jj = e.j + row / e.B;
+  float ssq = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float u[4] = {__uint_as_float(uw[i].x), __uint_as_float(uw[i].y), __uint_as_float(uw[i].z),
+                        __uint_as_float(uw[i].w)};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float w = v[4 * i + k];
+      if (e.pages) w *= e.inv_sqrt_L;
+      w += u[k];
+      v[4 * i + k] = w;
+      ssq += w * w;
+    }
+  }
+  store_bf16x32(e.zout + ((size_t)b * e.Nseq + jj) * e.d + col0, v);
+  store_bf16x32(e.z16 + (size_t)row * e.d + col0, v);
+  return ssq;
+}
+
 // The epilogue-side dependencies of a task, polled in parallel by the 128
 // epilogue threads (thread i polls flag i of a contiguous range; the polls
 // are acquire loads), then the epilogue barrier, which orders every epilogue
@@ -708,9 +767,7 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       } else if (ph == PH_W1) {
         epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);
       } else if (ph == PH_W2) {
-        // the residual u (a split's epilogue reads only tensor memory; the
-        // last split polls these before it sums the partial tiles)
-        if (g.S == 1) epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);
+        epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);   // the residual u
       } else {
         epi_poll_range(P, PH_W2, T.rb, 0, phase_flags(P.g[PH_W2]), (unsigned)(j + 1), tid);
       }
@@ -726,7 +783,27 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
         e.ssq_in = P.ssq_z; e.ssq_tiles = phase_flags(P.g[PH_W2]);
         if (row_ok) rs = row_scale_for<EPI_WKV>(e, row);
       }
-      if (row_ok && ph == PH_WO) epilogue_prefetch<EPI_WO>(e, row, col_base, g.N, g.BN);
+      // W_o: the residual x (an input of the layer, never written here) is
+      // loaded now, while the tile's MMAs run
+      const bool wo64 = ph == PH_WO && g.BN == 64;
+      // a W_2 split finishes 32 columns: their residual u, loaded now as well
+      const bool w2pre = ph == PH_W2 && g.S > 1 && flag_cols(g) == 32;
+      uint4 xw[8];   // W_o: 64 bf16 of x; a W_2 split: 32 fp32 of u (their bits)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xw[i] = make_uint4(0, 0, 0, 0);
+      if (w2pre && row_ok) {
+        const uint4* up = reinterpret_cast<const uint4*>(P.ep.u32 + (size_t)row * P.ep.d + col_base + T.split * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xw[i] = __ldcg(up + i);
+      } else if (wo64 && row_ok) {
+        const int b = row % P.ep.B, jj = j + row / P.ep.B, ch = jj / P.ep.xc;
+        const uint4* xp = reinterpret_cast<const uint4*>(
+            P.ep.x + (((size_t)ch * P.ep.B + b) * P.ep.xc + (jj - ch * P.ep.xc)) * P.ep.d + col_base);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xw[i] = __ldg(xp + i);
+      } else if (row_ok && ph == PH_WO) {
+        epilogue_prefetch<EPI_WO>(e, row, col_base, g.N, g.BN);
+      }
       // A wait that gives up (error word set) does not end the task: the four
       // epilogue warps must reach every named barrier together, so they run
       // on with whatever tensor memory holds.
@@ -741,7 +818,10 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       if (g.S == 1) {
         float ssq = 0.f;
         switch (ph) {
-          case PH_WO: ssq = epi_tile_tmem<EPI_WO>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi); break;
+          case PH_WO:
+            ssq = wo64 ? epi_wo_tile64(e, row, row_ok, col_base, taddr, two, xw, P.err)
+                       : epi_tile_tmem<EPI_WO>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi);
+            break;
           case PH_W1: epi_tile_tmem<EPI_W1>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi); break;
           case PH_W2: ssq = epi_tile_tmem<EPI_W2>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi); break;
           default: epi_tile_tmem<EPI_WKV>(e, row, row_ok, col_base, g.BN, taddr, two, rs, P.err, P, gi); break;
@@ -785,7 +865,6 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
           atom_add_acq_rel(cnt, 1u);
           poll_ge(cnt, (unsigned)(g.S * (j + 1)), P.err, 49, wait_site(ph, j, loc));
         }
-        epi_poll_range(P, PH_WO, T.rb, 0, P.g[PH_WO].tiles, (unsigned)(j + 1), tid);   // the residual u
         epi_bar();
         if (tid == 0) trace_ev(P, gi, 13);
         const int fc = flag_cols(g), c0 = T.split * fc;
@@ -802,7 +881,8 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
             for (int i = 0; i < 32; ++i) v[i] += __ldcg(src + (size_t)i * C::BM);
           }
           if (tid == 0 && c == c0) trace_ev(P, gi, 14);
-          if (row_ok) ssq += epilogue_chunk<EPI_W2>(e, row, col_base + c, g.N, v, 1.f, P.err);
+          if (w2pre) ssq += epi_w2_chunk_pre(e, row, row_ok, col_base + c, v, xw, P.err);
+          else if (row_ok) ssq += epilogue_chunk<EPI_W2>(e, row, col_base + c, g.N, v, 1.f, P.err);
         }
         if (row_ok && idx_ok(fu <= P.ep.d / 32, P.err, 15, fu, 2)) P.ssq_z[(size_t)fu * P.ep.B + row] = ssq;
       }
