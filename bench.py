@@ -58,7 +58,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="headline")
     ap.add_argument("--schedule", choices=["blocked", "naive"], default="blocked")
-    ap.add_argument("--driver", choices=["graph", "stream"], default="graph")
+    ap.add_argument("--driver", choices=["graph", "stream", "persistent"], default="graph")
+    ap.add_argument("--no-drivers", action="store_true",
+                    help="skip timing the headline with the other step-loop driver")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -497,7 +499,7 @@ def run_profile_case(args, R, torch, rtinputs):
         W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
              for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16").items()}
         x = torch.randn((B, N, d), device=dev, dtype=torch.bfloat16)
-        z, _, _ = R.layer_forward(x, W, H, driver="stream" if args.profile_case == "step" else "graph")
+        z, _, _ = R.layer_forward(x, W, H, driver="persistent" if args.profile_case == "step" else "graph")
     elif args.profile_case == "naive":
         B, N, d, H, dff = args.pB, args.lb, 1024, 16, 4096
         W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
@@ -645,12 +647,13 @@ def main():
     if args.schedule == "blocked" and not args.no_ablation:
         wsn = R.alloc_workspace(R.workspace_bytes(Bsz, N, d, H, dff, torch.bfloat16, "naive"), dev)
         outn = (torch.empty_like(z), torch.empty_like(K), torch.empty_like(V))
-        R.layer_forward(x, W, H, schedule="naive", driver=args.driver, out=outn, workspace=wsn)
+        ndrv = "graph" if args.driver == "persistent" else args.driver   # the naive schedule has no step kernel
+        R.layer_forward(x, W, H, schedule="naive", driver=ndrv, out=outn, workspace=wsn)
         torch.cuda.synchronize()
         n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n0.record(stream)
         for _ in range(args.ablation_steps):
-            R.layer_forward(x, W, H, schedule="naive", driver=args.driver, out=outn, workspace=wsn)
+            R.layer_forward(x, W, H, schedule="naive", driver=ndrv, out=outn, workspace=wsn)
         n1.record(stream)
         torch.cuda.synchronize()
         if R.sync_status(wsn) != 0:
@@ -663,6 +666,24 @@ def main():
                     "blocked_speedup": n_ms / ms_step}
         del wsn, outn
         torch.cuda.empty_cache()
+
+    # the same forward with the other step-loop driver (one kernel per phase,
+    # or the persistent step kernel): 1 warm-up, 2 timed
+    drivers = None
+    if args.schedule == "blocked" and not args.no_drivers and args.driver in ("graph", "persistent"):
+        other = "persistent" if args.driver == "graph" else "graph"
+        R.layer_forward(x, W, H, driver=other, out=(z, K, V), workspace=ws)
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(2):
+            R.layer_forward(x, W, H, driver=other, out=(z, K, V), workspace=ws)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        if R.sync_status(ws) != 0:
+            raise RuntimeError(f"device error with the {other} driver")
+        o_ms = d0.elapsed_time(d1) / 2
+        drivers = {args.driver: {"ms_per_step": ms_step}, other: {"ms_per_step": o_ms, "steps": 2}}
 
     # end to end through the public C ABI with HOST buffers (copies in the timed region)
     e2e = None
@@ -714,8 +735,9 @@ def main():
         "config": workload_config(args, cfg, world),
         "roofline": roofline, "step_roofline": step_roof, "kernels": kernels, "fold_levels": fold_levels,
         "ablation": ablation,
+        "drivers": drivers,
         "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": R.launch_count(Bsz, N, d, H, dff, torch.bfloat16, args.schedule) * args.steps,
+        "gpu_launches": R.launch_count(Bsz, N, d, H, dff, torch.bfloat16, args.schedule, args.driver) * args.steps,
         "clocks": clocks,
     }), flush=True)
 

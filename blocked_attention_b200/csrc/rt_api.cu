@@ -582,8 +582,9 @@ static cudaError_t launch_attend(const Plan& P, const T* qkv, const T* K, const 
 // bf16 forward
 // ---------------------------------------------------------------------------
 static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st, Timer* T,
-                        const HostIo* io = nullptr) {
+                        const HostIo* io = nullptr, bool persistent = false) {
   const Shape& s = P.s;
+  const bool steps = persistent && P.sp.ok;   // the persistent step kernel, else one kernel per phase
   char* ws = static_cast<char*>(X.ws);
   unsigned* err = reinterpret_cast<unsigned*>(ws + P.off_err);
   bf16* qkv = reinterpret_cast<bf16*>(ws + P.off_qkv);
@@ -695,7 +696,6 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
       !make_tmap(&tA_z, z16, d, B, 128) || !make_tmap(&tB_kv, wqkv + (size_t)d * d, d, 2 * d, bn_kv))
     return RT_ERR_INVALID_ARG;
   const float sc2 = s.sc2();
-  if (s.pages && !P.sp.ok) return RT_ERR_UNSUPPORTED;   // head normalisation lives in the step kernel
   const bool blocked = s.schedule == RT_SCHED_BLOCKED;
   // step j reads queries and temporary pairs of positions up to 2j + 1
   // (the fold of step j covers queries j + 1 .. 2j + 1, 0-based) and x of j
@@ -709,7 +709,7 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
     TimedScope ts(T, KC_ATTEND, st);
     RT_CK((launch_attend<bf16, 2>(P, qkv, K, V, m, l, o, a16, 0, sc2, st)));
   }
-  if (P.sp.ok) {
+  if (steps) {
     // persistent step kernel: one launch per segment of steps whose folds
     // have at most 8 keys; the segment's last fold (>= 16 keys) follows it
     StepsParams sp;
@@ -777,7 +777,7 @@ static int enqueue_bf16(const Plan& P, const Ptrs& X, const DevState& ds, cudaSt
       j = j1;
     }
   }
-  for (int j = 0; j < N && !P.sp.ok; ++j) {
+  for (int j = 0; j < N && !steps; ++j) {
     ep.j = j;
     {
       const int rc = project_through(std::min(N - 1, 2 * j + 1));
@@ -1018,7 +1018,7 @@ static int enqueue_chunked(const Plan& P, const Ptrs& X, const DevState& ds, cud
 }
 
 static int enqueue_forward(const Plan& P, const Ptrs& X, const DevState& ds, cudaStream_t st,
-                           Timer* T = nullptr, const HostIo* io = nullptr) {
+                           Timer* T = nullptr, const HostIo* io = nullptr, bool persistent = false) {
   if (P.s.chunk > 0) {
     if (io) return RT_ERR_UNSUPPORTED;
     return enqueue_chunked(P, X, ds, st, T);
@@ -1026,13 +1026,13 @@ static int enqueue_forward(const Plan& P, const Ptrs& X, const DevState& ds, cud
   if (io) {
     if (P.s.dtype != RT_BF16) return RT_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_io_mu);
-    return enqueue_bf16(P, X, ds, st, T, io);
+    return enqueue_bf16(P, X, ds, st, T, io, persistent);
   }
-  return P.s.dtype == RT_BF16 ? enqueue_bf16(P, X, ds, st, T) : enqueue_f32(P, X, st, T);
+  return P.s.dtype == RT_BF16 ? enqueue_bf16(P, X, ds, st, T, nullptr, persistent) : enqueue_f32(P, X, st, T);
 }
 
 // Kernels one forward launches (must mirror enqueue_bf16 / enqueue_f32).
-static long launch_count(const Shape& s) {
+static long launch_count(const Shape& s, int driver) {
   long folds = 0;
   if (s.schedule == RT_SCHED_BLOCKED)
     for (int t = 1; t <= s.N; ++t) folds += (std::min(lowbit(t), s.N - t) > 0) ? 1 : 0;
@@ -1042,7 +1042,7 @@ static long launch_count(const Shape& s) {
     return 2 + 5l * nchunks + (nchunks - 1);
   }
   if (s.dtype == RT_BF16) {
-    if (s.schedule == RT_SCHED_BLOCKED && plan_steps(s).ok) {
+    if (driver == RT_DRIVER_PERSISTENT && plan_steps(s).ok) {
       // finalise(position 1) + one step kernel per segment + the folds of
       // >= 16 keys that end segments (each finalises the next position)
       long segments = 0, big = 0;
@@ -1064,7 +1064,7 @@ static long launch_count(const Shape& s) {
 // ---------------------------------------------------------------------------
 struct GraphKey {
   uintptr_t p[15];
-  int v[11];
+  int v[12];
   bool operator<(const GraphKey& o) const {
     int c = std::memcmp(p, o.p, sizeof(p));
     if (c) return c < 0;
@@ -1080,14 +1080,22 @@ static std::map<GraphKey, GraphEntry> g_graphs;
 static unsigned long long g_graph_clock = 0;
 static constexpr size_t kMaxGraphs = 8;
 
+// The persistent driver takes the bf16 blocked forward at shapes the step
+// kernel's plan accepts.
+static bool persistent_ok(const Plan& P) {
+  return P.s.dtype == RT_BF16 && P.s.schedule == RT_SCHED_BLOCKED && P.s.chunk == 0 && P.sp.ok;
+}
+
 static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st, const HostIo* io = nullptr) {
+  const bool persistent = driver == RT_DRIVER_PERSISTENT;
+  if (persistent && !persistent_ok(P)) return RT_ERR_UNSUPPORTED;
   DevState* ds = nullptr;
   int rc = device_setup(&ds);
   if (rc != RT_OK) return rc;
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   RT_CK(cudaStreamIsCapturing(st, &cap));
   if (driver == RT_DRIVER_STREAM || cap != cudaStreamCaptureStatusNone)
-    return enqueue_forward(P, X, *ds, st, nullptr, io);
+    return enqueue_forward(P, X, *ds, st, nullptr, io, persistent);
 
   int dev = 0;
   RT_CK(cudaGetDevice(&dev));
@@ -1097,8 +1105,8 @@ static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st
                           io ? io->x_host : nullptr, io ? io->z_host : nullptr,
                           io ? io->K_host : nullptr, io ? io->V_host : nullptr};
   for (int i = 0; i < 15; ++i) key.p[i] = reinterpret_cast<uintptr_t>(ptrs[i]);
-  const int vals[11] = {P.s.B, P.s.N, P.s.d, P.s.H, P.s.d_ff, P.s.dtype, P.s.schedule, dev, P.s.pages, P.s.L,
-                        P.s.chunk};
+  const int vals[12] = {P.s.B, P.s.N, P.s.d, P.s.H, P.s.d_ff, P.s.dtype, P.s.schedule, dev, P.s.pages, P.s.L,
+                        P.s.chunk, driver};
   std::memcpy(key.v, vals, sizeof(vals));
 
   std::lock_guard<std::mutex> lk(g_graph_mu);
@@ -1108,11 +1116,11 @@ static int run_forward(const Plan& P, const Ptrs& X, int driver, cudaStream_t st
     cudaError_t ce = cudaSuccess;
     for (int attempt = 0; attempt < 2; ++attempt) {
       RT_CK(cudaStreamBeginCapture(ds->capture, cudaStreamCaptureModeThreadLocal));
-      rc = enqueue_forward(P, X, *ds, ds->capture, nullptr, io);
+      rc = enqueue_forward(P, X, *ds, ds->capture, nullptr, io, persistent);
       ce = cudaStreamEndCapture(ds->capture, &graph);
       // a capture that failed on the step kernel's cooperative launch is
       // recorded once more with plain launches
-      if ((rc == RT_ERR_CUDA || ce != cudaSuccess) && P.sp.ok && ds->coop && attempt == 0) {
+      if ((rc == RT_ERR_CUDA || ce != cudaSuccess) && persistent && ds->coop && attempt == 0) {
         if (graph) cudaGraphDestroy(graph);
         graph = nullptr;
         cudaGetLastError();
@@ -1183,7 +1191,8 @@ extern "C" int rt_layer_forward(const void* x, const void* W_q, const void* W_k,
   Shape s{B, N, d, H, d_ff, dtype, schedule};
   int rc = validate(s);
   if (rc != RT_OK) return rc;
-  if (driver != RT_DRIVER_GRAPH && driver != RT_DRIVER_STREAM) return RT_ERR_INVALID_ARG;
+  if (driver != RT_DRIVER_GRAPH && driver != RT_DRIVER_STREAM && driver != RT_DRIVER_PERSISTENT)
+    return RT_ERR_INVALID_ARG;
   if (!x || !W_q || !W_k || !W_v || !W_o || !W_1 || !W_2 || !z || !K || !V) return RT_ERR_INVALID_ARG;
   const void* all[10] = {x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V};
   for (const void* p : all)
@@ -1198,22 +1207,23 @@ extern "C" int rt_layer_forward(const void* x, const void* W_q, const void* W_k,
 extern "C" int rt_layer_forward_pages(const void* x, const void* W_q, const void* W_k, const void* W_v,
                                       const void* W_o, const void* W_1, const void* W_2, int B, int N, int d, int H,
                                       int d_ff, int L, void* z, void* K, void* V, void* workspace,
-                                      size_t workspace_bytes, void* stream) {
+                                      size_t workspace_bytes, void* stream, int driver) {
   Shape s{B, N, d, H, d_ff, RT_BF16, RT_SCHED_BLOCKED};
   s.pages = 1;
   s.L = L;
   int rc = validate(s);
   if (rc != RT_OK) return rc;
+  if (driver != RT_DRIVER_GRAPH && driver != RT_DRIVER_STREAM && driver != RT_DRIVER_PERSISTENT)
+    return RT_ERR_INVALID_ARG;
   if (!x || !W_q || !W_k || !W_v || !W_o || !W_1 || !W_2 || !z || !K || !V) return RT_ERR_INVALID_ARG;
   const void* all[10] = {x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V};
   for (const void* p : all)
     if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return RT_ERR_INVALID_ARG;
   const Plan P = make_plan(s);
-  if (!P.sp.ok) return RT_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < P.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return RT_ERR_WORKSPACE;
   Ptrs X{x, W_q, W_k, W_v, W_o, W_1, W_2, z, K, V, workspace};
-  return run_forward(P, X, RT_DRIVER_GRAPH, static_cast<cudaStream_t>(stream));
+  return run_forward(P, X, driver, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" size_t rt_layer_chunked_workspace_bytes(int B, int N, int d, int H, int d_ff, int C) {
@@ -1579,10 +1589,12 @@ extern "C" int rt_gemm_bf16(const void* A, const void* W, float* C, int M, int N
   return RT_OK;
 }
 
-extern "C" long rt_layer_launch_count(int B, int N, int d, int H, int d_ff, int dtype, int schedule) {
+extern "C" long rt_layer_launch_count(int B, int N, int d, int H, int d_ff, int dtype, int schedule, int driver) {
   Shape s{B, N, d, H, d_ff, dtype, schedule};
   if (validate(s) != RT_OK) return -1;
-  return launch_count(s);
+  if (driver != RT_DRIVER_GRAPH && driver != RT_DRIVER_STREAM && driver != RT_DRIVER_PERSISTENT) return -1;
+  if (driver == RT_DRIVER_PERSISTENT && !persistent_ok(make_plan(s))) return -1;
+  return launch_count(s, driver);
 }
 
 extern "C" int rt_layer_forward_timed(const void* x, const void* W_q, const void* W_k, const void* W_v,

@@ -18,10 +18,10 @@ RT_OK, RT_ERR_INVALID_ARG, RT_ERR_UNSUPPORTED, RT_ERR_WORKSPACE, RT_ERR_CUDA, RT
     0, -1, -2, -3, -4, -5, -6
 RT_F32, RT_BF16 = 0, 1
 RT_SCHED_BLOCKED, RT_SCHED_NAIVE = 0, 1
-RT_DRIVER_GRAPH, RT_DRIVER_STREAM = 0, 1
+RT_DRIVER_GRAPH, RT_DRIVER_STREAM, RT_DRIVER_PERSISTENT = 0, 1, 2
 
 SCHEDULES = {"blocked": RT_SCHED_BLOCKED, "naive": RT_SCHED_NAIVE}
-DRIVERS = {"graph": RT_DRIVER_GRAPH, "stream": RT_DRIVER_STREAM}
+DRIVERS = {"graph": RT_DRIVER_GRAPH, "stream": RT_DRIVER_STREAM, "persistent": RT_DRIVER_PERSISTENT}
 WEIGHT_NAMES = ("W_q", "W_k", "W_v", "W_o", "W_1", "W_2")
 
 EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_error_string",
@@ -89,7 +89,7 @@ def lib() -> ctypes.CDLL:
     L.rt_layer_forward_chunked.restype = i
     L.rt_layer_forward_chunked.argtypes = [vp] * 7 + [i] * 6 + [vp] * 4 + [sz, vp]
     L.rt_layer_forward_pages.restype = i
-    L.rt_layer_forward_pages.argtypes = [vp] * 7 + [i] * 6 + [vp] * 4 + [sz, vp]
+    L.rt_layer_forward_pages.argtypes = [vp] * 7 + [i] * 6 + [vp] * 4 + [sz, vp, i]
     L.rt_layer_sync_status.restype = i
     L.rt_layer_sync_status.argtypes = [vp, vp]
     L.rt_embed_forward.restype = i
@@ -101,7 +101,7 @@ def lib() -> ctypes.CDLL:
     L.rt_gemm_bf16.restype = i
     L.rt_gemm_bf16.argtypes = [vp, vp, fp, i, i, i, vp, vp]
     L.rt_layer_launch_count.restype = ctypes.c_long
-    L.rt_layer_launch_count.argtypes = [i] * 7
+    L.rt_layer_launch_count.argtypes = [i] * 8
     L.rt_layer_forward_timed.restype = i
     L.rt_layer_forward_timed.argtypes = [vp] * 7 + [i] * 7 + [vp] * 4 + [sz, vp, fp,
                                                                          ctypes.POINTER(ctypes.c_int), i]
@@ -202,7 +202,7 @@ def layer_forward(x: torch.Tensor, W: dict, H: int, d_ff: int | None = None, sch
 
 
 def layer_forward_pages(x: torch.Tensor, W: dict, H: int, L: int = 1, out=None,
-                        workspace: torch.Tensor | None = None, stream=None):
+                        workspace: torch.Tensor | None = None, stream=None, driver: str = "graph"):
     """rt_layer_forward_pages: the layer in the paper's own parameterisation
     (per-head unit-RMS queries and keys, no softmax scale, RMS without eps,
     branches scaled by 1/sqrt(L)); bf16 device tensors as in layer_forward."""
@@ -223,7 +223,7 @@ def layer_forward_pages(x: torch.Tensor, W: dict, H: int, L: int = 1, out=None,
         workspace = alloc_workspace(workspace_bytes(B, N, d, H, d_ff), x.device)
     rc = lib().rt_layer_forward_pages(_ptr(x), *[_ptr(W[n]) for n in WEIGHT_NAMES], B, N, d, H, d_ff, L,
                                       _ptr(z), _ptr(K), _ptr(V), _ptr(workspace),
-                                      ctypes.c_size_t(workspace.numel()), _stream(stream))
+                                      ctypes.c_size_t(workspace.numel()), _stream(stream), DRIVERS[driver])
     _check("rt_layer_forward_pages", rc)
     return z, K, V
 
@@ -287,8 +287,9 @@ def layer_forward_chunked(x: torch.Tensor, W: dict, H: int, C: int, out=None,
     return z, K, V
 
 
-def launch_count(B, N, d, H, d_ff, dtype=torch.bfloat16, schedule="blocked") -> int:
-    return int(lib().rt_layer_launch_count(B, N, d, H, d_ff, _dtype_code(dtype), SCHEDULES[schedule]))
+def launch_count(B, N, d, H, d_ff, dtype=torch.bfloat16, schedule="blocked", driver="graph") -> int:
+    return int(lib().rt_layer_launch_count(B, N, d, H, d_ff, _dtype_code(dtype), SCHEDULES[schedule],
+                                           DRIVERS[driver]))
 
 
 def layer_forward_timed(x: torch.Tensor, W: dict, H: int, out, workspace: torch.Tensor,

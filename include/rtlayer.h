@@ -73,10 +73,19 @@ typedef enum { RT_F32 = 0, RT_BF16 = 1 } rt_dtype;
  * Theta(N^2) traffic (the ablation of notes §4.1). Same result up to rounding. */
 typedef enum { RT_SCHED_BLOCKED = 0, RT_SCHED_NAIVE = 1 } rt_schedule;
 
-/* RT_DRIVER_GRAPH: the whole N-step loop is recorded once into a CUDA graph
- * (cached per argument set) and replayed with a single launch per call.
- * RT_DRIVER_STREAM: every kernel is launched from the host loop. */
-typedef enum { RT_DRIVER_GRAPH = 0, RT_DRIVER_STREAM = 1 } rt_driver;
+/* RT_DRIVER_GRAPH: the whole N-step loop (one kernel per phase of a step:
+ * W_o, W_1, W_2, W_kv GEMMs and the block fold) is recorded once into a
+ * CUDA graph (cached per argument set, consecutive kernels overlapped by
+ * programmatic dependent launch) and replayed with a single launch per call.
+ * RT_DRIVER_STREAM: the same kernels, each launched from the host loop.
+ * RT_DRIVER_PERSISTENT: bf16, blocked schedule only: the step loop as one
+ * persistent kernel per run of steps whose folds have at most 8 keys (every
+ * phase of every step inside it, ordered by flags in global memory), the
+ * folds of >= 16 keys between them; recorded into a cached graph like
+ * RT_DRIVER_GRAPH. RT_ERR_UNSUPPORTED for other dtypes, schedules or shapes
+ * whose per-phase flags exceed its flag table. Same results up to rounding
+ * order in all three. */
+typedef enum { RT_DRIVER_GRAPH = 0, RT_DRIVER_STREAM = 1, RT_DRIVER_PERSISTENT = 2 } rt_driver;
 
 /* Library version (major*10000 + minor*100 + patch). */
 int rt_version(void);
@@ -111,7 +120,7 @@ int rt_layer_forward(const void* x_dev,
 
 /* The layer in the paper's own parameterisation (paper §2 notation, §2.1 and
  * §2.2, rather than the single-layer configuration above), bf16, blocked
- * schedule, graph driver:
+ * schedule, driver as in rt_layer_forward:
  *   RMS(v) = sqrt(D) v / ||v|| (no eps, unit gain); RMS_h = the same over
  *   each head's 64 entries;
  *   r = RMS(x_t); q = RMS_h(W_q r); k~ = RMS_h(W_k r); v~ = W_v r
@@ -126,7 +135,8 @@ int rt_layer_forward_pages(const void* x_dev,
                            const void* W_o_dev, const void* W_1_dev, const void* W_2_dev,
                            int B, int N, int d, int H, int d_ff, int L,
                            void* z_dev, void* K_dev, void* V_dev,
-                           void* workspace_dev, size_t workspace_bytes, void* stream);
+                           void* workspace_dev, size_t workspace_bytes, void* stream,
+                           int driver);
 
 /* Device bytes rt_layer_forward_chunked needs for chunks of C positions;
  * 0 if unsupported. */
@@ -348,9 +358,10 @@ int rt_project_qkv_noalloc_status(void* stream);
  * Measurement
  * ------------------------------------------------------------------------ */
 
-/* Number of kernels one rt_layer_forward launches for this shape (the same
- * count whichever driver runs them); -1 for invalid arguments. */
-long rt_layer_launch_count(int B, int N, int d, int H, int d_ff, int dtype, int schedule);
+/* Number of kernels one rt_layer_forward launches for this shape with this
+ * driver (RT_DRIVER_GRAPH and RT_DRIVER_STREAM launch the same kernels); -1
+ * for invalid arguments or a shape the driver does not take. */
+long rt_layer_launch_count(int B, int N, int d, int H, int d_ff, int dtype, int schedule, int driver);
 
 /* Kernel classes reported by rt_layer_forward_timed. */
 enum {

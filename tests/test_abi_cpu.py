@@ -100,15 +100,24 @@ def _step_kernel_launches(N):
 
 
 def test_launch_count_matches_schedule(L):
-    # bf16 blocked: inv_rms + projection + finalise(position 1) + the step
-    # kernel's segments + the folds of >= 16 keys between them
+    G, S, P = R.RT_DRIVER_GRAPH, R.RT_DRIVER_STREAM, R.RT_DRIVER_PERSISTENT
     for N in (1, 2, 7, 16, 17, 64, 2048):
-        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0) == 3 + _step_kernel_launches(N)
-        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 1) == 2 + 5 * N
-    # the headline: 128 segments and 127 large folds
-    assert L.rt_layer_launch_count(512, 2048, 1024, 16, 4096, R.RT_BF16, 0) == 3 + 128 + 127
-    assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_F32, 0) == 2 + 8 * 8 + 7
-    assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_BF16, 0) == -1
+        folds = sum(1 for t in range(1, N + 1) if min(t & -t, N - t) > 0)
+        # per-kernel drivers: inv_rms + projection + finalise(position 1) + 4
+        # GEMMs per step + one fold per step that has one
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0, G) == 3 + 4 * N + folds
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0, S) == 3 + 4 * N + folds
+        # persistent: the step kernel's segments + the folds of >= 16 keys between them
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 0, P) == 3 + _step_kernel_launches(N)
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 1, G) == 2 + 5 * N
+        assert L.rt_layer_launch_count(4, N, 512, 8, 1024, R.RT_BF16, 1, P) == -1   # blocked only
+    # the headline: 2047 folds; persistent: 128 segments and 127 large folds
+    assert L.rt_layer_launch_count(512, 2048, 1024, 16, 4096, R.RT_BF16, 0, G) == 3 + 4 * 2048 + 2047
+    assert L.rt_layer_launch_count(512, 2048, 1024, 16, 4096, R.RT_BF16, 0, P) == 3 + 128 + 127
+    assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_F32, 0, G) == 2 + 8 * 8 + 7
+    assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_F32, 0, P) == -1
+    assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_F32, 0, 3) == -1
+    assert L.rt_layer_launch_count(4, 8, 64, 2, 256, R.RT_BF16, 0, R.RT_DRIVER_GRAPH) == -1
 
 
 def _fwd(L, ptr, B=2, N=8, d=64, H=2, d_ff=256, dtype=R.RT_F32, sched=0, driver=0, ws_bytes=1 << 30,
@@ -209,14 +218,15 @@ def test_recompute_validation_happens_before_any_launch(L):
 def test_pages_entry_point_validation_happens_before_any_launch(L):
     p = ctypes.c_void_p(1 << 40)
 
-    def call(Lv=1, d=128, H=2, ws_bytes=1 << 34):
+    def call(Lv=1, d=128, H=2, ws_bytes=1 << 34, driver=R.RT_DRIVER_GRAPH):
         return L.rt_layer_forward_pages(*([p] * 7), 2, 16, d, H, 256, Lv, p, p, p, p, ctypes.c_size_t(ws_bytes),
-                                        None)
+                                        None, driver)
     assert call(Lv=0) == R.RT_ERR_INVALID_ARG          # the stack depth L >= 1
     assert call(d=96, H=2) == R.RT_ERR_UNSUPPORTED       # bf16 needs d_h = 64
     assert call(ws_bytes=16) == R.RT_ERR_WORKSPACE
+    assert call(driver=7) == R.RT_ERR_INVALID_ARG
     assert L.rt_layer_forward_pages(None, *([p] * 6), 2, 16, 128, 2, 256, 1, p, p, p, p,
-                                    ctypes.c_size_t(1 << 34), None) == R.RT_ERR_INVALID_ARG
+                                    ctypes.c_size_t(1 << 34), None, R.RT_DRIVER_GRAPH) == R.RT_ERR_INVALID_ARG
 
 
 def test_chunked_entry_point_validation_happens_before_any_launch(L):

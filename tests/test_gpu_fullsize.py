@@ -26,13 +26,14 @@ def _filled_batch(B, N, d, seqs, seed):
     return x, xs
 
 
-def test_headline_config_sampled_sequences():
+@pytest.mark.parametrize("driver", ["graph", "persistent"])
+def test_headline_config_sampled_sequences(driver):
     from blocked_attention_b200 import rtlayer as R
     B, N, d, H, dff = 512, 2048, 1024, 16, 4096
     seqs = [0, 511]
     W = rtinputs.weights(0, d, dff, dtype="bf16")
     x, xs = _filled_batch(B, N, d, seqs, 0)
-    z, K, V = R.layer_forward(x, {k: to_device(v, "bf16") for k, v in W.items()}, H, driver="graph")
+    z, K, V = R.layer_forward(x, {k: to_device(v, "bf16") for k, v in W.items()}, H, driver=driver)
     torch.cuda.synchronize()
     zg, Kg, Vg = to_np(z[seqs]), to_np(K[:, seqs]).transpose(1, 0, 2), to_np(V[:, seqs]).transpose(1, 0, 2)
     del x, z, K, V

@@ -21,23 +21,27 @@ def rt():
     return R
 
 
+@pytest.mark.parametrize("driver", ["graph", "persistent"])
 @pytest.mark.parametrize("B,N,d,H,d_ff,L", [(3, 37, 128, 2, 256, 1), (2, 70, 128, 2, 256, 6),
                                             (130, 20, 192, 3, 320, 2), (1, 1, 64, 1, 64, 1)])
-def test_pages_parameterisation_matches_oracle(rt, B, N, d, H, d_ff, L):
+def test_pages_parameterisation_matches_oracle(rt, B, N, d, H, d_ff, L, driver):
     x, W = problem(B, N, d, H, d_ff, "bf16")
-    z, K, V = rt.layer_forward_pages(to_device(x, "bf16"), {k: to_device(v, "bf16") for k, v in W.items()}, H, L)
+    z, K, V = rt.layer_forward_pages(to_device(x, "bf16"), {k: to_device(v, "bf16") for k, v in W.items()}, H, L,
+                                     driver=driver)
     torch.cuda.synchronize()
     zr, Kr, Vr = O.rt_layer_pages(x, W, H, L)
     errs = (rel_err(to_np(z), zr), rel_err(to_np(K).transpose(1, 0, 2), Kr), rel_err(to_np(V).transpose(1, 0, 2), Vr))
     assert max(errs) <= TOL["bf16"], errs
 
 
-def test_pages_config_B64_N1024_d512_sampled(rt):
+@pytest.mark.parametrize("driver", ["graph", "persistent"])
+def test_pages_config_B64_N1024_d512_sampled(rt, driver):
     # the bf16 single-layer widths (B=64, N=1024, d=512, 8 heads of 64, d_ff=2048),
     # sampled sequences against the oracle; every fold kernel runs
     B, N, d, H, d_ff = 64, 1024, 512, 8, 2048
     x, W = problem(B, N, d, H, d_ff, "bf16")
-    z, K, V = rt.layer_forward_pages(to_device(x, "bf16"), {k: to_device(v, "bf16") for k, v in W.items()}, H, 1)
+    z, K, V = rt.layer_forward_pages(to_device(x, "bf16"), {k: to_device(v, "bf16") for k, v in W.items()}, H, 1,
+                                     driver=driver)
     torch.cuda.synchronize()
     seqs = [0, 63]
     zr, Kr, Vr = O.rt_layer_pages(x[seqs], W, H, 1)

@@ -143,10 +143,11 @@ def test_layer_f32_tiny_config(rt, schedule, driver):
     _check_layer(rt, 2, 64, 64, 2, 256, "f32", schedule=schedule, driver=driver)
 
 
+@pytest.mark.parametrize("driver", ["graph", "persistent"])
 @pytest.mark.parametrize("B,N,d,H,d_ff", [(3, 37, 128, 2, 256), (5, 100, 192, 3, 320), (1, 1, 64, 1, 64),
                                           (2, 2, 64, 1, 128), (130, 20, 128, 2, 256)])
-def test_layer_bf16_ragged_shapes(rt, B, N, d, H, d_ff):
-    _check_layer(rt, B, N, d, H, d_ff, "bf16")
+def test_layer_bf16_ragged_shapes(rt, B, N, d, H, d_ff, driver):
+    _check_layer(rt, B, N, d, H, d_ff, "bf16", driver=driver)
 
 
 def test_layer_f32_peaky_attention(rt):
@@ -203,6 +204,16 @@ def test_graph_replay_is_deterministic_and_matches_stream(rt):
     torch.cuda.synchronize()
     for a, b in zip(first, s):
         assert torch.equal(a, b)
+    # the persistent step kernel: replays are bitwise equal too (its W_2
+    # split partials are summed in split order), and it agrees with the
+    # per-kernel path up to rounding order
+    rt.layer_forward(xd, Wd, H, out=outs, workspace=ws, driver="persistent")
+    pfirst = [t.clone() for t in outs]
+    rt.layer_forward(xd, Wd, H, out=outs, workspace=ws, driver="persistent")
+    assert rt.sync_status(ws) == 0
+    for a, b, c in zip(pfirst, outs, first):
+        assert torch.equal(a, b)
+        assert rel_err(to_np(a), to_np(c)) < TOL["bf16"]
 
 
 def test_host_buffer_entry_point(rt):
@@ -223,7 +234,7 @@ def test_host_buffer_entry_point(rt):
 
 
 @pytest.mark.parametrize("pinned", [True, False])
-@pytest.mark.parametrize("driver", ["graph", "stream"])
+@pytest.mark.parametrize("driver", ["graph", "stream", "persistent"])
 def test_host_entry_matches_device_entry(rt, pinned, driver):
     # B=11 splits unevenly into the sequence chunks of the overlapped upload
     # and N=37 into its output ranges; pinned buffers take the overlapped
