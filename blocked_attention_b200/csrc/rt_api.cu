@@ -431,6 +431,9 @@ static Plan make_plan(const Shape& s) {
     P.t_w1 = choose_tiles(M, s.d_ff, s.d, kLayerSplitK);
     P.t_w2 = choose_tiles(M, s.d, s.d_ff, kLayerSplitK);
     P.t_wkv = choose_tiles(M, 2 * s.d, s.d, kLayerSplitK);
+    // the paper's parameterisation normalises every head of k inside the
+    // W_kv epilogue, which needs a head's 64 columns in one tile
+    if (s.pages && (P.t_wkv.bn < 64 || P.t_wkv.splits > 1)) P.t_wkv = TileCfg{64, 1};
   }
   P.total = off;
   return P;
