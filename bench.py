@@ -83,9 +83,10 @@ def parse():
                     help="activation-checkpoint recompute of K, V from z over all B*N rows")
     ap.add_argument("--backward", action="store_true",
                     help="backward pass (bf16 storage) at B=64 N=1024 d=512 H=8x64 d_ff=2048")
-    ap.add_argument("--profile-case", choices=["step", "fold", "fwd", "naive"],
+    ap.add_argument("--profile-case", choices=["step", "persistent", "fold", "fwd", "naive"],
                     help="run one small case for an ncu capture and exit: 'step' = one host-loop forward at "
-                         "B=512 N=64 d=1024 (the per-step GEMM shapes of the headline); 'fold' = one block fold "
+                         "B=512 N=64 d=1024 (the per-step GEMM shapes of the headline); 'persistent' = the same "
+                         "forward with the persistent step kernel; 'fold' = one block fold "
                          "of --lb keys into --lb queries at B=--pB H=16 (position-major); 'fwd' = one "
                          "graph-driver forward at the headline widths with N = --lb; 'naive' = one host-loop "
                          "naive-schedule forward at B=--pB, N=--lb, d=1024 H=16x64 d_ff=4096")
@@ -494,12 +495,13 @@ def run_next_rows(args, R, torch, rtinputs):
 
 def run_profile_case(args, R, torch, rtinputs):
     dev = torch.device("cuda", 0)
-    if args.profile_case in ("step", "fwd"):
-        B, N, d, H, dff = 512, (64 if args.profile_case == "step" else args.lb), 1024, 16, 4096
+    if args.profile_case in ("step", "persistent", "fwd"):
+        B, N, d, H, dff = 512, (args.lb if args.profile_case == "fwd" else 64), 1024, 16, 4096
         W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)
              for k, v in rtinputs.weights(args.seed, d, dff, dtype="bf16").items()}
         x = torch.randn((B, N, d), device=dev, dtype=torch.bfloat16)
-        z, _, _ = R.layer_forward(x, W, H, driver="persistent" if args.profile_case == "step" else "graph")
+        drv = {"step": "stream", "persistent": "persistent", "fwd": "graph"}[args.profile_case]
+        z, _, _ = R.layer_forward(x, W, H, driver=drv)
     elif args.profile_case == "naive":
         B, N, d, H, dff = args.pB, args.lb, 1024, 16, 4096
         W = {k: torch.from_numpy(v.astype("float32")).to(dev, torch.bfloat16)

@@ -272,15 +272,6 @@ __device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* src, float (&v)
   }
 }
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4& w, float (&v)[8]) {
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float2 f = __bfloat1622float2(p[k]);
-    v[2 * k] = f.x;
-    v[2 * k + 1] = f.y;
-  }
-}
 
 // Work split: a CTA of 128 threads holds 16 octets. With S = min(16, the
 // power of two >= max(nq, nk)) query slots per (b, h) pair, a CTA serves

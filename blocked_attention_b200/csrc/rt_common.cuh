@@ -137,6 +137,17 @@ __device__ __forceinline__ float gelu_as7126(float y) {
   return 0.5f * y * (1.0f + erf_as7126(y * 0.70710678118654752f));
 }
 
+// eight bf16 (one 16-byte word) to float
+__device__ __forceinline__ void unpack_bf16x8(const uint4& w, float (&v)[8]) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __bfloat1622float2(p[k]);
+    v[2 * k] = f.x;
+    v[2 * k + 1] = f.y;
+  }
+}
+
 // scale of an empty accumulator: exp2(m_old - m_new) with m_old = -inf -> 0
 __device__ __forceinline__ float rescale(float m_old, float m_new) {
   return (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
