@@ -40,7 +40,11 @@ METRIC = "RT-layer prefill tokens/s (B=512,N=2048,d=1024 bf16); % of roofline"
 # dram__bytes_write.sum of one launch), keyed by (kernel class, workload, hash
 # of the CUDA sources at capture time); reported as null once the sources
 # change.
-NCU_TRAFFIC: dict = {}
+NCU_TRAFFIC: dict = {
+    # dram__bytes_read.sum + dram__bytes_write.sum of one W_2 GEMM launch at the
+    # headline shapes (profiles/gemm_w2_B512_d1024_dff4096.md), valid for these sources
+    ("gemm_w2", "headline", "ccaeaeac93bb"): 14721536,
+}
 
 
 def src_hash() -> str:
