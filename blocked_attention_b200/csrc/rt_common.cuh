@@ -200,6 +200,49 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsign
   }
 }
 
+// ---------------------------------------------------------------------------
+// flags in global memory between CTAs of one kernel
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ unsigned ld_volatile_u32(const unsigned* p) {
+  return *reinterpret_cast<const volatile unsigned*>(p);
+}
+// Bounded poll until *f >= target (acquire). Returns at once once the error
+// word is set; a poll that runs out sets RT_DEVERR_TIMEOUT. Either way the
+// caller proceeds.
+// (debug build: a wait that runs out records `id` and `where`, and the value
+// it saw, after the error word)
+static __device__ __noinline__ void poll_ge(const unsigned* f, unsigned target, unsigned* err, unsigned id = 0,
+                                     long long where = 0) {
+  if (ld_acquire_u32(f) >= target) return;
+  const unsigned long long t0 = globaltimer();
+  for (unsigned it = 1;; ++it) {
+    __nanosleep(64);
+    const unsigned v = ld_acquire_u32(f);
+    if (v >= target) return;
+    if ((it & 15u) == 0) {
+      if (err && ld_volatile_u32(err) != 0) return;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        set_error(err, RT_DEVERR_TIMEOUT);
+        timeout_record(err, id, where, ((long long)v << 16) | (target & 0xffff));
+        return;
+      }
+    }
+  }
+}
+
 // Rings consumed by two issuers that take alternate stages: the previous
 // round of a slot may belong to the other issuer, and if that round's copy
 // has not landed yet when this issuer reaches the slot, a parity wait for

@@ -57,6 +57,7 @@
 #pragma once
 
 #include "rt_common.cuh"
+#include "rt_foldunits.cuh"
 #include "rt_gemm_tc.cuh"
 
 namespace rt {
@@ -121,22 +122,6 @@ struct StepsParams {
 // ---------------------------------------------------------------------------
 // synchronisation helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-__device__ __forceinline__ unsigned ld_volatile_u32(const unsigned* p) {
-  return *reinterpret_cast<const volatile unsigned*>(p);
-}
 // generic-proxy global stores <-> async-proxy (TMA) global accesses
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -145,30 +130,6 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // barrier of the four fold warps (named barrier 2, 128 threads)
 __device__ __forceinline__ void fold_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
-
-// Bounded poll until *f >= target (acquire). Returns at once once the error
-// word is set; a poll that runs out sets RT_DEVERR_TIMEOUT. Either way the
-// caller proceeds.
-// (debug build: a wait that runs out records `id` and `where`, and the value
-// it saw, after the error word)
-__device__ __noinline__ void poll_ge(const unsigned* f, unsigned target, unsigned* err, unsigned id = 0,
-                                     long long where = 0) {
-  if (ld_acquire_u32(f) >= target) return;
-  const unsigned long long t0 = globaltimer();
-  for (unsigned it = 1;; ++it) {
-    __nanosleep(64);
-    const unsigned v = ld_acquire_u32(f);
-    if (v >= target) return;
-    if ((it & 15u) == 0) {
-      if (ld_volatile_u32(err) != 0) return;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        set_error(err, RT_DEVERR_TIMEOUT);
-        timeout_record(err, id, where, ((long long)v << 16) | (target & 0xffff));
-        return;
-      }
-    }
-  }
-}
 
 // mbarrier wait bounded by time and abandoned once the error word is set.
 __device__ __forceinline__ bool mbar_wait_g(uint64_t* bar, unsigned parity, unsigned* err, unsigned id = 0,
@@ -315,145 +276,6 @@ __device__ __forceinline__ void slice_flags(const StepsParams& P, int ph, int kk
   }
 }
 
-// ---------------------------------------------------------------------------
-// small block fold (at most 8 keys), one task = one head of up to 32
-// sequences: every (sequence, query) unit is served by an octet of lanes
-// holding 8 of the head's 64 dims; each thread takes R units at a time and
-// issues all their loads before any use. With fin, the first query q0 is
-// finalised (temporary pair merged, a = o / l written, statistics not
-// stored); the other queries' (m, l, o) are updated in place, or written when
-// the fold is the first into them (init).
-// ---------------------------------------------------------------------------
-template <int NK, int R>
-__device__ __forceinline__ void fold_small_units(const StepsParams& P, int q0, int nq, int k0, int init, int h,
-                                                 int s0, int ns, int tid, int fin) {
-  const int B = P.ep.B, H = P.H, d = P.ep.d;
-  const int oct = tid >> 3, sl = tid & 7;
-  const unsigned omask = 0xFFu << ((tid & 31) & 24);
-  const int U = ns * nq;
-  const __nv_bfloat16* K = P.ep.Kout;
-  const __nv_bfloat16* V = P.ep.Vout;
-  for (int u0 = 0; u0 < U; u0 += 16 * R) {
-    uint4 qw[R], kw[R][NK], vw[R][NK], ktw[R], vtw[R];
-    float4 oa[R], ob[R];
-    float mo[R], lo[R];
-    bool live[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int u = u0 + r * 16 + oct;
-      bool act = u < U;
-      const int s = act ? u / nq : 0, qi = act ? u - s * nq : 0;
-      const int b = s0 + s;
-      const size_t row = (size_t)(q0 + qi) * B + b;
-      const __nv_bfloat16* qp = P.qkv + row * (size_t)(3 * d) + h * 64 + sl * 8;
-      qw[r] = ktw[r] = vtw[r] = make_uint4(0, 0, 0, 0);
-      act = act && idx_ok(b < B && q0 + qi < P.ep.Nseq && k0 >= 0 && k0 + NK <= q0 && h < H, P.err);
-      oa[r] = ob[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-      mo[r] = -INFINITY;
-      lo[r] = 0.f;
-#pragma unroll
-      for (int i = 0; i < NK; ++i) kw[r][i] = vw[r][i] = make_uint4(0, 0, 0, 0);
-      live[r] = act;
-      if (act) {
-        // k, v, m, l and o were written by other CTAs of this kernel: loads
-        // through L2 only (no stale L1 lines); q and the temporary pair come
-        // from the projection kernel
-        qw[r] = *reinterpret_cast<const uint4*>(qp);
-#pragma unroll
-        for (int i = 0; i < NK; ++i) {
-          const size_t kv = ((size_t)(k0 + i) * B + b) * d + h * 64 + sl * 8;
-          kw[r][i] = __ldcg(reinterpret_cast<const uint4*>(K + kv));
-          vw[r][i] = __ldcg(reinterpret_cast<const uint4*>(V + kv));
-        }
-        if (fin && qi == 0) {   // the finalised query's temporary pair
-          ktw[r] = *reinterpret_cast<const uint4*>(qp + d);
-          vtw[r] = *reinterpret_cast<const uint4*>(qp + 2 * d);
-        }
-        if (!init) {
-          const float* op = P.o + row * (size_t)d + h * 64 + sl * 8;
-          mo[r] = __ldcg(P.m + row * H + h);
-          lo[r] = __ldcg(P.l + row * H + h);
-          oa[r] = __ldcg(reinterpret_cast<const float4*>(op));
-          ob[r] = __ldcg(reinterpret_cast<const float4*>(op) + 1);
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int u = u0 + r * 16 + oct;
-      if (!live[r]) continue;   // whole octets together; shuffles stay inside the octet
-      const int s = u / nq, qi = u - s * nq;
-      const int b = s0 + s;
-      const size_t row = (size_t)(q0 + qi) * B + b;
-      float q[8];
-      unpack_bf16x8(qw[r], q);
-      float sc[NK];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < NK; ++i) {
-        float kk[8];
-        unpack_bf16x8(kw[r][i], kk);
-        float dot = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) dot += q[e] * kk[e];
-        dot += __shfl_xor_sync(omask, dot, 1);
-        dot += __shfl_xor_sync(omask, dot, 2);
-        dot += __shfl_xor_sync(omask, dot, 4);
-        sc[i] = dot * P.sc2;
-        mx = fmaxf(mx, sc[i]);
-      }
-      float oo[8] = {oa[r].x, oa[r].y, oa[r].z, oa[r].w, ob[r].x, ob[r].y, ob[r].z, ob[r].w};
-      const float mn = fmaxf(mo[r], mx);
-      const float al = rescale(mo[r], mn);
-      float ln = lo[r] * al;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) oo[e] *= al;
-#pragma unroll
-      for (int i = 0; i < NK; ++i) {
-        const float p = exp2f(sc[i] - mn);
-        float vv[8];
-        unpack_bf16x8(vw[r][i], vv);
-        ln += p;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) oo[e] += p * vv[e];
-      }
-      if (fin && qi == 0) {
-        float kt[8];
-        unpack_bf16x8(ktw[r], kt);
-        float dot = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) dot += q[e] * kt[e];
-        dot += __shfl_xor_sync(omask, dot, 1);
-        dot += __shfl_xor_sync(omask, dot, 2);
-        dot += __shfl_xor_sync(omask, dot, 4);
-        const float st = dot * P.sc2;
-        const float m2 = fmaxf(mn, st);
-        const float a2 = rescale(mn, m2), pt = exp2f(st - m2);
-        const float inv = 1.f / (ln * a2 + pt);
-        float vt[8];
-        unpack_bf16x8(vtw[r], vt);
-        uint4 w;
-        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          __nv_bfloat162 v2 = __floats2bfloat162_rn((oo[2 * k] * a2 + pt * vt[2 * k]) * inv,
-                                                    (oo[2 * k + 1] * a2 + pt * vt[2 * k + 1]) * inv);
-          wp[k] = *reinterpret_cast<uint32_t*>(&v2);
-        }
-        if (idx_ok(b < B && h < H, P.err, 16, b, h))
-          *reinterpret_cast<uint4*>(P.a16 + (size_t)b * d + h * 64 + sl * 8) = w;
-      } else {
-        float* op = P.o + row * (size_t)d + h * 64 + sl * 8;
-        if (sl == 0) {
-          P.m[row * H + h] = mn;
-          P.l[row * H + h] = ln;
-        }
-        reinterpret_cast<float4*>(op)[0] = make_float4(oo[0], oo[1], oo[2], oo[3]);
-        reinterpret_cast<float4*>(op)[1] = make_float4(oo[4], oo[5], oo[6], oo[7]);
-      }
-    }
-  }
-}
 
 // ---------------------------------------------------------------------------
 // epilogue of one GEMM tile (split == whole K): 32 columns at a time, the sum
@@ -903,6 +725,10 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
   } else {
     // ---------------- fold warps: the small folds (FOLD and DEFER tasks) ----------------
     const int ftid = threadIdx.x - 224;   // 0..127
+    FoldUnitArgs fa;
+    fa.B = P.ep.B; fa.H = P.H; fa.d = P.ep.d; fa.Nseq = P.ep.Nseq;
+    fa.K = P.ep.Kout; fa.V = P.ep.Vout; fa.qkv = P.qkv;
+    fa.m = P.m; fa.l = P.l; fa.o = P.o; fa.a16 = P.a16; fa.sc2 = P.sc2; fa.err = P.err;
     for_my_tasks(P, [&](int ph, int j, int loc, int gi) -> bool {
       if (ph < PH_FOLD) return true;
       if (ftid == 0) note_progress(P, 4, ph, j, loc);
@@ -931,16 +757,16 @@ __global__ void __launch_bounds__(StepsCfg::THREADS, 1) k_steps(const __grid_con
       const int init = t == lb ? 1 : 0;
       if (ns > 0 && urgent && nq > 0) {
         switch (lb) {
-          case 1: fold_small_units<1, 2>(P, t, 1, t - 1, init, h, s0, ns, ftid, 1); break;
-          case 2: fold_small_units<2, 2>(P, t, 1, t - 2, init, h, s0, ns, ftid, 1); break;
-          case 4: fold_small_units<4, 2>(P, t, 1, t - 4, init, h, s0, ns, ftid, 1); break;
-          default: fold_small_units<8, 1>(P, t, 1, t - 8, init, h, s0, ns, ftid, 1); break;
+          case 1: fold_units<1, 2>(fa, t, 1, t - 1, init, h, s0, ns, ftid, 1); break;
+          case 2: fold_units<2, 2>(fa, t, 1, t - 2, init, h, s0, ns, ftid, 1); break;
+          case 4: fold_units<4, 2>(fa, t, 1, t - 4, init, h, s0, ns, ftid, 1); break;
+          default: fold_units<8, 1>(fa, t, 1, t - 8, init, h, s0, ns, ftid, 1); break;
         }
       } else if (ns > 0 && !urgent && nq > 1) {
         switch (lb) {
-          case 2: fold_small_units<2, 2>(P, t + 1, nq - 1, t - 2, init, h, s0, ns, ftid, 0); break;
-          case 4: fold_small_units<4, 2>(P, t + 1, nq - 1, t - 4, init, h, s0, ns, ftid, 0); break;
-          default: fold_small_units<8, 1>(P, t + 1, nq - 1, t - 8, init, h, s0, ns, ftid, 0); break;
+          case 2: fold_units<2, 2>(fa, t + 1, nq - 1, t - 2, init, h, s0, ns, ftid, 0); break;
+          case 4: fold_units<4, 2>(fa, t + 1, nq - 1, t - 4, init, h, s0, ns, ftid, 0); break;
+          default: fold_units<8, 1>(fa, t + 1, nq - 1, t - 8, init, h, s0, ns, ftid, 0); break;
         }
       }
       if (ftid == 0) trace_ev(P, gi, 10);
