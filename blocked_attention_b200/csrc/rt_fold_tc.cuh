@@ -385,14 +385,21 @@ __global__ void __launch_bounds__(192, 1)
 // tile of 256 queries (tile A = queries 0..127, tile B = 128..255 of it), so
 // every K/V chunk feeds two 128-query tiles. 320 threads:
 //   warp 0 : TMA producer (Q of both tiles per item; K/V ring)
-//   warp 1 : MMA issuer, ping-pong order S_A(0) S_B(0) | PV_A(g) S_A(g+1)
-//            PV_B(g) S_B(g+1) | ..., so each tile's softmax overlaps the
-//            other tile's tensor-core work
-//   warps 2..5 (tile A), 6..9 (tile B): softmax, accumulate, merge
-// P is double-buffered per tile, so the softmax of chunk g + 1 runs while
-// the PV product of chunk g still reads P(g). Q is single-buffered: the
-// producer reloads it once the item's last S products have completed.
-// TMEM: S_A 0..127, S_B 128..255, O_A[2] 256/320, O_B[2] 384/448.
+//   warp 1 : MMA issuer, order S_A(0) S_B(0) | S_A(g+1) PV_A(g) S_B(g+1)
+//            PV_B(g) | ...: the next chunk's scores go ahead of this chunk's
+//            PV product, since the softmax frees S as soon as it has read it
+//   warps 2..5 (tile A), 6..9 (tile B): softmax and merge
+// Per chunk a softmax thread (one query row) reads its 128 scores from tensor
+// memory once and releases S; exponentials are taken against a reference
+// maximum that moves only when a chunk's maximum exceeds it by more than 8
+// (in log2 units; p <= 2^8 is exact enough in bf16), and only then are O and
+// l rescaled (O read, scaled and written back in tensor memory once the
+// previous PV product has completed). O accumulates over an item's chunks in
+// tensor memory (the first chunk's PV overwrites it) and is read once, at the
+// item's end, for the merge. P is double-buffered per tile in shared memory.
+// Q is single-buffered: the producer reloads it once the item's last S
+// products have completed.
+// TMEM: S_A 0..127, S_B 128..255, O_A 256..319, O_B 320..383.
 // ---------------------------------------------------------------------------
 // q . k over d_h = 64 bf16 elements (one thread; kept out of line so that the
 // finalising row's dot product adds no registers to the softmax loop)
@@ -439,8 +446,7 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* s_free = bars + 10;     // [tile]
   uint64_t* p_full = bars + 12;     // [tile][2]
   uint64_t* p_free = bars + 16;     // [tile][2]
-  uint64_t* o_full = bars + 20;     // [tile][2]
-  uint64_t* o_free = bars + 24;     // [tile][2]
+  uint64_t* o_done = bars + 20;     // [tile]: a PV product has completed (one phase per chunk)
   uint64_t* mma_done = bars + 28;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 29);
 
@@ -469,9 +475,9 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < 4; ++i) {
       mbar_init(&p_full[i], 4);
       mbar_init(&p_free[i], 1);
-      mbar_init(&o_full[i], 1);
-      mbar_init(&o_free[i], 4);
     }
+    mbar_init(&o_done[0], 1);
+    mbar_init(&o_done[1], 1);
     for (int i = 0; i < C::KVS; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
@@ -544,31 +550,30 @@ __global__ void __launch_bounds__(320, 1)
       };
       auto issue_pv = [&](int g, int t) -> bool {
         const int li = g / nch, c = g - li * nch;
-        const int st = g % C::KVS, ob = g & 1;
-        if (!mbar_wait(&p_full[t * 2 + ob], (g >> 1) & 1u, err) ||
-            !mbar_wait(&o_free[t * 2 + ob], ((g >> 1) & 1u) ^ 1u, err))
-          return false;
+        const int st = g % C::KVS, pb = g & 1;
+        if (!mbar_wait(&p_full[t * 2 + pb], (g >> 1) & 1u, err)) return false;
         tc_fence_after();
-        const uint8_t* pt = smem + C::OFF_P + (t * 2 + ob) * C::P_BYTES;
+        const uint8_t* pt = smem + C::OFF_P + (t * 2 + pb) * C::P_BYTES;
         const uint8_t* vt = smem + C::OFF_V + st * C::KV_BYTES;
+        // O accumulates over the item's chunks; its first chunk overwrites it
 #pragma unroll
         for (int ks = 0; ks < C::KC / 16; ++ks)
-          tc_mma_f16(tmem_base + 256 + t * 128 + ob * 64, smem_desc_sw128(pt + (ks >> 2) * 16384 + (ks & 3) * 32),
-                     smem_desc_sw128_mn(vt + ks * 16 * 128), idesc_o, ks != 0 ? 1u : 0u);
-        tc_commit(&o_full[t * 2 + ob]);
-        tc_commit(&p_free[t * 2 + ob]);
+          tc_mma_f16(tmem_base + 256 + t * 64, smem_desc_sw128(pt + (ks >> 2) * 16384 + (ks & 3) * 32),
+                     smem_desc_sw128_mn(vt + ks * 16 * 128), idesc_o, (ks != 0 || c != 0) ? 1u : 0u);
+        tc_commit(&o_done[t]);
+        tc_commit(&p_free[t * 2 + pb]);
         if (t == 1) tc_commit(&kv_empty[st]);
         (void)li;
-        (void)c;
         return true;
       };
       bool ok = true;
       if (total > 0) ok = issue_s(0, 0) && issue_s(0, 1);
+      // the next chunk's S products go ahead of this chunk's PV products
       for (int g = 0; g < total && ok; ++g) {
-        ok = issue_pv(g, 0);
-        if (ok && g + 1 < total) ok = issue_s(g + 1, 0);
-        if (ok) ok = issue_pv(g, 1);
+        if (g + 1 < total) ok = issue_s(g + 1, 0);
+        if (ok) ok = issue_pv(g, 0);
         if (ok && g + 1 < total) ok = issue_s(g + 1, 1);
+        if (ok) ok = issue_pv(g, 1);
       }
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, err);
@@ -582,33 +587,16 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t* const sP = smem + C::OFF_P + t * 2 * C::P_BYTES + r * 128;   // this row in P buffer 0
     uint64_t* const pfull = p_full + t * 2;
     uint64_t* const pfree = p_free + t * 2;
-    float m_run = -INFINITY, l_run = 0.f, alpha_prev = 0.f;
-    float oacc[64];
+    float m_ref = -INFINITY, m_true = -INFINITY, l_run = 0.f;   // reference and true row maximum
     bool ok = true;
+    const uint32_t obase = tmem_base + lane_base + 256 + t * 64;   // this row's O
 
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
       int v = 1;
       if (lane == 0) v = mbar_wait(bar, parity, err) ? 1 : 0;
       return __shfl_sync(0xffffffffu, v, 0) != 0;
     };
-    auto accumulate = [&](int g, float alpha) -> bool {
-      const int ob = g & 1;
-      if (!wait_warp(&o_full[t * 2 + ob], (g >> 1) & 1u)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t rv[32];
-        tmem_ld_32x32b_x32(tmem_base + lane_base + 256 + t * 128 + ob * 64 + half * 32, rv);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) oacc[half * 32 + i] = oacc[half * 32 + i] * alpha + __uint_as_float(rv[i]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_free[t * 2 + ob]);
-      return true;
-    };
-    auto merge = [&](int li) {
+    auto merge = [&](int li, const float (&oacc)[64]) {
       int b, h, st0;
       item_of(li, b, h, st0);
       const int qt0 = st0 + t * C::QT;
@@ -618,8 +606,8 @@ __global__ void __launch_bounds__(320, 1)
         float mg = -INFINITY, lg = 0.f;
         float* op = o + row * (size_t)d + h * C::DH;
         if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }
-        const float mn = fmaxf(mg, m_run);
-        const float ag = rescale(mg, mn), ab = rescale(m_run, mn);
+        const float mn = fmaxf(mg, m_ref);
+        const float ag = rescale(mg, mn), ab = rescale(m_ref, mn);
         const float ln = lg * ag + l_run * ab;
         if (fin && qt0 == q0 && r == 0) {
           const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * C::DH;   // q, then k_tmp at +d, v_tmp at +2d
@@ -658,47 +646,52 @@ __global__ void __launch_bounds__(320, 1)
 
     for (int g = 0; g < total && ok; ++g) {
       const int li = g / nch, c = g - li * nch;
-      if (c == 0) {
-        if (g > 0) {
-          if (!accumulate(g - 1, alpha_prev)) { ok = false; break; }
-          merge(li - 1);
-        }
-        m_run = -INFINITY;
-        l_run = 0.f;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) oacc[i] = 0.f;
-      }
       if (!wait_warp(&s_full[t], g & 1u)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t sbase = tmem_base + lane_base + t * 128;
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t rv[32];
-        tmem_ld_32x32b_x32(sbase + cc * 32, rv);
-        tmem_ld_wait();
+      // the row's 128 scores, read once; S is then free for the next chunk
+      uint32_t sv[4][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(rv[i]));
+      for (int cc = 0; cc < 4; ++cc) tmem_ld_32x32b_x32(tmem_base + lane_base + t * 128 + cc * 32, sv[cc]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[t]);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
+      mx *= sc2;
+      // The reference moves only when a row's chunk maximum passes it by
+      // more than 8; then O and l are rescaled, warp-wide (the warp's rows
+      // share the tensor-memory access) and after this chunk's exponentials,
+      // before its PV product may start.
+      float alpha = 1.f;
+      bool rescale_o = false;
+      if (c == 0) {
+        m_ref = mx;   // a new item: O is overwritten by this chunk's PV product
+        m_true = mx;
+        l_run = 0.f;
+      } else if (__any_sync(0xffffffffu, mx > m_ref + 8.f)) {
+        const float m_new = fmaxf(m_ref, mx);
+        alpha = rescale(m_ref, m_new);
+        m_ref = m_new;
+        rescale_o = true;
       }
-      const float m_new = fmaxf(m_run, mx * sc2);
-      const float alpha = rescale(m_run, m_new);
       // P buffer g % 2 must have been consumed by the PV product of chunk g - 2
       const int pb = g & 1;
       if (!wait_warp(pfree + pb, ((g >> 1) & 1u) ^ 1u)) { ok = false; break; }
       float lsum = 0.f;
       uint8_t* prow = sP + (pb ? C::P_BYTES : 0u);
-#pragma unroll 1
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t rv[32];
-        tmem_ld_32x32b_x32(sbase + cc * 32, rv);
-        tmem_ld_wait();
         uint8_t* atom = prow + (cc >> 1) * 16384;
 #pragma unroll
         for (int gq = 0; gq < 4; ++gq) {
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            p[e] = exp2f(__uint_as_float(rv[gq * 8 + e]) * sc2 - m_new);
+            p[e] = exp2f(__uint_as_float(sv[cc][gq * 8 + e]) * sc2 - m_ref);
             lsum += p[e];
           }
           uint4 w;
@@ -710,19 +703,52 @@ __global__ void __launch_bounds__(320, 1)
           *reinterpret_cast<uint4*>(atom + ((chunk ^ (r & 7)) << 4)) = w;
         }
       }
+      if (rescale_o) {
+        // O of chunks up to g - 1: its last PV product must have completed
+        if (!wait_warp(&o_done[t], (uint32_t)(g - 1) & 1u)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t ov[32];
+          tmem_ld_32x32b_x32(obase + half * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st_32x32b_x32(obase + half * 32, ov);
+        }
+        tmem_st_wait();
+      }
       l_run = l_run * alpha + lsum;
-      m_run = m_new;
+      m_true = fmaxf(m_true, mx);
       tc_fence_before();
       fence_async_shared();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&s_free[t]);
-        mbar_arrive(pfull + pb);
+      if (lane == 0) mbar_arrive(pfull + pb);
+      if (c == nch - 1) {
+        // the item's last chunk: O is final once its PV product completes
+        if (!wait_warp(&o_done[t], (uint32_t)g & 1u)) { ok = false; break; }
+        tc_fence_after();
+        float oacc[64];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t ov[32];
+          tmem_ld_32x32b_x32(obase + half * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) oacc[half * 32 + i] = __uint_as_float(ov[i]);
+        }
+        tc_fence_before();
+        // the statistics in canonical form: relative to the true maximum
+        if (m_true > m_ref) {
+          const float af = rescale(m_ref, m_true);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) oacc[i] *= af;
+          l_run *= af;
+          m_ref = m_true;
+        }
+        merge(li, oacc);
       }
-      if (c > 0 && !accumulate(g - 1, alpha_prev)) { ok = false; break; }
-      alpha_prev = alpha;
     }
-    if (ok && total > 0 && accumulate(total - 1, alpha_prev)) merge(my_items - 1);
   }
   __syncthreads();
   if (warp == 1) {
