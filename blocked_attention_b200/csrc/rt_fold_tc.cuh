@@ -656,11 +656,17 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[t]);
-      float mx = -INFINITY;
+      // row maximum and, below, row sum in 8 independent partials (a single
+      // running value would chain 128 dependent operations per chunk)
+      float mxp[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
+        for (int i = 0; i < 32; ++i) mxp[i & 7] = fmaxf(mxp[i & 7], __uint_as_float(sv[cc][i]));
+      float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                       fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
       mx *= sc2;
       // The reference moves only when a row's chunk maximum passes it by
       // more than 8; then O and l are rescaled, warp-wide (the warp's rows
@@ -681,7 +687,9 @@ __global__ void __launch_bounds__(320, 1)
       // P buffer g % 2 must have been consumed by the PV product of chunk g - 2
       const int pb = g & 1;
       if (!wait_warp(pfree + pb, ((g >> 1) & 1u) ^ 1u)) { ok = false; break; }
-      float lsum = 0.f;
+      float lsp[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lsp[e] = 0.f;
       uint8_t* prow = sP + (pb ? C::P_BYTES : 0u);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -692,7 +700,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             p[e] = exp2f(__uint_as_float(sv[cc][gq * 8 + e]) * sc2 - m_ref);
-            lsum += p[e];
+            lsp[e] += p[e];
           }
           uint4 w;
           w.x = pack_bf16x2(p[0], p[1]);
@@ -703,6 +711,7 @@ __global__ void __launch_bounds__(320, 1)
           *reinterpret_cast<uint4*>(atom + ((chunk ^ (r & 7)) << 4)) = w;
         }
       }
+      const float lsum = ((lsp[0] + lsp[1]) + (lsp[2] + lsp[3])) + ((lsp[4] + lsp[5]) + (lsp[6] + lsp[7]));
       if (rescale_o) {
         // O of chunks up to g - 1: its last PV product must have completed
         if (!wait_warp(&o_done[t], (uint32_t)(g - 1) & 1u)) { ok = false; break; }
