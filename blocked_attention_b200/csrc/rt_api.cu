@@ -530,18 +530,19 @@ static cudaError_t launch_fold(const T* Q, int q_stride, const T* K, const T* V,
     }
     if (fast && dh == 64 && nk >= 16 && nk % 16 == 0) {
       // pack 4 / 2 (b, h) pairs per CTA for 16- / 32-key blocks so that no warp idles
+      // blocks of 16 or 32 keys are one chunk: the single-buffered variant (5 CTAs per SM)
       if (nk <= 16) {
         dim3 grid((nq + 15) / 16, (pairs + 3) / 4);
-        return launch_pdl(k_fold_mma<4>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B,
-                          H, q0, nq, k0, nk, sc2, init, fin, err);
+        return launch_pdl(k_fold_mma<4, 1>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out,
+                          B, H, q0, nq, k0, nk, sc2, init, fin, err);
       }
       if (nk <= 32) {
         dim3 grid((nq + 31) / 32, (pairs + 1) / 2);
-        return launch_pdl(k_fold_mma<2>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B,
-                          H, q0, nq, k0, nk, sc2, init, fin, err);
+        return launch_pdl(k_fold_mma<2, 1>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out,
+                          B, H, q0, nq, k0, nk, sc2, init, fin, err);
       }
       dim3 grid((nq + 63) / 64, pairs);
-      return launch_pdl(k_fold_mma<1>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B, H,
+      return launch_pdl(k_fold_mma<1, 2>, grid, dim3(128), 0, st, Q, q_stride, K, V, kv_stride, m, l, o, a_out, B, H,
                         q0, nq, k0, nk, sc2, init, fin, err);
     }
     if (fast && dh == 64 && nk <= 8 && q_stride % 8 == 0 && kv_stride % 8 == 0) {

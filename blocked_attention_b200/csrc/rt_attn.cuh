@@ -656,8 +656,11 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 // P (b, h) pairs per CTA: P = 1 for blocks >= 64 keys (64 queries of one pair,
 // keys in 64-key chunks); P = 2 / 4 for 32- / 16-key blocks (64/P queries and
 // the 64/P keys of each pair share one 64-row tile), so no warp idles.
-template <int P>
-__global__ void __launch_bounds__(128)
+// NB = K/V chunk buffers: 2 (double-buffered chunks) for blocks of more than
+// one chunk, 1 for blocks of one chunk (16 keys at P = 4, 32 at P = 2), whose
+// smaller footprint (and register bound) lets 5 CTAs share an SM instead of 4.
+template <int P, int NB = 2>
+__global__ void __launch_bounds__(128, NB == 1 ? 5 : 4)
     k_fold_mma(const __nv_bfloat16* __restrict__ Q, int q_stride, const __nv_bfloat16* __restrict__ K,
                const __nv_bfloat16* __restrict__ V, int kv_stride, float* __restrict__ m,
                float* __restrict__ l, float* __restrict__ o, __nv_bfloat16* __restrict__ a_out, int B, int H,
@@ -665,10 +668,14 @@ __global__ void __launch_bounds__(128)
   using namespace mma_detail;
   constexpr int DH = 64, QT = 64, KC = 64, QTP = QT / P, KCP = KC / P;
   __shared__ __align__(128) __nv_bfloat16 sQ[QT * LDS];
-  __shared__ __align__(128) __nv_bfloat16 sK[2][KC * LDS];
-  __shared__ __align__(128) __nv_bfloat16 sV[2][KC * LDS];
+  __shared__ __align__(128) __nv_bfloat16 sK[NB][KC * LDS];
+  __shared__ __align__(128) __nv_bfloat16 sV[NB][KC * LDS];
   pdl_launch_dependents();
   pdl_wait();
+  if (NB == 1 && nk > KCP) {             // one buffer holds one chunk only
+    if (threadIdx.x == 0) set_error(err, RT_DEVERR_INDEX);
+    return;
+  }
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int npairs = B * H;
@@ -719,9 +726,9 @@ __global__ void __launch_bounds__(128)
   uint32_t qf[4][4];
 
   for (int ci = 0; ci < nchunks; ++ci) {
-    const int buf = ci & 1;
+    const int buf = NB == 2 ? (ci & 1) : 0;
     if (ci + 1 < nchunks) {
-      load_kv(buf ^ 1, (ci + 1) * KCP, min(KCP, nk - (ci + 1) * KCP));
+      load_kv(NB == 2 ? buf ^ 1 : 0, (ci + 1) * KCP, min(KCP, nk - (ci + 1) * KCP));
       cp_async_commit();
       cp_async_wait<1>();
     } else {
