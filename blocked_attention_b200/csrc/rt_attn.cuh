@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
   for (int i = 0; i < KMAX; ++i) {
     if (i < n) {
-      const float p = exp2f(s[i] - mn);
+      const float p = ex2_ftz(s[i] - mn);
       float vv[8];
       unpack_bf16x8(STAGED ? sv[i * 8] : v1w, vv);
       lo += p;
@@ -789,10 +789,10 @@ __global__ void __launch_bounds__(128, NB == 1 ? 5 : 4)
           float p[2][4];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            p[u][0] = exp2f(sacc[2 * kj + u][0] - mrow[0]);
-            p[u][1] = exp2f(sacc[2 * kj + u][1] - mrow[0]);
-            p[u][2] = exp2f(sacc[2 * kj + u][2] - mrow[1]);
-            p[u][3] = exp2f(sacc[2 * kj + u][3] - mrow[1]);
+            p[u][0] = ex2_ftz(sacc[2 * kj + u][0] - mrow[0]);
+            p[u][1] = ex2_ftz(sacc[2 * kj + u][1] - mrow[0]);
+            p[u][2] = ex2_ftz(sacc[2 * kj + u][2] - mrow[1]);
+            p[u][3] = ex2_ftz(sacc[2 * kj + u][3] - mrow[1]);
             lrow[0] += p[u][0] + p[u][1];
             lrow[1] += p[u][2] + p[u][3];
           }

@@ -148,6 +148,15 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& w, float (&v)[8]) {
   }
 }
 
+// 2^x on the special-function unit, results below 2^-126 flushed to zero
+// (ex2(-inf) = +0). For softmax weights of bf16 folds: a weight that small
+// is negligible against the row's largest (>= 2^-8 of the reference).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // scale of an empty accumulator: exp2(m_old - m_new) with m_old = -inf -> 0
 __device__ __forceinline__ float rescale(float m_old, float m_new) {
   return (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);

@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(192, 1)
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            p[e] = exp2f(__uint_as_float(rv[gq * 8 + e]) * sc2 - m_new);
+            p[e] = ex2_ftz(__uint_as_float(rv[gq * 8 + e]) * sc2 - m_new);
             lsum += p[e];
           }
           uint4 w;
@@ -568,8 +568,15 @@ __global__ void __launch_bounds__(320, 1)
       };
       bool ok = true;
       if (total > 0) ok = issue_s(0, 0) && issue_s(0, 1);
-      // the next chunk's S products go ahead of this chunk's PV products
+      // Within an item the next chunk's S products go ahead of this chunk's
+      // PV products. At an item's last chunk the PV products go first: the
+      // next item's S products wait for its Q tiles, and the merge must not.
       for (int g = 0; g < total && ok; ++g) {
+        if ((g + 1) % nch == 0) {
+          ok = issue_pv(g, 0) && issue_pv(g, 1);
+          if (ok && g + 1 < total) ok = issue_s(g + 1, 0) && issue_s(g + 1, 1);
+          continue;
+        }
         if (g + 1 < total) ok = issue_s(g + 1, 0);
         if (ok) ok = issue_pv(g, 0);
         if (ok && g + 1 < total) ok = issue_s(g + 1, 1);
@@ -596,52 +603,115 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) v = mbar_wait(bar, parity, err) ? 1 : 0;
       return __shfl_sync(0xffffffffu, v, 0) != 0;
     };
-    auto merge = [&](int li, const float (&oacc)[64]) {
-      int b, h, st0;
-      item_of(li, b, h, st0);
-      const int qt0 = st0 + t * C::QT;
-      const int nrows = min(C::QT, q0 + nq - qt0);   // may be <= 0 for an empty tile B
-      if (r < nrows && idx_ok(qt0 + r >= q0 && qt0 + r < q0 + nq && b < B && h < H, err)) {
-        const size_t row = (size_t)(qt0 + r) * B + b;
-        float mg = -INFINITY, lg = 0.f;
-        float* op = o + row * (size_t)d + h * C::DH;
-        if (!init) { mg = m[row * H + h]; lg = l[row * H + h]; }
-        const float mn = fmaxf(mg, m_ref);
-        const float ag = rescale(mg, mn), ab = rescale(m_ref, mn);
-        const float ln = lg * ag + l_run * ab;
-        if (fin && qt0 == q0 && r == 0) {
-          const __nv_bfloat16* tp = Q + row * (size_t)q_stride + h * C::DH;   // q, then k_tmp at +d, v_tmp at +2d
-          const float dot = dot64_bf16(tp, tp + d);
-          const float s2 = dot * sc2;
-          const float m2 = fmaxf(mn, s2);
-          const float a2 = rescale(mn, m2), pt = exp2f(s2 - m2);
-          const float inv = 1.f / (ln * a2 + pt);
-          __nv_bfloat16* ap = a_out + (size_t)b * d + h * C::DH;
+    // The merge runs warp-wide on coalesced rows: lane i owns columns 2i, 2i+1
+    // of each of the warp's 32 rows, so a row's 256 bytes of o move in one
+    // access. The running o of item li is loaded that way before the item's
+    // last PV product completes (its latency overlaps it); the block's
+    // result leaves tensor memory one row per thread and is transposed
+    // through this warp's own 4 KB slices of the tile's P buffer 0 (rows
+    // 32qq..32qq+31 of both key halves: columns 0-31 and 32-63, 128 bytes a
+    // row, 16-byte chunks XOR-swizzled by row). Both P buffers are idle from
+    // the item's last PV product until this warp writes its next P rows.
+    uint8_t* const stg = smem + C::OFF_P + t * 2 * C::P_BYTES + qq * 4096;
+    constexpr int NPRE = 12;   // rows of the running o loaded ahead (registers allow no more)
+    struct RowPos { int b, h, qt0, nrows; };
+    auto pos_of = [&](int li) {
+      RowPos p;
+      int st0;
+      item_of(li, p.b, p.h, st0);
+      p.qt0 = st0 + t * C::QT;
+      p.nrows = min(C::QT, q0 + nq - p.qt0);   // may be <= 0 for an empty tile B
+      return p;
+    };
+    auto load_prev = [&](const RowPos& p, float2 (&prev)[NPRE], float& mg, float& lg) {
+      mg = -INFINITY;
+      lg = 0.f;
+      if (!init && r < p.nrows) {   // this thread's row: its running maximum and sum
+        const size_t row = (size_t)(p.qt0 + r) * B + p.b;
+        mg = m[row * H + p.h];
+        lg = l[row * H + p.h];
+      }
+      const float* const o_w = o + ((size_t)(p.qt0 + qq * 32) * B + p.b) * d + p.h * C::DH + 2 * lane;
 #pragma unroll
-          for (int e = 0; e < C::DH; e += 2) {
-            float og0 = 0.f, og1 = 0.f;
-            if (!init) { og0 = op[e]; og1 = op[e + 1]; }
-            const float o0 = og0 * ag + oacc[e] * ab, o1 = og1 * ag + oacc[e + 1] * ab;
-            const float2 vt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tp + 2 * d + e));
-            *reinterpret_cast<__nv_bfloat162*>(ap + e) =
-                __floats2bfloat162_rn((o0 * a2 + pt * vt.x) * inv, (o1 * a2 + pt * vt.y) * inv);
-          }
-        } else {
-          m[row * H + h] = mn;
-          l[row * H + h] = ln;
+      for (int k = 0; k < NPRE; ++k) {
+        prev[k] = make_float2(0.f, 0.f);
+        if (!init && qq * 32 + k < p.nrows) prev[k] = *reinterpret_cast<const float2*>(o_w + k * (size_t)B * d);
+      }
+    };
+    // af: the factor that takes O from the lazy reference to the true maximum
+    auto merge = [&](const RowPos& p, float af, const float2 (&prev)[NPRE], float mg, float lg) {
+      const bool valid =
+          r < p.nrows && idx_ok(p.qt0 + r >= q0 && p.qt0 + r < q0 + nq && p.b < B && p.h < H, err);
+      const size_t row = (size_t)(p.qt0 + r) * B + p.b;
+      const float mn = fmaxf(mg, m_ref);
+      const float ag = rescale(mg, mn), ab = rescale(m_ref, mn);
+      const float abo = ab * af;   // on O, still relative to the lazy reference
+      const float ln = lg * ag + l_run * ab;
+      const bool fin_row = fin && p.qt0 == q0 && r == 0;   // lane 0 of warp 0 of the first tile
+      // finalisation of query q0 with its own temporary pair (q . k_tmp)
+      float a2 = 0.f, pt = 0.f, inv = 0.f;
+      if (fin_row && valid) {
+        const __nv_bfloat16* tp = Q + row * (size_t)q_stride + p.h * C::DH;   // q, k_tmp at +d
+        const float s2 = dot64_bf16(tp, tp + d) * sc2;
+        const float m2 = fmaxf(mn, s2);
+        a2 = rescale(mn, m2);
+        pt = exp2f(s2 - m2);
+        inv = 1.f / (ln * a2 + pt);
+      } else if (valid) {
+        m[row * H + p.h] = mn;
+        l[row * H + p.h] = ln;
+      }
+      // this row's new-block part, abo * O, from tensor memory into the staging slices
 #pragma unroll
-          for (int e = 0; e < C::DH; e += 4) {
-            float4 og = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (!init) og = *reinterpret_cast<const float4*>(op + e);
-            og.x = og.x * ag + oacc[e] * ab;
-            og.y = og.y * ag + oacc[e + 1] * ab;
-            og.z = og.z * ag + oacc[e + 2] * ab;
-            og.w = og.w * ag + oacc[e + 3] * ab;
-            *reinterpret_cast<float4*>(op + e) = og;
-          }
+      for (int half = 0; half < 2; ++half) {
+        uint32_t ov[32];
+        tmem_ld_32x32b_x32(obase + half * 32, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = half * 8 + jj;
+          const float4 v = make_float4(__uint_as_float(ov[4 * jj]) * abo, __uint_as_float(ov[4 * jj + 1]) * abo,
+                                       __uint_as_float(ov[4 * jj + 2]) * abo, __uint_as_float(ov[4 * jj + 3]) * abo);
+          *reinterpret_cast<float4*>(stg + half * 16384 + lane * 128 + (((j & 7) ^ (lane & 7)) << 4)) = v;
         }
       }
-      __syncwarp();   // reconverge the warp after the row-dependent branch
+      tc_fence_before();
+      __syncwarp();
+      const bool fin_warp = fin && p.qt0 == q0 && qq == 0;
+      a2 = __shfl_sync(0xffffffffu, a2, 0);
+      pt = __shfl_sync(0xffffffffu, pt, 0);
+      inv = __shfl_sync(0xffffffffu, inv, 0);
+      const uint32_t rd = (uint32_t)(lane >> 4) * 16384u + (uint32_t)(lane & 1) * 8u;
+      const size_t ostep = (size_t)B * d;   // floats from one query row of o to the next
+      float* const o_w = o + ((size_t)(p.qt0 + qq * 32) * B + p.b) * d + p.h * C::DH + 2 * lane;
+      const int nk_rows = min(32, p.nrows - qq * 32);   // rows of this warp in the block (warp-uniform)
+      auto put_row = [&](int k, float2 pk) {
+        const float agk = __shfl_sync(0xffffffffu, ag, k);
+        const float2 nb = *reinterpret_cast<const float2*>(stg + rd + k * 128 + ((((lane & 15) >> 1) ^ (k & 7)) << 4));
+        const float o0 = pk.x * agk + nb.x, o1 = pk.y * agk + nb.y;
+        if (fin_warp && k == 0) {
+          const __nv_bfloat16* vt_p = Q + ((size_t)p.qt0 * B + p.b) * q_stride + 2 * d + p.h * C::DH + 2 * lane;
+          const float2 vt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vt_p));
+          *reinterpret_cast<__nv_bfloat162*>(a_out + (size_t)p.b * d + p.h * C::DH + 2 * lane) =
+              __floats2bfloat162_rn((o0 * a2 + pt * vt.x) * inv, (o1 * a2 + pt * vt.y) * inv);
+        } else {
+          *reinterpret_cast<float2*>(o_w + k * ostep) = make_float2(o0, o1);
+        }
+      };
+      // the other rows' running o, all in flight together
+      float2 rest[32 - NPRE];
+#pragma unroll
+      for (int k = NPRE; k < 32; ++k) {
+        rest[k - NPRE] = make_float2(0.f, 0.f);
+        if (!init && k < nk_rows) rest[k - NPRE] = *reinterpret_cast<const float2*>(o_w + k * ostep);
+      }
+#pragma unroll
+      for (int k = 0; k < NPRE; ++k)
+        if (k < nk_rows) put_row(k, prev[k]);
+#pragma unroll
+      for (int k = NPRE; k < 32; ++k)
+        if (k < nk_rows) put_row(k, rest[k - NPRE]);
+      __syncwarp();   // the staging slices are rewritten by this warp's next P rows
     };
 
     for (int g = 0; g < total && ok; ++g) {
@@ -699,7 +769,7 @@ __global__ void __launch_bounds__(320, 1)
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            p[e] = exp2f(__uint_as_float(sv[cc][gq * 8 + e]) * sc2 - m_ref);
+            p[e] = ex2_ftz(__uint_as_float(sv[cc][gq * 8 + e]) * sc2 - m_ref);
             lsp[e] += p[e];
           }
           uint4 w;
@@ -735,27 +805,20 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) mbar_arrive(pfull + pb);
       if (c == nch - 1) {
         // the item's last chunk: O is final once its PV product completes
+        const RowPos pos = pos_of(li);
+        float2 prev[NPRE];   // the warp's first NPRE rows; the others load in the merge
+        float mg, lg;
+        load_prev(pos, prev, mg, lg);
         if (!wait_warp(&o_done[t], (uint32_t)g & 1u)) { ok = false; break; }
         tc_fence_after();
-        float oacc[64];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t ov[32];
-          tmem_ld_32x32b_x32(obase + half * 32, ov);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) oacc[half * 32 + i] = __uint_as_float(ov[i]);
-        }
-        tc_fence_before();
         // the statistics in canonical form: relative to the true maximum
+        float af = 1.f;
         if (m_true > m_ref) {
-          const float af = rescale(m_ref, m_true);
-#pragma unroll
-          for (int i = 0; i < 64; ++i) oacc[i] *= af;
+          af = rescale(m_ref, m_true);
           l_run *= af;
           m_ref = m_true;
         }
-        merge(li, oacc);
+        merge(pos, af, prev, mg, lg);
       }
     }
   }

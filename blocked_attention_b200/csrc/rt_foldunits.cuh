@@ -120,7 +120,7 @@ __device__ __forceinline__ void fold_units(const FoldUnitArgs& P, int q0, int nq
       for (int e = 0; e < 8; ++e) oo[e] *= al;
 #pragma unroll
       for (int i = 0; i < NK; ++i) {
-        const float p = exp2f(sc[i] - mn);
+        const float p = ex2_ftz(sc[i] - mn);
         float vv[8];
         unpack_bf16x8(vw[r][i], vv);
         ln += p;
