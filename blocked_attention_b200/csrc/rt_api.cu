@@ -271,8 +271,8 @@ static TileCfg choose_tiles(int M, int N, int K, bool allow_split) {
 // Per-step GEMMs may use cluster split-K (see choose_tiles).
 static constexpr bool kLayerSplitK = true;
 // Smallest block size that uses the tcgen05 folds (smaller ones: mma.sync);
-// measured at B = 512, d = 1024: mma.sync wins up to 256 keys, tcgen05 from 512.
-static constexpr int kFoldTcMinBlock = 512;
+// measured at B = 512, d = 1024: mma.sync wins up to 128 keys, tcgen05 from 256.
+static constexpr int kFoldTcMinBlock = 256;
 
 template <int BN, int EPI>
 static cudaError_t launch_tc_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
