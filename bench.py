@@ -222,7 +222,7 @@ def algorithmic_work(cfg: dict, schedule: str = "blocked") -> dict:
         else:
             warp_b += by
     w["fold_warp"] = ("hbm", warp_b)
-    w["fold_mma"] = ("hbm", mma_b)
+    w["fold_tensor"] = ("hbm", mma_b)
     return w
 
 

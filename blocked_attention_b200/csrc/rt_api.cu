@@ -456,7 +456,7 @@ struct HostIo {
 // per-kernel-class event timing (stream driver only)
 // ---------------------------------------------------------------------------
 enum KernelClass {
-  KC_INV_RMS = 0, KC_PROJ, KC_ATTEND, KC_WO, KC_W1, KC_W2, KC_WKV, KC_FOLD_WARP, KC_FOLD_MMA, KC_STEPS,
+  KC_INV_RMS = 0, KC_PROJ, KC_ATTEND, KC_WO, KC_W1, KC_W2, KC_WKV, KC_FOLD_WARP, KC_FOLD_TENSOR, KC_STEPS,
   KC_FOLD_LEVEL0 = 16,   // + log2(block size): per-level fold timing
   KC_COUNT = 32
 };
@@ -1639,7 +1639,7 @@ extern "C" int rt_layer_forward_timed(const void* x, const void* W_q, const void
     const int c = timer.cls[i];
     if (c < n_classes) { class_ms[c] += ms; class_launches[c] += 1; }
     if (c >= KC_FOLD_LEVEL0) {   // per-level folds also count towards the kernel that ran them
-      const int kc = (s.dtype == RT_BF16 && c - KC_FOLD_LEVEL0 >= 4) ? KC_FOLD_MMA : KC_FOLD_WARP;
+      const int kc = (s.dtype == RT_BF16 && c - KC_FOLD_LEVEL0 >= 4) ? KC_FOLD_TENSOR : KC_FOLD_WARP;
       if (kc < n_classes) { class_ms[kc] += ms; class_launches[kc] += 1; }
     }
   }

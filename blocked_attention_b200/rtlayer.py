@@ -35,7 +35,7 @@ EXPORTS = ("rt_version", "rt_status_string", "rt_last_cuda_error", "rt_cuda_erro
            "rt_layer_chunked_workspace_bytes", "rt_layer_forward_chunked")
 
 KERNEL_CLASSES = ("inv_rms", "proj", "attend", "gemm_wo", "gemm_w1", "gemm_w2", "gemm_wkv",
-                  "fold_warp", "fold_mma", "steps")
+                  "fold_warp", "fold_tensor", "steps")
 RT_KC_FOLD_LEVEL0 = 16
 RT_KC_COUNT = 32
 

@@ -373,7 +373,8 @@ enum {
   RT_KC_W2 = 5,      /* h W_2^T + residual = z_t                          */
   RT_KC_WKV = 6,     /* persistent pair rms(z_t) [W_k; W_v]^T             */
   RT_KC_FOLD_WARP = 7, /* block fold, small-block / warp kernels          */
-  RT_KC_FOLD_MMA = 8,  /* block fold, tensor-core kernel (block >= 16)    */
+  RT_KC_FOLD_TENSOR = 8, /* block fold on tensor cores (block >= 16: mma.sync
+                           below 256 keys, tcgen05 from 256)             */
   RT_KC_STEPS = 9,     /* persistent step kernel: a segment's W_o, W_1,
                           W_2, W_kv GEMMs and its folds of <= 8 keys       */
   RT_KC_FOLD_LEVEL0 = 16, /* + log2(block size): the same folds by level  */
