@@ -613,7 +613,7 @@ __global__ void __launch_bounds__(320, 1)
     // row, 16-byte chunks XOR-swizzled by row). Both P buffers are idle from
     // the item's last PV product until this warp writes its next P rows.
     uint8_t* const stg = smem + C::OFF_P + t * 2 * C::P_BYTES + qq * 4096;
-    constexpr int NPRE = 12;   // rows of the running o loaded ahead (registers allow no more)
+    constexpr int NPRE = 14;   // rows of the running o loaded ahead (registers allow no more)
     struct RowPos { int b, h, qt0, nrows; };
     auto pos_of = [&](int li) {
       RowPos p;
@@ -782,9 +782,19 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       const float lsum = ((lsp[0] + lsp[1]) + (lsp[2] + lsp[3])) + ((lsp[4] + lsp[5]) + (lsp[6] + lsp[7]));
+      // o_done completes one phase per PV product, and a parity wait only
+      // tells the phase it waits for from the one before it. Chunk g - 1's
+      // product has had no wait of its own (the next chunk's S products are
+      // issued ahead of it), so it is waited for here -- before this chunk's
+      // P is released, while chunk g's product cannot have started -- when O
+      // is rescaled and at an item's last chunk, whose merge then waits for
+      // phase g alone.
+      if ((rescale_o || c == nch - 1) && g > 0 && !wait_warp(&o_done[t], (uint32_t)(g - 1) & 1u)) {
+        ok = false;
+        break;
+      }
       if (rescale_o) {
-        // O of chunks up to g - 1: its last PV product must have completed
-        if (!wait_warp(&o_done[t], (uint32_t)(g - 1) & 1u)) { ok = false; break; }
+        // O of chunks up to g - 1 is final: rescale it
         tc_fence_after();
 #pragma unroll
         for (int half = 0; half < 2; ++half) {

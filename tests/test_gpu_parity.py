@@ -133,6 +133,45 @@ def test_block_fold_matches_oracle(rt, dtype, nk, nq, init_empty):
     np.testing.assert_array_equal(to_np(og)[untouched], o0[untouched].astype(np.float32))
 
 
+@pytest.mark.parametrize("nk,init_empty", [(256, False), (256, True), (384, False)])
+def test_block_fold_many_items_per_cta(rt, nk, init_empty):
+    # The two-tile tcgen05 fold with several (pair, 256-query) items per CTA
+    # (1280 items over the SMs) and two or three 128-key chunks per item: each
+    # item's merge must see every PV product of the item. Sampled pairs are
+    # checked against the oracle with the bound of test_block_fold_matches_oracle.
+    B, H, dh, nq = 64, 20, 64, 256
+    d = H * dh
+    npos = nk + nq + 2
+    rng = np.random.default_rng(nk * 11 + int(init_empty))
+    Q = rtinputs.to_grid(rng.standard_normal((npos, B, d)), "bf16")
+    Kc = rtinputs.to_grid(rng.standard_normal((npos, B, d)), "bf16")
+    Vc = rtinputs.to_grid(rng.standard_normal((npos, B, d)), "bf16")
+    m0 = rng.standard_normal((npos, B, H)) * 2
+    l0 = rng.uniform(0.5, 3.0, (npos, B, H))
+    o0 = rng.standard_normal((npos, B, d))
+    if init_empty:
+        m0[:] = -np.inf; l0[:] = 0; o0[:] = 0
+    k0, q0 = 1, 1 + nk
+    mg = torch.tensor((m0 * LOG2E).astype(np.float32), device="cuda")
+    lg = torch.tensor(l0.astype(np.float32), device="cuda")
+    og = torch.tensor(o0.astype(np.float32), device="cuda")
+    rt.block_fold(to_device(Q, "bf16"), to_device(Kc, "bf16"), to_device(Vc, "bf16"), mg, lg, og, H, dh,
+                  q0, nq, k0, nk)
+    torch.cuda.synchronize()
+    m_all, l_all, o_all = to_np(mg) / LOG2E, to_np(lg), to_np(og)
+    for pair in range(0, B * H, 37):
+        b, h = divmod(pair, H)
+        sl = slice(h * dh, (h + 1) * dh)
+        v = Vc[k0:k0 + nk, b, sl]
+        mr, lr, orr = O.block_fold(Q[q0:q0 + nq, b, sl], Kc[k0:k0 + nk, b, sl], v, m0[q0:q0 + nq, b, h].copy(),
+                                   l0[q0:q0 + nq, b, h].copy(), o0[q0:q0 + nq, b, sl].copy(), 1.0 / math.sqrt(dh))
+        m_got, l_got, o_got = m_all[q0:q0 + nq, b, h], l_all[q0:q0 + nq, b, h], o_all[q0:q0 + nq, b, sl]
+        assert np.max(np.abs(m_got - mr)) < 1e-4 * max(1.0, np.max(np.abs(mr)))
+        bound = 2.0 ** -9 * np.max(np.abs(v)) * 1.01 + 1e-5
+        assert np.max(np.abs(o_got / l_got[:, None] - orr / lr[:, None])) <= bound, (b, h)
+        assert rel_err(l_got, lr) < 2.0 ** -9 * 1.01
+
+
 # --------------------------------------------------------------------------
 # the layer
 # --------------------------------------------------------------------------
